@@ -1,0 +1,195 @@
+/*
+ * qmm.h -- C ABI of the packed 4-bit weight matmul library (libqmm.so) for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The library decodes and multiplies weights that stay packed in GPU memory:
+ *
+ *   IQ4_NL      18-byte blocks of 32 weights: a little-endian fp16 scale d,
+ *               then 16 bytes of 4-bit indices into the 16-entry non-linear
+ *               table {-127,-104,-83,-65,-49,-35,-22,-10,1,13,25,38,53,69,89,
+ *               113}; the low nibble of byte j is weight j of the block, the
+ *               high nibble weight j+16.  A row of k weights is k/32
+ *               consecutive blocks; rows follow each other.
+ *               ("Mark-Experimental-V3-8B", section "Quantization".)
+ *   FP4G16_F16  E2M1 codes, two per byte (low nibble = even k), row-major
+ *               [n][k/2]; one fp16 scale per 16 consecutive k, row-major
+ *               [n][k/16].  Weight = fp16(code * scale).
+ *   FP4G16_E4M3 the same codes; one E4M3FN byte scale per 16 consecutive k,
+ *               row-major [n][k/16], and one fp32 global scale g per matrix.
+ *               Weight = fp16(fp32(code * e4m3 * g)).
+ *               ("Mamb2_8B_FP4_Recall_SQ3.25", section "Representation",
+ *               paragraph "Weights": E2M1 codes with magnitudes 0, 0.5, 1,
+ *               1.5, 2, 3, 4, 6, 16-element groups along the input axis, an
+ *               E4M3FN block scale per group and an FP32 scale per matrix.)
+ *
+ * A weight matrix W is [n][k]: n output rows, k input columns; groups run
+ * along k.  Activations x are fp16 [m][k] row-major, outputs y are fp16
+ * [m][n] row-major (y = x W^T), accumulated in fp32.  fp16 values are passed
+ * as uint16_t bit patterns.
+ *
+ * Conventions shared by every entry point:
+ *   - Every pointer argument marked "device" must point to GPU global memory
+ *     of the current device; the caller allocates and owns all of it.  The
+ *     library allocates nothing on the device except its fixed error word and
+ *     keeps no pointer after a call returns.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream); all work
+ *     is enqueued on it and the call returns without synchronising.
+ *   - Argument checks happen on the host before anything is enqueued; on
+ *     failure nothing is launched and the status says why.  There is no CPU
+ *     fallback and no silent fallback: a shape or layout that no kernel
+ *     supports returns QMM_ERR_UNSUPPORTED_SHAPE.
+ *   - Errors that can only be seen on the device (a pipeline wait that ran
+ *     out, an expert id out of range) set a per-device error word;
+ *     qmm_sync_check() reports and clears it.
+ *   - Device base pointers must be 16-byte aligned (QMM_ERR_MISALIGNED
+ *     otherwise).
+ *   - Calls on different streams may run concurrently; they share no state
+ *     besides the error word.
+ */
+#ifndef QMM_H_
+#define QMM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QMM_OK = 0,
+  QMM_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad format */
+  QMM_ERR_UNSUPPORTED_SHAPE = 2, /* k not a multiple of the group, m out of range */
+  QMM_ERR_MISALIGNED = 3,        /* a device pointer is not 16-byte aligned */
+  QMM_ERR_NOT_SM100 = 4,         /* current device is not compute capability 10.0 */
+  QMM_ERR_CUDA = 5,              /* a CUDA runtime call failed (launch, attribute) */
+  QMM_ERR_TIMEOUT = 6,           /* a kernel wait ran out (reported by qmm_sync_check) */
+  QMM_ERR_DEVICE_FAULT = 7,      /* bad data seen on the device, e.g. expert id out of range */
+  QMM_ERR_WORKSPACE = 8          /* workspace missing or smaller than qmm_workspace_bytes() */
+} qmm_status;
+
+typedef enum {
+  QMM_FMT_IQ4_NL = 1,
+  QMM_FMT_FP4G16_F16 = 2,
+  QMM_FMT_FP4G16_E4M3 = 3
+} qmm_format;
+
+/* One packed matrix, or a stack of `num_experts` packed matrices of equal
+ * shape (the routed-expert tensor of the IQ4_NL model card: one contiguous
+ * [E][n][k] tensor per projection, "Mark-Experimental-V3-8B", section
+ * "Quantization", last bullet). */
+typedef struct {
+  int32_t fmt;            /* qmm_format */
+  int32_t reserved;       /* must be 0 */
+  int64_t n;              /* output rows */
+  int64_t k;              /* input columns: k % 32 == 0 (IQ4_NL), k % 16 == 0 (FP4) */
+  const void* data;       /* device: IQ4_NL blocks, or FP4 codes [n][k/2] */
+  const void* scales;     /* device: FP4 scales [n][k/16] (fp16 or E4M3FN); NULL for IQ4_NL */
+  float global_scale;     /* FP4G16_E4M3 only (fp32 g); ignored otherwise */
+  int32_t reserved2;      /* must be 0 */
+  int64_t num_experts;    /* 1 for a plain matrix */
+  int64_t expert_data_stride;  /* bytes between experts in `data` (>= qmm_data_bytes) */
+  int64_t expert_scale_stride; /* bytes between experts in `scales` */
+} qmm_weights;
+
+/* Bytes of the code/block array of one [n][k] matrix (IQ4_NL: n*k/32*18;
+ * FP4: n*k/2).  Returns 0 for an invalid format or shape. */
+size_t qmm_data_bytes(int32_t fmt, int64_t n, int64_t k);
+
+/* Bytes of the separate scale array of one matrix (IQ4_NL: 0; FP4G16_F16:
+ * n*k/16*2; FP4G16_E4M3: n*k/16). */
+size_t qmm_scale_bytes(int32_t fmt, int64_t n, int64_t k);
+
+/* qmm_data_bytes + qmm_scale_bytes (+4 for the FP4G16_E4M3 global scale, as
+ * the storage table of the FP4-G16 model card counts it). */
+size_t qmm_packed_bytes(int32_t fmt, int64_t n, int64_t k);
+
+/* Decode a packed matrix to resident fp16, bit-exactly as defined above (one
+ * rounding to fp16, round to nearest even, fp16 subnormals kept; for E4M3 the
+ * product is rounded to fp32 and then to fp16).  This is what the published
+ * runtime of the FP4-G16 model card does at load time
+ * ("Mamb2_8B_FP4_Recall_SQ3.25", section "Storage and runtime memory": all
+ * decoded FP16 weights stay resident).
+ *   w       weights (num_experts must be 1)
+ *   out     device, [n][k] fp16, written completely
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, NOT_SM100, CUDA. */
+qmm_status qmm_dequant(const qmm_weights* w, uint16_t* out, void* stream);
+
+/* Fused dequantise-and-multiply for decode batches: y[m][n] = sum_k
+ * x[m][k] * W[n][k] with the decoded fp16 weights, fp32 accumulation, one
+ * rounding of the sum to fp16.  For FP4G16_E4M3 the global scale g is applied
+ * to the fp32 sum instead of to each weight (the difference from the
+ * per-weight definition is one fp16 rounding of each weight).
+ *   x       device, [m][k] fp16
+ *   m       1..16
+ *   y       device, [m][n] fp16
+ *   ws      device workspace of ws_bytes (qmm_workspace_bytes(QMM_OP_GEMV, ...));
+ *           may be NULL when that is 0
+ * Errors: as qmm_dequant, plus WORKSPACE. */
+qmm_status qmm_gemv(const qmm_weights* w, const uint16_t* x, int64_t m, uint16_t* y, void* ws,
+                    size_t ws_bytes, void* stream);
+
+/* The same product for a prefill window (m up to any size; the kernel is a
+ * tensor-core GEMM that decodes weight tiles into shared memory).
+ *   x       device, [m][k] fp16;  y device, [m][n] fp16
+ * Errors: as qmm_gemv. */
+qmm_status qmm_gemm(const qmm_weights* w, const uint16_t* x, int64_t m, uint16_t* y, void* ws,
+                    size_t ws_bytes, void* stream);
+
+/* Bucket the t*topk (token, slot) pairs of a top-k routing by expert: a
+ * counting sort ("Mark-Experimental-V3-8B", section "Mixture-of-Experts
+ * (MoE)": 32 routed experts, top-4 per token).
+ *   topk_ids        device, [t][topk] int32 expert ids
+ *   expert_offsets  device, [num_experts+1] int32: pairs of expert e are
+ *                   pair_perm[offsets[e] .. offsets[e+1]-1]
+ *   pair_perm       device, [t*topk] int32 pair indices p = token*topk+slot,
+ *                   grouped by expert (order within an expert unspecified);
+ *                   ids outside [0, num_experts) are left out, their count is
+ *                   t*topk - offsets[num_experts], and the device error word
+ *                   records QMM_ERR_DEVICE_FAULT
+ *   ws              device workspace (qmm_workspace_bytes(QMM_OP_ROUTE, ...))
+ * Errors: INVALID_ARG, MISALIGNED, NOT_SM100, CUDA, WORKSPACE. */
+qmm_status qmm_route(const int32_t* topk_ids, int64_t t, int64_t topk, int64_t num_experts,
+                     int32_t* expert_offsets, int32_t* pair_perm, void* ws, size_t ws_bytes,
+                     void* stream);
+
+/* Routed-expert grouped GEMV: for every (token, slot) with e =
+ * topk_ids[token][slot] in range, y[token][slot][:] = W_e x_row, where x_row
+ * is x[token] (x_per_pair = 0, x is [t][k]) or x[token][slot]
+ * (x_per_pair = 1, x is [t][topk][k]).  Each expert's weights are read once
+ * for all of the pairs routed to it.  Pairs with an id out of range leave
+ * their y row untouched and set QMM_ERR_DEVICE_FAULT in the error word.
+ *   experts   a stack of num_experts matrices (expert_*_stride set)
+ *   y         device, [t][topk][n] fp16
+ *   ws        device workspace (qmm_workspace_bytes(QMM_OP_GROUPED, ...))
+ * Errors: as qmm_gemv. */
+qmm_status qmm_grouped_gemv(const qmm_weights* experts, const uint16_t* x, int32_t x_per_pair,
+                            const int32_t* topk_ids, int64_t t, int64_t topk, uint16_t* y, void* ws,
+                            size_t ws_bytes, void* stream);
+
+enum { QMM_OP_DEQUANT = 0, QMM_OP_GEMV = 1, QMM_OP_GEMM = 2, QMM_OP_ROUTE = 3, QMM_OP_GROUPED = 4 };
+
+/* Device workspace bytes an operation needs for these sizes (0 = none).
+ * `w` may be NULL for QMM_OP_ROUTE; `num_experts` is taken from `w` except
+ * for QMM_OP_ROUTE, where it is passed in `m`. */
+size_t qmm_workspace_bytes(int32_t op, const qmm_weights* w, int64_t m, int64_t t, int64_t topk);
+
+/* Synchronise `stream`, then read and clear this device's error word.
+ * Returns QMM_OK, QMM_ERR_TIMEOUT, QMM_ERR_DEVICE_FAULT or QMM_ERR_CUDA. */
+qmm_status qmm_sync_check(void* stream);
+
+/* Static text for a status code. */
+const char* qmm_status_string(int32_t status);
+
+/* Name of the kernel variant the last successful call on this host thread
+ * launched (for dispatch records next to timings); "" before any call. */
+const char* qmm_last_variant(void);
+
+/* Library version string. */
+const char* qmm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QMM_H_ */

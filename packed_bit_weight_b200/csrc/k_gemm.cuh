@@ -1,0 +1,293 @@
+// k_gemm.cuh -- prefill GEMM on packed FP4-G16 weights with 5th-generation
+// tensor cores (tcgen05, accumulators in tensor memory).
+//
+// Y[m][n] = sum_k X[m][k] W[n][k] for a prefill window (m = 2048 tokens in
+// the model card's evaluation protocol, "Mamb2_8B_FP4_Recall_SQ3.25",
+// section "Measured quality": windows of up to 2,048 targets).
+//
+// One CTA computes a 128 x BN tile of Y (128 tokens x BN weight rows).  Per
+// 64-wide k step:
+//   * warp 0 (one thread) loads the X tile [128 x 64] fp16 with a 2-D tensor
+//     map, 128-byte swizzle -- the canonical K-major operand layout;
+//   * warps 2-5 (128 threads) load the packed codes and scales of the BN
+//     weight rows straight from global memory (registers, one step ahead),
+//     decode them to fp16 (E2M1 -> f16x2 convert, one multiply by the group
+//     scale = the bit-exact dequantised weight) and store them into shared
+//     memory in the same swizzled K-major layout;
+//   * warp 1 (one thread) issues four tcgen05.mma (M=128, N=BN, K=16) per
+//     step from the two shared-memory descriptors into the fp32 accumulator
+//     in tensor memory and commits them to the stage's "empty" barrier.
+// A ring of STAGES stages decouples the three.  After the last step the MMA
+// thread commits to an "accumulator ready" barrier and warps 2-5 read the
+// accumulator with tcgen05.ld (each warp owns 32 TMEM lanes = 32 tokens),
+// round to fp16 and store Y.
+//
+// No TMA multicast is used.  Every wait is bounded (%globaltimer); on a
+// timeout the kernel raises the error word, drains its own copies and MMAs,
+// frees its tensor memory and returns.
+#pragma once
+#include "qmm_dev.cuh"
+
+namespace qmm {
+
+constexpr int kGemmBM = 128;
+constexpr int kGemmBK = 64;
+constexpr int kGemmThreads = 6 * 32;
+constexpr int kGemmDecodeThreads = 128;
+
+template <int BN, int STAGES>
+struct GemmCfg {
+  static constexpr int kABytes = kGemmBM * kGemmBK * 2;  // 16 KB
+  static constexpr int kBBytes = BN * kGemmBK * 2;        // 32 KB at BN=256
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = BN;                    // fp32 accumulator columns
+  static size_t smem_bytes() { return 1024 + (size_t)STAGES * kStageBytes + 256; }
+};
+
+// --- tcgen05 wrappers --------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive on `bar` once all tcgen05.mma issued so far by this thread complete.
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
+// 128 B, 8-row groups 1024 B apart (SBO), LBO unused (1), descriptor version 1.
+__device__ __forceinline__ uint64_t umma_desc_k128(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) | ((uint64_t)(1024u >> 4) << 32) |
+         ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+}
+
+// Instruction descriptor, kind::f16: fp16 A and B (K-major), fp32 D, M=128.
+__host__ __device__ constexpr uint32_t umma_idesc_f16(int n) {
+  return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+// Packed data of one weight row for one 64-wide k step.
+struct RowPack {
+  uint4 c0, c1;  // 32 code bytes (k0 .. k0+63)
+  uint2 s;       // fp16: 4 scales; E4M3: 4 bytes in s.x
+};
+
+template <int FMT>
+__device__ __forceinline__ void load_rowpack(RowPack& p, const uint8_t* __restrict__ codes,
+                                             const uint8_t* __restrict__ scales, int64_t row, int n, int k,
+                                             int k0) {
+  if (row < n) {
+    const uint8_t* cp = codes + row * (int64_t)(k >> 1) + (k0 >> 1);
+    p.c0 = ldg_nc128(cp);
+    p.c1 = ldg_nc128(cp + 16);
+    if (FMT == 2) {
+      p.s = *reinterpret_cast<const uint2*>(scales + (row * (int64_t)(k >> 4) + (k0 >> 4)) * 2);
+    } else {
+      p.s.x = *reinterpret_cast<const uint32_t*>(scales + row * (int64_t)(k >> 4) + (k0 >> 4));
+      p.s.y = 0;
+    }
+  } else {
+    p.c0 = make_uint4(0, 0, 0, 0);
+    p.c1 = p.c0;
+    p.s = make_uint2(0, 0);
+  }
+}
+
+// Decode one row's 64 weights and store them as 8 swizzled 16-byte chunks.
+template <int FMT>
+__device__ __forceinline__ void store_row(const RowPack& p, uint32_t b_stage, int r) {
+  uint32_t sc[4];  // f16x2 broadcast scale per group of 16 (= two chunks)
+  if (FMT == 2) {
+    sc[0] = bcast_lo(p.s.x); sc[1] = bcast_hi(p.s.x); sc[2] = bcast_lo(p.s.y); sc[3] = bcast_hi(p.s.y);
+  } else {
+    const uint32_t e01 = e4m3x2_to_f16x2(p.s.x & 0xFFFFu), e23 = e4m3x2_to_f16x2(p.s.x >> 16);
+    sc[0] = bcast_lo(e01); sc[1] = bcast_hi(e01); sc[2] = bcast_lo(e23); sc[3] = bcast_hi(e23);
+  }
+  const uint32_t q[8] = {p.c0.x, p.c0.y, p.c0.z, p.c0.w, p.c1.x, p.c1.y, p.c1.z, p.c1.w};
+  const uint32_t row_base = b_stage + (uint32_t)r * 128u;
+  const uint32_t sw = (uint32_t)(r & 7);
+#pragma unroll
+  for (int c = 0; c < 8; c++) {  // chunk c = k 8c .. 8c+7 = code word q[c]
+    uint32_t w[4];
+    e2m1x8_to_f16x2(q[c], w);
+    const uint32_t s = sc[c >> 1];
+    sts128(row_base + ((c ^ sw) << 4), hmul2(w[0], s), hmul2(w[1], s), hmul2(w[2], s), hmul2(w[3], s));
+  }
+}
+
+template <int FMT, int BN, int STAGES>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_fp4_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const uint8_t* __restrict__ codes,
+                       const uint8_t* __restrict__ scales, uint16_t* __restrict__ y, int m, int n, int k, float g) {
+  using C = GemmCfg<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t base = (smem_addr(smem_raw) + 1023u) & ~1023u;
+  const uint32_t a_s = base;                                  // STAGES x 16 KB
+  const uint32_t b_s = a_s + STAGES * C::kABytes;             // STAGES x BN*128 B
+  const uint32_t bars = b_s + STAGES * C::kBBytes;            // full[S], empty[S], accum
+  const uint32_t tmem_slot = bars + 8 * (2 * STAGES + 1);
+  uint32_t* tmem_slot_ptr = reinterpret_cast<uint32_t*>(smem_raw + (tmem_slot - smem_addr(smem_raw)));
+  __shared__ volatile int s_abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tiles = (n + BN - 1) / BN;
+  const int tile_n = blockIdx.x % n_tiles, tile_m = blockIdx.x / n_tiles;
+  const int m0 = tile_m * kGemmBM, n0 = tile_n * BN;
+  const int ksteps = k / kGemmBK;
+  // the last weight-row tile may be half as wide: issue N = 128 there
+  const int n_valid = min(BN, n - n0);
+  const int n_mma = (n_valid <= BN / 2) ? BN / 2 : BN;
+
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    for (int s = 0; s < STAGES; s++) {
+      mbar_init(bars + 8 * s, 1 + kGemmDecodeThreads);  // full: TMA arrive(+tx) + decode threads
+      mbar_init(bars + 8 * (STAGES + s), 1);             // empty: MMA commit
+    }
+    mbar_init(bars + 8 * (2 * STAGES), 1);               // accumulator ready
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot_ptr;
+  const uint32_t accum_bar = bars + 8 * (2 * STAGES);
+
+  if (warp == 0) {
+    // ---------------------------- X loader --------------------------------
+    if (lane == 0) {
+      prefetch_tmap(&tm_x);
+      int issued = 0;
+      for (int ks = 0; ks < ksteps; ks++) {
+        const int s = ks % STAGES;
+        const uint32_t ph = (uint32_t)(ks / STAGES) & 1u;
+        if (s_abort || !mbar_wait(bars + 8 * (STAGES + s), ph ^ 1u)) { s_abort = 1; break; }
+        mbar_arrive_expect_tx(bars + 8 * s, C::kABytes);
+        tma_load_2d(a_s + s * C::kABytes, &tm_x, ks * kGemmBK, m0, bars + 8 * s);
+        issued++;
+      }
+      // drain: the last use of every stage must have landed
+      for (int s = 0; s < STAGES && s < issued; s++) {
+        const int last = issued - 1 - ((issued - 1 - s) % STAGES);
+        mbar_wait(bars + 8 * s, (uint32_t)(last / STAGES) & 1u);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------- MMA issuer ------------------------------
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_f16(n_mma);
+      for (int ks = 0; ks < ksteps; ks++) {
+        const int s = ks % STAGES;
+        const uint32_t ph = (uint32_t)(ks / STAGES) & 1u;
+        if (s_abort || !mbar_wait(bars + 8 * s, ph)) { s_abort = 1; break; }
+        tc_fence_after();
+        const uint64_t da = umma_desc_k128(a_s + s * C::kABytes);
+        const uint64_t db = umma_desc_k128(b_s + s * C::kBBytes);
+#pragma unroll
+        for (int kk = 0; kk < kGemmBK / 16; kk++)  // +32 bytes per K=16 inside the swizzle row
+          umma_f16(tmem, da + (uint64_t)(2 * kk), db + (uint64_t)(2 * kk), idesc, (ks | kk) != 0);
+        umma_commit(bars + 8 * (STAGES + s));  // frees the stage when these MMAs are done
+      }
+      umma_commit(accum_bar);  // all issued MMAs complete -> accumulator ready
+    }
+  } else {
+    // ---------------------- decode producers + epilogue ----------------------
+    const int t = threadIdx.x - 64;  // 0..127: weight rows t and t+128 of the tile
+    RowPack cur[BN / 128], nxt[BN / 128];
+#pragma unroll
+    for (int h = 0; h < BN / 128; h++) load_rowpack<FMT>(cur[h], codes, scales, (int64_t)n0 + t + 128 * h, n, k, 0);
+    for (int ks = 0; ks < ksteps; ks++) {
+      const int s = ks % STAGES;
+      const uint32_t ph = (uint32_t)(ks / STAGES) & 1u;
+      if (ks + 1 < ksteps) {
+#pragma unroll
+        for (int h = 0; h < BN / 128; h++)
+          load_rowpack<FMT>(nxt[h], codes, scales, (int64_t)n0 + t + 128 * h, n, k, (ks + 1) * kGemmBK);
+      }
+      if (s_abort || !mbar_wait(bars + 8 * (STAGES + s), ph ^ 1u)) { s_abort = 1; break; }
+#pragma unroll
+      for (int h = 0; h < BN / 128; h++) store_row<FMT>(cur[h], b_s + s * C::kBBytes, t + 128 * h);
+      fence_proxy_async_shared();  // generic-proxy stores -> visible to the tensor core
+      mbar_arrive(bars + 8 * s);
+#pragma unroll
+      for (int h = 0; h < BN / 128; h++) cur[h] = nxt[h];
+    }
+    // epilogue: warp q = warp % 4 owns TMEM lanes 32q .. 32q+31 (tokens)
+    const bool ready = mbar_wait(accum_bar, 0);
+    tc_fence_after();
+    if (ready && !s_abort) {
+      const int q = warp & 3;
+      const int row = m0 + 32 * q + lane;
+      const float gs = (FMT == 3) ? g : 1.0f;
+      for (int j = 0; j < n_mma / 32; j++) {
+        uint32_t r[32];
+        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(32 * j), r);
+        tmem_ld_wait();
+        const int col = n0 + 32 * j;
+        if (row < m && col < n) {
+          uint32_t h[16];
+#pragma unroll
+          for (int i = 0; i < 16; i++)
+            h[i] = f32x2_to_f16x2(__uint_as_float(r[2 * i]) * gs, __uint_as_float(r[2 * i + 1]) * gs);
+          uint16_t* yp = y + (int64_t)row * n + col;
+          if (col + 32 <= n && (n & 7) == 0) {
+            uint4* y4 = reinterpret_cast<uint4*>(yp);
+#pragma unroll
+            for (int i = 0; i < 4; i++) y4[i] = make_uint4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
+          } else {
+            for (int i = 0; i < 32 && col + i < n; i++) yp[i] = (uint16_t)((h[i >> 1] >> (16 * (i & 1))) & 0xFFFFu);
+          }
+        }
+      }
+    }
+  }
+
+  // teardown: nothing of ours may still write shared or tensor memory
+  if (warp == 1 && lane == 0 && s_abort) mbar_wait(accum_bar, 0);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace qmm

@@ -1,0 +1,450 @@
+// qmm_lib.cu -- libqmm.so: the C ABI declared in include/qmm.h.
+//
+// Host side: argument validation, kernel-variant selection, TMA descriptor
+// encoding and launches.  All arithmetic of the path runs in the sm_100a
+// kernels included below; there is no host or CPU fallback.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/qmm.h"
+#include "k_dequant.cuh"
+#include "k_gemv.cuh"
+#include "k_gemm.cuh"
+#include "k_grouped.cuh"
+
+namespace qmm {
+
+static thread_local char t_variant[160] = "";
+
+static void set_variant(const char* fmt, ...) __attribute__((format(printf, 1, 2)));
+static void set_variant(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_variant, sizeof(t_variant), fmt, ap);
+  va_end(ap);
+}
+
+struct DevInfo {
+  bool init = false;
+  bool sm100 = false;
+  int sms = 0;
+  size_t smem_optin = 0;
+};
+static DevInfo g_dev[64];
+static std::mutex g_mu;
+
+static qmm_status device_info(DevInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return QMM_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DevInfo& d = g_dev[dev];
+  if (!d.init) {
+    int major = 0, minor = 0, sms = 0, optin = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+      return QMM_ERR_CUDA;
+    d.sm100 = (major == 10 && minor == 0);
+    d.sms = sms;
+    d.smem_optin = (size_t)optin;
+    d.init = true;
+  }
+  *out = &d;
+  return d.sm100 ? QMM_OK : QMM_ERR_NOT_SM100;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static bool valid_fmt(int32_t f) { return f == QMM_FMT_IQ4_NL || f == QMM_FMT_FP4G16_F16 || f == QMM_FMT_FP4G16_E4M3; }
+
+static qmm_status check_weights(const qmm_weights* w, bool allow_experts) {
+  if (!w) return QMM_ERR_INVALID_ARG;
+  if (!valid_fmt(w->fmt) || w->reserved != 0 || w->reserved2 != 0) return QMM_ERR_INVALID_ARG;
+  if (w->n < 0 || w->k < 0 || w->num_experts < 1) return QMM_ERR_INVALID_ARG;
+  if (!allow_experts && w->num_experts != 1) return QMM_ERR_INVALID_ARG;
+  if (w->n > INT32_MAX || w->k > INT32_MAX) return QMM_ERR_UNSUPPORTED_SHAPE;
+  if (w->fmt == QMM_FMT_IQ4_NL ? (w->k % 32) : (w->k % 16)) return QMM_ERR_UNSUPPORTED_SHAPE;
+  if (w->n > 0 && w->k > 0) {
+    if (!w->data) return QMM_ERR_INVALID_ARG;
+    if (w->fmt != QMM_FMT_IQ4_NL && !w->scales) return QMM_ERR_INVALID_ARG;
+    if (!aligned16(w->data) || (w->scales && !aligned16(w->scales))) return QMM_ERR_MISALIGNED;
+  }
+  return QMM_OK;
+}
+
+static qmm_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? QMM_OK : QMM_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// TMA descriptors (driver entry point fetched through the runtime, so the
+// library needs no link-time libcuda).
+// ---------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+static bool get_encoder() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_encode) return true;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || !fn)
+    return false;
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return true;
+}
+
+// 2-D map over a row-major [rows][cols] array of `elem`-byte elements.
+static bool make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem, uint64_t cols,
+                        uint64_t rows, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  if (!get_encoder()) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * (uint64_t)elem};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+static int grid_for(int64_t items, int per_block, int sms, int waves = 8) {
+  int64_t b = (items + per_block - 1) / per_block;
+  int64_t cap = (int64_t)sms * waves;
+  if (b > cap) b = cap;
+  if (b < 1) b = 1;
+  return (int)b;
+}
+
+// ---------------------------------------------------------------------------
+// GEMV dispatch
+// ---------------------------------------------------------------------------
+template <int FMT, int MT, int NT>
+static qmm_status launch_gemv_tma(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st,
+                                  const DevInfo* di) {
+  using C = GemvTmaCfg<FMT, MT>;
+  const int n = (int)w->n, k = (int)w->k;
+  CUtensorMap tc, ts;
+  if (!make_map_2d(&tc, w->data, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)k / 2, (uint64_t)n, 128, C::RT,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+    return QMM_ERR_CUDA;
+  if (FMT == 2) {
+    if (!make_map_2d(&ts, w->scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)k / 16, (uint64_t)n, 16, C::RT,
+                     CU_TENSOR_MAP_SWIZZLE_NONE))
+      return QMM_ERR_CUDA;
+  } else {
+    if (!make_map_2d(&ts, w->scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)k / 16, (uint64_t)n, 16, C::RT,
+                     CU_TENSOR_MAP_SWIZZLE_NONE))
+      return QMM_ERR_CUDA;
+  }
+  const size_t budget = di->smem_optin - 1024;  // room for the static shared words
+  int depth = 16;
+  while (depth > 2 && C::smem_bytes(depth) > budget) depth--;
+  const size_t smem = C::smem_bytes(depth);
+  auto kern = gemv_fp4_tma_kernel<FMT, MT, NT>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return QMM_ERR_CUDA;
+  const int tiles = (n + C::RT - 1) / C::RT;
+  const int grid = tiles < di->sms ? tiles : di->sms;
+  kern<<<grid, kGemvThreads, smem, st>>>(tc, ts, x, y, n, k, m, w->global_scale, tiles, depth);
+  set_variant("gemv_fp4_tma<fmt=%d,rt=%d,nt=%d,depth=%d,grid=%d>", FMT, C::RT, NT, depth, grid);
+  return launch_status();
+}
+
+template <int FMT>
+static qmm_status gemv_fmt(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st,
+                           const DevInfo* di) {
+  const int64_t n = w->n, k = w->k;
+  if (FMT != 1 && k % kChunkK == 0 && k >= 8 * kChunkK && n >= 16) {
+    if (m <= 8) return launch_gemv_tma<FMT, 1, 1>(w, x, m, y, st, di);
+    return launch_gemv_tma<FMT, 1, 2>(w, x, m, y, st, di);
+  }
+  const int64_t tiles = (n + 15) / 16;
+  const int64_t blocks = (tiles + 3) / 4;
+  if (blocks > INT32_MAX) return QMM_ERR_UNSUPPORTED_SHAPE;
+  gemv_generic_kernel<FMT><<<(unsigned)blocks, 128, 0, st>>>(static_cast<const uint8_t*>(w->data),
+                                                             static_cast<const uint8_t*>(w->scales), w->global_scale,
+                                                             x, y, n, k, m);
+  set_variant("gemv_generic<fmt=%d>", FMT);
+  return launch_status();
+}
+
+// ---------------------------------------------------------------------------
+// GEMM dispatch
+// ---------------------------------------------------------------------------
+template <int FMT>
+static qmm_status launch_gemm_tc(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st,
+                                 const DevInfo* di) {
+  constexpr int BN = 256, STAGES = 4;
+  using C = GemmCfg<BN, STAGES>;
+  const int n = (int)w->n, k = (int)w->k;
+  CUtensorMap tx;
+  if (!make_map_2d(&tx, x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)k, (uint64_t)m, kGemmBK, kGemmBM,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+    return QMM_ERR_CUDA;
+  const size_t smem = C::smem_bytes();
+  if (smem > di->smem_optin - 1024) return QMM_ERR_CUDA;
+  auto kern = gemm_fp4_tc_kernel<FMT, BN, STAGES>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return QMM_ERR_CUDA;
+  const int64_t tiles = (int64_t)((m + kGemmBM - 1) / kGemmBM) * ((n + BN - 1) / BN);
+  if (tiles > INT32_MAX) return QMM_ERR_UNSUPPORTED_SHAPE;
+  kern<<<(unsigned)tiles, kGemmThreads, smem, st>>>(tx, static_cast<const uint8_t*>(w->data),
+                                                    static_cast<const uint8_t*>(w->scales), y, m, n, k,
+                                                    w->global_scale);
+  set_variant("gemm_fp4_tc<fmt=%d,bm=128,bn=%d,bk=64,stages=%d,tiles=%lld>", FMT, BN, STAGES, (long long)tiles);
+  return launch_status();
+}
+
+// Any shape the tensor-core kernel does not take: the decode-batch kernel
+// over 16-token slices of x (a GPU path, recorded as such).
+template <int FMT>
+static qmm_status gemm_by_gemv(const qmm_weights* w, const uint16_t* x, int64_t m, uint16_t* y, cudaStream_t st,
+                               const DevInfo* di) {
+  for (int64_t m0 = 0; m0 < m; m0 += 16) {
+    const int mm = (int)((m - m0) < 16 ? (m - m0) : 16);
+    qmm_weights w1 = *w;
+    const int64_t tiles = (w->n + 15) / 16;
+    gemv_generic_kernel<FMT><<<(unsigned)((tiles + 3) / 4), 128, 0, st>>>(
+        static_cast<const uint8_t*>(w1.data), static_cast<const uint8_t*>(w1.scales), w1.global_scale,
+        x + m0 * w->k, y + m0 * w->n, w->n, w->k, mm);
+    if (cudaGetLastError() != cudaSuccess) return QMM_ERR_CUDA;
+  }
+  set_variant("gemm_by_gemv_generic<fmt=%d>", FMT);
+  return QMM_OK;
+}
+
+template <int FMT>
+static qmm_status launch_grouped(const qmm_weights* w, const uint16_t* x, int x_per_pair, int64_t topk,
+                                 const int32_t* offsets, const int32_t* perm, uint16_t* y, cudaStream_t st) {
+  const int64_t tiles = (w->n + 15) / 16;
+  const int64_t items = tiles * w->num_experts;
+  const int64_t blocks = (items + 3) / 4;
+  if (blocks > INT32_MAX) return QMM_ERR_UNSUPPORTED_SHAPE;
+  grouped_gemv_kernel<FMT><<<(unsigned)blocks, 128, 0, st>>>(
+      static_cast<const uint8_t*>(w->data), w->expert_data_stride, static_cast<const uint8_t*>(w->scales),
+      w->expert_scale_stride, w->global_scale, x, x_per_pair, (int)topk, offsets, perm, y, w->n, w->k,
+      (int)w->num_experts);
+  return launch_status();
+}
+
+}  // namespace qmm
+
+using namespace qmm;
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+size_t qmm_data_bytes(int32_t fmt, int64_t n, int64_t k) {
+  if (!valid_fmt(fmt) || n < 0 || k < 0) return 0;
+  if (fmt == QMM_FMT_IQ4_NL) return (k % 32) ? 0 : (size_t)n * (size_t)(k / 32) * 18u;
+  return (k % 16) ? 0 : (size_t)n * (size_t)(k / 2);
+}
+
+size_t qmm_scale_bytes(int32_t fmt, int64_t n, int64_t k) {
+  if (!valid_fmt(fmt) || n < 0 || k < 0 || fmt == QMM_FMT_IQ4_NL || (k % 16)) return 0;
+  return (size_t)n * (size_t)(k / 16) * (fmt == QMM_FMT_FP4G16_F16 ? 2u : 1u);
+}
+
+size_t qmm_packed_bytes(int32_t fmt, int64_t n, int64_t k) {
+  return qmm_data_bytes(fmt, n, k) + qmm_scale_bytes(fmt, n, k) + (fmt == QMM_FMT_FP4G16_E4M3 ? 4u : 0u);
+}
+
+const char* qmm_status_string(int32_t s) {
+  switch (s) {
+    case QMM_OK: return "ok";
+    case QMM_ERR_INVALID_ARG: return "invalid argument";
+    case QMM_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case QMM_ERR_MISALIGNED: return "device pointer not 16-byte aligned";
+    case QMM_ERR_NOT_SM100: return "current device is not sm_100 (B200)";
+    case QMM_ERR_CUDA: return "CUDA runtime error";
+    case QMM_ERR_TIMEOUT: return "a kernel pipeline wait timed out";
+    case QMM_ERR_DEVICE_FAULT: return "bad data seen on the device (expert id out of range)";
+    case QMM_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+const char* qmm_last_variant(void) { return t_variant; }
+
+const char* qmm_version(void) { return "qmm 0.1 (sm_100a)"; }
+
+qmm_status qmm_dequant(const qmm_weights* w, uint16_t* out, void* stream) {
+  qmm_status s = check_weights(w, false);
+  if (s != QMM_OK) return s;
+  DevInfo* di = nullptr;
+  if ((s = device_info(&di)) != QMM_OK) return s;
+  const int64_t total = w->n * w->k;
+  if (total == 0) return QMM_OK;
+  if (!out) return QMM_ERR_INVALID_ARG;
+  if (!aligned16(out)) return QMM_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const uint8_t* data = static_cast<const uint8_t*>(w->data);
+  const uint8_t* sc = static_cast<const uint8_t*>(w->scales);
+  if (w->fmt == QMM_FMT_IQ4_NL) {
+    const int64_t nb = total / 32;
+    dequant_iq4nl_kernel<<<grid_for(nb, 256, di->sms), 256, 0, st>>>(data, out, nb);
+    set_variant("dequant_iq4nl");
+  } else if (w->fmt == QMM_FMT_FP4G16_F16) {
+    const int64_t ng = total / 16;
+    dequant_fp4_kernel<2><<<grid_for(ng, 256, di->sms), 256, 0, st>>>(data, sc, 1.0f, out, ng);
+    set_variant("dequant_fp4<fmt=2>");
+  } else {
+    const int64_t ng = total / 16;
+    dequant_fp4_kernel<3><<<grid_for(ng, 256, di->sms), 256, 0, st>>>(data, sc, w->global_scale, out, ng);
+    set_variant("dequant_fp4<fmt=3>");
+  }
+  return launch_status();
+}
+
+static qmm_status zero_output(uint16_t* y, int64_t count, cudaStream_t st, const DevInfo* di) {
+  zero_fill_kernel<<<grid_for(count, 256, di->sms), 256, 0, st>>>(y, count);
+  set_variant("zero_fill");
+  return launch_status();
+}
+
+qmm_status qmm_gemv(const qmm_weights* w, const uint16_t* x, int64_t m, uint16_t* y, void* ws, size_t ws_bytes,
+                    void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  qmm_status s = check_weights(w, false);
+  if (s != QMM_OK) return s;
+  if (m < 0) return QMM_ERR_INVALID_ARG;
+  if (m > 16) return QMM_ERR_UNSUPPORTED_SHAPE;
+  DevInfo* di = nullptr;
+  if ((s = device_info(&di)) != QMM_OK) return s;
+  if (m == 0 || w->n == 0) return QMM_OK;
+  if (!y || (w->k > 0 && !x)) return QMM_ERR_INVALID_ARG;
+  if (!aligned16(y) || (x && !aligned16(x))) return QMM_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (w->k == 0) return zero_output(y, m * w->n, st, di);
+  switch (w->fmt) {
+    case QMM_FMT_IQ4_NL: return gemv_fmt<1>(w, x, (int)m, y, st, di);
+    case QMM_FMT_FP4G16_F16: return gemv_fmt<2>(w, x, (int)m, y, st, di);
+    default: return gemv_fmt<3>(w, x, (int)m, y, st, di);
+  }
+}
+
+qmm_status qmm_gemm(const qmm_weights* w, const uint16_t* x, int64_t m, uint16_t* y, void* ws, size_t ws_bytes,
+                    void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  qmm_status s = check_weights(w, false);
+  if (s != QMM_OK) return s;
+  if (m < 0) return QMM_ERR_INVALID_ARG;
+  if (m > INT32_MAX) return QMM_ERR_UNSUPPORTED_SHAPE;
+  DevInfo* di = nullptr;
+  if ((s = device_info(&di)) != QMM_OK) return s;
+  if (m == 0 || w->n == 0) return QMM_OK;
+  if (!y || (w->k > 0 && !x)) return QMM_ERR_INVALID_ARG;
+  if (!aligned16(y) || (x && !aligned16(x))) return QMM_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (w->k == 0) return zero_output(y, m * w->n, st, di);
+  const bool tc = w->fmt != QMM_FMT_IQ4_NL && w->k % kGemmBK == 0 && m >= 64;
+  switch (w->fmt) {
+    case QMM_FMT_IQ4_NL: return gemm_by_gemv<1>(w, x, m, y, st, di);
+    case QMM_FMT_FP4G16_F16: return tc ? launch_gemm_tc<2>(w, x, (int)m, y, st, di) : gemm_by_gemv<2>(w, x, m, y, st, di);
+    default: return tc ? launch_gemm_tc<3>(w, x, (int)m, y, st, di) : gemm_by_gemv<3>(w, x, m, y, st, di);
+  }
+}
+
+static size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+static qmm_status check_routing(const int32_t* ids, int64_t t, int64_t topk, int64_t num_experts) {
+  if (t < 0 || topk < 0 || num_experts < 1) return QMM_ERR_INVALID_ARG;
+  if (num_experts > kRouteMaxExperts || t * topk > INT32_MAX / 2) return QMM_ERR_UNSUPPORTED_SHAPE;
+  if (t * topk > 0 && !ids) return QMM_ERR_INVALID_ARG;
+  if (ids && !aligned16(ids)) return QMM_ERR_MISALIGNED;
+  return QMM_OK;
+}
+
+qmm_status qmm_route(const int32_t* topk_ids, int64_t t, int64_t topk, int64_t num_experts, int32_t* expert_offsets,
+                     int32_t* pair_perm, void* ws, size_t ws_bytes, void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  qmm_status s = check_routing(topk_ids, t, topk, num_experts);
+  if (s != QMM_OK) return s;
+  if (!expert_offsets || (t * topk > 0 && !pair_perm)) return QMM_ERR_INVALID_ARG;
+  if (!aligned16(expert_offsets) || (pair_perm && !aligned16(pair_perm))) return QMM_ERR_MISALIGNED;
+  DevInfo* di = nullptr;
+  if ((s = device_info(&di)) != QMM_OK) return s;
+  route_kernel<<<1, kRouteThreads, 0, static_cast<cudaStream_t>(stream)>>>(topk_ids, (int)(t * topk),
+                                                                          (int)num_experts, expert_offsets, pair_perm);
+  set_variant("route_stable_counting_sort");
+  return launch_status();
+}
+
+static qmm_status check_expert_strides(const qmm_weights* w) {
+  const size_t db = qmm_data_bytes(w->fmt, w->n, w->k), sb = qmm_scale_bytes(w->fmt, w->n, w->k);
+  if (w->num_experts > 1) {
+    if (w->expert_data_stride < (int64_t)db || (sb && w->expert_scale_stride < (int64_t)sb)) return QMM_ERR_INVALID_ARG;
+    if ((w->expert_data_stride & 15) || (sb && (w->expert_scale_stride & 15))) return QMM_ERR_MISALIGNED;
+  }
+  return QMM_OK;
+}
+
+qmm_status qmm_grouped_gemv(const qmm_weights* experts, const uint16_t* x, int32_t x_per_pair, const int32_t* topk_ids,
+                            int64_t t, int64_t topk, uint16_t* y, void* ws, size_t ws_bytes, void* stream) {
+  qmm_status s = check_weights(experts, true);
+  if (s != QMM_OK) return s;
+  if ((s = check_expert_strides(experts)) != QMM_OK) return s;
+  if ((s = check_routing(topk_ids, t, topk, experts->num_experts)) != QMM_OK) return s;
+  if (x_per_pair != 0 && x_per_pair != 1) return QMM_ERR_INVALID_ARG;
+  DevInfo* di = nullptr;
+  if ((s = device_info(&di)) != QMM_OK) return s;
+  const int64_t P = t * topk;
+  if (P == 0 || experts->n == 0) return QMM_OK;
+  if (!y || (experts->k > 0 && !x)) return QMM_ERR_INVALID_ARG;
+  if (!aligned16(y) || (x && !aligned16(x))) return QMM_ERR_MISALIGNED;
+  const size_t need = qmm_workspace_bytes(QMM_OP_GROUPED, experts, 0, t, topk);
+  if (!ws || ws_bytes < need) return QMM_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QMM_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t* offsets = static_cast<int32_t*>(ws);
+  int32_t* perm = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + align256(4 * (size_t)(experts->num_experts + 1)));
+  route_kernel<<<1, kRouteThreads, 0, st>>>(topk_ids, (int)P, (int)experts->num_experts, offsets, perm);
+  if (cudaGetLastError() != cudaSuccess) return QMM_ERR_CUDA;
+  if (experts->k == 0) {
+    // every routed pair's row is an empty sum
+    zero_fill_kernel<<<grid_for(P * experts->n, 256, di->sms), 256, 0, st>>>(y, P * experts->n);
+    set_variant("route+zero_fill");
+    return launch_status();
+  }
+  switch (experts->fmt) {
+    case QMM_FMT_IQ4_NL: s = launch_grouped<1>(experts, x, x_per_pair, topk, offsets, perm, y, st); break;
+    case QMM_FMT_FP4G16_F16: s = launch_grouped<2>(experts, x, x_per_pair, topk, offsets, perm, y, st); break;
+    default: s = launch_grouped<3>(experts, x, x_per_pair, topk, offsets, perm, y, st); break;
+  }
+  set_variant("route+grouped_gemv_generic<fmt=%d>", experts->fmt);
+  return s;
+}
+
+size_t qmm_workspace_bytes(int32_t op, const qmm_weights* w, int64_t m, int64_t t, int64_t topk) {
+  if (op == QMM_OP_GROUPED) {
+    if (!w || w->num_experts < 1 || t < 0 || topk < 0) return 0;
+    return align256(4 * (size_t)(w->num_experts + 1)) + align256(4 * (size_t)(t * topk));
+  }
+  (void)m;
+  return 0;
+}
+
+qmm_status qmm_sync_check(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return QMM_ERR_CUDA;
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_err_word, sizeof(v)) != cudaSuccess) return QMM_ERR_CUDA;
+  if (v == 0) return QMM_OK;
+  if (cudaMemcpyToSymbol(g_err_word, &zero, sizeof(zero)) != cudaSuccess) return QMM_ERR_CUDA;
+  if (v & ERR_TIMEOUT) return QMM_ERR_TIMEOUT;
+  return QMM_ERR_DEVICE_FAULT;
+}
+
+}  // extern "C"

@@ -1,0 +1,215 @@
+"""ctypes binding of libqmm.so (include/qmm.h).
+
+Argument marshalling only: every function here takes torch tensors, checks
+that they are CUDA tensors of the right element size, passes raw device
+pointers and the current CUDA stream to the C ABI, and raises ``QmmError`` on
+a non-OK status.  No arithmetic of the path happens in Python, and there is
+no fallback: if the library is missing the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+from . import _build
+
+FMT_IQ4_NL = 1
+FMT_FP4G16_F16 = 2
+FMT_FP4G16_E4M3 = 3
+
+OP_DEQUANT, OP_GEMV, OP_GEMM, OP_ROUTE, OP_GROUPED = 0, 1, 2, 3, 4
+
+STATUS = {0: "QMM_OK", 1: "QMM_ERR_INVALID_ARG", 2: "QMM_ERR_UNSUPPORTED_SHAPE", 3: "QMM_ERR_MISALIGNED",
+          4: "QMM_ERR_NOT_SM100", 5: "QMM_ERR_CUDA", 6: "QMM_ERR_TIMEOUT", 7: "QMM_ERR_DEVICE_FAULT",
+          8: "QMM_ERR_WORKSPACE"}
+
+
+class QmmError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__("%s: %s (%s)" % (where, STATUS.get(status, status), _lib().qmm_status_string(status).decode()))
+
+
+class qmm_weights(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int32), ("reserved", ctypes.c_int32), ("n", ctypes.c_int64), ("k", ctypes.c_int64),
+                ("data", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("global_scale", ctypes.c_float),
+                ("reserved2", ctypes.c_int32), ("num_experts", ctypes.c_int64),
+                ("expert_data_stride", ctypes.c_int64), ("expert_scale_stride", ctypes.c_int64)]
+
+
+_L = None
+LIB_PATH = _build.LIB
+
+
+def _lib():
+    global _L
+    if _L is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libqmm.so is not built (expected at %s); run __graft_entry__.build()" % LIB_PATH)
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+        W = ctypes.POINTER(qmm_weights)
+        sigs = {
+            "qmm_data_bytes": (sz, [i32, i64, i64]),
+            "qmm_scale_bytes": (sz, [i32, i64, i64]),
+            "qmm_packed_bytes": (sz, [i32, i64, i64]),
+            "qmm_dequant": (i32, [W, vp, vp]),
+            "qmm_gemv": (i32, [W, vp, i64, vp, vp, sz, vp]),
+            "qmm_gemm": (i32, [W, vp, i64, vp, vp, sz, vp]),
+            "qmm_route": (i32, [vp, i64, i64, i64, vp, vp, vp, sz, vp]),
+            "qmm_grouped_gemv": (i32, [W, vp, i32, vp, i64, i64, vp, vp, sz, vp]),
+            "qmm_workspace_bytes": (sz, [i32, W, i64, i64, i64]),
+            "qmm_sync_check": (i32, [vp]),
+            "qmm_status_string": (ctypes.c_char_p, [i32]),
+            "qmm_last_variant": (ctypes.c_char_p, []),
+            "qmm_version": (ctypes.c_char_p, []),
+        }
+        for name, (res, args) in sigs.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _L = L
+    return _L
+
+
+def lib():
+    return _lib()
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise QmmError(status, where)
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: torch.Tensor | None, esize: int | None = None, name: str = "tensor"):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if esize is not None and t.element_size() != esize:
+        raise ValueError("%s must have %d-byte elements" % (name, esize))
+    return ctypes.c_void_p(t.data_ptr())
+
+
+@dataclass
+class PackedWeights:
+    """Device tensors of one packed matrix (or expert stack) plus its C descriptor."""
+    fmt: int
+    n: int
+    k: int
+    data: torch.Tensor
+    scales: torch.Tensor | None
+    global_scale: float = 1.0
+    experts: int = 1
+
+    def desc(self) -> qmm_weights:
+        d = qmm_weights()
+        d.fmt, d.reserved, d.n, d.k = self.fmt, 0, self.n, self.k
+        d.data = ctypes.c_void_p(self.data.data_ptr()) if self.data is not None else None
+        d.scales = ctypes.c_void_p(self.scales.data_ptr()) if self.scales is not None else None
+        d.global_scale, d.reserved2, d.num_experts = float(self.global_scale), 0, self.experts
+        d.expert_data_stride = self.data.numel() // self.experts if self.data is not None else 0
+        d.expert_scale_stride = (self.scales.numel() * self.scales.element_size() // self.experts
+                                 if self.scales is not None else 0)
+        return d
+
+    @property
+    def nbytes(self) -> int:
+        return self.data.numel() + (0 if self.scales is None else self.scales.numel() * self.scales.element_size())
+
+    @staticmethod
+    def from_host(p, device="cuda") -> "PackedWeights":
+        """From a ``synth.Packed`` (numpy bytes) to device tensors."""
+        data = torch.from_numpy(p.data).to(device)
+        scales = None if p.scales is None else torch.from_numpy(p.scales).to(device)
+        return PackedWeights(p.fmt, p.n, p.k, data, scales, p.global_scale, p.experts)
+
+
+# ---------------------------------------------------------------------------
+# Entry points (same names as the C ABI)
+# ---------------------------------------------------------------------------
+def qmm_data_bytes(fmt: int, n: int, k: int) -> int:
+    return _lib().qmm_data_bytes(fmt, n, k)
+
+
+def qmm_scale_bytes(fmt: int, n: int, k: int) -> int:
+    return _lib().qmm_scale_bytes(fmt, n, k)
+
+
+def qmm_packed_bytes(fmt: int, n: int, k: int) -> int:
+    return _lib().qmm_packed_bytes(fmt, n, k)
+
+
+def qmm_workspace_bytes(op: int, w: PackedWeights | None, m: int = 0, t: int = 0, topk: int = 0) -> int:
+    d = w.desc() if w is not None else None
+    return _lib().qmm_workspace_bytes(op, ctypes.byref(d) if d is not None else None, m, t, topk)
+
+
+def qmm_dequant(w: PackedWeights, out: torch.Tensor, stream=None) -> torch.Tensor:
+    d = w.desc()
+    _check(_lib().qmm_dequant(ctypes.byref(d), _ptr(out, 2, "out"), _stream(stream)), "qmm_dequant")
+    return out
+
+
+def _ws(ws):
+    return (_ptr(ws, None, "ws"), 0 if ws is None else ws.numel() * ws.element_size())
+
+
+def qmm_gemv(w: PackedWeights, x: torch.Tensor, y: torch.Tensor, ws: torch.Tensor | None = None,
+             stream=None) -> torch.Tensor:
+    d = w.desc()
+    wp, wb = _ws(ws)
+    m = x.shape[0] if x.dim() == 2 else 1
+    _check(_lib().qmm_gemv(ctypes.byref(d), _ptr(x, 2, "x"), m, _ptr(y, 2, "y"), wp, wb, _stream(stream)), "qmm_gemv")
+    return y
+
+
+def qmm_gemm(w: PackedWeights, x: torch.Tensor, y: torch.Tensor, ws: torch.Tensor | None = None,
+             stream=None) -> torch.Tensor:
+    d = w.desc()
+    wp, wb = _ws(ws)
+    _check(_lib().qmm_gemm(ctypes.byref(d), _ptr(x, 2, "x"), x.shape[0], _ptr(y, 2, "y"), wp, wb, _stream(stream)),
+           "qmm_gemm")
+    return y
+
+
+def qmm_route(topk_ids: torch.Tensor, num_experts: int, offsets: torch.Tensor, perm: torch.Tensor,
+              ws: torch.Tensor | None = None, stream=None):
+    t, topk = topk_ids.shape
+    wp, wb = _ws(ws)
+    _check(_lib().qmm_route(_ptr(topk_ids, 4, "topk_ids"), t, topk, num_experts, _ptr(offsets, 4, "offsets"),
+                            _ptr(perm, 4, "perm"), wp, wb, _stream(stream)), "qmm_route")
+    return offsets, perm
+
+
+def qmm_grouped_gemv(w: PackedWeights, x: torch.Tensor, topk_ids: torch.Tensor, y: torch.Tensor,
+                     x_per_pair: bool = False, ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    d = w.desc()
+    t, topk = topk_ids.shape
+    wp, wb = _ws(ws)
+    _check(_lib().qmm_grouped_gemv(ctypes.byref(d), _ptr(x, 2, "x"), int(bool(x_per_pair)),
+                                   _ptr(topk_ids, 4, "topk_ids"), t, topk, _ptr(y, 2, "y"), wp, wb,
+                                   _stream(stream)), "qmm_grouped_gemv")
+    return y
+
+
+def qmm_sync_check(stream=None) -> int:
+    return _lib().qmm_sync_check(_stream(stream))
+
+
+def qmm_last_variant() -> str:
+    return _lib().qmm_last_variant().decode()
+
+
+def qmm_version() -> str:
+    return _lib().qmm_version().decode()

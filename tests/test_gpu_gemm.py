@@ -1,0 +1,89 @@
+"""GPU parity: qmm_gemm (tcgen05 prefill GEMM) against the oracle within
+|y - y_ref| <= 1e-3 * sum_k |w_k x_k| (+2^-24), plus exact special cases."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import check_tol, dev, from_dev_u16, nz, to_dev_u16
+from packed_bit_weight_b200 import qmm, synth
+
+pytestmark = pytest.mark.gpu
+
+
+def run_gemm(w, x_bits, canary=64):
+    m = x_bits.shape[0]
+    x = to_dev_u16(x_bits)
+    yb = torch.full((m * w.n + canary,), 0x5A5A, dtype=torch.int16, device="cuda")
+    y = yb[: m * w.n].view(m, w.n)
+    qmm.qmm_gemm(w, x, y)
+    st = qmm.qmm_sync_check()
+    assert st == 0, "qmm_sync_check -> %s" % qmm.STATUS.get(st, st)
+    assert bool((yb[m * w.n:] == 0x5A5A).all()), "write past the end of y"
+    return from_dev_u16(y)
+
+
+@pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3])
+@pytest.mark.parametrize("m,n,k", [(128, 256, 64), (128, 256, 256), (256, 384, 512), (200, 300, 1024),
+                                   (64, 128, 128), (384, 1000, 2048)])
+def test_gemm_vs_oracle(fmt, m, n, k):
+    rng = np.random.default_rng(500 + m + n + k + fmt)
+    p = synth.gen_fp4(rng, n, k, fmt)
+    x = synth.gen_x(rng, m, k)
+    y = run_gemm(dev(p), x)
+    assert qmm.qmm_last_variant().startswith("gemm_fp4_tc"), qmm.qmm_last_variant()
+    yref, absy = oracle.matmul(fmt, n, k, p.data, p.scales, p.global_scale, x)
+    check_tol(y, yref, absy, "gemm m=%d n=%d k=%d" % (m, n, k))
+
+
+@pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3])
+def test_gemm_identity_rows_give_decoded_weights(fmt):
+    """X = [I | 0]: row i of Y is column i of the decoded W, bit-exactly."""
+    rng = np.random.default_rng(9)
+    m, n, k = 128, 512, 256
+    p = synth.gen_fp4(rng, n, k, fmt)
+    x = np.zeros((m, k), dtype=np.uint16)
+    x[np.arange(m), np.arange(m)] = 0x3C00
+    y = run_gemm(dev(p), x)
+    deq = oracle.dequant(fmt, n, k, p.data, p.scales, p.global_scale)
+    # a sum that starts from +0 returns +0 for a -0 weight: compare values
+    # bit-exactly with the sign of zero normalised
+    assert np.array_equal(nz(y), nz(deq[:, :m].T))
+
+
+def test_gemm_small_m_uses_decode_kernel_and_agrees():
+    rng = np.random.default_rng(4)
+    p = synth.gen_fp4(rng, 300, 512)
+    x = synth.gen_x(rng, 20, 512)
+    y = run_gemm(dev(p), x)
+    assert qmm.qmm_last_variant().startswith("gemm_by_gemv")
+    yref, absy = oracle.matmul(p.fmt, p.n, p.k, p.data, p.scales, 1.0, x)
+    check_tol(y, yref, absy, "small m")
+
+
+def test_gemm_iq4nl():
+    rng = np.random.default_rng(6)
+    p = synth.gen_iq4nl(rng, 100, 256)
+    x = synth.gen_x(rng, 40, 256)
+    y = run_gemm(dev(p), x)
+    yref, absy = oracle.matmul(p.fmt, p.n, p.k, p.data, None, 1.0, x)
+    check_tol(y, yref, absy, "iq4 gemm")
+
+
+@pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3])
+def test_config5_prefill_full_size_sampled(fmt):
+    p, x = synth.make_prefill(fmt)
+    w = dev(p)
+    y = run_gemm(w, x)
+    assert qmm.qmm_last_variant().startswith("gemm_fp4_tc")
+    rng = np.random.default_rng(44)
+    mi = np.concatenate([[0, 0, p.k and 2047, 2047], rng.integers(0, 2048, 1500)])
+    ri = np.concatenate([[0, p.n - 1, 0, p.n - 1], rng.integers(0, p.n, 1500)])
+    # plus one full row and one full column of the output
+    ys, as_ = oracle.matmul_sampled(p.fmt, p.n, p.k, p.data, p.scales, p.global_scale, x, mi, ri)
+    check_tol(y[mi, ri], ys, as_, "prefill sampled")
+    col = np.full(2048, 18559)
+    ys, as_ = oracle.matmul_sampled(p.fmt, p.n, p.k, p.data, p.scales, p.global_scale, x, np.arange(2048), col)
+    check_tol(y[np.arange(2048), col], ys, as_, "prefill last column")
+    y2 = run_gemm(w, x)
+    assert np.array_equal(y, y2)  # deterministic

@@ -1,0 +1,109 @@
+"""GPU parity: qmm_gemv against the oracle within |y - y_ref| <= 1e-3 *
+sum_k |w_k x_k| (+2^-24), plus exact special cases and edge cases."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import check_tol, dev, from_dev_u16, nz, run_gemv, to_dev_u16
+from packed_bit_weight_b200 import qmm, synth
+
+pytestmark = pytest.mark.gpu
+
+FMTS = [synth.FMT_IQ4_NL, synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3]
+
+
+def _case(fmt, n, k, m, seed):
+    rng = np.random.default_rng(seed)
+    p = synth.gen_weights(rng, fmt, n, k)
+    x = synth.gen_x(rng, m, k)
+    return p, x
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("n,k,m", [(1, 32, 1), (37, 64, 1), (256, 512, 1), (100, 160, 3), (64, 1024, 8),
+                                   (45, 2048, 9), (1000, 2048, 1), (1000, 2048, 5), (999, 4096, 16),
+                                   (2000, 4096, 4)])
+def test_gemv_vs_oracle(fmt, n, k, m):
+    p, x = _case(fmt, n, k, m, 1000 + n + k + m + fmt)
+    w = dev(p)
+    y = run_gemv(w, x)
+    yref, absy = oracle.matmul(fmt, n, k, p.data, p.scales, p.global_scale, x)
+    check_tol(y, yref, absy, "%s n=%d k=%d m=%d [%s]" % (fmt, n, k, m, qmm.qmm_last_variant()))
+
+
+def test_fast_path_is_used_for_streaming_shapes():
+    p, x = _case(synth.FMT_FP4G16_F16, 1000, 4096, 1, 5)
+    run_gemv(dev(p), x)
+    assert qmm.qmm_last_variant().startswith("gemv_fp4_tma")
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_one_hot_gives_the_decoded_column_bit_exactly(fmt):
+    n, k = 300, 4096
+    p, _ = _case(fmt, n, k, 1, 77)
+    w = dev(p)
+    deq = oracle.dequant(fmt, n, k, p.data, p.scales, p.global_scale)
+    for col in (0, 1, 777, 4095):
+        x = np.zeros((1, k), dtype=np.uint16)
+        x[0, col] = 0x3C00
+        y = run_gemv(w, x)
+        assert np.array_equal(nz(y[0]), nz(deq[:, col])), (fmt, col, qmm.qmm_last_variant())
+
+
+@pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3])
+def test_config2_in_proj_full(fmt):
+    p, x = synth.make_gemv(synth.FP4_IN_PROJ, fmt)
+    w = dev(p)
+    y = run_gemv(w, x)
+    assert qmm.qmm_last_variant().startswith("gemv_fp4_tma")
+    yref, absy = oracle.matmul(fmt, p.n, p.k, p.data, p.scales, p.global_scale, x)
+    check_tol(y, yref, absy, "in_proj")
+    y2 = run_gemv(w, x)
+    assert np.array_equal(y, y2)                      # deterministic
+
+
+def test_config1_iq4nl_tiny():
+    p, x = synth.make_gemv(synth.IQ4_TINY)
+    y = run_gemv(dev(p), x)
+    yref, absy = oracle.matmul(p.fmt, p.n, p.k, p.data, None, 1.0, x)
+    check_tol(y, yref, absy, "iq4 tiny")
+
+
+@pytest.mark.parametrize("m", [1, 4, 16])
+def test_config3_sweep(m):
+    mats = synth.make_sweep()
+    rng = np.random.default_rng(31 + m)
+    for name, (p, xall) in mats.items():
+        x = xall[:m]
+        w = dev(p)
+        y = run_gemv(w, x)
+        if p.n <= 4096:
+            yref, absy = oracle.matmul(p.fmt, p.n, p.k, p.data, p.scales, p.global_scale, x)
+            check_tol(y, yref, absy, name)
+        else:  # LM head: sampled outputs, first and last rows included
+            ri = np.concatenate([[0, p.n - 1], rng.integers(0, p.n, 600)])
+            mi = rng.integers(0, m, ri.size)
+            ys, as_ = oracle.matmul_sampled(p.fmt, p.n, p.k, p.data, p.scales, p.global_scale, x, mi, ri)
+            check_tol(y[mi, ri], ys, as_, name)
+        del w
+
+
+def test_gemv_edge_cases():
+    p, x = _case(synth.FMT_FP4G16_F16, 64, 256, 2, 3)
+    w = dev(p)
+    xd = to_dev_u16(x)
+    y = torch.zeros((2, 64), dtype=torch.int16, device="cuda")
+    qmm.qmm_gemv(w, xd[:0], y[:0])                                    # m = 0: no-op
+    with pytest.raises(qmm.QmmError) as e:                              # m = 17
+        qmm.qmm_gemv(w, torch.zeros((17, 256), dtype=torch.int16, device="cuda"),
+                     torch.zeros((17, 64), dtype=torch.int16, device="cuda"))
+    assert e.value.status == 2
+    wk0 = qmm.PackedWeights(w.fmt, 64, 0, w.data, w.scales)            # k = 0: y = 0
+    y.fill_(77)
+    qmm.qmm_gemv(wk0, xd[:, :0].contiguous(), y)
+    assert qmm.qmm_sync_check() == 0 and bool((y == 0).all())
+    yb = torch.zeros((2 * 64 + 8,), dtype=torch.int16, device="cuda")
+    with pytest.raises(qmm.QmmError) as e:
+        qmm.qmm_gemv(w, xd, yb[1:129].view(2, 64))                      # misaligned y
+    assert e.value.status == 3

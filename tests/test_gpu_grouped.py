@@ -1,0 +1,108 @@
+"""GPU parity: routing bucket sort (exact) and the routed-expert grouped GEMV
+against the oracle (tolerance as for the GEMV)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import check_tol, dev, from_dev_u16, to_dev_u16
+from packed_bit_weight_b200 import qmm, synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _route_gpu(ids, E):
+    t, topk = ids.shape
+    d_ids = torch.from_numpy(ids).cuda()
+    off = torch.full((E + 1,), -7, dtype=torch.int32, device="cuda")
+    perm = torch.full((max(1, t * topk),), -7, dtype=torch.int32, device="cuda")
+    qmm.qmm_route(d_ids, E, off, perm)
+    st = qmm.qmm_sync_check()
+    return off.cpu().numpy(), perm.cpu().numpy()[: t * topk], st
+
+
+@pytest.mark.parametrize("t,topk,E", [(64, 4, 32), (1, 1, 1), (7, 3, 5), (3000, 4, 32), (1024, 8, 256), (5, 2, 200)])
+def test_route_matches_oracle(t, topk, E):
+    rng = np.random.default_rng(t * 7 + E)
+    ids = synth.gen_topk(rng, t, topk, E)
+    off, perm, st = _route_gpu(ids, E)
+    assert st == 0
+    ooff, operm, bad = oracle.route(ids, E)
+    assert bad == 0
+    assert np.array_equal(off, ooff)
+    assert np.array_equal(perm, operm)        # the GPU sort is stable too
+
+
+def test_route_flags_out_of_range_ids():
+    ids = synth.gen_topk(np.random.default_rng(1), 16, 2, 8)
+    ids[3, 1] = 8
+    ids[0, 0] = -2
+    off, perm, st = _route_gpu(ids, 8)
+    assert st == 7  # QMM_ERR_DEVICE_FAULT
+    ooff, operm, bad = oracle.route(ids, 8)
+    assert bad == 2 and np.array_equal(off, ooff) and np.array_equal(perm[: off[8]], operm[: ooff[8]])
+
+
+def _grouped(w, x_bits, ids, x_per_pair):
+    t, topk = ids.shape
+    x = to_dev_u16(x_bits)
+    d_ids = torch.from_numpy(ids).cuda()
+    y = torch.full((t, topk, w.n), 0x5A5A, dtype=torch.int16, device="cuda")
+    nb = qmm.qmm_workspace_bytes(qmm.OP_GROUPED, w, 0, t, topk)
+    ws = torch.empty((nb,), dtype=torch.uint8, device="cuda")
+    qmm.qmm_grouped_gemv(w, x, d_ids, y, x_per_pair=x_per_pair, ws=ws)
+    st = qmm.qmm_sync_check()
+    return from_dev_u16(y), st
+
+
+@pytest.mark.parametrize("fmt", [synth.FMT_IQ4_NL, synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3])
+@pytest.mark.parametrize("E,n,k,t,topk,per_pair", [(6, 40, 64, 9, 2, False), (4, 33, 256, 70, 3, True),
+                                                    (8, 128, 512, 3, 4, False)])
+def test_grouped_vs_oracle(fmt, E, n, k, t, topk, per_pair):
+    rng = np.random.default_rng(E * 100 + n + k + fmt)
+    p = synth.gen_weights(rng, fmt, n, k, experts=E)
+    x = synth.gen_x(rng, t, topk, k) if per_pair else synth.gen_x(rng, t, k)
+    ids = synth.gen_topk(rng, t, topk, E)
+    y, st = _grouped(dev(p), x, ids, per_pair)
+    assert st == 0
+    if per_pair:
+        yref = np.empty((t, topk, n)); absy = np.empty((t, topk, n))
+        for s in range(topk):
+            for tok in range(t):
+                e = ids[tok, s]
+                de = p.data[e * p.data_stride:(e + 1) * p.data_stride]
+                se = None if p.scales is None else p.scales[e * p.scale_stride:(e + 1) * p.scale_stride]
+                yy, aa = oracle.matmul(fmt, n, k, de, se, p.global_scale, x[tok, s][None])
+                yref[tok, s], absy[tok, s] = yy[0], aa[0]
+    else:
+        yref, absy = oracle.grouped_gemv(fmt, n, k, p.data, p.data_stride, p.scales, p.scale_stride,
+                                         p.global_scale, E, x, ids)
+    check_tol(y, yref, absy, "grouped %s" % qmm.qmm_last_variant())
+
+
+def test_config4_experts_sampled():
+    wgu, wdn, x_gu, x_dn, ids = synth.make_experts()
+    for w, x, per_pair in ((wgu, x_gu, False), (wdn, x_dn, True)):
+        y, st = _grouped(dev(w), x, ids, per_pair)
+        assert st == 0
+        rng = np.random.default_rng(8)
+        for tok in rng.integers(0, 64, 6):
+            for s in range(4):
+                e = ids[tok, s]
+                de = w.data[e * w.data_stride:(e + 1) * w.data_stride]
+                xr = x[tok, s][None] if per_pair else x[tok][None]
+                rows = rng.integers(0, w.n, 64)
+                ys, as_ = oracle.matmul_sampled(w.fmt, w.n, w.k, de, None, 1.0, xr, np.zeros(64, np.int64), rows)
+                check_tol(y[tok, s, rows], ys, as_, "config4")
+
+
+def test_grouped_rejects_small_workspace():
+    rng = np.random.default_rng(2)
+    p = synth.gen_iq4nl(rng, 32, 64, experts=4)
+    w = dev(p)
+    ids = torch.from_numpy(synth.gen_topk(rng, 8, 2, 4)).cuda()
+    x = to_dev_u16(synth.gen_x(rng, 8, 64))
+    y = torch.empty((8, 2, 32), dtype=torch.int16, device="cuda")
+    with pytest.raises(qmm.QmmError) as e:
+        qmm.qmm_grouped_gemv(w, x, ids, y, ws=torch.empty((16,), dtype=torch.uint8, device="cuda"))
+    assert e.value.status == 8
