@@ -30,8 +30,9 @@
  * Conventions shared by every entry point:
  *   - Every pointer argument marked "device" must point to GPU global memory
  *     of the current device; the caller allocates and owns all of it.  The
- *     library allocates nothing on the device except its fixed error word and
- *     keeps no pointer after a call returns.
+ *     library allocates nothing on the device; its only device memory is its
+ *     fixed error word and the fixed scratch array of
+ *     qmm_grouped_gemv_noalloc, and it keeps no pointer after a call returns.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream); all work
  *     is enqueued on it and the call returns without synchronising.
  *   - Argument checks happen on the host before anything is enqueued; on
@@ -166,6 +167,33 @@ qmm_status qmm_route(const int32_t* topk_ids, int64_t t, int64_t topk, int64_t n
 qmm_status qmm_grouped_gemv(const qmm_weights* experts, const uint16_t* x, int32_t x_per_pair,
                             const int32_t* topk_ids, int64_t t, int64_t topk, uint16_t* y, void* ws,
                             size_t ws_bytes, void* stream);
+
+/* Allocation-free variant of qmm_grouped_gemv.  The pages have no
+ * counterpart: this entry point exists for callers that cannot allocate
+ * device memory, so cannot supply the routing workspace qmm_grouped_gemv
+ * asks for -- for example a host runtime that hands out all device memory
+ * from its own fixed pool and forbids other allocations, or a latency-bound
+ * serving loop that must not block in the allocator.
+ *
+ * Same arguments and result as qmm_grouped_gemv, minus the workspace.  The
+ * routing offsets and pair permutation live instead in one fixed array of
+ * the library's own device memory (258 KiB, held by every GPU that loads the
+ * library until the process exits).  Limits: t*topk <= 65536 pairs and
+ * num_experts <= 256; larger calls return QMM_ERR_UNSUPPORTED_SHAPE and
+ * launch nothing.  The call allocates nothing: no cudaMalloc, no cudaFree, no
+ * allocating library routine.
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and caches it; make that
+ * first call before any stream capture.  Every call on a device uses the
+ * same array and it keeps the last call's contents (each call rewrites every
+ * entry it reads, so nothing needs clearing): two calls whose kernels
+ * overlap on the GPU -- on different streams, or from different host
+ * threads -- race on it and must be serialised by the caller.
+ * Errors: as qmm_grouped_gemv, except QMM_ERR_WORKSPACE. */
+qmm_status qmm_grouped_gemv_noalloc(const qmm_weights* experts, const uint16_t* x, int32_t x_per_pair,
+                                    const int32_t* topk_ids, int64_t t, int64_t topk, uint16_t* y,
+                                    void* stream);
 
 enum { QMM_OP_DEQUANT = 0, QMM_OP_GEMV = 1, QMM_OP_GEMM = 2, QMM_OP_ROUTE = 3, QMM_OP_GROUPED = 4 };
 

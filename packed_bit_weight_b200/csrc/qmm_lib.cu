@@ -234,6 +234,33 @@ static qmm_status launch_grouped(const qmm_weights* w, const uint16_t* x, int x_
   return launch_status();
 }
 
+// ---------------------------------------------------------------------------
+// Fixed device scratch for qmm_grouped_gemv_noalloc
+// ---------------------------------------------------------------------------
+// Routing offsets (first kNoAllocOffsetInts words) and the pair permutation
+// (next kNoAllocMaxPairs words) for callers that cannot hand the library a
+// workspace.  Every GPU that loads the library holds this array (258 KiB)
+// until the process exits; all calls on a device share it.
+constexpr int64_t kNoAllocMaxPairs = 65536;
+constexpr int kNoAllocOffsetInts = 512;  // >= kRouteMaxExperts + 1; keeps the permutation 256-byte aligned
+static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocOffsetInts + kNoAllocMaxPairs];
+static int32_t* g_noalloc_addr[64];  // device address of g_noalloc_scratch, per device
+
+// The host-side name g_noalloc_scratch is only a stand-in; the kernels need
+// the device address, fetched once per device with that device current.
+static qmm_status noalloc_scratch(int32_t** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return QMM_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return QMM_ERR_CUDA;
+    g_noalloc_addr[dev] = static_cast<int32_t*>(p);
+  }
+  *out = g_noalloc_addr[dev];
+  return QMM_OK;
+}
+
 }  // namespace qmm
 
 using namespace qmm;
@@ -434,6 +461,43 @@ size_t qmm_workspace_bytes(int32_t op, const qmm_weights* w, int64_t m, int64_t 
   }
   (void)m;
   return 0;
+}
+
+qmm_status qmm_grouped_gemv_noalloc(const qmm_weights* experts, const uint16_t* x, int32_t x_per_pair,
+                                    const int32_t* topk_ids, int64_t t, int64_t topk, uint16_t* y, void* stream) {
+  qmm_status s = check_weights(experts, true);
+  if (s != QMM_OK) return s;
+  if ((s = check_expert_strides(experts)) != QMM_OK) return s;
+  if ((s = check_routing(topk_ids, t, topk, experts->num_experts)) != QMM_OK) return s;
+  if (x_per_pair != 0 && x_per_pair != 1) return QMM_ERR_INVALID_ARG;
+  if (t * topk > kNoAllocMaxPairs) return QMM_ERR_UNSUPPORTED_SHAPE;  // beyond the fixed scratch
+  DevInfo* di = nullptr;
+  if ((s = device_info(&di)) != QMM_OK) return s;
+  const int64_t P = t * topk;
+  if (P == 0 || experts->n == 0) return QMM_OK;
+  if (!y || (experts->k > 0 && !x)) return QMM_ERR_INVALID_ARG;
+  if (!aligned16(y) || (x && !aligned16(x))) return QMM_ERR_MISALIGNED;
+  int32_t* scratch = nullptr;
+  if ((s = noalloc_scratch(&scratch)) != QMM_OK) return s;
+  // The routing kernel rewrites offsets[0..E] and every permutation slot the
+  // grouped kernel reads, so nothing in the shared array has to be cleared.
+  int32_t* offsets = scratch;
+  int32_t* perm = scratch + kNoAllocOffsetInts;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  route_kernel<<<1, kRouteThreads, 0, st>>>(topk_ids, (int)P, (int)experts->num_experts, offsets, perm);
+  if (cudaGetLastError() != cudaSuccess) return QMM_ERR_CUDA;
+  if (experts->k == 0) {
+    zero_fill_kernel<<<grid_for(P * experts->n, 256, di->sms), 256, 0, st>>>(y, P * experts->n);
+    set_variant("noalloc:route+zero_fill");
+    return launch_status();
+  }
+  switch (experts->fmt) {
+    case QMM_FMT_IQ4_NL: s = launch_grouped<1>(experts, x, x_per_pair, topk, offsets, perm, y, st); break;
+    case QMM_FMT_FP4G16_F16: s = launch_grouped<2>(experts, x, x_per_pair, topk, offsets, perm, y, st); break;
+    default: s = launch_grouped<3>(experts, x, x_per_pair, topk, offsets, perm, y, st); break;
+  }
+  set_variant("noalloc:route+grouped_gemv_generic<fmt=%d>", experts->fmt);
+  return s;
 }
 
 qmm_status qmm_sync_check(void* stream) {

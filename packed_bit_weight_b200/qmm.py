@@ -61,6 +61,7 @@ def _lib():
             "qmm_gemm": (i32, [W, vp, i64, vp, vp, sz, vp]),
             "qmm_route": (i32, [vp, i64, i64, i64, vp, vp, vp, sz, vp]),
             "qmm_grouped_gemv": (i32, [W, vp, i32, vp, i64, i64, vp, vp, sz, vp]),
+            "qmm_grouped_gemv_noalloc": (i32, [W, vp, i32, vp, i64, i64, vp, vp]),
             "qmm_workspace_bytes": (sz, [i32, W, i64, i64, i64]),
             "qmm_sync_check": (i32, [vp]),
             "qmm_status_string": (ctypes.c_char_p, [i32]),
@@ -200,6 +201,19 @@ def qmm_grouped_gemv(w: PackedWeights, x: torch.Tensor, topk_ids: torch.Tensor, 
     _check(_lib().qmm_grouped_gemv(ctypes.byref(d), _ptr(x, 2, "x"), int(bool(x_per_pair)),
                                    _ptr(topk_ids, 4, "topk_ids"), t, topk, _ptr(y, 2, "y"), wp, wb,
                                    _stream(stream)), "qmm_grouped_gemv")
+    return y
+
+
+def qmm_grouped_gemv_noalloc(w: PackedWeights, x: torch.Tensor, topk_ids: torch.Tensor, y: torch.Tensor,
+                             x_per_pair: bool = False, stream=None) -> torch.Tensor:
+    """qmm_grouped_gemv without a workspace: the routing scratch is the
+    library's own fixed device array (at most 65536 pairs, 256 experts; calls
+    that overlap on the GPU race on it)."""
+    d = w.desc()
+    t, topk = topk_ids.shape
+    _check(_lib().qmm_grouped_gemv_noalloc(ctypes.byref(d), _ptr(x, 2, "x"), int(bool(x_per_pair)),
+                                           _ptr(topk_ids, 4, "topk_ids"), t, topk, _ptr(y, 2, "y"),
+                                           _stream(stream)), "qmm_grouped_gemv_noalloc")
     return y
 
 
