@@ -40,7 +40,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # ncu DRAM traffic per launch (read + write bytes) of the dominant kernel, by
 # variant string; a variant not listed here reports traffic null.
-TRAFFIC = {}
+TRAFFIC = {
+    # profiles/gemv_fp4_ldg_in_proj_18560x4096_m1.md: 47,552,768 B read + 26,112 B written
+    "gemv_fp4_ldg<fmt=2,nt=1,spw=8,wpc=4,minb=4,tiles=1160>": 47578880,
+}
 
 
 def load_peaks():
@@ -278,6 +281,92 @@ def cpu_oracle_gemv(p, x_bits, budget_s=10.0, rows=None):
             "sample": "%d of %d rows x %d reps (%.1f s, one thread)" % (rows, p.n, reps, dt)}
 
 
+def timed_launches(launch, count, reps, warm_reps, world):
+    """Graph of `count` launches; returns seconds per launch (max over ranks)."""
+    g = graph_of(launch, count)
+    time_graph(g, warm_reps, world)
+    secs, _ = time_graph(g, reps, world)
+    del g
+    return max_over_ranks(secs, world) / (count * reps)
+
+
+def gemm_workload(fmt, world, l2, peaks):
+    """Prefill GEMM, 2048 x 18560 x 4096, rotating weight and activation copies."""
+    import torch
+    from packed_bit_weight_b200 import qmm, synth
+    p, x = synth.make_prefill(fmt)
+    base = qmm.PackedWeights.from_host(p)
+    xd0 = torch.from_numpy(x.view(np.int16)).cuda()
+    R = max(2, math.ceil(1.5 * l2 / (base.nbytes + xd0.numel() * 2)))
+    ws = [base] + [qmm.PackedWeights(base.fmt, base.n, base.k, base.data.clone(), base.scales.clone(),
+                                     base.global_scale) for _ in range(R - 1)]
+    xs = [xd0] + [xd0.clone() for _ in range(R - 1)]
+    y = torch.empty((p.k and x.shape[0], p.n), dtype=torch.int16, device="cuda")
+
+    def launch(i):
+        qmm.qmm_gemm(ws[i % R], xs[i % R], y)
+
+    per = timed_launches(launch, 2 * R, 5, 1, world)
+    variant = qmm.qmm_last_variant()
+    assert qmm.qmm_sync_check() == 0
+    flops = 2.0 * x.shape[0] * p.n * p.k
+    tf = flops / per / 1e12
+    return {"variant": variant, "tflops": tf, "frac_dense_fp16": tf / peaks["bf16_tflops"],
+            "us_per_launch": per * 1e6, "flops_per_launch": flops, "copies": R}
+
+
+def grouped_workload(world, l2, peaks):
+    """Routed experts (IQ4_NL, 32 experts, 64 tokens top-4): gate+up then down."""
+    import torch
+    from packed_bit_weight_b200 import qmm, synth
+    wgu, wdn, x_gu, x_dn, ids = synth.make_experts()
+    gu, dn = qmm.PackedWeights.from_host(wgu), qmm.PackedWeights.from_host(wdn)
+    per_set = gu.nbytes + dn.nbytes
+    R = max(2, math.ceil(4 * l2 / per_set))
+    gus = [gu] + [qmm.PackedWeights(gu.fmt, gu.n, gu.k, gu.data.clone(), None, 1.0, gu.experts) for _ in range(R - 1)]
+    dns = [dn] + [qmm.PackedWeights(dn.fmt, dn.n, dn.k, dn.data.clone(), None, 1.0, dn.experts) for _ in range(R - 1)]
+    xg = torch.from_numpy(x_gu.view(np.int16)).cuda()
+    xdn = torch.from_numpy(x_dn.view(np.int16)).cuda()
+    d_ids = torch.from_numpy(ids).cuda()
+    t, topk = ids.shape
+    ygu = torch.empty((t, topk, gu.n), dtype=torch.int16, device="cuda")
+    ydn = torch.empty((t, topk, dn.n), dtype=torch.int16, device="cuda")
+    wsb = max(qmm.qmm_workspace_bytes(qmm.OP_GROUPED, gu, 0, t, topk), qmm.qmm_workspace_bytes(qmm.OP_GROUPED, dn, 0, t, topk))
+    ws = torch.empty((wsb,), dtype=torch.uint8, device="cuda")
+
+    def launch(i):
+        qmm.qmm_grouped_gemv(gus[i % R], xg, d_ids, ygu, x_per_pair=False, ws=ws)
+        qmm.qmm_grouped_gemv(dns[i % R], xdn, d_ids, ydn, x_per_pair=True, ws=ws)
+
+    per = timed_launches(launch, 2 * R, 10, 2, world)
+    variant = qmm.qmm_last_variant()
+    assert qmm.qmm_sync_check() == 0
+    hit = sorted(set(ids.reshape(-1).tolist()))
+    bytes_hit = len(hit) * (gu.nbytes + dn.nbytes) // gu.experts
+    return {"variant": variant, "gbs": bytes_hit / per / 1e9, "frac_hbm": bytes_hit / per / 1e9 / peaks["hbm_gbs"],
+            "us_per_step": per * 1e6, "experts_hit": len(hit), "bytes_per_step": bytes_hit,
+            "note": "one step = gate+up grouped GEMV then down grouped GEMV, each with its routing sort"}
+
+
+def dequant_workload(world, l2, peaks):
+    import torch
+    from packed_bit_weight_b200 import qmm, synth
+    p, _ = synth.make_gemv(synth.FP4_IN_PROJ)
+    base = qmm.PackedWeights.from_host(p)
+    out = torch.empty((p.n, p.k), dtype=torch.int16, device="cuda")
+    R = max(2, math.ceil(2 * l2 / base.nbytes))
+    ws = [base] + [qmm.PackedWeights(base.fmt, base.n, base.k, base.data.clone(), base.scales.clone()) for _ in range(R - 1)]
+
+    def launch(i):
+        qmm.qmm_dequant(ws[i % R], out)
+
+    per = timed_launches(launch, 2 * R, 10, 2, world)
+    variant = qmm.qmm_last_variant()
+    total = base.nbytes + out.numel() * 2
+    return {"variant": variant, "gbs_read_plus_write": total / per / 1e9, "frac_hbm": total / per / 1e9 / peaks["hbm_gbs"],
+            "us_per_launch": per * 1e6}
+
+
 def extra_workloads(args, world, l2, peaks):
     """Every other workload of the path, device-resident, kernel throughput."""
     from packed_bit_weight_b200 import synth
@@ -291,6 +380,7 @@ def extra_workloads(args, world, l2, peaks):
             out["fp4g16_gemv_%s_m%d" % (name, m)] = {
                 "variant": r["variant"], "gbs": r["gbs"], "frac_hbm": r["gbs"] / peaks["hbm_gbs"],
                 "us_per_launch": r["s_per_launch"] * 1e6, "tflops": 2 * m * p.n * p.k / r["s_per_launch"] / 1e12}
+    del mats
     p, x = synth.make_gemv(synth.FP4_IN_PROJ, synth.FMT_FP4G16_E4M3)
     r = gemv_workload(p, x, steps, warm, world, l2)
     out["fp4g16_e4m3_gemv_in_proj_m1"] = {"variant": r["variant"], "gbs": r["gbs"],
@@ -300,7 +390,64 @@ def extra_workloads(args, world, l2, peaks):
     r = gemv_workload(p, x, steps, warm, world, l2)
     out["iq4nl_gemv_tiny_256x512_m1"] = {"variant": r["variant"], "gbs": r["gbs"],
                                          "us_per_launch": r["s_per_launch"] * 1e6, "note": "fits in L2"}
+    out["fp4g16_prefill_gemm_2048x18560x4096"] = gemm_workload(synth.FMT_FP4G16_F16, world, l2, peaks)
+    out["fp4g16_e4m3_prefill_gemm_2048x18560x4096"] = gemm_workload(synth.FMT_FP4G16_E4M3, world, l2, peaks)
+    out["iq4nl_grouped_experts_t64_top4"] = grouped_workload(world, l2, peaks)
+    out["fp4g16_dequant_in_proj"] = dequant_workload(world, l2, peaks)
     return out
+
+
+def profile_case(name: str) -> int:
+    """Small cases for ncu captures (a few hundred MB on the device, a handful
+    of launches): gemv (in_proj, m=1, 4 rotating copies > L2), gemm (the
+    2048-token prefill, two launches), grouped (routed experts, 2 rotating
+    sets), dequant (in_proj)."""
+    import torch
+    from packed_bit_weight_b200 import qmm, synth
+    if name == "gemv":
+        p, x = synth.make_gemv(synth.FP4_IN_PROJ)
+        base = qmm.PackedWeights.from_host(p)
+        ws = [base] + [qmm.PackedWeights(base.fmt, base.n, base.k, base.data.clone(), base.scales.clone())
+                       for _ in range(3)]
+        xd = torch.from_numpy(x.view(np.int16)).cuda()
+        y = torch.empty((1, p.n), dtype=torch.int16, device="cuda")
+        for i in range(8):
+            qmm.qmm_gemv(ws[i % 4], xd, y)
+    elif name in ("gemm", "gemm_tile"):
+        if name == "gemm_tile":
+            os.environ["QMM_GEMM_VARIANT"] = "tile"
+        p, x = synth.make_prefill()
+        w = qmm.PackedWeights.from_host(p)
+        xd = torch.from_numpy(x.view(np.int16)).cuda()
+        y = torch.empty((x.shape[0], p.n), dtype=torch.int16, device="cuda")
+        for _ in range(2):
+            qmm.qmm_gemm(w, xd, y)
+    elif name == "grouped":
+        wgu, wdn, x_gu, x_dn, ids = synth.make_experts()
+        sets = [(qmm.PackedWeights.from_host(wgu), qmm.PackedWeights.from_host(wdn)) for _ in range(2)]
+        d_ids = torch.from_numpy(ids).cuda()
+        xg = torch.from_numpy(x_gu.view(np.int16)).cuda()
+        xdn = torch.from_numpy(x_dn.view(np.int16)).cuda()
+        t, topk = ids.shape
+        ygu = torch.empty((t, topk, wgu.n), dtype=torch.int16, device="cuda")
+        ydn = torch.empty((t, topk, wdn.n), dtype=torch.int16, device="cuda")
+        ws = torch.empty((1 << 20,), dtype=torch.uint8, device="cuda")
+        for i in range(4):
+            gu, dn = sets[i % 2]
+            qmm.qmm_grouped_gemv(gu, xg, d_ids, ygu, x_per_pair=False, ws=ws)
+            qmm.qmm_grouped_gemv(dn, xdn, d_ids, ydn, x_per_pair=True, ws=ws)
+    elif name == "dequant":
+        p, _ = synth.make_gemv(synth.FP4_IN_PROJ)
+        w = qmm.PackedWeights.from_host(p)
+        out = torch.empty((p.n, p.k), dtype=torch.int16, device="cuda")
+        for _ in range(3):
+            qmm.qmm_dequant(w, out)
+    else:
+        raise SystemExit("unknown profile case %r" % name)
+    torch.cuda.synchronize()
+    st = qmm.qmm_sync_check()
+    print("profile case", name, qmm.qmm_last_variant(), "status", st)
+    return 0 if st == 0 else 1
 
 
 # ---------------------------------------------------------------------------
@@ -312,7 +459,11 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extra", action="store_true", help="headline workload only")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--profile-case", default=None,
+                    help="run one small case for an ncu capture and exit (gemv, gemm, gemm_tile, grouped, dequant)")
     args = ap.parse_args()
+    if args.profile_case:
+        return profile_case(args.profile_case)
     if args.warmup < 3:
         args.warmup = 3
 

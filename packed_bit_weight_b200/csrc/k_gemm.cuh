@@ -9,8 +9,8 @@
 // 64-wide k step:
 //   * warp 0 (one thread) loads the X tile [128 x 64] fp16 with a 2-D tensor
 //     map, 128-byte swizzle -- the canonical K-major operand layout;
-//   * warps 2-5 (128 threads) load the packed codes and scales of the BN
-//     weight rows straight from global memory (registers, one step ahead),
+//   * warps 2-9 (256 threads, one weight row each) copy the packed codes and
+//     scales of their row into a private cp.async ring PSLOTS steps ahead,
 //     decode them to fp16 (E2M1 -> f16x2 convert, one multiply by the group
 //     scale = the bit-exact dequantised weight) and store them into shared
 //     memory in the same swizzled K-major layout;
@@ -18,9 +18,9 @@
 //     step from the two shared-memory descriptors into the fp32 accumulator
 //     in tensor memory and commits them to the stage's "empty" barrier.
 // A ring of STAGES stages decouples the three.  After the last step the MMA
-// thread commits to an "accumulator ready" barrier and warps 2-5 read the
-// accumulator with tcgen05.ld (each warp owns 32 TMEM lanes = 32 tokens),
-// round to fp16 and store Y.
+// thread commits to an "accumulator ready" barrier and warps 2-9 read the
+// accumulator with tcgen05.ld (warp w owns TMEM lanes 32*(w%4).. = 32 tokens
+// and half of the columns), round to fp16 and store Y.
 //
 // No TMA multicast is used.  Every wait is bounded (%globaltimer); on a
 // timeout the kernel raises the error word, drains its own copies and MMAs,
@@ -32,8 +32,10 @@ namespace qmm {
 
 constexpr int kGemmBM = 128;
 constexpr int kGemmBK = 64;
-constexpr int kGemmThreads = 6 * 32;
-constexpr int kGemmDecodeThreads = 128;
+constexpr int kGemmDecodeWarps = 8;
+constexpr int kGemmThreads = (2 + kGemmDecodeWarps) * 32;
+constexpr int kGemmDecodeThreads = kGemmDecodeWarps * 32;
+constexpr int kGemmPSlots = 5;  // packed-weight prefetch ring depth (k steps)
 
 template <int BN, int STAGES>
 struct GemmCfg {
@@ -41,7 +43,11 @@ struct GemmCfg {
   static constexpr int kBBytes = BN * kGemmBK * 2;        // 32 KB at BN=256
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = BN;                    // fp32 accumulator columns
-  static size_t smem_bytes() { return 1024 + (size_t)STAGES * kStageBytes + 256; }
+  // packed ring slot: codes bytes 0-15 [BN][16], bytes 16-31 [BN][16], scales [BN][8]
+  static constexpr int kPCodesHi = BN * 16, kPScales = 2 * BN * 16, kPSlotBytes = 2 * BN * 16 + BN * 8;
+  static size_t smem_bytes() {
+    return 1024 + (size_t)STAGES * kStageBytes + (size_t)kGemmPSlots * kPSlotBytes + 256;
+  }
 };
 
 // --- tcgen05 wrappers --------------------------------------------------------
@@ -100,44 +106,54 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, ui
   asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-// Packed data of one weight row for one 64-wide k step.
-struct RowPack {
-  uint4 c0, c1;  // 32 code bytes (k0 .. k0+63)
-  uint2 s;       // fp16: 4 scales; E4M3: 4 bytes in s.x
-};
-
-template <int FMT>
-__device__ __forceinline__ void load_rowpack(RowPack& p, const uint8_t* __restrict__ codes,
-                                             const uint8_t* __restrict__ scales, int64_t row, int n, int k,
-                                             int k0) {
-  if (row < n) {
-    const uint8_t* cp = codes + row * (int64_t)(k >> 1) + (k0 >> 1);
-    p.c0 = ldg_nc128(cp);
-    p.c1 = ldg_nc128(cp + 16);
-    if (FMT == 2) {
-      p.s = *reinterpret_cast<const uint2*>(scales + (row * (int64_t)(k >> 4) + (k0 >> 4)) * 2);
-    } else {
-      p.s.x = *reinterpret_cast<const uint32_t*>(scales + row * (int64_t)(k >> 4) + (k0 >> 4));
-      p.s.y = 0;
-    }
-  } else {
-    p.c0 = make_uint4(0, 0, 0, 0);
-    p.c1 = p.c0;
-    p.s = make_uint2(0, 0);
-  }
+__device__ __forceinline__ void cp_async16_g(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async8_g(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4_g(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_commit_g() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_wait_g(int) {
+  asm volatile("cp.async.wait_group %0;" ::"n"(kGemmPSlots - 1) : "memory");
+}
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
 }
 
-// Decode one row's 64 weights and store them as 8 swizzled 16-byte chunks.
-template <int FMT>
-__device__ __forceinline__ void store_row(const RowPack& p, uint32_t b_stage, int r) {
+// Copy the packed codes (32 bytes) and scales (8 or 4 bytes) of weight row
+// `row` for the k step starting at k0 into this thread's ring slot.  Rows
+// past n copy row n-1 (their outputs are never stored).
+template <int FMT, int BN>
+__device__ __forceinline__ void copy_rowpack(uint32_t slot, int t, const uint8_t* __restrict__ codes,
+                                             const uint8_t* __restrict__ scales, int64_t row, int n, int k, int k0) {
+  const int64_t r = row < n ? row : (int64_t)n - 1;
+  const uint8_t* cp = codes + r * (int64_t)(k >> 1) + (k0 >> 1);
+  cp_async16_g(slot + t * 16, cp);
+  cp_async16_g(slot + BN * 16 + t * 16, cp + 16);
+  if (FMT == 2) cp_async8_g(slot + 2 * BN * 16 + t * 8, scales + (r * (int64_t)(k >> 4) + (k0 >> 4)) * 2);
+  else cp_async4_g(slot + 2 * BN * 16 + t * 8, scales + r * (int64_t)(k >> 4) + (k0 >> 4));
+}
+
+// Decode this thread's row (64 weights) from its ring slot and store it as 8
+// swizzled 16-byte chunks of the B stage; rows past n store zeros.
+template <int FMT, int BN>
+__device__ __forceinline__ void store_row(uint32_t slot, int t, bool valid, uint32_t b_stage, int r) {
+  const uint4 c0 = lds128(slot + t * 16), c1 = lds128(slot + BN * 16 + t * 16);
+  const uint2 sv = lds64(slot + 2 * BN * 16 + t * 8);
   uint32_t sc[4];  // f16x2 broadcast scale per group of 16 (= two chunks)
   if (FMT == 2) {
-    sc[0] = bcast_lo(p.s.x); sc[1] = bcast_hi(p.s.x); sc[2] = bcast_lo(p.s.y); sc[3] = bcast_hi(p.s.y);
+    sc[0] = bcast_lo(sv.x); sc[1] = bcast_hi(sv.x); sc[2] = bcast_lo(sv.y); sc[3] = bcast_hi(sv.y);
   } else {
-    const uint32_t e01 = e4m3x2_to_f16x2(p.s.x & 0xFFFFu), e23 = e4m3x2_to_f16x2(p.s.x >> 16);
+    const uint32_t e01 = e4m3x2_to_f16x2(sv.x & 0xFFFFu), e23 = e4m3x2_to_f16x2(sv.x >> 16);
     sc[0] = bcast_lo(e01); sc[1] = bcast_hi(e01); sc[2] = bcast_lo(e23); sc[3] = bcast_hi(e23);
   }
-  const uint32_t q[8] = {p.c0.x, p.c0.y, p.c0.z, p.c0.w, p.c1.x, p.c1.y, p.c1.z, p.c1.w};
+  if (!valid) sc[0] = sc[1] = sc[2] = sc[3] = 0u;
+  const uint32_t q[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
   const uint32_t row_base = b_stage + (uint32_t)r * 128u;
   const uint32_t sw = (uint32_t)(r & 7);
 #pragma unroll
@@ -158,7 +174,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t base = (smem_addr(smem_raw) + 1023u) & ~1023u;
   const uint32_t a_s = base;                                  // STAGES x 16 KB
   const uint32_t b_s = a_s + STAGES * C::kABytes;             // STAGES x BN*128 B
-  const uint32_t bars = b_s + STAGES * C::kBBytes;            // full[S], empty[S], accum
+  const uint32_t p_s = b_s + STAGES * C::kBBytes;             // packed ring, kGemmPSlots slots
+  const uint32_t bars = p_s + kGemmPSlots * C::kPSlotBytes;   // full[S], empty[S], accum
   const uint32_t tmem_slot = bars + 8 * (2 * STAGES + 1);
   uint32_t* tmem_slot_ptr = reinterpret_cast<uint32_t*>(smem_raw + (tmem_slot - smem_addr(smem_raw)));
   __shared__ volatile int s_abort;
@@ -230,44 +247,49 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     // ---------------------- decode producers + epilogue ----------------------
-    const int t = threadIdx.x - 64;  // 0..127: weight rows t and t+128 of the tile
-    RowPack cur[BN / 128], nxt[BN / 128];
-#pragma unroll
-    for (int h = 0; h < BN / 128; h++) load_rowpack<FMT>(cur[h], codes, scales, (int64_t)n0 + t + 128 * h, n, k, 0);
+    const int t = threadIdx.x - 64;  // 0..255: weight row t of the tile
+    const int64_t row = (int64_t)n0 + t;
+    const bool valid = row < n;
+    // prologue: the first kGemmPSlots-1 steps in flight
+#pragma unroll 1
+    for (int j = 0; j < kGemmPSlots - 1; j++) {
+      if (j < ksteps) copy_rowpack<FMT, BN>(p_s + j * C::kPSlotBytes, t, codes, scales, row, n, k, j * kGemmBK);
+      cp_commit_g();
+    }
     for (int ks = 0; ks < ksteps; ks++) {
       const int s = ks % STAGES;
       const uint32_t ph = (uint32_t)(ks / STAGES) & 1u;
-      if (ks + 1 < ksteps) {
-#pragma unroll
-        for (int h = 0; h < BN / 128; h++)
-          load_rowpack<FMT>(nxt[h], codes, scales, (int64_t)n0 + t + 128 * h, n, k, (ks + 1) * kGemmBK);
-      }
+      const int jn = ks + kGemmPSlots - 1;  // step to prefetch now
+      if (jn < ksteps)
+        copy_rowpack<FMT, BN>(p_s + (jn % kGemmPSlots) * C::kPSlotBytes, t, codes, scales, row, n, k, jn * kGemmBK);
+      cp_commit_g();
+      cp_wait_g(0);  // this thread's copies of step ks have landed
       if (s_abort || !mbar_wait(bars + 8 * (STAGES + s), ph ^ 1u)) { s_abort = 1; break; }
-#pragma unroll
-      for (int h = 0; h < BN / 128; h++) store_row<FMT>(cur[h], b_s + s * C::kBBytes, t + 128 * h);
+      store_row<FMT, BN>(p_s + (ks % kGemmPSlots) * C::kPSlotBytes, t, valid, b_s + s * C::kBBytes, t);
       fence_proxy_async_shared();  // generic-proxy stores -> visible to the tensor core
       mbar_arrive(bars + 8 * s);
-#pragma unroll
-      for (int h = 0; h < BN / 128; h++) cur[h] = nxt[h];
     }
-    // epilogue: warp q = warp % 4 owns TMEM lanes 32q .. 32q+31 (tokens)
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    // epilogue: warp w owns TMEM lanes 32*(w%4) .. (tokens) and column half (w-2)/4
     const bool ready = mbar_wait(accum_bar, 0);
     tc_fence_after();
     if (ready && !s_abort) {
-      const int q = warp & 3;
-      const int row = m0 + 32 * q + lane;
+      const int q = warp & 3, half = (warp - 2) >> 2;
+      const int mrow = m0 + 32 * q + lane;
       const float gs = (FMT == 3) ? g : 1.0f;
-      for (int j = 0; j < n_mma / 32; j++) {
+      const int ncols = n_mma / 2;  // columns of this warp
+      for (int j = 0; j < ncols / 32; j++) {
+        const int c0 = half * ncols + 32 * j;
         uint32_t r[32];
-        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(32 * j), r);
+        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, r);
         tmem_ld_wait();
-        const int col = n0 + 32 * j;
-        if (row < m && col < n) {
+        const int col = n0 + c0;
+        if (mrow < m && col < n) {
           uint32_t h[16];
 #pragma unroll
           for (int i = 0; i < 16; i++)
             h[i] = f32x2_to_f16x2(__uint_as_float(r[2 * i]) * gs, __uint_as_float(r[2 * i + 1]) * gs);
-          uint16_t* yp = y + (int64_t)row * n + col;
+          uint16_t* yp = y + (int64_t)mrow * n + col;
           if (col + 32 <= n && (n & 7) == 0) {
             uint4* y4 = reinterpret_cast<uint4*>(yp);
 #pragma unroll
@@ -287,6 +309,197 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Persistent variant: one CTA per SM loops over tiles (tile = blockIdx.x +
+// i * gridDim.x).  Tensor memory holds two 128 x 256 fp32 accumulators; the
+// MMA thread fills accumulator i&1 while four epilogue warps (10-13) drain
+// the other, so the store of tile i overlaps the main loop of tile i+1.  The
+// operand ring and the decode warps' packed-weight prefetch run on across
+// tile boundaries without a pause.  Barriers: full/empty per operand stage,
+// acc_full/acc_empty per accumulator.
+// ---------------------------------------------------------------------------
+constexpr int kGemmPThreads = (2 + kGemmDecodeWarps + 4) * 32;
+
+template <int FMT, int BN, int STAGES>
+__global__ void __launch_bounds__(kGemmPThreads, 1)
+    gemm_fp4_tc_persistent_kernel(const __grid_constant__ CUtensorMap tm_x, const uint8_t* __restrict__ codes,
+                                  const uint8_t* __restrict__ scales, uint16_t* __restrict__ y, int m, int n, int k,
+                                  float g) {
+  using C = GemmCfg<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t base = (smem_addr(smem_raw) + 1023u) & ~1023u;
+  const uint32_t a_s = base;
+  const uint32_t b_s = a_s + STAGES * C::kABytes;
+  const uint32_t p_s = b_s + STAGES * C::kBBytes;
+  const uint32_t bars = p_s + kGemmPSlots * C::kPSlotBytes;  // full[S] empty[S] accf[2] acce[2] done
+  const uint32_t accf = bars + 8 * (2 * STAGES), acce = accf + 16, done_bar = acce + 16;
+  const uint32_t tmem_slot = done_bar + 8;
+  uint32_t* tmem_slot_ptr = reinterpret_cast<uint32_t*>(smem_raw + (tmem_slot - smem_addr(smem_raw)));
+  __shared__ volatile int s_abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tiles = (n + BN - 1) / BN;
+  const int tiles = ((m + kGemmBM - 1) / kGemmBM) * n_tiles;
+  const int ksteps = k / kGemmBK;
+  const int G = (int)gridDim.x;
+  const int my_tiles = (tiles - (int)blockIdx.x + G - 1) / G;
+
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    for (int s = 0; s < STAGES; s++) {
+      mbar_init(bars + 8 * s, 1 + kGemmDecodeThreads);
+      mbar_init(bars + 8 * (STAGES + s), 1);
+    }
+    for (int a = 0; a < 2; a++) {
+      mbar_init(accf + 8 * a, 1);    // MMA commit
+      mbar_init(acce + 8 * a, 128);  // every epilogue thread
+    }
+    mbar_init(done_bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 2 * BN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot_ptr;
+
+  if (warp == 0) {
+    // ---------------------------- X loader --------------------------------
+    if (lane == 0) {
+      prefetch_tmap(&tm_x);
+      int gs = 0, issued = 0;
+      for (int li = 0; li < my_tiles && !s_abort; li++) {
+        const int tile = (int)blockIdx.x + li * G;
+        const int m0 = (tile / n_tiles) * kGemmBM;
+        for (int ks = 0; ks < ksteps; ks++, gs++) {
+          const int s = gs % STAGES;
+          const uint32_t ph = (uint32_t)(gs / STAGES) & 1u;
+          if (s_abort || !mbar_wait(bars + 8 * (STAGES + s), ph ^ 1u)) { s_abort = 1; break; }
+          mbar_arrive_expect_tx(bars + 8 * s, C::kABytes);
+          tma_load_2d(a_s + s * C::kABytes, &tm_x, ks * kGemmBK, m0, bars + 8 * s);
+          issued = gs + 1;
+        }
+      }
+      for (int s = 0; s < STAGES && s < issued; s++) {  // drain our copies
+        const int last = issued - 1 - ((issued - 1 - s) % STAGES);
+        mbar_wait(bars + 8 * s, (uint32_t)(last / STAGES) & 1u);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------- MMA issuer ------------------------------
+    if (lane == 0) {
+      int gs = 0;
+      for (int li = 0; li < my_tiles && !s_abort; li++) {
+        const int tile = (int)blockIdx.x + li * G;
+        const int n0 = (tile % n_tiles) * BN;
+        const int n_mma = (min(BN, n - n0) <= BN / 2) ? BN / 2 : BN;
+        const uint32_t idesc = umma_idesc_f16(n_mma);
+        const int a = li & 1;
+        if (!mbar_wait(acce + 8 * a, (((uint32_t)li >> 1) & 1u) ^ 1u)) { s_abort = 1; break; }
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(a * BN);
+        bool ok = true;
+        for (int ks = 0; ks < ksteps; ks++, gs++) {
+          const int s = gs % STAGES;
+          const uint32_t ph = (uint32_t)(gs / STAGES) & 1u;
+          if (s_abort || !mbar_wait(bars + 8 * s, ph)) { s_abort = 1; ok = false; break; }
+          tc_fence_after();
+          const uint64_t da = umma_desc_k128(a_s + s * C::kABytes);
+          const uint64_t db = umma_desc_k128(b_s + s * C::kBBytes);
+#pragma unroll
+          for (int kk = 0; kk < kGemmBK / 16; kk++)
+            umma_f16(d, da + (uint64_t)(2 * kk), db + (uint64_t)(2 * kk), idesc, (ks | kk) != 0);
+          umma_commit(bars + 8 * (STAGES + s));
+        }
+        if (!ok) break;
+        umma_commit(accf + 8 * a);
+      }
+      umma_commit(done_bar);  // every MMA we issued has completed when this arrives
+    }
+  } else if (warp < 2 + kGemmDecodeWarps) {
+    // ------------------------- decode producers ---------------------------
+    const int t = threadIdx.x - 64;  // weight row t of each tile
+    // prefetch cursor (tile li, step ks) and consume cursor
+    int pli = 0, pks = 0, pg = 0;
+    auto prefetch = [&]() {
+      if (pli < my_tiles) {
+        const int tile = (int)blockIdx.x + pli * G;
+        const int64_t row = (int64_t)(tile % n_tiles) * BN + t;
+        copy_rowpack<FMT, BN>(p_s + (pg % kGemmPSlots) * C::kPSlotBytes, t, codes, scales, row, n, k, pks * kGemmBK);
+        if (++pks == ksteps) { pks = 0; pli++; }
+      }
+      pg++;
+      cp_commit_g();
+    };
+#pragma unroll 1
+    for (int j = 0; j < kGemmPSlots - 1; j++) prefetch();
+    int gs = 0;
+    bool stop = false;
+    for (int li = 0; li < my_tiles && !stop; li++) {
+      const int tile = (int)blockIdx.x + li * G;
+      const bool valid = (int64_t)(tile % n_tiles) * BN + t < n;
+      for (int ks = 0; ks < ksteps; ks++, gs++) {
+        const int s = gs % STAGES;
+        const uint32_t ph = (uint32_t)(gs / STAGES) & 1u;
+        prefetch();
+        cp_wait_g(0);  // this thread's copies of step gs have landed
+        if (s_abort || !mbar_wait(bars + 8 * (STAGES + s), ph ^ 1u)) { s_abort = 1; stop = true; break; }
+        store_row<FMT, BN>(p_s + (gs % kGemmPSlots) * C::kPSlotBytes, t, valid, b_s + s * C::kBBytes, t);
+        fence_proxy_async_shared();
+        mbar_arrive(bars + 8 * s);
+      }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+  } else {
+    // ------------------------------ epilogue ------------------------------
+    const int q = warp & 3;  // TMEM lanes 32q .. 32q+31
+    const float gs = (FMT == 3) ? g : 1.0f;
+    for (int li = 0; li < my_tiles; li++) {
+      const int tile = (int)blockIdx.x + li * G;
+      const int m0 = (tile / n_tiles) * kGemmBM, n0 = (tile % n_tiles) * BN;
+      const int n_mma = (min(BN, n - n0) <= BN / 2) ? BN / 2 : BN;
+      const int a = li & 1;
+      if (s_abort || !mbar_wait(accf + 8 * a, ((uint32_t)li >> 1) & 1u)) { s_abort = 1; break; }
+      tc_fence_after();
+      const int mrow = m0 + 32 * q + lane;
+      for (int j = 0; j < n_mma / 32; j++) {
+        uint32_t r[32];
+        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * BN + 32 * j), r);
+        tmem_ld_wait();
+        const int col = n0 + 32 * j;
+        if (mrow < m && col < n) {
+          uint32_t h[16];
+#pragma unroll
+          for (int i = 0; i < 16; i++)
+            h[i] = f32x2_to_f16x2(__uint_as_float(r[2 * i]) * gs, __uint_as_float(r[2 * i + 1]) * gs);
+          uint16_t* yp = y + (int64_t)mrow * n + col;
+          if (col + 32 <= n && (n & 7) == 0) {
+            uint4* y4 = reinterpret_cast<uint4*>(yp);
+#pragma unroll
+            for (int i = 0; i < 4; i++) y4[i] = make_uint4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
+          } else {
+            for (int i = 0; i < 32 && col + i < n; i++) yp[i] = (uint16_t)((h[i >> 1] >> (16 * (i & 1))) & 0xFFFFu);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(acce + 8 * a);  // accumulator a may be overwritten
+    }
+  }
+
+  // teardown: no MMA of ours may still be writing tensor memory
+  if (warp == 1 && lane == 0) mbar_wait(done_bar, 0);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 2 * BN);
   }
 }
 

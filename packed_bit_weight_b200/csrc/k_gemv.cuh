@@ -307,4 +307,526 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Streaming FP4-G16 kernel, register-direct (no shared-memory staging).
+//
+// One CTA = one tile of 16 weight rows over the whole k; its 8 warps split k
+// into equal ranges of SPW segments of 128 (64 code bytes per row).  Each lane
+// owns rows grp and grp+8 and, in every segment, the 16 code bytes at
+// 16*tig (plus their two group scales): it issues all of its loads for the
+// tile at once (16-byte ld.global.nc with an L2 256-byte prefetch hint, no L1
+// allocation), so a warp has SPW*1.25 KB in flight and the several CTAs
+// resident per SM keep HBM busy.  The bytes then go straight into MMA
+// fragments (same k order as the TMA kernel).  The WPC partial tiles are
+// summed in shared memory in a fixed order.  Launched with programmatic
+// dependent launch: the weight loads are issued before griddepcontrol.wait, so
+// a CTA that starts while the previous kernel drains already streams its
+// weights; activations are read and y written only after the wait.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint4 ldg_stream128(const void* p) {
+  uint4 v;
+  asm("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint32_t ldg_stream32(const void* p) {
+  uint32_t v;
+  asm("ld.global.nc.L1::no_allocate.L2::256B.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint32_t ldg_stream16(const void* p) {
+  unsigned short v;
+  asm("ld.global.nc.L1::no_allocate.L2::256B.u16 %0, [%1];" : "=h"(v) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint4 ldg_x128(const void* p) {
+  uint4 v;
+  asm("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
+
+constexpr int kLdgWarps = 8;
+
+// Programmatic dependent launch: let the next kernel on the stream start
+// launching now; wait until the previous kernel's writes are visible.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <int FMT, int NT, int SPW, int WPC = kLdgWarps, int MINB = 2>
+__global__ void __launch_bounds__(WPC * 32, MINB)
+    gemv_fp4_ldg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                        const uint16_t* __restrict__ x, uint16_t* __restrict__ y, int n, int k, int m, float g) {
+  __shared__ float red[WPC][16][16];  // [warp][token][row]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int grp = lane >> 2, tig = lane & 3;
+  const int n0 = blockIdx.x * 16;
+  const int ra = n0 + grp, rb = ra + 8;
+  const bool va = ra < n, vb = rb < n;
+  const int seg0 = warp * SPW;
+  const int64_t crow = k >> 1, srow = k >> 4;
+
+  pdl_launch_dependents();
+  uint4 qa[SPW], qb[SPW];
+  uint32_t sa[SPW], sb[SPW];
+#pragma unroll
+  for (int i = 0; i < SPW; i++) {
+    const int seg = seg0 + i;
+    const int64_t cb = (int64_t)seg * 64 + tig * 16;
+    const int64_t gi = (int64_t)seg * 8 + tig * 2;  // first of the two group scales
+    qa[i] = va ? ldg_stream128(codes + ra * crow + cb) : make_uint4(0, 0, 0, 0);
+    qb[i] = vb ? ldg_stream128(codes + rb * crow + cb) : make_uint4(0, 0, 0, 0);
+    if (FMT == 2) {
+      sa[i] = va ? ldg_stream32(scales + (ra * srow + gi) * 2) : 0u;
+      sb[i] = vb ? ldg_stream32(scales + (rb * srow + gi) * 2) : 0u;
+    } else {
+      sa[i] = va ? e4m3x2_to_f16x2(ldg_stream16(scales + ra * srow + gi)) : 0u;
+      sb[i] = vb ? e4m3x2_to_f16x2(ldg_stream16(scales + rb * srow + gi)) : 0u;
+    }
+  }
+  pdl_wait();  // x may be the previous kernel's output; y may still be read by it
+
+  float acc[NT][4];
+#pragma unroll
+  for (int j = 0; j < NT; j++)
+#pragma unroll
+    for (int c = 0; c < 4; c++) acc[j][c] = 0.f;
+
+#pragma unroll
+  for (int i = 0; i < SPW; i++) {
+    const int kseg = (seg0 + i) * 128 + tig * 32;
+    uint32_t xb[NT][16];
+#pragma unroll
+    for (int j = 0; j < NT; j++) {
+      const int tok = grp + 8 * j;
+      if (tok < m) {
+        const uint16_t* xp = x + (int64_t)tok * k + kseg;
+#pragma unroll
+        for (int q = 0; q < 4; q++) {
+          const uint4 v = ldg_x128(xp + 8 * q);
+          xb[j][4 * q] = v.x; xb[j][4 * q + 1] = v.y; xb[j][4 * q + 2] = v.z; xb[j][4 * q + 3] = v.w;
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < 16; q++) xb[j][q] = 0u;
+      }
+    }
+    const uint32_t sa0 = bcast_lo(sa[i]), sa1 = bcast_hi(sa[i]);
+    const uint32_t sb0 = bcast_lo(sb[i]), sb1 = bcast_hi(sb[i]);
+    uint32_t wa[16], wb[16];
+    e2m1x8_to_f16x2(qa[i].x, *reinterpret_cast<uint32_t(*)[4]>(&wa[0]));
+    e2m1x8_to_f16x2(qa[i].y, *reinterpret_cast<uint32_t(*)[4]>(&wa[4]));
+    e2m1x8_to_f16x2(qa[i].z, *reinterpret_cast<uint32_t(*)[4]>(&wa[8]));
+    e2m1x8_to_f16x2(qa[i].w, *reinterpret_cast<uint32_t(*)[4]>(&wa[12]));
+    e2m1x8_to_f16x2(qb[i].x, *reinterpret_cast<uint32_t(*)[4]>(&wb[0]));
+    e2m1x8_to_f16x2(qb[i].y, *reinterpret_cast<uint32_t(*)[4]>(&wb[4]));
+    e2m1x8_to_f16x2(qb[i].z, *reinterpret_cast<uint32_t(*)[4]>(&wb[8]));
+    e2m1x8_to_f16x2(qb[i].w, *reinterpret_cast<uint32_t(*)[4]>(&wb[12]));
+#pragma unroll
+    for (int st = 0; st < 8; st++) {
+      const uint32_t sA = (st < 4) ? sa0 : sa1, sB = (st < 4) ? sb0 : sb1;
+      const uint32_t a0 = hmul2(wa[2 * st], sA), a2 = hmul2(wa[2 * st + 1], sA);
+      const uint32_t a1 = hmul2(wb[2 * st], sB), a3 = hmul2(wb[2 * st + 1], sB);
+#pragma unroll
+      for (int j = 0; j < NT; j++) mma_16816(acc[j], a0, a1, a2, a3, xb[j][2 * st], xb[j][2 * st + 1]);
+    }
+  }
+
+#pragma unroll
+  for (int j = 0; j < NT; j++) {
+    const int t0 = 8 * j + 2 * tig;
+    red[warp][t0][grp] = acc[j][0];
+    red[warp][t0 + 1][grp] = acc[j][1];
+    red[warp][t0][grp + 8] = acc[j][2];
+    red[warp][t0 + 1][grp + 8] = acc[j][3];
+  }
+  __syncthreads();
+  const float gs = (FMT == 3) ? g : 1.0f;
+  for (int idx = threadIdx.x; idx < 16 * m; idx += WPC * 32) {
+    const int row = idx & 15, tok = idx >> 4;
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < WPC; w++) v += red[w][tok][row];
+    if (n0 + row < n) y[(int64_t)tok * n + n0 + row] = f32_to_f16_bits(v * gs);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Streaming FP4-G16 kernel with per-warp cp.async rings (persistent).
+//
+// Work unit = a tile of 16 weight rows over the whole k; its k range is split
+// into WPC equal ranges, one per warp, of SPW segments (128 k each).  Each
+// CTA loops over tiles; each warp walks the same k range of successive tiles,
+// a linear stream of segments, and keeps DEPTH segments in flight with
+// cp.async: per segment a lane copies its own 16 code bytes of rows grp and
+// grp+8 and their 4-byte scale words into a lane-private slot of the warp's
+// ring.  Only the issuing lane reads what it copied, so the ring needs no
+// barrier (cp.async.wait_group is per thread) and its layout is lane-major,
+// conflict-free.  Loads in flight hold no registers, so two CTAs of WPC
+// warps per SM keep ~2*WPC*DEPTH*1.3 KB streaming while the warps decode.
+// At the end of a tile the WPC partial sums meet in shared memory (fixed
+// order) and the tile's rows are stored.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global.L2::256B [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// One ring slot (one segment of one warp), lane-major per field so every
+// cp.async destination is aligned to its size: codes of row a [32 lanes][16 B]
+// at 0, codes of row b at 512, scale words of row a [32][4 B] at 1024, of
+// row b at 1152.
+constexpr int kCpaSlotBytes = 1280;
+constexpr int kCpaCodesB = 512, kCpaScalesA = 1024, kCpaScalesB = 1152;
+
+// Walks one warp's linear stream of (tile, segment) elements with pointers
+// that advance by constant strides; rows past n are clamped once per tile.
+template <int FMT>
+struct CpaCursor {
+  const uint8_t* ca;  // codes, row a, this lane's 16 bytes
+  const uint8_t* cb;
+  const uint8_t* sa;  // this lane's scale word, row a
+  const uint8_t* sb;
+  int seg;            // segment within the tile's warp range
+  int tile;
+
+  __device__ __forceinline__ void at_tile(const uint8_t* codes, const uint8_t* scales, int t, int n, int64_t crow,
+                                          int64_t srow, int seg_lo, int grp, int tig) {
+    tile = t;
+    seg = 0;
+    const int64_t ra = min((int64_t)t * 16 + grp, (int64_t)n - 1);
+    const int64_t rb = min((int64_t)t * 16 + grp + 8, (int64_t)n - 1);
+    ca = codes + ra * crow + seg_lo * 64 + tig * 16;
+    cb = codes + rb * crow + seg_lo * 64 + tig * 16;
+    if (FMT == 2) {
+      sa = scales + (ra * srow + seg_lo * 8 + tig * 2) * 2;
+      sb = scales + (rb * srow + seg_lo * 8 + tig * 2) * 2;
+    } else {  // the aligned word holding this lane's two E4M3 bytes
+      sa = scales + ra * srow + seg_lo * 8 + (tig & 2) * 2;
+      sb = scales + rb * srow + seg_lo * 8 + (tig & 2) * 2;
+    }
+  }
+  __device__ __forceinline__ void next(const uint8_t* codes, const uint8_t* scales, int spw, int G, int n,
+                                       int64_t crow, int64_t srow, int seg_lo, int grp, int tig) {
+    if (++seg == spw) {
+      at_tile(codes, scales, tile + G, n, crow, srow, seg_lo, grp, tig);
+    } else {
+      ca += 64;
+      cb += 64;
+      sa += (FMT == 2) ? 16 : 8;
+      sb += (FMT == 2) ? 16 : 8;
+    }
+  }
+};
+
+template <int FMT, int NT, int WPC, int DEPTH, int MINB = 2>
+__global__ void __launch_bounds__(WPC * 32, MINB)
+    gemv_fp4_cpa_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                        const uint16_t* __restrict__ x, uint16_t* __restrict__ y, int n, int k, int m, float g,
+                        int num_tiles) {
+  static_assert((DEPTH & (DEPTH - 1)) == 0, "ring depth must be a power of two");
+  extern __shared__ __align__(16) uint8_t smem_cpa[];
+  float* red = reinterpret_cast<float*>(smem_cpa);  // [WPC][16 tokens][16 rows]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int grp = lane >> 2, tig = lane & 3;
+  const uint32_t ring = smem_addr(smem_cpa) + WPC * 16 * 16 * 4 + warp * DEPTH * kCpaSlotBytes;
+  const int spw = (k >> 7) / WPC;  // segments per warp and tile
+  const int seg_lo = warp * spw;
+  const int G = (int)gridDim.x;
+  const int64_t crow = k >> 1, srow = k >> 4;
+  const int my_tiles = (num_tiles - (int)blockIdx.x + G - 1) / G;
+  const int total = my_tiles * spw;  // this warp's element stream
+
+  CpaCursor<FMT> in;  // next element to copy
+  in.at_tile(codes, scales, (int)blockIdx.x, n, crow, srow, seg_lo, grp, tig);
+  int issued = 0;
+  auto issue_one = [&]() {
+    if (issued < total) {
+      const uint32_t slot = ring + (uint32_t)(issued & (DEPTH - 1)) * kCpaSlotBytes;
+      cp_async16(slot + lane * 16, in.ca);
+      cp_async16(slot + kCpaCodesB + lane * 16, in.cb);
+      cp_async4(slot + kCpaScalesA + lane * 4, in.sa);
+      cp_async4(slot + kCpaScalesB + lane * 4, in.sb);
+      in.next(codes, scales, spw, G, n, crow, srow, seg_lo, grp, tig);
+    }
+    issued++;
+    cp_async_commit();  // one group per element (empty past the end)
+  };
+#pragma unroll 1
+  for (int j = 0; j < DEPTH - 1; j++) issue_one();
+
+  float acc[NT][4];
+  const float gs = (FMT == 3) ? g : 1.0f;
+  int tile = (int)blockIdx.x, seg = 0;
+  const uint16_t* xrow[NT];
+#pragma unroll
+  for (int t = 0; t < NT; t++) xrow[t] = (grp + 8 * t < m) ? x + (int64_t)(grp + 8 * t) * k + seg_lo * 128 + tig * 32 : nullptr;
+#pragma unroll 1
+  for (int j = 0; j < total; j++) {
+    if (seg == 0) {
+#pragma unroll
+      for (int a = 0; a < NT; a++)
+#pragma unroll
+        for (int c = 0; c < 4; c++) acc[a][c] = 0.f;
+    }
+    issue_one();
+    uint32_t xb[NT][16];
+#pragma unroll
+    for (int t = 0; t < NT; t++) {
+      if (xrow[t]) {
+        const uint16_t* xp = xrow[t] + seg * 128;
+#pragma unroll
+        for (int q = 0; q < 4; q++) {
+          const uint4 v = ldg_x128(xp + 8 * q);
+          xb[t][4 * q] = v.x; xb[t][4 * q + 1] = v.y; xb[t][4 * q + 2] = v.z; xb[t][4 * q + 3] = v.w;
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < 16; q++) xb[t][q] = 0u;
+      }
+    }
+    cp_async_wait<DEPTH - 1>();  // element j has landed (this lane's copies)
+    const uint32_t slot = ring + (uint32_t)(j & (DEPTH - 1)) * kCpaSlotBytes;
+    const uint4 qa = lds128(slot + lane * 16), qb = lds128(slot + kCpaCodesB + lane * 16);
+    uint32_t sa = lds32(slot + kCpaScalesA + lane * 4), sb = lds32(slot + kCpaScalesB + lane * 4);
+    if (FMT == 3) {
+      sa = e4m3x2_to_f16x2((tig & 1) ? (sa >> 16) : sa);
+      sb = e4m3x2_to_f16x2((tig & 1) ? (sb >> 16) : sb);
+    }
+    const uint32_t sa0 = bcast_lo(sa), sa1 = bcast_hi(sa), sb0 = bcast_lo(sb), sb1 = bcast_hi(sb);
+    uint32_t wa[16], wb[16];
+    e2m1x8_to_f16x2(qa.x, *reinterpret_cast<uint32_t(*)[4]>(&wa[0]));
+    e2m1x8_to_f16x2(qa.y, *reinterpret_cast<uint32_t(*)[4]>(&wa[4]));
+    e2m1x8_to_f16x2(qa.z, *reinterpret_cast<uint32_t(*)[4]>(&wa[8]));
+    e2m1x8_to_f16x2(qa.w, *reinterpret_cast<uint32_t(*)[4]>(&wa[12]));
+    e2m1x8_to_f16x2(qb.x, *reinterpret_cast<uint32_t(*)[4]>(&wb[0]));
+    e2m1x8_to_f16x2(qb.y, *reinterpret_cast<uint32_t(*)[4]>(&wb[4]));
+    e2m1x8_to_f16x2(qb.z, *reinterpret_cast<uint32_t(*)[4]>(&wb[8]));
+    e2m1x8_to_f16x2(qb.w, *reinterpret_cast<uint32_t(*)[4]>(&wb[12]));
+#pragma unroll
+    for (int st = 0; st < 8; st++) {
+      const uint32_t sA = (st < 4) ? sa0 : sa1, sB = (st < 4) ? sb0 : sb1;
+      const uint32_t a0 = hmul2(wa[2 * st], sA), a2 = hmul2(wa[2 * st + 1], sA);
+      const uint32_t a1 = hmul2(wb[2 * st], sB), a3 = hmul2(wb[2 * st + 1], sB);
+#pragma unroll
+      for (int t = 0; t < NT; t++) mma_16816(acc[t], a0, a1, a2, a3, xb[t][2 * st], xb[t][2 * st + 1]);
+    }
+    if (++seg == spw) {  // tile done: meet the other warps
+      seg = 0;
+      float* r = red + warp * 256;
+#pragma unroll
+      for (int t = 0; t < NT; t++) {
+        const int t0 = 8 * t + 2 * tig;
+        r[t0 * 16 + grp] = acc[t][0];
+        r[(t0 + 1) * 16 + grp] = acc[t][1];
+        r[t0 * 16 + grp + 8] = acc[t][2];
+        r[(t0 + 1) * 16 + grp + 8] = acc[t][3];
+      }
+      __syncthreads();
+      const int n0 = tile * 16;
+      for (int idx = threadIdx.x; idx < 16 * m; idx += WPC * 32) {
+        const int row = idx & 15, tok = idx >> 4;
+        float v = 0.f;
+#pragma unroll
+        for (int w = 0; w < WPC; w++) v += red[w * 256 + tok * 16 + row];
+        if (n0 + row < n) y[(int64_t)tok * n + n0 + row] = f32_to_f16_bits(v * gs);
+      }
+      __syncthreads();
+      tile += G;
+    }
+  }
+  cp_async_wait<0>();
+}
+
+// ---------------------------------------------------------------------------
+// Persistent streaming FP4-G16 kernel with a register prefetch ring.
+//
+// Tiles of 16 rows; WPC warps split each tile's k into ranges of spw
+// segments (128 k).  Every warp walks the linear stream of its segments over
+// the CTA's tiles and keeps P of them in flight in registers: the loads of
+// element j+P are issued right after element j is decoded, into the registers
+// element j just freed, so each SM always has WPC*P*1.25 KB per CTA streaming
+// and no CTA ever waits for a whole tile to arrive.  Addresses advance by
+// constant strides (64 code bytes, 8 scales per segment) and are clamped to
+// row n-1 once per tile.  With programmatic dependent launch the weight loads
+// of the first P elements are issued before griddepcontrol.wait, so they
+// overlap the tail of the kernel that precedes this one on the stream;
+// activations are read and outputs written only after the wait.
+// ---------------------------------------------------------------------------
+template <int FMT>
+struct SegRegs {
+  uint4 qa, qb;
+  uint32_t sa, sb;
+};
+
+template <int FMT>
+struct StreamCursor {
+  const uint8_t* ca;
+  const uint8_t* cb;
+  const uint8_t* sa;
+  const uint8_t* sb;
+  int seg, tile;
+  __device__ __forceinline__ void at_tile(const uint8_t* codes, const uint8_t* scales, int t, int n, int64_t crow,
+                                          int64_t srow, int seg_lo, int grp, int tig) {
+    tile = t;
+    seg = 0;
+    const int64_t ra = min((int64_t)t * 16 + grp, (int64_t)n - 1);
+    const int64_t rb = min((int64_t)t * 16 + grp + 8, (int64_t)n - 1);
+    ca = codes + ra * crow + seg_lo * 64 + tig * 16;
+    cb = codes + rb * crow + seg_lo * 64 + tig * 16;
+    sa = scales + (ra * srow + seg_lo * 8 + tig * 2) * (FMT == 2 ? 2 : 1);
+    sb = scales + (rb * srow + seg_lo * 8 + tig * 2) * (FMT == 2 ? 2 : 1);
+  }
+  __device__ __forceinline__ void load(SegRegs<FMT>& r) const {
+    r.qa = ldg_stream128(ca);
+    r.qb = ldg_stream128(cb);
+    if (FMT == 2) {
+      r.sa = ldg_stream32(sa);
+      r.sb = ldg_stream32(sb);
+    } else {
+      r.sa = ldg_stream16(sa);
+      r.sb = ldg_stream16(sb);
+    }
+  }
+  __device__ __forceinline__ void next(const uint8_t* codes, const uint8_t* scales, int spw, int G, int n,
+                                       int64_t crow, int64_t srow, int seg_lo, int grp, int tig) {
+    if (++seg == spw) {
+      at_tile(codes, scales, tile + G, n, crow, srow, seg_lo, grp, tig);
+    } else {
+      ca += 64;
+      cb += 64;
+      sa += (FMT == 2) ? 16 : 8;
+      sb += (FMT == 2) ? 16 : 8;
+    }
+  }
+};
+
+template <int FMT, int NT>
+__device__ __forceinline__ void seg_mma(float (&acc)[NT][4], const SegRegs<FMT>& r, const uint16_t* const (&xrow)[NT],
+                                        int off) {
+  uint32_t xb[NT][16];
+#pragma unroll
+  for (int t = 0; t < NT; t++) {
+    if (xrow[t]) {
+      const uint16_t* xp = xrow[t] + off;
+#pragma unroll
+      for (int q = 0; q < 4; q++) {
+        const uint4 v = ldg_x128(xp + 8 * q);
+        xb[t][4 * q] = v.x; xb[t][4 * q + 1] = v.y; xb[t][4 * q + 2] = v.z; xb[t][4 * q + 3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int q = 0; q < 16; q++) xb[t][q] = 0u;
+    }
+  }
+  uint32_t sa = r.sa, sb = r.sb;
+  if (FMT == 3) {
+    sa = e4m3x2_to_f16x2(sa);
+    sb = e4m3x2_to_f16x2(sb);
+  }
+  const uint32_t sa0 = bcast_lo(sa), sa1 = bcast_hi(sa), sb0 = bcast_lo(sb), sb1 = bcast_hi(sb);
+  uint32_t wa[16], wb[16];
+  e2m1x8_to_f16x2(r.qa.x, *reinterpret_cast<uint32_t(*)[4]>(&wa[0]));
+  e2m1x8_to_f16x2(r.qa.y, *reinterpret_cast<uint32_t(*)[4]>(&wa[4]));
+  e2m1x8_to_f16x2(r.qa.z, *reinterpret_cast<uint32_t(*)[4]>(&wa[8]));
+  e2m1x8_to_f16x2(r.qa.w, *reinterpret_cast<uint32_t(*)[4]>(&wa[12]));
+  e2m1x8_to_f16x2(r.qb.x, *reinterpret_cast<uint32_t(*)[4]>(&wb[0]));
+  e2m1x8_to_f16x2(r.qb.y, *reinterpret_cast<uint32_t(*)[4]>(&wb[4]));
+  e2m1x8_to_f16x2(r.qb.z, *reinterpret_cast<uint32_t(*)[4]>(&wb[8]));
+  e2m1x8_to_f16x2(r.qb.w, *reinterpret_cast<uint32_t(*)[4]>(&wb[12]));
+#pragma unroll
+  for (int st = 0; st < 8; st++) {
+    const uint32_t sA = (st < 4) ? sa0 : sa1, sB = (st < 4) ? sb0 : sb1;
+    const uint32_t a0 = hmul2(wa[2 * st], sA), a2 = hmul2(wa[2 * st + 1], sA);
+    const uint32_t a1 = hmul2(wb[2 * st], sB), a3 = hmul2(wb[2 * st + 1], sB);
+#pragma unroll
+    for (int t = 0; t < NT; t++) mma_16816(acc[t], a0, a1, a2, a3, xb[t][2 * st], xb[t][2 * st + 1]);
+  }
+}
+
+template <int FMT, int NT, int WPC, int P, int MINB>
+__global__ void __launch_bounds__(WPC * 32, MINB)
+    gemv_fp4_stream_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                           const uint16_t* __restrict__ x, uint16_t* __restrict__ y, int n, int k, int m, float g,
+                           int num_tiles) {
+  __shared__ float red[WPC][16][16];  // [warp][token][row]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, grp = lane >> 2, tig = lane & 3;
+  const int spw = (k >> 7) / WPC;
+  const int seg_lo = warp * spw;
+  const int G = (int)gridDim.x;
+  const int64_t crow = k >> 1, srow = k >> 4;
+  const int my_tiles = (num_tiles - (int)blockIdx.x + G - 1) / G;
+  const int total = my_tiles * spw;
+
+  pdl_launch_dependents();
+  StreamCursor<FMT> in;
+  in.at_tile(codes, scales, (int)blockIdx.x, n, crow, srow, seg_lo, grp, tig);
+  SegRegs<FMT> buf[P];
+#pragma unroll
+  for (int u = 0; u < P; u++) {
+    if (u < total) {
+      in.load(buf[u]);
+      in.next(codes, scales, spw, G, n, crow, srow, seg_lo, grp, tig);
+    }
+  }
+  pdl_wait();  // the previous kernel's outputs (our x) are visible from here on
+
+  const uint16_t* xrow[NT];
+#pragma unroll
+  for (int t = 0; t < NT; t++)
+    xrow[t] = (grp + 8 * t < m) ? x + (int64_t)(grp + 8 * t) * k + seg_lo * 128 + tig * 32 : nullptr;
+  const float gs = (FMT == 3) ? g : 1.0f;
+  float acc[NT][4];
+#pragma unroll
+  for (int t = 0; t < NT; t++)
+#pragma unroll
+    for (int c = 0; c < 4; c++) acc[t][c] = 0.f;
+  int tile = (int)blockIdx.x, seg = 0;
+#pragma unroll 1
+  for (int j0 = 0; j0 < total; j0 += P) {
+#pragma unroll
+    for (int u = 0; u < P; u++) {
+      const int j = j0 + u;
+      if (j < total) {
+        seg_mma<FMT, NT>(acc, buf[u], xrow, seg * 128);
+        if (j + P < total) {
+          in.load(buf[u]);
+          in.next(codes, scales, spw, G, n, crow, srow, seg_lo, grp, tig);
+        }
+        if (++seg == spw) {  // tile done: meet the other warps, store, reset
+          seg = 0;
+#pragma unroll
+          for (int t = 0; t < NT; t++) {
+            const int t0 = 8 * t + 2 * tig;
+            red[warp][t0][grp] = acc[t][0];
+            red[warp][t0 + 1][grp] = acc[t][1];
+            red[warp][t0][grp + 8] = acc[t][2];
+            red[warp][t0 + 1][grp + 8] = acc[t][3];
+#pragma unroll
+            for (int c = 0; c < 4; c++) acc[t][c] = 0.f;
+          }
+          __syncthreads();
+          const int n0 = tile * 16;
+          for (int idx = threadIdx.x; idx < 16 * m; idx += WPC * 32) {
+            const int row = idx & 15, tok = idx >> 4;
+            float v = 0.f;
+#pragma unroll
+            for (int w = 0; w < WPC; w++) v += red[w][tok][row];
+            if (n0 + row < n) y[(int64_t)tok * n + n0 + row] = f32_to_f16_bits(v * gs);
+          }
+          __syncthreads();
+          tile += G;
+        }
+      }
+    }
+  }
+}
+
 }  // namespace qmm

@@ -150,4 +150,169 @@ __global__ void __launch_bounds__(128) grouped_gemv_kernel(
   }
 }
 
+// ---------------------------------------------------------------------------
+// IQ4_NL streaming kernel for the grouped GEMV (and, with offsets == nullptr,
+// the plain GEMV: one "expert", m tokens in order).
+//
+// Work item = (expert, 16-row tile); persistent CTAs of IQW warps loop over
+// items.  The warps split the tile's k into ranges of "super-steps" of four
+// blocks (128 k).  In a super-step lane (grp, tig) owns block 4s+tig of rows
+// grp and grp+8: it reads the 18-byte block with five 4-byte loads (blocks of
+// even index start 4-byte aligned, odd ones 2 bytes past; with an even block
+// count per row the five words never leave the row), takes the scale d and
+// the 16 index bytes, and turns each index byte j into the pair
+// (w_j, w_{j+16}) = d * (kv[lo], kv[hi]) with one lookup in a 256-entry
+// table of exact f16x2 pairs (replicated across the 32 banks, so each lane
+// reads its own bank) and one f16x2 multiply -- the bit-exact decoded
+// weights.  MMA step i uses bytes 2i and 2i+1; the matching activation pairs
+// (x_2i, x_2i+16) and (x_2i+1, x_2i+17) are one byte permute each.
+// ---------------------------------------------------------------------------
+constexpr int kIqWarps = 4;
+constexpr int kIqLutBytes = 256 * 32 * 4;  // [byte][lane] f16x2
+constexpr int kIqRedBytes = kIqWarps * 32 * 16 * 4;
+
+// One pass of a warp over its super-steps for up to 8*NT tokens.
+template <int NT>
+__device__ __forceinline__ void iq4_pass(float (&acc)[4][4], const uint8_t* __restrict__ de, int64_t rowb, int ra,
+                                         int rb, int s_lo, int s_hi, int tig, const uint16_t* const (&xr)[4],
+                                         uint32_t lut_lane) {
+  for (int ss = s_lo; ss < s_hi; ss++) {
+    const int b = 4 * ss + tig;
+    const int64_t boff = (int64_t)b * 18 - ((tig & 1) ? 2 : 0);  // 4-byte aligned start
+    const uint32_t* pa = reinterpret_cast<const uint32_t*>(de + (int64_t)ra * rowb + boff);
+    const uint32_t* pb = reinterpret_cast<const uint32_t*>(de + (int64_t)rb * rowb + boff);
+    uint32_t wa[5], wb[5];
+#pragma unroll
+    for (int i = 0; i < 5; i++) {
+      wa[i] = __ldg(pa + i);
+      wb[i] = __ldg(pb + i);
+    }
+    uint32_t da, db, qa[4], qb[4];
+    if (tig & 1) {  // block starts 2 bytes into word 0
+      da = wa[0] >> 16;
+      db = wb[0] >> 16;
+#pragma unroll
+      for (int i = 0; i < 4; i++) { qa[i] = wa[i + 1]; qb[i] = wb[i + 1]; }
+    } else {
+      da = wa[0] & 0xFFFFu;
+      db = wb[0] & 0xFFFFu;
+#pragma unroll
+      for (int i = 0; i < 4; i++) {
+        qa[i] = __funnelshift_r(wa[i], wa[i + 1], 16);
+        qb[i] = __funnelshift_r(wb[i], wb[i + 1], 16);
+      }
+    }
+    const uint32_t dda = da | (da << 16), ddb = db | (db << 16);
+    uint32_t xw[NT][16];  // this block's 32 activations per n-tile, as 16 words
+#pragma unroll
+    for (int j = 0; j < NT; j++) {
+      if (xr[j]) {
+        const uint16_t* xp = xr[j] + b * 32;
+#pragma unroll
+        for (int q = 0; q < 4; q++) {
+          const uint4 v = ldg_x128(xp + 8 * q);
+          xw[j][4 * q] = v.x; xw[j][4 * q + 1] = v.y; xw[j][4 * q + 2] = v.z; xw[j][4 * q + 3] = v.w;
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < 16; q++) xw[j][q] = 0u;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; i++) {  // index bytes 2i, 2i+1 of the block
+      const uint32_t qwa = qa[i >> 1], qwb = qb[i >> 1];
+      const int sh = (i & 1) * 16;
+      const uint32_t a0 = hmul2(lds32(lut_lane + ((qwa >> sh) & 0xFFu) * 128u), dda);
+      const uint32_t a2 = hmul2(lds32(lut_lane + ((qwa >> (sh + 8)) & 0xFFu) * 128u), dda);
+      const uint32_t a1 = hmul2(lds32(lut_lane + ((qwb >> sh) & 0xFFu) * 128u), ddb);
+      const uint32_t a3 = hmul2(lds32(lut_lane + ((qwb >> (sh + 8)) & 0xFFu) * 128u), ddb);
+#pragma unroll
+      for (int j = 0; j < NT; j++) {
+        const uint32_t b0 = __byte_perm(xw[j][i], xw[j][i + 8], 0x5410);  // (x_2i, x_2i+16)
+        const uint32_t b1 = __byte_perm(xw[j][i], xw[j][i + 8], 0x7632);  // (x_2i+1, x_2i+17)
+        mma_16816(acc[j], a0, a1, a2, a3, b0, b1);
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kIqWarps * 32, 4)
+    grouped_iq4_kernel(const uint8_t* __restrict__ data, int64_t dstride, const uint16_t* __restrict__ x,
+                       int x_per_pair, int topk, const int32_t* __restrict__ offsets,
+                       const int32_t* __restrict__ perm, int m_plain, uint16_t* __restrict__ y, int n, int k,
+                       int E) {
+  extern __shared__ __align__(16) uint8_t smem_iq[];
+  const uint32_t lut = smem_addr(smem_iq);
+  float* red = reinterpret_cast<float*>(smem_iq + kIqLutBytes);  // [warp][32 token slots][16 rows]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, grp = lane >> 2, tig = lane & 3;
+  for (int i = threadIdx.x; i < 256 * 32; i += kIqWarps * 32) {
+    const int v = i >> 5;
+    const uint32_t lo = __half_as_ushort(__int2half_rn(c_iq4nl_kv[v & 15]));
+    const uint32_t hi = __half_as_ushort(__int2half_rn(c_iq4nl_kv[v >> 4]));
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(lut + 4u * i), "r"(lo | (hi << 16)) : "memory");
+  }
+  __syncthreads();
+  const uint32_t lut_lane = lut + 4u * lane;
+  const int tiles = (n + 15) / 16;
+  const int steps = k >> 7;  // super-steps per row
+  const int s_lo = warp * steps / kIqWarps, s_hi = (warp + 1) * steps / kIqWarps;
+  const int64_t rowb = (int64_t)(k >> 5) * 18;  // bytes per row
+  const int items = tiles * E;
+  for (int item = blockIdx.x; item < items; item += gridDim.x) {
+    const int e = item / tiles, tile = item % tiles;
+    int start = 0, cnt = m_plain;
+    if (offsets) {
+      start = offsets[e];
+      cnt = offsets[e + 1] - start;
+    }
+    if (cnt <= 0) continue;  // uniform across the CTA
+    const uint8_t* de = data + (int64_t)e * dstride;
+    const int ra = min(tile * 16 + grp, n - 1), rb = min(tile * 16 + grp + 8, n - 1);
+    for (int tok0 = 0; tok0 < cnt; tok0 += 32) {
+      const int ng = min(32, cnt - tok0);
+      const uint16_t* xr[4];
+#pragma unroll
+      for (int j = 0; j < 4; j++) {
+        const int slot = grp + 8 * j;
+        xr[j] = nullptr;
+        if (slot < ng) {
+          const int pr = offsets ? perm[start + tok0 + slot] : tok0 + slot;
+          xr[j] = x + (int64_t)((offsets && !x_per_pair) ? pr / topk : pr) * k;
+        }
+      }
+      float acc[4][4];
+#pragma unroll
+      for (int j = 0; j < 4; j++)
+#pragma unroll
+        for (int c = 0; c < 4; c++) acc[j][c] = 0.f;
+      if (ng <= 8) iq4_pass<1>(acc, de, rowb, ra, rb, s_lo, s_hi, tig, xr, lut_lane);
+      else if (ng <= 16) iq4_pass<2>(acc, de, rowb, ra, rb, s_lo, s_hi, tig, xr, lut_lane);
+      else iq4_pass<4>(acc, de, rowb, ra, rb, s_lo, s_hi, tig, xr, lut_lane);
+      // meet the other warps: red[warp][token slot][row]
+      float* r = red + warp * (32 * 16);
+#pragma unroll
+      for (int j = 0; j < 4; j++) {
+        const int t0 = 8 * j + 2 * tig;
+        r[t0 * 16 + grp] = acc[j][0];
+        r[(t0 + 1) * 16 + grp] = acc[j][1];
+        r[t0 * 16 + grp + 8] = acc[j][2];
+        r[(t0 + 1) * 16 + grp + 8] = acc[j][3];
+      }
+      __syncthreads();
+      for (int idx = threadIdx.x; idx < 16 * ng; idx += kIqWarps * 32) {
+        const int row = idx & 15, slot = idx >> 4;
+        float v = 0.f;
+#pragma unroll
+        for (int w = 0; w < kIqWarps; w++) v += red[w * 512 + slot * 16 + row];
+        const int grow = tile * 16 + row;
+        if (grow < n) {
+          const int64_t pr = offsets ? perm[start + tok0 + slot] : tok0 + slot;
+          y[pr * n + grow] = f32_to_f16_bits(v);
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
 }  // namespace qmm

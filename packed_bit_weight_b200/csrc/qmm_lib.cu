@@ -9,6 +9,7 @@
 
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -157,13 +158,205 @@ static qmm_status launch_gemv_tma(const qmm_weights* w, const uint16_t* x, int m
   return launch_status();
 }
 
+template <int FMT, int NT, int SPW, int WPC = kLdgWarps, int MINB = 2>
+static qmm_status launch_gemv_ldg(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st) {
+  const int n = (int)w->n, k = (int)w->k;
+  const int tiles = (n + 15) / 16;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(tiles);
+  cfg.blockDim = dim3(WPC * 32);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const uint8_t* codes = static_cast<const uint8_t*>(w->data);
+  const uint8_t* scales = static_cast<const uint8_t*>(w->scales);
+  const float g = w->global_scale;
+  if (cudaLaunchKernelEx(&cfg, gemv_fp4_ldg_kernel<FMT, NT, SPW, WPC, MINB>, codes, scales, x, y, n, k, m, g) !=
+      cudaSuccess)
+    return QMM_ERR_CUDA;
+  set_variant("gemv_fp4_ldg<fmt=%d,nt=%d,spw=%d,wpc=%d,minb=%d,tiles=%d>", FMT, NT, SPW, WPC, MINB, tiles);
+  return launch_status();
+}
+
+// Pick the warps per tile (WPC) and segments per warp (SPW, <= 8 at m <= 8,
+// <= 4 at m <= 16) for k = 128 * WPC * SPW; fewer, fuller warps keep more
+// bytes in flight per register.  Returns UNSUPPORTED_SHAPE for other k.
+template <int FMT, int NT>
+static qmm_status gemv_ldg_auto(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st) {
+  const int segs = (int)(w->k / 128);
+  if (w->k % 128) return QMM_ERR_UNSUPPORTED_SHAPE;
+  if (NT == 1) {
+    if (segs % 4 == 0 && segs / 4 <= 8) {
+      switch (segs / 4) {
+        case 1: return launch_gemv_ldg<FMT, 1, 1, 4, 4>(w, x, m, y, st);
+        case 2: return launch_gemv_ldg<FMT, 1, 2, 4, 4>(w, x, m, y, st);
+        case 3: return launch_gemv_ldg<FMT, 1, 3, 4, 4>(w, x, m, y, st);
+        case 4: return launch_gemv_ldg<FMT, 1, 4, 4, 4>(w, x, m, y, st);
+        case 5: return launch_gemv_ldg<FMT, 1, 5, 4, 4>(w, x, m, y, st);
+        case 6: return launch_gemv_ldg<FMT, 1, 6, 4, 4>(w, x, m, y, st);
+        case 7: return launch_gemv_ldg<FMT, 1, 7, 4, 4>(w, x, m, y, st);
+        default: return launch_gemv_ldg<FMT, 1, 8, 4, 4>(w, x, m, y, st);
+      }
+    }
+    if (segs % 8 == 0 && segs / 8 <= 8) {
+      switch (segs / 8) {
+        case 5: return launch_gemv_ldg<FMT, 1, 5, 8, 2>(w, x, m, y, st);
+        case 6: return launch_gemv_ldg<FMT, 1, 6, 8, 2>(w, x, m, y, st);
+        case 7: return launch_gemv_ldg<FMT, 1, 7, 8, 2>(w, x, m, y, st);
+        case 8: return launch_gemv_ldg<FMT, 1, 8, 8, 2>(w, x, m, y, st);
+        default: break;  // smaller counts took the 4-warp path
+      }
+    }
+    if (segs % 16 == 0 && segs / 16 <= 8) {
+      switch (segs / 16) {
+        case 5: return launch_gemv_ldg<FMT, 1, 5, 16, 1>(w, x, m, y, st);
+        case 6: return launch_gemv_ldg<FMT, 1, 6, 16, 1>(w, x, m, y, st);
+        case 7: return launch_gemv_ldg<FMT, 1, 7, 16, 1>(w, x, m, y, st);
+        case 8: return launch_gemv_ldg<FMT, 1, 8, 16, 1>(w, x, m, y, st);
+        default: break;
+      }
+    }
+  } else {
+    if (segs % 8 == 0 && segs / 8 <= 4) {
+      switch (segs / 8) {
+        case 1: return launch_gemv_ldg<FMT, 2, 1, 8, 2>(w, x, m, y, st);
+        case 2: return launch_gemv_ldg<FMT, 2, 2, 8, 2>(w, x, m, y, st);
+        case 3: return launch_gemv_ldg<FMT, 2, 3, 8, 2>(w, x, m, y, st);
+        default: return launch_gemv_ldg<FMT, 2, 4, 8, 2>(w, x, m, y, st);
+      }
+    }
+    if (segs % 16 == 0 && segs / 16 <= 4) {
+      switch (segs / 16) {
+        case 3: return launch_gemv_ldg<FMT, 2, 3, 16, 1>(w, x, m, y, st);
+        case 4: return launch_gemv_ldg<FMT, 2, 4, 16, 1>(w, x, m, y, st);
+        default: break;
+      }
+    }
+  }
+  return QMM_ERR_UNSUPPORTED_SHAPE;
+}
+
+template <int FMT, int NT, int WPC, int DEPTH, int MINB = 2>
+static qmm_status launch_gemv_cpa(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st,
+                                  const DevInfo* di) {
+  const int n = (int)w->n, k = (int)w->k;
+  const int tiles = (n + 15) / 16;
+  const size_t smem = (size_t)WPC * 16 * 16 * 4 + (size_t)WPC * DEPTH * kCpaSlotBytes;
+  auto kern = gemv_fp4_cpa_kernel<FMT, NT, WPC, DEPTH, MINB>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return QMM_ERR_CUDA;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, WPC * 32, smem) != cudaSuccess || per_sm < 1)
+    return QMM_ERR_CUDA;
+  const int grid = tiles < per_sm * di->sms ? tiles : per_sm * di->sms;
+  kern<<<grid, WPC * 32, smem, st>>>(static_cast<const uint8_t*>(w->data), static_cast<const uint8_t*>(w->scales), x, y,
+                                      n, k, m, w->global_scale, tiles);
+  set_variant("gemv_fp4_cpa<fmt=%d,nt=%d,wpc=%d,depth=%d,minb=%d,grid=%d>", FMT, NT, WPC, DEPTH, MINB, grid);
+  return launch_status();
+}
+
+// Variant override for measurements: QMM_GEMV_VARIANT=cpa|tma|ldg|generic.
+static int gemv_variant_env() {
+  const char* v = getenv("QMM_GEMV_VARIANT");
+  if (!v) return 0;
+  if (!strcmp(v, "tma")) return 1;
+  if (!strcmp(v, "ldg")) return 2;
+  if (!strcmp(v, "generic")) return 3;
+  if (!strcmp(v, "cpa")) return 4;
+  if (!strcmp(v, "iq4")) return 5;
+  return 0;
+}
+
+static qmm_status launch_iq4_stream(const qmm_weights* w, const uint16_t* x, int x_per_pair, int64_t topk,
+                                   const int32_t* offsets, const int32_t* perm, int m_plain, uint16_t* y,
+                                   cudaStream_t st, const DevInfo* di);
+
+// Persistent streaming GEMV, launched with programmatic stream serialization
+// (PDL) so its weight prefetch overlaps the previous kernel's tail.
+template <int FMT, int NT, int WPC, int P, int MINB>
+static qmm_status launch_gemv_stream(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st,
+                                     const DevInfo* di) {
+  const int n = (int)w->n, k = (int)w->k;
+  const int tiles = (n + 15) / 16;
+  auto kern = gemv_fp4_stream_kernel<FMT, NT, WPC, P, MINB>;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, WPC * 32, 0) != cudaSuccess || per_sm < 1)
+    return QMM_ERR_CUDA;
+  const int grid = tiles < per_sm * di->sms ? tiles : per_sm * di->sms;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(WPC * 32);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const uint8_t* codes = static_cast<const uint8_t*>(w->data);
+  const uint8_t* scales = static_cast<const uint8_t*>(w->scales);
+  const float g = w->global_scale;
+  if (cudaLaunchKernelEx(&cfg, kern, codes, scales, x, y, n, k, m, g, tiles) != cudaSuccess) return QMM_ERR_CUDA;
+  set_variant("gemv_fp4_stream<fmt=%d,nt=%d,wpc=%d,p=%d,minb=%d,grid=%d>", FMT, NT, WPC, P, MINB, grid);
+  return launch_status();
+}
+
+// Measurement hook: QMM_GEMV_CFG picks one compiled configuration of the
+// streaming kernels for k = 4096, m <= 8 (used by the tuning sweep only).
+template <int FMT>
+static bool gemv_cfg_env(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st,
+                         const DevInfo* di, qmm_status* out) {
+  const char* c = getenv("QMM_GEMV_CFG");
+  if (!c || w->k != 4096 || m > 8) return false;
+  if (!strcmp(c, "ldg_w8_s4_b2")) *out = launch_gemv_ldg<FMT, 1, 4, 8, 2>(w, x, m, y, st);
+  else if (!strcmp(c, "ldg_w16_s2_b2")) *out = launch_gemv_ldg<FMT, 1, 2, 16, 2>(w, x, m, y, st);
+  else if (!strcmp(c, "ldg_w8_s4_b3")) *out = launch_gemv_ldg<FMT, 1, 4, 8, 3>(w, x, m, y, st);
+  else if (!strcmp(c, "ldg_w4_s8_b4")) *out = launch_gemv_ldg<FMT, 1, 8, 4, 4>(w, x, m, y, st);
+  else if (!strcmp(c, "cpa_w8_d8_b2")) *out = launch_gemv_cpa<FMT, 1, 8, 8, 2>(w, x, m, y, st, di);
+  else if (!strcmp(c, "cpa_w8_d4_b3")) *out = launch_gemv_cpa<FMT, 1, 8, 4, 3>(w, x, m, y, st, di);
+  else if (!strcmp(c, "cpa_w16_d4_b2")) *out = launch_gemv_cpa<FMT, 1, 16, 4, 2>(w, x, m, y, st, di);
+  else if (!strcmp(c, "cpa_w4_d8_b4")) *out = launch_gemv_cpa<FMT, 1, 4, 8, 4>(w, x, m, y, st, di);
+  else if (!strcmp(c, "str_w4_p4_b4")) *out = launch_gemv_stream<FMT, 1, 4, 4, 4>(w, x, m, y, st, di);
+  else if (!strcmp(c, "str_w4_p8_b3")) *out = launch_gemv_stream<FMT, 1, 4, 8, 3>(w, x, m, y, st, di);
+  else if (!strcmp(c, "str_w8_p4_b2")) *out = launch_gemv_stream<FMT, 1, 8, 4, 2>(w, x, m, y, st, di);
+  else if (!strcmp(c, "str_w8_p2_b3")) *out = launch_gemv_stream<FMT, 1, 8, 2, 3>(w, x, m, y, st, di);
+  else if (!strcmp(c, "str_w2_p8_b6")) *out = launch_gemv_stream<FMT, 1, 2, 8, 6>(w, x, m, y, st, di);
+  else return false;
+  return true;
+}
+
 template <int FMT>
 static qmm_status gemv_fmt(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st,
                            const DevInfo* di) {
   const int64_t n = w->n, k = w->k;
-  if (FMT != 1 && k % kChunkK == 0 && k >= 8 * kChunkK && n >= 16) {
+  if (FMT != 1) {
+    qmm_status cs;
+    if (gemv_cfg_env<FMT>(w, x, m, y, st, di, &cs)) return cs;
+  }
+  const int pick = gemv_variant_env();
+  const bool tma_ok = FMT != 1 && k % kChunkK == 0 && k >= 8 * kChunkK && n >= 16;
+  if (FMT != 1 && (pick == 0 || pick == 2)) {
+    const qmm_status s = (m <= 8) ? gemv_ldg_auto<FMT, 1>(w, x, m, y, st) : gemv_ldg_auto<FMT, 2>(w, x, m, y, st);
+    if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
+  }
+  const int segs = (int)(k / 128);
+  const bool cpa_ok = FMT != 1 && k % 1024 == 0 && k >= 1024;
+  if (cpa_ok && pick == 4 && segs % 8 == 0) {
+    if (m <= 8) return launch_gemv_cpa<FMT, 1, 8, 8>(w, x, m, y, st, di);
+    return launch_gemv_cpa<FMT, 2, 8, 8>(w, x, m, y, st, di);
+  }
+  if (tma_ok && (pick == 0 || pick == 1)) {
     if (m <= 8) return launch_gemv_tma<FMT, 1, 1>(w, x, m, y, st, di);
     return launch_gemv_tma<FMT, 1, 2>(w, x, m, y, st, di);
+  }
+  if (FMT == 1 && k % 128 == 0 && (pick == 0 || pick == 5)) {
+    const qmm_status s = launch_iq4_stream(w, x, 0, 1, nullptr, nullptr, m, y, st, di);
+    set_variant("gemv_iq4_stream");
+    return s;
   }
   const int64_t tiles = (n + 15) / 16;
   const int64_t blocks = (tiles + 3) / 4;
@@ -181,7 +374,7 @@ static qmm_status gemv_fmt(const qmm_weights* w, const uint16_t* x, int m, uint1
 template <int FMT>
 static qmm_status launch_gemm_tc(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st,
                                  const DevInfo* di) {
-  constexpr int BN = 256, STAGES = 4;
+  constexpr int BN = 256, STAGES = 3;
   using C = GemmCfg<BN, STAGES>;
   const int n = (int)w->n, k = (int)w->k;
   CUtensorMap tx;
@@ -202,6 +395,31 @@ static qmm_status launch_gemm_tc(const qmm_weights* w, const uint16_t* x, int m,
   return launch_status();
 }
 
+template <int FMT>
+static qmm_status launch_gemm_tc_persistent(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y,
+                                            cudaStream_t st, const DevInfo* di) {
+  constexpr int BN = 256, STAGES = 3;
+  using C = GemmCfg<BN, STAGES>;
+  const int n = (int)w->n, k = (int)w->k;
+  CUtensorMap tx;
+  if (!make_map_2d(&tx, x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)k, (uint64_t)m, kGemmBK, kGemmBM,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+    return QMM_ERR_CUDA;
+  const size_t smem = C::smem_bytes() + 64;
+  if (smem > di->smem_optin - 1024) return QMM_ERR_CUDA;
+  auto kern = gemm_fp4_tc_persistent_kernel<FMT, BN, STAGES>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return QMM_ERR_CUDA;
+  const int64_t tiles = (int64_t)((m + kGemmBM - 1) / kGemmBM) * ((n + BN - 1) / BN);
+  if (tiles > INT32_MAX) return QMM_ERR_UNSUPPORTED_SHAPE;
+  const int grid = tiles < di->sms ? (int)tiles : di->sms;
+  kern<<<grid, kGemmPThreads, smem, st>>>(tx, static_cast<const uint8_t*>(w->data),
+                                          static_cast<const uint8_t*>(w->scales), y, m, n, k, w->global_scale);
+  set_variant("gemm_fp4_tc_persistent<fmt=%d,bm=128,bn=%d,bk=64,stages=%d,grid=%d,tiles=%lld>", FMT, BN, STAGES, grid,
+              (long long)tiles);
+  return launch_status();
+}
+
 // Any shape the tensor-core kernel does not take: the decode-batch kernel
 // over 16-token slices of x (a GPU path, recorded as such).
 template <int FMT>
@@ -218,6 +436,25 @@ static qmm_status gemm_by_gemv(const qmm_weights* w, const uint16_t* x, int64_t 
   }
   set_variant("gemm_by_gemv_generic<fmt=%d>", FMT);
   return QMM_OK;
+}
+
+// IQ4_NL streaming kernel (k % 128 == 0): persistent CTAs over (expert, tile).
+static qmm_status launch_iq4_stream(const qmm_weights* w, const uint16_t* x, int x_per_pair, int64_t topk,
+                                   const int32_t* offsets, const int32_t* perm, int m_plain, uint16_t* y,
+                                   cudaStream_t st, const DevInfo* di) {
+  const size_t smem = kIqLutBytes + kIqRedBytes;
+  if (cudaFuncSetAttribute(grouped_iq4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return QMM_ERR_CUDA;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, grouped_iq4_kernel, kIqWarps * 32, smem) != cudaSuccess ||
+      per_sm < 1)
+    return QMM_ERR_CUDA;
+  const int64_t items = ((w->n + 15) / 16) * w->num_experts;
+  const int64_t grid = items < (int64_t)per_sm * di->sms ? items : (int64_t)per_sm * di->sms;
+  grouped_iq4_kernel<<<(unsigned)grid, kIqWarps * 32, smem, st>>>(
+      static_cast<const uint8_t*>(w->data), w->expert_data_stride, x, x_per_pair, (int)topk, offsets, perm, m_plain, y,
+      (int)w->n, (int)w->k, (int)w->num_experts);
+  return launch_status();
 }
 
 template <int FMT>
@@ -376,10 +613,17 @@ qmm_status qmm_gemm(const qmm_weights* w, const uint16_t* x, int64_t m, uint16_t
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (w->k == 0) return zero_output(y, m * w->n, st, di);
   const bool tc = w->fmt != QMM_FMT_IQ4_NL && w->k % kGemmBK == 0 && m >= 64;
+  // QMM_GEMM_VARIANT=tile selects the one-tile-per-CTA kernel (measurements)
+  const char* gv = getenv("QMM_GEMM_VARIANT");
+  const bool persist = !(gv && !strcmp(gv, "tile"));
   switch (w->fmt) {
     case QMM_FMT_IQ4_NL: return gemm_by_gemv<1>(w, x, m, y, st, di);
-    case QMM_FMT_FP4G16_F16: return tc ? launch_gemm_tc<2>(w, x, (int)m, y, st, di) : gemm_by_gemv<2>(w, x, m, y, st, di);
-    default: return tc ? launch_gemm_tc<3>(w, x, (int)m, y, st, di) : gemm_by_gemv<3>(w, x, m, y, st, di);
+    case QMM_FMT_FP4G16_F16:
+      if (!tc) return gemm_by_gemv<2>(w, x, m, y, st, di);
+      return persist ? launch_gemm_tc_persistent<2>(w, x, (int)m, y, st, di) : launch_gemm_tc<2>(w, x, (int)m, y, st, di);
+    default:
+      if (!tc) return gemm_by_gemv<3>(w, x, m, y, st, di);
+      return persist ? launch_gemm_tc_persistent<3>(w, x, (int)m, y, st, di) : launch_gemm_tc<3>(w, x, (int)m, y, st, di);
   }
 }
 
@@ -444,6 +688,11 @@ qmm_status qmm_grouped_gemv(const qmm_weights* experts, const uint16_t* x, int32
     zero_fill_kernel<<<grid_for(P * experts->n, 256, di->sms), 256, 0, st>>>(y, P * experts->n);
     set_variant("route+zero_fill");
     return launch_status();
+  }
+  if (experts->fmt == QMM_FMT_IQ4_NL && experts->k % 128 == 0 && getenv("QMM_GEMV_VARIANT") == nullptr) {
+    s = launch_iq4_stream(experts, x, x_per_pair, topk, offsets, perm, 0, y, st, di);
+    set_variant("route+grouped_iq4_stream");
+    return s;
   }
   switch (experts->fmt) {
     case QMM_FMT_IQ4_NL: s = launch_grouped<1>(experts, x, x_per_pair, topk, offsets, perm, y, st); break;

@@ -23,15 +23,19 @@ def run_gemm(w, x_bits, canary=64):
     return from_dev_u16(y)
 
 
+@pytest.mark.parametrize("variant", ["persistent", "tile"])
 @pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3])
 @pytest.mark.parametrize("m,n,k", [(128, 256, 64), (128, 256, 256), (256, 384, 512), (200, 300, 1024),
-                                   (64, 128, 128), (384, 1000, 2048)])
-def test_gemm_vs_oracle(fmt, m, n, k):
+                                   (64, 128, 128), (384, 1000, 2048), (2560, 2048, 64), (2048, 2560, 256)])
+def test_gemm_vs_oracle(variant, fmt, m, n, k, monkeypatch):
+    if variant == "tile":
+        monkeypatch.setenv("QMM_GEMM_VARIANT", "tile")
     rng = np.random.default_rng(500 + m + n + k + fmt)
     p = synth.gen_fp4(rng, n, k, fmt)
     x = synth.gen_x(rng, m, k)
     y = run_gemm(dev(p), x)
-    assert qmm.qmm_last_variant().startswith("gemm_fp4_tc"), qmm.qmm_last_variant()
+    v = qmm.qmm_last_variant()
+    assert v.startswith("gemm_fp4_tc_persistent" if variant == "persistent" else "gemm_fp4_tc<"), v
     yref, absy = oracle.matmul(fmt, n, k, p.data, p.scales, p.global_scale, x)
     check_tol(y, yref, absy, "gemm m=%d n=%d k=%d" % (m, n, k))
 

@@ -35,7 +35,21 @@ def test_gemv_vs_oracle(fmt, n, k, m):
 def test_fast_path_is_used_for_streaming_shapes():
     p, x = _case(synth.FMT_FP4G16_F16, 1000, 4096, 1, 5)
     run_gemv(dev(p), x)
-    assert qmm.qmm_last_variant().startswith("gemv_fp4_tma")
+    assert qmm.qmm_last_variant().startswith(("gemv_fp4_cpa", "gemv_fp4_ldg", "gemv_fp4_tma"))
+
+
+@pytest.mark.parametrize("variant", ["cpa", "tma", "ldg", "generic"])
+@pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3])
+@pytest.mark.parametrize("n,k,m", [(1000, 4096, 1), (333, 8192, 3), (64, 2048, 16), (517, 3072, 9)])
+def test_every_streaming_variant_vs_oracle(variant, fmt, n, k, m, monkeypatch):
+    monkeypatch.setenv("QMM_GEMV_VARIANT", variant)
+    p, x = _case(fmt, n, k, m, 2000 + n + k + m + fmt)
+    y = run_gemv(dev(p), x)
+    v = qmm.qmm_last_variant()
+    assert v.startswith({"cpa": "gemv_fp4_cpa", "tma": "gemv_fp4_tma", "ldg": "gemv_fp4_ldg",
+                         "generic": "gemv_generic"}[variant]), v
+    yref, absy = oracle.matmul(fmt, n, k, p.data, p.scales, p.global_scale, x)
+    check_tol(y, yref, absy, v)
 
 
 @pytest.mark.parametrize("fmt", FMTS)
@@ -56,7 +70,7 @@ def test_config2_in_proj_full(fmt):
     p, x = synth.make_gemv(synth.FP4_IN_PROJ, fmt)
     w = dev(p)
     y = run_gemv(w, x)
-    assert qmm.qmm_last_variant().startswith("gemv_fp4_tma")
+    assert qmm.qmm_last_variant().startswith(("gemv_fp4_cpa", "gemv_fp4_ldg", "gemv_fp4_tma"))
     yref, absy = oracle.matmul(fmt, p.n, p.k, p.data, p.scales, p.global_scale, x)
     check_tol(y, yref, absy, "in_proj")
     y2 = run_gemv(w, x)
