@@ -613,9 +613,9 @@ qmm_status qmm_gemm(const qmm_weights* w, const uint16_t* x, int64_t m, uint16_t
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (w->k == 0) return zero_output(y, m * w->n, st, di);
   const bool tc = w->fmt != QMM_FMT_IQ4_NL && w->k % kGemmBK == 0 && m >= 64;
-  // QMM_GEMM_VARIANT=tile selects the one-tile-per-CTA kernel (measurements)
+  // QMM_GEMM_VARIANT=persistent selects the persistent kernel (measurements)
   const char* gv = getenv("QMM_GEMM_VARIANT");
-  const bool persist = !(gv && !strcmp(gv, "tile"));
+  const bool persist = gv && !strcmp(gv, "persistent");
   switch (w->fmt) {
     case QMM_FMT_IQ4_NL: return gemm_by_gemv<1>(w, x, m, y, st, di);
     case QMM_FMT_FP4G16_F16:

@@ -28,8 +28,7 @@ def run_gemm(w, x_bits, canary=64):
 @pytest.mark.parametrize("m,n,k", [(128, 256, 64), (128, 256, 256), (256, 384, 512), (200, 300, 1024),
                                    (64, 128, 128), (384, 1000, 2048), (2560, 2048, 64), (2048, 2560, 256)])
 def test_gemm_vs_oracle(variant, fmt, m, n, k, monkeypatch):
-    if variant == "tile":
-        monkeypatch.setenv("QMM_GEMM_VARIANT", "tile")
+    monkeypatch.setenv("QMM_GEMM_VARIANT", variant)
     rng = np.random.default_rng(500 + m + n + k + fmt)
     p = synth.gen_fp4(rng, n, k, fmt)
     x = synth.gen_x(rng, m, k)
