@@ -413,9 +413,9 @@ def profile_case(name: str) -> int:
         y = torch.empty((1, p.n), dtype=torch.int16, device="cuda")
         for i in range(8):
             qmm.qmm_gemv(ws[i % 4], xd, y)
-    elif name in ("gemm", "gemm_persistent"):
-        if name == "gemm_persistent":
-            os.environ["QMM_GEMM_VARIANT"] = "persistent"
+    elif name in ("gemm", "gemm_tile"):
+        if name == "gemm_tile":
+            os.environ["QMM_GEMM_VARIANT"] = "tile"
         p, x = synth.make_prefill()
         w = qmm.PackedWeights.from_host(p)
         xd = torch.from_numpy(x.view(np.int16)).cuda()
@@ -460,7 +460,7 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="headline workload only")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--profile-case", default=None,
-                    help="run one small case for an ncu capture and exit (gemv, gemm, gemm_persistent, grouped, dequant)")
+                    help="run one small case for an ncu capture and exit (gemv, gemm, gemm_tile, grouped, dequant)")
     args = ap.parse_args()
     if args.profile_case:
         return profile_case(args.profile_case)

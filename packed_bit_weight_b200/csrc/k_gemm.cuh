@@ -322,6 +322,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // acc_full/acc_empty per accumulator.
 // ---------------------------------------------------------------------------
 constexpr int kGemmPThreads = (2 + kGemmDecodeWarps + 4) * 32;
+constexpr int kGemmChunkSteps = 4;  // k steps per cooperatively staged packed chunk (256 k)
+
+// Staged packed chunk for BN=256 rows: codes [256][128 B] (16-byte unit u of
+// row r at unit u ^ (r & 7), so the eight rows of a read phase hit eight
+// different bank groups), then scales [256][32 B] (fp16: 16-byte half h at
+// h ^ ((r >> 2) & 1); E4M3: the row's 16 bytes unswizzled).
+constexpr int kStageCodes = 256 * 128;
+constexpr int kStageScales = 256 * 32;
+constexpr int kStageBytes = kStageCodes + kStageScales;
+
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
 
 template <int FMT, int BN, int STAGES>
 __global__ void __launch_bounds__(kGemmPThreads, 1)
@@ -333,10 +346,11 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
   const uint32_t base = (smem_addr(smem_raw) + 1023u) & ~1023u;
   const uint32_t a_s = base;
   const uint32_t b_s = a_s + STAGES * C::kABytes;
-  const uint32_t p_s = b_s + STAGES * C::kBBytes;
-  const uint32_t bars = p_s + kGemmPSlots * C::kPSlotBytes;  // full[S] empty[S] accf[2] acce[2] done
+  const uint32_t p_s = b_s + STAGES * C::kBBytes;            // 2 staged packed chunks
+  const uint32_t bars = p_s + 2 * kStageBytes;                // full[S] empty[S] accf[2] acce[2] done cf[2] ce[2]
   const uint32_t accf = bars + 8 * (2 * STAGES), acce = accf + 16, done_bar = acce + 16;
-  const uint32_t tmem_slot = done_bar + 8;
+  const uint32_t cfull = done_bar + 8, cempty = cfull + 16;
+  const uint32_t tmem_slot = cempty + 16;
   uint32_t* tmem_slot_ptr = reinterpret_cast<uint32_t*>(smem_raw + (tmem_slot - smem_addr(smem_raw)));
   __shared__ volatile int s_abort;
 
@@ -358,6 +372,10 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
       mbar_init(acce + 8 * a, 128);  // every epilogue thread
     }
     mbar_init(done_bar, 1);
+    for (int c = 0; c < 2; c++) {
+      mbar_init(cfull + 8 * c, kGemmDecodeThreads);   // every decode thread's copies landed
+      mbar_init(cempty + 8 * c, kGemmDecodeThreads);  // every decode thread done reading
+    }
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -424,36 +442,85 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
     }
   } else if (warp < 2 + kGemmDecodeWarps) {
     // ------------------------- decode producers ---------------------------
-    const int t = threadIdx.x - 64;  // weight row t of each tile
-    // prefetch cursor (tile li, step ks) and consume cursor
-    int pli = 0, pks = 0, pg = 0;
-    auto prefetch = [&]() {
-      if (pli < my_tiles) {
-        const int tile = (int)blockIdx.x + pli * G;
-        const int64_t row = (int64_t)(tile % n_tiles) * BN + t;
-        copy_rowpack<FMT, BN>(p_s + (pg % kGemmPSlots) * C::kPSlotBytes, t, codes, scales, row, n, k, pks * kGemmBK);
-        if (++pks == ksteps) { pks = 0; pli++; }
+    // Packed weights arrive in chunks of 4 k steps, copied cooperatively (8
+    // threads per 128-byte row piece of codes, so a warp instruction touches
+    // 4 cache lines) into a 2-slot staging ring; thread t then decodes row t.
+    const int t = threadIdx.x - 64;
+    const int nck = ksteps / kGemmChunkSteps;  // chunks per tile
+    const int total_ck = my_tiles * nck;
+    const int64_t crow = k >> 1, srow = k >> 4;
+    auto issue_chunk = [&](int c) -> bool {
+      const int slot = c & 1;
+      if (!mbar_wait(cempty + 8 * slot, (((uint32_t)c >> 1) & 1u) ^ 1u)) return false;
+      const int tile = (int)blockIdx.x + (c / nck) * G;
+      const int n0 = (tile % n_tiles) * BN;
+      const int kc = (c % nck) * (kGemmChunkSteps * kGemmBK);  // first k of the chunk
+      const uint32_t dst = p_s + slot * kStageBytes;
+#pragma unroll
+      for (int i = 0; i < 8; i++) {  // codes: 256 rows x 8 units of 16 bytes
+        const int pc = i * kGemmDecodeThreads + t;
+        const int r = pc >> 3, u = pc & 7;
+        const int64_t gr = min((int64_t)n0 + r, (int64_t)n - 1);
+        cp_async16_g(dst + r * 128 + ((u ^ (r & 7)) << 4), codes + gr * crow + (kc >> 1) + u * 16);
       }
-      pg++;
-      cp_commit_g();
+      if (FMT == 2) {
+#pragma unroll
+        for (int i = 0; i < 2; i++) {  // scales: 256 rows x 2 halves of 16 bytes
+          const int pc = i * kGemmDecodeThreads + t;
+          const int r = pc >> 1, h = pc & 1;
+          const int64_t gr = min((int64_t)n0 + r, (int64_t)n - 1);
+          cp_async16_g(dst + kStageCodes + r * 32 + ((h ^ ((r >> 2) & 1)) << 4),
+                       scales + (gr * srow + (kc >> 4)) * 2 + h * 16);
+        }
+      } else {  // E4M3: 16 bytes per row, copied whole; words read swizzled
+        const int r = t;
+        const int64_t gr = min((int64_t)n0 + r, (int64_t)n - 1);
+        cp_async16_g(dst + kStageCodes + r * 32, scales + gr * srow + (kc >> 4));
+      }
+      cp_async_mbar_arrive_noinc(cfull + 8 * slot);
+      return true;
     };
-#pragma unroll 1
-    for (int j = 0; j < kGemmPSlots - 1; j++) prefetch();
+    bool stop = !issue_chunk(0);
     int gs = 0;
-    bool stop = false;
-    for (int li = 0; li < my_tiles && !stop; li++) {
-      const int tile = (int)blockIdx.x + li * G;
+    for (int c = 0; c < total_ck && !stop; c++) {
+      if (c + 1 < total_ck && !issue_chunk(c + 1)) { s_abort = 1; break; }
+      const int slot = c & 1;
+      if (s_abort || !mbar_wait(cfull + 8 * slot, ((uint32_t)c >> 1) & 1u)) { s_abort = 1; break; }
+      const int tile = (int)blockIdx.x + (c / nck) * G;
       const bool valid = (int64_t)(tile % n_tiles) * BN + t < n;
-      for (int ks = 0; ks < ksteps; ks++, gs++) {
+      const uint32_t src = p_s + slot * kStageBytes;
+      for (int j = 0; j < kGemmChunkSteps; j++, gs++) {
         const int s = gs % STAGES;
         const uint32_t ph = (uint32_t)(gs / STAGES) & 1u;
-        prefetch();
-        cp_wait_g(0);  // this thread's copies of step gs have landed
+        // this row's 32 code bytes (units 2j, 2j+1) and 4 scales of step j
+        const uint4 c0 = lds128(src + t * 128 + (((2 * j) ^ (t & 7)) << 4));
+        const uint4 c1 = lds128(src + t * 128 + (((2 * j + 1) ^ (t & 7)) << 4));
+        uint32_t sc[4];
+        if (FMT == 2) {
+          const uint32_t half = (uint32_t)((j >> 1) ^ ((t >> 2) & 1));
+          const uint2 sv = lds64(src + kStageCodes + t * 32 + (half << 4) + (j & 1) * 8);
+          sc[0] = bcast_lo(sv.x); sc[1] = bcast_hi(sv.x); sc[2] = bcast_lo(sv.y); sc[3] = bcast_hi(sv.y);
+        } else {
+          const uint32_t sw = lds32(src + kStageCodes + t * 32 + j * 4);
+          const uint32_t e01 = e4m3x2_to_f16x2(sw & 0xFFFFu), e23 = e4m3x2_to_f16x2(sw >> 16);
+          sc[0] = bcast_lo(e01); sc[1] = bcast_hi(e01); sc[2] = bcast_lo(e23); sc[3] = bcast_hi(e23);
+        }
+        if (!valid) sc[0] = sc[1] = sc[2] = sc[3] = 0u;
         if (s_abort || !mbar_wait(bars + 8 * (STAGES + s), ph ^ 1u)) { s_abort = 1; stop = true; break; }
-        store_row<FMT, BN>(p_s + (gs % kGemmPSlots) * C::kPSlotBytes, t, valid, b_s + s * C::kBBytes, t);
+        const uint32_t q[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        const uint32_t row_base = b_s + s * C::kBBytes + (uint32_t)t * 128u;
+        const uint32_t swz = (uint32_t)(t & 7);
+#pragma unroll
+        for (int cc = 0; cc < 8; cc++) {
+          uint32_t w4[4];
+          e2m1x8_to_f16x2(q[cc], w4);
+          const uint32_t sv = sc[cc >> 1];
+          sts128(row_base + ((cc ^ swz) << 4), hmul2(w4[0], sv), hmul2(w4[1], sv), hmul2(w4[2], sv), hmul2(w4[3], sv));
+        }
         fence_proxy_async_shared();
         mbar_arrive(bars + 8 * s);
       }
+      mbar_arrive(cempty + 8 * slot);  // this thread is done with the staged chunk
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
   } else {

@@ -171,35 +171,45 @@ constexpr int kIqWarps = 4;
 constexpr int kIqLutBytes = 256 * 32 * 4;  // [byte][lane] f16x2
 constexpr int kIqRedBytes = kIqWarps * 32 * 16 * 4;
 
-// One pass of a warp over its super-steps for up to 8*NT tokens.
-template <int NT>
+// One pass of a warp over its super-steps (at most SMAX) for up to 8*NT
+// tokens.  All block loads of the pass are issued first, so a warp has up to
+// SMAX * 1.25 KB in flight before it decodes anything.
+template <int NT, int SMAX>
 __device__ __forceinline__ void iq4_pass(float (&acc)[4][4], const uint8_t* __restrict__ de, int64_t rowb, int ra,
                                          int rb, int s_lo, int s_hi, int tig, const uint16_t* const (&xr)[4],
                                          uint32_t lut_lane) {
-  for (int ss = s_lo; ss < s_hi; ss++) {
-    const int b = 4 * ss + tig;
-    const int64_t boff = (int64_t)b * 18 - ((tig & 1) ? 2 : 0);  // 4-byte aligned start
-    const uint32_t* pa = reinterpret_cast<const uint32_t*>(de + (int64_t)ra * rowb + boff);
-    const uint32_t* pb = reinterpret_cast<const uint32_t*>(de + (int64_t)rb * rowb + boff);
-    uint32_t wa[5], wb[5];
+  uint32_t wa[SMAX][5], wb[SMAX][5];
 #pragma unroll
-    for (int i = 0; i < 5; i++) {
-      wa[i] = __ldg(pa + i);
-      wb[i] = __ldg(pb + i);
+  for (int u = 0; u < SMAX; u++) {
+    if (s_lo + u < s_hi) {
+      const int b = 4 * (s_lo + u) + tig;
+      const int64_t boff = (int64_t)b * 18 - ((tig & 1) ? 2 : 0);  // 4-byte aligned start
+      const uint32_t* pa = reinterpret_cast<const uint32_t*>(de + (int64_t)ra * rowb + boff);
+      const uint32_t* pb = reinterpret_cast<const uint32_t*>(de + (int64_t)rb * rowb + boff);
+#pragma unroll
+      for (int i = 0; i < 5; i++) {
+        wa[u][i] = __ldg(pa + i);
+        wb[u][i] = __ldg(pb + i);
+      }
     }
+  }
+#pragma unroll
+  for (int u = 0; u < SMAX; u++) {
+    if (s_lo + u >= s_hi) break;
+    const int b = 4 * (s_lo + u) + tig;
     uint32_t da, db, qa[4], qb[4];
     if (tig & 1) {  // block starts 2 bytes into word 0
-      da = wa[0] >> 16;
-      db = wb[0] >> 16;
+      da = wa[u][0] >> 16;
+      db = wb[u][0] >> 16;
 #pragma unroll
-      for (int i = 0; i < 4; i++) { qa[i] = wa[i + 1]; qb[i] = wb[i + 1]; }
+      for (int i = 0; i < 4; i++) { qa[i] = wa[u][i + 1]; qb[i] = wb[u][i + 1]; }
     } else {
-      da = wa[0] & 0xFFFFu;
-      db = wb[0] & 0xFFFFu;
+      da = wa[u][0] & 0xFFFFu;
+      db = wb[u][0] & 0xFFFFu;
 #pragma unroll
       for (int i = 0; i < 4; i++) {
-        qa[i] = __funnelshift_r(wa[i], wa[i + 1], 16);
-        qb[i] = __funnelshift_r(wb[i], wb[i + 1], 16);
+        qa[i] = __funnelshift_r(wa[u][i], wa[u][i + 1], 16);
+        qb[i] = __funnelshift_r(wb[u][i], wb[u][i + 1], 16);
       }
     }
     const uint32_t dda = da | (da << 16), ddb = db | (db << 16);
@@ -236,6 +246,16 @@ __device__ __forceinline__ void iq4_pass(float (&acc)[4][4], const uint8_t* __re
   }
 }
 
+// Passes over a warp range longer than SMAX super-steps are split in chunks.
+template <int NT>
+__device__ __forceinline__ void iq4_range(float (&acc)[4][4], const uint8_t* __restrict__ de, int64_t rowb, int ra,
+                                          int rb, int s_lo, int s_hi, int tig, const uint16_t* const (&xr)[4],
+                                          uint32_t lut_lane) {
+  constexpr int SMAX = (NT == 1) ? 3 : 2;
+  for (int s0 = s_lo; s0 < s_hi; s0 += SMAX)
+    iq4_pass<NT, SMAX>(acc, de, rowb, ra, rb, s0, min(s0 + SMAX, s_hi), tig, xr, lut_lane);
+}
+
 __global__ void __launch_bounds__(kIqWarps * 32, 4)
     grouped_iq4_kernel(const uint8_t* __restrict__ data, int64_t dstride, const uint16_t* __restrict__ x,
                        int x_per_pair, int topk, const int32_t* __restrict__ offsets,
@@ -268,8 +288,8 @@ __global__ void __launch_bounds__(kIqWarps * 32, 4)
     if (cnt <= 0) continue;  // uniform across the CTA
     const uint8_t* de = data + (int64_t)e * dstride;
     const int ra = min(tile * 16 + grp, n - 1), rb = min(tile * 16 + grp + 8, n - 1);
-    for (int tok0 = 0; tok0 < cnt; tok0 += 32) {
-      const int ng = min(32, cnt - tok0);
+    for (int tok0 = 0; tok0 < cnt; tok0 += 16) {  // up to 16 gathered tokens per pass
+      const int ng = min(16, cnt - tok0);
       const uint16_t* xr[4];
 #pragma unroll
       for (int j = 0; j < 4; j++) {
@@ -285,9 +305,8 @@ __global__ void __launch_bounds__(kIqWarps * 32, 4)
       for (int j = 0; j < 4; j++)
 #pragma unroll
         for (int c = 0; c < 4; c++) acc[j][c] = 0.f;
-      if (ng <= 8) iq4_pass<1>(acc, de, rowb, ra, rb, s_lo, s_hi, tig, xr, lut_lane);
-      else if (ng <= 16) iq4_pass<2>(acc, de, rowb, ra, rb, s_lo, s_hi, tig, xr, lut_lane);
-      else iq4_pass<4>(acc, de, rowb, ra, rb, s_lo, s_hi, tig, xr, lut_lane);
+      if (ng <= 8) iq4_range<1>(acc, de, rowb, ra, rb, s_lo, s_hi, tig, xr, lut_lane);
+      else iq4_range<2>(acc, de, rowb, ra, rb, s_lo, s_hi, tig, xr, lut_lane);
       // meet the other warps: red[warp][token slot][row]
       float* r = red + warp * (32 * 16);
 #pragma unroll

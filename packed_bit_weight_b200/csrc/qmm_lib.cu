@@ -405,8 +405,8 @@ static qmm_status launch_gemm_tc_persistent(const qmm_weights* w, const uint16_t
   if (!make_map_2d(&tx, x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)k, (uint64_t)m, kGemmBK, kGemmBM,
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return QMM_ERR_CUDA;
-  const size_t smem = C::smem_bytes() + 64;
-  if (smem > di->smem_optin - 1024) return QMM_ERR_CUDA;
+  const size_t smem = 1024 + (size_t)STAGES * C::kStageBytes + 2 * (size_t)kStageBytes + 256;
+  if (smem > di->smem_optin) return QMM_ERR_CUDA;
   auto kern = gemm_fp4_tc_persistent_kernel<FMT, BN, STAGES>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return QMM_ERR_CUDA;
@@ -613,9 +613,10 @@ qmm_status qmm_gemm(const qmm_weights* w, const uint16_t* x, int64_t m, uint16_t
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (w->k == 0) return zero_output(y, m * w->n, st, di);
   const bool tc = w->fmt != QMM_FMT_IQ4_NL && w->k % kGemmBK == 0 && m >= 64;
-  // QMM_GEMM_VARIANT=persistent selects the persistent kernel (measurements)
+  // persistent kernel when k is a multiple of its 256-wide staging chunk;
+  // QMM_GEMM_VARIANT=tile selects the one-tile-per-CTA kernel (measurements)
   const char* gv = getenv("QMM_GEMM_VARIANT");
-  const bool persist = gv && !strcmp(gv, "persistent");
+  const bool persist = !(gv && !strcmp(gv, "tile")) && w->k % (kGemmChunkSteps * kGemmBK) == 0;
   switch (w->fmt) {
     case QMM_FMT_IQ4_NL: return gemm_by_gemv<1>(w, x, m, y, st, di);
     case QMM_FMT_FP4G16_F16:
