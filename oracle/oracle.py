@@ -38,6 +38,10 @@ PINS = {
     "matmul_sampled": "equals matmul on every sampled coordinate (tests/test_oracle_matmul.py)",
     "route": "brute-force bucket check (tests/test_oracle_matmul.py)",
     "grouped_gemv": "per-pair loop of the plain product (tests/test_oracle_matmul.py)",
+    "router_topk": "softmax sums to 1, brute-force top-k, zero-weight and one-hot special cases "
+                   "(tests/test_oracle_moe.py)",
+    "silu/swiglu": "closed forms: silu(0)=0, silu(ln 3)=0.75 ln 3, odd/even split, limits (tests/test_oracle_moe.py)",
+    "combine": "linearity and the one-slot special case (tests/test_oracle_moe.py)",
 }
 
 
@@ -80,6 +84,11 @@ def lib():
         L.orc_route.argtypes = [vp, i64, i64, i64, vp, vp]
         L.orc_route.restype = i64
         L.orc_grouped_gemv.argtypes = [i32, i64, i64, vp, i64, vp, i64, f32, i64, vp, vp, i64, i64, vp, vp]
+        L.orc_router_topk.argtypes = [vp, vp, vp, i64, i64, i64, i64, vp, vp, vp, vp]
+        L.orc_silu.argtypes = [ctypes.c_double]
+        L.orc_silu.restype = ctypes.c_double
+        L.orc_swiglu.argtypes = [vp, i64, i64, vp]
+        L.orc_combine.argtypes = [vp, vp, i64, i64, i64, vp]
         _lib = L
     return _lib
 
@@ -188,3 +197,42 @@ def grouped_gemv(fmt, n, k, data, data_stride, scales, scale_stride, global_scal
     lib().orc_grouped_gemv(fmt, n, k, _p(data), int(data_stride), _p(scales), int(scale_stride),
                            float(global_scale), num_experts, _p(x_bits), _p(ids), t, topk, _p(y), _p(a))
     return y, a
+
+
+# -- mixture-of-experts block ---------------------------------------------------
+def router_topk(x_bits, w_bits, bias, topk):
+    """(logits fp32 [t][E], ids [t][topk], g [t][topk] double, probs [t][E])."""
+    x_bits = _c(x_bits, np.uint16)
+    w_bits = _c(w_bits, np.uint16)
+    bias = _c(bias, np.float32)
+    t, k = x_bits.shape
+    E = w_bits.shape[0]
+    logits = np.empty((t, E), dtype=np.float32)
+    ids = np.empty((t, topk), dtype=np.int32)
+    g = np.empty((t, topk), dtype=np.float64)
+    probs = np.empty((t, E), dtype=np.float64)
+    lib().orc_router_topk(_p(x_bits), _p(w_bits), _p(bias), t, k, E, topk, _p(logits), _p(ids), _p(g), _p(probs))
+    return logits, ids, g, probs
+
+
+def silu(z: float) -> float:
+    return lib().orc_silu(float(z))
+
+
+def swiglu(gu):
+    """gu [pairs][2f] double -> h [pairs][f] = SiLU(gate) * up."""
+    gu = _c(gu, np.float64)
+    pairs, f2 = gu.shape
+    h = np.empty((pairs, f2 // 2), dtype=np.float64)
+    lib().orc_swiglu(_p(gu), pairs, f2 // 2, _p(h))
+    return h
+
+
+def combine(y, g):
+    """y [t][topk][n], g [t][topk] -> out [t][n] = sum_s g y."""
+    y = _c(y, np.float64)
+    g = _c(g, np.float64)
+    t, topk, n = y.shape
+    out = np.empty((t, n), dtype=np.float64)
+    lib().orc_combine(_p(y), _p(g), t, topk, n, _p(out))
+    return out

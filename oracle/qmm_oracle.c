@@ -331,3 +331,77 @@ void orc_grouped_gemv(int fmt, int64_t n, int64_t k, const uint8_t* data, int64_
   free(yr);
   free(ar);
 }
+
+/* ---------------------------------------------------------------------- */
+/* Mixture-of-experts block around the grouped GEMV [MARK-M]:             */
+/*   s_{t,e} = Softmax_e(x_t W_router^T + b_e), the top-k experts by s    */
+/*   carry weights g_i = s_{t,i}; a routed expert is                       */
+/*   F(x) = (SiLU(x W_gate) * (x W_up)) W_down; the routed part of the    */
+/*   layer output is sum_i g_i F_i(x).                                     */
+/* Readings: W_router is a dense fp16 [E][k] matrix and b an fp32 [E]       */
+/* vector; g_i is the softmax score itself (no renormalisation over the    */
+/* top-k); the top-k is decided on the logits rounded to fp32 (the         */
+/* precision the GPU decides in), larger first, ties to the lower expert   */
+/* index.                                                                  */
+/* ---------------------------------------------------------------------- */
+
+/* logits[t][e] = fp32(sum_k x[t][k] * w[e][k] (double) + b[e]);
+ * ids[t][j], g[t][j] (double): the top-k experts and their softmax scores;
+ * probs[t][e] (double, may be NULL): the full softmax. */
+void orc_router_topk(const uint16_t* x, const uint16_t* w, const float* b, int64_t t, int64_t k, int64_t E,
+                     int64_t topk, float* logits, int32_t* ids, double* g, double* probs) {
+  double* p = (double*)malloc(sizeof(double) * (size_t)(E > 0 ? E : 1));
+  char* taken = (char*)malloc((size_t)(E > 0 ? E : 1));
+  for (int64_t i = 0; i < t; i++) {
+    double mx = -INFINITY;
+    for (int64_t e = 0; e < E; e++) {
+      double s = 0.0;
+      for (int64_t kk = 0; kk < k; kk++) s += orc_f16_to_f64(x[i * k + kk]) * orc_f16_to_f64(w[e * k + kk]);
+      float z = (float)(s + (double)b[e]);
+      logits[i * E + e] = z;
+      if ((double)z > mx) mx = (double)z;
+    }
+    double den = 0.0;
+    for (int64_t e = 0; e < E; e++) {
+      p[e] = exp((double)logits[i * E + e] - mx);
+      den += p[e];
+    }
+    for (int64_t e = 0; e < E; e++) {
+      p[e] /= den;
+      if (probs) probs[i * E + e] = p[e];
+      taken[e] = 0;
+    }
+    for (int64_t j = 0; j < topk; j++) {
+      int64_t best = -1;
+      for (int64_t e = 0; e < E; e++) {
+        if (taken[e]) continue;
+        if (best < 0 || logits[i * E + e] > logits[i * E + best]) best = e;
+      }
+      taken[best] = 1;
+      ids[i * topk + j] = (int32_t)best;
+      g[i * topk + j] = p[best];
+    }
+  }
+  free(p);
+  free(taken);
+}
+
+/* SiLU(z) = z / (1 + exp(-z)). */
+double orc_silu(double z) { return z / (1.0 + exp(-z)); }
+
+/* h[p][j] = SiLU(gu[p][j]) * gu[p][f + j] for the gate+up product rows
+ * gu[p] = [gate (f values) | up (f values)] of each (token, slot) pair. */
+void orc_swiglu(const double* gu, int64_t pairs, int64_t f, double* h) {
+  for (int64_t p = 0; p < pairs; p++)
+    for (int64_t j = 0; j < f; j++) h[p * f + j] = orc_silu(gu[p * 2 * f + j]) * gu[p * 2 * f + f + j];
+}
+
+/* out[t][j] = sum_s g[t][s] * y[t][s][j]. */
+void orc_combine(const double* y, const double* g, int64_t t, int64_t topk, int64_t n, double* out) {
+  for (int64_t i = 0; i < t; i++)
+    for (int64_t j = 0; j < n; j++) {
+      double s = 0.0;
+      for (int64_t q = 0; q < topk; q++) s += g[i * topk + q] * y[(i * topk + q) * n + j];
+      out[i * n + j] = s;
+    }
+}
