@@ -171,6 +171,15 @@ constexpr int kIqWarps = 4;
 constexpr int kIqLutBytes = 256 * 32 * 4;  // [byte][lane] f16x2
 constexpr int kIqRedBytes = kIqWarps * 32 * 16 * 4;
 
+// Shared address of the table entry for byte `b` (compile-time 0..3) of q:
+// one byte permute (zero-extended byte) and one multiply-add.
+__device__ __forceinline__ uint32_t lut_addr(uint32_t q, int b, uint32_t lut_lane) {
+  const uint32_t byte = __byte_perm(q, 0u, 0x4440u | (uint32_t)b);
+  uint32_t a;
+  asm("mad.lo.u32 %0, %1, 128, %2;" : "=r"(a) : "r"(byte), "r"(lut_lane));
+  return a;
+}
+
 // One pass of a warp over its super-steps (at most SMAX) for up to 8*NT
 // tokens.  All block loads of the pass are issued first, so a warp has up to
 // SMAX * 1.25 KB in flight before it decodes anything.
@@ -231,11 +240,11 @@ __device__ __forceinline__ void iq4_pass(float (&acc)[4][4], const uint8_t* __re
 #pragma unroll
     for (int i = 0; i < 8; i++) {  // index bytes 2i, 2i+1 of the block
       const uint32_t qwa = qa[i >> 1], qwb = qb[i >> 1];
-      const int sh = (i & 1) * 16;
-      const uint32_t a0 = hmul2(lds32(lut_lane + ((qwa >> sh) & 0xFFu) * 128u), dda);
-      const uint32_t a2 = hmul2(lds32(lut_lane + ((qwa >> (sh + 8)) & 0xFFu) * 128u), dda);
-      const uint32_t a1 = hmul2(lds32(lut_lane + ((qwb >> sh) & 0xFFu) * 128u), ddb);
-      const uint32_t a3 = hmul2(lds32(lut_lane + ((qwb >> (sh + 8)) & 0xFFu) * 128u), ddb);
+      const int bs = (i & 1) * 2;  // byte of the word
+      const uint32_t a0 = hmul2(lds32(lut_addr(qwa, bs, lut_lane)), dda);
+      const uint32_t a2 = hmul2(lds32(lut_addr(qwa, bs + 1, lut_lane)), dda);
+      const uint32_t a1 = hmul2(lds32(lut_addr(qwb, bs, lut_lane)), ddb);
+      const uint32_t a3 = hmul2(lds32(lut_addr(qwb, bs + 1, lut_lane)), ddb);
 #pragma unroll
       for (int j = 0; j < NT; j++) {
         const uint32_t b0 = __byte_perm(xw[j][i], xw[j][i + 8], 0x5410);  // (x_2i, x_2i+16)
@@ -307,15 +316,17 @@ __global__ void __launch_bounds__(kIqWarps * 32, 4)
         for (int c = 0; c < 4; c++) acc[j][c] = 0.f;
       if (ng <= 8) iq4_range<1>(acc, de, rowb, ra, rb, s_lo, s_hi, tig, xr, lut_lane);
       else iq4_range<2>(acc, de, rowb, ra, rb, s_lo, s_hi, tig, xr, lut_lane);
-      // meet the other warps: red[warp][token slot][row]
+      // meet the other warps: red[warp][token slot][row] (used token tiles only)
       float* r = red + warp * (32 * 16);
 #pragma unroll
-      for (int j = 0; j < 4; j++) {
-        const int t0 = 8 * j + 2 * tig;
-        r[t0 * 16 + grp] = acc[j][0];
-        r[(t0 + 1) * 16 + grp] = acc[j][1];
-        r[t0 * 16 + grp + 8] = acc[j][2];
-        r[(t0 + 1) * 16 + grp + 8] = acc[j][3];
+      for (int j = 0; j < 2; j++) {
+        if (8 * j < ng) {
+          const int t0 = 8 * j + 2 * tig;
+          r[t0 * 16 + grp] = acc[j][0];
+          r[(t0 + 1) * 16 + grp] = acc[j][1];
+          r[t0 * 16 + grp + 8] = acc[j][2];
+          r[(t0 + 1) * 16 + grp + 8] = acc[j][3];
+        }
       }
       __syncthreads();
       for (int idx = threadIdx.x; idx < 16 * ng; idx += kIqWarps * 32) {

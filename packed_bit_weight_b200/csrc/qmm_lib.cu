@@ -162,22 +162,30 @@ template <int FMT, int NT, int SPW, int WPC = kLdgWarps, int MINB = 2>
 static qmm_status launch_gemv_ldg(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st) {
   const int n = (int)w->n, k = (int)w->k;
   const int tiles = (n + 15) / 16;
+  // Measurement knobs: QMM_GEMV_NOPDL=1 drops programmatic dependent launch,
+  // QMM_GEMV_SMEM_PAD=<bytes> reserves unused shared memory per CTA (caps
+  // the CTAs per SM).
+  const char* nopdl = getenv("QMM_GEMV_NOPDL");
+  const char* pad = getenv("QMM_GEMV_SMEM_PAD");
+  const int pad_bytes = pad ? atoi(pad) : 0;
+  auto kern = gemv_fp4_ldg_kernel<FMT, NT, SPW, WPC, MINB>;
+  if (pad_bytes > 0 &&
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pad_bytes) != cudaSuccess)
+    return QMM_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(tiles);
   cfg.blockDim = dim3(WPC * 32);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = pad_bytes > 0 ? pad_bytes : 0;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = (nopdl && nopdl[0] == '1') ? 0 : 1;
   const uint8_t* codes = static_cast<const uint8_t*>(w->data);
   const uint8_t* scales = static_cast<const uint8_t*>(w->scales);
   const float g = w->global_scale;
-  if (cudaLaunchKernelEx(&cfg, gemv_fp4_ldg_kernel<FMT, NT, SPW, WPC, MINB>, codes, scales, x, y, n, k, m, g) !=
-      cudaSuccess)
-    return QMM_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kern, codes, scales, x, y, n, k, m, g) != cudaSuccess) return QMM_ERR_CUDA;
   set_variant("gemv_fp4_ldg<fmt=%d,nt=%d,spw=%d,wpc=%d,minb=%d,tiles=%d>", FMT, NT, SPW, WPC, MINB, tiles);
   return launch_status();
 }
