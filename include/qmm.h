@@ -195,11 +195,67 @@ qmm_status qmm_grouped_gemv_noalloc(const qmm_weights* experts, const uint16_t* 
                                     const int32_t* topk_ids, int64_t t, int64_t topk, uint16_t* y,
                                     void* stream);
 
-enum { QMM_OP_DEQUANT = 0, QMM_OP_GEMV = 1, QMM_OP_GEMM = 2, QMM_OP_ROUTE = 3, QMM_OP_GROUPED = 4 };
+/* Router of a mixture-of-experts layer ("Mark-Experimental-V3-8B", section
+ * "Mixture-of-Experts (MoE)": s_{t,e} = Softmax(x_t W_router + b_e), the 4
+ * experts of largest score are active, each weighted by g_i).
+ * For every token: z_e = fp32(sum_k x[k] w_router[e][k] + bias[e]) with the
+ * sum taken in fp64 (every fp16 product is exact there) and rounded once;
+ * s = softmax(z) in fp32; topk_ids = the topk experts of largest z, larger
+ * first, equal z to the lower index; topk_weights = their s (no
+ * renormalisation over the chosen experts).
+ *   x             device, [t][k] fp16 activations
+ *   w_router      device, [num_experts][k] fp16 (a quantised router is
+ *                 decoded once with qmm_dequant)
+ *   bias          device, [num_experts] fp32 (the b_e of the formula)
+ *   topk_ids      device, [t][topk] int32 out
+ *   topk_weights  device, [t][topk] fp32 out
+ *   logits        device, [t][num_experts] fp32 out (z), or NULL
+ * Limits: 1 <= topk <= num_experts <= 256, k % 8 == 0.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, NOT_SM100, CUDA. */
+qmm_status qmm_router_topk(const uint16_t* x, const uint16_t* w_router, const float* bias, int64_t t,
+                           int64_t k, int64_t num_experts, int64_t topk, int32_t* topk_ids,
+                           float* topk_weights, float* logits, void* stream);
+
+/* Routed-expert block of a mixture-of-experts layer ("Mark-Experimental-V3-8B",
+ * section "Mixture-of-Experts (MoE)": F_i(x) = (SiLU(x W_gate) * (x W_up))
+ * W_down, output sum over the chosen experts of g_i F_i(x); the expert
+ * weights are contiguous 3-D tensors ffn_gate_exps / ffn_up_exps /
+ * ffn_down_exps, section "Quantization"):
+ *   out[t][:] = sum_s topk_weights[t][s] * W_down,e (h_{t,s}),
+ *   h_{t,s}   = fp16(SiLU(W_gate,e x_t) * (W_up,e x_t)),  e = topk_ids[t][s].
+ * Three kernels after the routing sort: gate and up are multiplied in one
+ * pass over the same row tiles with SiLU(gate) * up applied before the only
+ * fp16 rounding of h; the down projection multiplies each expert's pairs,
+ * scales them by g in fp32 and keeps them in fp32; a last pass adds a
+ * token's slots in slot order and rounds once to fp16.  The shared experts
+ * of the formula are this same call with ids {0, 1} and weights 1.
+ *   gate, up     IQ4_NL stacks of num_experts matrices [f][d] (same f, d, E)
+ *   down         IQ4_NL stack of num_experts matrices [d][f]
+ *   x            device, [t][d] fp16
+ *   topk_ids     device, [t][topk] int32 (ids out of range: their pairs are
+ *                left out, QMM_ERR_DEVICE_FAULT set in the error word)
+ *   topk_weights device, [t][topk] fp32
+ *   out          device, [t][d] fp16
+ *   ws           device workspace (qmm_workspace_bytes(QMM_OP_MOE, gate, 0,
+ *                t, topk)), laid out as offsets [E+1] int32 | pair_perm
+ *                [t*topk] int32 | h [t*topk][f] fp16 | g-scaled slot outputs
+ *                [t*topk][d] fp32, each part starting on a 256-byte
+ *                boundary; after the call h is readable there (pairs with an
+ *                out-of-range id hold stale data)
+ * Limits: d % 128 == 0, f % 128 == 0 (whole 4-block super-steps per row).
+ * Errors: as qmm_grouped_gemv. */
+qmm_status qmm_moe_routed(const qmm_weights* gate, const qmm_weights* up, const qmm_weights* down,
+                          const uint16_t* x, const int32_t* topk_ids, const float* topk_weights,
+                          int64_t t, int64_t topk, uint16_t* out, void* ws, size_t ws_bytes,
+                          void* stream);
+
+enum { QMM_OP_DEQUANT = 0, QMM_OP_GEMV = 1, QMM_OP_GEMM = 2, QMM_OP_ROUTE = 3, QMM_OP_GROUPED = 4,
+       QMM_OP_MOE = 5 };
 
 /* Device workspace bytes an operation needs for these sizes (0 = none).
  * `w` may be NULL for QMM_OP_ROUTE; `num_experts` is taken from `w` except
- * for QMM_OP_ROUTE, where it is passed in `m`. */
+ * for QMM_OP_ROUTE, where it is passed in `m`.  For QMM_OP_MOE `w` is the
+ * gate stack (f = w->n, d = w->k). */
 size_t qmm_workspace_bytes(int32_t op, const qmm_weights* w, int64_t m, int64_t t, int64_t topk);
 
 /* Synchronise `stream`, then read and clear this device's error word.

@@ -265,14 +265,29 @@ __device__ __forceinline__ void iq4_range(float (&acc)[4][4], const uint8_t* __r
     iq4_pass<NT, SMAX>(acc, de, rowb, ra, rb, s0, min(s0 + SMAX, s_hi), tig, xr, lut_lane);
 }
 
+// Epilogue of the IQ4_NL expert kernel.
+//   IQ_OUT_F16: y[pair][row] = fp16(acc)                        (plain product)
+//   IQ_SWIGLU:  the item multiplies the same 16-row tile of two matrices (gate,
+//               up) and writes y[pair][row] = fp16(SiLU(gate) * up), with
+//               SiLU(z) = z / (1 + e^-z) in fp32 ("Mark-Experimental-V3-8B",
+//               section "Mixture-of-Experts (MoE)": F = (SiLU(x W_gate) *
+//               (x W_up)) W_down).
+//   IQ_SCALED_F32: yf[pair][row] = gw[pair] * acc in fp32 (the routing weight
+//               g_i of the pair applied in the down projection; the slots of a
+//               token are added by combine_kernel).
+enum { IQ_OUT_F16 = 0, IQ_SWIGLU = 1, IQ_SCALED_F32 = 2 };
+constexpr int kIqGateBytes = 16 * 16 * 4;  // [token slot][row] fp32 gate values
+
+template <int MODE>
 __global__ void __launch_bounds__(kIqWarps * 32, 4)
-    grouped_iq4_kernel(const uint8_t* __restrict__ data, int64_t dstride, const uint16_t* __restrict__ x,
-                       int x_per_pair, int topk, const int32_t* __restrict__ offsets,
-                       const int32_t* __restrict__ perm, int m_plain, uint16_t* __restrict__ y, int n, int k,
-                       int E) {
+    grouped_iq4_kernel(const uint8_t* __restrict__ data, int64_t dstride, const uint8_t* __restrict__ data2,
+                       int64_t dstride2, const uint16_t* __restrict__ x, int x_per_pair, int topk,
+                       const int32_t* __restrict__ offsets, const int32_t* __restrict__ perm, int m_plain,
+                       void* __restrict__ yout, const float* __restrict__ gw, int n, int k, int E) {
   extern __shared__ __align__(16) uint8_t smem_iq[];
   const uint32_t lut = smem_addr(smem_iq);
   float* red = reinterpret_cast<float*>(smem_iq + kIqLutBytes);  // [warp][32 token slots][16 rows]
+  float* gsm = reinterpret_cast<float*>(smem_iq + kIqLutBytes + kIqRedBytes);  // IQ_SWIGLU gate values
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, grp = lane >> 2, tig = lane & 3;
   for (int i = threadIdx.x; i < 256 * 32; i += kIqWarps * 32) {
     const int v = i >> 5;
@@ -287,6 +302,7 @@ __global__ void __launch_bounds__(kIqWarps * 32, 4)
   const int s_lo = warp * steps / kIqWarps, s_hi = (warp + 1) * steps / kIqWarps;
   const int64_t rowb = (int64_t)(k >> 5) * 18;  // bytes per row
   const int items = tiles * E;
+  constexpr int kHalves = (MODE == IQ_SWIGLU) ? 2 : 1;
   for (int item = blockIdx.x; item < items; item += gridDim.x) {
     const int e = item / tiles, tile = item % tiles;
     int start = 0, cnt = m_plain;
@@ -295,7 +311,6 @@ __global__ void __launch_bounds__(kIqWarps * 32, 4)
       cnt = offsets[e + 1] - start;
     }
     if (cnt <= 0) continue;  // uniform across the CTA
-    const uint8_t* de = data + (int64_t)e * dstride;
     const int ra = min(tile * 16 + grp, n - 1), rb = min(tile * 16 + grp + 8, n - 1);
     for (int tok0 = 0; tok0 < cnt; tok0 += 16) {  // up to 16 gathered tokens per pass
       const int ng = min(16, cnt - tok0);
@@ -309,38 +324,55 @@ __global__ void __launch_bounds__(kIqWarps * 32, 4)
           xr[j] = x + (int64_t)((offsets && !x_per_pair) ? pr / topk : pr) * k;
         }
       }
-      float acc[4][4];
+#pragma unroll 1
+      for (int half = 0; half < kHalves; half++) {
+        const uint8_t* de = half ? data2 + (int64_t)e * dstride2 : data + (int64_t)e * dstride;
+        float acc[4][4];
 #pragma unroll
-      for (int j = 0; j < 4; j++)
+        for (int j = 0; j < 4; j++)
 #pragma unroll
-        for (int c = 0; c < 4; c++) acc[j][c] = 0.f;
-      if (ng <= 8) iq4_range<1>(acc, de, rowb, ra, rb, s_lo, s_hi, tig, xr, lut_lane);
-      else iq4_range<2>(acc, de, rowb, ra, rb, s_lo, s_hi, tig, xr, lut_lane);
-      // meet the other warps: red[warp][token slot][row] (used token tiles only)
-      float* r = red + warp * (32 * 16);
+          for (int c = 0; c < 4; c++) acc[j][c] = 0.f;
+        if (ng <= 8) iq4_range<1>(acc, de, rowb, ra, rb, s_lo, s_hi, tig, xr, lut_lane);
+        else iq4_range<2>(acc, de, rowb, ra, rb, s_lo, s_hi, tig, xr, lut_lane);
+        // meet the other warps: red[warp][token slot][row] (used token tiles only)
+        float* r = red + warp * (32 * 16);
 #pragma unroll
-      for (int j = 0; j < 2; j++) {
-        if (8 * j < ng) {
-          const int t0 = 8 * j + 2 * tig;
-          r[t0 * 16 + grp] = acc[j][0];
-          r[(t0 + 1) * 16 + grp] = acc[j][1];
-          r[t0 * 16 + grp + 8] = acc[j][2];
-          r[(t0 + 1) * 16 + grp + 8] = acc[j][3];
+        for (int j = 0; j < 2; j++) {
+          if (8 * j < ng) {
+            const int t0 = 8 * j + 2 * tig;
+            r[t0 * 16 + grp] = acc[j][0];
+            r[(t0 + 1) * 16 + grp] = acc[j][1];
+            r[t0 * 16 + grp + 8] = acc[j][2];
+            r[(t0 + 1) * 16 + grp + 8] = acc[j][3];
+          }
         }
-      }
-      __syncthreads();
-      for (int idx = threadIdx.x; idx < 16 * ng; idx += kIqWarps * 32) {
-        const int row = idx & 15, slot = idx >> 4;
-        float v = 0.f;
+        __syncthreads();
+        for (int idx = threadIdx.x; idx < 16 * ng; idx += kIqWarps * 32) {
+          const int row = idx & 15, slot = idx >> 4;
+          float v = 0.f;
 #pragma unroll
-        for (int w = 0; w < kIqWarps; w++) v += red[w * 512 + slot * 16 + row];
-        const int grow = tile * 16 + row;
-        if (grow < n) {
-          const int64_t pr = offsets ? perm[start + tok0 + slot] : tok0 + slot;
-          y[pr * n + grow] = f32_to_f16_bits(v);
+          for (int w = 0; w < kIqWarps; w++) v += red[w * 512 + slot * 16 + row];
+          if (MODE == IQ_SWIGLU && half == 0) {
+            gsm[idx] = v;  // gate value, kept for the up pass
+            continue;
+          }
+          const int grow = tile * 16 + row;
+          if (grow < n) {
+            const int64_t pr = offsets ? perm[start + tok0 + slot] : tok0 + slot;
+            if (MODE == IQ_SCALED_F32) {
+              static_cast<float*>(yout)[pr * n + grow] = gw[pr] * v;
+            } else {
+              float o = v;
+              if (MODE == IQ_SWIGLU) {
+                const float gv = gsm[idx];
+                o = gv / (1.0f + expf(-gv)) * v;
+              }
+              static_cast<uint16_t*>(yout)[pr * n + grow] = f32_to_f16_bits(o);
+            }
+          }
         }
+        __syncthreads();
       }
-      __syncthreads();
     }
   }
 }

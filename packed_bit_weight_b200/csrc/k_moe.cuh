@@ -1,0 +1,115 @@
+// k_moe.cuh -- the pieces around the routed-expert GEMVs of a mixture-of-
+// experts layer ("Mark-Experimental-V3-8B", section "Mixture-of-Experts
+// (MoE)": s = Softmax(x W_router + b), top-4 experts with weights g_i,
+// F(x) = (SiLU(x W_gate) * (x W_up)) W_down, routed output sum_i g_i F_i(x)).
+//
+// router_topk_kernel: one CTA per token; warps take experts, lanes split k;
+//   the dot product is accumulated in fp64 (products of fp16 values are exact
+//   there) and rounded once, with the bias, to an fp32 logit; softmax in fp32;
+//   the top-k is taken on the fp32 logits, larger first, ties to the lower
+//   expert index; g = the softmax score of each chosen expert.
+// combine_kernel: out[t][j] = sum_s g[t][s] * y[t][s][j]: the down
+//   projection's epilogue already scaled each slot by g in fp32; the slots are
+//   added in slot order (deterministic) and rounded once to fp16.
+// (SiLU(gate) * up is fused into the grouped IQ4_NL kernel's epilogue.)
+#pragma once
+#include "qmm_dev.cuh"
+
+namespace qmm {
+
+constexpr int kRouterMaxExperts = 256;
+constexpr int kRouterMaxTopk = 16;
+
+__global__ void __launch_bounds__(256) router_topk_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ w,
+                                                          const float* __restrict__ b, int k, int E, int topk,
+                                                          int32_t* __restrict__ ids, float* __restrict__ g,
+                                                          float* __restrict__ logits_out) {
+  __shared__ float z[kRouterMaxExperts];
+  const int tok = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint16_t* xr = x + (int64_t)tok * k;
+  for (int e = warp; e < E; e += 8) {
+    const uint16_t* wr = w + (int64_t)e * k;
+    double s = 0.0;
+    for (int kk = lane * 8; kk < k; kk += 256) {
+      const uint4 xv = *reinterpret_cast<const uint4*>(xr + kk);
+      const uint4 wv = *reinterpret_cast<const uint4*>(wr + kk);
+      const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w}, ws[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+      for (int i = 0; i < 4; i++) {
+        const float2 xf = f16x2_to_f32x2(xs[i]), wf = f16x2_to_f32x2(ws[i]);
+        s = fma((double)xf.x, (double)wf.x, s);
+        s = fma((double)xf.y, (double)wf.y, s);
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, off);
+    if (lane == 0) {
+      const float zz = __double2float_rn(s + (double)b[e]);
+      z[e] = zz;
+      if (logits_out) logits_out[(int64_t)tok * E + e] = zz;
+    }
+  }
+  __syncthreads();
+  if (warp != 0) return;
+  float mx = -INFINITY;
+  for (int e = lane; e < E; e += 32) mx = fmaxf(mx, z[e]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+  float den = 0.f;
+  for (int e = lane; e < E; e += 32) den += expf(z[e] - mx);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xFFFFFFFFu, den, off);
+  uint32_t taken = 0u;  // bit i: expert lane + 32 i already chosen
+  for (int j = 0; j < topk; j++) {
+    float bv = -INFINITY;
+    int be = E;  // larger logit first, ties to the lower index
+    for (int i = 0, e = lane; e < E; i++, e += 32) {
+      if ((taken >> i) & 1u) continue;
+      const float v = z[e];
+      if (v > bv || (v == bv && e < be)) { bv = v; be = e; }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
+      const int oe = __shfl_xor_sync(0xFFFFFFFFu, be, off);
+      if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+    }
+    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+    if (lane == 0) {
+      ids[(int64_t)tok * topk + j] = be;
+      g[(int64_t)tok * topk + j] = expf(bv - mx) / den;
+    }
+  }
+}
+
+// out[t][j] = fp16(sum_s yg[t][s][j]): the slots' g-scaled fp32 outputs
+// added in slot order, 8 outputs per thread (n % 8 == 0).  Slots whose
+// expert id is out of range were never computed and are left out.
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ yg, const int32_t* __restrict__ ids,
+                                                      int E, int t, int topk, int n, uint16_t* __restrict__ out) {
+  const int64_t per_tok = n / 8;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < (int64_t)t * per_tok;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t tok = i / per_tok;
+    const int j = (int)(i % per_tok) * 8;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int s = 0; s < topk; s++) {
+      const int e = ids[tok * topk + s];
+      if (e < 0 || e >= E) continue;
+      const float* src = yg + (tok * topk + s) * n + j;
+      const float4 v0 = *reinterpret_cast<const float4*>(src);
+      const float4 v1 = *reinterpret_cast<const float4*>(src + 4);
+      acc[0] += v0.x; acc[1] += v0.y; acc[2] += v0.z; acc[3] += v0.w;
+      acc[4] += v1.x; acc[5] += v1.y; acc[6] += v1.z; acc[7] += v1.w;
+    }
+    uint4 o;
+    o.x = f32x2_to_f16x2(acc[0], acc[1]);
+    o.y = f32x2_to_f16x2(acc[2], acc[3]);
+    o.z = f32x2_to_f16x2(acc[4], acc[5]);
+    o.w = f32x2_to_f16x2(acc[6], acc[7]);
+    *reinterpret_cast<uint4*>(out + tok * n + j) = o;
+  }
+}
+
+}  // namespace qmm

@@ -18,6 +18,7 @@
 #include "k_gemv.cuh"
 #include "k_gemm.cuh"
 #include "k_grouped.cuh"
+#include "k_moe.cuh"
 
 namespace qmm {
 
@@ -447,22 +448,34 @@ static qmm_status gemm_by_gemv(const qmm_weights* w, const uint16_t* x, int64_t 
 }
 
 // IQ4_NL streaming kernel (k % 128 == 0): persistent CTAs over (expert, tile).
-static qmm_status launch_iq4_stream(const qmm_weights* w, const uint16_t* x, int x_per_pair, int64_t topk,
-                                   const int32_t* offsets, const int32_t* perm, int m_plain, uint16_t* y,
-                                   cudaStream_t st, const DevInfo* di) {
-  const size_t smem = kIqLutBytes + kIqRedBytes;
-  if (cudaFuncSetAttribute(grouped_iq4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+// MODE selects the epilogue (IQ_OUT_F16, IQ_SWIGLU with w2 the up matrix,
+// IQ_SCALED_F32 with gw the per-pair weights and an fp32 output).
+template <int MODE>
+static qmm_status launch_iq4_mode(const qmm_weights* w, const qmm_weights* w2, const uint16_t* x, int x_per_pair,
+                                  int64_t topk, const int32_t* offsets, const int32_t* perm, int m_plain, void* y,
+                                  const float* gw, cudaStream_t st, const DevInfo* di) {
+  const size_t smem = kIqLutBytes + kIqRedBytes + kIqGateBytes;
+  if (cudaFuncSetAttribute(grouped_iq4_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
     return QMM_ERR_CUDA;
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, grouped_iq4_kernel, kIqWarps * 32, smem) != cudaSuccess ||
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, grouped_iq4_kernel<MODE>, kIqWarps * 32, smem) !=
+          cudaSuccess ||
       per_sm < 1)
     return QMM_ERR_CUDA;
   const int64_t items = ((w->n + 15) / 16) * w->num_experts;
   const int64_t grid = items < (int64_t)per_sm * di->sms ? items : (int64_t)per_sm * di->sms;
-  grouped_iq4_kernel<<<(unsigned)grid, kIqWarps * 32, smem, st>>>(
-      static_cast<const uint8_t*>(w->data), w->expert_data_stride, x, x_per_pair, (int)topk, offsets, perm, m_plain, y,
-      (int)w->n, (int)w->k, (int)w->num_experts);
+  grouped_iq4_kernel<MODE><<<(unsigned)grid, kIqWarps * 32, smem, st>>>(
+      static_cast<const uint8_t*>(w->data), w->expert_data_stride,
+      w2 ? static_cast<const uint8_t*>(w2->data) : nullptr, w2 ? w2->expert_data_stride : 0, x, x_per_pair,
+      (int)topk, offsets, perm, m_plain, y, gw, (int)w->n, (int)w->k, (int)w->num_experts);
   return launch_status();
+}
+
+static qmm_status launch_iq4_stream(const qmm_weights* w, const uint16_t* x, int x_per_pair, int64_t topk,
+                                   const int32_t* offsets, const int32_t* perm, int m_plain, uint16_t* y,
+                                   cudaStream_t st, const DevInfo* di) {
+  return launch_iq4_mode<IQ_OUT_F16>(w, nullptr, x, x_per_pair, topk, offsets, perm, m_plain, y, nullptr, st, di);
 }
 
 template <int FMT>
@@ -713,9 +726,12 @@ qmm_status qmm_grouped_gemv(const qmm_weights* experts, const uint16_t* x, int32
 }
 
 size_t qmm_workspace_bytes(int32_t op, const qmm_weights* w, int64_t m, int64_t t, int64_t topk) {
-  if (op == QMM_OP_GROUPED) {
-    if (!w || w->num_experts < 1 || t < 0 || topk < 0) return 0;
-    return align256(4 * (size_t)(w->num_experts + 1)) + align256(4 * (size_t)(t * topk));
+  if (op == QMM_OP_GROUPED || op == QMM_OP_MOE) {
+    if (!w || w->num_experts < 1 || t < 0 || topk < 0 || w->n < 0 || w->k < 0) return 0;
+    size_t b = align256(4 * (size_t)(w->num_experts + 1)) + align256(4 * (size_t)(t * topk));
+    if (op == QMM_OP_MOE)  // h [t*topk][f] fp16, g-scaled slot outputs [t*topk][d] fp32
+      b += align256(2 * (size_t)(t * topk) * (size_t)w->n) + align256(4 * (size_t)(t * topk) * (size_t)w->k);
+    return b;
   }
   (void)m;
   return 0;
@@ -756,6 +772,75 @@ qmm_status qmm_grouped_gemv_noalloc(const qmm_weights* experts, const uint16_t* 
   }
   set_variant("noalloc:route+grouped_gemv_generic<fmt=%d>", experts->fmt);
   return s;
+}
+
+qmm_status qmm_router_topk(const uint16_t* x, const uint16_t* w_router, const float* bias, int64_t t, int64_t k,
+                           int64_t num_experts, int64_t topk, int32_t* topk_ids, float* topk_weights, float* logits,
+                           void* stream) {
+  if (t < 0 || k < 0 || num_experts < 1 || topk < 1 || topk > num_experts) return QMM_ERR_INVALID_ARG;
+  if (num_experts > kRouterMaxExperts || k % 8 || t > INT32_MAX) return QMM_ERR_UNSUPPORTED_SHAPE;
+  DevInfo* di = nullptr;
+  qmm_status s = device_info(&di);
+  if (s != QMM_OK) return s;
+  if (t == 0) return QMM_OK;
+  if (!bias || !topk_ids || !topk_weights || (k > 0 && (!x || !w_router))) return QMM_ERR_INVALID_ARG;
+  if ((x && !aligned16(x)) || (w_router && !aligned16(w_router)) || !aligned16(bias) || !aligned16(topk_ids) ||
+      !aligned16(topk_weights) || (logits && !aligned16(logits)))
+    return QMM_ERR_MISALIGNED;
+  router_topk_kernel<<<(unsigned)t, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      x, w_router, bias, (int)k, (int)num_experts, (int)topk, topk_ids, topk_weights, logits);
+  set_variant("router_topk");
+  return launch_status();
+}
+
+qmm_status qmm_moe_routed(const qmm_weights* gate, const qmm_weights* up, const qmm_weights* down, const uint16_t* x,
+                          const int32_t* topk_ids, const float* topk_weights, int64_t t, int64_t topk, uint16_t* out,
+                          void* ws, size_t ws_bytes, void* stream) {
+  qmm_status s;
+  for (const qmm_weights* w : {gate, up, down}) {
+    if ((s = check_weights(w, true)) != QMM_OK) return s;
+    if ((s = check_expert_strides(w)) != QMM_OK) return s;
+    if (w->fmt != QMM_FMT_IQ4_NL) return QMM_ERR_UNSUPPORTED_SHAPE;
+  }
+  const int64_t f = gate->n, d = gate->k, E = gate->num_experts;
+  if (up->n != f || up->k != d || down->n != d || down->k != f || up->num_experts != E || down->num_experts != E)
+    return QMM_ERR_INVALID_ARG;
+  if ((s = check_routing(topk_ids, t, topk, E)) != QMM_OK) return s;
+  if (d % 128 || f % 128 || d > INT32_MAX / 2 || f > INT32_MAX / 2) return QMM_ERR_UNSUPPORTED_SHAPE;
+  DevInfo* di = nullptr;
+  if ((s = device_info(&di)) != QMM_OK) return s;
+  const int64_t P = t * topk;
+  if (P == 0 || d == 0) return QMM_OK;
+  if (!out || !x || !topk_weights) return QMM_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(x) || !aligned16(topk_weights)) return QMM_ERR_MISALIGNED;
+  const size_t need = qmm_workspace_bytes(QMM_OP_MOE, gate, 0, t, topk);
+  if (!ws || ws_bytes < need) return QMM_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QMM_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* p = static_cast<char*>(ws);
+  int32_t* offsets = reinterpret_cast<int32_t*>(p);
+  p += align256(4 * (size_t)(E + 1));
+  int32_t* perm = reinterpret_cast<int32_t*>(p);
+  p += align256(4 * (size_t)P);
+  uint16_t* h = reinterpret_cast<uint16_t*>(p);
+  p += align256(2 * (size_t)P * (size_t)f);
+  float* yg = reinterpret_cast<float*>(p);
+  route_kernel<<<1, kRouteThreads, 0, st>>>(topk_ids, (int)P, (int)E, offsets, perm);
+  if (cudaGetLastError() != cudaSuccess) return QMM_ERR_CUDA;
+  if (f == 0) {
+    // h is empty: every slot output is an empty sum
+    zero_fill_kernel<<<grid_for(t * d, 256, di->sms), 256, 0, st>>>(out, t * d);
+    set_variant("moe:route+zero_fill");
+    return launch_status();
+  }
+  if ((s = launch_iq4_mode<IQ_SWIGLU>(gate, up, x, 0, topk, offsets, perm, 0, h, nullptr, st, di)) != QMM_OK)
+    return s;
+  if ((s = launch_iq4_mode<IQ_SCALED_F32>(down, nullptr, h, 1, topk, offsets, perm, 0, yg, topk_weights, st, di)) !=
+      QMM_OK)
+    return s;
+  combine_kernel<<<grid_for(t * (d / 8), 256, di->sms), 256, 0, st>>>(yg, topk_ids, (int)E, (int)t, (int)topk, (int)d, out);
+  set_variant("moe:route+gate_up_swiglu_iq4+down_scaled_iq4+combine");
+  return launch_status();
 }
 
 qmm_status qmm_sync_check(void* stream) {

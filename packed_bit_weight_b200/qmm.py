@@ -20,7 +20,7 @@ FMT_IQ4_NL = 1
 FMT_FP4G16_F16 = 2
 FMT_FP4G16_E4M3 = 3
 
-OP_DEQUANT, OP_GEMV, OP_GEMM, OP_ROUTE, OP_GROUPED = 0, 1, 2, 3, 4
+OP_DEQUANT, OP_GEMV, OP_GEMM, OP_ROUTE, OP_GROUPED, OP_MOE = 0, 1, 2, 3, 4, 5
 
 STATUS = {0: "QMM_OK", 1: "QMM_ERR_INVALID_ARG", 2: "QMM_ERR_UNSUPPORTED_SHAPE", 3: "QMM_ERR_MISALIGNED",
           4: "QMM_ERR_NOT_SM100", 5: "QMM_ERR_CUDA", 6: "QMM_ERR_TIMEOUT", 7: "QMM_ERR_DEVICE_FAULT",
@@ -62,6 +62,8 @@ def _lib():
             "qmm_route": (i32, [vp, i64, i64, i64, vp, vp, vp, sz, vp]),
             "qmm_grouped_gemv": (i32, [W, vp, i32, vp, i64, i64, vp, vp, sz, vp]),
             "qmm_grouped_gemv_noalloc": (i32, [W, vp, i32, vp, i64, i64, vp, vp]),
+            "qmm_router_topk": (i32, [vp, vp, vp, i64, i64, i64, i64, vp, vp, vp, vp]),
+            "qmm_moe_routed": (i32, [W, W, W, vp, vp, vp, i64, i64, vp, vp, sz, vp]),
             "qmm_workspace_bytes": (sz, [i32, W, i64, i64, i64]),
             "qmm_sync_check": (i32, [vp]),
             "qmm_status_string": (ctypes.c_char_p, [i32]),
@@ -112,6 +114,8 @@ class PackedWeights:
     scales: torch.Tensor | None
     global_scale: float = 1.0
     experts: int = 1
+    data_stride: int | None = None    # bytes between experts (default: data split evenly)
+    scale_stride: int | None = None
 
     def desc(self) -> qmm_weights:
         d = qmm_weights()
@@ -119,10 +123,26 @@ class PackedWeights:
         d.data = ctypes.c_void_p(self.data.data_ptr()) if self.data is not None else None
         d.scales = ctypes.c_void_p(self.scales.data_ptr()) if self.scales is not None else None
         d.global_scale, d.reserved2, d.num_experts = float(self.global_scale), 0, self.experts
-        d.expert_data_stride = self.data.numel() // self.experts if self.data is not None else 0
-        d.expert_scale_stride = (self.scales.numel() * self.scales.element_size() // self.experts
-                                 if self.scales is not None else 0)
+        if self.data_stride is not None:
+            d.expert_data_stride = self.data_stride
+        else:
+            d.expert_data_stride = self.data.numel() // self.experts if self.data is not None else 0
+        if self.scale_stride is not None:
+            d.expert_scale_stride = self.scale_stride
+        else:
+            d.expert_scale_stride = (self.scales.numel() * self.scales.element_size() // self.experts
+                                     if self.scales is not None else 0)
         return d
+
+    def rows(self, r0: int, r1: int) -> "PackedWeights":
+        """View of rows [r0, r1) of every matrix of the stack (no copy): e.g.
+        the gate and up halves of an expert stack stored as [E][2f][k]."""
+        db, sb = qmm_data_bytes(self.fmt, 1, self.k), qmm_scale_bytes(self.fmt, 1, self.k)
+        d = self.desc()
+        data = self.data.view(torch.uint8).reshape(-1)[r0 * db:]
+        scales = None if self.scales is None else self.scales.view(torch.uint8).reshape(-1)[r0 * sb:]
+        return PackedWeights(self.fmt, r1 - r0, self.k, data, scales, self.global_scale, self.experts,
+                             d.expert_data_stride, d.expert_scale_stride)
 
     @property
     def nbytes(self) -> int:
@@ -215,6 +235,32 @@ def qmm_grouped_gemv_noalloc(w: PackedWeights, x: torch.Tensor, topk_ids: torch.
                                            _ptr(topk_ids, 4, "topk_ids"), t, topk, _ptr(y, 2, "y"),
                                            _stream(stream)), "qmm_grouped_gemv_noalloc")
     return y
+
+
+def qmm_router_topk(x: torch.Tensor, w_router: torch.Tensor, bias: torch.Tensor, topk: int,
+                    topk_ids: torch.Tensor, topk_weights: torch.Tensor, logits: torch.Tensor | None = None,
+                    stream=None):
+    """Router logits (fp64 sums rounded once to fp32), fp32 softmax and the
+    top-k experts with their softmax weights."""
+    t, k = x.shape
+    E = w_router.shape[0]
+    _check(_lib().qmm_router_topk(_ptr(x, 2, "x"), _ptr(w_router, 2, "w_router"), _ptr(bias, 4, "bias"), t, k, E,
+                                  topk, _ptr(topk_ids, 4, "topk_ids"), _ptr(topk_weights, 4, "topk_weights"),
+                                  _ptr(logits, 4, "logits"), _stream(stream)), "qmm_router_topk")
+    return topk_ids, topk_weights
+
+
+def qmm_moe_routed(gate: PackedWeights, up: PackedWeights, down: PackedWeights, x: torch.Tensor,
+                   topk_ids: torch.Tensor, topk_weights: torch.Tensor, out: torch.Tensor,
+                   ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """out[t] = sum_s g[t][s] * W_down,e (SiLU(W_gate,e x_t) * W_up,e x_t)."""
+    dg, du, dd = gate.desc(), up.desc(), down.desc()
+    t, topk = topk_ids.shape
+    wp, wb = _ws(ws)
+    _check(_lib().qmm_moe_routed(ctypes.byref(dg), ctypes.byref(du), ctypes.byref(dd), _ptr(x, 2, "x"),
+                                 _ptr(topk_ids, 4, "topk_ids"), _ptr(topk_weights, 4, "topk_weights"), t, topk,
+                                 _ptr(out, 2, "out"), wp, wb, _stream(stream)), "qmm_moe_routed")
+    return out
 
 
 def qmm_sync_check(stream=None) -> int:

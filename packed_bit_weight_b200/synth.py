@@ -109,6 +109,14 @@ def gen_topk(rng: np.random.Generator, t: int, topk: int, experts: int) -> np.nd
     return ids
 
 
+def gen_router(rng: np.random.Generator, experts: int, k: int):
+    """Router weights [experts][k] as fp16 bits, N(0, 1/k) so that the logits
+    of N(0,1) activations are about N(0,1), and an fp32 bias N(0, 0.1^2)."""
+    w = _fp16_bits(rng.standard_normal((experts, k), dtype=np.float32) / np.float32(np.sqrt(max(k, 1))))
+    b = (rng.standard_normal(experts, dtype=np.float32) * np.float32(0.1)).astype(np.float32)
+    return w, b
+
+
 # ---------------------------------------------------------------------------
 # The five workloads
 # ---------------------------------------------------------------------------
@@ -165,6 +173,18 @@ def make_experts(experts=32, gate_up=(1792, 2560), down=(2560, 896), t=64, topk=
     x_dn = gen_x(rng, t, topk, down[1])
     ids = gen_topk(rng, t, topk, experts)
     return wgu, wdn, x_gu, x_dn, ids
+
+
+def make_moe(experts=32, f=896, d=2560, t=64, topk=4, seed=None):
+    """Routed-expert block inputs: gate+up stack [E][2f][d] (gate rows, then
+    up rows, as the grouped GEMV's stack), down stack [E][d][f], activations
+    [t][d], router weights [E][d] fp16 and bias [E] fp32."""
+    rng = np.random.default_rng(IQ4_EXPERTS.seed + 100 if seed is None else seed)
+    wgu = gen_iq4nl(rng, 2 * f, d, experts)
+    wdn = gen_iq4nl(rng, d, f, experts)
+    x = gen_x(rng, t, d)
+    wr, br = gen_router(rng, experts, d)
+    return wgu, wdn, x, wr, br
 
 
 def make_prefill(fmt: int = FMT_FP4G16_F16, m=None, n=None, k=None):

@@ -21,7 +21,8 @@ def _declared():
 
 def test_header_declares_the_boundary():
     names = _declared()
-    for want in ("qmm_dequant", "qmm_gemv", "qmm_gemm", "qmm_route", "qmm_grouped_gemv", "qmm_sync_check"):
+    for want in ("qmm_dequant", "qmm_gemv", "qmm_gemm", "qmm_route", "qmm_grouped_gemv", "qmm_router_topk",
+                 "qmm_moe_routed", "qmm_sync_check"):
         assert want in names
 
 
@@ -44,6 +45,25 @@ def test_size_functions_match_the_oracle():
     assert qmm.qmm_packed_bytes(3, 18560, 4096) == 42762244
     assert qmm.qmm_data_bytes(1, 1, 48) == 0          # k not a multiple of 32: invalid
     assert qmm.qmm_data_bytes(9, 1, 32) == 0          # bad format
+
+
+def test_moe_workspace_size():
+    """Host-side size rule of the routed-expert block's workspace: routing
+    offsets and permutation, h in fp16 and the fp32 slot outputs, each
+    rounded up to 256 bytes."""
+    from packed_bit_weight_b200 import qmm
+    import torch
+    a = lambda v: (v + 255) // 256 * 256
+    E, f, d, t, topk = 32, 896, 2560, 64, 4
+    gate = qmm.PackedWeights(1, f, d, torch.zeros(E * qmm.qmm_data_bytes(1, f, d), dtype=torch.uint8), None,
+                             1.0, E)
+    P = t * topk
+    want = a(4 * (E + 1)) + a(4 * P) + a(2 * P * f) + a(4 * P * d)
+    assert qmm.qmm_workspace_bytes(qmm.OP_MOE, gate, 0, t, topk) == want
+    assert qmm.qmm_workspace_bytes(qmm.OP_GROUPED, gate, 0, t, topk) == a(4 * (E + 1)) + a(4 * P)
+    view = gate.rows(f // 2, f)
+    assert view.desc().expert_data_stride == gate.desc().expert_data_stride
+    assert view.data.data_ptr() - gate.data.data_ptr() == (f // 2) * qmm.qmm_data_bytes(1, 1, d)
 
 
 def test_product_path_does_not_import_the_oracle():
