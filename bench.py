@@ -348,6 +348,46 @@ def grouped_workload(world, l2, peaks):
             "note": "one step = gate+up grouped GEMV then down grouped GEMV, each with its routing sort"}
 
 
+def moe_workload(world, l2, peaks, t=64, topk=4):
+    """Routed-expert MoE block (IQ4_NL, 32 experts, f=896, d=2560): router
+    top-4 then the fused gate/up + SiLU, the g-scaled down and the combine."""
+    import torch
+    from packed_bit_weight_b200 import qmm, synth
+    wgu, wdn, x, wr, br = synth.make_moe(t=t, topk=topk)
+    f = wgu.n // 2
+    gu0, dn0 = qmm.PackedWeights.from_host(wgu), qmm.PackedWeights.from_host(wdn)
+    per_set = gu0.nbytes + dn0.nbytes
+    R = max(2, math.ceil(4 * l2 / per_set))
+    sets = [(gu0, dn0)] + [(qmm.PackedWeights(1, gu0.n, gu0.k, gu0.data.clone(), None, 1.0, gu0.experts),
+                            qmm.PackedWeights(1, dn0.n, dn0.k, dn0.data.clone(), None, 1.0, dn0.experts))
+                           for _ in range(R - 1)]
+    views = [(gu.rows(0, f), gu.rows(f, 2 * f), dn) for gu, dn in sets]
+    xd = torch.from_numpy(x.view(np.int16)).cuda()
+    wrd = torch.from_numpy(wr.view(np.int16)).cuda()
+    brd = torch.from_numpy(br).cuda()
+    E = wgu.experts
+    ids = torch.empty((t, topk), dtype=torch.int32, device="cuda")
+    g = torch.empty((t, topk), dtype=torch.float32, device="cuda")
+    out = torch.empty((t, wgu.k), dtype=torch.int16, device="cuda")
+    ws = torch.empty((qmm.qmm_workspace_bytes(qmm.OP_MOE, views[0][0], 0, t, topk),), dtype=torch.uint8,
+                     device="cuda")
+
+    def launch(i):
+        gate, up, dn = views[i % R]
+        qmm.qmm_router_topk(xd, wrd, brd, topk, ids, g)
+        qmm.qmm_moe_routed(gate, up, dn, xd, ids, g, out, ws=ws)
+
+    per = timed_launches(launch, 2 * R, 10, 2, world)
+    variant = qmm.qmm_last_variant()
+    assert qmm.qmm_sync_check() == 0
+    hit = sorted(set(ids.cpu().numpy().reshape(-1).tolist()))
+    bytes_hit = len(hit) * per_set // E + wr.nbytes
+    return {"variant": "router_topk+" + variant, "gbs": bytes_hit / per / 1e9,
+            "frac_hbm": bytes_hit / per / 1e9 / peaks["hbm_gbs"], "us_per_step": per * 1e6,
+            "experts_hit": len(hit), "bytes_per_step": bytes_hit, "tokens": t,
+            "note": "one step = router top-4 + routed-expert block (5 kernels); bytes = weights of the experts hit"}
+
+
 def dequant_workload(world, l2, peaks):
     import torch
     from packed_bit_weight_b200 import qmm, synth
@@ -393,6 +433,8 @@ def extra_workloads(args, world, l2, peaks):
     out["fp4g16_prefill_gemm_2048x18560x4096"] = gemm_workload(synth.FMT_FP4G16_F16, world, l2, peaks)
     out["fp4g16_e4m3_prefill_gemm_2048x18560x4096"] = gemm_workload(synth.FMT_FP4G16_E4M3, world, l2, peaks)
     out["iq4nl_grouped_experts_t64_top4"] = grouped_workload(world, l2, peaks)
+    out["iq4nl_moe_block_t64_top4"] = moe_workload(world, l2, peaks, t=64)
+    out["iq4nl_moe_block_t1_top4"] = moe_workload(world, l2, peaks, t=1)
     out["fp4g16_dequant_in_proj"] = dequant_workload(world, l2, peaks)
     return out
 
@@ -401,7 +443,8 @@ def profile_case(name: str) -> int:
     """Small cases for ncu captures (a few hundred MB on the device, a handful
     of launches): gemv (in_proj, m=1, 4 rotating copies > L2), gemm (the
     2048-token prefill, two launches), grouped (routed experts, 2 rotating
-    sets), dequant (in_proj)."""
+    sets), moe (router + routed-expert block, 2 rotating sets), dequant
+    (in_proj)."""
     import torch
     from packed_bit_weight_b200 import qmm, synth
     if name == "gemv":
@@ -436,6 +479,22 @@ def profile_case(name: str) -> int:
             gu, dn = sets[i % 2]
             qmm.qmm_grouped_gemv(gu, xg, d_ids, ygu, x_per_pair=False, ws=ws)
             qmm.qmm_grouped_gemv(dn, xdn, d_ids, ydn, x_per_pair=True, ws=ws)
+    elif name == "moe":
+        wgu, wdn, x, wr, br = synth.make_moe()
+        f = wgu.n // 2
+        sets = [(qmm.PackedWeights.from_host(wgu), qmm.PackedWeights.from_host(wdn)) for _ in range(2)]
+        xd = torch.from_numpy(x.view(np.int16)).cuda()
+        t, topk = x.shape[0], 4
+        ids = torch.empty((t, topk), dtype=torch.int32, device="cuda")
+        g = torch.empty((t, topk), dtype=torch.float32, device="cuda")
+        out = torch.empty((t, wgu.k), dtype=torch.int16, device="cuda")
+        ws = torch.empty((qmm.qmm_workspace_bytes(qmm.OP_MOE, sets[0][0].rows(0, f), 0, t, topk),),
+                         dtype=torch.uint8, device="cuda")
+        for i in range(4):
+            gu, dn = sets[i % 2]
+            qmm.qmm_router_topk(xd, torch.from_numpy(wr.view(np.int16)).cuda(), torch.from_numpy(br).cuda(), topk,
+                                ids, g)
+            qmm.qmm_moe_routed(gu.rows(0, f), gu.rows(f, 2 * f), dn, xd, ids, g, out, ws=ws)
     elif name == "dequant":
         p, _ = synth.make_gemv(synth.FP4_IN_PROJ)
         w = qmm.PackedWeights.from_host(p)

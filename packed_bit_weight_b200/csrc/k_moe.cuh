@@ -4,8 +4,9 @@
 // F(x) = (SiLU(x W_gate) * (x W_up)) W_down, routed output sum_i g_i F_i(x)).
 //
 // router_topk_kernel: one CTA per token; warps take experts, lanes split k;
-//   the dot product is accumulated in fp64 (products of fp16 values are exact
-//   there) and rounded once, with the bias, to an fp32 logit; softmax in fp32;
+//   every fp16 x fp16 product is exact in fp32 and the dot product is
+//   accumulated in fp64, then rounded once, with the bias, to an fp32 logit;
+//   softmax in fp32;
 //   the top-k is taken on the fp32 logits, larger first, ties to the lower
 //   expert index; g = the softmax score of each chosen expert.
 // combine_kernel: out[t][j] = sum_s g[t][s] * y[t][s][j]: the down
@@ -20,6 +21,22 @@ namespace qmm {
 constexpr int kRouterMaxExperts = 256;
 constexpr int kRouterMaxTopk = 16;
 
+// Router logits: warp w takes experts w, w+8, w+16, w+24 (then the next 32),
+// lanes take 8 consecutive k of every 256; each fp16 x fp16 product is exact
+// in fp32 and is added in fp64.  Loads of four k-chunks are issued before
+// their products so the warp keeps several memory requests in flight.
+constexpr int kRouterEB = 4;  // experts per warp per pass
+
+__device__ __forceinline__ void router_acc8(double& s, const uint4& xv, const uint4& wv) {
+  const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w}, ws[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+  for (int i = 0; i < 4; i++) {
+    const float2 xf = f16x2_to_f32x2(xs[i]), wf = f16x2_to_f32x2(ws[i]);
+    s += (double)(xf.x * wf.x);  // exact product
+    s += (double)(xf.y * wf.y);
+  }
+}
+
 __global__ void __launch_bounds__(256) router_topk_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ w,
                                                           const float* __restrict__ b, int k, int E, int topk,
                                                           int32_t* __restrict__ ids, float* __restrict__ g,
@@ -28,26 +45,45 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const uint16_t* __rest
   const int tok = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint16_t* xr = x + (int64_t)tok * k;
-  for (int e = warp; e < E; e += 8) {
-    const uint16_t* wr = w + (int64_t)e * k;
-    double s = 0.0;
-    for (int kk = lane * 8; kk < k; kk += 256) {
-      const uint4 xv = *reinterpret_cast<const uint4*>(xr + kk);
-      const uint4 wv = *reinterpret_cast<const uint4*>(wr + kk);
-      const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w}, ws[4] = {wv.x, wv.y, wv.z, wv.w};
+  for (int e0 = warp; e0 < E; e0 += 8 * kRouterEB) {
+    double s[kRouterEB];
+    const uint16_t* wr[kRouterEB];
 #pragma unroll
-      for (int i = 0; i < 4; i++) {
-        const float2 xf = f16x2_to_f32x2(xs[i]), wf = f16x2_to_f32x2(ws[i]);
-        s = fma((double)xf.x, (double)wf.x, s);
-        s = fma((double)xf.y, (double)wf.y, s);
+    for (int j = 0; j < kRouterEB; j++) {
+      s[j] = 0.0;
+      const int e = e0 + 8 * j;
+      wr[j] = w + (int64_t)(e < E ? e : e0) * k;
+    }
+    int kk = lane * 8;
+    for (; kk + 3 * 256 < k; kk += 4 * 256) {
+      uint4 xv[4], wv[4][kRouterEB];
+#pragma unroll
+      for (int u = 0; u < 4; u++) {
+        xv[u] = *reinterpret_cast<const uint4*>(xr + kk + u * 256);
+#pragma unroll
+        for (int j = 0; j < kRouterEB; j++) wv[u][j] = *reinterpret_cast<const uint4*>(wr[j] + kk + u * 256);
       }
+#pragma unroll
+      for (int u = 0; u < 4; u++)
+#pragma unroll
+        for (int j = 0; j < kRouterEB; j++) router_acc8(s[j], xv[u], wv[u][j]);
+    }
+    for (; kk < k; kk += 256) {
+      const uint4 xv = *reinterpret_cast<const uint4*>(xr + kk);
+#pragma unroll
+      for (int j = 0; j < kRouterEB; j++) router_acc8(s[j], xv, *reinterpret_cast<const uint4*>(wr[j] + kk));
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, off);
-    if (lane == 0) {
-      const float zz = __double2float_rn(s + (double)b[e]);
-      z[e] = zz;
-      if (logits_out) logits_out[(int64_t)tok * E + e] = zz;
+    for (int j = 0; j < kRouterEB; j++) {
+      double v = s[j];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
+      const int e = e0 + 8 * j;
+      if (lane == 0 && e < E) {
+        const float zz = __double2float_rn(v + (double)b[e]);
+        z[e] = zz;
+        if (logits_out) logits_out[(int64_t)tok * E + e] = zz;
+      }
     }
   }
   __syncthreads();

@@ -18,6 +18,7 @@
 #include "k_gemv.cuh"
 #include "k_gemm.cuh"
 #include "k_grouped.cuh"
+#include "k_iq4p.cuh"
 #include "k_moe.cuh"
 
 namespace qmm {
@@ -277,8 +278,16 @@ static int gemv_variant_env() {
   if (!strcmp(v, "generic")) return 3;
   if (!strcmp(v, "cpa")) return 4;
   if (!strcmp(v, "iq4")) return 5;
+  if (!strcmp(v, "iq4p")) return 6;
   return 0;
 }
+
+// Persistent IQ4_NL kernel (k_iq4p.cuh).  Returns QMM_ERR_UNSUPPORTED_SHAPE,
+// having launched nothing, when the shape is outside what it takes.
+template <int MODE>
+static qmm_status launch_iq4_persist(const qmm_weights* w0, const qmm_weights* w1, const uint16_t* x, int x_per_pair,
+                                     int64_t topk, const int32_t* ids, int64_t P, int m_plain, void* y,
+                                     const float* gw, cudaStream_t st, const DevInfo* di);
 
 static qmm_status launch_iq4_stream(const qmm_weights* w, const uint16_t* x, int x_per_pair, int64_t topk,
                                    const int32_t* offsets, const int32_t* perm, int m_plain, uint16_t* y,
@@ -361,6 +370,10 @@ static qmm_status gemv_fmt(const qmm_weights* w, const uint16_t* x, int m, uint1
   if (tma_ok && (pick == 0 || pick == 1)) {
     if (m <= 8) return launch_gemv_tma<FMT, 1, 1>(w, x, m, y, st, di);
     return launch_gemv_tma<FMT, 1, 2>(w, x, m, y, st, di);
+  }
+  if (FMT == 1 && pick == 6) {  // persistent kernel: measured slower than the streaming one, kept selectable
+    const qmm_status s = launch_iq4_persist<IQ_OUT_F16>(w, nullptr, x, 0, 1, nullptr, 0, m, y, nullptr, st, di);
+    if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
   }
   if (FMT == 1 && k % 128 == 0 && (pick == 0 || pick == 5)) {
     const qmm_status s = launch_iq4_stream(w, x, 0, 1, nullptr, nullptr, m, y, st, di);
@@ -469,6 +482,67 @@ static qmm_status launch_iq4_mode(const qmm_weights* w, const qmm_weights* w2, c
       static_cast<const uint8_t*>(w->data), w->expert_data_stride,
       w2 ? static_cast<const uint8_t*>(w2->data) : nullptr, w2 ? w2->expert_data_stride : 0, x, x_per_pair,
       (int)topk, offsets, perm, m_plain, y, gw, (int)w->n, (int)w->k, (int)w->num_experts);
+  return launch_status();
+}
+
+template <int MODE>
+static qmm_status launch_iq4_persist(const qmm_weights* w0, const qmm_weights* w1, const uint16_t* x, int x_per_pair,
+                                     int64_t topk, const int32_t* ids, int64_t P, int m_plain, void* y,
+                                     const float* gw, cudaStream_t st, const DevInfo* di) {
+  const int64_t n = w0->n, k = w0->k;
+  const int E = ids ? (int)w0->num_experts : 1;
+  const int H = (MODE == IQ_SWIGLU) ? 2 : 1;
+  if (w0->fmt != QMM_FMT_IQ4_NL || (w1 && w1->fmt != QMM_FMT_IQ4_NL)) return QMM_ERR_UNSUPPORTED_SHAPE;
+  if (k % 128 || n % 16 || k > (1 << 20) || n > INT32_MAX / 2) return QMM_ERR_UNSUPPORTED_SHAPE;
+  if (ids && (P > kPxMaxPairs || E > kRouteMaxExperts)) return QMM_ERR_UNSUPPORTED_SHAPE;
+  if (!ids && m_plain > 16) return QMM_ERR_UNSUPPORTED_SHAPE;
+  const int steps = (int)(k / 128);
+  int W = (steps + 1) / 2;  // about two 128-wide super-steps per consumer warp per tile
+  if (W > kPxMaxWarps) W = kPxMaxWarps;
+  if (W < 1) W = 1;
+  const uint32_t limit = 232448u - 256u;  // opt-in shared memory per block, less the static part
+  int S = 0, XB = 0;
+  for (int xb = kPxMaxXBuf; xb >= 1 && !S; xb--)
+    for (int s = kPxMaxStages; s >= 2; s--)
+      if (px_layout((int)k, E, (int)P, W, s, xb, H).total <= limit) {
+        S = s;
+        XB = xb;
+        break;
+      }
+  if (!S) return QMM_ERR_UNSUPPORTED_SHAPE;
+  const PxLayout L = px_layout((int)k, E, (int)P, W, S, XB, H);
+  if (cudaFuncSetAttribute(iq4_persist_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total) !=
+      cudaSuccess)
+    return QMM_ERR_CUDA;
+  PxArgs a;
+  a.data0 = static_cast<const uint8_t*>(w0->data);
+  a.data1 = w1 ? static_cast<const uint8_t*>(w1->data) : nullptr;
+  a.dstride0 = w0->expert_data_stride;
+  a.dstride1 = w1 ? w1->expert_data_stride : 0;
+  a.x = x;
+  a.x_per_pair = x_per_pair;
+  a.topk = (int)topk;
+  a.ids = ids;
+  a.P = (int)P;
+  a.m_plain = m_plain;
+  a.y = y;
+  a.gw = gw;
+  a.n = (int)n;
+  a.k = (int)k;
+  a.E = E;
+  a.W = W;
+  a.S = S;
+  a.XB = XB;
+  // items exist only for routed experts, known on the device: one CTA per SM
+  // (plain product: no more CTAs than items)
+  int64_t grid = di->sms;
+  if (!ids) {
+    const int64_t items = (n / 16) * ((m_plain + 15) / 16);
+    if (items < grid) grid = items;
+  }
+  if (grid < 1) grid = 1;
+  iq4_persist_kernel<MODE><<<(unsigned)grid, 32 * (W + 1), L.total, st>>>(a);
+  set_variant("iq4_persist<mode=%d,W=%d,S=%d,XB=%d,grid=%d>", MODE, W, S, XB, (int)grid);
   return launch_status();
 }
 
@@ -701,6 +775,13 @@ qmm_status qmm_grouped_gemv(const qmm_weights* experts, const uint16_t* x, int32
   if (!ws || ws_bytes < need) return QMM_ERR_WORKSPACE;
   if (!aligned16(ws)) return QMM_ERR_MISALIGNED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int pick = gemv_variant_env();
+  if (experts->fmt == QMM_FMT_IQ4_NL && experts->k > 0 && pick == 6) {
+    // persistent kernel (buckets the ids itself, no routing pass); measured
+    // slower than route + streaming kernel on the routed-expert shapes
+    s = launch_iq4_persist<IQ_OUT_F16>(experts, nullptr, x, x_per_pair, topk, topk_ids, P, 0, y, nullptr, st, di);
+    if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
+  }
   int32_t* offsets = static_cast<int32_t*>(ws);
   int32_t* perm = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + align256(4 * (size_t)(experts->num_experts + 1)));
   route_kernel<<<1, kRouteThreads, 0, st>>>(topk_ids, (int)P, (int)experts->num_experts, offsets, perm);
@@ -711,7 +792,7 @@ qmm_status qmm_grouped_gemv(const qmm_weights* experts, const uint16_t* x, int32
     set_variant("route+zero_fill");
     return launch_status();
   }
-  if (experts->fmt == QMM_FMT_IQ4_NL && experts->k % 128 == 0 && getenv("QMM_GEMV_VARIANT") == nullptr) {
+  if (experts->fmt == QMM_FMT_IQ4_NL && experts->k % 128 == 0 && (pick == 0 || pick == 5)) {
     s = launch_iq4_stream(experts, x, x_per_pair, topk, offsets, perm, 0, y, st, di);
     set_variant("route+grouped_iq4_stream");
     return s;
@@ -825,6 +906,20 @@ qmm_status qmm_moe_routed(const qmm_weights* gate, const qmm_weights* up, const 
   uint16_t* h = reinterpret_cast<uint16_t*>(p);
   p += align256(2 * (size_t)P * (size_t)f);
   float* yg = reinterpret_cast<float*>(p);
+  if (f > 0 && gemv_variant_env() == 6) {
+    // persistent kernels (each buckets the ids itself): gate/up + SiLU, then
+    // the g-scaled down product, then the slot sum
+    s = launch_iq4_persist<IQ_SWIGLU>(gate, up, x, 0, topk, topk_ids, P, 0, h, nullptr, st, di);
+    if (s == QMM_OK)
+      s = launch_iq4_persist<IQ_SCALED_F32>(down, nullptr, h, 1, topk, topk_ids, P, 0, yg, topk_weights, st, di);
+    if (s == QMM_OK) {
+      combine_kernel<<<grid_for(t * (d / 8), 256, di->sms), 256, 0, st>>>(yg, topk_ids, (int)E, (int)t, (int)topk,
+                                                                           (int)d, out);
+      set_variant("moe:gate_up_swiglu_iq4_persist+down_scaled_iq4_persist+combine");
+      return launch_status();
+    }
+    if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
+  }
   route_kernel<<<1, kRouteThreads, 0, st>>>(topk_ids, (int)P, (int)E, offsets, perm);
   if (cudaGetLastError() != cudaSuccess) return QMM_ERR_CUDA;
   if (f == 0) {

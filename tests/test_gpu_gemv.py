@@ -121,3 +121,23 @@ def test_gemv_edge_cases():
     with pytest.raises(qmm.QmmError) as e:
         qmm.qmm_gemv(w, xd, yb[1:129].view(2, 64))                      # misaligned y
     assert e.value.status == 3
+
+
+@pytest.mark.parametrize("variant", [None, "iq4p", "generic"])
+@pytest.mark.parametrize("n,k,m", [(256, 512, 1), (2000, 4096, 5), (48, 2560, 16), (4096, 8192, 2)])
+def test_iq4nl_kernels_vs_oracle(variant, n, k, m, monkeypatch):
+    """Each IQ4_NL GEMV kernel: the streaming kernel (default for k % 128 ==
+    0), the persistent kernel (k % 128 == 0 and n % 16 == 0 while 16
+    activation rows and two weight tiles fit in shared memory, k <= 2560 or
+    so; a shape it does not take goes to the generic kernel) and the generic
+    one."""
+    if variant:
+        monkeypatch.setenv("QMM_GEMV_VARIANT", variant)
+    p, x = _case(synth.FMT_IQ4_NL, n, k, m, 3000 + n + k + m)
+    y = run_gemv(dev(p), x)
+    v = qmm.qmm_last_variant()
+    want = {None: ("gemv_iq4_stream",), "iq4p": ("iq4_persist",) if k <= 2560 else ("gemv_generic",),
+            "generic": ("gemv_generic",)}[variant]
+    assert v.startswith(want), v
+    yref, absy = oracle.matmul(synth.FMT_IQ4_NL, n, k, p.data, None, 1.0, x)
+    check_tol(y, yref, absy, v)

@@ -106,3 +106,39 @@ def test_grouped_rejects_small_workspace():
     with pytest.raises(qmm.QmmError) as e:
         qmm.qmm_grouped_gemv(w, x, ids, y, ws=torch.empty((16,), dtype=torch.uint8, device="cuda"))
     assert e.value.status == 8
+
+
+@pytest.mark.parametrize("variant", [None, "iq4p"])
+@pytest.mark.parametrize("E,n,k,t,topk,per_pair", [(3, 64, 256, 50, 2, False), (5, 48, 384, 200, 3, True),
+                                                    (2, 16, 128, 2100, 2, False), (32, 32, 128, 1, 4, True)])
+def test_grouped_iq4_many_pairs_per_expert(variant, E, n, k, t, topk, per_pair, monkeypatch):
+    """IQ4_NL experts with more than 16 pairs each (several token groups per
+    expert, whose row tiles land on different CTAs), with the routed streaming
+    kernel (default) and the persistent kernel; t * topk = 4200 is past the
+    persistent kernel's pair limit (a forced variant that does not take a
+    shape leaves it to the generic kernel)."""
+    if variant:
+        monkeypatch.setenv("QMM_GEMV_VARIANT", variant)
+    rng = np.random.default_rng(E * 1000 + n + k + t)
+    p = synth.gen_weights(rng, synth.FMT_IQ4_NL, n, k, experts=E)
+    x = synth.gen_x(rng, t, topk, k) if per_pair else synth.gen_x(rng, t, k)
+    ids = synth.gen_topk(rng, t, topk, E)
+    y, st = _grouped(dev(p), x, ids, per_pair)
+    v = qmm.qmm_last_variant()
+    assert st == 0, v
+    if variant == "iq4p":
+        assert v.startswith("iq4_persist" if t * topk <= 4096 else "route+grouped_gemv_generic"), v
+    else:
+        assert "iq4_stream" in v, v
+    if per_pair:
+        xs = x.reshape(t * topk, k)
+        yref = np.empty((t * topk, n)); absy = np.empty((t * topk, n))
+        for e in range(E):
+            sel = np.flatnonzero(ids.reshape(-1) == e)
+            if len(sel):
+                de = p.data[e * p.data_stride:(e + 1) * p.data_stride]
+                yref[sel], absy[sel] = oracle.matmul(synth.FMT_IQ4_NL, n, k, de, None, 1.0, xs[sel])
+        yref, absy = yref.reshape(t, topk, n), absy.reshape(t, topk, n)
+    else:
+        yref, absy = oracle.grouped_gemv(synth.FMT_IQ4_NL, n, k, p.data, p.data_stride, None, 0, 1.0, E, x, ids)
+    check_tol(y, yref, absy, "grouped iq4 %s" % v)

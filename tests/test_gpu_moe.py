@@ -141,17 +141,24 @@ def _moe_reference_stages(wgu, wdn, x, ids, g, f, h_gpu):
     return h_ref, h_bound, out_ref, out_abs
 
 
+@pytest.mark.parametrize("variant", [None, "iq4p"])
 @pytest.mark.parametrize("E,f,d,t,topk", [(6, 128, 256, 9, 2), (4, 256, 128, 40, 4), (2, 128, 384, 5, 2),
                                           (32, 896, 2560, 64, 4), (32, 896, 2560, 1, 4)])
-def test_moe_routed_vs_oracle(E, f, d, t, topk):
+def test_moe_routed_vs_oracle(E, f, d, t, topk, variant, monkeypatch):
+    """Default: route + streaming kernels; iq4p: the persistent kernels (each
+    buckets the ids itself)."""
+    if variant:
+        monkeypatch.setenv("QMM_GEMV_VARIANT", variant)
     rng = np.random.default_rng(E * 31 + f + d + t)
     wgu = synth.gen_iq4nl(rng, 2 * f, d, E)
     wdn = synth.gen_iq4nl(rng, d, f, E)
     x = synth.gen_x(rng, t, d)
     wr, br = synth.gen_router(rng, E, d)
     ids, g = _check_router(x, wr, br, topk)
-    out, h, st, variant = _moe_gpu(wgu, wdn, x, ids, g, f)
-    assert st == 0, variant
+    out, h, st, used = _moe_gpu(wgu, wdn, x, ids, g, f)
+    assert st == 0, used
+    assert ("iq4_persist" in used) == (variant == "iq4p"), used
+    variant = used
     h_ref, h_bound, out_ref, out_abs = _moe_reference_stages(wgu, wdn, x, ids, g, f, h)
     err = np.abs(f16(h) - h_ref)
     assert np.all(err <= h_bound), ("h", float((err / h_bound).max()), variant)
