@@ -121,6 +121,11 @@ qmm_status qmm_dequant(const qmm_weights* w, uint16_t* out, void* stream);
  * rounding of the sum to fp16.  For FP4G16_E4M3 the global scale g is applied
  * to the fp32 sum instead of to each weight (the difference from the
  * per-weight definition is one fp16 rounding of each weight).
+ * The FP4 kernels are launched with programmatic dependent launch: they start
+ * reading W while the kernel before them on the stream is still running (x
+ * and y wait for it).  So W must not be written by the kernel that
+ * immediately precedes this call on the stream; any other operation in
+ * between (a copy, an event, another library call) restores full ordering.
  *   x       device, [m][k] fp16
  *   m       1..16
  *   y       device, [m][n] fp16

@@ -97,17 +97,6 @@ __host__ __device__ inline PxLayout px_layout(int k, int E, int P, int W, int S,
   return L;
 }
 
-// bar.sync on a named barrier that also returns the OR of every thread's flag.
-__device__ __forceinline__ bool named_bar_or(int id, int threads, bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}"
-      : "=r"(r)
-      : "r"((uint32_t)v), "r"(id), "r"(threads)
-      : "memory");
-  return r != 0;
-}
-
 // Decode and multiply the super-steps [s_lo, s_hi) of one 16-row tile held in
 // shared memory at `tile` against up to 8*NT token rows at xrow0 (slot grp)
 // and xrow1 (slot grp+8).  Two super-steps are loaded before either is used.
@@ -368,7 +357,7 @@ __global__ void __launch_bounds__(kPxMaxThreads, 1) iq4_persist_kernel(const PxA
     if (e != ce || g != cg) {
       if (xf > 0 && lane == 0) mbar_arrive(xempty + 8u * ((xf - 1u) % (uint32_t)XB));
       const uint32_t xb = xf % (uint32_t)XB;
-      if (!mbar_wait(xfull + 8u * xb, (xf / XB) & 1u)) fail = true;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(xfull + 8u * xb, (xf / XB) & 1u))) fail = true;
       xbase = sb + L.xbuf + xb * 16u * xs;
       xf++;
       ce = e;
@@ -385,7 +374,7 @@ __global__ void __launch_bounds__(kPxMaxThreads, 1) iq4_persist_kernel(const PxA
 #pragma unroll
     for (int h = 0; h < H; h++) {
       const uint32_t slot = st % (uint32_t)S;
-      if (!fail && !s_abort && mbar_wait(full + 8u * slot, (st / S) & 1u)) {
+      if (__all_sync(0xFFFFFFFFu, !fail && !s_abort && mbar_wait(full + 8u * slot, (st / S) & 1u))) {
         const uint32_t t0 = sb + L.ring + slot * tb;
         if (ng <= 8) px_range<1>(acc[h], t0, rowb, grp, tig, s_lo, s_hi, xrow0, xrow1, lut_lane);
         else px_range<2>(acc[h], t0, rowb, grp, tig, s_lo, s_hi, xrow0, xrow1, lut_lane);

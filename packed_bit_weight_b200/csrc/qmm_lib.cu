@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -18,6 +19,7 @@
 #include "k_gemv.cuh"
 #include "k_gemm.cuh"
 #include "k_grouped.cuh"
+#include "k_gemv_ring.cuh"
 #include "k_iq4p.cuh"
 #include "k_moe.cuh"
 
@@ -192,6 +194,48 @@ static qmm_status launch_gemv_ldg(const qmm_weights* w, const uint16_t* x, int m
   return launch_status();
 }
 
+// Persistent ring GEMV (k_gemv_ring.cuh): one CTA per SM, whole 16-row tiles
+// in a ring of 2..4 stages (at most 96 KB, so the next launch's CTA fits
+// beside it), programmatic dependent launch.  Needs k % 256 == 0 and a tile of
+// at most 48 KB (k <= 4096 with fp16 scales).  Measurement knobs:
+// QMM_RING_STAGES=<2..4>, QMM_GEMV_NOPDL=1.
+template <int FMT, int NT, int CW, int SPW, bool XSM>
+static qmm_status launch_gemv_ring(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st,
+                                   const DevInfo* di) {
+  const int64_t n = w->n, k = w->k;
+  if (k % 256 || k < 256 || k > 128 * CW * SPW || n < 1 || n > INT32_MAX - 16) return QMM_ERR_UNSUPPORTED_SHAPE;
+  const uint32_t stage = ring_stage_bytes(FMT, (int)k);
+  int stages = (int)std::min<uint32_t>(kRingMaxStages, kRingStageBudget / stage);
+  if (const char* e = getenv("QMM_RING_STAGES")) stages = atoi(e);
+  if (stages < 2 || stages > kRingMaxStages) return QMM_ERR_UNSUPPORTED_SHAPE;
+  const uint32_t xs_bytes = XSM ? 2u * (uint32_t)m * (uint32_t)k : 0u;
+  if (xs_bytes > kRingXsMax) return QMM_ERR_UNSUPPORTED_SHAPE;
+  const uint32_t smem = ring_smem_bytes<CW, NT>(FMT, (int)k, stages, xs_bytes);
+  if (smem > di->smem_optin) return QMM_ERR_UNSUPPORTED_SHAPE;
+  auto kern = gemv_fp4_ring_kernel<FMT, NT, CW, SPW, XSM>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return QMM_ERR_CUDA;
+  const int64_t tiles = (n + 15) / 16;
+  const int64_t grid = std::min<int64_t>(tiles, (int64_t)di->sms);
+  const char* nopdl = getenv("QMM_GEMV_NOPDL");
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(32 * (CW + 1));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = (nopdl && nopdl[0] == '1') ? 0 : 1;
+  if (cudaLaunchKernelEx(&cfg, kern, static_cast<const uint8_t*>(w->data), static_cast<const uint8_t*>(w->scales), x,
+                         y, (int)n, (int)k, m, w->global_scale, stages) != cudaSuccess)
+    return QMM_ERR_CUDA;
+  set_variant("gemv_fp4_ring<fmt=%d,nt=%d,cw=%d,xsm=%d,stages=%d,grid=%d,smem=%u>", FMT, NT, CW, (int)XSM, stages,
+              (int)grid, smem);
+  return launch_status();
+}
+
 // Pick the warps per tile (WPC) and segments per warp (SPW, <= 8 at m <= 8,
 // <= 4 at m <= 16) for k = 128 * WPC * SPW; fewer, fuller warps keep more
 // bytes in flight per register.  Returns UNSUPPORTED_SHAPE for other k.
@@ -279,6 +323,7 @@ static int gemv_variant_env() {
   if (!strcmp(v, "cpa")) return 4;
   if (!strcmp(v, "iq4")) return 5;
   if (!strcmp(v, "iq4p")) return 6;
+  if (!strcmp(v, "ring")) return 7;
   return 0;
 }
 
@@ -356,6 +401,17 @@ static qmm_status gemv_fmt(const qmm_weights* w, const uint16_t* x, int m, uint1
     if (gemv_cfg_env<FMT>(w, x, m, y, st, di, &cs)) return cs;
   }
   const int pick = gemv_variant_env();
+  if constexpr (FMT != 1) {
+    if (pick == 7) {
+      const bool xsm = 2 * m * k <= (int64_t)kRingXsMax;
+      const char* cwe = getenv("QMM_RING_CW");  // measurement knob: 16 consumer warps at m <= 8
+      const qmm_status s = (m > 8) ? launch_gemv_ring<FMT, 2, 8, 4, false>(w, x, m, y, st, di)
+                           : (cwe && atoi(cwe) == 16) ? launch_gemv_ring<FMT, 1, 16, 2, false>(w, x, m, y, st, di)
+                           : xsm ? launch_gemv_ring<FMT, 1, 8, 4, true>(w, x, m, y, st, di)
+                                 : launch_gemv_ring<FMT, 1, 8, 4, false>(w, x, m, y, st, di);
+      if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
+    }
+  }
   const bool tma_ok = FMT != 1 && k % kChunkK == 0 && k >= 8 * kChunkK && n >= 16;
   if (FMT != 1 && (pick == 0 || pick == 2)) {
     const qmm_status s = (m <= 8) ? gemv_ldg_auto<FMT, 1>(w, x, m, y, st) : gemv_ldg_auto<FMT, 2>(w, x, m, y, st);

@@ -38,7 +38,7 @@ def test_fast_path_is_used_for_streaming_shapes():
     assert qmm.qmm_last_variant().startswith(("gemv_fp4_cpa", "gemv_fp4_ldg", "gemv_fp4_tma"))
 
 
-@pytest.mark.parametrize("variant", ["cpa", "tma", "ldg", "generic"])
+@pytest.mark.parametrize("variant", ["cpa", "tma", "ldg", "generic", "ring"])
 @pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3])
 @pytest.mark.parametrize("n,k,m", [(1000, 4096, 1), (333, 8192, 3), (64, 2048, 16), (517, 3072, 9)])
 def test_every_streaming_variant_vs_oracle(variant, fmt, n, k, m, monkeypatch):
@@ -46,8 +46,9 @@ def test_every_streaming_variant_vs_oracle(variant, fmt, n, k, m, monkeypatch):
     p, x = _case(fmt, n, k, m, 2000 + n + k + m + fmt)
     y = run_gemv(dev(p), x)
     v = qmm.qmm_last_variant()
-    assert v.startswith({"cpa": "gemv_fp4_cpa", "tma": "gemv_fp4_tma", "ldg": "gemv_fp4_ldg",
-                         "generic": "gemv_generic"}[variant]), v
+    want = {"cpa": "gemv_fp4_cpa", "tma": "gemv_fp4_tma", "ldg": "gemv_fp4_ldg", "generic": "gemv_generic",
+            "ring": "gemv_fp4_ring" if k <= 4096 else "gemv_generic"}[variant]  # ring: tiles of <= 48 KB
+    assert v.startswith(want), v
     yref, absy = oracle.matmul(fmt, n, k, p.data, p.scales, p.global_scale, x)
     check_tol(y, yref, absy, v)
 
