@@ -353,45 +353,17 @@ constexpr int kLdgWarps = 8;
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-template <int FMT, int NT, int SPW, int WPC = kLdgWarps, int MINB = 2>
-__global__ void __launch_bounds__(WPC * 32, MINB)
-    gemv_fp4_ldg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
-                        const uint16_t* __restrict__ x, uint16_t* __restrict__ y, int n, int k, int m, float g) {
-  __shared__ float red[WPC][16][16];  // [warp][token][row]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int grp = lane >> 2, tig = lane & 3;
-  const int n0 = blockIdx.x * 16;
-  const int ra = n0 + grp, rb = ra + 8;
-  const bool va = ra < n, vb = rb < n;
-  const int seg0 = warp * SPW;
-  const int64_t crow = k >> 1, srow = k >> 4;
-
-  pdl_launch_dependents();
-  uint4 qa[SPW], qb[SPW];
-  uint32_t sa[SPW], sb[SPW];
-#pragma unroll
-  for (int i = 0; i < SPW; i++) {
-    const int seg = seg0 + i;
-    const int64_t cb = (int64_t)seg * 64 + tig * 16;
-    const int64_t gi = (int64_t)seg * 8 + tig * 2;  // first of the two group scales
-    qa[i] = va ? ldg_stream128(codes + ra * crow + cb) : make_uint4(0, 0, 0, 0);
-    qb[i] = vb ? ldg_stream128(codes + rb * crow + cb) : make_uint4(0, 0, 0, 0);
-    if (FMT == 2) {
-      sa[i] = va ? ldg_stream32(scales + (ra * srow + gi) * 2) : 0u;
-      sb[i] = vb ? ldg_stream32(scales + (rb * srow + gi) * 2) : 0u;
-    } else {
-      sa[i] = va ? e4m3x2_to_f16x2(ldg_stream16(scales + ra * srow + gi)) : 0u;
-      sb[i] = vb ? e4m3x2_to_f16x2(ldg_stream16(scales + rb * srow + gi)) : 0u;
-    }
-  }
-  pdl_wait();  // x may be the previous kernel's output; y may still be read by it
-
-  float acc[NT][4];
-#pragma unroll
-  for (int j = 0; j < NT; j++)
-#pragma unroll
-    for (int c = 0; c < 4; c++) acc[j][c] = 0.f;
-
+// Decode and multiply a warp's SPW segments of one 16-row tile, held in
+// registers (code bytes qa/qb of rows grp and grp+8, group-scale pairs sa/sb
+// as f16x2), against tokens grp and grp+8 (when < m) read from global memory.
+// Measured alternatives, both slower on the in_proj shape: loading a clamped
+// token row in every lane instead of zero-filling the columns past m (27 %:
+// 8x the L1 traffic), and zero-filling once before the segment loop (18 %:
+// the compiler then keeps fewer of the tile's loads in flight).
+template <int FMT, int NT, int SPW>
+__device__ __forceinline__ void ldg_tile_mma(float (&acc)[NT][4], const uint4 (&qa)[SPW], const uint4 (&qb)[SPW],
+                                             const uint32_t (&sa)[SPW], const uint32_t (&sb)[SPW], int seg0, int grp,
+                                             int tig, const uint16_t* __restrict__ x, int k, int m) {
 #pragma unroll
   for (int i = 0; i < SPW; i++) {
     const int kseg = (seg0 + i) * 128 + tig * 32;
@@ -431,7 +403,15 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
       for (int j = 0; j < NT; j++) mma_16816(acc[j], a0, a1, a2, a3, xb[j][2 * st], xb[j][2 * st + 1]);
     }
   }
+}
 
+// The WPC warps' partial sums of one tile meet in shared memory and are added
+// in warp order (deterministic); rows n0.. of y are stored.  Ends with every
+// thread past a __syncthreads, so `red` may be reused afterwards only after
+// another one.
+template <int FMT, int NT, int WPC>
+__device__ __forceinline__ void ldg_tile_store(float (&red)[WPC][16][16], const float (&acc)[NT][4], int warp, int grp,
+                                               int tig, int n0, int n, int m, float g, uint16_t* __restrict__ y) {
 #pragma unroll
   for (int j = 0; j < NT; j++) {
     const int t0 = 8 * j + 2 * tig;
@@ -449,6 +429,151 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
     for (int w = 0; w < WPC; w++) v += red[w][tok][row];
     if (n0 + row < n) y[(int64_t)tok * n + n0 + row] = f32_to_f16_bits(v * gs);
   }
+}
+
+template <int FMT, int NT, int SPW, int WPC = kLdgWarps, int MINB = 2>
+__global__ void __launch_bounds__(WPC * 32, MINB)
+    gemv_fp4_ldg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                        const uint16_t* __restrict__ x, uint16_t* __restrict__ y, int n, int k, int m, float g) {
+  __shared__ float red[WPC][16][16];  // [warp][token][row]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int grp = lane >> 2, tig = lane & 3;
+  const int n0 = blockIdx.x * 16;
+  const int ra = n0 + grp, rb = ra + 8;
+  const bool va = ra < n, vb = rb < n;
+  const int seg0 = warp * SPW;
+  const int64_t crow = k >> 1, srow = k >> 4;
+
+  pdl_launch_dependents();
+  uint4 qa[SPW], qb[SPW];
+  uint32_t sa[SPW], sb[SPW];
+#pragma unroll
+  for (int i = 0; i < SPW; i++) {
+    const int seg = seg0 + i;
+    const int64_t cb = (int64_t)seg * 64 + tig * 16;
+    const int64_t gi = (int64_t)seg * 8 + tig * 2;  // first of the two group scales
+    qa[i] = va ? ldg_stream128(codes + ra * crow + cb) : make_uint4(0, 0, 0, 0);
+    qb[i] = vb ? ldg_stream128(codes + rb * crow + cb) : make_uint4(0, 0, 0, 0);
+    if (FMT == 2) {
+      sa[i] = va ? ldg_stream32(scales + (ra * srow + gi) * 2) : 0u;
+      sb[i] = vb ? ldg_stream32(scales + (rb * srow + gi) * 2) : 0u;
+    } else {
+      sa[i] = va ? e4m3x2_to_f16x2(ldg_stream16(scales + ra * srow + gi)) : 0u;
+      sb[i] = vb ? e4m3x2_to_f16x2(ldg_stream16(scales + rb * srow + gi)) : 0u;
+    }
+  }
+  pdl_wait();  // x may be the previous kernel's output; y may still be read by it
+
+  float acc[NT][4];
+#pragma unroll
+  for (int j = 0; j < NT; j++)
+#pragma unroll
+    for (int c = 0; c < 4; c++) acc[j][c] = 0.f;
+  ldg_tile_mma<FMT, NT, SPW>(acc, qa, qb, sa, sb, seg0, grp, tig, x, k, m);
+  ldg_tile_store<FMT, NT, WPC>(red, acc, warp, grp, tig, n0, n, m, g, y);
+}
+
+// ---------------------------------------------------------------------------
+// Two tiles per CTA, all bytes in flight at once.  The CTA of block b loads
+// tile 2b into registers exactly as gemv_fp4_ldg does, and thread 0 copies
+// tile 2b+1 (its 16 code rows and 16 scale rows are two contiguous ranges)
+// into shared memory with two bulk copies.  With half as many CTAs the whole
+// matrix fits in one wave of resident CTAs (registers plus shared memory hold
+// a tile each), so no second wave waits for the first wave's arithmetic.
+// Tile 2b+1 is then read from shared memory in the same lane layout.
+// ---------------------------------------------------------------------------
+template <int FMT>
+__host__ __device__ inline uint32_t dual_smem_bytes(int k) {
+  return 16u * ((uint32_t)k / 2u + ((FMT == 2) ? (uint32_t)k / 8u : (uint32_t)k / 16u)) + 16u;
+}
+
+template <int FMT, int NT, int SPW, int WPC, int MINB>
+__global__ void __launch_bounds__(WPC * 32, MINB)
+    gemv_fp4_dual_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                         const uint16_t* __restrict__ x, uint16_t* __restrict__ y, int n, int k, int m, float g) {
+  extern __shared__ __align__(128) uint8_t smem_dual[];
+  __shared__ float red[WPC][16][16];  // [warp][token][row]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int grp = lane >> 2, tig = lane & 3;
+  const int seg0 = warp * SPW;
+  const int64_t crow = k >> 1, srow = k >> 4;
+  const uint32_t sbytes = (FMT == 2) ? (uint32_t)k / 8u : (uint32_t)k / 16u;  // scale bytes per row
+  const int n0 = blockIdx.x * 32, n1 = n0 + 16;
+  const uint32_t sbase = smem_addr(smem_dual);
+  const uint32_t bar = sbase + 16u * ((uint32_t)crow + sbytes);
+
+  pdl_launch_dependents();
+  uint4 qa[SPW], qb[SPW];
+  uint32_t sa[SPW], sb[SPW];
+  {
+    const int ra = n0 + grp, rb = ra + 8;
+    const bool va = ra < n, vb = rb < n;
+#pragma unroll
+    for (int i = 0; i < SPW; i++) {
+      const int seg = seg0 + i;
+      const int64_t cb = (int64_t)seg * 64 + tig * 16;
+      const int64_t gi = (int64_t)seg * 8 + tig * 2;
+      qa[i] = va ? ldg_stream128(codes + ra * crow + cb) : make_uint4(0, 0, 0, 0);
+      qb[i] = vb ? ldg_stream128(codes + rb * crow + cb) : make_uint4(0, 0, 0, 0);
+      if (FMT == 2) {
+        sa[i] = va ? ldg_stream32(scales + (ra * srow + gi) * 2) : 0u;
+        sb[i] = vb ? ldg_stream32(scales + (rb * srow + gi) * 2) : 0u;
+      } else {
+        sa[i] = va ? e4m3x2_to_f16x2(ldg_stream16(scales + ra * srow + gi)) : 0u;
+        sb[i] = vb ? e4m3x2_to_f16x2(ldg_stream16(scales + rb * srow + gi)) : 0u;
+      }
+    }
+  }
+  const int rows1 = min(16, n - n1);  // rows of the second tile (<= 0: none)
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+    if (rows1 > 0) {
+      mbar_arrive_expect_tx(bar, (uint32_t)rows1 * ((uint32_t)crow + sbytes));
+      bulk_load(sbase, codes + (int64_t)n1 * crow, (uint32_t)rows1 * (uint32_t)crow, bar);
+      bulk_load(sbase + 16u * (uint32_t)crow, scales + (int64_t)n1 * sbytes, (uint32_t)rows1 * sbytes, bar);
+    }
+  }
+  __syncthreads();  // the barrier is initialised before anyone waits on it
+  pdl_wait();       // x may be the previous kernel's output; y may still be read by it
+
+  float acc[NT][4];
+#pragma unroll
+  for (int j = 0; j < NT; j++)
+#pragma unroll
+    for (int c = 0; c < 4; c++) acc[j][c] = 0.f;
+  ldg_tile_mma<FMT, NT, SPW>(acc, qa, qb, sa, sb, seg0, grp, tig, x, k, m);
+  ldg_tile_store<FMT, NT, WPC>(red, acc, warp, grp, tig, n0, n, m, g, y);
+  if (rows1 <= 0) return;
+
+  // second tile: every lane waits for the copies (bounded); the verdict is
+  // made warp-uniform so the MMAs never run in a diverged warp
+  const bool ready = __all_sync(0xFFFFFFFFu, mbar_wait(bar, 0));
+  if (ready) {
+    const uint8_t* cs = smem_dual + grp * crow + tig * 16;
+    const uint8_t* ss = smem_dual + 16 * crow + grp * sbytes;
+#pragma unroll
+    for (int i = 0; i < SPW; i++) {
+      const int seg = seg0 + i;
+      qa[i] = *reinterpret_cast<const uint4*>(cs + seg * 64);
+      qb[i] = *reinterpret_cast<const uint4*>(cs + 8 * crow + seg * 64);
+      if (FMT == 2) {
+        sa[i] = *reinterpret_cast<const uint32_t*>(ss + seg * 16 + tig * 4);
+        sb[i] = *reinterpret_cast<const uint32_t*>(ss + 8u * sbytes + seg * 16 + tig * 4);
+      } else {
+        sa[i] = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(ss + seg * 8 + tig * 2));
+        sb[i] = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(ss + 8u * sbytes + seg * 8 + tig * 2));
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < NT; j++)
+#pragma unroll
+      for (int c = 0; c < 4; c++) acc[j][c] = 0.f;
+    ldg_tile_mma<FMT, NT, SPW>(acc, qa, qb, sa, sb, seg0, grp, tig, x, k, m);
+  }
+  // the first tile's sums have been read from `red`; the store below holds
+  // barriers, so it runs in every thread or in none
+  if (__syncthreads_and(ready)) ldg_tile_store<FMT, NT, WPC>(red, acc, warp, grp, tig, n1, n, m, g, y);
 }
 
 // ---------------------------------------------------------------------------

@@ -236,6 +236,50 @@ static qmm_status launch_gemv_ring(const qmm_weights* w, const uint16_t* x, int 
   return launch_status();
 }
 
+// Two tiles per CTA (k_gemv.cuh, gemv_fp4_dual_kernel): one in registers, one
+// bulk-copied into shared memory, so the whole matrix is in flight in one wave.
+template <int FMT, int NT, int SPW, int WPC, int MINB>
+static qmm_status launch_gemv_dual(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st,
+                                   const DevInfo* di) {
+  const int64_t n = w->n, k = w->k;
+  if (k != 128 * WPC * SPW || n < 1 || n > INT32_MAX - 32) return QMM_ERR_UNSUPPORTED_SHAPE;
+  const uint32_t smem = dual_smem_bytes<FMT>((int)k);
+  if (smem > di->smem_optin) return QMM_ERR_UNSUPPORTED_SHAPE;
+  auto kern = gemv_fp4_dual_kernel<FMT, NT, SPW, WPC, MINB>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return QMM_ERR_CUDA;
+  const int64_t blocks = (n + 31) / 32;
+  const char* nopdl = getenv("QMM_GEMV_NOPDL");
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.blockDim = dim3(WPC * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = (nopdl && nopdl[0] == '1') ? 0 : 1;
+  if (cudaLaunchKernelEx(&cfg, kern, static_cast<const uint8_t*>(w->data), static_cast<const uint8_t*>(w->scales), x,
+                         y, (int)n, (int)k, m, w->global_scale) != cudaSuccess)
+    return QMM_ERR_CUDA;
+  set_variant("gemv_fp4_dual<fmt=%d,nt=%d,spw=%d,wpc=%d,minb=%d,blocks=%d,smem=%u>", FMT, NT, SPW, WPC, MINB,
+              (int)blocks, smem);
+  return launch_status();
+}
+
+template <int FMT>
+static qmm_status gemv_dual_auto(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st,
+                                 const DevInfo* di) {
+  if (m > 8 || w->k % 512) return QMM_ERR_UNSUPPORTED_SHAPE;
+  switch (w->k / 512) {
+    case 4: return launch_gemv_dual<FMT, 1, 4, 4, 4>(w, x, m, y, st, di);
+    case 6: return launch_gemv_dual<FMT, 1, 6, 4, 4>(w, x, m, y, st, di);
+    case 8: return launch_gemv_dual<FMT, 1, 8, 4, 4>(w, x, m, y, st, di);
+    default: return QMM_ERR_UNSUPPORTED_SHAPE;
+  }
+}
+
 // Pick the warps per tile (WPC) and segments per warp (SPW, <= 8 at m <= 8,
 // <= 4 at m <= 16) for k = 128 * WPC * SPW; fewer, fuller warps keep more
 // bytes in flight per register.  Returns UNSUPPORTED_SHAPE for other k.
@@ -324,6 +368,7 @@ static int gemv_variant_env() {
   if (!strcmp(v, "iq4")) return 5;
   if (!strcmp(v, "iq4p")) return 6;
   if (!strcmp(v, "ring")) return 7;
+  if (!strcmp(v, "dual")) return 8;
   return 0;
 }
 
@@ -402,6 +447,10 @@ static qmm_status gemv_fmt(const qmm_weights* w, const uint16_t* x, int m, uint1
   }
   const int pick = gemv_variant_env();
   if constexpr (FMT != 1) {
+    if (pick == 8) {
+      const qmm_status s = gemv_dual_auto<FMT>(w, x, m, y, st, di);
+      if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
+    }
     if (pick == 7) {
       const bool xsm = 2 * m * k <= (int64_t)kRingXsMax;
       const char* cwe = getenv("QMM_RING_CW");  // measurement knob: 16 consumer warps at m <= 8

@@ -38,7 +38,7 @@ def test_fast_path_is_used_for_streaming_shapes():
     assert qmm.qmm_last_variant().startswith(("gemv_fp4_cpa", "gemv_fp4_ldg", "gemv_fp4_tma"))
 
 
-@pytest.mark.parametrize("variant", ["cpa", "tma", "ldg", "generic", "ring"])
+@pytest.mark.parametrize("variant", ["cpa", "tma", "ldg", "generic", "ring", "dual"])
 @pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3])
 @pytest.mark.parametrize("n,k,m", [(1000, 4096, 1), (333, 8192, 3), (64, 2048, 16), (517, 3072, 9)])
 def test_every_streaming_variant_vs_oracle(variant, fmt, n, k, m, monkeypatch):
@@ -47,7 +47,8 @@ def test_every_streaming_variant_vs_oracle(variant, fmt, n, k, m, monkeypatch):
     y = run_gemv(dev(p), x)
     v = qmm.qmm_last_variant()
     want = {"cpa": "gemv_fp4_cpa", "tma": "gemv_fp4_tma", "ldg": "gemv_fp4_ldg", "generic": "gemv_generic",
-            "ring": "gemv_fp4_ring" if k <= 4096 else "gemv_generic"}[variant]  # ring: tiles of <= 48 KB
+            "ring": "gemv_fp4_ring" if k <= 4096 else "gemv_generic",  # ring: tiles of <= 48 KB
+            "dual": "gemv_fp4_dual" if m <= 8 and k in (2048, 3072, 4096) else "gemv_generic"}[variant]
     assert v.startswith(want), v
     yref, absy = oracle.matmul(fmt, n, k, p.data, p.scales, p.global_scale, x)
     check_tol(y, yref, absy, v)
@@ -141,4 +142,18 @@ def test_iq4nl_kernels_vs_oracle(variant, n, k, m, monkeypatch):
             "generic": ("gemv_generic",)}[variant]
     assert v.startswith(want), v
     yref, absy = oracle.matmul(synth.FMT_IQ4_NL, n, k, p.data, None, 1.0, x)
+    check_tol(y, yref, absy, v)
+
+
+@pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3])
+@pytest.mark.parametrize("n,k,m", [(1010, 4096, 1), (1010, 3072, 5), (31, 2048, 8), (17, 4096, 2), (16, 4096, 1)])
+def test_dual_tile_kernel_ragged(fmt, n, k, m, monkeypatch):
+    """Two tiles per CTA (registers + a bulk copy into shared memory): a last
+    CTA whose second tile is partial, absent, or the only partial one."""
+    monkeypatch.setenv("QMM_GEMV_VARIANT", "dual")
+    p, x = _case(fmt, n, k, m, 4000 + n + k + m + fmt)
+    y = run_gemv(dev(p), x)
+    v = qmm.qmm_last_variant()
+    assert v.startswith("gemv_fp4_dual"), v
+    yref, absy = oracle.matmul(fmt, n, k, p.data, p.scales, p.global_scale, x)
     check_tol(y, yref, absy, v)
