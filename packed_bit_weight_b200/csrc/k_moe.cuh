@@ -3,7 +3,8 @@
 // (MoE)": s = Softmax(x W_router + b), top-4 experts with weights g_i,
 // F(x) = (SiLU(x W_gate) * (x W_up)) W_down, routed output sum_i g_i F_i(x)).
 //
-// router_topk_kernel: one CTA per token; warps take experts, lanes split k;
+// router_topk_kernel: one CTA of 32 warps per token; warps take experts,
+//   lanes split k;
 //   every fp16 x fp16 product is exact in fp32 and the dot product is
 //   accumulated in fp64, then rounded once, with the bias, to an fp32 logit;
 //   softmax in fp32;
@@ -21,11 +22,14 @@ namespace qmm {
 constexpr int kRouterMaxExperts = 256;
 constexpr int kRouterMaxTopk = 16;
 
-// Router logits: warp w takes experts w, w+8, w+16, w+24 (then the next 32),
-// lanes take 8 consecutive k of every 256; each fp16 x fp16 product is exact
-// in fp32 and is added in fp64.  Loads of four k-chunks are issued before
-// their products so the warp keeps several memory requests in flight.
-constexpr int kRouterEB = 4;  // experts per warp per pass
+// Router logits: 32 warps per token; warp w takes experts w, w+32, ...; lanes
+// take 8 consecutive k of every 256.  Each fp16 x fp16 product is exact in
+// fp32 and is added in fp64, into two partial sums (alternate chunks: two
+// independent add chains); four chunks' loads are issued before their
+// products.  (Eight warps with four experts each measured 11 us per token:
+// the fp64 adds and conversions are long-latency and two warps per scheduler
+// did not hide them.)
+constexpr int kRouterThreads = 1024;
 
 __device__ __forceinline__ void router_acc8(double& s, const uint4& xv, const uint4& wv) {
   const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w}, ws[4] = {wv.x, wv.y, wv.z, wv.w};
@@ -37,53 +41,42 @@ __device__ __forceinline__ void router_acc8(double& s, const uint4& xv, const ui
   }
 }
 
-__global__ void __launch_bounds__(256) router_topk_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ w,
-                                                          const float* __restrict__ b, int k, int E, int topk,
-                                                          int32_t* __restrict__ ids, float* __restrict__ g,
-                                                          float* __restrict__ logits_out) {
+__global__ void __launch_bounds__(kRouterThreads) router_topk_kernel(const uint16_t* __restrict__ x,
+                                                                     const uint16_t* __restrict__ w,
+                                                                     const float* __restrict__ b, int k, int E,
+                                                                     int topk, int32_t* __restrict__ ids,
+                                                                     float* __restrict__ g,
+                                                                     float* __restrict__ logits_out) {
   __shared__ float z[kRouterMaxExperts];
   const int tok = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int kWarps = kRouterThreads / 32;
   const uint16_t* xr = x + (int64_t)tok * k;
-  for (int e0 = warp; e0 < E; e0 += 8 * kRouterEB) {
-    double s[kRouterEB];
-    const uint16_t* wr[kRouterEB];
-#pragma unroll
-    for (int j = 0; j < kRouterEB; j++) {
-      s[j] = 0.0;
-      const int e = e0 + 8 * j;
-      wr[j] = w + (int64_t)(e < E ? e : e0) * k;
-    }
+  for (int e = warp; e < E; e += kWarps) {
+    const uint16_t* wr = w + (int64_t)e * k;
+    double s0 = 0.0, s1 = 0.0;
     int kk = lane * 8;
     for (; kk + 3 * 256 < k; kk += 4 * 256) {
-      uint4 xv[4], wv[4][kRouterEB];
+      uint4 xv[4], wv[4];
 #pragma unroll
       for (int u = 0; u < 4; u++) {
         xv[u] = *reinterpret_cast<const uint4*>(xr + kk + u * 256);
-#pragma unroll
-        for (int j = 0; j < kRouterEB; j++) wv[u][j] = *reinterpret_cast<const uint4*>(wr[j] + kk + u * 256);
+        wv[u] = *reinterpret_cast<const uint4*>(wr + kk + u * 256);
       }
-#pragma unroll
-      for (int u = 0; u < 4; u++)
-#pragma unroll
-        for (int j = 0; j < kRouterEB; j++) router_acc8(s[j], xv[u], wv[u][j]);
+      router_acc8(s0, xv[0], wv[0]);
+      router_acc8(s1, xv[1], wv[1]);
+      router_acc8(s0, xv[2], wv[2]);
+      router_acc8(s1, xv[3], wv[3]);
     }
-    for (; kk < k; kk += 256) {
-      const uint4 xv = *reinterpret_cast<const uint4*>(xr + kk);
+    for (; kk < k; kk += 256)
+      router_acc8(s0, *reinterpret_cast<const uint4*>(xr + kk), *reinterpret_cast<const uint4*>(wr + kk));
+    double v = s0 + s1;
 #pragma unroll
-      for (int j = 0; j < kRouterEB; j++) router_acc8(s[j], xv, *reinterpret_cast<const uint4*>(wr[j] + kk));
-    }
-#pragma unroll
-    for (int j = 0; j < kRouterEB; j++) {
-      double v = s[j];
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
-      const int e = e0 + 8 * j;
-      if (lane == 0 && e < E) {
-        const float zz = __double2float_rn(v + (double)b[e]);
-        z[e] = zz;
-        if (logits_out) logits_out[(int64_t)tok * E + e] = zz;
-      }
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
+    if (lane == 0) {
+      const float zz = __double2float_rn(v + (double)b[e]);
+      z[e] = zz;
+      if (logits_out) logits_out[(int64_t)tok * E + e] = zz;
     }
   }
   __syncthreads();

@@ -210,6 +210,13 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
                : "memory");
 }
 
+// Bulk prefetch of a global byte range into L2 (no shared memory, no
+// completion; a hint): address 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+               : "memory");
+}
+
 // bar.sync on a named barrier that also returns the OR of every thread's flag.
 __device__ __forceinline__ bool named_bar_or(int id, int threads, bool v) {
   uint32_t r;

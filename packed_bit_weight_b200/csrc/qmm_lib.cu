@@ -583,10 +583,13 @@ static qmm_status launch_iq4_mode(const qmm_weights* w, const qmm_weights* w2, c
     return QMM_ERR_CUDA;
   const int64_t items = ((w->n + 15) / 16) * w->num_experts;
   const int64_t grid = items < (int64_t)per_sm * di->sms ? items : (int64_t)per_sm * di->sms;
+  int pf = 0;  // items of L2 prefetch ahead per CTA (measurement knob QMM_IQ4_PF)
+  if (const char* e = getenv("QMM_IQ4_PF")) pf = atoi(e);
+  if (pf < 0 || pf > 8) return QMM_ERR_INVALID_ARG;
   grouped_iq4_kernel<MODE><<<(unsigned)grid, kIqWarps * 32, smem, st>>>(
       static_cast<const uint8_t*>(w->data), w->expert_data_stride,
       w2 ? static_cast<const uint8_t*>(w2->data) : nullptr, w2 ? w2->expert_data_stride : 0, x, x_per_pair,
-      (int)topk, offsets, perm, m_plain, y, gw, (int)w->n, (int)w->k, (int)w->num_experts);
+      (int)topk, offsets, perm, m_plain, y, gw, (int)w->n, (int)w->k, (int)w->num_experts, pf);
   return launch_status();
 }
 
@@ -973,7 +976,7 @@ qmm_status qmm_router_topk(const uint16_t* x, const uint16_t* w_router, const fl
   if ((x && !aligned16(x)) || (w_router && !aligned16(w_router)) || !aligned16(bias) || !aligned16(topk_ids) ||
       !aligned16(topk_weights) || (logits && !aligned16(logits)))
     return QMM_ERR_MISALIGNED;
-  router_topk_kernel<<<(unsigned)t, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+  router_topk_kernel<<<(unsigned)t, kRouterThreads, 0, static_cast<cudaStream_t>(stream)>>>(
       x, w_router, bias, (int)k, (int)num_experts, (int)topk, topk_ids, topk_weights, logits);
   set_variant("router_topk");
   return launch_status();
