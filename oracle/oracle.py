@@ -15,6 +15,7 @@ import numpy as np
 FMT_IQ4_NL = 1
 FMT_FP4G16_F16 = 2
 FMT_FP4G16_E4M3 = 3
+FMT_MXFP4 = 4
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "qmm_oracle.c")
@@ -29,6 +30,7 @@ PINS = {
                    "(tests/test_oracle_codecs.py)",
     "e2m1_to_f64": "printed magnitude list (tests/golden/e2m1_magnitudes.txt)",
     "iq4nl_value": "printed codebook (tests/golden/iq4nl_codebook.txt)",
+    "e8m0_to_f64": "all 256 bytes vs torch float8_e8m0fnu (tests/test_oracle_codecs.py)",
     "data_bytes/scale_bytes": "byte identities from the model-card storage table "
                               "(tests/test_oracle_sizes.py)",
     "dequant": "hand-built blocks with hand-written expected values (tests/golden/*.txt), "
@@ -69,6 +71,8 @@ def lib():
         L.orc_f64_to_f16.restype = ctypes.c_uint16
         L.orc_e4m3_to_f64.argtypes = [ctypes.c_uint8]
         L.orc_e4m3_to_f64.restype = ctypes.c_double
+        L.orc_e8m0_to_f64.argtypes = [ctypes.c_uint8]
+        L.orc_e8m0_to_f64.restype = ctypes.c_double
         L.orc_e2m1_to_f64.argtypes = [ctypes.c_uint8]
         L.orc_e2m1_to_f64.restype = ctypes.c_double
         L.orc_iq4nl_value.argtypes = [i32]
@@ -112,6 +116,10 @@ def f64_to_f16(v: float) -> int:
 
 def e4m3_to_f64(b: int) -> float:
     return lib().orc_e4m3_to_f64(int(b))
+
+
+def e8m0_to_f64(b: int) -> float:
+    return lib().orc_e8m0_to_f64(int(b))
 
 
 def e2m1_to_f64(nib: int) -> float:

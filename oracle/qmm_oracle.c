@@ -20,6 +20,9 @@
  *             per matrix; the weights are decoded to FP16.
  *   [MAMBA-S] same page, section "Storage and runtime memory": the decoded
  *             weights are held as resident FP16 tensors.
+ *   [ZQ-MX]   "1bit.gg zyphra", section "What these numbers say": MXFP4
+ *             experts are E2M1 codes, 32 per group, with one E8M0 scale byte
+ *             per group (the OCP microscaling format).
  *
  * Readings where the pages are silent (each is listed in the design notes):
  *   - IQ4_NL block: scale first, little-endian; low nibble of qs[j] is weight
@@ -32,6 +35,9 @@
  *     subnormals kept): w = fp16(code * scale).  For the E4M3FN variant the
  *     product code * e4m3 * g is rounded to fp32 first (the FP32 global
  *     scale is an fp32 multiply) and then to fp16.
+ *   - MXFP4: the codes are laid out as for FP4-G16; the scales are a
+ *     separate row-major [n][k/32] array of E8M0 bytes; w = fp16(code *
+ *     2^(e-127)), one rounding; e = 0xFF is NaN.
  *   - The matrix product is y[m][n] = sum_k w16[n][k] * x[m][k], evaluated
  *     here in double precision in ascending k.
  *
@@ -45,6 +51,7 @@
 #define ORC_FMT_IQ4_NL 1
 #define ORC_FMT_FP4G16_F16 2
 #define ORC_FMT_FP4G16_E4M3 3
+#define ORC_FMT_MXFP4 4
 
 /* ---------------------------------------------------------------------- */
 /* IEEE 754 binary16 (half precision): 1 sign, 5 exponent (bias 15),      */
@@ -141,6 +148,15 @@ double orc_e2m1_to_f64(uint8_t nib) {
   return sign ? -v : v;
 }
 
+/* ---------------------------------------------------------------------- */
+/* OCP MX E8M0 scale: an unsigned biased exponent, value 2^(e-127); no     */
+/* sign, no zero; only 0xFF is NaN ([ZQ-MX] names the type).               */
+/* ---------------------------------------------------------------------- */
+double orc_e8m0_to_f64(uint8_t b) {
+  if (b == 0xFF) return NAN;
+  return ldexp(1.0, (int)b - 127);
+}
+
 /* The IQ4_NL non-linear table printed in [MARK-Q]. */
 static const int orc_iq4nl_table[16] = {-127, -104, -83, -65, -49, -35, -22, -10,
                                         1,    13,   25,  38,  53,  69,  89,  113};
@@ -162,6 +178,7 @@ int64_t orc_data_bytes(int fmt, int64_t n, int64_t k) {
 int64_t orc_scale_bytes(int fmt, int64_t n, int64_t k) {
   if (fmt == ORC_FMT_FP4G16_F16) return n * (k / 16) * 2;
   if (fmt == ORC_FMT_FP4G16_E4M3) return n * (k / 16) * 1;
+  if (fmt == ORC_FMT_MXFP4) return n * (k / 32) * 1; /* [ZQ-MX]: one byte per 32 */
   return 0;
 }
 
@@ -198,6 +215,11 @@ void orc_dequant_row(int fmt, int64_t n, int64_t k, const uint8_t* data, const u
     if (fmt == ORC_FMT_FP4G16_F16) {
       const uint8_t* sp = scales + (row * (k / 16) + g) * 2;
       double s = orc_f16_to_f64((uint16_t)(sp[0] | (sp[1] << 8)));
+      out[kk] = orc_f64_to_f16(c * s);
+    } else if (fmt == ORC_FMT_MXFP4) {
+      /* c has two significant bits and the scale is a power of two from
+       * 2^-127 to 2^127, so the double product is exact. */
+      double s = orc_e8m0_to_f64(scales[row * (k / 32) + kk / 32]);
       out[kk] = orc_f64_to_f16(c * s);
     } else {
       double e = orc_e4m3_to_f64(scales[row * (k / 16) + g]);

@@ -14,6 +14,9 @@ routing):
   E4M3FN variant of the model card, ``s = |N(0,1)| * 0.05`` in fp32,
   ``g = max(s) / 448`` and block scale ``e4m3(s / g)`` (round to nearest even,
   by torch's float8_e4m3fn cast).
+* MXFP4: the same codes and one E8M0 byte per 32 consecutive K elements,
+  ``127 + floor(log2(|N(0,1)| * 0.05))`` (the power of two at or below the
+  draw, clipped to 0..254).
 * IQ4_NL: per 32-weight block a scale ``d = fp16(|N(0,1)| * 0.002)`` and 16
   bytes of uniform random nibble pairs.
 * Activations: ``fp16(N(0,1))``.
@@ -32,7 +35,9 @@ import numpy as np
 FMT_IQ4_NL = 1
 FMT_FP4G16_F16 = 2
 FMT_FP4G16_E4M3 = 3
-FMT_NAMES = {FMT_IQ4_NL: "iq4_nl", FMT_FP4G16_F16: "fp4g16_f16", FMT_FP4G16_E4M3: "fp4g16_e4m3"}
+FMT_MXFP4 = 4
+FMT_NAMES = {FMT_IQ4_NL: "iq4_nl", FMT_FP4G16_F16: "fp4g16_f16", FMT_FP4G16_E4M3: "fp4g16_e4m3",
+             FMT_MXFP4: "mxfp4"}
 
 
 @dataclass
@@ -64,9 +69,14 @@ def _fp16_bits(a: np.ndarray) -> np.ndarray:
 
 
 def gen_fp4(rng: np.random.Generator, n: int, k: int, fmt: int = FMT_FP4G16_F16, experts: int = 1) -> Packed:
-    if k % 16:
-        raise ValueError("FP4-G16 needs k % 16 == 0")
+    if k % 16 or (fmt == FMT_MXFP4 and k % 32):
+        raise ValueError("FP4-G16 needs k % 16 == 0, MXFP4 k % 32 == 0")
     codes = rng.integers(0, 256, size=(experts, n, k // 2), dtype=np.uint8)
+    if fmt == FMT_MXFP4:
+        s = np.abs(rng.standard_normal((experts, n, k // 32), dtype=np.float32)) * np.float32(0.05)
+        with np.errstate(divide="ignore"):
+            e = np.clip(127.0 + np.floor(np.log2(s.astype(np.float64))), 0, 254).astype(np.uint8)
+        return Packed(fmt, n, k, codes.reshape(-1), e.reshape(-1), 1.0, experts)
     s = np.abs(rng.standard_normal((experts, n, k // 16), dtype=np.float32)) * np.float32(0.05)
     if fmt == FMT_FP4G16_F16:
         return Packed(fmt, n, k, codes.reshape(-1), _fp16_bits(s).view(np.uint8).reshape(-1), 1.0, experts)

@@ -21,7 +21,9 @@ def golden_lines(name):
 
 
 def parse_value(tok: str) -> float:
-    """Decimal, or '<int>p<exp>' meaning int * 2^exp (exact)."""
+    """Decimal, 'inf'/'-inf', or '<int>p<exp>' meaning int * 2^exp (exact)."""
+    if tok in ("inf", "-inf"):
+        return float(tok)
     if "p" in tok:
         mant, ex = tok.split("p")
         return float(int(mant)) * 2.0 ** int(ex)

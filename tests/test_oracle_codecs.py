@@ -69,6 +69,17 @@ def test_e4m3_all_bytes_match_torch():
     assert sum(math.isnan(g) for g in got) == 2
 
 
+def test_e8m0_all_bytes_match_torch():
+    """OCP E8M0 (the MXFP4 scale): all 256 bytes against torch's
+    float8_e8m0fnu; 0x7f is 1, 0x00 is 2^-127, 0xff the only NaN."""
+    allb = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = allb.view(torch.float8_e8m0fnu).to(torch.float64).numpy()
+    got = np.array([oracle.e8m0_to_f64(b) for b in range(256)])
+    assert all(_same(g, r) for g, r in zip(got, ref))
+    assert got[0x7F] == 1.0 and got[0x00] == 2.0 ** -127 and got[0xFE] == 2.0 ** 127 and math.isnan(got[0xFF])
+    assert sum(math.isnan(g) for g in got) == 1
+
+
 def test_e2m1_matches_printed_magnitudes():
     mags = [float(t) for t in golden_lines("e2m1_magnitudes.txt")[0].split()]
     assert mags == sorted(mags) and len(mags) == 8

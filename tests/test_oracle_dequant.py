@@ -168,3 +168,60 @@ def test_fp4_e4m3_all_scale_bytes_vs_numpy_rounding(g):
     nan_e = ((exp & 0x7C00) == 0x7C00) & ((exp & 0x3FF) != 0)
     assert np.array_equal(nan_g, nan_e)
     assert np.array_equal(got[~nan_g], exp[~nan_e])
+
+
+# -- MXFP4 (E2M1 codes, one E8M0 scale byte per 32) ---------------------------
+def _mx_cases():
+    lines = golden_lines("mxfp4_rows_handmade.txt")
+    cases = []
+    for i in range(0, len(lines), 3):
+        codes = np.array([int(t, 16) for t in lines[i].split()[1:]], dtype=np.uint8)
+        scale = np.array([int(lines[i + 1].split()[1], 16)], dtype=np.uint8)
+        exp = [parse_value(t) for t in lines[i + 2].split()[1:]]
+        assert len(codes) == 16 and len(exp) == 32
+        cases.append((codes, scale, exp))
+    return cases
+
+
+def test_mxfp4_handmade_rows():
+    cases = _mx_cases()
+    assert len(cases) == 6
+    for codes, scale, exp in cases:
+        got = oracle.dequant(oracle.FMT_MXFP4, 1, 32, codes, scale)
+        assert np.array_equal(got[0], _to_bits(exp)), (scale, got)
+
+
+def test_mxfp4_nan_scale():
+    """E8M0 0xFF is NaN: every weight of its group is NaN, zeros included."""
+    codes = np.array([0x10, 0x32, 0x54, 0x76, 0x98, 0xBA, 0xDC, 0xFE] * 2, dtype=np.uint8)
+    got = oracle.dequant(oracle.FMT_MXFP4, 1, 32, codes, np.array([0xFF], dtype=np.uint8))[0]
+    assert np.all(((got & 0x7C00) == 0x7C00) & ((got & 0x3FF) != 0))
+
+
+def test_mxfp4_mutations_are_caught():
+    """A swapped nibble convention, a reversed code pair order, a flipped
+    nibble and a scale off by one are each visible in the golden rows."""
+    codes, scale, exp = _mx_cases()[5]
+    ref = _to_bits(exp)
+    muts = [(((codes & 0x0F) << 4) | (codes >> 4), scale),                  # swapped nibble convention
+            (np.concatenate([codes[1::-1], codes[2:]]), scale),             # reversed byte (pair) order
+            (codes ^ np.array([0x01] + [0] * 15, dtype=np.uint8), scale),   # one flipped nibble bit
+            (codes, scale + 1), (codes, scale - 1)]                          # scale off by one
+    for c, s in muts:
+        assert not np.array_equal(oracle.dequant(oracle.FMT_MXFP4, 1, 32, c, s)[0], ref)
+
+
+def test_mxfp4_all_scale_bytes_vs_numpy_rounding():
+    """Every E8M0 byte x every code: fp16(code * 2^(e-127)) rounded by numpy
+    from the exact double product."""
+    e2m1 = np.array([oracle.e2m1_to_f64(c) for c in range(16)], dtype=np.float64)
+    n = 256
+    codes = np.tile(np.array([0x10, 0x32, 0x54, 0x76, 0x98, 0xBA, 0xDC, 0xFE] * 2, dtype=np.uint8), (n, 1))
+    got = oracle.dequant(oracle.FMT_MXFP4, n, 32, codes.reshape(-1), np.arange(256, dtype=np.uint8))
+    with np.errstate(all="ignore"):
+        scale = np.where(np.arange(256) == 255, np.nan, np.ldexp(1.0, np.arange(256) - 127))
+        exp = (scale[:, None] * np.tile(e2m1, 2)[None, :]).astype(np.float16).view(np.uint16)
+    nan_g = ((got & 0x7C00) == 0x7C00) & ((got & 0x3FF) != 0)
+    nan_e = ((exp & 0x7C00) == 0x7C00) & ((exp & 0x3FF) != 0)
+    assert np.array_equal(nan_g, nan_e) and nan_g[255].all() and not nan_g[:255].any()
+    assert np.array_equal(got[~nan_g], exp[~nan_e])

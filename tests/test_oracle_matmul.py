@@ -41,6 +41,11 @@ def _weights_exact(w):
             if w.fmt == synth.FMT_FP4G16_F16:
                 s = float(w.scales.view(np.uint16).reshape(n, k // 16)[r, kk // 16].view(np.float16))
                 out[r, kk] = Fraction(float(np.float16(c * s)))
+            elif w.fmt == synth.FMT_MXFP4:
+                import torch
+                e = float(torch.tensor([w.scales.reshape(n, k // 32)[r, kk // 32]], dtype=torch.uint8)
+                          .view(torch.float8_e8m0fnu).double())
+                out[r, kk] = Fraction(float(np.float16(c * e)))
             else:
                 import torch
                 e = float(torch.tensor([w.scales.reshape(n, k // 16)[r, kk // 16]], dtype=torch.uint8)
@@ -51,7 +56,7 @@ def _weights_exact(w):
 
 @pytest.mark.parametrize("fmt,n,k,m", [(synth.FMT_IQ4_NL, 8, 64, 3), (synth.FMT_IQ4_NL, 5, 32, 1),
                                        (synth.FMT_FP4G16_F16, 8, 32, 2), (synth.FMT_FP4G16_F16, 3, 64, 4),
-                                       (synth.FMT_FP4G16_E4M3, 6, 48, 2)])
+                                       (synth.FMT_FP4G16_E4M3, 6, 48, 2), (synth.FMT_MXFP4, 4, 64, 3)])
 def test_brute_force_exact(fmt, n, k, m):
     rng = np.random.default_rng(7 + n + k)
     w = synth.gen_weights(rng, fmt, n, k)
@@ -67,7 +72,7 @@ def test_brute_force_exact(fmt, n, k, m):
             assert abs(Fraction(a[i, r]) - absum) <= Fraction(2 * k, 2 ** 53) * absum
 
 
-@pytest.mark.parametrize("fmt", [synth.FMT_IQ4_NL, synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3])
+@pytest.mark.parametrize("fmt", [synth.FMT_IQ4_NL, synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3, synth.FMT_MXFP4])
 def test_one_hot_gives_decoded_column(fmt):
     rng = np.random.default_rng(11)
     n, k = 16, 64

@@ -61,3 +61,13 @@ def test_iq4nl_sizes():
 def test_fp4_sizes():
     assert oracle.data_bytes(oracle.FMT_FP4G16_F16, 18560, 4096) + oracle.scale_bytes(oracle.FMT_FP4G16_F16, 18560, 4096) == 47513600
     assert oracle.data_bytes(oracle.FMT_FP4G16_E4M3, 18560, 4096) + oracle.scale_bytes(oracle.FMT_FP4G16_E4M3, 18560, 4096) + 4 == 42762244
+
+
+def test_mxfp4_sizes():
+    """MXFP4 ("1bit.gg zyphra": E8M0 scale byte and 32 E2M1 codes per group):
+    16 code bytes and 1 scale byte per 32 weights, 4.25 bits per weight."""
+    assert oracle.data_bytes(oracle.FMT_MXFP4, 1, 32) == 16
+    assert oracle.scale_bytes(oracle.FMT_MXFP4, 1, 32) == 1
+    n, k = 2560, 896
+    total = oracle.data_bytes(oracle.FMT_MXFP4, n, k) + oracle.scale_bytes(oracle.FMT_MXFP4, n, k)
+    assert total == n * k * 17 // 32 and 8 * total / (n * k) == 4.25
