@@ -426,12 +426,18 @@ def extra_workloads(args, world, l2, peaks):
     out["fp4g16_e4m3_gemv_in_proj_m1"] = {"variant": r["variant"], "gbs": r["gbs"],
                                           "frac_hbm": r["gbs"] / peaks["hbm_gbs"],
                                           "us_per_launch": r["s_per_launch"] * 1e6}
+    p, x = synth.make_gemv(synth.FP4_IN_PROJ, synth.FMT_MXFP4)
+    r = gemv_workload(p, x, steps, warm, world, l2)
+    out["mxfp4_gemv_in_proj_m1"] = {"variant": r["variant"], "gbs": r["gbs"], "frac_hbm": r["gbs"] / peaks["hbm_gbs"],
+                                    "us_per_launch": r["s_per_launch"] * 1e6,
+                                    "note": "E2M1 codes + one E8M0 byte per 32 (4.25 bits per weight)"}
     p, x = synth.make_gemv(synth.IQ4_TINY)
     r = gemv_workload(p, x, steps, warm, world, l2)
     out["iq4nl_gemv_tiny_256x512_m1"] = {"variant": r["variant"], "gbs": r["gbs"],
                                          "us_per_launch": r["s_per_launch"] * 1e6, "note": "fits in L2"}
     out["fp4g16_prefill_gemm_2048x18560x4096"] = gemm_workload(synth.FMT_FP4G16_F16, world, l2, peaks)
     out["fp4g16_e4m3_prefill_gemm_2048x18560x4096"] = gemm_workload(synth.FMT_FP4G16_E4M3, world, l2, peaks)
+    out["mxfp4_prefill_gemm_2048x18560x4096"] = gemm_workload(synth.FMT_MXFP4, world, l2, peaks)
     out["iq4nl_grouped_experts_t64_top4"] = grouped_workload(world, l2, peaks)
     out["iq4nl_moe_block_t64_top4"] = moe_workload(world, l2, peaks, t=64)
     out["iq4nl_moe_block_t1_top4"] = moe_workload(world, l2, peaks, t=1)

@@ -72,7 +72,13 @@ typedef enum {
 typedef enum {
   QMM_FMT_IQ4_NL = 1,
   QMM_FMT_FP4G16_F16 = 2,
-  QMM_FMT_FP4G16_E4M3 = 3
+  QMM_FMT_FP4G16_E4M3 = 3,
+  /* E2M1 codes laid out as for FP4-G16 plus one OCP E8M0 scale byte per 32
+   * consecutive k, a separate [n][k/32] array ("1bit.gg zyphra", section
+   * "What these numbers say": MXFP4 experts, E8M0 scale bytes and 32 E2M1
+   * codes per group).  w = fp16(code * 2^(e-127)), one rounding; e = 0xFF
+   * is NaN.  k % 32 == 0. */
+  QMM_FMT_MXFP4 = 4
 } qmm_format;
 
 /* One packed matrix, or a stack of `num_experts` packed matrices of equal
@@ -83,9 +89,10 @@ typedef struct {
   int32_t fmt;            /* qmm_format */
   int32_t reserved;       /* must be 0 */
   int64_t n;              /* output rows */
-  int64_t k;              /* input columns: k % 32 == 0 (IQ4_NL), k % 16 == 0 (FP4) */
+  int64_t k;              /* input columns: k % 32 == 0 (IQ4_NL, MXFP4), k % 16 == 0 (FP4-G16) */
   const void* data;       /* device: IQ4_NL blocks, or FP4 codes [n][k/2] */
-  const void* scales;     /* device: FP4 scales [n][k/16] (fp16 or E4M3FN); NULL for IQ4_NL */
+  const void* scales;     /* device: FP4-G16 scales [n][k/16] (fp16 or E4M3FN), MXFP4 [n][k/32]
+                           * E8M0 bytes; NULL for IQ4_NL */
   float global_scale;     /* FP4G16_E4M3 only (fp32 g); ignored otherwise */
   int32_t reserved2;      /* must be 0 */
   int64_t num_experts;    /* 1 for a plain matrix */
@@ -98,7 +105,7 @@ typedef struct {
 size_t qmm_data_bytes(int32_t fmt, int64_t n, int64_t k);
 
 /* Bytes of the separate scale array of one matrix (IQ4_NL: 0; FP4G16_F16:
- * n*k/16*2; FP4G16_E4M3: n*k/16). */
+ * n*k/16*2; FP4G16_E4M3: n*k/16; MXFP4: n*k/32). */
 size_t qmm_scale_bytes(int32_t fmt, int64_t n, int64_t k);
 
 /* qmm_data_bytes + qmm_scale_bytes (+4 for the FP4G16_E4M3 global scale, as

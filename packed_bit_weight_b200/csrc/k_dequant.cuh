@@ -49,6 +49,34 @@ __global__ void __launch_bounds__(256) dequant_fp4_kernel(const uint8_t* __restr
   }
 }
 
+// MXFP4: one thread per 32-weight group (16 code bytes, one E8M0 byte);
+// fp16(code * 2^(e-127)), one rounding ("1bit.gg zyphra", MXFP4 experts).
+__global__ void __launch_bounds__(256) dequant_mxfp4_kernel(const uint8_t* __restrict__ codes,
+                                                            const uint8_t* __restrict__ scales,
+                                                            uint16_t* __restrict__ out, int64_t groups) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < groups; i += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 q = *reinterpret_cast<const uint4*>(codes + i * 16);
+    const uint32_t b = scales[i];
+    uint32_t w[16];
+    e2m1x8_to_f16x2(q.x, *reinterpret_cast<uint32_t(*)[4]>(&w[0]));
+    e2m1x8_to_f16x2(q.y, *reinterpret_cast<uint32_t(*)[4]>(&w[4]));
+    e2m1x8_to_f16x2(q.z, *reinterpret_cast<uint32_t(*)[4]>(&w[8]));
+    e2m1x8_to_f16x2(q.w, *reinterpret_cast<uint32_t(*)[4]>(&w[12]));
+    if (e8m0_f16_ok(b)) {
+      const uint32_t ss = e8m0_to_f16x2(b);
+#pragma unroll
+      for (int j = 0; j < 16; j++) w[j] = hmul2(w[j], ss);
+    } else {
+      const float sf = e8m0_to_f32(b);
+#pragma unroll
+      for (int j = 0; j < 16; j++) w[j] = mx_scale_any(w[j], sf);
+    }
+    uint4* o = reinterpret_cast<uint4*>(out + i * 32);
+#pragma unroll
+    for (int j = 0; j < 4; j++) o[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+  }
+}
+
 // IQ4_NL: one thread per 18-byte block (2-byte aligned: read as 9 halves).
 __global__ void __launch_bounds__(256) dequant_iq4nl_kernel(const uint8_t* __restrict__ blocks,
                                                             uint16_t* __restrict__ out, int64_t nblocks) {

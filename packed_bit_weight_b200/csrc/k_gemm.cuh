@@ -472,6 +472,10 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
           cp_async16_g(dst + kStageCodes + r * 32 + ((h ^ ((r >> 2) & 1)) << 4),
                        scales + (gr * srow + (kc >> 4)) * 2 + h * 16);
         }
+      } else if (FMT == 4) {  // MXFP4: 8 E8M0 bytes per row (one per 32 k)
+        const int r = t;
+        const int64_t gr = min((int64_t)n0 + r, (int64_t)n - 1);
+        cp_async8_g(dst + kStageCodes + r * 32, scales + gr * (srow >> 1) + (kc >> 5));
       } else {  // E4M3: 16 bytes per row, copied whole; words read swizzled
         const int r = t;
         const int64_t gr = min((int64_t)n0 + r, (int64_t)n - 1);
@@ -496,10 +500,23 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
         const uint4 c0 = lds128(src + t * 128 + (((2 * j) ^ (t & 7)) << 4));
         const uint4 c1 = lds128(src + t * 128 + (((2 * j + 1) ^ (t & 7)) << 4));
         uint32_t sc[4];
+        bool mx_wide = false;  // MXFP4 scale that is not an fp16 value: two fp16 factors
+        uint32_t mx0a = 0u, mx0b = 0u, mx1a = 0u, mx1b = 0u;
         if (FMT == 2) {
           const uint32_t half = (uint32_t)((j >> 1) ^ ((t >> 2) & 1));
           const uint2 sv = lds64(src + kStageCodes + t * 32 + (half << 4) + (j & 1) * 8);
           sc[0] = bcast_lo(sv.x); sc[1] = bcast_hi(sv.x); sc[2] = bcast_lo(sv.y); sc[3] = bcast_hi(sv.y);
+        } else if (FMT == 4) {  // two E8M0 bytes for this step's 64 k
+          const uint32_t sw = lds32(src + kStageCodes + t * 32 + (j >> 1) * 4) >> ((j & 1) * 16);
+          const uint32_t b0 = sw & 0xFFu, b1 = (sw >> 8) & 0xFFu;
+          mx_wide = !(e8m0_f16_ok(b0) && e8m0_f16_ok(b1));
+          if (mx_wide) {  // rare: two fp16 factors per group
+            e8m0_f16_factors(b0, mx0a, mx0b);
+            e8m0_f16_factors(b1, mx1a, mx1b);
+          }
+          const int v0 = (int)b0 - 127, v1 = (int)b1 - 127;  // the power itself when it is an fp16 value
+          sc[0] = sc[1] = f16x2_pow2(v0 < -24 ? -24 : (v0 > 15 ? 15 : v0));
+          sc[2] = sc[3] = f16x2_pow2(v1 < -24 ? -24 : (v1 > 15 ? 15 : v1));
         } else {
           const uint32_t sw = lds32(src + kStageCodes + t * 32 + j * 4);
           const uint32_t e01 = e4m3x2_to_f16x2(sw & 0xFFFFu), e23 = e4m3x2_to_f16x2(sw >> 16);
@@ -510,12 +527,25 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
         const uint32_t q[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
         const uint32_t row_base = b_s + s * C::kBBytes + (uint32_t)t * 128u;
         const uint32_t swz = (uint32_t)(t & 7);
+        if (FMT == 4 && mx_wide) {
+          if (!valid) mx0a = mx0b = mx1a = mx1b = 0u;
 #pragma unroll
-        for (int cc = 0; cc < 8; cc++) {
-          uint32_t w4[4];
-          e2m1x8_to_f16x2(q[cc], w4);
-          const uint32_t sv = sc[cc >> 1];
-          sts128(row_base + ((cc ^ swz) << 4), hmul2(w4[0], sv), hmul2(w4[1], sv), hmul2(w4[2], sv), hmul2(w4[3], sv));
+          for (int cc = 0; cc < 8; cc++) {
+            uint32_t w4[4];
+            e2m1x8_to_f16x2(q[cc], w4);
+            const uint32_t fa = (cc < 4) ? mx0a : mx1a, fb = (cc < 4) ? mx0b : mx1b;
+            sts128(row_base + ((cc ^ swz) << 4), hmul2(hmul2(w4[0], fa), fb), hmul2(hmul2(w4[1], fa), fb),
+                   hmul2(hmul2(w4[2], fa), fb), hmul2(hmul2(w4[3], fa), fb));
+          }
+        } else {
+#pragma unroll
+          for (int cc = 0; cc < 8; cc++) {
+            uint32_t w4[4];
+            e2m1x8_to_f16x2(q[cc], w4);
+            const uint32_t sv = sc[cc >> 1];
+            sts128(row_base + ((cc ^ swz) << 4), hmul2(w4[0], sv), hmul2(w4[1], sv), hmul2(w4[2], sv),
+                   hmul2(w4[3], sv));
+          }
         }
         fence_proxy_async_shared();
         mbar_arrive(bars + 8 * s);

@@ -43,6 +43,10 @@ __device__ __forceinline__ uint32_t generic_pair(const uint8_t* __restrict__ dat
   } else {
     const uint32_t byte = data[row * (k >> 1) + (kk >> 1)];
     const uint32_t c = e2m1x2_to_f16x2(byte);
+    if (FMT == 4) {  // MXFP4: one E8M0 byte per 32
+      const uint32_t e = scales[row * (k >> 5) + (kk >> 5)];
+      return e8m0_f16_ok(e) ? hmul2(c, e8m0_to_f16x2(e)) : mx_scale_any(c, e8m0_to_f32(e));
+    }
     const int64_t gi = row * (k >> 4) + (kk >> 4);
     if (FMT == 2) {
       const uint32_t s = reinterpret_cast<const uint16_t*>(scales)[gi];
@@ -335,6 +339,11 @@ __device__ __forceinline__ uint32_t ldg_stream32(const void* p) {
   asm("ld.global.nc.L1::no_allocate.L2::256B.u32 %0, [%1];" : "=r"(v) : "l"(p));
   return v;
 }
+__device__ __forceinline__ uint32_t ldg_stream8(const void* p) {
+  unsigned short v;
+  asm("ld.global.nc.L1::no_allocate.L2::256B.u8 %0, [%1];" : "=h"(v) : "l"(p));
+  return v;
+}
 __device__ __forceinline__ uint32_t ldg_stream16(const void* p) {
   unsigned short v;
   asm("ld.global.nc.L1::no_allocate.L2::256B.u16 %0, [%1];" : "=h"(v) : "l"(p));
@@ -383,8 +392,13 @@ __device__ __forceinline__ void ldg_tile_mma(float (&acc)[NT][4], const uint4 (&
         for (int q = 0; q < 16; q++) xb[j][q] = 0u;
       }
     }
-    const uint32_t sa0 = bcast_lo(sa[i]), sa1 = bcast_hi(sa[i]);
-    const uint32_t sb0 = bcast_lo(sb[i]), sb1 = bcast_hi(sb[i]);
+    // group scales as f16x2: two fp16 groups per lane (FP4-G16), or one
+    // E8M0 group (MXFP4: a power of two, applied as two fp16 factors so that
+    // scales outside the fp16 range round exactly once too)
+    uint32_t sa0, sa1, sb0, sb1;
+    // FP4-G16: the two groups' scales; MXFP4: the one group's two fp16
+    // factors (the first is 1 when the scale is an fp16 value)
+    sa0 = bcast_lo(sa[i]); sa1 = bcast_hi(sa[i]); sb0 = bcast_lo(sb[i]); sb1 = bcast_hi(sb[i]);
     uint32_t wa[16], wb[16];
     e2m1x8_to_f16x2(qa[i].x, *reinterpret_cast<uint32_t(*)[4]>(&wa[0]));
     e2m1x8_to_f16x2(qa[i].y, *reinterpret_cast<uint32_t(*)[4]>(&wa[4]));
@@ -396,9 +410,15 @@ __device__ __forceinline__ void ldg_tile_mma(float (&acc)[NT][4], const uint4 (&
     e2m1x8_to_f16x2(qb[i].w, *reinterpret_cast<uint32_t(*)[4]>(&wb[12]));
 #pragma unroll
     for (int st = 0; st < 8; st++) {
-      const uint32_t sA = (st < 4) ? sa0 : sa1, sB = (st < 4) ? sb0 : sb1;
-      const uint32_t a0 = hmul2(wa[2 * st], sA), a2 = hmul2(wa[2 * st + 1], sA);
-      const uint32_t a1 = hmul2(wb[2 * st], sB), a3 = hmul2(wb[2 * st + 1], sB);
+      uint32_t a0, a1, a2, a3;
+      if (FMT == 4) {  // the lane's one group: code * f1 exact, * f2 rounds once
+        a0 = hmul2(hmul2(wa[2 * st], sa0), sa1); a2 = hmul2(hmul2(wa[2 * st + 1], sa0), sa1);
+        a1 = hmul2(hmul2(wb[2 * st], sb0), sb1); a3 = hmul2(hmul2(wb[2 * st + 1], sb0), sb1);
+      } else {  // group st/4 of the lane's two
+        const uint32_t sA = (st < 4) ? sa0 : sa1, sB = (st < 4) ? sb0 : sb1;
+        a0 = hmul2(wa[2 * st], sA); a2 = hmul2(wa[2 * st + 1], sA);
+        a1 = hmul2(wb[2 * st], sB); a3 = hmul2(wb[2 * st + 1], sB);
+      }
 #pragma unroll
       for (int j = 0; j < NT; j++) mma_16816(acc[j], a0, a1, a2, a3, xb[j][2 * st], xb[j][2 * st + 1]);
     }
@@ -457,6 +477,9 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
     if (FMT == 2) {
       sa[i] = va ? ldg_stream32(scales + (ra * srow + gi) * 2) : 0u;
       sb[i] = vb ? ldg_stream32(scales + (rb * srow + gi) * 2) : 0u;
+    } else if (FMT == 4) {  // the lane's 32 k are one MXFP4 group: one E8M0 byte (127 = 1 for rows past n)
+      sa[i] = e8m0_f16_factor_pair(va ? ldg_stream8(scales + ra * (srow >> 1) + seg * 4 + tig) : 127u);
+      sb[i] = e8m0_f16_factor_pair(vb ? ldg_stream8(scales + rb * (srow >> 1) + seg * 4 + tig) : 127u);
     } else {
       sa[i] = va ? e4m3x2_to_f16x2(ldg_stream16(scales + ra * srow + gi)) : 0u;
       sb[i] = vb ? e4m3x2_to_f16x2(ldg_stream16(scales + rb * srow + gi)) : 0u;

@@ -70,6 +70,47 @@ __device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
   return d;
 }
 
+// MXFP4 group scale: an OCP E8M0 byte b is 2^(b-127); 0xFF is NaN.
+// e8m0_f16_ok: 2^(b-127) is an fp16 value (2^-24 .. 2^15, b in [103, 142]),
+// so one f16x2 multiply by e8m0_to_f16x2(b) rounds code * scale exactly once.
+__device__ __forceinline__ bool e8m0_f16_ok(uint32_t b) { return b - 103u <= 39u; }
+__device__ __forceinline__ uint32_t e8m0_to_f16x2(uint32_t b) {
+  const int s = (int)b - 127;
+  const uint32_t h = (s >= -14) ? (uint32_t)(s + 15) << 10 : 1u << (s + 24);  // normal or subnormal 2^s
+  return h | (h << 16);
+}
+// Any E8M0 byte as two fp16 factors f1, f2 (f16x2 broadcasts) such that
+// fp16((code * f1) * f2) == fp16(code * 2^(b-127)) for every E2M1 code with
+// the first product exact: 2^(b-127) = f1 * f2 when that fits (f1 = 1 inside
+// the fp16 range; f1 = 2^-14 below it; f1 = 2^15 above it, where a first
+// product that overflows means the true one does too); below 2^-38 and
+// above 2^30 the clamped factors round to the same zero / infinity; 0xFF
+// gives f2 = NaN.
+__device__ __forceinline__ uint32_t f16x2_pow2(int v) {  // 2^v, v in [-24, 15]
+  const uint32_t h = (v >= -14) ? (uint32_t)(v + 15) << 10 : 1u << (v + 24);
+  return h | (h << 16);
+}
+__device__ __forceinline__ void e8m0_f16_factors(uint32_t b, uint32_t& f1, uint32_t& f2) {
+  const int s = (int)b - 127;
+  const int a = (s < -24) ? -14 : ((s > 15) ? 15 : 0);
+  int r = s - a;
+  r = r < -24 ? -24 : (r > 15 ? 15 : r);
+  f1 = f16x2_pow2(a);
+  f2 = (b == 255u) ? 0x7E007E00u : f16x2_pow2(r);
+}
+
+// The two factors of e8m0_f16_factors packed as two fp16 halves (f1 low).
+__device__ __forceinline__ uint32_t e8m0_f16_factor_pair(uint32_t b) {
+  uint32_t f1, f2;
+  e8m0_f16_factors(b, f1, f2);
+  return (f1 & 0xFFFFu) | (f2 << 16);
+}
+
+// 2^(b-127) as fp32 for every byte (b = 0: the fp32 subnormal 2^-127).
+__device__ __forceinline__ float e8m0_to_f32(uint32_t b) {
+  return b == 0u ? __uint_as_float(0x00400000u) : (b == 255u ? __uint_as_float(0x7FC00000u) : __uint_as_float(b << 23));
+}
+
 // Broadcast the low / high f16 of a word to both halves.
 __device__ __forceinline__ uint32_t bcast_lo(uint32_t v) { return __byte_perm(v, v, 0x1010); }
 __device__ __forceinline__ uint32_t bcast_hi(uint32_t v) { return __byte_perm(v, v, 0x3232); }
@@ -101,6 +142,16 @@ __device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a
       "{%0,%1,%2,%3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// ---------------------------------------------------------------------------
+// fp16(code * scale) for the two exact code values of f16x2 c and any MXFP4
+// scale s (fp32 from e8m0_to_f32): the fp32 product is exact (two
+// significant bits times a power of two, fp32 subnormals kept), the narrowing
+// rounds once.
+__device__ __forceinline__ uint32_t mx_scale_any(uint32_t c, float s) {
+  const float2 f = f16x2_to_f32x2(c);
+  return f32x2_to_f16x2(f.x * s, f.y * s);
 }
 
 // ---------------------------------------------------------------------------

@@ -67,7 +67,10 @@ static qmm_status device_info(DevInfo** out) {
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-static bool valid_fmt(int32_t f) { return f == QMM_FMT_IQ4_NL || f == QMM_FMT_FP4G16_F16 || f == QMM_FMT_FP4G16_E4M3; }
+static bool valid_fmt(int32_t f) {
+  return f == QMM_FMT_IQ4_NL || f == QMM_FMT_FP4G16_F16 || f == QMM_FMT_FP4G16_E4M3 || f == QMM_FMT_MXFP4;
+}
+static int64_t fmt_group(int32_t f) { return (f == QMM_FMT_IQ4_NL || f == QMM_FMT_MXFP4) ? 32 : 16; }
 
 static qmm_status check_weights(const qmm_weights* w, bool allow_experts) {
   if (!w) return QMM_ERR_INVALID_ARG;
@@ -75,7 +78,7 @@ static qmm_status check_weights(const qmm_weights* w, bool allow_experts) {
   if (w->n < 0 || w->k < 0 || w->num_experts < 1) return QMM_ERR_INVALID_ARG;
   if (!allow_experts && w->num_experts != 1) return QMM_ERR_INVALID_ARG;
   if (w->n > INT32_MAX || w->k > INT32_MAX) return QMM_ERR_UNSUPPORTED_SHAPE;
-  if (w->fmt == QMM_FMT_IQ4_NL ? (w->k % 32) : (w->k % 16)) return QMM_ERR_UNSUPPORTED_SHAPE;
+  if (w->k % fmt_group(w->fmt)) return QMM_ERR_UNSUPPORTED_SHAPE;
   if (w->n > 0 && w->k > 0) {
     if (!w->data) return QMM_ERR_INVALID_ARG;
     if (w->fmt != QMM_FMT_IQ4_NL && !w->scales) return QMM_ERR_INVALID_ARG;
@@ -441,12 +444,15 @@ template <int FMT>
 static qmm_status gemv_fmt(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st,
                            const DevInfo* di) {
   const int64_t n = w->n, k = w->k;
-  if (FMT != 1) {
+  // FP4-G16 (fp16 or E4M3 scale per 16) has every streaming variant; MXFP4
+  // the register kernel and the generic one
+  constexpr bool kG16 = FMT == 2 || FMT == 3;
+  if constexpr (kG16) {
     qmm_status cs;
     if (gemv_cfg_env<FMT>(w, x, m, y, st, di, &cs)) return cs;
   }
   const int pick = gemv_variant_env();
-  if constexpr (FMT != 1) {
+  if constexpr (kG16) {
     if (pick == 8) {
       const qmm_status s = gemv_dual_auto<FMT>(w, x, m, y, st, di);
       if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
@@ -461,20 +467,22 @@ static qmm_status gemv_fmt(const qmm_weights* w, const uint16_t* x, int m, uint1
       if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
     }
   }
-  const bool tma_ok = FMT != 1 && k % kChunkK == 0 && k >= 8 * kChunkK && n >= 16;
   if (FMT != 1 && (pick == 0 || pick == 2)) {
     const qmm_status s = (m <= 8) ? gemv_ldg_auto<FMT, 1>(w, x, m, y, st) : gemv_ldg_auto<FMT, 2>(w, x, m, y, st);
     if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
   }
-  const int segs = (int)(k / 128);
-  const bool cpa_ok = FMT != 1 && k % 1024 == 0 && k >= 1024;
-  if (cpa_ok && pick == 4 && segs % 8 == 0) {
-    if (m <= 8) return launch_gemv_cpa<FMT, 1, 8, 8>(w, x, m, y, st, di);
-    return launch_gemv_cpa<FMT, 2, 8, 8>(w, x, m, y, st, di);
-  }
-  if (tma_ok && (pick == 0 || pick == 1)) {
-    if (m <= 8) return launch_gemv_tma<FMT, 1, 1>(w, x, m, y, st, di);
-    return launch_gemv_tma<FMT, 1, 2>(w, x, m, y, st, di);
+  if constexpr (kG16) {
+    const int segs = (int)(k / 128);
+    const bool cpa_ok = k % 1024 == 0 && k >= 1024;
+    if (cpa_ok && pick == 4 && segs % 8 == 0) {
+      if (m <= 8) return launch_gemv_cpa<FMT, 1, 8, 8>(w, x, m, y, st, di);
+      return launch_gemv_cpa<FMT, 2, 8, 8>(w, x, m, y, st, di);
+    }
+    const bool tma_ok = k % kChunkK == 0 && k >= 8 * kChunkK && n >= 16;
+    if (tma_ok && (pick == 0 || pick == 1)) {
+      if (m <= 8) return launch_gemv_tma<FMT, 1, 1>(w, x, m, y, st, di);
+      return launch_gemv_tma<FMT, 1, 2>(w, x, m, y, st, di);
+    }
   }
   if (FMT == 1 && pick == 6) {  // persistent kernel: measured slower than the streaming one, kept selectable
     const qmm_status s = launch_iq4_persist<IQ_OUT_F16>(w, nullptr, x, 0, 1, nullptr, 0, m, y, nullptr, st, di);
@@ -712,12 +720,14 @@ extern "C" {
 
 size_t qmm_data_bytes(int32_t fmt, int64_t n, int64_t k) {
   if (!valid_fmt(fmt) || n < 0 || k < 0) return 0;
-  if (fmt == QMM_FMT_IQ4_NL) return (k % 32) ? 0 : (size_t)n * (size_t)(k / 32) * 18u;
-  return (k % 16) ? 0 : (size_t)n * (size_t)(k / 2);
+  if (k % fmt_group(fmt)) return 0;
+  if (fmt == QMM_FMT_IQ4_NL) return (size_t)n * (size_t)(k / 32) * 18u;
+  return (size_t)n * (size_t)(k / 2);
 }
 
 size_t qmm_scale_bytes(int32_t fmt, int64_t n, int64_t k) {
-  if (!valid_fmt(fmt) || n < 0 || k < 0 || fmt == QMM_FMT_IQ4_NL || (k % 16)) return 0;
+  if (!valid_fmt(fmt) || n < 0 || k < 0 || fmt == QMM_FMT_IQ4_NL || (k % fmt_group(fmt))) return 0;
+  if (fmt == QMM_FMT_MXFP4) return (size_t)n * (size_t)(k / 32);
   return (size_t)n * (size_t)(k / 16) * (fmt == QMM_FMT_FP4G16_F16 ? 2u : 1u);
 }
 
@@ -764,6 +774,10 @@ qmm_status qmm_dequant(const qmm_weights* w, uint16_t* out, void* stream) {
     const int64_t ng = total / 16;
     dequant_fp4_kernel<2><<<grid_for(ng, 256, di->sms), 256, 0, st>>>(data, sc, 1.0f, out, ng);
     set_variant("dequant_fp4<fmt=2>");
+  } else if (w->fmt == QMM_FMT_MXFP4) {
+    const int64_t ng = total / 32;
+    dequant_mxfp4_kernel<<<grid_for(ng, 256, di->sms), 256, 0, st>>>(data, sc, out, ng);
+    set_variant("dequant_mxfp4");
   } else {
     const int64_t ng = total / 16;
     dequant_fp4_kernel<3><<<grid_for(ng, 256, di->sms), 256, 0, st>>>(data, sc, w->global_scale, out, ng);
@@ -796,6 +810,7 @@ qmm_status qmm_gemv(const qmm_weights* w, const uint16_t* x, int64_t m, uint16_t
   switch (w->fmt) {
     case QMM_FMT_IQ4_NL: return gemv_fmt<1>(w, x, (int)m, y, st, di);
     case QMM_FMT_FP4G16_F16: return gemv_fmt<2>(w, x, (int)m, y, st, di);
+    case QMM_FMT_MXFP4: return gemv_fmt<4>(w, x, (int)m, y, st, di);
     default: return gemv_fmt<3>(w, x, (int)m, y, st, di);
   }
 }
@@ -825,6 +840,9 @@ qmm_status qmm_gemm(const qmm_weights* w, const uint16_t* x, int64_t m, uint16_t
     case QMM_FMT_FP4G16_F16:
       if (!tc) return gemm_by_gemv<2>(w, x, m, y, st, di);
       return persist ? launch_gemm_tc_persistent<2>(w, x, (int)m, y, st, di) : launch_gemm_tc<2>(w, x, (int)m, y, st, di);
+    case QMM_FMT_MXFP4:  // the persistent kernel only (its 256-wide staging chunk holds 8 E8M0 bytes a row)
+      if (!tc || !persist) return gemm_by_gemv<4>(w, x, m, y, st, di);
+      return launch_gemm_tc_persistent<4>(w, x, (int)m, y, st, di);
     default:
       if (!tc) return gemm_by_gemv<3>(w, x, m, y, st, di);
       return persist ? launch_gemm_tc_persistent<3>(w, x, (int)m, y, st, di) : launch_gemm_tc<3>(w, x, (int)m, y, st, di);
@@ -908,6 +926,7 @@ qmm_status qmm_grouped_gemv(const qmm_weights* experts, const uint16_t* x, int32
   switch (experts->fmt) {
     case QMM_FMT_IQ4_NL: s = launch_grouped<1>(experts, x, x_per_pair, topk, offsets, perm, y, st); break;
     case QMM_FMT_FP4G16_F16: s = launch_grouped<2>(experts, x, x_per_pair, topk, offsets, perm, y, st); break;
+    case QMM_FMT_MXFP4: s = launch_grouped<4>(experts, x, x_per_pair, topk, offsets, perm, y, st); break;
     default: s = launch_grouped<3>(experts, x, x_per_pair, topk, offsets, perm, y, st); break;
   }
   set_variant("route+grouped_gemv_generic<fmt=%d>", experts->fmt);
@@ -957,6 +976,7 @@ qmm_status qmm_grouped_gemv_noalloc(const qmm_weights* experts, const uint16_t* 
   switch (experts->fmt) {
     case QMM_FMT_IQ4_NL: s = launch_grouped<1>(experts, x, x_per_pair, topk, offsets, perm, y, st); break;
     case QMM_FMT_FP4G16_F16: s = launch_grouped<2>(experts, x, x_per_pair, topk, offsets, perm, y, st); break;
+    case QMM_FMT_MXFP4: s = launch_grouped<4>(experts, x, x_per_pair, topk, offsets, perm, y, st); break;
     default: s = launch_grouped<3>(experts, x, x_per_pair, topk, offsets, perm, y, st); break;
   }
   set_variant("noalloc:route+grouped_gemv_generic<fmt=%d>", experts->fmt);

@@ -12,6 +12,7 @@ import ctypes
 import os
 from dataclasses import dataclass
 
+import numpy as np
 import torch
 
 from . import _build
@@ -19,6 +20,7 @@ from . import _build
 FMT_IQ4_NL = 1
 FMT_FP4G16_F16 = 2
 FMT_FP4G16_E4M3 = 3
+FMT_MXFP4 = 4
 
 OP_DEQUANT, OP_GEMV, OP_GEMM, OP_ROUTE, OP_GROUPED, OP_MOE = 0, 1, 2, 3, 4, 5
 
@@ -150,7 +152,22 @@ class PackedWeights:
 
     @staticmethod
     def from_host(p, device="cuda") -> "PackedWeights":
-        """From a ``synth.Packed`` (numpy bytes) to device tensors."""
+        """From a ``synth.Packed`` (numpy bytes) to device tensors.  An expert
+        stack whose per-expert byte counts are not multiples of 16 (e.g.
+        MXFP4 scales of an odd row count) is copied with each expert padded
+        to 16 bytes, as the expert strides of the C ABI require."""
+        ds, ss = p.data_stride, p.scale_stride
+        if p.experts > 1 and (ds % 16 or ss % 16):
+            pd, ps = -(-ds // 16) * 16, -(-ss // 16) * 16
+            d = np.zeros((p.experts, pd), dtype=np.uint8)
+            d[:, :ds] = p.data.reshape(p.experts, ds)
+            sc = None
+            if p.scales is not None:
+                sc = np.zeros((p.experts, ps), dtype=np.uint8)
+                sc[:, :ss] = p.scales.reshape(p.experts, ss)
+                sc = torch.from_numpy(sc.reshape(-1)).to(device)
+            return PackedWeights(p.fmt, p.n, p.k, torch.from_numpy(d.reshape(-1)).to(device), sc, p.global_scale,
+                                 p.experts, pd, ps if p.scales is not None else None)
         data = torch.from_numpy(p.data).to(device)
         scales = None if p.scales is None else torch.from_numpy(p.scales).to(device)
         return PackedWeights(p.fmt, p.n, p.k, data, scales, p.global_scale, p.experts)

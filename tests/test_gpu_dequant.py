@@ -9,7 +9,7 @@ from packed_bit_weight_b200 import qmm, synth
 
 pytestmark = pytest.mark.gpu
 
-FMTS = [synth.FMT_IQ4_NL, synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3]
+FMTS = [synth.FMT_IQ4_NL, synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3, synth.FMT_MXFP4]
 
 
 def _deq(w):
@@ -73,3 +73,13 @@ def test_dequant_empty_and_errors():
         qmm.qmm_dequant(w, out[1:129])                                   # 2-byte offset: misaligned
     assert e.value.status == 3
     assert qmm.qmm_sync_check() == 0
+
+
+def test_dequant_mxfp4_every_scale_byte_and_code():
+    """All 256 E8M0 bytes x all 16 codes: the bytes whose power of two is an
+    fp16 value take one f16x2 multiply, the others the fp32 path."""
+    codes = np.tile(np.array([0x10, 0x32, 0x54, 0x76, 0x98, 0xBA, 0xDC, 0xFE] * 2, dtype=np.uint8), 256)
+    p = synth.Packed(synth.FMT_MXFP4, 256, 32, codes, np.arange(256, dtype=np.uint8))
+    got = _deq(dev(p))
+    exp = oracle.dequant(p.fmt, p.n, p.k, p.data, p.scales)
+    assert nan_class_equal(got, exp)

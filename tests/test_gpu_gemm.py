@@ -24,7 +24,7 @@ def run_gemm(w, x_bits, canary=64):
 
 
 @pytest.mark.parametrize("variant", ["persistent", "tile"])
-@pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3])
+@pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3, synth.FMT_MXFP4])
 @pytest.mark.parametrize("m,n,k", [(128, 256, 64), (128, 256, 256), (256, 384, 512), (200, 300, 1024),
                                    (64, 128, 128), (384, 1000, 2048), (2560, 2048, 64), (2048, 2560, 256)])
 def test_gemm_vs_oracle(variant, fmt, m, n, k, monkeypatch):
@@ -34,14 +34,18 @@ def test_gemm_vs_oracle(variant, fmt, m, n, k, monkeypatch):
     x = synth.gen_x(rng, m, k)
     y = run_gemm(dev(p), x)
     v = qmm.qmm_last_variant()
-    # the persistent kernel stages packed weights in 256-wide k chunks
-    want = "gemm_fp4_tc_persistent" if (variant == "persistent" and k % 256 == 0) else "gemm_fp4_tc<"
+    # the persistent kernel stages packed weights in 256-wide k chunks; MXFP4
+    # has only that tensor-core kernel (other k: the decode kernel per row block)
+    if fmt == synth.FMT_MXFP4:
+        want = "gemm_fp4_tc_persistent" if (variant == "persistent" and k % 256 == 0) else "gemm_by_gemv"
+    else:
+        want = "gemm_fp4_tc_persistent" if (variant == "persistent" and k % 256 == 0) else "gemm_fp4_tc<"
     assert v.startswith(want), v
     yref, absy = oracle.matmul(fmt, n, k, p.data, p.scales, p.global_scale, x)
     check_tol(y, yref, absy, "gemm m=%d n=%d k=%d" % (m, n, k))
 
 
-@pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3])
+@pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3, synth.FMT_MXFP4])
 def test_gemm_identity_rows_give_decoded_weights(fmt):
     """X = [I | 0]: row i of Y is column i of the decoded W, bit-exactly."""
     rng = np.random.default_rng(9)
@@ -92,3 +96,19 @@ def test_config5_prefill_full_size_sampled(fmt):
     check_tol(y[np.arange(2048), col], ys, as_, "prefill last column")
     y2 = run_gemm(w, x)
     assert np.array_equal(y, y2)  # deterministic
+
+
+def test_gemm_mxfp4_small_and_normal_scales():
+    """The tensor-core decode of MXFP4 groups through f16x2 (E8M0 103..142)
+    and through fp32 (0..102) in one tile."""
+    rng = np.random.default_rng(31)
+    m, n, k = 256, 512, 1024
+    p = synth.gen_fp4(rng, n, k, synth.FMT_MXFP4)
+    sc = p.scales.copy()
+    sc[::5] = rng.integers(0, 131, size=sc[::5].size)
+    p = synth.Packed(p.fmt, n, k, p.data, sc)
+    x = synth.gen_x(rng, m, k)
+    y = run_gemm(dev(p), x)
+    assert qmm.qmm_last_variant().startswith("gemm_fp4_tc_persistent<fmt=4")
+    yref, absy = oracle.matmul(p.fmt, n, k, p.data, p.scales, 1.0, x)
+    check_tol(y, yref, absy, "gemm mxfp4 scales")

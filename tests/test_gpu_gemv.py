@@ -5,12 +5,12 @@ import pytest
 import torch
 
 import oracle
-from gpu_util import check_tol, dev, from_dev_u16, nz, run_gemv, to_dev_u16
+from gpu_util import check_tol, dev, f16, from_dev_u16, nz, run_gemv, to_dev_u16
 from packed_bit_weight_b200 import qmm, synth
 
 pytestmark = pytest.mark.gpu
 
-FMTS = [synth.FMT_IQ4_NL, synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3]
+FMTS = [synth.FMT_IQ4_NL, synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3, synth.FMT_MXFP4]
 
 
 def _case(fmt, n, k, m, seed):
@@ -157,3 +157,51 @@ def test_dual_tile_kernel_ragged(fmt, n, k, m, monkeypatch):
     assert v.startswith("gemv_fp4_dual"), v
     yref, absy = oracle.matmul(fmt, n, k, p.data, p.scales, p.global_scale, x)
     check_tol(y, yref, absy, v)
+
+
+@pytest.mark.parametrize("variant", [None, "generic"])
+@pytest.mark.parametrize("m", [1, 5, 16])
+def test_mxfp4_small_and_normal_scales(variant, m, monkeypatch):
+    """MXFP4 groups scaled by one f16x2 multiply (E8M0 103..142) and groups
+    scaled through fp32 (0..102: subnormal and zero weights) in the same
+    warp."""
+    if variant:
+        monkeypatch.setenv("QMM_GEMV_VARIANT", variant)
+    rng = np.random.default_rng(77 + m)
+    n, k = 96, 4096
+    p = synth.gen_fp4(rng, n, k, synth.FMT_MXFP4)
+    sc = p.scales.copy()
+    sc[::7] = rng.integers(0, 131, size=sc[::7].size)
+    sc[:103] = np.arange(103)
+    p = synth.Packed(p.fmt, n, k, p.data, sc)
+    x = synth.gen_x(rng, m, k)
+    y = run_gemv(dev(p), x)
+    v = qmm.qmm_last_variant()
+    assert v.startswith("gemv_generic" if variant else "gemv_fp4_ldg"), v
+    yref, absy = oracle.matmul(p.fmt, n, k, p.data, p.scales, 1.0, x)
+    check_tol(y, yref, absy, v)
+
+
+@pytest.mark.parametrize("variant", [None, "generic"])
+def test_mxfp4_huge_scales_overflow_like_the_oracle(variant, monkeypatch):
+    """E8M0 bytes 143..254 turn codes >= 1 into fp16 infinities; 0xFF is NaN.
+    The outputs of those rows are infinite or NaN exactly where the oracle's
+    are, with the same sign."""
+    if variant:
+        monkeypatch.setenv("QMM_GEMV_VARIANT", variant)
+    rng = np.random.default_rng(5)
+    n, k, m = 32, 512, 2
+    p = synth.gen_fp4(rng, n, k, synth.FMT_MXFP4)
+    sc = p.scales.copy().reshape(n, k // 32)
+    sc[0:8, 3] = [143, 150, 160, 180, 200, 220, 240, 254]   # one huge group in rows 0..7
+    sc[8, :] = 0xFF                            # a NaN row
+    p = synth.Packed(p.fmt, n, k, p.data, sc.reshape(-1))
+    x = synth.gen_x(rng, m, k)
+    y = f16(run_gemv(dev(p), x))
+    with np.errstate(all="ignore"):
+        yref, _ = oracle.matmul(p.fmt, n, k, p.data, p.scales, 1.0, x)
+    big = ~np.isfinite(yref)
+    assert big[:, :9].all() and not big[:, 9:].any()
+    assert np.array_equal(np.isnan(y[big]), np.isnan(yref[big]))
+    nn = big & ~np.isnan(yref)
+    assert np.array_equal(y[nn], yref[nn])      # +-inf, same sign

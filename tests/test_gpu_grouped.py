@@ -55,7 +55,7 @@ def _grouped(w, x_bits, ids, x_per_pair):
     return from_dev_u16(y), st
 
 
-@pytest.mark.parametrize("fmt", [synth.FMT_IQ4_NL, synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3])
+@pytest.mark.parametrize("fmt", [synth.FMT_IQ4_NL, synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3, synth.FMT_MXFP4])
 @pytest.mark.parametrize("E,n,k,t,topk,per_pair", [(6, 40, 64, 9, 2, False), (4, 33, 256, 70, 3, True),
                                                     (8, 128, 512, 3, 4, False)])
 def test_grouped_vs_oracle(fmt, E, n, k, t, topk, per_pair):
