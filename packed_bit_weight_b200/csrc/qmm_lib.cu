@@ -21,6 +21,7 @@
 #include "k_grouped.cuh"
 #include "k_gemv_ring.cuh"
 #include "k_iq4p.cuh"
+#include "k_iq4w.cuh"
 #include "k_moe.cuh"
 
 namespace qmm {
@@ -372,8 +373,15 @@ static int gemv_variant_env() {
   if (!strcmp(v, "iq4p")) return 6;
   if (!strcmp(v, "ring")) return 7;
   if (!strcmp(v, "dual")) return 8;
+  if (!strcmp(v, "iq4w")) return 9;
   return 0;
 }
+
+// Warp-per-tile IQ4_NL kernel (k_iq4w.cuh); UNSUPPORTED_SHAPE launches nothing.
+template <int MODE>
+static qmm_status launch_iq4_warp(const qmm_weights* w0, const qmm_weights* w1, const uint16_t* x, int x_per_pair,
+                                  int64_t topk, const int32_t* offsets, const int32_t* perm, int m_plain, void* y,
+                                  const float* gw, cudaStream_t st, const DevInfo* di);
 
 // Persistent IQ4_NL kernel (k_iq4p.cuh).  Returns QMM_ERR_UNSUPPORTED_SHAPE,
 // having launched nothing, when the shape is outside what it takes.
@@ -483,6 +491,10 @@ static qmm_status gemv_fmt(const qmm_weights* w, const uint16_t* x, int m, uint1
       if (m <= 8) return launch_gemv_tma<FMT, 1, 1>(w, x, m, y, st, di);
       return launch_gemv_tma<FMT, 1, 2>(w, x, m, y, st, di);
     }
+  }
+  if (FMT == 1 && pick == 9) {
+    const qmm_status s = launch_iq4_warp<IQ_OUT_F16>(w, nullptr, x, 0, 1, nullptr, nullptr, m, y, nullptr, st, di);
+    if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
   }
   if (FMT == 1 && pick == 6) {  // persistent kernel: measured slower than the streaming one, kept selectable
     const qmm_status s = launch_iq4_persist<IQ_OUT_F16>(w, nullptr, x, 0, 1, nullptr, 0, m, y, nullptr, st, di);
@@ -598,6 +610,46 @@ static qmm_status launch_iq4_mode(const qmm_weights* w, const qmm_weights* w2, c
       static_cast<const uint8_t*>(w->data), w->expert_data_stride,
       w2 ? static_cast<const uint8_t*>(w2->data) : nullptr, w2 ? w2->expert_data_stride : 0, x, x_per_pair,
       (int)topk, offsets, perm, m_plain, y, gw, (int)w->n, (int)w->k, (int)w->num_experts, pf);
+  return launch_status();
+}
+
+// Warp-per-tile IQ4_NL kernel (k_iq4w.cuh): persistent, two CTAs of 8 warps
+// per SM, items from the routing sort (offsets/perm) or the plain product.
+template <int MODE>
+static qmm_status launch_iq4_warp(const qmm_weights* w0, const qmm_weights* w1, const uint16_t* x, int x_per_pair,
+                                  int64_t topk, const int32_t* offsets, const int32_t* perm, int m_plain, void* y,
+                                  const float* gw, cudaStream_t st, const DevInfo* di) {
+  const int64_t n = w0->n, k = w0->k;
+  if (w0->fmt != QMM_FMT_IQ4_NL || (w1 && w1->fmt != QMM_FMT_IQ4_NL)) return QMM_ERR_UNSUPPORTED_SHAPE;
+  if (k % 128 || k < 128 || n < 1 || n > INT32_MAX / 2 || k > INT32_MAX / 2) return QMM_ERR_UNSUPPORTED_SHAPE;
+  if (offsets && w0->num_experts > kIqwMaxExperts) return QMM_ERR_UNSUPPORTED_SHAPE;
+  const size_t smem = kIqLutBytes;
+  if (cudaFuncSetAttribute(iq4_warp_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return QMM_ERR_CUDA;
+  int64_t grid = 2 * (int64_t)di->sms;
+  if (!offsets) {
+    const int64_t items = ((n + 15) / 16) * ((m_plain + 15) / 16);
+    grid = std::min<int64_t>(grid, (items + kIqwWarps - 1) / kIqwWarps);
+  }
+  IqwArgs a;
+  a.data0 = static_cast<const uint8_t*>(w0->data);
+  a.data1 = w1 ? static_cast<const uint8_t*>(w1->data) : nullptr;
+  a.dstride0 = w0->expert_data_stride;
+  a.dstride1 = w1 ? w1->expert_data_stride : 0;
+  a.x = x;
+  a.x_per_pair = x_per_pair;
+  a.topk = (int)topk;
+  a.offsets = offsets;
+  a.perm = perm;
+  a.m_plain = m_plain;
+  a.y = y;
+  a.gw = gw;
+  a.n = (int)n;
+  a.k = (int)k;
+  a.E = offsets ? (int)w0->num_experts : 1;
+  iq4_warp_kernel<MODE><<<(unsigned)std::max<int64_t>(grid, 1), kIqwWarps * 32, smem, st>>>(a);
+  set_variant("iq4_warp<mode=%d,grid=%d>", MODE, (int)grid);
   return launch_status();
 }
 
@@ -918,6 +970,13 @@ qmm_status qmm_grouped_gemv(const qmm_weights* experts, const uint16_t* x, int32
     set_variant("route+zero_fill");
     return launch_status();
   }
+  if (experts->fmt == QMM_FMT_IQ4_NL && pick == 9) {
+    s = launch_iq4_warp<IQ_OUT_F16>(experts, nullptr, x, x_per_pair, topk, offsets, perm, 0, y, nullptr, st, di);
+    if (s != QMM_ERR_UNSUPPORTED_SHAPE) {
+      set_variant("route+grouped_iq4_warp");
+      return s;
+    }
+  }
   if (experts->fmt == QMM_FMT_IQ4_NL && experts->k % 128 == 0 && (pick == 0 || pick == 5)) {
     s = launch_iq4_stream(experts, x, x_per_pair, topk, offsets, perm, 0, y, st, di);
     set_variant("route+grouped_iq4_stream");
@@ -1055,6 +1114,18 @@ qmm_status qmm_moe_routed(const qmm_weights* gate, const qmm_weights* up, const 
     zero_fill_kernel<<<grid_for(t * d, 256, di->sms), 256, 0, st>>>(out, t * d);
     set_variant("moe:route+zero_fill");
     return launch_status();
+  }
+  if (gemv_variant_env() == 9) {  // warp-per-tile kernels
+    s = launch_iq4_warp<IQ_SWIGLU>(gate, up, x, 0, topk, offsets, perm, 0, h, nullptr, st, di);
+    if (s == QMM_OK)
+      s = launch_iq4_warp<IQ_SCALED_F32>(down, nullptr, h, 1, topk, offsets, perm, 0, yg, topk_weights, st, di);
+    if (s == QMM_OK) {
+      combine_kernel<<<grid_for(t * (d / 8), 256, di->sms), 256, 0, st>>>(yg, topk_ids, (int)E, (int)t, (int)topk,
+                                                                           (int)d, out);
+      set_variant("moe:route+gate_up_swiglu_iq4_warp+down_scaled_iq4_warp+combine");
+      return launch_status();
+    }
+    if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
   }
   if ((s = launch_iq4_mode<IQ_SWIGLU>(gate, up, x, 0, topk, offsets, perm, 0, h, nullptr, st, di)) != QMM_OK)
     return s;

@@ -108,7 +108,7 @@ def test_grouped_rejects_small_workspace():
     assert e.value.status == 8
 
 
-@pytest.mark.parametrize("variant", [None, "iq4p"])
+@pytest.mark.parametrize("variant", [None, "iq4p", "iq4w"])
 @pytest.mark.parametrize("E,n,k,t,topk,per_pair", [(3, 64, 256, 50, 2, False), (5, 48, 384, 200, 3, True),
                                                     (2, 16, 128, 2100, 2, False), (32, 32, 128, 1, 4, True)])
 def test_grouped_iq4_many_pairs_per_expert(variant, E, n, k, t, topk, per_pair, monkeypatch):
@@ -128,6 +128,8 @@ def test_grouped_iq4_many_pairs_per_expert(variant, E, n, k, t, topk, per_pair, 
     assert st == 0, v
     if variant == "iq4p":
         assert v.startswith("iq4_persist" if t * topk <= 4096 else "route+grouped_gemv_generic"), v
+    elif variant == "iq4w":
+        assert v.startswith("route+grouped_iq4_warp"), v
     else:
         assert "iq4_stream" in v, v
     if per_pair:

@@ -141,7 +141,7 @@ def _moe_reference_stages(wgu, wdn, x, ids, g, f, h_gpu):
     return h_ref, h_bound, out_ref, out_abs
 
 
-@pytest.mark.parametrize("variant", [None, "iq4p"])
+@pytest.mark.parametrize("variant", [None, "iq4p", "iq4w"])
 @pytest.mark.parametrize("E,f,d,t,topk", [(6, 128, 256, 9, 2), (4, 256, 128, 40, 4), (2, 128, 384, 5, 2),
                                           (32, 896, 2560, 64, 4), (32, 896, 2560, 1, 4)])
 def test_moe_routed_vs_oracle(E, f, d, t, topk, variant, monkeypatch):
@@ -158,6 +158,7 @@ def test_moe_routed_vs_oracle(E, f, d, t, topk, variant, monkeypatch):
     out, h, st, used = _moe_gpu(wgu, wdn, x, ids, g, f)
     assert st == 0, used
     assert ("iq4_persist" in used) == (variant == "iq4p"), used
+    assert ("iq4_warp" in used) == (variant == "iq4w"), used
     variant = used
     h_ref, h_bound, out_ref, out_abs = _moe_reference_stages(wgu, wdn, x, ids, g, f, h)
     err = np.abs(f16(h) - h_ref)
