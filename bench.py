@@ -298,8 +298,9 @@ def gemm_workload(fmt, world, l2, peaks):
     base = qmm.PackedWeights.from_host(p)
     xd0 = torch.from_numpy(x.view(np.int16)).cuda()
     R = max(2, math.ceil(1.5 * l2 / (base.nbytes + xd0.numel() * 2)))
-    ws = [base] + [qmm.PackedWeights(base.fmt, base.n, base.k, base.data.clone(), base.scales.clone(),
-                                     base.global_scale) for _ in range(R - 1)]
+    ws = [base] + [qmm.PackedWeights(base.fmt, base.n, base.k, base.data.clone(),
+                                     None if base.scales is None else base.scales.clone(), base.global_scale)
+                   for _ in range(R - 1)]
     xs = [xd0] + [xd0.clone() for _ in range(R - 1)]
     y = torch.empty((p.k and x.shape[0], p.n), dtype=torch.int16, device="cuda")
 
@@ -438,6 +439,7 @@ def extra_workloads(args, world, l2, peaks):
     out["fp4g16_prefill_gemm_2048x18560x4096"] = gemm_workload(synth.FMT_FP4G16_F16, world, l2, peaks)
     out["fp4g16_e4m3_prefill_gemm_2048x18560x4096"] = gemm_workload(synth.FMT_FP4G16_E4M3, world, l2, peaks)
     out["mxfp4_prefill_gemm_2048x18560x4096"] = gemm_workload(synth.FMT_MXFP4, world, l2, peaks)
+    out["iq4nl_prefill_gemm_2048x18560x4096"] = gemm_workload(synth.FMT_IQ4_NL, world, l2, peaks)
     out["iq4nl_grouped_experts_t64_top4"] = grouped_workload(world, l2, peaks)
     out["iq4nl_moe_block_t64_top4"] = moe_workload(world, l2, peaks, t=64)
     out["iq4nl_moe_block_t1_top4"] = moe_workload(world, l2, peaks, t=1)

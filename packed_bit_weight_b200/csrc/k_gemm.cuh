@@ -332,6 +332,38 @@ constexpr int kStageCodes = 256 * 128;
 constexpr int kStageScales = 256 * 32;
 constexpr int kStageBytes = kStageCodes + kStageScales;
 
+// IQ4_NL ("Mark-Experimental-V3-8B", section "Quantization": 18-byte blocks
+// per 32 weights, fp16 d then 16 bytes of indices into the printed table):
+// a 256-k chunk of a row is 8 blocks = 144 bytes, copied as 9 units into
+// [256][144 B]; the 4 KB after them in staging slot 0 hold a 256-entry table
+// of exact f16x2 pairs (kv[i & 15], kv[i >> 4]) in 4 bank-interleaved copies
+// (copy c of entry i at word 4i + c; a thread reads copy lane & 3).
+constexpr int kStageIq4Row = 144;
+constexpr int kStageIq4Lut = 256 * kStageIq4Row;  // 36,864: table offset inside slot 0
+static_assert(kStageIq4Lut + 256 * 4 * 4 <= kStageBytes, "IQ4_NL table fits in the staging slot");
+
+// Decode the 16 index bytes Q[0..3] of one IQ4_NL block (scale dd, f16x2
+// broadcast) into its 32 weights as four 8-weight chunks in k order: chunk 0
+// = low nibbles of bytes 0..7 (weights 0..7), 1 = low of 8..15, 2 = high of
+// 0..7 (weights 16..23), 3 = high of 8..15.  Two adjacent nibbles of the same
+// kind form one table index, so each lookup yields two consecutive weights,
+// exact; one f16x2 multiply by d rounds each once.
+__device__ __forceinline__ void iq4_block_chunks(const uint32_t (&Q)[4], uint32_t dd, uint32_t lut_copy,
+                                                 uint32_t (&out)[16]) {
+#pragma unroll
+  for (int i = 0; i < 4; i++) {
+    const uint32_t lo = Q[i] & 0x0F0F0F0Fu, hi = (Q[i] >> 4) & 0x0F0F0F0Fu;
+    const uint32_t ul = lo | (lo >> 4), uh = hi | (hi >> 4);  // bytes 0 and 2: (n0 | n1 << 4), (n2 | n3 << 4)
+    const uint32_t l0 = lds32(lut_copy + ((ul & 0xFFu) << 4)), l1 = lds32(lut_copy + (((ul >> 16) & 0xFFu) << 4));
+    const uint32_t h0 = lds32(lut_copy + ((uh & 0xFFu) << 4)), h1 = lds32(lut_copy + (((uh >> 16) & 0xFFu) << 4));
+    // bytes 4i..4i+3: low nibbles are weights 4i..4i+3, high ones 16+4i..
+    out[(i >> 1) * 4 + (i & 1) * 2] = hmul2(l0, dd);
+    out[(i >> 1) * 4 + (i & 1) * 2 + 1] = hmul2(l1, dd);
+    out[8 + (i >> 1) * 4 + (i & 1) * 2] = hmul2(h0, dd);
+    out[8 + (i >> 1) * 4 + (i & 1) * 2 + 1] = hmul2(h1, dd);
+  }
+}
+
 __device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint32_t bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
@@ -381,6 +413,14 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
   if (warp == 1) {
     tmem_alloc(tmem_slot, 2 * BN);
     tmem_relinquish();
+  }
+  if (FMT == 1) {  // IQ4_NL pair table, 4 interleaved copies, in staging slot 0's spare tail
+    for (int i = threadIdx.x; i < 256 * 4; i += blockDim.x) {
+      const int v = i >> 2;
+      const uint32_t lo = __half_as_ushort(__int2half_rn(c_iq4nl_kv[v & 15]));
+      const uint32_t hi = __half_as_ushort(__int2half_rn(c_iq4nl_kv[v >> 4]));
+      asm volatile("st.shared.u32 [%0], %1;" ::"r"(p_s + kStageIq4Lut + 4u * i), "r"(lo | (hi << 16)) : "memory");
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -456,6 +496,18 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
       const int n0 = (tile % n_tiles) * BN;
       const int kc = (c % nck) * (kGemmChunkSteps * kGemmBK);  // first k of the chunk
       const uint32_t dst = p_s + slot * kStageBytes;
+      if (FMT == 1) {  // IQ4_NL: 256 rows x 9 units of 16 bytes (8 blocks of 18 bytes)
+        const int64_t rowb = (int64_t)(k >> 5) * 18;
+#pragma unroll
+        for (int i = 0; i < 9; i++) {
+          const int pc = i * kGemmDecodeThreads + t;
+          const int r = pc / 9, u = pc - r * 9;
+          const int64_t gr = min((int64_t)n0 + r, (int64_t)n - 1);
+          cp_async16_g(dst + r * kStageIq4Row + u * 16, codes + gr * rowb + (int64_t)(kc >> 5) * 18 + u * 16);
+        }
+        cp_async_mbar_arrive_noinc(cfull + 8 * slot);
+        return true;
+      }
 #pragma unroll
       for (int i = 0; i < 8; i++) {  // codes: 256 rows x 8 units of 16 bytes
         const int pc = i * kGemmDecodeThreads + t;
@@ -496,6 +548,37 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
       for (int j = 0; j < kGemmChunkSteps; j++, gs++) {
         const int s = gs % STAGES;
         const uint32_t ph = (uint32_t)(gs / STAGES) & 1u;
+        if (FMT == 1) {
+          // this row's two blocks of step j: 36 bytes from byte 36j of the row
+          uint32_t w[9];
+#pragma unroll
+          for (int i = 0; i < 9; i++) w[i] = lds32(src + t * kStageIq4Row + j * 36 + 4 * i);
+          uint32_t qa[4], qb[4];
+#pragma unroll
+          for (int i = 0; i < 4; i++) {
+            qa[i] = __funnelshift_r(w[i], w[i + 1], 16);  // block 0: index bytes 2..17 of the 36
+            qb[i] = w[5 + i];                              // block 1: bytes 20..35
+          }
+          uint32_t da = w[0] & 0xFFFFu, db = w[4] >> 16;
+          da = valid ? (da | (da << 16)) : 0u;
+          db = valid ? (db | (db << 16)) : 0u;
+          if (s_abort || !mbar_wait(bars + 8 * (STAGES + s), ph ^ 1u)) { s_abort = 1; stop = true; break; }
+          const uint32_t lut_copy = p_s + kStageIq4Lut + 4u * (uint32_t)(t & 3);
+          const uint32_t row_base = b_s + s * C::kBBytes + (uint32_t)t * 128u;
+          const uint32_t swz = (uint32_t)(t & 7);
+          uint32_t o[16];
+          iq4_block_chunks(qa, da, lut_copy, o);
+#pragma unroll
+          for (int cc = 0; cc < 4; cc++)
+            sts128(row_base + ((cc ^ swz) << 4), o[4 * cc], o[4 * cc + 1], o[4 * cc + 2], o[4 * cc + 3]);
+          iq4_block_chunks(qb, db, lut_copy, o);
+#pragma unroll
+          for (int cc = 0; cc < 4; cc++)
+            sts128(row_base + (((cc + 4) ^ swz) << 4), o[4 * cc], o[4 * cc + 1], o[4 * cc + 2], o[4 * cc + 3]);
+          fence_proxy_async_shared();
+          mbar_arrive(bars + 8 * s);
+          continue;
+        }
         // this row's 32 code bytes (units 2j, 2j+1) and 4 scales of step j
         const uint4 c0 = lds128(src + t * 128 + (((2 * j) ^ (t & 7)) << 4));
         const uint4 c1 = lds128(src + t * 128 + (((2 * j + 1) ^ (t & 7)) << 4));

@@ -882,13 +882,15 @@ qmm_status qmm_gemm(const qmm_weights* w, const uint16_t* x, int64_t m, uint16_t
   if (!aligned16(y) || (x && !aligned16(x))) return QMM_ERR_MISALIGNED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (w->k == 0) return zero_output(y, m * w->n, st, di);
-  const bool tc = w->fmt != QMM_FMT_IQ4_NL && w->k % kGemmBK == 0 && m >= 64;
+  const bool tc = w->k % kGemmBK == 0 && m >= 64;
   // persistent kernel when k is a multiple of its 256-wide staging chunk;
   // QMM_GEMM_VARIANT=tile selects the one-tile-per-CTA kernel (measurements)
   const char* gv = getenv("QMM_GEMM_VARIANT");
   const bool persist = !(gv && !strcmp(gv, "tile")) && w->k % (kGemmChunkSteps * kGemmBK) == 0;
   switch (w->fmt) {
-    case QMM_FMT_IQ4_NL: return gemm_by_gemv<1>(w, x, m, y, st, di);
+    case QMM_FMT_IQ4_NL:  // the persistent kernel only (256-wide staging chunk = 8 blocks = 144 bytes a row)
+      if (!tc || !persist) return gemm_by_gemv<1>(w, x, m, y, st, di);
+      return launch_gemm_tc_persistent<1>(w, x, (int)m, y, st, di);
     case QMM_FMT_FP4G16_F16:
       if (!tc) return gemm_by_gemv<2>(w, x, m, y, st, di);
       return persist ? launch_gemm_tc_persistent<2>(w, x, (int)m, y, st, di) : launch_gemm_tc<2>(w, x, (int)m, y, st, di);

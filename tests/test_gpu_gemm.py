@@ -112,3 +112,38 @@ def test_gemm_mxfp4_small_and_normal_scales():
     assert qmm.qmm_last_variant().startswith("gemm_fp4_tc_persistent<fmt=4")
     yref, absy = oracle.matmul(p.fmt, n, k, p.data, p.scales, 1.0, x)
     check_tol(y, yref, absy, "gemm mxfp4 scales")
+
+
+@pytest.mark.parametrize("m,n,k", [(128, 256, 256), (200, 300, 1024), (384, 1000, 2048), (64, 17, 512),
+                                   (2048, 1792, 2560), (256, 512, 384)])
+def test_gemm_iq4nl_tensor_cores(m, n, k):
+    """IQ4_NL prefill on the persistent tcgen05 kernel (k % 256 == 0; other k
+    take the decode kernel per 16-row slice): ragged m and n tiles, one
+    routed expert's gate+up shape."""
+    rng = np.random.default_rng(600 + m + n + k)
+    p = synth.gen_iq4nl(rng, n, k)
+    x = synth.gen_x(rng, m, k)
+    y = run_gemm(dev(p), x)
+    v = qmm.qmm_last_variant()
+    assert v.startswith("gemm_fp4_tc_persistent<fmt=1" if k % 256 == 0 else "gemm_by_gemv"), v
+    if m * n * k > 2 ** 31:
+        rows = rng.integers(0, m, 48)
+        cols = rng.integers(0, n, 48)
+        ys, as_ = oracle.matmul_sampled(p.fmt, n, k, p.data, None, 1.0, x, rows, cols)
+        check_tol(y[rows, cols], ys, as_, v)
+    else:
+        yref, absy = oracle.matmul(p.fmt, n, k, p.data, None, 1.0, x)
+        check_tol(y, yref, absy, v)
+
+
+def test_gemm_iq4nl_identity_rows_give_decoded_weights():
+    """X = [I | 0]: row i of Y is column i of the decoded IQ4_NL W, bit-exactly."""
+    rng = np.random.default_rng(10)
+    m, n, k = 128, 512, 256
+    p = synth.gen_iq4nl(rng, n, k)
+    x = np.zeros((m, k), dtype=np.uint16)
+    x[np.arange(m), np.arange(m)] = 0x3C00
+    y = run_gemm(dev(p), x)
+    assert qmm.qmm_last_variant().startswith("gemm_fp4_tc_persistent<fmt=1")
+    deq = oracle.dequant(p.fmt, n, k, p.data, None)
+    assert np.array_equal(nz(y), nz(deq[:, :m].T))
