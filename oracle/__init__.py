@@ -13,6 +13,6 @@ Parity status of each function is stated in ``PINS`` below.
 from .oracle import (  # noqa: F401
     FMT_IQ4_NL, FMT_FP4G16_F16, FMT_FP4G16_E4M3, FMT_MXFP4, PINS, build, lib,
     f16_to_f64, f64_to_f16, e4m3_to_f64, e8m0_to_f64, e2m1_to_f64, iq4nl_value,
-    data_bytes, scale_bytes, dequant, dequant_row, matmul, matmul_sampled,
+    data_bytes, scale_bytes, dequant, dequant_row, quantize, matmul, matmul_sampled,
     route, grouped_gemv, router_topk, silu, swiglu, combine,
 )

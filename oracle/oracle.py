@@ -44,6 +44,9 @@ PINS = {
                    "(tests/test_oracle_moe.py)",
     "silu/swiglu": "closed forms: silu(0)=0, silu(ln 3)=0.75 ln 3, odd/even split, limits (tests/test_oracle_moe.py)",
     "combine": "linearity and the one-slot special case (tests/test_oracle_moe.py)",
+    "quantize": "exact recovery of codes from power-of-two scaled weights, hand-written rows "
+                "(tests/golden/quantize_handmade.txt), error bound, optimality against numpy-rounded "
+                "candidates (tests/test_oracle_quantize.py); the scale choice itself is parity unpinned",
 }
 
 
@@ -84,6 +87,7 @@ def lib():
         L.orc_dequant_row.argtypes = [i32, i64, i64, vp, vp, f32, i64, vp]
         L.orc_dequant.argtypes = [i32, i64, i64, vp, vp, f32, vp]
         L.orc_matmul.argtypes = [i32, i64, i64, vp, vp, f32, vp, i64, vp, vp]
+        L.orc_quantize.argtypes = [i32, i64, i64, vp, vp, vp]
         L.orc_matmul_sampled.argtypes = [i32, i64, i64, vp, vp, f32, vp, i64, vp, vp, i64, vp, vp]
         L.orc_route.argtypes = [vp, i64, i64, i64, vp, vp]
         L.orc_route.restype = i64
@@ -157,6 +161,21 @@ def dequant_row(fmt, n, k, data, scales, global_scale, row):
 
 
 # -- products --------------------------------------------------------------------
+def quantize(fmt, n, k, w_bits):
+    """fp16 weights [n][k] (bit patterns) -> (data, scales) packed bytes:
+    FP4G16_F16 (fp16 scale amax/6), MXFP4 (E8M0 exponent floor(log2 amax) - 2)
+    or IQ4_NL (d = m / -127); each weight the nearest decoded value, ties to
+    the lowest code."""
+    if fmt not in (FMT_FP4G16_F16, FMT_MXFP4, FMT_IQ4_NL):
+        raise ValueError("no encoder for this format")
+    w_bits = _c(w_bits, np.uint16).reshape(n, k)
+    data = np.zeros(data_bytes(fmt, n, k), dtype=np.uint8)
+    sb = scale_bytes(fmt, n, k)
+    scales = np.zeros(max(sb, 1), dtype=np.uint8)
+    lib().orc_quantize(fmt, n, k, _p(w_bits), _p(data), _p(scales))
+    return data, (scales[:sb] if sb else None)
+
+
 def matmul(fmt, n, k, data, scales, global_scale, x_bits):
     """(y, absy): y[m][n] = sum_k w16[n][k] x[m][k] in double, absy = sum |w x|."""
     data = _c(data, np.uint8)

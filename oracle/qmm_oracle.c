@@ -239,6 +239,94 @@ void orc_dequant(int fmt, int64_t n, int64_t k, const uint8_t* data, const uint8
 }
 
 /* ---------------------------------------------------------------------- */
+/* Encoders: fp16 weights -> packed bytes.  The pages fix the formats but   */
+/* not the quantiser; the readings below take the plainest choice of scale */
+/* and then the nearest representable weight ("parity unpinned" for the   */
+/* scale choice; the nearest-value step is pinned by the tests).           */
+/*   FP4-G16 (fp16 scale): s = fp16(amax / 6) per group of 16, amax = the  */
+/*     largest |w| of the group (6 = the largest E2M1 magnitude).           */
+/*   MXFP4: e = floor(log2(amax)) - 2 + 127 clamped to [0, 254] (the OCP MX */
+/*     shared exponent; 2 = the E2M1 maximum's exponent), e = 0 for amax = 0.*/
+/*   IQ4_NL: d = fp16(m / -127), m the first element of largest |w| of the  */
+/*     block, so that it maps to the table's -127 entry.                    */
+/* Then each weight takes the code whose decoded value (exactly as the      */
+/* decoders define it) is nearest; on equal distance the lowest code (FP4:  */
+/* 0..7 are +0, 0.5, .. 6, 8..15 their negatives; IQ4_NL: table order).     */
+/* A NaN weight takes code 0.                                               */
+/* ---------------------------------------------------------------------- */
+static int orc_nearest_code(double w, const double* cand, int ncand) {
+  int best = 0;
+  double be = fabs(w - cand[0]);
+  for (int i = 1; i < ncand; i++) {
+    double e = fabs(w - cand[i]);
+    if (e < be) { be = e; best = i; }
+  }
+  return best;
+}
+
+/* w [n][k] fp16 bits -> data (codes or blocks) and scales, in the layouts of
+ * orc_dequant_row.  fmt: FP4G16_F16, MXFP4 or IQ4_NL (E4M3 is not encoded). */
+void orc_quantize(int fmt, int64_t n, int64_t k, const uint16_t* w, uint8_t* data, uint8_t* scales) {
+  double cand[16];
+  for (int64_t r = 0; r < n; r++) {
+    const uint16_t* wr = w + r * k;
+    if (fmt == ORC_FMT_IQ4_NL) {
+      for (int64_t b = 0; b < k / 32; b++) {
+        double m = 0.0, am = 0.0;
+        for (int j = 0; j < 32; j++) {
+          double v = orc_f16_to_f64(wr[b * 32 + j]);
+          if (fabs(v) > am) { am = fabs(v); m = v; }
+        }
+        uint16_t dbits = orc_f64_to_f16(m / -127.0);
+        double d = orc_f16_to_f64(dbits);
+        for (int i = 0; i < 16; i++) cand[i] = orc_f16_to_f64(orc_f64_to_f16(d * (double)orc_iq4nl_table[i]));
+        uint8_t* blk = data + (r * (k / 32) + b) * 18;
+        blk[0] = (uint8_t)(dbits & 0xFF);
+        blk[1] = (uint8_t)(dbits >> 8);
+        for (int j = 0; j < 16; j++) {
+          int lo = orc_nearest_code(orc_f16_to_f64(wr[b * 32 + j]), cand, 16);
+          int hi = orc_nearest_code(orc_f16_to_f64(wr[b * 32 + j + 16]), cand, 16);
+          blk[2 + j] = (uint8_t)(lo | (hi << 4));
+        }
+      }
+      continue;
+    }
+    const int g = (fmt == ORC_FMT_MXFP4) ? 32 : 16;
+    for (int64_t q = 0; q < k / g; q++) {
+      double am = 0.0;
+      for (int j = 0; j < g; j++) {
+        double v = fabs(orc_f16_to_f64(wr[q * g + j]));
+        if (v > am) am = v;
+      }
+      double sc;
+      if (fmt == ORC_FMT_MXFP4) {
+        int e = 0;
+        if (am > 0.0) {
+          int ex;
+          frexp(am, &ex); /* am = fr * 2^ex, fr in [0.5, 1): floor(log2(am)) = ex - 1 */
+          e = ex - 1 - 2 + 127;
+          if (e < 0) e = 0;
+          if (e > 254) e = 254;
+        }
+        scales[r * (k / 32) + q] = (uint8_t)e;
+        sc = orc_e8m0_to_f64((uint8_t)e);
+      } else {
+        uint16_t sbits = orc_f64_to_f16(am / 6.0);
+        scales[(r * (k / 16) + q) * 2] = (uint8_t)(sbits & 0xFF);
+        scales[(r * (k / 16) + q) * 2 + 1] = (uint8_t)(sbits >> 8);
+        sc = orc_f16_to_f64(sbits);
+      }
+      for (int c = 0; c < 16; c++) cand[c] = orc_f16_to_f64(orc_f64_to_f16(orc_e2m1_to_f64((uint8_t)c) * sc));
+      for (int j = 0; j < g; j += 2) {
+        int c0 = orc_nearest_code(orc_f16_to_f64(wr[q * g + j]), cand, 16);
+        int c1 = orc_nearest_code(orc_f16_to_f64(wr[q * g + j + 1]), cand, 16);
+        data[r * (k / 2) + (q * g + j) / 2] = (uint8_t)(c0 | (c1 << 4));
+      }
+    }
+  }
+}
+
+/* ---------------------------------------------------------------------- */
 /* Matrix product on the decoded weights                                  */
 /* ---------------------------------------------------------------------- */
 
