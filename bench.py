@@ -389,6 +389,31 @@ def moe_workload(world, l2, peaks, t=64, topk=4):
             "note": "one step = router top-4 + routed-expert block (5 kernels); bytes = weights of the experts hit"}
 
 
+def quantize_workload(fmt, world, l2, peaks):
+    """Encode resident fp16 in_proj weights (18560 x 4096) to a packed format."""
+    import torch
+    from packed_bit_weight_b200 import qmm, synth
+    p, _ = synth.make_gemv(synth.FP4_IN_PROJ)
+    n, k = p.n, p.k
+    w0 = torch.empty((n, k), dtype=torch.int16, device="cuda")
+    qmm.qmm_dequant(qmm.PackedWeights.from_host(p), w0)
+    R = max(2, math.ceil(2 * l2 / (w0.numel() * 2)))
+    ws = [w0] + [w0.clone() for _ in range(R - 1)]
+    data = torch.empty((qmm.qmm_data_bytes(fmt, n, k),), dtype=torch.uint8, device="cuda")
+    sb = qmm.qmm_scale_bytes(fmt, n, k)
+    sc = torch.empty((max(sb, 16),), dtype=torch.uint8, device="cuda") if sb else None
+
+    def launch(i):
+        qmm.qmm_quantize(fmt, ws[i % R], data, sc)
+
+    per = timed_launches(launch, 2 * R, 5, 1, world)
+    variant = qmm.qmm_last_variant()
+    assert qmm.qmm_sync_check() == 0
+    moved = n * k * 2 + data.numel() + sb
+    return {"variant": variant, "gbs_read_plus_write": moved / per / 1e9, "frac_hbm": moved / per / 1e9 / peaks["hbm_gbs"],
+            "us_per_launch": per * 1e6, "note": "fp16 in, packed out; one thread per group, distances in fp64"}
+
+
 def dequant_workload(world, l2, peaks):
     import torch
     from packed_bit_weight_b200 import qmm, synth
@@ -444,6 +469,8 @@ def extra_workloads(args, world, l2, peaks):
     out["iq4nl_moe_block_t64_top4"] = moe_workload(world, l2, peaks, t=64)
     out["iq4nl_moe_block_t1_top4"] = moe_workload(world, l2, peaks, t=1)
     out["fp4g16_dequant_in_proj"] = dequant_workload(world, l2, peaks)
+    out["fp4g16_quantize_in_proj"] = quantize_workload(synth.FMT_FP4G16_F16, world, l2, peaks)
+    out["iq4nl_quantize_in_proj"] = quantize_workload(synth.FMT_IQ4_NL, world, l2, peaks)
     return out
 
 

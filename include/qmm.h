@@ -123,6 +123,26 @@ size_t qmm_packed_bytes(int32_t fmt, int64_t n, int64_t k);
  * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, NOT_SM100, CUDA. */
 qmm_status qmm_dequant(const qmm_weights* w, uint16_t* out, void* stream);
 
+/* Encode resident fp16 weights into a packed format (the inverse direction
+ * of qmm_dequant, for callers that hold fp16 checkpoints).  The formats are
+ * the pages' ("Mamb2_8B_FP4_Recall_SQ3.25", section "Representation";
+ * "1bit.gg zyphra", MXFP4 experts; "Mark-Experimental-V3-8B", section
+ * "Quantization"); the pages do not give the quantiser, so the scale is the
+ * plainest reading: FP4G16_F16 s = fp16(amax / 6) per 16; MXFP4 E8M0 e =
+ * floor(log2 amax) - 2 + 127 in [0, 254] per 32 (0 for an all-zero group,
+ * 254 when amax is infinite); IQ4_NL d = fp16(m / -127) per 32, m the first
+ * element of largest |w| (it maps to the table's -127 entry).  Each weight
+ * then takes the code whose decoded value (exactly as qmm_dequant decodes
+ * it) is nearest, the lowest code on equal distance, code 0 for NaN.
+ *   fmt     QMM_FMT_FP4G16_F16, QMM_FMT_MXFP4 or QMM_FMT_IQ4_NL
+ *           (FP4G16_E4M3: UNSUPPORTED_SHAPE, its global scale is matrix-wide)
+ *   w       device, [n][k] fp16 (k a multiple of the format's group)
+ *   data    device, qmm_data_bytes(fmt, n, k) bytes, written completely
+ *   scales  device, qmm_scale_bytes(fmt, n, k) bytes (NULL for IQ4_NL)
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, NOT_SM100, CUDA. */
+qmm_status qmm_quantize(int32_t fmt, const uint16_t* w, int64_t n, int64_t k, void* data, void* scales,
+                        void* stream);
+
 /* Fused dequantise-and-multiply for decode batches: y[m][n] = sum_k
  * x[m][k] * W[n][k] with the decoded fp16 weights, fp32 accumulation, one
  * rounding of the sum to fp16.  For FP4G16_E4M3 the global scale g is applied

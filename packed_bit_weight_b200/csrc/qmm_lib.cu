@@ -22,6 +22,7 @@
 #include "k_gemv_ring.cuh"
 #include "k_iq4p.cuh"
 #include "k_iq4w.cuh"
+#include "k_quant.cuh"
 #include "k_moe.cuh"
 
 namespace qmm {
@@ -834,6 +835,36 @@ qmm_status qmm_dequant(const qmm_weights* w, uint16_t* out, void* stream) {
     const int64_t ng = total / 16;
     dequant_fp4_kernel<3><<<grid_for(ng, 256, di->sms), 256, 0, st>>>(data, sc, w->global_scale, out, ng);
     set_variant("dequant_fp4<fmt=3>");
+  }
+  return launch_status();
+}
+
+qmm_status qmm_quantize(int32_t fmt, const uint16_t* w, int64_t n, int64_t k, void* data, void* scales, void* stream) {
+  if (!valid_fmt(fmt) || n < 0 || k < 0) return QMM_ERR_INVALID_ARG;
+  if (fmt == QMM_FMT_FP4G16_E4M3) return QMM_ERR_UNSUPPORTED_SHAPE;  // needs a matrix-wide global scale: not encoded
+  if (k % fmt_group(fmt) || n > INT32_MAX || k > INT32_MAX) return QMM_ERR_UNSUPPORTED_SHAPE;
+  qmm_status s;
+  DevInfo* di = nullptr;
+  if ((s = device_info(&di)) != QMM_OK) return s;
+  const int64_t total = n * k;
+  if (total == 0) return QMM_OK;
+  if (!w || !data || (fmt != QMM_FMT_IQ4_NL && !scales)) return QMM_ERR_INVALID_ARG;
+  if (!aligned16(w) || !aligned16(data) || (scales && !aligned16(scales))) return QMM_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* d = static_cast<uint8_t*>(data);
+  uint8_t* sc = static_cast<uint8_t*>(scales);
+  if (fmt == QMM_FMT_IQ4_NL) {
+    const int64_t nb = total / 32;
+    quantize_iq4nl_kernel<<<grid_for(nb, 128, di->sms), 128, 0, st>>>(w, d, nb);
+    set_variant("quantize_iq4nl");
+  } else if (fmt == QMM_FMT_MXFP4) {
+    const int64_t ng = total / 32;
+    quantize_fp4_kernel<4><<<grid_for(ng, 128, di->sms), 128, 0, st>>>(w, d, sc, ng);
+    set_variant("quantize_fp4<fmt=4>");
+  } else {
+    const int64_t ng = total / 16;
+    quantize_fp4_kernel<2><<<grid_for(ng, 128, di->sms), 128, 0, st>>>(w, d, sc, ng);
+    set_variant("quantize_fp4<fmt=2>");
   }
   return launch_status();
 }

@@ -59,6 +59,7 @@ def _lib():
             "qmm_scale_bytes": (sz, [i32, i64, i64]),
             "qmm_packed_bytes": (sz, [i32, i64, i64]),
             "qmm_dequant": (i32, [W, vp, vp]),
+            "qmm_quantize": (i32, [i32, vp, i64, i64, vp, vp, vp]),
             "qmm_gemv": (i32, [W, vp, i64, vp, vp, sz, vp]),
             "qmm_gemm": (i32, [W, vp, i64, vp, vp, sz, vp]),
             "qmm_route": (i32, [vp, i64, i64, i64, vp, vp, vp, sz, vp]),
@@ -197,6 +198,14 @@ def qmm_dequant(w: PackedWeights, out: torch.Tensor, stream=None) -> torch.Tenso
     d = w.desc()
     _check(_lib().qmm_dequant(ctypes.byref(d), _ptr(out, 2, "out"), _stream(stream)), "qmm_dequant")
     return out
+
+
+def qmm_quantize(fmt: int, w: torch.Tensor, data: torch.Tensor, scales: torch.Tensor | None = None,
+                 stream=None) -> None:
+    """fp16 weights w [n][k] (2-byte elements) -> packed data / scales."""
+    n, k = w.shape
+    _check(_lib().qmm_quantize(fmt, _ptr(w, 2, "w"), n, k, _ptr(data, None, "data"), _ptr(scales, None, "scales"),
+                               _stream(stream)), "qmm_quantize")
 
 
 def _ws(ws):

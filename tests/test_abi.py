@@ -22,7 +22,7 @@ def _declared():
 def test_header_declares_the_boundary():
     names = _declared()
     for want in ("qmm_dequant", "qmm_gemv", "qmm_gemm", "qmm_route", "qmm_grouped_gemv", "qmm_router_topk",
-                 "qmm_moe_routed", "qmm_sync_check"):
+                 "qmm_moe_routed", "qmm_sync_check", "qmm_quantize"):
         assert want in names
 
 
@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol():
 def test_size_functions_match_the_oracle():
     import oracle
     from packed_bit_weight_b200 import qmm
-    for fmt in (1, 2, 3):
+    for fmt in (1, 2, 3, 4):
         for n, k in ((256, 512), (18560, 4096), (1792, 2560), (2560, 896), (3, 64), (0, 32)):
             assert qmm.qmm_data_bytes(fmt, n, k) == oracle.data_bytes(fmt, n, k)
             assert qmm.qmm_scale_bytes(fmt, n, k) == oracle.scale_bytes(fmt, n, k)
