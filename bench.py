@@ -113,15 +113,20 @@ class ClockSampler:
 # collective: every rank runs independent replicas of the workload)
 # ---------------------------------------------------------------------------
 def dist_init():
+    """One process per GPU over NCCL; without a GPU (the CPU tests of this
+    plumbing) the same steps run over gloo."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     import torch
     if world > 1:
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
     elif torch.cuda.is_available():
         torch.cuda.set_device(local)
     return world, rank, local
@@ -138,9 +143,16 @@ def max_over_ranks(v: float, world: int) -> float:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_throughput(bytes_per_launch: int, launches: int, seconds_max: float, world: int) -> float:
+    """Whole-job GB/s of N independent replicas: every rank streams the same
+    bytes per launch; the job takes as long as its slowest rank."""
+    return world * bytes_per_launch * launches / seconds_max / 1e9
 
 
 # ---------------------------------------------------------------------------
@@ -594,7 +606,7 @@ def main():
     r = gemv_workload(p, x, args.steps, args.warmup, world, l2, sampler)
     secs = max_over_ranks(r["seconds"], world)
     launches = r["launches"]
-    value = world * r["bytes_per_launch"] * launches / secs / 1e9
+    value = replica_throughput(r["bytes_per_launch"], launches, secs, world)
     per_launch = secs / launches
     achieved = r["bytes_per_launch"] / per_launch / 1e9
     e2e = gemv_e2e(p, x, max(200, min(5000, args.steps // 4)), world)
