@@ -188,6 +188,7 @@ __device__ __forceinline__ void iq4_pass(float (&acc)[4][4], const uint8_t* __re
                                          int rb, int s_lo, int s_hi, int tig, const uint16_t* const (&xr)[4],
                                          uint32_t lut_lane) {
   uint32_t wa[SMAX][5], wb[SMAX][5];
+  uint32_t xs[SMAX][NT][16];  // the pass's activation words, loaded with the weights
 #pragma unroll
   for (int u = 0; u < SMAX; u++) {
     if (s_lo + u < s_hi) {
@@ -199,6 +200,20 @@ __device__ __forceinline__ void iq4_pass(float (&acc)[4][4], const uint8_t* __re
       for (int i = 0; i < 5; i++) {
         wa[u][i] = __ldg(pa + i);
         wb[u][i] = __ldg(pb + i);
+      }
+#pragma unroll
+      for (int j = 0; j < NT; j++) {
+        if (xr[j]) {
+          const uint16_t* xp = xr[j] + b * 32;
+#pragma unroll
+          for (int q = 0; q < 4; q++) {
+            const uint4 v = ldg_x128(xp + 8 * q);
+            xs[u][j][4 * q] = v.x; xs[u][j][4 * q + 1] = v.y; xs[u][j][4 * q + 2] = v.z; xs[u][j][4 * q + 3] = v.w;
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 16; q++) xs[u][j][q] = 0u;
+        }
       }
     }
   }
@@ -222,21 +237,7 @@ __device__ __forceinline__ void iq4_pass(float (&acc)[4][4], const uint8_t* __re
       }
     }
     const uint32_t dda = da | (da << 16), ddb = db | (db << 16);
-    uint32_t xw[NT][16];  // this block's 32 activations per n-tile, as 16 words
-#pragma unroll
-    for (int j = 0; j < NT; j++) {
-      if (xr[j]) {
-        const uint16_t* xp = xr[j] + b * 32;
-#pragma unroll
-        for (int q = 0; q < 4; q++) {
-          const uint4 v = ldg_x128(xp + 8 * q);
-          xw[j][4 * q] = v.x; xw[j][4 * q + 1] = v.y; xw[j][4 * q + 2] = v.z; xw[j][4 * q + 3] = v.w;
-        }
-      } else {
-#pragma unroll
-        for (int q = 0; q < 16; q++) xw[j][q] = 0u;
-      }
-    }
+    const uint32_t (&xw)[NT][16] = xs[u];  // this block's 32 activations per n-tile, as 16 words
 #pragma unroll
     for (int i = 0; i < 8; i++) {  // index bytes 2i, 2i+1 of the block
       const uint32_t qwa = qa[i >> 1], qwb = qb[i >> 1];
@@ -260,7 +261,7 @@ template <int NT>
 __device__ __forceinline__ void iq4_range(float (&acc)[4][4], const uint8_t* __restrict__ de, int64_t rowb, int ra,
                                           int rb, int s_lo, int s_hi, int tig, const uint16_t* const (&xr)[4],
                                           uint32_t lut_lane) {
-  constexpr int SMAX = (NT == 1) ? 3 : 2;
+  constexpr int SMAX = (NT == 1) ? 2 : 1;  // super-steps per pass (their weights and activations in registers)
   for (int s0 = s_lo; s0 < s_hi; s0 += SMAX)
     iq4_pass<NT, SMAX>(acc, de, rowb, ra, rb, s0, min(s0 + SMAX, s_hi), tig, xr, lut_lane);
 }
