@@ -246,7 +246,8 @@ void orc_dequant(int fmt, int64_t n, int64_t k, const uint8_t* data, const uint8
 /*   FP4-G16 (fp16 scale): s = fp16(amax / 6) per group of 16, amax = the  */
 /*     largest |w| of the group (6 = the largest E2M1 magnitude).           */
 /*   MXFP4: e = floor(log2(amax)) - 2 + 127 clamped to [0, 254] (the OCP MX */
-/*     shared exponent; 2 = the E2M1 maximum's exponent), e = 0 for amax = 0.*/
+/*     shared exponent; 2 = the E2M1 maximum's exponent), e = 0 for amax = 0,*/
+/*     254 for an infinite amax.                                            */
 /*   IQ4_NL: d = fp16(m / -127), m the first element of largest |w| of the  */
 /*     block, so that it maps to the table's -127 entry.                    */
 /* Then each weight takes the code whose decoded value (exactly as the      */
@@ -301,7 +302,9 @@ void orc_quantize(int fmt, int64_t n, int64_t k, const uint16_t* w, uint8_t* dat
       double sc;
       if (fmt == ORC_FMT_MXFP4) {
         int e = 0;
-        if (am > 0.0) {
+        if (isinf(am)) {
+          e = 254; /* an infinite weight: the largest scale */
+        } else if (am > 0.0) {
           int ex;
           frexp(am, &ex); /* am = fr * 2^ex, fr in [0.5, 1): floor(log2(am)) = ex - 1 */
           e = ex - 1 - 2 + 127;
