@@ -349,6 +349,19 @@ __device__ __forceinline__ uint32_t ldg_stream16(const void* p) {
   asm("ld.global.nc.L1::no_allocate.L2::256B.u16 %0, [%1];" : "=h"(v) : "l"(p));
   return v;
 }
+// 256-bit streaming loads (sm_100): 32 contiguous bytes per lane, so the
+// four lanes of a weight row cover a whole 128-byte line per instruction.
+// p must be 32-byte aligned.
+__device__ __forceinline__ void ldg_stream256(const void* p, uint4& lo, uint4& hi) {
+  asm("ld.global.nc.L1::no_allocate.L2::256B.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+      : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w), "=r"(hi.x), "=r"(hi.y), "=r"(hi.z), "=r"(hi.w)
+      : "l"(p));
+}
+__device__ __forceinline__ uint2 ldg_stream64(const void* p) {
+  uint2 v;
+  asm("ld.global.nc.L1::no_allocate.L2::256B.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+  return v;
+}
 __device__ __forceinline__ uint4 ldg_x128(const void* p) {
   uint4 v;
   asm("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
@@ -369,13 +382,17 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 // token row in every lane instead of zero-filling the columns past m (27 %:
 // 8x the L1 traffic), and zero-filling once before the segment loop (18 %:
 // the compiler then keeps fewer of the tile's loads in flight).
-template <int FMT, int NT, int SPW>
+// WIDE: the lane's bytes of two consecutive segments 2w, 2w+1 are the 32
+// contiguous bytes at 32*tig of a 256-k span (one 256-bit load), so segment
+// 2w+h holds k = 256w + 64*tig + 32h + [0, 32) instead of 128s + 32*tig.
+template <int FMT, int NT, int SPW, bool WIDE = false>
 __device__ __forceinline__ void ldg_tile_mma(float (&acc)[NT][4], const uint4 (&qa)[SPW], const uint4 (&qb)[SPW],
                                              const uint32_t (&sa)[SPW], const uint32_t (&sb)[SPW], int seg0, int grp,
                                              int tig, const uint16_t* __restrict__ x, int k, int m) {
 #pragma unroll
   for (int i = 0; i < SPW; i++) {
-    const int kseg = (seg0 + i) * 128 + tig * 32;
+    const int s = seg0 + i;
+    const int kseg = WIDE ? (s >> 1) * 256 + tig * 64 + (s & 1) * 32 : s * 128 + tig * 32;
     uint32_t xb[NT][16];
 #pragma unroll
     for (int j = 0; j < NT; j++) {
@@ -451,10 +468,15 @@ __device__ __forceinline__ void ldg_tile_store(float (&red)[WPC][16][16], const 
   }
 }
 
-template <int FMT, int NT, int SPW, int WPC = kLdgWarps, int MINB = 2>
+// WIDE (k % 256 == 0, SPW even, codes 32-byte aligned): each lane loads its
+// bytes of two segments with one 256-bit load per row, and their scales with
+// one load (8 B fp16, 4 B E4M3, 2 B E8M0), the segment pairing of
+// ldg_tile_mma's WIDE layout.
+template <int FMT, int NT, int SPW, int WPC = kLdgWarps, int MINB = 2, bool WIDE = false>
 __global__ void __launch_bounds__(WPC * 32, MINB)
     gemv_fp4_ldg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
                         const uint16_t* __restrict__ x, uint16_t* __restrict__ y, int n, int k, int m, float g) {
+  static_assert(!WIDE || SPW % 2 == 0, "WIDE pairs segments");
   __shared__ float red[WPC][16][16];  // [warp][token][row]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int grp = lane >> 2, tig = lane & 3;
@@ -467,6 +489,32 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
   pdl_launch_dependents();
   uint4 qa[SPW], qb[SPW];
   uint32_t sa[SPW], sb[SPW];
+  if (WIDE) {
+#pragma unroll
+    for (int p = 0; p < SPW / 2; p++) {
+      const int64_t w2 = (seg0 >> 1) + p;  // 256-k span
+      const int64_t cb = w2 * 128 + tig * 32;
+      const uint4 z = make_uint4(0, 0, 0, 0);
+      qa[2 * p] = z; qa[2 * p + 1] = z; qb[2 * p] = z; qb[2 * p + 1] = z;
+      if (va) ldg_stream256(codes + ra * crow + cb, qa[2 * p], qa[2 * p + 1]);
+      if (vb) ldg_stream256(codes + rb * crow + cb, qb[2 * p], qb[2 * p + 1]);
+      if (FMT == 2) {  // four fp16 group scales: groups 16*w2 + 4*tig .. +3
+        const uint2 s0 = va ? ldg_stream64(scales + (ra * srow + w2 * 16 + tig * 4) * 2) : make_uint2(0, 0);
+        const uint2 s1 = vb ? ldg_stream64(scales + (rb * srow + w2 * 16 + tig * 4) * 2) : make_uint2(0, 0);
+        sa[2 * p] = s0.x; sa[2 * p + 1] = s0.y; sb[2 * p] = s1.x; sb[2 * p + 1] = s1.y;
+      } else if (FMT == 4) {  // two E8M0 bytes: MX groups 8*w2 + 2*tig, +1 (127 = 1 for rows past n)
+        const uint32_t s0 = va ? ldg_stream16(scales + ra * (srow >> 1) + w2 * 8 + tig * 2) : 0x7F7Fu;
+        const uint32_t s1 = vb ? ldg_stream16(scales + rb * (srow >> 1) + w2 * 8 + tig * 2) : 0x7F7Fu;
+        sa[2 * p] = e8m0_f16_factor_pair(s0 & 0xFFu); sa[2 * p + 1] = e8m0_f16_factor_pair(s0 >> 8);
+        sb[2 * p] = e8m0_f16_factor_pair(s1 & 0xFFu); sb[2 * p + 1] = e8m0_f16_factor_pair(s1 >> 8);
+      } else {  // four E4M3 group scales
+        const uint32_t s0 = va ? ldg_stream32(scales + ra * srow + w2 * 16 + tig * 4) : 0u;
+        const uint32_t s1 = vb ? ldg_stream32(scales + rb * srow + w2 * 16 + tig * 4) : 0u;
+        sa[2 * p] = e4m3x2_to_f16x2(s0 & 0xFFFFu); sa[2 * p + 1] = e4m3x2_to_f16x2(s0 >> 16);
+        sb[2 * p] = e4m3x2_to_f16x2(s1 & 0xFFFFu); sb[2 * p + 1] = e4m3x2_to_f16x2(s1 >> 16);
+      }
+    }
+  } else {
 #pragma unroll
   for (int i = 0; i < SPW; i++) {
     const int seg = seg0 + i;
@@ -485,6 +533,7 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
       sb[i] = vb ? e4m3x2_to_f16x2(ldg_stream16(scales + rb * srow + gi)) : 0u;
     }
   }
+  }
   pdl_wait();  // x may be the previous kernel's output; y may still be read by it
 
   float acc[NT][4];
@@ -492,7 +541,7 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
   for (int j = 0; j < NT; j++)
 #pragma unroll
     for (int c = 0; c < 4; c++) acc[j][c] = 0.f;
-  ldg_tile_mma<FMT, NT, SPW>(acc, qa, qb, sa, sb, seg0, grp, tig, x, k, m);
+  ldg_tile_mma<FMT, NT, SPW, WIDE>(acc, qa, qb, sa, sb, seg0, grp, tig, x, k, m);
   ldg_tile_store<FMT, NT, WPC>(red, acc, warp, grp, tig, n0, n, m, g, y);
 }
 

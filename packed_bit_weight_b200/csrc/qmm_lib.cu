@@ -167,7 +167,7 @@ static qmm_status launch_gemv_tma(const qmm_weights* w, const uint16_t* x, int m
   return launch_status();
 }
 
-template <int FMT, int NT, int SPW, int WPC = kLdgWarps, int MINB = 2>
+template <int FMT, int NT, int SPW, int WPC = kLdgWarps, int MINB = 2, bool WIDE = false>
 static qmm_status launch_gemv_ldg(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st) {
   const int n = (int)w->n, k = (int)w->k;
   const int tiles = (n + 15) / 16;
@@ -177,7 +177,7 @@ static qmm_status launch_gemv_ldg(const qmm_weights* w, const uint16_t* x, int m
   const char* nopdl = getenv("QMM_GEMV_NOPDL");
   const char* pad = getenv("QMM_GEMV_SMEM_PAD");
   const int pad_bytes = pad ? atoi(pad) : 0;
-  auto kern = gemv_fp4_ldg_kernel<FMT, NT, SPW, WPC, MINB>;
+  auto kern = gemv_fp4_ldg_kernel<FMT, NT, SPW, WPC, MINB, WIDE>;
   if (pad_bytes > 0 &&
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pad_bytes) != cudaSuccess)
     return QMM_ERR_CUDA;
@@ -195,8 +195,31 @@ static qmm_status launch_gemv_ldg(const qmm_weights* w, const uint16_t* x, int m
   const uint8_t* scales = static_cast<const uint8_t*>(w->scales);
   const float g = w->global_scale;
   if (cudaLaunchKernelEx(&cfg, kern, codes, scales, x, y, n, k, m, g) != cudaSuccess) return QMM_ERR_CUDA;
-  set_variant("gemv_fp4_ldg<fmt=%d,nt=%d,spw=%d,wpc=%d,minb=%d,tiles=%d>", FMT, NT, SPW, WPC, MINB, tiles);
+  set_variant("gemv_fp4_ldg<fmt=%d,nt=%d,spw=%d,wpc=%d,minb=%d,wide=%d,tiles=%d>", FMT, NT, SPW, WPC, MINB,
+              WIDE ? 1 : 0, tiles);
   return launch_status();
+}
+
+// The 256-bit-load layout where the shape and alignment allow it (k % 256 ==
+// 0 for segment pairs, an even segment count per warp, 32-byte-aligned codes)
+// and it measured faster: MXFP4 (one 2-byte scale load instead of two 1-byte
+// loads per pair; in_proj m = 1 12.2 vs 13.1 us on B200).  For FP4-G16 it
+// measured slower at every shape (in_proj m = 1 11.3 vs 10.4 us: 109 vs 98
+// registers).  QMM_GEMV_WIDE=0/1 forces either layout (measurement knob).
+static bool ldg_wide_ok(const qmm_weights* w) {
+  if (w->k % 256 != 0 || (reinterpret_cast<uintptr_t>(w->data) & 31u) != 0) return false;
+  const char* e = getenv("QMM_GEMV_WIDE");
+  if (e && e[0]) return e[0] == '1';
+  return w->fmt == QMM_FMT_MXFP4;
+}
+
+template <int FMT, int NT, int SPW, int WPC, int MINB>
+static qmm_status launch_gemv_ldg_pick(bool wide, const qmm_weights* w, const uint16_t* x, int m, uint16_t* y,
+                                       cudaStream_t st) {
+  if constexpr (SPW % 2 == 0) {
+    if (wide) return launch_gemv_ldg<FMT, NT, SPW, WPC, MINB, true>(w, x, m, y, st);
+  }
+  return launch_gemv_ldg<FMT, NT, SPW, WPC, MINB, false>(w, x, m, y, st);
 }
 
 // Persistent ring GEMV (k_gemv_ring.cuh): one CTA per SM, whole 16-row tiles
@@ -292,50 +315,51 @@ template <int FMT, int NT>
 static qmm_status gemv_ldg_auto(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st) {
   const int segs = (int)(w->k / 128);
   if (w->k % 128) return QMM_ERR_UNSUPPORTED_SHAPE;
+  const bool wide = ldg_wide_ok(w);
   if (NT == 1) {
     if (segs % 4 == 0 && segs / 4 <= 8) {
       switch (segs / 4) {
-        case 1: return launch_gemv_ldg<FMT, 1, 1, 4, 4>(w, x, m, y, st);
-        case 2: return launch_gemv_ldg<FMT, 1, 2, 4, 4>(w, x, m, y, st);
-        case 3: return launch_gemv_ldg<FMT, 1, 3, 4, 4>(w, x, m, y, st);
-        case 4: return launch_gemv_ldg<FMT, 1, 4, 4, 4>(w, x, m, y, st);
-        case 5: return launch_gemv_ldg<FMT, 1, 5, 4, 4>(w, x, m, y, st);
-        case 6: return launch_gemv_ldg<FMT, 1, 6, 4, 4>(w, x, m, y, st);
-        case 7: return launch_gemv_ldg<FMT, 1, 7, 4, 4>(w, x, m, y, st);
-        default: return launch_gemv_ldg<FMT, 1, 8, 4, 4>(w, x, m, y, st);
+        case 1: return launch_gemv_ldg_pick<FMT, 1, 1, 4, 4>(wide, w, x, m, y, st);
+        case 2: return launch_gemv_ldg_pick<FMT, 1, 2, 4, 4>(wide, w, x, m, y, st);
+        case 3: return launch_gemv_ldg_pick<FMT, 1, 3, 4, 4>(wide, w, x, m, y, st);
+        case 4: return launch_gemv_ldg_pick<FMT, 1, 4, 4, 4>(wide, w, x, m, y, st);
+        case 5: return launch_gemv_ldg_pick<FMT, 1, 5, 4, 4>(wide, w, x, m, y, st);
+        case 6: return launch_gemv_ldg_pick<FMT, 1, 6, 4, 4>(wide, w, x, m, y, st);
+        case 7: return launch_gemv_ldg_pick<FMT, 1, 7, 4, 4>(wide, w, x, m, y, st);
+        default: return launch_gemv_ldg_pick<FMT, 1, 8, 4, 4>(wide, w, x, m, y, st);
       }
     }
     if (segs % 8 == 0 && segs / 8 <= 8) {
       switch (segs / 8) {
-        case 5: return launch_gemv_ldg<FMT, 1, 5, 8, 2>(w, x, m, y, st);
-        case 6: return launch_gemv_ldg<FMT, 1, 6, 8, 2>(w, x, m, y, st);
-        case 7: return launch_gemv_ldg<FMT, 1, 7, 8, 2>(w, x, m, y, st);
-        case 8: return launch_gemv_ldg<FMT, 1, 8, 8, 2>(w, x, m, y, st);
+        case 5: return launch_gemv_ldg_pick<FMT, 1, 5, 8, 2>(wide, w, x, m, y, st);
+        case 6: return launch_gemv_ldg_pick<FMT, 1, 6, 8, 2>(wide, w, x, m, y, st);
+        case 7: return launch_gemv_ldg_pick<FMT, 1, 7, 8, 2>(wide, w, x, m, y, st);
+        case 8: return launch_gemv_ldg_pick<FMT, 1, 8, 8, 2>(wide, w, x, m, y, st);
         default: break;  // smaller counts took the 4-warp path
       }
     }
     if (segs % 16 == 0 && segs / 16 <= 8) {
       switch (segs / 16) {
-        case 5: return launch_gemv_ldg<FMT, 1, 5, 16, 1>(w, x, m, y, st);
-        case 6: return launch_gemv_ldg<FMT, 1, 6, 16, 1>(w, x, m, y, st);
-        case 7: return launch_gemv_ldg<FMT, 1, 7, 16, 1>(w, x, m, y, st);
-        case 8: return launch_gemv_ldg<FMT, 1, 8, 16, 1>(w, x, m, y, st);
+        case 5: return launch_gemv_ldg_pick<FMT, 1, 5, 16, 1>(wide, w, x, m, y, st);
+        case 6: return launch_gemv_ldg_pick<FMT, 1, 6, 16, 1>(wide, w, x, m, y, st);
+        case 7: return launch_gemv_ldg_pick<FMT, 1, 7, 16, 1>(wide, w, x, m, y, st);
+        case 8: return launch_gemv_ldg_pick<FMT, 1, 8, 16, 1>(wide, w, x, m, y, st);
         default: break;
       }
     }
   } else {
     if (segs % 8 == 0 && segs / 8 <= 4) {
       switch (segs / 8) {
-        case 1: return launch_gemv_ldg<FMT, 2, 1, 8, 2>(w, x, m, y, st);
-        case 2: return launch_gemv_ldg<FMT, 2, 2, 8, 2>(w, x, m, y, st);
-        case 3: return launch_gemv_ldg<FMT, 2, 3, 8, 2>(w, x, m, y, st);
-        default: return launch_gemv_ldg<FMT, 2, 4, 8, 2>(w, x, m, y, st);
+        case 1: return launch_gemv_ldg_pick<FMT, 2, 1, 8, 2>(wide, w, x, m, y, st);
+        case 2: return launch_gemv_ldg_pick<FMT, 2, 2, 8, 2>(wide, w, x, m, y, st);
+        case 3: return launch_gemv_ldg_pick<FMT, 2, 3, 8, 2>(wide, w, x, m, y, st);
+        default: return launch_gemv_ldg_pick<FMT, 2, 4, 8, 2>(wide, w, x, m, y, st);
       }
     }
     if (segs % 16 == 0 && segs / 16 <= 4) {
       switch (segs / 16) {
-        case 3: return launch_gemv_ldg<FMT, 2, 3, 16, 1>(w, x, m, y, st);
-        case 4: return launch_gemv_ldg<FMT, 2, 4, 16, 1>(w, x, m, y, st);
+        case 3: return launch_gemv_ldg_pick<FMT, 2, 3, 16, 1>(wide, w, x, m, y, st);
+        case 4: return launch_gemv_ldg_pick<FMT, 2, 4, 16, 1>(wide, w, x, m, y, st);
         default: break;
       }
     }

@@ -54,6 +54,47 @@ def test_every_streaming_variant_vs_oracle(variant, fmt, n, k, m, monkeypatch):
     check_tol(y, yref, absy, v)
 
 
+@pytest.mark.parametrize("wide", ["0", "1"])
+@pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3, synth.FMT_MXFP4])
+@pytest.mark.parametrize("n,k,m", [(1000, 4096, 1), (333, 8192, 3), (517, 3072, 9), (64, 2048, 16),
+                                   (77, 1536, 5), (40, 1024, 1), (129, 2048, 8)])
+def test_register_kernel_both_load_layouts(wide, fmt, n, k, m, monkeypatch):
+    """The register GEMV with 128-bit loads and with 256-bit loads (segment
+    pairs; taken when k % 256 == 0, the warp's segment count is even and the
+    codes are 32-byte aligned)."""
+    monkeypatch.setenv("QMM_GEMV_VARIANT", "ldg")
+    monkeypatch.setenv("QMM_GEMV_WIDE", wide)
+    p, x = _case(fmt, n, k, m, 3000 + n + k + m + fmt)
+    y = run_gemv(dev(p), x)
+    v = qmm.qmm_last_variant()
+    assert v.startswith("gemv_fp4_ldg"), v
+    spw = int(v.split("spw=")[1].split(",")[0])
+    expect_wide = wide == "1" and k % 256 == 0 and spw % 2 == 0
+    assert ("wide=1" in v) == expect_wide, v
+    yref, absy = oracle.matmul(fmt, n, k, p.data, p.scales, p.global_scale, x)
+    check_tol(y, yref, absy, v)
+
+
+@pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_MXFP4])
+def test_codes_16_byte_aligned_take_the_128_bit_layout(fmt):
+    """Codes that are 16- but not 32-byte aligned (legal in the ABI) must not
+    reach the 256-bit loads."""
+    n, k, m = 300, 4096, 2
+    p, x = _case(fmt, n, k, m, 91 + fmt)
+    w = dev(p)
+    buf = torch.zeros(w.data.numel() + 48, dtype=torch.uint8, device="cuda")
+    off = 16 if (buf.data_ptr() + 16) % 32 else 48
+    shifted = buf[off:off + w.data.numel()]
+    shifted.copy_(w.data.view(torch.uint8).reshape(-1))
+    assert shifted.data_ptr() % 32 == 16
+    w2 = qmm.PackedWeights(w.fmt, w.n, w.k, shifted, w.scales, w.global_scale)
+    y = run_gemv(w2, x)
+    v = qmm.qmm_last_variant()
+    assert v.startswith("gemv_fp4_ldg") and "wide=0" in v, v
+    yref, absy = oracle.matmul(fmt, n, k, p.data, p.scales, p.global_scale, x)
+    check_tol(y, yref, absy, v)
+
+
 @pytest.mark.parametrize("fmt", FMTS)
 def test_one_hot_gives_the_decoded_column_bit_exactly(fmt):
     n, k = 300, 4096
