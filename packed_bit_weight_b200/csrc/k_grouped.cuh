@@ -28,6 +28,9 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
   __shared__ int fill[kRouteMaxExperts];
   __shared__ int wcnt[kRouteThreads / 32][kRouteMaxExperts];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // a kernel launched after this one with programmatic dependent launch may
+  // start now (it waits for this kernel's results before reading them)
+  asm volatile("griddepcontrol.launch_dependents;" :::);
   for (int e = tid; e < E; e += kRouteThreads) cnt[e] = 0;
   __syncthreads();
   bool bad = false;

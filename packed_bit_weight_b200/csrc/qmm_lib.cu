@@ -22,6 +22,7 @@
 #include "k_gemv_ring.cuh"
 #include "k_iq4p.cuh"
 #include "k_iq4w.cuh"
+#include "k_iq4t.cuh"
 #include "k_quant.cuh"
 #include "k_moe.cuh"
 
@@ -399,8 +400,15 @@ static int gemv_variant_env() {
   if (!strcmp(v, "ring")) return 7;
   if (!strcmp(v, "dual")) return 8;
   if (!strcmp(v, "iq4w")) return 9;
+  if (!strcmp(v, "iq4t")) return 10;
   return 0;
 }
+
+// Tile-resident IQ4_NL kernel (k_iq4t.cuh); UNSUPPORTED_SHAPE launches nothing.
+template <int MODE>
+static qmm_status launch_iq4_tile(const qmm_weights* w0, const qmm_weights* w1, const uint16_t* x, int x_per_pair,
+                                  int64_t topk, const int32_t* offsets, const int32_t* perm, int64_t P, int m_plain,
+                                  void* y, const float* gw, cudaStream_t st);
 
 // Warp-per-tile IQ4_NL kernel (k_iq4w.cuh); UNSUPPORTED_SHAPE launches nothing.
 template <int MODE>
@@ -516,6 +524,10 @@ static qmm_status gemv_fmt(const qmm_weights* w, const uint16_t* x, int m, uint1
       if (m <= 8) return launch_gemv_tma<FMT, 1, 1>(w, x, m, y, st, di);
       return launch_gemv_tma<FMT, 1, 2>(w, x, m, y, st, di);
     }
+  }
+  if (FMT == 1 && pick == 10) {
+    const qmm_status s = launch_iq4_tile<IQ_OUT_F16>(w, nullptr, x, 0, 1, nullptr, nullptr, 0, m, y, nullptr, st);
+    if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
   }
   if (FMT == 1 && pick == 9) {
     const qmm_status s = launch_iq4_warp<IQ_OUT_F16>(w, nullptr, x, 0, 1, nullptr, nullptr, m, y, nullptr, st, di);
@@ -654,7 +666,7 @@ static qmm_status launch_iq4_warp(const qmm_weights* w0, const qmm_weights* w1, 
     return QMM_ERR_CUDA;
   int64_t grid = 2 * (int64_t)di->sms;
   if (!offsets) {
-    const int64_t items = ((n + 15) / 16) * ((m_plain + 15) / 16);
+    const int64_t items = ((n + 31) / 32) * ((m_plain + 15) / 16);  // tile pairs x token groups
     grid = std::min<int64_t>(grid, (items + kIqwWarps - 1) / kIqwWarps);
   }
   IqwArgs a;
@@ -676,6 +688,88 @@ static qmm_status launch_iq4_warp(const qmm_weights* w0, const qmm_weights* w1, 
   iq4_warp_kernel<MODE><<<(unsigned)std::max<int64_t>(grid, 1), kIqwWarps * 32, smem, st>>>(a);
   set_variant("iq4_warp<mode=%d,grid=%d>", MODE, (int)grid);
   return launch_status();
+}
+
+// Tile-resident IQ4_NL kernel (k_iq4t.cuh): one CTA per (expert, item of S
+// tiles), programmatic dependent launch.  The weights are loaded before the
+// dependency wait when most experts are expected to have pairs (P >= 4E:
+// fewer than 2 % of the experts empty for uniform routing) or for the plain
+// product; QMM_IQ4T_SPEC=0/1 forces either (measurement knob).
+template <int MODE, int S, int SPW, int kMaxReg, bool W16>
+static qmm_status launch_iq4_tile_cfg(const qmm_weights* w0, const qmm_weights* w1, const uint16_t* x, int x_per_pair,
+                                      int64_t topk, const int32_t* offsets, const int32_t* perm, int64_t P,
+                                      int m_plain, void* y, const float* gw, cudaStream_t st) {
+  const int steps = (int)(w0->k / 128), wpc = steps / SPW;
+  const int64_t tiles = (w0->n + 15) / 16;
+  const int64_t ipe = (MODE == IQ_SWIGLU) ? tiles : (tiles + S - 1) / S;
+  const int64_t E = offsets ? w0->num_experts : 1;
+  const int64_t grid = E * ipe;
+  if (grid < 1 || grid > INT32_MAX) return QMM_ERR_UNSUPPORTED_SHAPE;
+  auto kern = iq4_tile_kernel<MODE, S, SPW, kMaxReg, W16>;
+  const uint32_t smem = iqt_smem_bytes(S, wpc);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return QMM_ERR_CUDA;
+  IqtArgs a;
+  a.data0 = static_cast<const uint8_t*>(w0->data);
+  a.data1 = w1 ? static_cast<const uint8_t*>(w1->data) : nullptr;
+  a.dstride0 = w0->expert_data_stride;
+  a.dstride1 = w1 ? w1->expert_data_stride : 0;
+  a.x = x;
+  a.x_per_pair = x_per_pair;
+  a.topk = (int)topk;
+  a.offsets = offsets;
+  a.perm = perm;
+  a.m_plain = m_plain;
+  a.y = y;
+  a.gw = gw;
+  a.n = (int)w0->n;
+  a.k = (int)w0->k;
+  a.E = (int)E;
+  a.items_per_expert = (int)ipe;
+  a.spec = (!offsets || P >= 4 * E) ? 1 : 0;
+  if (const char* e = getenv("QMM_IQ4T_SPEC")) a.spec = (e[0] == '1') ? 1 : 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(wpc * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return QMM_ERR_CUDA;
+  set_variant("iq4_tile<mode=%d,s=%d,spw=%d,wpc=%d,w16=%d,spec=%d,grid=%d>", MODE, S, SPW, wpc, W16 ? 1 : 0, a.spec,
+              (int)grid);
+  return launch_status();
+}
+
+// Needs k % 128 == 0 and k <= 4096 (at most 16 warps of at most two
+// super-steps); returns QMM_ERR_UNSUPPORTED_SHAPE, having launched nothing,
+// otherwise.
+template <int MODE>
+static qmm_status launch_iq4_tile(const qmm_weights* w0, const qmm_weights* w1, const uint16_t* x, int x_per_pair,
+                                  int64_t topk, const int32_t* offsets, const int32_t* perm, int64_t P, int m_plain,
+                                  void* y, const float* gw, cudaStream_t st) {
+  if (w0->fmt != QMM_FMT_IQ4_NL || (w1 && w1->fmt != QMM_FMT_IQ4_NL)) return QMM_ERR_UNSUPPORTED_SHAPE;
+  const int64_t k = w0->k, n = w0->n;
+  if (k % 128 || k < 128 || n < 1 || n > INT32_MAX / 2) return QMM_ERR_UNSUPPORTED_SHAPE;
+  const int64_t steps = k / 128;
+  // registers: 96 keeps two CTAs of up to 10 warps (three of 7) per SM
+  if (steps % 2 == 0 && steps / 2 <= kIqtMaxWarps)  // k % 256 == 0: rows 16-byte aligned
+    return launch_iq4_tile_cfg<MODE, 2, 2, 96, true>(w0, w1, x, x_per_pair, topk, offsets, perm, P, m_plain, y, gw,
+                                                     st);
+  if (steps <= kIqtMaxWarps) {
+    const char* e = getenv("QMM_IQ4T_S");  // measurement knob: tiles per item at one super-step per warp
+    if constexpr (MODE != IQ_SWIGLU) {
+      if (!(e && e[0] == '2'))
+        return launch_iq4_tile_cfg<MODE, 4, 1, 128, false>(w0, w1, x, x_per_pair, topk, offsets, perm, P, m_plain, y,
+                                                           gw, st);
+    }
+    return launch_iq4_tile_cfg<MODE, 2, 1, 96, false>(w0, w1, x, x_per_pair, topk, offsets, perm, P, m_plain, y, gw,
+                                                      st);
+  }
+  return QMM_ERR_UNSUPPORTED_SHAPE;
 }
 
 template <int MODE>
@@ -1027,6 +1121,16 @@ qmm_status qmm_grouped_gemv(const qmm_weights* experts, const uint16_t* x, int32
     set_variant("route+zero_fill");
     return launch_status();
   }
+  // IQ4_NL: the tile-resident kernel when most experts have pairs (its
+  // weight loads then overlap the routing pass), else the streaming kernel
+  const bool iq4_tile = pick == 10 || (pick == 0 && P >= 4 * experts->num_experts);
+  if (experts->fmt == QMM_FMT_IQ4_NL && iq4_tile) {
+    s = launch_iq4_tile<IQ_OUT_F16>(experts, nullptr, x, x_per_pair, topk, offsets, perm, P, 0, y, nullptr, st);
+    if (s != QMM_ERR_UNSUPPORTED_SHAPE) {
+      set_variant("route+grouped_iq4_tile");
+      return s;
+    }
+  }
   if (experts->fmt == QMM_FMT_IQ4_NL && pick == 9) {
     s = launch_iq4_warp<IQ_OUT_F16>(experts, nullptr, x, x_per_pair, topk, offsets, perm, 0, y, nullptr, st, di);
     if (s != QMM_ERR_UNSUPPORTED_SHAPE) {
@@ -1171,6 +1275,21 @@ qmm_status qmm_moe_routed(const qmm_weights* gate, const qmm_weights* up, const 
     zero_fill_kernel<<<grid_for(t * d, 256, di->sms), 256, 0, st>>>(out, t * d);
     set_variant("moe:route+zero_fill");
     return launch_status();
+  }
+  // tile-resident kernels when most experts have pairs (measured faster at
+  // 64 tokens, slower at 1), else the streaming kernels
+  const int pick = gemv_variant_env();
+  if (pick == 10 || (pick == 0 && P >= 4 * E)) {
+    s = launch_iq4_tile<IQ_SWIGLU>(gate, up, x, 0, topk, offsets, perm, P, 0, h, nullptr, st);
+    if (s == QMM_OK)
+      s = launch_iq4_tile<IQ_SCALED_F32>(down, nullptr, h, 1, topk, offsets, perm, P, 0, yg, topk_weights, st);
+    if (s == QMM_OK) {
+      combine_kernel<<<grid_for(t * (d / 8), 256, di->sms), 256, 0, st>>>(yg, topk_ids, (int)E, (int)t, (int)topk,
+                                                                           (int)d, out);
+      set_variant("moe:route+gate_up_swiglu_iq4_tile+down_scaled_iq4_tile+combine");
+      return launch_status();
+    }
+    if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
   }
   if (gemv_variant_env() == 9) {  // warp-per-tile kernels
     s = launch_iq4_warp<IQ_SWIGLU>(gate, up, x, 0, topk, offsets, perm, 0, h, nullptr, st, di);

@@ -166,7 +166,7 @@ def test_gemv_edge_cases():
     assert e.value.status == 3
 
 
-@pytest.mark.parametrize("variant", [None, "iq4p", "iq4w", "generic"])
+@pytest.mark.parametrize("variant", [None, "iq4p", "iq4w", "iq4t", "generic"])
 @pytest.mark.parametrize("n,k,m", [(256, 512, 1), (2000, 4096, 5), (48, 2560, 16), (4096, 8192, 2)])
 def test_iq4nl_kernels_vs_oracle(variant, n, k, m, monkeypatch):
     """Each IQ4_NL GEMV kernel: the streaming kernel (default for k % 128 ==
@@ -180,7 +180,8 @@ def test_iq4nl_kernels_vs_oracle(variant, n, k, m, monkeypatch):
     y = run_gemv(dev(p), x)
     v = qmm.qmm_last_variant()
     want = {None: ("gemv_iq4_stream",), "iq4p": ("iq4_persist",) if k <= 2560 else ("gemv_generic",),
-            "iq4w": ("iq4_warp",), "generic": ("gemv_generic",)}[variant]
+            "iq4w": ("iq4_warp",), "iq4t": ("iq4_tile",) if k <= 4096 else ("gemv_generic",),
+            "generic": ("gemv_generic",)}[variant]
     assert v.startswith(want), v
     yref, absy = oracle.matmul(synth.FMT_IQ4_NL, n, k, p.data, None, 1.0, x)
     check_tol(y, yref, absy, v)

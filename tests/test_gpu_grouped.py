@@ -108,15 +108,15 @@ def test_grouped_rejects_small_workspace():
     assert e.value.status == 8
 
 
-@pytest.mark.parametrize("variant", [None, "iq4p", "iq4w"])
+@pytest.mark.parametrize("variant", [None, "iq4p", "iq4w", "iq4t"])
 @pytest.mark.parametrize("E,n,k,t,topk,per_pair", [(3, 64, 256, 50, 2, False), (5, 48, 384, 200, 3, True),
                                                     (2, 16, 128, 2100, 2, False), (32, 32, 128, 1, 4, True)])
 def test_grouped_iq4_many_pairs_per_expert(variant, E, n, k, t, topk, per_pair, monkeypatch):
     """IQ4_NL experts with more than 16 pairs each (several token groups per
-    expert, whose row tiles land on different CTAs), with the routed streaming
-    kernel (default) and the persistent kernel; t * topk = 4200 is past the
-    persistent kernel's pair limit (a forced variant that does not take a
-    shape leaves it to the generic kernel)."""
+    expert, whose row tiles land on different CTAs), with the default kernel
+    (tile-resident, or streaming when t * topk < 4 E) and the opt-in ones;
+    t * topk = 4200 is past the persistent kernel's pair limit (a forced
+    variant that does not take a shape leaves it to the generic kernel)."""
     if variant:
         monkeypatch.setenv("QMM_GEMV_VARIANT", variant)
     rng = np.random.default_rng(E * 1000 + n + k + t)
@@ -130,8 +130,11 @@ def test_grouped_iq4_many_pairs_per_expert(variant, E, n, k, t, topk, per_pair, 
         assert v.startswith("iq4_persist" if t * topk <= 4096 else "route+grouped_gemv_generic"), v
     elif variant == "iq4w":
         assert v.startswith("route+grouped_iq4_warp"), v
+    elif variant == "iq4t":
+        assert v.startswith("route+grouped_iq4_tile"), v
     else:
-        assert "iq4_stream" in v, v
+        # default: the tile-resident kernel when t * topk >= 4 E, else the streaming one
+        assert ("iq4_tile" if t * topk >= 4 * E else "iq4_stream") in v, v
     if per_pair:
         xs = x.reshape(t * topk, k)
         yref = np.empty((t * topk, n)); absy = np.empty((t * topk, n))
@@ -144,3 +147,38 @@ def test_grouped_iq4_many_pairs_per_expert(variant, E, n, k, t, topk, per_pair, 
     else:
         yref, absy = oracle.grouped_gemv(synth.FMT_IQ4_NL, n, k, p.data, p.data_stride, None, 0, 1.0, E, x, ids)
     check_tol(y, yref, absy, "grouped iq4 %s" % v)
+
+
+@pytest.mark.parametrize("spec", ["0", "1"])
+@pytest.mark.parametrize("tiles_per_item", ["2", "4"])
+@pytest.mark.parametrize("E,n,k,t,topk,per_pair", [(32, 1792, 2560, 64, 4, False), (32, 2560, 896, 64, 4, True),
+                                                    (32, 2560, 896, 1, 4, True), (7, 1000, 1152, 37, 3, False),
+                                                    (4, 72, 4096, 20, 2, False)])
+def test_grouped_iq4_tile_kernel(spec, tiles_per_item, E, n, k, t, topk, per_pair, monkeypatch):
+    """The tile-resident IQ4_NL kernel with its weight loads before and after
+    the dependency wait, two or four tiles per CTA at one super-step per warp
+    (k = 896, 1152), ragged last items (n = 1000, 72) and the routed-expert
+    shapes (gate+up 1792 x 2560, down 2560 x 896 at 64 and 1 tokens)."""
+    monkeypatch.setenv("QMM_GEMV_VARIANT", "iq4t")
+    monkeypatch.setenv("QMM_IQ4T_SPEC", spec)
+    monkeypatch.setenv("QMM_IQ4T_S", tiles_per_item)
+    rng = np.random.default_rng(E * 7 + n + k + t)
+    p = synth.gen_weights(rng, synth.FMT_IQ4_NL, n, k, experts=E)
+    x = synth.gen_x(rng, t, topk, k) if per_pair else synth.gen_x(rng, t, k)
+    ids = synth.gen_topk(rng, t, topk, E)
+    y, st = _grouped(dev(p), x, ids, per_pair)
+    v = qmm.qmm_last_variant()
+    assert st == 0 and v.startswith("route+grouped_iq4_tile"), v
+    if per_pair:
+        xs = x.reshape(t * topk, k)
+        yref = np.empty((t * topk, n)); absy = np.empty((t * topk, n))
+        for e in range(E):
+            sel = np.flatnonzero(ids.reshape(-1) == e)
+            if len(sel):
+                de = p.data[e * p.data_stride:(e + 1) * p.data_stride]
+                yref[sel], absy[sel] = oracle.matmul(synth.FMT_IQ4_NL, n, k, de, None, 1.0, xs[sel])
+        yref, absy = yref.reshape(t, topk, n), absy.reshape(t, topk, n)
+    else:
+        yref, absy = oracle.grouped_gemv(synth.FMT_IQ4_NL, n, k, p.data, p.data_stride, None, 0, 1.0, E, x, ids)
+    check_tol(y, yref, absy, "grouped iq4 tile %s" % v)
+
