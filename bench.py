@@ -242,8 +242,9 @@ def gemv_workload(p, x_bits, steps, warmup, world, l2, sampler=None, graph_len=1
 
 
 def gemv_e2e(p, x_bits, steps, world):
-    """Same GEMV through the public Python API with host buffers: pinned x
-    host->device, the call, y device->host, every step."""
+    """Same GEMV through the public API with host buffers (qmm_gemv_host):
+    pinned x host->device, the product, y device->host, every step, in one
+    library call per step."""
     import torch
     from packed_bit_weight_b200 import qmm
     w = qmm.PackedWeights.from_host(p)
@@ -253,16 +254,15 @@ def gemv_e2e(p, x_bits, steps, world):
     xd = torch.empty_like(xh, device="cuda")
     yd = torch.empty((m, p.n), dtype=torch.int16, device="cuda")
 
+    st = torch.cuda.current_stream()
+
     def step():
-        xd.copy_(xh, non_blocking=True)
-        qmm.qmm_gemv(w, xd, yd)
-        yh.copy_(yd, non_blocking=True)
+        qmm.qmm_gemv_host(w, xh, yh, xd, yd, stream=st)
 
     for _ in range(20):
         step()
     torch.cuda.synchronize()
     barrier(world)
-    st = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(st)
     for _ in range(steps):

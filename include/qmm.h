@@ -162,6 +162,26 @@ qmm_status qmm_quantize(int32_t fmt, const uint16_t* w, int64_t n, int64_t k, vo
 qmm_status qmm_gemv(const qmm_weights* w, const uint16_t* x, int64_t m, uint16_t* y, void* ws,
                     size_t ws_bytes, void* stream);
 
+/* qmm_gemv with host-resident activations and outputs, in one call (a
+ * serving step's whole round trip), enqueued on `stream`: x_host reaches
+ * x_dev, the product is formed, y lands in y_host.  Page-locked host buffers
+ * (cudaHostAlloc, torch pin_memory) are used in place through their device
+ * mapping: a copy kernel reads x_host into x_dev while the GEMV, launched
+ * with programmatic dependent launch, already streams W, and the GEMV stores
+ * y straight into y_host (y_dev is then unused).  Pageable buffers go through
+ * cudaMemcpyAsync (synchronous to the host) and y_dev.  y_host holds the
+ * result once the stream reaches the end of this call's work.
+ *   x_host  host, [m][k] fp16 (16-byte aligned for the in-place path)
+ *   y_host  host, [m][n] fp16 (16-byte aligned for the in-place path)
+ *   x_dev   device, [m][k] fp16 staging buffer (16-byte aligned)
+ *   y_dev   device, [m][n] fp16 staging buffer (16-byte aligned)
+ * The whole [m][k] and [m][n] ranges must lie in the buffers the caller
+ * passes (a page-locked range is read and written by the GPU directly).
+ * Errors: as qmm_gemv; CUDA when a copy cannot be enqueued (the kernel may
+ * then already be queued). */
+qmm_status qmm_gemv_host(const qmm_weights* w, const uint16_t* x_host, int64_t m, uint16_t* y_host,
+                         uint16_t* x_dev, uint16_t* y_dev, void* stream);
+
 /* The same product for a prefill window (m up to any size; the kernel is a
  * tensor-core GEMM that decodes weight tiles into shared memory).
  *   x       device, [m][k] fp16;  y device, [m][n] fp16

@@ -1016,6 +1016,64 @@ qmm_status qmm_gemv(const qmm_weights* w, const uint16_t* x, int64_t m, uint16_t
   }
 }
 
+// Device address of bytes [p, p + bytes) of page-locked host memory mapped
+// into the current device's address space (16-byte aligned), else nullptr
+// (pageable memory, or a range whose ends are not in the same mapping).
+static void* mapped_host_alias(const void* p, size_t bytes) {
+  if (!p || bytes == 0) return nullptr;
+  cudaPointerAttributes a, b;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  if (a.type != cudaMemoryTypeHost || !a.devicePointer || (reinterpret_cast<uintptr_t>(a.devicePointer) & 15u))
+    return nullptr;
+  const char* last = static_cast<const char*>(p) + bytes - 1;
+  if (cudaPointerGetAttributes(&b, last) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  if (b.type != cudaMemoryTypeHost || !b.devicePointer ||
+      static_cast<char*>(b.devicePointer) - static_cast<char*>(a.devicePointer) != (ptrdiff_t)(bytes - 1))
+    return nullptr;
+  return a.devicePointer;
+}
+
+qmm_status qmm_gemv_host(const qmm_weights* w, const uint16_t* x_host, int64_t m, uint16_t* y_host, uint16_t* x_dev,
+                         uint16_t* y_dev, void* stream) {
+  qmm_status s = check_weights(w, false);
+  if (s != QMM_OK) return s;
+  if (m < 0) return QMM_ERR_INVALID_ARG;
+  if (m > 16) return QMM_ERR_UNSUPPORTED_SHAPE;
+  if (m == 0 || w->n == 0) return QMM_OK;
+  if (!y_host || !y_dev || (w->k > 0 && (!x_host || !x_dev))) return QMM_ERR_INVALID_ARG;
+  if (!aligned16(y_dev) || (x_dev && !aligned16(x_dev))) return QMM_ERR_MISALIGNED;  // before anything is queued
+  DevInfo* di = nullptr;
+  if ((s = device_info(&di)) != QMM_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t xb = 2 * (size_t)m * (size_t)w->k, yb = 2 * (size_t)m * (size_t)w->n;
+  // Page-locked host buffers are used in place through their device mapping:
+  // a copy kernel brings x in (the GEMV's weight stream starts meanwhile) and
+  // the GEMV stores y straight to host memory.  Pageable buffers go through
+  // the copy engine.
+  const void* xa = mapped_host_alias(x_host, xb);
+  void* ya = mapped_host_alias(y_host, yb);
+  if (xb) {
+    if (xa && xb % 16 == 0) {
+      const int64_t n16 = (int64_t)(xb / 16);
+      fetch16_kernel<<<(unsigned)std::min<int64_t>((n16 + 255) / 256, di->sms), 256, 0, st>>>(
+          static_cast<const uint4*>(xa), reinterpret_cast<uint4*>(x_dev), n16);
+      if (cudaGetLastError() != cudaSuccess) return QMM_ERR_CUDA;
+    } else if (cudaMemcpyAsync(x_dev, x_host, xb, cudaMemcpyHostToDevice, st) != cudaSuccess) {
+      return QMM_ERR_CUDA;
+    }
+  }
+  if (ya) return qmm_gemv(w, x_dev, m, static_cast<uint16_t*>(ya), nullptr, 0, stream);
+  if ((s = qmm_gemv(w, x_dev, m, y_dev, nullptr, 0, stream)) != QMM_OK) return s;
+  if (cudaMemcpyAsync(y_host, y_dev, yb, cudaMemcpyDeviceToHost, st) != cudaSuccess) return QMM_ERR_CUDA;
+  return QMM_OK;
+}
+
 qmm_status qmm_gemm(const qmm_weights* w, const uint16_t* x, int64_t m, uint16_t* y, void* ws, size_t ws_bytes,
                     void* stream) {
   (void)ws;

@@ -61,6 +61,7 @@ def _lib():
             "qmm_dequant": (i32, [W, vp, vp]),
             "qmm_quantize": (i32, [i32, vp, i64, i64, vp, vp, vp]),
             "qmm_gemv": (i32, [W, vp, i64, vp, vp, sz, vp]),
+            "qmm_gemv_host": (i32, [W, vp, i64, vp, vp, vp, vp]),
             "qmm_gemm": (i32, [W, vp, i64, vp, vp, sz, vp]),
             "qmm_route": (i32, [vp, i64, i64, i64, vp, vp, vp, sz, vp]),
             "qmm_grouped_gemv": (i32, [W, vp, i32, vp, i64, i64, vp, vp, sz, vp]),
@@ -121,6 +122,18 @@ class PackedWeights:
     scale_stride: int | None = None
 
     def desc(self) -> qmm_weights:
+        """The C descriptor, rebuilt only when a field or a buffer changed."""
+        key = (self.fmt, self.n, self.k, None if self.data is None else self.data.data_ptr(),
+               None if self.scales is None else self.scales.data_ptr(), self.global_scale, self.experts,
+               self.data_stride, self.scale_stride)
+        cached = self.__dict__.get("_desc")
+        if cached is not None and cached[0] == key:
+            return cached[1]
+        d = self._build_desc()
+        self.__dict__["_desc"] = (key, d)
+        return d
+
+    def _build_desc(self) -> qmm_weights:
         d = qmm_weights()
         d.fmt, d.reserved, d.n, d.k = self.fmt, 0, self.n, self.k
         d.data = ctypes.c_void_p(self.data.data_ptr()) if self.data is not None else None
@@ -219,6 +232,28 @@ def qmm_gemv(w: PackedWeights, x: torch.Tensor, y: torch.Tensor, ws: torch.Tenso
     m = x.shape[0] if x.dim() == 2 else 1
     _check(_lib().qmm_gemv(ctypes.byref(d), _ptr(x, 2, "x"), m, _ptr(y, 2, "y"), wp, wb, _stream(stream)), "qmm_gemv")
     return y
+
+
+def _host_ptr(t: torch.Tensor, esize: int, name: str):
+    if t.is_cuda:
+        raise ValueError("%s must be a host tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if t.element_size() != esize:
+        raise ValueError("%s must have %d-byte elements" % (name, esize))
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def qmm_gemv_host(w: PackedWeights, x_host: torch.Tensor, y_host: torch.Tensor, x_dev: torch.Tensor,
+                  y_dev: torch.Tensor, stream=None) -> torch.Tensor:
+    """qmm_gemv on host tensors in one library call: x_host -> x_dev, the
+    product into y_dev, y_dev -> y_host, enqueued on the stream (asynchronous
+    when the host tensors are pinned)."""
+    d = w.desc()
+    m = x_host.shape[0] if x_host.dim() == 2 else 1
+    _check(_lib().qmm_gemv_host(ctypes.byref(d), _host_ptr(x_host, 2, "x_host"), m, _host_ptr(y_host, 2, "y_host"),
+                                _ptr(x_dev, 2, "x_dev"), _ptr(y_dev, 2, "y_dev"), _stream(stream)), "qmm_gemv_host")
+    return y_host
 
 
 def qmm_gemm(w: PackedWeights, x: torch.Tensor, y: torch.Tensor, ws: torch.Tensor | None = None,

@@ -247,3 +247,49 @@ def test_mxfp4_huge_scales_overflow_like_the_oracle(variant, monkeypatch):
     assert np.array_equal(np.isnan(y[big]), np.isnan(yref[big]))
     nn = big & ~np.isnan(yref)
     assert np.array_equal(y[nn], yref[nn])      # +-inf, same sign
+
+
+@pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_IQ4_NL, synth.FMT_MXFP4])
+@pytest.mark.parametrize("pinned", [True, False])
+def test_gemv_host_round_trip(fmt, pinned):
+    """qmm_gemv_host: host x in, host y out in one call, the same result as
+    qmm_gemv on device buffers (bit-exact) and within tolerance of the
+    oracle."""
+    n, k, m = 1000, 4096, 3
+    p, x = _case(fmt, n, k, m, 5000 + fmt)
+    w = dev(p)
+    xh = torch.from_numpy(x.view(np.int16).copy())
+    yh = torch.full((m, n), 0x5A5A, dtype=torch.int16)
+    if pinned:
+        xh, yh = xh.pin_memory(), yh.pin_memory()
+    xd = torch.empty((m, k), dtype=torch.int16, device="cuda")
+    yd = torch.empty((m, n), dtype=torch.int16, device="cuda")
+    qmm.qmm_gemv_host(w, xh, yh, xd, yd)
+    torch.cuda.synchronize()
+    assert qmm.qmm_sync_check() == 0
+    got = yh.numpy().view(np.uint16)
+    yref_dev = run_gemv(w, x)
+    assert np.array_equal(got, yref_dev)
+    yref, absy = oracle.matmul(fmt, n, k, p.data, p.scales, p.global_scale, x)
+    check_tol(got, yref, absy, "gemv_host %d" % fmt)
+
+
+def test_gemv_host_argument_errors():
+    p, x = _case(synth.FMT_FP4G16_F16, 64, 256, 2, 9)
+    w = dev(p)
+    xh = torch.from_numpy(x.view(np.int16).copy())
+    yh = torch.empty((2, 64), dtype=torch.int16)
+    xd = torch.empty((2, 256), dtype=torch.int16, device="cuda")
+    yd = torch.empty((2, 64), dtype=torch.int16, device="cuda")
+    with pytest.raises(ValueError):
+        qmm.qmm_gemv_host(w, xd, yh, xd, yd)                  # device tensor as the host input
+    with pytest.raises(ValueError):
+        qmm.qmm_gemv_host(w, xh, yh, xh, yd)                  # host tensor as the device staging buffer
+    big = torch.zeros((17, 256), dtype=torch.int16)
+    with pytest.raises(qmm.QmmError) as e:
+        qmm.qmm_gemv_host(w, big, torch.empty((17, 64), dtype=torch.int16), torch.empty((17, 256), dtype=torch.int16,
+                          device="cuda"), torch.empty((17, 64), dtype=torch.int16, device="cuda"))
+    assert e.value.status == 2                                  # m > 16: UNSUPPORTED_SHAPE
+    with pytest.raises(qmm.QmmError) as e:
+        qmm.qmm_gemv_host(w, xh, yh, xd, torch.zeros((2 * 64 + 8,), dtype=torch.int16, device="cuda")[1:129])
+    assert e.value.status == 3                                  # misaligned y staging buffer
