@@ -7,7 +7,7 @@
 // IQ4_NL product (one "expert", m tokens in order).
 //
 // One CTA per work item = (expert, S sources): with IQ_SWIGLU the gate and
-// the up tile of the same 16 rows (S = 2), otherwise S neighbouring 16-row
+// up tiles of S/2 neighbouring 16-row tiles, otherwise S neighbouring 16-row
 // tiles of the matrix.  The CTA's WPC warps split k into ranges of SPW
 // super-steps (128 k = four 18-byte blocks per row); in a super-step lane
 // (grp, tig) owns block 4s + tig of rows grp and grp+8 of every source.  Each
@@ -42,7 +42,6 @@
 
 namespace qmm {
 
-constexpr int kIqtMaxWarps = 16;
 constexpr int kIqtGroup = 16;  // token slots per pass (two MMA n-tiles)
 
 struct IqtArgs {
@@ -164,9 +163,13 @@ __device__ __forceinline__ void iqt_load(uint32_t (&w)[SPW][S][2][6], const uint
   }
 }
 
+// Threads a CTA of this register budget may have.
+__host__ __device__ constexpr int iqt_max_threads(int maxreg) { return (65536 / maxreg) & ~31; }
+
 template <int MODE, int S, int SPW, int MAXREG, bool W16>
-__global__ void __launch_bounds__(kIqtMaxWarps * 32) __maxnreg__(MAXREG) iq4_tile_kernel(const IqtArgs a) {
-  static_assert(MODE != IQ_SWIGLU || S == 2, "SwiGLU items are a gate and an up tile");
+__global__ void __launch_bounds__(iqt_max_threads(MAXREG)) __maxnreg__(MAXREG) iq4_tile_kernel(const IqtArgs a) {
+  static_assert(MODE != IQ_SWIGLU || S % 2 == 0, "SwiGLU items are gate and up tiles of the same rows");
+  constexpr int kOut = (MODE == IQ_SWIGLU) ? S / 2 : S;  // output tiles per item
   extern __shared__ __align__(16) uint8_t smem_iqt[];
   const uint32_t lut = smem_addr(smem_iqt);
   float* red = reinterpret_cast<float*>(smem_iqt + kIqLutBytes);  // [warp][source][slot][row]
@@ -191,9 +194,9 @@ __global__ void __launch_bounds__(kIqtMaxWarps * 32) __maxnreg__(MAXREG) iq4_til
 #pragma unroll
   for (int s = 0; s < S; s++) {
     const uint8_t* base;
-    if (MODE == IQ_SWIGLU) {
-      row0[s] = item * 16;
-      base = (s ? a.data1 + (int64_t)e * a.dstride1 : a.data0 + (int64_t)e * a.dstride0);
+    if (MODE == IQ_SWIGLU) {  // sources 2q, 2q+1: gate and up of output tile q
+      row0[s] = (item * kOut + (s >> 1)) * 16;
+      base = ((s & 1) ? a.data1 + (int64_t)e * a.dstride1 : a.data0 + (int64_t)e * a.dstride0);
     } else {
       row0[s] = (item * S + s) * 16;
       base = a.data0 + (int64_t)e * a.dstride0;
@@ -256,15 +259,15 @@ __global__ void __launch_bounds__(kIqtMaxWarps * 32) __maxnreg__(MAXREG) iq4_til
       }
     }
     __syncthreads();
-    constexpr int kOut = (MODE == IQ_SWIGLU) ? 1 : S;  // output tiles per item
     for (int idx = threadIdx.x; idx < kOut * 16 * ng; idx += blockDim.x) {
-      const int row = idx & 15, slot = (idx >> 4) % ng, s = (idx >> 4) / ng;
-      const int grow = row0[0] + s * 16 + row;
+      const int row = idx & 15, slot = (idx >> 4) % ng, q = (idx >> 4) / ng;
+      const int grow = (item * kOut + q) * 16 + row;
       if (grow >= a.n) continue;
+      const int sv = (MODE == IQ_SWIGLU) ? 2 * q : q;  // source of the value (the gate for SwiGLU)
       float v = 0.f, u = 0.f;
       for (int wi = 0; wi < wpc; wi++) {
-        v += red[((wi * S + s) * kIqtGroup + slot) * 16 + row];
-        if (MODE == IQ_SWIGLU) u += red[((wi * S + 1) * kIqtGroup + slot) * 16 + row];
+        v += red[((wi * S + sv) * kIqtGroup + slot) * 16 + row];
+        if (MODE == IQ_SWIGLU) u += red[((wi * S + sv + 1) * kIqtGroup + slot) * 16 + row];
       }
       const int64_t pr = a.offsets ? a.perm[start + g0 + slot] : g0 + slot;
       if (MODE == IQ_SCALED_F32) {

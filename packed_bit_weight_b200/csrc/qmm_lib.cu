@@ -701,7 +701,9 @@ static qmm_status launch_iq4_tile_cfg(const qmm_weights* w0, const qmm_weights* 
                                       int m_plain, void* y, const float* gw, cudaStream_t st) {
   const int steps = (int)(w0->k / 128), wpc = steps / SPW;
   const int64_t tiles = (w0->n + 15) / 16;
-  const int64_t ipe = (MODE == IQ_SWIGLU) ? tiles : (tiles + S - 1) / S;
+  constexpr int kOut = (MODE == IQ_SWIGLU) ? S / 2 : S;  // output tiles per item
+  const int64_t ipe = (tiles + kOut - 1) / kOut;
+  if (wpc * 32 > iqt_max_threads(kMaxReg)) return QMM_ERR_UNSUPPORTED_SHAPE;
   const int64_t E = offsets ? w0->num_experts : 1;
   const int64_t grid = E * ipe;
   if (grid < 1 || grid > INT32_MAX) return QMM_ERR_UNSUPPORTED_SHAPE;
@@ -755,20 +757,18 @@ static qmm_status launch_iq4_tile(const qmm_weights* w0, const qmm_weights* w1, 
   const int64_t k = w0->k, n = w0->n;
   if (k % 128 || k < 128 || n < 1 || n > INT32_MAX / 2) return QMM_ERR_UNSUPPORTED_SHAPE;
   const int64_t steps = k / 128;
-  // registers: 96 keeps two CTAs of up to 10 warps (three of 7) per SM
-  if (steps % 2 == 0 && steps / 2 <= kIqtMaxWarps)  // k % 256 == 0: rows 16-byte aligned
+  // Items of S tiles (sources) whose activation fragments are shared; each
+  // warp holds S * SPW blocks per row pair in registers.  k % 256 == 0 (rows
+  // 16-byte aligned): two tiles, two super-steps per warp, 96 registers (two
+  // CTAs of up to 10 warps per SM).  Otherwise four tiles, one super-step per
+  // warp, 128 registers.  Four tiles at one super-step per warp for k = 2560
+  // would need 20 warps of ~128 registers (more than an SM holds).
+  if (steps % 2 == 0 && steps / 2 <= iqt_max_threads(96) / 32)
     return launch_iq4_tile_cfg<MODE, 2, 2, 96, true>(w0, w1, x, x_per_pair, topk, offsets, perm, P, m_plain, y, gw,
                                                      st);
-  if (steps <= kIqtMaxWarps) {
-    const char* e = getenv("QMM_IQ4T_S");  // measurement knob: tiles per item at one super-step per warp
-    if constexpr (MODE != IQ_SWIGLU) {
-      if (!(e && e[0] == '2'))
-        return launch_iq4_tile_cfg<MODE, 4, 1, 128, false>(w0, w1, x, x_per_pair, topk, offsets, perm, P, m_plain, y,
-                                                           gw, st);
-    }
-    return launch_iq4_tile_cfg<MODE, 2, 1, 96, false>(w0, w1, x, x_per_pair, topk, offsets, perm, P, m_plain, y, gw,
-                                                      st);
-  }
+  if (steps <= iqt_max_threads(128) / 32)
+    return launch_iq4_tile_cfg<MODE, 4, 1, 128, false>(w0, w1, x, x_per_pair, topk, offsets, perm, P, m_plain, y, gw,
+                                                       st);
   return QMM_ERR_UNSUPPORTED_SHAPE;
 }
 

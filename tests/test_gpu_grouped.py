@@ -150,18 +150,17 @@ def test_grouped_iq4_many_pairs_per_expert(variant, E, n, k, t, topk, per_pair, 
 
 
 @pytest.mark.parametrize("spec", ["0", "1"])
-@pytest.mark.parametrize("tiles_per_item", ["2", "4"])
 @pytest.mark.parametrize("E,n,k,t,topk,per_pair", [(32, 1792, 2560, 64, 4, False), (32, 2560, 896, 64, 4, True),
                                                     (32, 2560, 896, 1, 4, True), (7, 1000, 1152, 37, 3, False),
                                                     (4, 72, 4096, 20, 2, False)])
-def test_grouped_iq4_tile_kernel(spec, tiles_per_item, E, n, k, t, topk, per_pair, monkeypatch):
+def test_grouped_iq4_tile_kernel(spec, E, n, k, t, topk, per_pair, monkeypatch):
     """The tile-resident IQ4_NL kernel with its weight loads before and after
-    the dependency wait, two or four tiles per CTA at one super-step per warp
-    (k = 896, 1152), ragged last items (n = 1000, 72) and the routed-expert
-    shapes (gate+up 1792 x 2560, down 2560 x 896 at 64 and 1 tokens)."""
+    the dependency wait, items of two tiles (two super-steps per warp, k %
+    256 == 0) or four (one super-step per warp: k = 896, 1152), ragged last
+    items (n = 1000, 72) and the routed-expert shapes (gate+up 1792 x 2560,
+    down 2560 x 896 at 64 and 1 tokens)."""
     monkeypatch.setenv("QMM_GEMV_VARIANT", "iq4t")
     monkeypatch.setenv("QMM_IQ4T_SPEC", spec)
-    monkeypatch.setenv("QMM_IQ4T_S", tiles_per_item)
     rng = np.random.default_rng(E * 7 + n + k + t)
     p = synth.gen_weights(rng, synth.FMT_IQ4_NL, n, k, experts=E)
     x = synth.gen_x(rng, t, topk, k) if per_pair else synth.gen_x(rng, t, k)
