@@ -177,6 +177,15 @@ __global__ void __launch_bounds__(iqt_max_threads(MAXREG)) __maxnreg__(MAXREG) i
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, grp = lane >> 2, tig = lane & 3;
   const int e = blockIdx.x / a.items_per_expert, item = blockIdx.x - e * a.items_per_expert;
   pdl_launch_dependents();
+  int start = 0, cnt = a.m_plain;
+  if (!a.spec) {  // most experts may be empty: find out before any other work
+    pdl_wait();
+    if (a.offsets) {
+      start = a.offsets[e];
+      cnt = a.offsets[e + 1] - start;
+    }
+    if (cnt <= 0) return;
+  }
   // pair table: entry v (an index byte) = (kv[v & 15], kv[v >> 4]) as f16x2,
   // one copy per bank; each store covers four banks
   for (int i = threadIdx.x; i < 256 * 8; i += blockDim.x) {
@@ -206,15 +215,17 @@ __global__ void __launch_bounds__(iqt_max_threads(MAXREG)) __maxnreg__(MAXREG) i
   }
   const int s0 = warp * SPW;
   uint32_t w[SPW][S][2][6];
-  if (a.spec) iqt_load<S, SPW, W16>(w, rp, s0, tig);
-  pdl_wait();  // routing, activations and the output buffer follow the previous kernel
-  int start = 0, cnt = a.m_plain;
-  if (a.offsets) {
-    start = a.offsets[e];
-    cnt = a.offsets[e + 1] - start;
+  if (a.spec) {
+    iqt_load<S, SPW, W16>(w, rp, s0, tig);
+    pdl_wait();  // routing, activations and the output buffer follow the previous kernel
+    if (a.offsets) {
+      start = a.offsets[e];
+      cnt = a.offsets[e + 1] - start;
+    }
+    if (cnt <= 0) return;  // the whole CTA: an expert without pairs
+  } else {
+    iqt_load<S, SPW, W16>(w, rp, s0, tig);
   }
-  if (cnt <= 0) return;  // the whole CTA: an expert without pairs
-  if (!a.spec) iqt_load<S, SPW, W16>(w, rp, s0, tig);
   __syncthreads();  // the pair table is complete
   const uint32_t lut_lane = lut + 4u * lane;
 

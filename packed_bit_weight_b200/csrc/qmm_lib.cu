@@ -1179,9 +1179,10 @@ qmm_status qmm_grouped_gemv(const qmm_weights* experts, const uint16_t* x, int32
     set_variant("route+zero_fill");
     return launch_status();
   }
-  // IQ4_NL: the tile-resident kernel when most experts have pairs (its
-  // weight loads then overlap the routing pass), else the streaming kernel
-  const bool iq4_tile = pick == 10 || (pick == 0 && P >= 4 * experts->num_experts);
+  // IQ4_NL: the tile-resident kernel (its weight loads overlap the routing
+  // pass when most experts have pairs); QMM_GEMV_VARIANT=iq4 keeps the
+  // streaming kernel
+  const bool iq4_tile = pick == 10 || pick == 0;
   if (experts->fmt == QMM_FMT_IQ4_NL && iq4_tile) {
     s = launch_iq4_tile<IQ_OUT_F16>(experts, nullptr, x, x_per_pair, topk, offsets, perm, P, 0, y, nullptr, st);
     if (s != QMM_ERR_UNSUPPORTED_SHAPE) {
@@ -1334,10 +1335,10 @@ qmm_status qmm_moe_routed(const qmm_weights* gate, const qmm_weights* up, const 
     set_variant("moe:route+zero_fill");
     return launch_status();
   }
-  // tile-resident kernels when most experts have pairs (measured faster at
-  // 64 tokens, slower at 1), else the streaming kernels
+  // tile-resident kernels (measured faster than the streaming ones at 1, 4,
+  // 16 and 64 tokens); QMM_GEMV_VARIANT=iq4 keeps the streaming kernels
   const int pick = gemv_variant_env();
-  if (pick == 10 || (pick == 0 && P >= 4 * E)) {
+  if (pick == 10 || pick == 0) {
     s = launch_iq4_tile<IQ_SWIGLU>(gate, up, x, 0, topk, offsets, perm, P, 0, h, nullptr, st);
     if (s == QMM_OK)
       s = launch_iq4_tile<IQ_SCALED_F32>(down, nullptr, h, 1, topk, offsets, perm, P, 0, yg, topk_weights, st);

@@ -108,13 +108,13 @@ def test_grouped_rejects_small_workspace():
     assert e.value.status == 8
 
 
-@pytest.mark.parametrize("variant", [None, "iq4p", "iq4w", "iq4t"])
+@pytest.mark.parametrize("variant", [None, "iq4", "iq4p", "iq4w", "iq4t"])
 @pytest.mark.parametrize("E,n,k,t,topk,per_pair", [(3, 64, 256, 50, 2, False), (5, 48, 384, 200, 3, True),
                                                     (2, 16, 128, 2100, 2, False), (32, 32, 128, 1, 4, True)])
 def test_grouped_iq4_many_pairs_per_expert(variant, E, n, k, t, topk, per_pair, monkeypatch):
     """IQ4_NL experts with more than 16 pairs each (several token groups per
-    expert, whose row tiles land on different CTAs), with the default kernel
-    (tile-resident, or streaming when t * topk < 4 E) and the opt-in ones;
+    expert, whose row tiles land on different CTAs), with the default
+    (tile-resident) kernel and the opt-in ones;
     t * topk = 4200 is past the persistent kernel's pair limit (a forced
     variant that does not take a shape leaves it to the generic kernel)."""
     if variant:
@@ -132,9 +132,10 @@ def test_grouped_iq4_many_pairs_per_expert(variant, E, n, k, t, topk, per_pair, 
         assert v.startswith("route+grouped_iq4_warp"), v
     elif variant == "iq4t":
         assert v.startswith("route+grouped_iq4_tile"), v
+    elif variant == "iq4":
+        assert v.startswith("route+grouped_iq4_stream"), v
     else:
-        # default: the tile-resident kernel when t * topk >= 4 E, else the streaming one
-        assert ("iq4_tile" if t * topk >= 4 * E else "iq4_stream") in v, v
+        assert "iq4_tile" in v, v  # default: the tile-resident kernel
     if per_pair:
         xs = x.reshape(t * topk, k)
         yref = np.empty((t * topk, n)); absy = np.empty((t * topk, n))

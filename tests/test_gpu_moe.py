@@ -141,13 +141,13 @@ def _moe_reference_stages(wgu, wdn, x, ids, g, f, h_gpu):
     return h_ref, h_bound, out_ref, out_abs
 
 
-@pytest.mark.parametrize("variant", [None, "iq4p", "iq4w", "iq4t"])
+@pytest.mark.parametrize("variant", [None, "iq4", "iq4p", "iq4w", "iq4t"])
 @pytest.mark.parametrize("E,f,d,t,topk", [(6, 128, 256, 9, 2), (4, 256, 128, 40, 4), (2, 128, 384, 5, 2),
                                           (32, 896, 2560, 64, 4), (32, 896, 2560, 1, 4)])
 def test_moe_routed_vs_oracle(E, f, d, t, topk, variant, monkeypatch):
-    """Default: route + tile-resident kernels when t * topk >= 4 E, else route
-    + streaming kernels; iq4p: the persistent kernels (each buckets the ids
-    itself); iq4w, iq4t: the warp-per-tile and tile-resident kernels."""
+    """Default (and iq4t): route + tile-resident kernels; iq4: route +
+    streaming kernels; iq4p: the persistent kernels (each buckets the ids
+    itself); iq4w: the warp-per-tile kernels."""
     if variant:
         monkeypatch.setenv("QMM_GEMV_VARIANT", variant)
     rng = np.random.default_rng(E * 31 + f + d + t)
@@ -160,7 +160,7 @@ def test_moe_routed_vs_oracle(E, f, d, t, topk, variant, monkeypatch):
     assert st == 0, used
     assert ("iq4_persist" in used) == (variant == "iq4p"), used
     assert ("iq4_warp" in used) == (variant == "iq4w"), used
-    assert ("iq4_tile" in used) == (variant == "iq4t" or (variant is None and t * topk >= 4 * E)), used
+    assert ("iq4_tile" in used) == (variant in ("iq4t", None)), used
     variant = used
     h_ref, h_bound, out_ref, out_abs = _moe_reference_stages(wgu, wdn, x, ids, g, f, h)
     err = np.abs(f16(h) - h_ref)
