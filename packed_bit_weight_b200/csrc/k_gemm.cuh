@@ -368,16 +368,25 @@ __device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint32_t bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 
-template <int FMT, int BN, int STAGES>
+// MH = 2: tiles of 256 tokens x BN = 128 weight rows, two M=128 MMAs per k16
+// step that share the decoded weight tile and accumulate into two halves of
+// the accumulator: half the weight decode per FLOP of MH = 1 (128 x 256),
+// the same tensor memory (2 accumulators x 256 columns) and operand bytes
+// per stage (32 + 16 KB instead of 16 + 32 KB).  Decode thread t then owns
+// 32 of the 64 k of row t % 128.
+template <int FMT, int BN, int STAGES, int MH = 1>
 __global__ void __launch_bounds__(kGemmPThreads, 1)
     gemm_fp4_tc_persistent_kernel(const __grid_constant__ CUtensorMap tm_x, const uint8_t* __restrict__ codes,
                                   const uint8_t* __restrict__ scales, uint16_t* __restrict__ y, int m, int n, int k,
                                   float g) {
   using C = GemmCfg<BN, STAGES>;
+  static_assert(MH == 1 || (MH == 2 && BN * MH == kGemmDecodeThreads), "one decode thread per row half");
+  constexpr uint32_t kA = MH * C::kABytes;  // X bytes per stage
+  constexpr int kBM = MH * kGemmBM;         // tokens per tile
   extern __shared__ uint8_t smem_raw[];
   const uint32_t base = (smem_addr(smem_raw) + 1023u) & ~1023u;
   const uint32_t a_s = base;
-  const uint32_t b_s = a_s + STAGES * C::kABytes;
+  const uint32_t b_s = a_s + STAGES * kA;
   const uint32_t p_s = b_s + STAGES * C::kBBytes;            // 2 staged packed chunks
   const uint32_t bars = p_s + 2 * kStageBytes;                // full[S] empty[S] accf[2] acce[2] done cf[2] ce[2]
   const uint32_t accf = bars + 8 * (2 * STAGES), acce = accf + 16, done_bar = acce + 16;
@@ -388,7 +397,7 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_tiles = (n + BN - 1) / BN;
-  const int tiles = ((m + kGemmBM - 1) / kGemmBM) * n_tiles;
+  const int tiles = ((m + kBM - 1) / kBM) * n_tiles;
   const int ksteps = k / kGemmBK;
   const int G = (int)gridDim.x;
   const int my_tiles = (tiles - (int)blockIdx.x + G - 1) / G;
@@ -411,7 +420,7 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 2 * BN);
+    tmem_alloc(tmem_slot, 2 * MH * BN);
     tmem_relinquish();
   }
   if (FMT == 1) {  // IQ4_NL pair table, 4 interleaved copies, in staging slot 0's spare tail
@@ -434,13 +443,13 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
       int gs = 0, issued = 0;
       for (int li = 0; li < my_tiles && !s_abort; li++) {
         const int tile = (int)blockIdx.x + li * G;
-        const int m0 = (tile / n_tiles) * kGemmBM;
+        const int m0 = (tile / n_tiles) * kBM;
         for (int ks = 0; ks < ksteps; ks++, gs++) {
           const int s = gs % STAGES;
           const uint32_t ph = (uint32_t)(gs / STAGES) & 1u;
           if (s_abort || !mbar_wait(bars + 8 * (STAGES + s), ph ^ 1u)) { s_abort = 1; break; }
-          mbar_arrive_expect_tx(bars + 8 * s, C::kABytes);
-          tma_load_2d(a_s + s * C::kABytes, &tm_x, ks * kGemmBK, m0, bars + 8 * s);
+          mbar_arrive_expect_tx(bars + 8 * s, kA);
+          tma_load_2d(a_s + s * kA, &tm_x, ks * kGemmBK, m0, bars + 8 * s);  // box of kBM rows
           issued = gs + 1;
         }
       }
@@ -461,18 +470,20 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
         const int a = li & 1;
         if (!mbar_wait(acce + 8 * a, (((uint32_t)li >> 1) & 1u) ^ 1u)) { s_abort = 1; break; }
         tc_fence_after();
-        const uint32_t d = tmem + (uint32_t)(a * BN);
+        const uint32_t d = tmem + (uint32_t)(a * MH * BN);
         bool ok = true;
         for (int ks = 0; ks < ksteps; ks++, gs++) {
           const int s = gs % STAGES;
           const uint32_t ph = (uint32_t)(gs / STAGES) & 1u;
           if (s_abort || !mbar_wait(bars + 8 * s, ph)) { s_abort = 1; ok = false; break; }
           tc_fence_after();
-          const uint64_t da = umma_desc_k128(a_s + s * C::kABytes);
           const uint64_t db = umma_desc_k128(b_s + s * C::kBBytes);
 #pragma unroll
           for (int kk = 0; kk < kGemmBK / 16; kk++)
-            umma_f16(d, da + (uint64_t)(2 * kk), db + (uint64_t)(2 * kk), idesc, (ks | kk) != 0);
+#pragma unroll
+            for (int h = 0; h < MH; h++)  // M-half h: X rows 128h.. of the stage, accumulator columns h*BN..
+              umma_f16(d + (uint32_t)(h * BN), umma_desc_k128(a_s + s * kA + h * C::kABytes) + (uint64_t)(2 * kk),
+                       db + (uint64_t)(2 * kk), idesc, (ks | kk) != 0);
           umma_commit(bars + 8 * (STAGES + s));
         }
         if (!ok) break;
@@ -486,6 +497,7 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
     // threads per 128-byte row piece of codes, so a warp instruction touches
     // 4 cache lines) into a 2-slot staging ring; thread t then decodes row t.
     const int t = threadIdx.x - 64;
+    const int rt = t % BN, hf = t / BN;  // row of the tile; with MH = 2 the 32-k half of each step
     const int nck = ksteps / kGemmChunkSteps;  // chunks per tile
     const int total_ck = my_tiles * nck;
     const int64_t crow = k >> 1, srow = k >> 4;
@@ -499,8 +511,9 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
       if (FMT == 1) {  // IQ4_NL: 256 rows x 9 units of 16 bytes (8 blocks of 18 bytes)
         const int64_t rowb = (int64_t)(k >> 5) * 18;
 #pragma unroll
-        for (int i = 0; i < 9; i++) {
+        for (int i = 0; i < (9 * BN + kGemmDecodeThreads - 1) / kGemmDecodeThreads; i++) {
           const int pc = i * kGemmDecodeThreads + t;
+          if (pc >= 9 * BN) break;
           const int r = pc / 9, u = pc - r * 9;
           const int64_t gr = min((int64_t)n0 + r, (int64_t)n - 1);
           cp_async16_g(dst + r * kStageIq4Row + u * 16, codes + gr * rowb + (int64_t)(kc >> 5) * 18 + u * 16);
@@ -509,7 +522,7 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
         return true;
       }
 #pragma unroll
-      for (int i = 0; i < 8; i++) {  // codes: 256 rows x 8 units of 16 bytes
+      for (int i = 0; i < 8 * BN / kGemmDecodeThreads; i++) {  // codes: BN rows x 8 units of 16 bytes
         const int pc = i * kGemmDecodeThreads + t;
         const int r = pc >> 3, u = pc & 7;
         const int64_t gr = min((int64_t)n0 + r, (int64_t)n - 1);
@@ -517,7 +530,7 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
       }
       if (FMT == 2) {
 #pragma unroll
-        for (int i = 0; i < 2; i++) {  // scales: 256 rows x 2 halves of 16 bytes
+        for (int i = 0; i < 2 * BN / kGemmDecodeThreads; i++) {  // scales: BN rows x 2 halves of 16 bytes
           const int pc = i * kGemmDecodeThreads + t;
           const int r = pc >> 1, h = pc & 1;
           const int64_t gr = min((int64_t)n0 + r, (int64_t)n - 1);
@@ -527,11 +540,11 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
       } else if (FMT == 4) {  // MXFP4: 8 E8M0 bytes per row (one per 32 k)
         const int r = t;
         const int64_t gr = min((int64_t)n0 + r, (int64_t)n - 1);
-        cp_async8_g(dst + kStageCodes + r * 32, scales + gr * (srow >> 1) + (kc >> 5));
+        if (r < BN) cp_async8_g(dst + kStageCodes + r * 32, scales + gr * (srow >> 1) + (kc >> 5));
       } else {  // E4M3: 16 bytes per row, copied whole; words read swizzled
         const int r = t;
         const int64_t gr = min((int64_t)n0 + r, (int64_t)n - 1);
-        cp_async16_g(dst + kStageCodes + r * 32, scales + gr * srow + (kc >> 4));
+        if (r < BN) cp_async16_g(dst + kStageCodes + r * 32, scales + gr * srow + (kc >> 4));
       }
       cp_async_mbar_arrive_noinc(cfull + 8 * slot);
       return true;
@@ -543,7 +556,7 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
       const int slot = c & 1;
       if (s_abort || !mbar_wait(cfull + 8 * slot, ((uint32_t)c >> 1) & 1u)) { s_abort = 1; break; }
       const int tile = (int)blockIdx.x + (c / nck) * G;
-      const bool valid = (int64_t)(tile % n_tiles) * BN + t < n;
+      const bool valid = (int64_t)(tile % n_tiles) * BN + rt < n;
       const uint32_t src = p_s + slot * kStageBytes;
       for (int j = 0; j < kGemmChunkSteps; j++, gs++) {
         const int s = gs % STAGES;
@@ -552,7 +565,7 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
           // this row's two blocks of step j: 36 bytes from byte 36j of the row
           uint32_t w[9];
 #pragma unroll
-          for (int i = 0; i < 9; i++) w[i] = lds32(src + t * kStageIq4Row + j * 36 + 4 * i);
+          for (int i = 0; i < 9; i++) w[i] = lds32(src + rt * kStageIq4Row + j * 36 + 4 * i);
           uint32_t qa[4], qb[4];
 #pragma unroll
           for (int i = 0; i < 4; i++) {
@@ -564,33 +577,47 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
           db = valid ? (db | (db << 16)) : 0u;
           if (s_abort || !mbar_wait(bars + 8 * (STAGES + s), ph ^ 1u)) { s_abort = 1; stop = true; break; }
           const uint32_t lut_copy = p_s + kStageIq4Lut + 4u * (uint32_t)(t & 3);
-          const uint32_t row_base = b_s + s * C::kBBytes + (uint32_t)t * 128u;
-          const uint32_t swz = (uint32_t)(t & 7);
+          const uint32_t row_base = b_s + s * C::kBBytes + (uint32_t)rt * 128u;
+          const uint32_t swz = (uint32_t)(rt & 7);
           uint32_t o[16];
-          iq4_block_chunks(qa, da, lut_copy, o);
+          if (MH == 1 || hf == 0) {
+            iq4_block_chunks(qa, da, lut_copy, o);
 #pragma unroll
-          for (int cc = 0; cc < 4; cc++)
-            sts128(row_base + ((cc ^ swz) << 4), o[4 * cc], o[4 * cc + 1], o[4 * cc + 2], o[4 * cc + 3]);
-          iq4_block_chunks(qb, db, lut_copy, o);
+            for (int cc = 0; cc < 4; cc++)
+              sts128(row_base + ((cc ^ swz) << 4), o[4 * cc], o[4 * cc + 1], o[4 * cc + 2], o[4 * cc + 3]);
+          }
+          if (MH == 1 || hf == 1) {
+            iq4_block_chunks(qb, db, lut_copy, o);
 #pragma unroll
-          for (int cc = 0; cc < 4; cc++)
-            sts128(row_base + (((cc + 4) ^ swz) << 4), o[4 * cc], o[4 * cc + 1], o[4 * cc + 2], o[4 * cc + 3]);
+            for (int cc = 0; cc < 4; cc++)
+              sts128(row_base + (((cc + 4) ^ swz) << 4), o[4 * cc], o[4 * cc + 1], o[4 * cc + 2], o[4 * cc + 3]);
+          }
           fence_proxy_async_shared();
           mbar_arrive(bars + 8 * s);
           continue;
         }
-        // this row's 32 code bytes (units 2j, 2j+1) and 4 scales of step j
-        const uint4 c0 = lds128(src + t * 128 + (((2 * j) ^ (t & 7)) << 4));
-        const uint4 c1 = lds128(src + t * 128 + (((2 * j + 1) ^ (t & 7)) << 4));
+        // this row's 32 code bytes (units 2j, 2j+1) and 4 scales of step j;
+        // with MH = 2 this thread takes unit 2j + hf (chunks 4hf .. 4hf+3)
+        constexpr int kCh = 8 / MH;                 // 16-byte output chunks of this thread
+        const int ch0 = (MH == 2) ? 4 * hf : 0;     // its first chunk
+        uint32_t q[8];
+        {
+          const uint4 c0 = lds128(src + rt * 128 + (((2 * j + (MH == 2 ? hf : 0)) ^ (rt & 7)) << 4));
+          q[0] = c0.x; q[1] = c0.y; q[2] = c0.z; q[3] = c0.w;
+          if (MH == 1) {
+            const uint4 c1 = lds128(src + rt * 128 + (((2 * j + 1) ^ (rt & 7)) << 4));
+            q[4] = c1.x; q[5] = c1.y; q[6] = c1.z; q[7] = c1.w;
+          }
+        }
         uint32_t sc[4];
         bool mx_wide = false;  // MXFP4 scale that is not an fp16 value: two fp16 factors
         uint32_t mx0a = 0u, mx0b = 0u, mx1a = 0u, mx1b = 0u;
         if (FMT == 2) {
-          const uint32_t half = (uint32_t)((j >> 1) ^ ((t >> 2) & 1));
-          const uint2 sv = lds64(src + kStageCodes + t * 32 + (half << 4) + (j & 1) * 8);
+          const uint32_t half = (uint32_t)((j >> 1) ^ ((rt >> 2) & 1));
+          const uint2 sv = lds64(src + kStageCodes + rt * 32 + (half << 4) + (j & 1) * 8);
           sc[0] = bcast_lo(sv.x); sc[1] = bcast_hi(sv.x); sc[2] = bcast_lo(sv.y); sc[3] = bcast_hi(sv.y);
         } else if (FMT == 4) {  // two E8M0 bytes for this step's 64 k
-          const uint32_t sw = lds32(src + kStageCodes + t * 32 + (j >> 1) * 4) >> ((j & 1) * 16);
+          const uint32_t sw = lds32(src + kStageCodes + rt * 32 + (j >> 1) * 4) >> ((j & 1) * 16);
           const uint32_t b0 = sw & 0xFFu, b1 = (sw >> 8) & 0xFFu;
           mx_wide = !(e8m0_f16_ok(b0) && e8m0_f16_ok(b1));
           if (mx_wide) {  // rare: two fp16 factors per group
@@ -601,30 +628,31 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
           sc[0] = sc[1] = f16x2_pow2(v0 < -24 ? -24 : (v0 > 15 ? 15 : v0));
           sc[2] = sc[3] = f16x2_pow2(v1 < -24 ? -24 : (v1 > 15 ? 15 : v1));
         } else {
-          const uint32_t sw = lds32(src + kStageCodes + t * 32 + j * 4);
+          const uint32_t sw = lds32(src + kStageCodes + rt * 32 + j * 4);
           const uint32_t e01 = e4m3x2_to_f16x2(sw & 0xFFFFu), e23 = e4m3x2_to_f16x2(sw >> 16);
           sc[0] = bcast_lo(e01); sc[1] = bcast_hi(e01); sc[2] = bcast_lo(e23); sc[3] = bcast_hi(e23);
         }
         if (!valid) sc[0] = sc[1] = sc[2] = sc[3] = 0u;
         if (s_abort || !mbar_wait(bars + 8 * (STAGES + s), ph ^ 1u)) { s_abort = 1; stop = true; break; }
-        const uint32_t q[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-        const uint32_t row_base = b_s + s * C::kBBytes + (uint32_t)t * 128u;
-        const uint32_t swz = (uint32_t)(t & 7);
+        const uint32_t row_base = b_s + s * C::kBBytes + (uint32_t)rt * 128u;
+        const uint32_t swz = (uint32_t)(rt & 7);
         if (FMT == 4 && mx_wide) {
           if (!valid) mx0a = mx0b = mx1a = mx1b = 0u;
 #pragma unroll
-          for (int cc = 0; cc < 8; cc++) {
+          for (int c = 0; c < kCh; c++) {
+            const int cc = ch0 + c;
             uint32_t w4[4];
-            e2m1x8_to_f16x2(q[cc], w4);
+            e2m1x8_to_f16x2(q[c], w4);
             const uint32_t fa = (cc < 4) ? mx0a : mx1a, fb = (cc < 4) ? mx0b : mx1b;
             sts128(row_base + ((cc ^ swz) << 4), hmul2(hmul2(w4[0], fa), fb), hmul2(hmul2(w4[1], fa), fb),
                    hmul2(hmul2(w4[2], fa), fb), hmul2(hmul2(w4[3], fa), fb));
           }
         } else {
 #pragma unroll
-          for (int cc = 0; cc < 8; cc++) {
+          for (int c = 0; c < kCh; c++) {
+            const int cc = ch0 + c;
             uint32_t w4[4];
-            e2m1x8_to_f16x2(q[cc], w4);
+            e2m1x8_to_f16x2(q[c], w4);
             const uint32_t sv = sc[cc >> 1];
             sts128(row_base + ((cc ^ swz) << 4), hmul2(w4[0], sv), hmul2(w4[1], sv), hmul2(w4[2], sv),
                    hmul2(w4[3], sv));
@@ -642,15 +670,16 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
     const float gs = (FMT == 3) ? g : 1.0f;
     for (int li = 0; li < my_tiles; li++) {
       const int tile = (int)blockIdx.x + li * G;
-      const int m0 = (tile / n_tiles) * kGemmBM, n0 = (tile % n_tiles) * BN;
+      const int m0 = (tile / n_tiles) * kBM, n0 = (tile % n_tiles) * BN;
       const int n_mma = (min(BN, n - n0) <= BN / 2) ? BN / 2 : BN;
       const int a = li & 1;
       if (s_abort || !mbar_wait(accf + 8 * a, ((uint32_t)li >> 1) & 1u)) { s_abort = 1; break; }
       tc_fence_after();
-      const int mrow = m0 + 32 * q + lane;
-      for (int j = 0; j < n_mma / 32; j++) {
+      for (int jj = 0; jj < MH * (n_mma / 32); jj++) {
+        const int mh = jj / (n_mma / 32), j = jj - mh * (n_mma / 32);  // M-half, 32-column group
+        const int mrow = m0 + 128 * mh + 32 * q + lane;
         uint32_t r[32];
-        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * BN + 32 * j), r);
+        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * MH * BN + mh * BN + 32 * j), r);
         tmem_ld_wait();
         const int col = n0 + 32 * j;
         if (mrow < m && col < n) {
@@ -679,7 +708,7 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 2 * BN);
+    tmem_dealloc(tmem, 2 * MH * BN);
   }
 }
 

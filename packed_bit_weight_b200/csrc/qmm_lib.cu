@@ -579,29 +579,43 @@ static qmm_status launch_gemm_tc(const qmm_weights* w, const uint16_t* x, int m,
   return launch_status();
 }
 
-template <int FMT>
-static qmm_status launch_gemm_tc_persistent(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y,
-                                            cudaStream_t st, const DevInfo* di) {
-  constexpr int BN = 256, STAGES = 3;
+// MH = 1: 128-token x 256-row tiles; MH = 2: 256 x 128 (half the weight
+// decode per FLOP, two MMAs per k16 step sharing the decoded weights).
+template <int FMT, int MH>
+static qmm_status launch_gemm_tc_persistent_mh(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y,
+                                               cudaStream_t st, const DevInfo* di) {
+  constexpr int BN = 256 / MH, STAGES = 3, BM = kGemmBM * MH;
   using C = GemmCfg<BN, STAGES>;
   const int n = (int)w->n, k = (int)w->k;
   CUtensorMap tx;
-  if (!make_map_2d(&tx, x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)k, (uint64_t)m, kGemmBK, kGemmBM,
+  if (!make_map_2d(&tx, x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)k, (uint64_t)m, kGemmBK, BM,
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return QMM_ERR_CUDA;
-  const size_t smem = 1024 + (size_t)STAGES * C::kStageBytes + 2 * (size_t)kStageBytes + 256;
+  const size_t smem = 1024 + (size_t)STAGES * (MH * C::kABytes + C::kBBytes) + 2 * (size_t)kStageBytes + 256;
   if (smem > di->smem_optin) return QMM_ERR_CUDA;
-  auto kern = gemm_fp4_tc_persistent_kernel<FMT, BN, STAGES>;
+  auto kern = gemm_fp4_tc_persistent_kernel<FMT, BN, STAGES, MH>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return QMM_ERR_CUDA;
-  const int64_t tiles = (int64_t)((m + kGemmBM - 1) / kGemmBM) * ((n + BN - 1) / BN);
+  const int64_t tiles = (int64_t)((m + BM - 1) / BM) * ((n + BN - 1) / BN);
   if (tiles > INT32_MAX) return QMM_ERR_UNSUPPORTED_SHAPE;
   const int grid = tiles < di->sms ? (int)tiles : di->sms;
   kern<<<grid, kGemmPThreads, smem, st>>>(tx, static_cast<const uint8_t*>(w->data),
                                           static_cast<const uint8_t*>(w->scales), y, m, n, k, w->global_scale);
-  set_variant("gemm_fp4_tc_persistent<fmt=%d,bm=128,bn=%d,bk=64,stages=%d,grid=%d,tiles=%lld>", FMT, BN, STAGES, grid,
-              (long long)tiles);
+  set_variant("gemm_fp4_tc_persistent<fmt=%d,bm=%d,bn=%d,bk=64,stages=%d,grid=%d,tiles=%lld>", FMT, BM, BN, STAGES,
+              grid, (long long)tiles);
   return launch_status();
+}
+
+// 256-token tiles from m = 256 up (2048 x 18560 x 4096 on B200: FP4-G16
+// 949 vs 871 TFLOP/s, E4M3 995 vs 882, MXFP4 957 vs 766, IQ4_NL 685 vs 470),
+// 128-token tiles below.  QMM_GEMM_MH=1/2 forces either (measurement knob).
+template <int FMT>
+static qmm_status launch_gemm_tc_persistent(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y,
+                                            cudaStream_t st, const DevInfo* di) {
+  const char* e = getenv("QMM_GEMM_MH");
+  const bool two = (e && e[0]) ? e[0] == '2' : m >= 256;
+  if (two) return launch_gemm_tc_persistent_mh<FMT, 2>(w, x, m, y, st, di);
+  return launch_gemm_tc_persistent_mh<FMT, 1>(w, x, m, y, st, di);
 }
 
 // Any shape the tensor-core kernel does not take: the decode-batch kernel

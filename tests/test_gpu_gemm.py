@@ -147,3 +147,52 @@ def test_gemm_iq4nl_identity_rows_give_decoded_weights():
     assert qmm.qmm_last_variant().startswith("gemm_fp4_tc_persistent<fmt=1")
     deq = oracle.dequant(p.fmt, n, k, p.data, None)
     assert np.array_equal(nz(y), nz(deq[:, :m].T))
+
+
+@pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3, synth.FMT_MXFP4, synth.FMT_IQ4_NL])
+@pytest.mark.parametrize("m,n,k", [(256, 128, 256), (200, 300, 1024), (300, 1000, 512), (64, 17, 512),
+                                   (2048, 640, 2560), (520, 200, 768)])
+def test_gemm_256_token_tiles(fmt, m, n, k, monkeypatch):
+    """The persistent kernel with 256-token x 128-row tiles (two M=128 MMAs
+    per k16 step on the same decoded weights, two accumulator halves): ragged
+    m (the second half partly or wholly past m) and n (64-row last tiles)."""
+    monkeypatch.setenv("QMM_GEMM_MH", "2")
+    rng = np.random.default_rng(700 + m + n + k + fmt)
+    p = synth.gen_weights(rng, fmt, n, k)
+    x = synth.gen_x(rng, m, k)
+    y = run_gemm(dev(p), x)
+    v = qmm.qmm_last_variant()
+    assert v.startswith("gemm_fp4_tc_persistent<fmt=%d,bm=256,bn=128" % fmt), v
+    yref, absy = oracle.matmul(fmt, n, k, p.data, p.scales, p.global_scale, x)
+    check_tol(y, yref, absy, v)
+
+
+@pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_MXFP4, synth.FMT_IQ4_NL])
+def test_gemm_256_token_tiles_identity_rows(fmt, monkeypatch):
+    """X = [I | 0] over 256 tokens: both accumulator halves return the decoded
+    weight columns bit-exactly."""
+    monkeypatch.setenv("QMM_GEMM_MH", "2")
+    rng = np.random.default_rng(11 + fmt)
+    m, n, k = 256, 384, 512
+    p = synth.gen_weights(rng, fmt, n, k)
+    x = np.zeros((m, k), dtype=np.uint16)
+    x[np.arange(m), np.arange(m)] = 0x3C00
+    y = run_gemm(dev(p), x)
+    assert qmm.qmm_last_variant().startswith("gemm_fp4_tc_persistent<fmt=%d,bm=256" % fmt)
+    deq = oracle.dequant(fmt, n, k, p.data, p.scales, p.global_scale)
+    assert np.array_equal(nz(y), nz(deq[:, :m].T))
+
+
+@pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_IQ4_NL])
+@pytest.mark.parametrize("m,n,k", [(128, 256, 256), (200, 300, 1024)])
+def test_gemm_128_token_tiles_forced(fmt, m, n, k, monkeypatch):
+    """The 128-token x 256-row tiles (the default below m = 256), forced."""
+    monkeypatch.setenv("QMM_GEMM_MH", "1")
+    rng = np.random.default_rng(800 + m + n + k + fmt)
+    p = synth.gen_weights(rng, fmt, n, k)
+    x = synth.gen_x(rng, m, k)
+    y = run_gemm(dev(p), x)
+    v = qmm.qmm_last_variant()
+    assert v.startswith("gemm_fp4_tc_persistent<fmt=%d,bm=128,bn=256" % fmt), v
+    yref, absy = oracle.matmul(fmt, n, k, p.data, p.scales, p.global_scale, x)
+    check_tol(y, yref, absy, v)
