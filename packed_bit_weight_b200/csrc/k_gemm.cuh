@@ -372,15 +372,16 @@ __device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint32_t bar) {
 // step that share the decoded weight tile and accumulate into two halves of
 // the accumulator: half the weight decode per FLOP of MH = 1 (128 x 256),
 // the same tensor memory (2 accumulators x 256 columns) and operand bytes
-// per stage (32 + 16 KB instead of 16 + 32 KB).  Decode thread t then owns
-// 32 of the 64 k of row t % 128.
+// per stage (32 + 16 KB instead of 16 + 32 KB).  With BN = 128 (either MH)
+// decode thread t owns 32 of the 64 k of row t % 128.
 template <int FMT, int BN, int STAGES, int MH = 1>
 __global__ void __launch_bounds__(kGemmPThreads, 1)
     gemm_fp4_tc_persistent_kernel(const __grid_constant__ CUtensorMap tm_x, const uint8_t* __restrict__ codes,
                                   const uint8_t* __restrict__ scales, uint16_t* __restrict__ y, int m, int n, int k,
                                   float g) {
   using C = GemmCfg<BN, STAGES>;
-  static_assert(MH == 1 || (MH == 2 && BN * MH == kGemmDecodeThreads), "one decode thread per row half");
+  constexpr int TPR = kGemmDecodeThreads / BN;  // decode threads per weight row: 1, or 2 (32 k each)
+  static_assert((TPR == 1 || TPR == 2) && BN * TPR == kGemmDecodeThreads, "one or two decode threads per row");
   constexpr uint32_t kA = MH * C::kABytes;  // X bytes per stage
   constexpr int kBM = MH * kGemmBM;         // tokens per tile
   extern __shared__ uint8_t smem_raw[];
@@ -497,7 +498,7 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
     // threads per 128-byte row piece of codes, so a warp instruction touches
     // 4 cache lines) into a 2-slot staging ring; thread t then decodes row t.
     const int t = threadIdx.x - 64;
-    const int rt = t % BN, hf = t / BN;  // row of the tile; with MH = 2 the 32-k half of each step
+    const int rt = t % BN, hf = t / BN;  // row of the tile; with TPR = 2 the 32-k half of each step
     const int nck = ksteps / kGemmChunkSteps;  // chunks per tile
     const int total_ck = my_tiles * nck;
     const int64_t crow = k >> 1, srow = k >> 4;
@@ -580,13 +581,13 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
           const uint32_t row_base = b_s + s * C::kBBytes + (uint32_t)rt * 128u;
           const uint32_t swz = (uint32_t)(rt & 7);
           uint32_t o[16];
-          if (MH == 1 || hf == 0) {
+          if (TPR == 1 || hf == 0) {
             iq4_block_chunks(qa, da, lut_copy, o);
 #pragma unroll
             for (int cc = 0; cc < 4; cc++)
               sts128(row_base + ((cc ^ swz) << 4), o[4 * cc], o[4 * cc + 1], o[4 * cc + 2], o[4 * cc + 3]);
           }
-          if (MH == 1 || hf == 1) {
+          if (TPR == 1 || hf == 1) {
             iq4_block_chunks(qb, db, lut_copy, o);
 #pragma unroll
             for (int cc = 0; cc < 4; cc++)
@@ -597,14 +598,14 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
           continue;
         }
         // this row's 32 code bytes (units 2j, 2j+1) and 4 scales of step j;
-        // with MH = 2 this thread takes unit 2j + hf (chunks 4hf .. 4hf+3)
-        constexpr int kCh = 8 / MH;                 // 16-byte output chunks of this thread
-        const int ch0 = (MH == 2) ? 4 * hf : 0;     // its first chunk
+        // with TPR = 2 this thread takes unit 2j + hf (chunks 4hf .. 4hf+3)
+        constexpr int kCh = 8 / TPR;                // 16-byte output chunks of this thread
+        const int ch0 = (TPR == 2) ? 4 * hf : 0;    // its first chunk
         uint32_t q[8];
         {
-          const uint4 c0 = lds128(src + rt * 128 + (((2 * j + (MH == 2 ? hf : 0)) ^ (rt & 7)) << 4));
+          const uint4 c0 = lds128(src + rt * 128 + (((2 * j + (TPR == 2 ? hf : 0)) ^ (rt & 7)) << 4));
           q[0] = c0.x; q[1] = c0.y; q[2] = c0.z; q[3] = c0.w;
-          if (MH == 1) {
+          if (TPR == 1) {
             const uint4 c1 = lds128(src + rt * 128 + (((2 * j + 1) ^ (rt & 7)) << 4));
             q[4] = c1.x; q[5] = c1.y; q[6] = c1.z; q[7] = c1.w;
           }

@@ -581,10 +581,10 @@ static qmm_status launch_gemm_tc(const qmm_weights* w, const uint16_t* x, int m,
 
 // MH = 1: 128-token x 256-row tiles; MH = 2: 256 x 128 (half the weight
 // decode per FLOP, two MMAs per k16 step sharing the decoded weights).
-template <int FMT, int MH>
+template <int FMT, int MH, int BN = 256 / MH>
 static qmm_status launch_gemm_tc_persistent_mh(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y,
                                                cudaStream_t st, const DevInfo* di) {
-  constexpr int BN = 256 / MH, STAGES = 3, BM = kGemmBM * MH;
+  constexpr int STAGES = 3, BM = kGemmBM * MH;
   using C = GemmCfg<BN, STAGES>;
   const int n = (int)w->n, k = (int)w->k;
   CUtensorMap tx;

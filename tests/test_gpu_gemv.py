@@ -293,3 +293,4 @@ def test_gemv_host_argument_errors():
     with pytest.raises(qmm.QmmError) as e:
         qmm.qmm_gemv_host(w, xh, yh, xd, torch.zeros((2 * 64 + 8,), dtype=torch.int16, device="cuda")[1:129])
     assert e.value.status == 3                                  # misaligned y staging buffer
+
