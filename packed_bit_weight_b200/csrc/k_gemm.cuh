@@ -348,14 +348,16 @@ static_assert(kStageIq4Lut + 256 * 4 * 4 <= kStageBytes, "IQ4_NL table fits in t
 // 0..7 (weights 16..23), 3 = high of 8..15.  Two adjacent nibbles of the same
 // kind form one table index, so each lookup yields two consecutive weights,
 // exact; one f16x2 multiply by d rounds each once.
+// LSH: log2 of a table entry's bytes (4 bytes per copy, 2^(LSH-2) copies).
+template <int LSH = 4>
 __device__ __forceinline__ void iq4_block_chunks(const uint32_t (&Q)[4], uint32_t dd, uint32_t lut_copy,
                                                  uint32_t (&out)[16]) {
 #pragma unroll
   for (int i = 0; i < 4; i++) {
     const uint32_t lo = Q[i] & 0x0F0F0F0Fu, hi = (Q[i] >> 4) & 0x0F0F0F0Fu;
     const uint32_t ul = lo | (lo >> 4), uh = hi | (hi >> 4);  // bytes 0 and 2: (n0 | n1 << 4), (n2 | n3 << 4)
-    const uint32_t l0 = lds32(lut_copy + ((ul & 0xFFu) << 4)), l1 = lds32(lut_copy + (((ul >> 16) & 0xFFu) << 4));
-    const uint32_t h0 = lds32(lut_copy + ((uh & 0xFFu) << 4)), h1 = lds32(lut_copy + (((uh >> 16) & 0xFFu) << 4));
+    const uint32_t l0 = lds32(lut_copy + ((ul & 0xFFu) << LSH)), l1 = lds32(lut_copy + (((ul >> 16) & 0xFFu) << LSH));
+    const uint32_t h0 = lds32(lut_copy + ((uh & 0xFFu) << LSH)), h1 = lds32(lut_copy + (((uh >> 16) & 0xFFu) << LSH));
     // bytes 4i..4i+3: low nibbles are weights 4i..4i+3, high ones 16+4i..
     out[(i >> 1) * 4 + (i & 1) * 2] = hmul2(l0, dd);
     out[(i >> 1) * 4 + (i & 1) * 2 + 1] = hmul2(l1, dd);
@@ -382,6 +384,11 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
   using C = GemmCfg<BN, STAGES>;
   constexpr int TPR = kGemmDecodeThreads / BN;  // decode threads per weight row: 1, or 2 (32 k each)
   static_assert((TPR == 1 || TPR == 2) && BN * TPR == kGemmDecodeThreads, "one or two decode threads per row");
+  // IQ4_NL pair table after the staged rows of slot 0: 16 word-interleaved
+  // copies when 128 rows leave room (two lanes per copy), else 4
+  constexpr int kLutC = (BN == 128) ? 16 : 4, kLutLsh = (BN == 128) ? 6 : 4;
+  constexpr uint32_t kLutOff = (uint32_t)BN * kStageIq4Row;
+  static_assert(kLutOff + 256u * kLutC * 4u <= (uint32_t)kStageBytes, "IQ4_NL table fits in staging slot 0");
   constexpr uint32_t kA = MH * C::kABytes;  // X bytes per stage
   constexpr int kBM = MH * kGemmBM;         // tokens per tile
   extern __shared__ uint8_t smem_raw[];
@@ -424,12 +431,12 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
     tmem_alloc(tmem_slot, 2 * MH * BN);
     tmem_relinquish();
   }
-  if (FMT == 1) {  // IQ4_NL pair table, 4 interleaved copies, in staging slot 0's spare tail
-    for (int i = threadIdx.x; i < 256 * 4; i += blockDim.x) {
-      const int v = i >> 2;
+  if (FMT == 1) {  // IQ4_NL pair table, kLutC interleaved copies, in staging slot 0's spare tail
+    for (int i = threadIdx.x; i < 256 * kLutC; i += blockDim.x) {
+      const int v = i / kLutC;
       const uint32_t lo = __half_as_ushort(__int2half_rn(c_iq4nl_kv[v & 15]));
       const uint32_t hi = __half_as_ushort(__int2half_rn(c_iq4nl_kv[v >> 4]));
-      asm volatile("st.shared.u32 [%0], %1;" ::"r"(p_s + kStageIq4Lut + 4u * i), "r"(lo | (hi << 16)) : "memory");
+      asm volatile("st.shared.u32 [%0], %1;" ::"r"(p_s + kLutOff + 4u * i), "r"(lo | (hi << 16)) : "memory");
     }
   }
   tc_fence_before();
@@ -509,7 +516,7 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
       const int n0 = (tile % n_tiles) * BN;
       const int kc = (c % nck) * (kGemmChunkSteps * kGemmBK);  // first k of the chunk
       const uint32_t dst = p_s + slot * kStageBytes;
-      if (FMT == 1) {  // IQ4_NL: 256 rows x 9 units of 16 bytes (8 blocks of 18 bytes)
+      if (FMT == 1) {  // IQ4_NL: BN rows x 9 units of 16 bytes (8 blocks of 18 bytes), unit-major [9][BN][16 B]
         const int64_t rowb = (int64_t)(k >> 5) * 18;
 #pragma unroll
         for (int i = 0; i < (9 * BN + kGemmDecodeThreads - 1) / kGemmDecodeThreads; i++) {
@@ -517,7 +524,7 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
           if (pc >= 9 * BN) break;
           const int r = pc / 9, u = pc - r * 9;
           const int64_t gr = min((int64_t)n0 + r, (int64_t)n - 1);
-          cp_async16_g(dst + r * kStageIq4Row + u * 16, codes + gr * rowb + (int64_t)(kc >> 5) * 18 + u * 16);
+          cp_async16_g(dst + u * (BN * 16) + r * 16, codes + gr * rowb + (int64_t)(kc >> 5) * 18 + u * 16);
         }
         cp_async_mbar_arrive_noinc(cfull + 8 * slot);
         return true;
@@ -559,14 +566,24 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
       const int tile = (int)blockIdx.x + (c / nck) * G;
       const bool valid = (int64_t)(tile % n_tiles) * BN + rt < n;
       const uint32_t src = p_s + slot * kStageBytes;
+#pragma unroll  // (IQ4_NL selects its words by j)
       for (int j = 0; j < kGemmChunkSteps; j++, gs++) {
         const int s = gs % STAGES;
         const uint32_t ph = (uint32_t)(gs / STAGES) & 1u;
         if (FMT == 1) {
-          // this row's two blocks of step j: 36 bytes from byte 36j of the row
+          // this row's two blocks of step j: 36 bytes from byte 36j of the row,
+          // inside its 16-byte units 2j .. 2j+2 (36j = 32j + 4j: the span
+          // starts j words into unit 2j); a warp's 32 rows read each unit as
+          // 512 contiguous bytes
+          uint32_t uw[12];
+#pragma unroll
+          for (int u = 0; u < 3; u++) {
+            const uint4 v = lds128(src + (2 * j + u) * (BN * 16) + rt * 16);
+            uw[4 * u] = v.x; uw[4 * u + 1] = v.y; uw[4 * u + 2] = v.z; uw[4 * u + 3] = v.w;
+          }
           uint32_t w[9];
 #pragma unroll
-          for (int i = 0; i < 9; i++) w[i] = lds32(src + rt * kStageIq4Row + j * 36 + 4 * i);
+          for (int i = 0; i < 9; i++) w[i] = (j == 0) ? uw[i] : (j == 1) ? uw[i + 1] : (j == 2) ? uw[i + 2] : uw[i + 3];
           uint32_t qa[4], qb[4];
 #pragma unroll
           for (int i = 0; i < 4; i++) {
@@ -577,18 +594,18 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
           da = valid ? (da | (da << 16)) : 0u;
           db = valid ? (db | (db << 16)) : 0u;
           if (s_abort || !mbar_wait(bars + 8 * (STAGES + s), ph ^ 1u)) { s_abort = 1; stop = true; break; }
-          const uint32_t lut_copy = p_s + kStageIq4Lut + 4u * (uint32_t)(t & 3);
+          const uint32_t lut_copy = p_s + kLutOff + 4u * (uint32_t)(t & (kLutC - 1));
           const uint32_t row_base = b_s + s * C::kBBytes + (uint32_t)rt * 128u;
           const uint32_t swz = (uint32_t)(rt & 7);
           uint32_t o[16];
           if (TPR == 1 || hf == 0) {
-            iq4_block_chunks(qa, da, lut_copy, o);
+            iq4_block_chunks<kLutLsh>(qa, da, lut_copy, o);
 #pragma unroll
             for (int cc = 0; cc < 4; cc++)
               sts128(row_base + ((cc ^ swz) << 4), o[4 * cc], o[4 * cc + 1], o[4 * cc + 2], o[4 * cc + 3]);
           }
           if (TPR == 1 || hf == 1) {
-            iq4_block_chunks(qb, db, lut_copy, o);
+            iq4_block_chunks<kLutLsh>(qb, db, lut_copy, o);
 #pragma unroll
             for (int cc = 0; cc < 4; cc++)
               sts128(row_base + (((cc + 4) ^ swz) << 4), o[4 * cc], o[4 * cc + 1], o[4 * cc + 2], o[4 * cc + 3]);
