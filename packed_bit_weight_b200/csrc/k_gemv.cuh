@@ -362,6 +362,12 @@ __device__ __forceinline__ uint2 ldg_stream64(const void* p) {
   asm("ld.global.nc.L1::no_allocate.L2::256B.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
   return v;
 }
+// 256-bit activation load (L1-allocating; p 32-byte aligned).
+__device__ __forceinline__ void ldg_x256(const void* p, uint4& lo, uint4& hi) {
+  asm("ld.global.nc.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+      : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w), "=r"(hi.x), "=r"(hi.y), "=r"(hi.z), "=r"(hi.w)
+      : "l"(p));
+}
 __device__ __forceinline__ uint4 ldg_x128(const void* p) {
   uint4 v;
   asm("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
@@ -385,7 +391,9 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 // WIDE: the lane's bytes of two consecutive segments 2w, 2w+1 are the 32
 // contiguous bytes at 32*tig of a 256-k span (one 256-bit load), so segment
 // 2w+h holds k = 256w + 64*tig + 32h + [0, 32) instead of 128s + 32*tig.
-template <int FMT, int NT, int SPW, bool WIDE = false>
+// XW: the token row's 64 bytes per segment as two 256-bit loads (x rows
+// 32-byte aligned).
+template <int FMT, int NT, int SPW, bool WIDE = false, bool XW = false>
 __device__ __forceinline__ void ldg_tile_mma(float (&acc)[NT][4], const uint4 (&qa)[SPW], const uint4 (&qb)[SPW],
                                              const uint32_t (&sa)[SPW], const uint32_t (&sb)[SPW], int seg0, int grp,
                                              int tig, const uint16_t* __restrict__ x, int k, int m) {
@@ -399,10 +407,20 @@ __device__ __forceinline__ void ldg_tile_mma(float (&acc)[NT][4], const uint4 (&
       const int tok = grp + 8 * j;
       if (tok < m) {
         const uint16_t* xp = x + (int64_t)tok * k + kseg;
+        if (XW) {
 #pragma unroll
-        for (int q = 0; q < 4; q++) {
-          const uint4 v = ldg_x128(xp + 8 * q);
-          xb[j][4 * q] = v.x; xb[j][4 * q + 1] = v.y; xb[j][4 * q + 2] = v.z; xb[j][4 * q + 3] = v.w;
+          for (int q = 0; q < 2; q++) {
+            uint4 lo, hi;
+            ldg_x256(xp + 16 * q, lo, hi);
+            xb[j][8 * q] = lo.x; xb[j][8 * q + 1] = lo.y; xb[j][8 * q + 2] = lo.z; xb[j][8 * q + 3] = lo.w;
+            xb[j][8 * q + 4] = hi.x; xb[j][8 * q + 5] = hi.y; xb[j][8 * q + 6] = hi.z; xb[j][8 * q + 7] = hi.w;
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 4; q++) {
+            const uint4 v = ldg_x128(xp + 8 * q);
+            xb[j][4 * q] = v.x; xb[j][4 * q + 1] = v.y; xb[j][4 * q + 2] = v.z; xb[j][4 * q + 3] = v.w;
+          }
         }
       } else {
 #pragma unroll
@@ -472,7 +490,7 @@ __device__ __forceinline__ void ldg_tile_store(float (&red)[WPC][16][16], const 
 // bytes of two segments with one 256-bit load per row, and their scales with
 // one load (8 B fp16, 4 B E4M3, 2 B E8M0), the segment pairing of
 // ldg_tile_mma's WIDE layout.
-template <int FMT, int NT, int SPW, int WPC = kLdgWarps, int MINB = 2, bool WIDE = false>
+template <int FMT, int NT, int SPW, int WPC = kLdgWarps, int MINB = 2, bool WIDE = false, bool XW = false>
 __global__ void __launch_bounds__(WPC * 32, MINB)
     gemv_fp4_ldg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
                         const uint16_t* __restrict__ x, uint16_t* __restrict__ y, int n, int k, int m, float g) {
@@ -541,7 +559,7 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
   for (int j = 0; j < NT; j++)
 #pragma unroll
     for (int c = 0; c < 4; c++) acc[j][c] = 0.f;
-  ldg_tile_mma<FMT, NT, SPW, WIDE>(acc, qa, qb, sa, sb, seg0, grp, tig, x, k, m);
+  ldg_tile_mma<FMT, NT, SPW, WIDE, XW>(acc, qa, qb, sa, sb, seg0, grp, tig, x, k, m);
   ldg_tile_store<FMT, NT, WPC>(red, acc, warp, grp, tig, n0, n, m, g, y);
 }
 

@@ -168,7 +168,7 @@ static qmm_status launch_gemv_tma(const qmm_weights* w, const uint16_t* x, int m
   return launch_status();
 }
 
-template <int FMT, int NT, int SPW, int WPC = kLdgWarps, int MINB = 2, bool WIDE = false>
+template <int FMT, int NT, int SPW, int WPC = kLdgWarps, int MINB = 2, bool WIDE = false, bool XW = false>
 static qmm_status launch_gemv_ldg(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st) {
   const int n = (int)w->n, k = (int)w->k;
   const int tiles = (n + 15) / 16;
@@ -178,7 +178,7 @@ static qmm_status launch_gemv_ldg(const qmm_weights* w, const uint16_t* x, int m
   const char* nopdl = getenv("QMM_GEMV_NOPDL");
   const char* pad = getenv("QMM_GEMV_SMEM_PAD");
   const int pad_bytes = pad ? atoi(pad) : 0;
-  auto kern = gemv_fp4_ldg_kernel<FMT, NT, SPW, WPC, MINB, WIDE>;
+  auto kern = gemv_fp4_ldg_kernel<FMT, NT, SPW, WPC, MINB, WIDE, XW>;
   if (pad_bytes > 0 &&
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pad_bytes) != cudaSuccess)
     return QMM_ERR_CUDA;
@@ -196,8 +196,8 @@ static qmm_status launch_gemv_ldg(const qmm_weights* w, const uint16_t* x, int m
   const uint8_t* scales = static_cast<const uint8_t*>(w->scales);
   const float g = w->global_scale;
   if (cudaLaunchKernelEx(&cfg, kern, codes, scales, x, y, n, k, m, g) != cudaSuccess) return QMM_ERR_CUDA;
-  set_variant("gemv_fp4_ldg<fmt=%d,nt=%d,spw=%d,wpc=%d,minb=%d,wide=%d,tiles=%d>", FMT, NT, SPW, WPC, MINB,
-              WIDE ? 1 : 0, tiles);
+  set_variant("gemv_fp4_ldg<fmt=%d,nt=%d,spw=%d,wpc=%d,minb=%d,wide=%d,xw=%d,tiles=%d>", FMT, NT, SPW, WPC, MINB,
+              WIDE ? 1 : 0, XW ? 1 : 0, tiles);
   return launch_status();
 }
 
@@ -217,9 +217,15 @@ static bool ldg_wide_ok(const qmm_weights* w) {
 template <int FMT, int NT, int SPW, int WPC, int MINB>
 static qmm_status launch_gemv_ldg_pick(bool wide, const qmm_weights* w, const uint16_t* x, int m, uint16_t* y,
                                        cudaStream_t st) {
+  // 256-bit activation loads when x is 32-byte aligned (QMM_GEMV_XW=0 turns
+  // them off: measurement knob)
+  const char* xe = getenv("QMM_GEMV_XW");
+  const bool xw = (reinterpret_cast<uintptr_t>(x) & 31u) == 0 && !(xe && xe[0] == '0');
   if constexpr (SPW % 2 == 0) {
+    if (wide && xw) return launch_gemv_ldg<FMT, NT, SPW, WPC, MINB, true, true>(w, x, m, y, st);
     if (wide) return launch_gemv_ldg<FMT, NT, SPW, WPC, MINB, true>(w, x, m, y, st);
   }
+  if (xw) return launch_gemv_ldg<FMT, NT, SPW, WPC, MINB, false, true>(w, x, m, y, st);
   return launch_gemv_ldg<FMT, NT, SPW, WPC, MINB, false>(w, x, m, y, st);
 }
 
