@@ -294,3 +294,30 @@ def test_gemv_host_argument_errors():
         qmm.qmm_gemv_host(w, xh, yh, xd, torch.zeros((2 * 64 + 8,), dtype=torch.int16, device="cuda")[1:129])
     assert e.value.status == 3                                  # misaligned y staging buffer
 
+
+
+@pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3, synth.FMT_MXFP4])
+@pytest.mark.parametrize("n,k,m", [(1000, 4096, 1), (333, 8192, 4), (517, 2048, 16)])
+@pytest.mark.parametrize("how", ["knob", "x16"])
+def test_register_kernel_128_bit_activation_loads(fmt, n, k, m, how, monkeypatch):
+    """The 16-byte activation loads: forced by QMM_GEMV_XW=0, or taken
+    because x is 16- but not 32-byte aligned (legal in the ABI)."""
+    p, xb = _case(fmt, n, k, m, 7000 + n + k + m + fmt)
+    w = dev(p)
+    if how == "knob":
+        monkeypatch.setenv("QMM_GEMV_XW", "0")
+        y = run_gemv(w, xb)
+    else:
+        buf = torch.zeros(m * k + 32, dtype=torch.int16, device="cuda")
+        off = 8 if (buf.data_ptr() + 16) % 32 else 24
+        xs = buf[off:off + m * k].view(m, k)
+        assert xs.data_ptr() % 32 == 16
+        xs.copy_(to_dev_u16(xb))
+        yd = torch.empty((m, n), dtype=torch.int16, device="cuda")
+        qmm.qmm_gemv(w, xs, yd)
+        assert qmm.qmm_sync_check() == 0
+        y = from_dev_u16(yd)
+    v = qmm.qmm_last_variant()
+    assert v.startswith("gemv_fp4_ldg") and "xw=0" in v, v
+    yref, absy = oracle.matmul(fmt, n, k, p.data, p.scales, p.global_scale, xb)
+    check_tol(y, yref, absy, v)
