@@ -309,7 +309,7 @@ def test_register_kernel_128_bit_activation_loads(fmt, n, k, m, how, monkeypatch
         y = run_gemv(w, xb)
     else:
         buf = torch.zeros(m * k + 32, dtype=torch.int16, device="cuda")
-        off = 8 if (buf.data_ptr() + 16) % 32 else 24
+        off = 8 if buf.data_ptr() % 32 == 0 else 0  # elements: x starts 16 bytes past a 32-byte boundary
         xs = buf[off:off + m * k].view(m, k)
         assert xs.data_ptr() % 32 == 16
         xs.copy_(to_dev_u16(xb))
