@@ -42,7 +42,14 @@
 
 namespace qmm {
 
-constexpr int kIqtGroup = 16;  // token slots per pass (two MMA n-tiles)
+constexpr int kIqtGroup = 16;      // token slots per pass (two MMA n-tiles)
+constexpr int kIqtMaxPairs = 1024;  // in-kernel routing: at most this many (token, slot) pairs
+// ... and the dispatch uses it up to one warp's worth: warp 0 reads the ids
+// 32 at a time, each read after the previous ballot, so at 256 pairs (64
+// tokens, top-4) the eight dependent reads per CTA cost more than the routing
+// pass they replace (routed experts 108 vs 92 us); at 4 pairs it saves the
+// pass (MoE block t = 1 34.9 vs 36.1 us).
+constexpr int kIqtInKernelRoutePairs = 32;
 
 struct IqtArgs {
   const uint8_t* data0;  // expert stack (gate when IQ_SWIGLU)
@@ -50,8 +57,10 @@ struct IqtArgs {
   int64_t dstride0, dstride1;
   const uint16_t* x;
   int x_per_pair, topk;
-  const int32_t* offsets;  // [E+1] pair offsets per expert (nullptr: plain product of m_plain rows)
+  const int32_t* offsets;  // [E+1] pair offsets per expert (nullptr: plain product of m_plain rows, or ids)
   const int32_t* perm;     // [P] pair ids sorted by expert
+  const int32_t* ids;      // [P] expert of each pair: the CTA finds its expert's pairs itself (offsets unused)
+  int P;
   int m_plain;
   void* y;
   const float* gw;  // IQ_SCALED_F32: per-pair weights
@@ -166,8 +175,35 @@ __device__ __forceinline__ void iqt_load(uint32_t (&w)[SPW][S][2][6], const uint
 // Threads a CTA of this register budget may have.
 __host__ __device__ constexpr int iqt_max_threads(int maxreg) { return (65536 / maxreg) & ~31; }
 
+// In-kernel routing (a.ids): warp 0 collects the pairs p whose id is this
+// CTA's expert, in increasing p (the order of the stable routing sort), into
+// shared memory; any id outside [0, E) raises ERR_BAD_EXPERT and is left out.
+// Returns the count to every thread (ends with a barrier).
+__device__ __forceinline__ int iqt_collect_pairs(const IqtArgs& a, int e, int* s_pairs, int* s_cnt) {
+  if ((threadIdx.x >> 5) == 0) {
+    const int lane = threadIdx.x & 31;
+    const unsigned lt = (1u << lane) - 1u;
+    int n = 0;
+    bool bad = false;
+    for (int p0 = 0; p0 < a.P; p0 += 32) {
+      const int p = p0 + lane;
+      const int id = p < a.P ? a.ids[p] : -1;
+      bad |= p < a.P && (id < 0 || id >= a.E);
+      const unsigned mask = __ballot_sync(0xFFFFFFFFu, id == e);
+      if (id == e) s_pairs[n + __popc(mask & lt)] = p;
+      n += __popc(mask);
+    }
+    if (__any_sync(0xFFFFFFFFu, bad) && lane == 0 && e == 0 && blockIdx.x == 0) raise_error(ERR_BAD_EXPERT);
+    if (lane == 0) *s_cnt = n;
+  }
+  __syncthreads();
+  return *s_cnt;
+}
+
 template <int MODE, int S, int SPW, int MAXREG, bool W16>
 __global__ void __launch_bounds__(iqt_max_threads(MAXREG)) __maxnreg__(MAXREG) iq4_tile_kernel(const IqtArgs a) {
+  __shared__ int s_pairs[kIqtMaxPairs];
+  __shared__ int s_cnt;
   static_assert(MODE != IQ_SWIGLU || S % 2 == 0, "SwiGLU items are gate and up tiles of the same rows");
   constexpr int kOut = (MODE == IQ_SWIGLU) ? S / 2 : S;  // output tiles per item
   extern __shared__ __align__(16) uint8_t smem_iqt[];
@@ -180,7 +216,9 @@ __global__ void __launch_bounds__(iqt_max_threads(MAXREG)) __maxnreg__(MAXREG) i
   int start = 0, cnt = a.m_plain;
   if (!a.spec) {  // most experts may be empty: find out before any other work
     pdl_wait();
-    if (a.offsets) {
+    if (a.ids) {
+      cnt = iqt_collect_pairs(a, e, s_pairs, &s_cnt);
+    } else if (a.offsets) {
       start = a.offsets[e];
       cnt = a.offsets[e + 1] - start;
     }
@@ -218,7 +256,9 @@ __global__ void __launch_bounds__(iqt_max_threads(MAXREG)) __maxnreg__(MAXREG) i
   if (a.spec) {
     iqt_load<S, SPW, W16>(w, rp, s0, tig);
     pdl_wait();  // routing, activations and the output buffer follow the previous kernel
-    if (a.offsets) {
+    if (a.ids) {
+      cnt = iqt_collect_pairs(a, e, s_pairs, &s_cnt);
+    } else if (a.offsets) {
       start = a.offsets[e];
       cnt = a.offsets[e + 1] - start;
     }
@@ -237,8 +277,8 @@ __global__ void __launch_bounds__(iqt_max_threads(MAXREG)) __maxnreg__(MAXREG) i
 #pragma unroll
     for (int j = 0; j < 2; j++) {
       const int slot = (grp + 8 * j < ng) ? grp + 8 * j : 0;
-      const int pr = a.offsets ? a.perm[start + g0 + slot] : g0 + slot;
-      const int row = (a.offsets && !a.x_per_pair) ? pr / a.topk : pr;
+      const int pr = a.ids ? s_pairs[g0 + slot] : a.offsets ? a.perm[start + g0 + slot] : g0 + slot;
+      const int row = ((a.ids || a.offsets) && !a.x_per_pair) ? pr / a.topk : pr;
       xr[j] = a.x + (int64_t)row * a.k;
     }
     float acc[S][2][4];
@@ -280,7 +320,7 @@ __global__ void __launch_bounds__(iqt_max_threads(MAXREG)) __maxnreg__(MAXREG) i
         v += red[((wi * S + sv) * kIqtGroup + slot) * 16 + row];
         if (MODE == IQ_SWIGLU) u += red[((wi * S + sv + 1) * kIqtGroup + slot) * 16 + row];
       }
-      const int64_t pr = a.offsets ? a.perm[start + g0 + slot] : g0 + slot;
+      const int64_t pr = a.ids ? s_pairs[g0 + slot] : a.offsets ? a.perm[start + g0 + slot] : g0 + slot;
       if (MODE == IQ_SCALED_F32) {
         static_cast<float*>(a.y)[pr * a.n + grow] = a.gw[pr] * v;
       } else if (MODE == IQ_SWIGLU) {

@@ -48,6 +48,9 @@ __global__ void __launch_bounds__(kRouterThreads) router_topk_kernel(const uint1
                                                                      float* __restrict__ g,
                                                                      float* __restrict__ logits_out) {
   __shared__ float z[kRouterMaxExperts];
+  // a kernel launched after this one with programmatic dependent launch (the
+  // routed-expert kernels) may start now; it waits for these results
+  asm volatile("griddepcontrol.launch_dependents;" :::);
   const int tok = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int kWarps = kRouterThreads / 32;

@@ -414,7 +414,7 @@ static int gemv_variant_env() {
 template <int MODE>
 static qmm_status launch_iq4_tile(const qmm_weights* w0, const qmm_weights* w1, const uint16_t* x, int x_per_pair,
                                   int64_t topk, const int32_t* offsets, const int32_t* perm, int64_t P, int m_plain,
-                                  void* y, const float* gw, cudaStream_t st);
+                                  void* y, const float* gw, cudaStream_t st, const int32_t* ids = nullptr);
 
 // Warp-per-tile IQ4_NL kernel (k_iq4w.cuh); UNSUPPORTED_SHAPE launches nothing.
 template <int MODE>
@@ -718,14 +718,15 @@ static qmm_status launch_iq4_warp(const qmm_weights* w0, const qmm_weights* w1, 
 template <int MODE, int S, int SPW, int kMaxReg, bool W16>
 static qmm_status launch_iq4_tile_cfg(const qmm_weights* w0, const qmm_weights* w1, const uint16_t* x, int x_per_pair,
                                       int64_t topk, const int32_t* offsets, const int32_t* perm, int64_t P,
-                                      int m_plain, void* y, const float* gw, cudaStream_t st) {
+                                      int m_plain, void* y, const float* gw, cudaStream_t st, const int32_t* ids) {
   const int steps = (int)(w0->k / 128), wpc = steps / SPW;
   const int64_t tiles = (w0->n + 15) / 16;
   constexpr int kOut = (MODE == IQ_SWIGLU) ? S / 2 : S;  // output tiles per item
   const int64_t ipe = (tiles + kOut - 1) / kOut;
   if (wpc * 32 > iqt_max_threads(kMaxReg)) return QMM_ERR_UNSUPPORTED_SHAPE;
-  const int64_t E = offsets ? w0->num_experts : 1;
+  const int64_t E = (offsets || ids) ? w0->num_experts : 1;
   const int64_t grid = E * ipe;
+  if (ids && P > kIqtMaxPairs) return QMM_ERR_UNSUPPORTED_SHAPE;
   if (grid < 1 || grid > INT32_MAX) return QMM_ERR_UNSUPPORTED_SHAPE;
   auto kern = iq4_tile_kernel<MODE, S, SPW, kMaxReg, W16>;
   const uint32_t smem = iqt_smem_bytes(S, wpc);
@@ -739,8 +740,10 @@ static qmm_status launch_iq4_tile_cfg(const qmm_weights* w0, const qmm_weights* 
   a.x = x;
   a.x_per_pair = x_per_pair;
   a.topk = (int)topk;
-  a.offsets = offsets;
-  a.perm = perm;
+  a.offsets = ids ? nullptr : offsets;
+  a.perm = ids ? nullptr : perm;
+  a.ids = ids;
+  a.P = (int)P;
   a.m_plain = m_plain;
   a.y = y;
   a.gw = gw;
@@ -748,7 +751,7 @@ static qmm_status launch_iq4_tile_cfg(const qmm_weights* w0, const qmm_weights* 
   a.k = (int)w0->k;
   a.E = (int)E;
   a.items_per_expert = (int)ipe;
-  a.spec = (!offsets || P >= 4 * E) ? 1 : 0;
+  a.spec = ((!offsets && !ids) || P >= 4 * E) ? 1 : 0;
   if (const char* e = getenv("QMM_IQ4T_SPEC")) a.spec = (e[0] == '1') ? 1 : 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
@@ -761,8 +764,8 @@ static qmm_status launch_iq4_tile_cfg(const qmm_weights* w0, const qmm_weights* 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return QMM_ERR_CUDA;
-  set_variant("iq4_tile<mode=%d,s=%d,spw=%d,wpc=%d,w16=%d,spec=%d,grid=%d>", MODE, S, SPW, wpc, W16 ? 1 : 0, a.spec,
-              (int)grid);
+  set_variant("iq4_tile<mode=%d,s=%d,spw=%d,wpc=%d,w16=%d,spec=%d,route=%s,grid=%d>", MODE, S, SPW, wpc, W16 ? 1 : 0,
+              a.spec, ids ? "in_kernel" : "sorted", (int)grid);
   return launch_status();
 }
 
@@ -772,7 +775,7 @@ static qmm_status launch_iq4_tile_cfg(const qmm_weights* w0, const qmm_weights* 
 template <int MODE>
 static qmm_status launch_iq4_tile(const qmm_weights* w0, const qmm_weights* w1, const uint16_t* x, int x_per_pair,
                                   int64_t topk, const int32_t* offsets, const int32_t* perm, int64_t P, int m_plain,
-                                  void* y, const float* gw, cudaStream_t st) {
+                                  void* y, const float* gw, cudaStream_t st, const int32_t* ids) {
   if (w0->fmt != QMM_FMT_IQ4_NL || (w1 && w1->fmt != QMM_FMT_IQ4_NL)) return QMM_ERR_UNSUPPORTED_SHAPE;
   const int64_t k = w0->k, n = w0->n;
   if (k % 128 || k < 128 || n < 1 || n > INT32_MAX / 2) return QMM_ERR_UNSUPPORTED_SHAPE;
@@ -785,10 +788,10 @@ static qmm_status launch_iq4_tile(const qmm_weights* w0, const qmm_weights* w1, 
   // would need 20 warps of ~128 registers (more than an SM holds).
   if (steps % 2 == 0 && steps / 2 <= iqt_max_threads(96) / 32)
     return launch_iq4_tile_cfg<MODE, 2, 2, 96, true>(w0, w1, x, x_per_pair, topk, offsets, perm, P, m_plain, y, gw,
-                                                     st);
+                                                     st, ids);
   if (steps <= iqt_max_threads(128) / 32)
     return launch_iq4_tile_cfg<MODE, 4, 1, 128, false>(w0, w1, x, x_per_pair, topk, offsets, perm, P, m_plain, y, gw,
-                                                       st);
+                                                       st, ids);
   return QMM_ERR_UNSUPPORTED_SHAPE;
 }
 
@@ -1189,6 +1192,19 @@ qmm_status qmm_grouped_gemv(const qmm_weights* experts, const uint16_t* x, int32
     s = launch_iq4_persist<IQ_OUT_F16>(experts, nullptr, x, x_per_pair, topk, topk_ids, P, 0, y, nullptr, st, di);
     if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
   }
+  // IQ4_NL: the tile-resident kernel (its weight loads overlap the previous
+  // kernel when most experts have pairs); up to kIqtInKernelRoutePairs pairs
+  // each CTA finds its expert's pairs itself, so no routing pass runs.
+  // QMM_GEMV_VARIANT=iq4 keeps the streaming kernel.
+  const bool iq4_tile = pick == 10 || pick == 0;
+  if (experts->fmt == QMM_FMT_IQ4_NL && experts->k > 0 && iq4_tile && P <= kIqtInKernelRoutePairs) {
+    s = launch_iq4_tile<IQ_OUT_F16>(experts, nullptr, x, x_per_pair, topk, nullptr, nullptr, P, 0, y, nullptr, st,
+                                    topk_ids);
+    if (s != QMM_ERR_UNSUPPORTED_SHAPE) {
+      set_variant("grouped_iq4_tile+in_kernel_route");
+      return s;
+    }
+  }
   int32_t* offsets = static_cast<int32_t*>(ws);
   int32_t* perm = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + align256(4 * (size_t)(experts->num_experts + 1)));
   route_kernel<<<1, kRouteThreads, 0, st>>>(topk_ids, (int)P, (int)experts->num_experts, offsets, perm);
@@ -1199,11 +1215,7 @@ qmm_status qmm_grouped_gemv(const qmm_weights* experts, const uint16_t* x, int32
     set_variant("route+zero_fill");
     return launch_status();
   }
-  // IQ4_NL: the tile-resident kernel (its weight loads overlap the routing
-  // pass when most experts have pairs); QMM_GEMV_VARIANT=iq4 keeps the
-  // streaming kernel
-  const bool iq4_tile = pick == 10 || pick == 0;
-  if (experts->fmt == QMM_FMT_IQ4_NL && iq4_tile) {
+  if (experts->fmt == QMM_FMT_IQ4_NL && iq4_tile) {  // more pairs: after the routing sort
     s = launch_iq4_tile<IQ_OUT_F16>(experts, nullptr, x, x_per_pair, topk, offsets, perm, P, 0, y, nullptr, st);
     if (s != QMM_ERR_UNSUPPORTED_SHAPE) {
       set_variant("route+grouped_iq4_tile");
@@ -1347,6 +1359,25 @@ qmm_status qmm_moe_routed(const qmm_weights* gate, const qmm_weights* up, const 
     }
     if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
   }
+  // tile-resident kernels (measured faster than the streaming ones at 1, 4,
+  // 16 and 64 tokens); up to kIqtInKernelRoutePairs pairs each CTA finds its
+  // expert's pairs itself, so no routing pass runs.  QMM_GEMV_VARIANT=iq4
+  // keeps the streaming kernels.
+  const int pick = gemv_variant_env();
+  const bool tile = pick == 10 || pick == 0;
+  if (f > 0 && tile && P <= kIqtInKernelRoutePairs) {
+    s = launch_iq4_tile<IQ_SWIGLU>(gate, up, x, 0, topk, nullptr, nullptr, P, 0, h, nullptr, st, topk_ids);
+    if (s == QMM_OK)
+      s = launch_iq4_tile<IQ_SCALED_F32>(down, nullptr, h, 1, topk, nullptr, nullptr, P, 0, yg, topk_weights, st,
+                                         topk_ids);
+    if (s == QMM_OK) {
+      combine_kernel<<<grid_for(t * (d / 8), 256, di->sms), 256, 0, st>>>(yg, topk_ids, (int)E, (int)t, (int)topk,
+                                                                           (int)d, out);
+      set_variant("moe:gate_up_swiglu_iq4_tile+down_scaled_iq4_tile+combine(in-kernel routing)");
+      return launch_status();
+    }
+    if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
+  }
   route_kernel<<<1, kRouteThreads, 0, st>>>(topk_ids, (int)P, (int)E, offsets, perm);
   if (cudaGetLastError() != cudaSuccess) return QMM_ERR_CUDA;
   if (f == 0) {
@@ -1355,10 +1386,7 @@ qmm_status qmm_moe_routed(const qmm_weights* gate, const qmm_weights* up, const 
     set_variant("moe:route+zero_fill");
     return launch_status();
   }
-  // tile-resident kernels (measured faster than the streaming ones at 1, 4,
-  // 16 and 64 tokens); QMM_GEMV_VARIANT=iq4 keeps the streaming kernels
-  const int pick = gemv_variant_env();
-  if (pick == 10 || pick == 0) {
+  if (tile) {  // more pairs: after the routing sort
     s = launch_iq4_tile<IQ_SWIGLU>(gate, up, x, 0, topk, offsets, perm, P, 0, h, nullptr, st);
     if (s == QMM_OK)
       s = launch_iq4_tile<IQ_SCALED_F32>(down, nullptr, h, 1, topk, offsets, perm, P, 0, yg, topk_weights, st);
@@ -1370,7 +1398,7 @@ qmm_status qmm_moe_routed(const qmm_weights* gate, const qmm_weights* up, const 
     }
     if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
   }
-  if (gemv_variant_env() == 9) {  // warp-per-tile kernels
+  if (pick == 9) {  // warp-per-tile kernels
     s = launch_iq4_warp<IQ_SWIGLU>(gate, up, x, 0, topk, offsets, perm, 0, h, nullptr, st, di);
     if (s == QMM_OK)
       s = launch_iq4_warp<IQ_SCALED_F32>(down, nullptr, h, 1, topk, offsets, perm, 0, yg, topk_weights, st, di);

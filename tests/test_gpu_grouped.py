@@ -131,7 +131,7 @@ def test_grouped_iq4_many_pairs_per_expert(variant, E, n, k, t, topk, per_pair, 
     elif variant == "iq4w":
         assert v.startswith("route+grouped_iq4_warp"), v
     elif variant == "iq4t":
-        assert v.startswith("route+grouped_iq4_tile"), v
+        assert "grouped_iq4_tile" in v, v
     elif variant == "iq4":
         assert v.startswith("route+grouped_iq4_stream"), v
     else:
@@ -153,13 +153,16 @@ def test_grouped_iq4_many_pairs_per_expert(variant, E, n, k, t, topk, per_pair, 
 @pytest.mark.parametrize("spec", ["0", "1"])
 @pytest.mark.parametrize("E,n,k,t,topk,per_pair", [(32, 1792, 2560, 64, 4, False), (32, 2560, 896, 64, 4, True),
                                                     (32, 2560, 896, 1, 4, True), (7, 1000, 1152, 37, 3, False),
-                                                    (4, 72, 4096, 20, 2, False)])
+                                                    (4, 72, 4096, 20, 2, False), (2, 72, 4096, 16, 2, False),
+                                                    (3, 100, 896, 10, 3, True)])
 def test_grouped_iq4_tile_kernel(spec, E, n, k, t, topk, per_pair, monkeypatch):
     """The tile-resident IQ4_NL kernel with its weight loads before and after
     the dependency wait, items of two tiles (two super-steps per warp, k %
     256 == 0) or four (one super-step per warp: k = 896, 1152), ragged last
-    items (n = 1000, 72) and the routed-expert shapes (gate+up 1792 x 2560,
-    down 2560 x 896 at 64 and 1 tokens)."""
+    items (n = 1000, 72), the routed-expert shapes (gate+up 1792 x 2560, down
+    2560 x 896 at 64 and 1 tokens), and routing inside the kernel (at most 32
+    pairs; 16 tokens x 2 over 2 experts puts more than one token group on an
+    expert)."""
     monkeypatch.setenv("QMM_GEMV_VARIANT", "iq4t")
     monkeypatch.setenv("QMM_IQ4T_SPEC", spec)
     rng = np.random.default_rng(E * 7 + n + k + t)
@@ -168,7 +171,7 @@ def test_grouped_iq4_tile_kernel(spec, E, n, k, t, topk, per_pair, monkeypatch):
     ids = synth.gen_topk(rng, t, topk, E)
     y, st = _grouped(dev(p), x, ids, per_pair)
     v = qmm.qmm_last_variant()
-    assert st == 0 and v.startswith("route+grouped_iq4_tile"), v
+    assert st == 0 and "grouped_iq4_tile" in v, v
     if per_pair:
         xs = x.reshape(t * topk, k)
         yref = np.empty((t * topk, n)); absy = np.empty((t * topk, n))
@@ -182,3 +185,28 @@ def test_grouped_iq4_tile_kernel(spec, E, n, k, t, topk, per_pair, monkeypatch):
         yref, absy = oracle.grouped_gemv(synth.FMT_IQ4_NL, n, k, p.data, p.data_stride, None, 0, 1.0, E, x, ids)
     check_tol(y, yref, absy, "grouped iq4 tile %s" % v)
 
+
+
+@pytest.mark.parametrize("variant", [None, "iq4"])
+def test_grouped_iq4_out_of_range_ids_are_left_out_and_flagged(variant, monkeypatch):
+    """IQ4_NL experts with ids outside [0, E): the default kernel routes in
+    the kernel (no routing pass), the streaming one after the routing sort;
+    both flag QMM_ERR_DEVICE_FAULT, leave those pairs' rows unwritten and
+    compute every other pair."""
+    if variant:
+        monkeypatch.setenv("QMM_GEMV_VARIANT", variant)
+    rng = np.random.default_rng(1234)
+    E, n, k, t, topk = 6, 64, 256, 12, 2  # 24 pairs: routed inside the kernel by default
+    p = synth.gen_weights(rng, synth.FMT_IQ4_NL, n, k, experts=E)
+    x = synth.gen_x(rng, t, k)
+    ids = synth.gen_topk(rng, t, topk, E)
+    ids[3, 1] = E
+    ids[7, 0] = -1
+    y, st = _grouped(dev(p), x, ids, False)
+    v = qmm.qmm_last_variant()
+    assert st == 7, v  # QMM_ERR_DEVICE_FAULT
+    valid = (ids >= 0) & (ids < E)
+    assert np.all(y[~valid] == 0x5A5A), v
+    yref, absy = oracle.grouped_gemv(synth.FMT_IQ4_NL, n, k, p.data, p.data_stride, None, 0, 1.0, E, x,
+                                     np.where(valid, ids, 0))
+    check_tol(y[valid], yref[valid], absy[valid], "bad ids %s" % v)
