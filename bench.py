@@ -14,6 +14,11 @@ back-to-back launches, bracketed by a barrier and synchronisation, timed with
 CUDA events on the launching stream, max over ranks.  The weights rotate over
 enough device copies to exceed 4x the L2 size, so every step streams from HBM.
 
+``e2e``: the same GEMV through ``qmm_gemv_host`` (the call a serving loop
+makes with host buffers): every step brings the token's activations in from
+pinned host memory and writes y back to pinned host memory, timed the same
+way.
+
 ``--impl reference`` times the CPU oracle (plain C, one host thread) on a
 bounded sample of the same workload instead.
 """
