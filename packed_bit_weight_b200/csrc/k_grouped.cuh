@@ -223,7 +223,6 @@ __device__ __forceinline__ void iq4_pass(float (&acc)[4][4], const uint8_t* __re
 #pragma unroll
   for (int u = 0; u < SMAX; u++) {
     if (s_lo + u >= s_hi) break;
-    const int b = 4 * (s_lo + u) + tig;
     uint32_t da, db, qa[4], qb[4];
     if (tig & 1) {  // block starts 2 bytes into word 0
       da = wa[u][0] >> 16;
