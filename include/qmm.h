@@ -212,9 +212,14 @@ qmm_status qmm_route(const int32_t* topk_ids, int64_t t, int64_t topk, int64_t n
  * (x_per_pair = 1, x is [t][topk][k]).  Each expert's weights are read once
  * for all of the pairs routed to it.  Pairs with an id out of range leave
  * their y row untouched and set QMM_ERR_DEVICE_FAULT in the error word.
+ * IQ4_NL experts are launched with programmatic dependent launch (their
+ * weights may be read while the kernel before them on the stream still
+ * runs, as for qmm_gemv: the experts must not be written by that kernel).
  *   experts   a stack of num_experts matrices (expert_*_stride set)
  *   y         device, [t][topk][n] fp16
- *   ws        device workspace (qmm_workspace_bytes(QMM_OP_GROUPED, ...))
+ *   ws        device workspace (qmm_workspace_bytes(QMM_OP_GROUPED, ...));
+ *             scratch for the routing sort (IQ4_NL with at most 32 pairs
+ *             routes inside the expert kernel and leaves it untouched)
  * Errors: as qmm_gemv. */
 qmm_status qmm_grouped_gemv(const qmm_weights* experts, const uint16_t* x, int32_t x_per_pair,
                             const int32_t* topk_ids, int64_t t, int64_t topk, uint16_t* y, void* ws,
@@ -275,12 +280,15 @@ qmm_status qmm_router_topk(const uint16_t* x, const uint16_t* w_router, const fl
  * ffn_down_exps, section "Quantization"):
  *   out[t][:] = sum_s topk_weights[t][s] * W_down,e (h_{t,s}),
  *   h_{t,s}   = fp16(SiLU(W_gate,e x_t) * (W_up,e x_t)),  e = topk_ids[t][s].
- * Three kernels after the routing sort: gate and up are multiplied in one
+ * Three kernels after the routing sort (up to 32 pairs the expert kernels
+ * route themselves and no sort runs): gate and up are multiplied in one
  * pass over the same row tiles with SiLU(gate) * up applied before the only
  * fp16 rounding of h; the down projection multiplies each expert's pairs,
  * scales them by g in fp32 and keeps them in fp32; a last pass adds a
  * token's slots in slot order and rounds once to fp16.  The shared experts
- * of the formula are this same call with ids {0, 1} and weights 1.
+ * of the formula are this same call with ids {0, 1} and weights 1.  The
+ * expert kernels use programmatic dependent launch: gate/up/down must not be
+ * written by the kernel that immediately precedes this call.
  *   gate, up     IQ4_NL stacks of num_experts matrices [f][d] (same f, d, E)
  *   down         IQ4_NL stack of num_experts matrices [d][f]
  *   x            device, [t][d] fp16
@@ -293,7 +301,8 @@ qmm_status qmm_router_topk(const uint16_t* x, const uint16_t* w_router, const fl
  *                [t*topk] int32 | h [t*topk][f] fp16 | g-scaled slot outputs
  *                [t*topk][d] fp32, each part starting on a 256-byte
  *                boundary; after the call h is readable there (pairs with an
- *                out-of-range id hold stale data)
+ *                out-of-range id hold stale data; offsets and pair_perm are
+ *                written only when the routing sort runs)
  * Limits: d % 128 == 0, f % 128 == 0 (whole 4-block super-steps per row).
  * Errors: as qmm_grouped_gemv. */
 qmm_status qmm_moe_routed(const qmm_weights* gate, const qmm_weights* up, const qmm_weights* down,
