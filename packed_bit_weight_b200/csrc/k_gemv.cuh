@@ -636,7 +636,7 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
   ldg_tile_store<FMT, NT, WPC>(red, acc, warp, grp, tig, n0, n, m, g, y);
   if (rows1 <= 0) return;
 
-  // second tile: every lane waits for the copies (bounded); the verdict is
+  // second tile: every lane waits for the copies (bounded); the decision is
   // made warp-uniform so the MMAs never run in a diverged warp
   const bool ready = __all_sync(0xFFFFFFFFu, mbar_wait(bar, 0));
   if (ready) {

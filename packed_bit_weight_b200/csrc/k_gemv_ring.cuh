@@ -221,7 +221,7 @@ __global__ void __maxnreg__((65536 / (2 * 32 * (CW + 1))) & ~7)
 #pragma unroll
         for (int c = 0; c < 4; c++) acc[i][j][c] = 0.f;
     const uint32_t slot = it % S;
-    // every lane waits (each needs the copies visible); the verdict is made
+    // every lane waits (each needs the copies visible); the decision is made
     // warp-uniform so the MMAs below never run in a diverged warp
     const bool ready = __all_sync(0xFFFFFFFFu, !fail && mbar_wait(full + 8u * slot, (it / S) & 1u));
     // this warp's segments s = cw + i*CW (at most SPW, k <= 128*CW*SPW) are read
