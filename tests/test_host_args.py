@@ -65,3 +65,88 @@ def test_binding_rejects_device_tensors_as_host_buffers():
         qmm.qmm_gemv_host(w, xh, yh, xh, yh)
     with pytest.raises(ValueError):                        # host buffers must be contiguous
         qmm.qmm_gemv_host(w, xh.view(-1)[:128].view(1, 128).t(), yh, xh, yh)
+
+
+def _stack(fmt=1, n=64, k=256, experts=4, data_stride=None, scale_stride=None):
+    d = _desc(fmt=fmt, n=n, k=k, scales=None if fmt == 1 else FAKE + (1 << 20))
+    d.num_experts = experts
+    db, sb = qmm.qmm_data_bytes(fmt, n, k), qmm.qmm_scale_bytes(fmt, n, k)
+    d.expert_data_stride = db if data_stride is None else data_stride
+    d.expert_scale_stride = sb if scale_stride is None else scale_stride
+    return d
+
+
+def _vp(a):
+    return ctypes.c_void_p(a) if a else None
+
+
+def test_gemm_argument_errors():
+    L = qmm._lib()
+    assert L.qmm_gemm(None, _vp(FAKE), 4, _vp(FAKE), None, 0, None) == INVALID
+    assert L.qmm_gemm(ctypes.byref(_desc()), _vp(FAKE), -1, _vp(FAKE), None, 0, None) == INVALID
+    assert L.qmm_gemm(ctypes.byref(_desc(k=250)), _vp(FAKE), 4, _vp(FAKE), None, 0, None) == UNSUPPORTED
+
+
+def test_grouped_argument_errors():
+    L = qmm._lib()
+    ids = _vp(FAKE + (4 << 20))
+
+    def call(d, t=8, topk=2, per_pair=0, ids=ids):
+        return L.qmm_grouped_gemv(ctypes.byref(d), _vp(FAKE), per_pair, ids, t, topk, _vp(FAKE), None, 0, None)
+
+    assert call(_stack(data_stride=100)) == INVALID                        # stride below one matrix
+    assert call(_stack(data_stride=qmm.qmm_data_bytes(1, 64, 256) + 8)) == MISALIGNED
+    assert call(_stack(), t=-1) == INVALID
+    assert call(_stack(experts=257)) == UNSUPPORTED                         # at most 256 experts
+    assert call(_stack(), ids=None) == INVALID                              # pairs but no ids
+    assert call(_stack(), ids=_vp(FAKE + 4)) == MISALIGNED
+    assert call(_stack(), per_pair=2) == INVALID
+    assert call(_stack(fmt=2, scale_stride=4)) == INVALID                  # FP4 scale stride below one matrix
+
+
+def test_route_argument_errors():
+    L = qmm._lib()
+    ids = _vp(FAKE)
+    assert L.qmm_route(ids, 8, 2, 4, None, _vp(FAKE + 256), None, 0, None) == INVALID   # no offsets
+    assert L.qmm_route(ids, 8, 2, 4, _vp(FAKE + 256), None, None, 0, None) == INVALID   # no permutation
+    assert L.qmm_route(ids, 8, 2, 4, _vp(FAKE + 8), _vp(FAKE + 256), None, 0, None) == MISALIGNED
+    assert L.qmm_route(ids, 8, 2, 0, _vp(FAKE + 256), _vp(FAKE + 512), None, 0, None) == INVALID  # no experts
+
+
+def test_moe_argument_errors():
+    L = qmm._lib()
+    E, f, d = 4, 128, 256
+    gate, up, down = _stack(n=f, k=d, experts=E), _stack(n=f, k=d, experts=E), _stack(n=d, k=f, experts=E)
+
+    def call(g=gate, u=up, dn=down, t=8, topk=2):
+        return L.qmm_moe_routed(ctypes.byref(g), ctypes.byref(u), ctypes.byref(dn), _vp(FAKE), _vp(FAKE + 4096),
+                                _vp(FAKE + 8192), t, topk, _vp(FAKE), None, 0, None)
+
+    assert call(g=_stack(fmt=2, n=f, k=d, experts=E)) == UNSUPPORTED       # the expert kernels are IQ4_NL
+    assert call(u=_stack(n=f + 16, k=d, experts=E)) == INVALID             # gate and up differ
+    assert call(dn=_stack(n=d, k=f, experts=E + 1)) == INVALID             # expert counts differ
+    assert call(t=-1) == INVALID
+    g2, u2 = _stack(n=f, k=160, experts=E), _stack(n=f, k=160, experts=E)
+    assert call(g=g2, u=u2, dn=_stack(n=160, k=f, experts=E)) == UNSUPPORTED  # d % 128 != 0
+
+
+def test_router_and_quantize_argument_errors():
+    L = qmm._lib()
+    p = _vp(FAKE)
+    # x, w_router, bias, t, k, E, topk, ids, weights, logits, stream
+    assert L.qmm_router_topk(p, p, p, 4, 256, 8, 9, p, p, None, None) == INVALID        # topk > E
+    assert L.qmm_router_topk(p, p, p, 4, 250, 8, 2, p, p, None, None) == UNSUPPORTED    # k % 8
+    assert L.qmm_router_topk(p, p, p, 4, 256, 300, 2, p, p, None, None) == UNSUPPORTED  # too many experts
+    assert L.qmm_router_topk(p, p, p, -1, 256, 8, 2, p, p, None, None) == INVALID
+    # fmt, w, n, k, data, scales, stream
+    assert L.qmm_quantize(9, p, 4, 256, p, p, None) == INVALID
+    assert L.qmm_quantize(3, p, 4, 256, p, p, None) == UNSUPPORTED      # E4M3 needs a matrix-wide scale
+    assert L.qmm_quantize(2, p, 4, 250, p, p, None) == UNSUPPORTED
+    assert L.qmm_quantize(2, p, -1, 256, p, p, None) == INVALID
+
+
+def test_workspace_size_rejects_bad_descriptors():
+    L = qmm._lib()
+    assert L.qmm_workspace_bytes(qmm.OP_GROUPED, None, 0, 8, 2) == 0
+    assert L.qmm_workspace_bytes(qmm.OP_GROUPED, ctypes.byref(_stack()), 0, -1, 2) == 0
+    assert L.qmm_workspace_bytes(qmm.OP_GROUPED, ctypes.byref(_stack()), 0, 8, 2) > 0
