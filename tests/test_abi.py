@@ -3,6 +3,7 @@ declares (no GPU needed: no compute call is made)."""
 import ctypes
 import os
 import re
+import subprocess
 
 import pytest
 
@@ -74,3 +75,53 @@ def test_product_path_does_not_import_the_oracle():
             if fn.endswith((".py", ".cu", ".cuh", ".h")):
                 src = open(os.path.join(dirpath, fn)).read()
                 assert "import oracle" not in src and "from oracle" not in src and "qmm_oracle" not in src, fn
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "qmm.h"
+
+int main(void) {
+  qmm_weights w;
+  memset(&w, 0, sizeof w);
+  w.fmt = QMM_FMT_FP4G16_F16;
+  w.n = 18560;
+  w.k = 4096;
+  w.num_experts = 1;
+  w.data = (const void*)(uintptr_t)0x10000;
+  w.scales = (const void*)(uintptr_t)0x20000;
+  /* in_proj at fp16 scales: 47,513,600 packed bytes */
+  if (qmm_packed_bytes(QMM_FMT_FP4G16_F16, 18560, 4096) != 47513600u) return 1;
+  if (qmm_data_bytes(QMM_FMT_IQ4_NL, 256, 512) != 73728u) return 2;
+  if (qmm_scale_bytes(QMM_FMT_MXFP4, 4, 64) != 8u) return 3;
+  if (qmm_packed_bytes(99, 4, 64) != 0u) return 4;
+  /* argument errors return before any device call */
+  w.fmt = 99;
+  if (qmm_gemv(&w, (const uint16_t*)(uintptr_t)0x30000, 1, (uint16_t*)(uintptr_t)0x40000, NULL, 0, NULL)
+      != QMM_ERR_INVALID_ARG) return 5;
+  if (qmm_gemv(NULL, NULL, 1, NULL, NULL, 0, NULL) != QMM_ERR_INVALID_ARG) return 6;
+  if (strlen(qmm_status_string(QMM_ERR_MISALIGNED)) == 0) return 7;
+  printf("ok\n");
+  return 0;
+}
+"""
+
+
+@pytest.mark.parametrize("lang", ["c", "c++"])
+def test_plain_c_client_links_and_calls_the_library(tmp_path, lang):
+    """The header is valid C99 and C++ (no C++ or torch types cross the
+    boundary), and a C program linked against libqmm.so alone reaches the
+    size queries and the host-side argument checks."""
+    from packed_bit_weight_b200 import _build
+    lib = _build.build()
+    src = tmp_path / ("client.c" if lang == "c" else "client.cpp")
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    cc = ["gcc", "-std=c99"] if lang == "c" else ["g++", "-std=c++17"]
+    cmd = cc + ["-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                lib, "-Wl,-rpath," + os.path.dirname(lib)]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
