@@ -1,9 +1,10 @@
 """ctypes binding of libqmm.so (include/qmm.h).
 
 Argument marshalling only: every function here takes torch tensors, checks
-that they are CUDA tensors of the right element size, passes raw device
-pointers and the current CUDA stream to the C ABI, and raises ``QmmError`` on
-a non-OK status.  No arithmetic of the path happens in Python, and there is
+that they are CUDA tensors of the right element size and that each holds at
+least the bytes the call will read or write (the C ABI takes bare pointers
+and cannot see a buffer's extent), passes raw device pointers and the current
+CUDA stream to the C ABI, and raises ``QmmError`` on a non-OK status.  No arithmetic of the path happens in Python, and there is
 no fallback: if the library is missing the first call raises.
 """
 from __future__ import annotations
@@ -96,6 +97,14 @@ def _stream(stream=None):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _need(t: torch.Tensor | None, nbytes: int, name: str) -> None:
+    """Refuse a tensor smaller than the bytes the C call touches through its
+    pointer: an undersized buffer would otherwise be an out-of-bounds access
+    on the device instead of an error here.  None is left to the C checks."""
+    if t is not None and t.nbytes < nbytes:
+        raise ValueError("%s holds %d bytes; the call reads or writes %d" % (name, t.nbytes, nbytes))
+
+
 def _ptr(t: torch.Tensor | None, esize: int | None = None, name: str = "tensor"):
     if t is None:
         return None
@@ -123,9 +132,9 @@ class PackedWeights:
 
     def desc(self) -> qmm_weights:
         """The C descriptor, rebuilt only when a field or a buffer changed."""
-        key = (self.fmt, self.n, self.k, None if self.data is None else self.data.data_ptr(),
-               None if self.scales is None else self.scales.data_ptr(), self.global_scale, self.experts,
-               self.data_stride, self.scale_stride)
+        key = (self.fmt, self.n, self.k, None if self.data is None else (self.data.data_ptr(), self.data.numel()),
+               None if self.scales is None else (self.scales.data_ptr(), self.scales.numel()), self.global_scale,
+               self.experts, self.data_stride, self.scale_stride)
         cached = self.__dict__.get("_desc")
         if cached is not None and cached[0] == key:
             return cached[1]
@@ -148,6 +157,12 @@ class PackedWeights:
         else:
             d.expert_scale_stride = (self.scales.numel() * self.scales.element_size() // self.experts
                                      if self.scales is not None else 0)
+        # every expert's codes and scales must lie inside the tensors (the
+        # sizes are 0 for a shape the C checks reject anyway)
+        last = max(int(self.experts), 1) - 1
+        db, sb = qmm_data_bytes(self.fmt, self.n, self.k), qmm_scale_bytes(self.fmt, self.n, self.k)
+        _need(self.data, last * d.expert_data_stride + db if db else 0, "data")
+        _need(self.scales, last * d.expert_scale_stride + sb if sb else 0, "scales")
         return d
 
     def rows(self, r0: int, r1: int) -> "PackedWeights":
@@ -209,6 +224,7 @@ def qmm_workspace_bytes(op: int, w: PackedWeights | None, m: int = 0, t: int = 0
 
 def qmm_dequant(w: PackedWeights, out: torch.Tensor, stream=None) -> torch.Tensor:
     d = w.desc()
+    _need(out, 2 * w.n * w.k, "out")
     _check(_lib().qmm_dequant(ctypes.byref(d), _ptr(out, 2, "out"), _stream(stream)), "qmm_dequant")
     return out
 
@@ -217,6 +233,8 @@ def qmm_quantize(fmt: int, w: torch.Tensor, data: torch.Tensor, scales: torch.Te
                  stream=None) -> None:
     """fp16 weights w [n][k] (2-byte elements) -> packed data / scales."""
     n, k = w.shape
+    _need(data, qmm_data_bytes(fmt, n, k), "data")
+    _need(scales, qmm_scale_bytes(fmt, n, k), "scales")
     _check(_lib().qmm_quantize(fmt, _ptr(w, 2, "w"), n, k, _ptr(data, None, "data"), _ptr(scales, None, "scales"),
                                _stream(stream)), "qmm_quantize")
 
@@ -230,6 +248,8 @@ def qmm_gemv(w: PackedWeights, x: torch.Tensor, y: torch.Tensor, ws: torch.Tenso
     d = w.desc()
     wp, wb = _ws(ws)
     m = x.shape[0] if x.dim() == 2 else 1
+    _need(x, 2 * m * w.k, "x")
+    _need(y, 2 * m * w.n, "y")
     _check(_lib().qmm_gemv(ctypes.byref(d), _ptr(x, 2, "x"), m, _ptr(y, 2, "y"), wp, wb, _stream(stream)), "qmm_gemv")
     return y
 
@@ -251,6 +271,11 @@ def qmm_gemv_host(w: PackedWeights, x_host: torch.Tensor, y_host: torch.Tensor, 
     when the host tensors are pinned)."""
     d = w.desc()
     m = x_host.shape[0] if x_host.dim() == 2 else 1
+    xb, yb = 2 * m * w.k, 2 * m * w.n
+    _need(x_host, xb, "x_host")
+    _need(x_dev, xb, "x_dev")
+    _need(y_host, yb, "y_host")
+    _need(y_dev, yb, "y_dev")
     _check(_lib().qmm_gemv_host(ctypes.byref(d), _host_ptr(x_host, 2, "x_host"), m, _host_ptr(y_host, 2, "y_host"),
                                 _ptr(x_dev, 2, "x_dev"), _ptr(y_dev, 2, "y_dev"), _stream(stream)), "qmm_gemv_host")
     return y_host
@@ -260,6 +285,8 @@ def qmm_gemm(w: PackedWeights, x: torch.Tensor, y: torch.Tensor, ws: torch.Tenso
              stream=None) -> torch.Tensor:
     d = w.desc()
     wp, wb = _ws(ws)
+    _need(x, 2 * x.shape[0] * w.k, "x")
+    _need(y, 2 * x.shape[0] * w.n, "y")
     _check(_lib().qmm_gemm(ctypes.byref(d), _ptr(x, 2, "x"), x.shape[0], _ptr(y, 2, "y"), wp, wb, _stream(stream)),
            "qmm_gemm")
     return y
@@ -269,15 +296,24 @@ def qmm_route(topk_ids: torch.Tensor, num_experts: int, offsets: torch.Tensor, p
               ws: torch.Tensor | None = None, stream=None):
     t, topk = topk_ids.shape
     wp, wb = _ws(ws)
+    _need(offsets, 4 * (num_experts + 1), "offsets")
+    _need(perm, 4 * t * topk, "perm")
     _check(_lib().qmm_route(_ptr(topk_ids, 4, "topk_ids"), t, topk, num_experts, _ptr(offsets, 4, "offsets"),
                             _ptr(perm, 4, "perm"), wp, wb, _stream(stream)), "qmm_route")
     return offsets, perm
 
 
+def _need_grouped(w: PackedWeights, x, topk_ids, y, x_per_pair):
+    t, topk = topk_ids.shape
+    _need(x, 2 * w.k * (t * topk if x_per_pair else t), "x")
+    _need(y, 2 * t * topk * w.n, "y")
+    return t, topk
+
+
 def qmm_grouped_gemv(w: PackedWeights, x: torch.Tensor, topk_ids: torch.Tensor, y: torch.Tensor,
                      x_per_pair: bool = False, ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     d = w.desc()
-    t, topk = topk_ids.shape
+    t, topk = _need_grouped(w, x, topk_ids, y, x_per_pair)
     wp, wb = _ws(ws)
     _check(_lib().qmm_grouped_gemv(ctypes.byref(d), _ptr(x, 2, "x"), int(bool(x_per_pair)),
                                    _ptr(topk_ids, 4, "topk_ids"), t, topk, _ptr(y, 2, "y"), wp, wb,
@@ -291,7 +327,7 @@ def qmm_grouped_gemv_noalloc(w: PackedWeights, x: torch.Tensor, topk_ids: torch.
     library's own fixed device array (at most 65536 pairs, 256 experts; calls
     that overlap on the GPU race on it)."""
     d = w.desc()
-    t, topk = topk_ids.shape
+    t, topk = _need_grouped(w, x, topk_ids, y, x_per_pair)
     _check(_lib().qmm_grouped_gemv_noalloc(ctypes.byref(d), _ptr(x, 2, "x"), int(bool(x_per_pair)),
                                            _ptr(topk_ids, 4, "topk_ids"), t, topk, _ptr(y, 2, "y"),
                                            _stream(stream)), "qmm_grouped_gemv_noalloc")
@@ -305,6 +341,10 @@ def qmm_router_topk(x: torch.Tensor, w_router: torch.Tensor, bias: torch.Tensor,
     top-k experts with their softmax weights."""
     t, k = x.shape
     E = w_router.shape[0]
+    for tt, nb, name in ((w_router, 2 * E * k, "w_router"), (bias, 4 * E, "bias"),
+                         (topk_ids, 4 * t * topk, "topk_ids"), (topk_weights, 4 * t * topk, "topk_weights"),
+                         (logits, 4 * t * E, "logits")):
+        _need(tt, nb, name)
     _check(_lib().qmm_router_topk(_ptr(x, 2, "x"), _ptr(w_router, 2, "w_router"), _ptr(bias, 4, "bias"), t, k, E,
                                   topk, _ptr(topk_ids, 4, "topk_ids"), _ptr(topk_weights, 4, "topk_weights"),
                                   _ptr(logits, 4, "logits"), _stream(stream)), "qmm_router_topk")
@@ -318,6 +358,9 @@ def qmm_moe_routed(gate: PackedWeights, up: PackedWeights, down: PackedWeights, 
     dg, du, dd = gate.desc(), up.desc(), down.desc()
     t, topk = topk_ids.shape
     wp, wb = _ws(ws)
+    _need(x, 2 * t * gate.k, "x")
+    _need(topk_weights, 4 * t * topk, "topk_weights")
+    _need(out, 2 * t * down.n, "out")
     _check(_lib().qmm_moe_routed(ctypes.byref(dg), ctypes.byref(du), ctypes.byref(dd), _ptr(x, 2, "x"),
                                  _ptr(topk_ids, 4, "topk_ids"), _ptr(topk_weights, 4, "topk_weights"), t, topk,
                                  _ptr(out, 2, "out"), wp, wb, _stream(stream)), "qmm_moe_routed")

@@ -150,3 +150,63 @@ def test_workspace_size_rejects_bad_descriptors():
     assert L.qmm_workspace_bytes(qmm.OP_GROUPED, None, 0, 8, 2) == 0
     assert L.qmm_workspace_bytes(qmm.OP_GROUPED, ctypes.byref(_stack()), 0, -1, 2) == 0
     assert L.qmm_workspace_bytes(qmm.OP_GROUPED, ctypes.byref(_stack()), 0, 8, 2) > 0
+
+
+def _pw(fmt=2, n=64, k=256, experts=1, short=0, scales_short=0):
+    torch = pytest.importorskip("torch")
+    db, sb = qmm.qmm_data_bytes(fmt, n, k) * experts, qmm.qmm_scale_bytes(fmt, n, k) * experts
+    sc = torch.zeros(sb - scales_short, dtype=torch.uint8) if sb else None
+    return qmm.PackedWeights(fmt, n, k, torch.zeros(db - short, dtype=torch.uint8), sc, 1.0, experts)
+
+
+def _short(fn, *a, **kw):
+    with pytest.raises(ValueError, match="holds"):
+        fn(*a, **kw)
+
+
+def test_binding_refuses_undersized_weight_tensors():
+    _short(lambda: _pw(short=16).desc())
+    _short(lambda: _pw(scales_short=2).desc())
+    _short(lambda: _pw(fmt=1, experts=3, short=18).desc())          # last expert's last block missing
+    _pw(fmt=1, experts=3).desc()                                     # exact sizes pass
+    _pw(fmt=2, k=250).desc()                                         # bad shape: left to the C checks
+
+
+def test_binding_refuses_undersized_buffers():
+    torch = pytest.importorskip("torch")
+    i16, i32, f32 = torch.int16, torch.int32, torch.float32
+    w = _pw()
+    z = lambda *s, dt=i16: torch.zeros(*s, dtype=dt)
+    _short(qmm.qmm_gemv, w, z(2, 256), z(2 * 64 - 1))                # y one element short
+    _short(qmm.qmm_gemv, w, z(2, 255), z(2, 64))                     # x rows shorter than k
+    _short(qmm.qmm_gemm, w, z(300, 256), z(299, 64))
+    _short(qmm.qmm_dequant, w, z(64 * 256 - 8))
+    _short(qmm.qmm_gemv_host, w, z(2, 256), z(2, 64), z(2, 256), z(2, 63))
+    _short(qmm.qmm_quantize, 2, z(64, 256), torch.zeros(64 * 128 - 1, dtype=torch.uint8),
+           torch.zeros(64 * 16 * 2, dtype=torch.uint8))
+    _short(qmm.qmm_quantize, 2, z(64, 256), torch.zeros(64 * 128, dtype=torch.uint8),
+           torch.zeros(64 * 16 * 2 - 1, dtype=torch.uint8))
+    ids = z(8, 2, dt=i32)
+    _short(qmm.qmm_route, ids, 4, z(4, dt=i32), z(16, dt=i32))       # offsets need E + 1
+    _short(qmm.qmm_route, ids, 4, z(5, dt=i32), z(15, dt=i32))       # perm needs t * topk
+    e = _pw(fmt=1, experts=4)
+    _short(qmm.qmm_grouped_gemv, e, z(8, 256), ids, z(8, 2, 63))
+    _short(qmm.qmm_grouped_gemv, e, z(8, 256), ids, z(8, 2, 64), x_per_pair=True)   # one x row per pair
+    _short(qmm.qmm_grouped_gemv_noalloc, e, z(7, 256), ids, z(8, 2, 64))
+    _short(qmm.qmm_router_topk, z(8, 256), z(4, 255), z(4, dt=f32), 2, ids, z(8, 2, dt=f32))
+    _short(qmm.qmm_router_topk, z(8, 256), z(4, 256), z(4, dt=f32), 2, ids, z(8, 2, dt=f32), z(8, 3, dt=f32))
+    g, u, d = _pw(fmt=1, n=128, k=256, experts=4), _pw(fmt=1, n=128, k=256, experts=4), _pw(fmt=1, n=256, k=128,
+                                                                                            experts=4)
+    _short(qmm.qmm_moe_routed, g, u, d, z(8, 256), ids, z(8, 1, dt=f32), z(8, 256))
+    _short(qmm.qmm_moe_routed, g, u, d, z(8, 256), ids, z(8, 2, dt=f32), z(8, 255))
+
+
+def test_binding_size_checks_pass_exact_buffers_on_to_the_device_check():
+    """Exactly sized buffers pass the size checks and are refused only
+    because they are host tensors (the device check that follows)."""
+    torch = pytest.importorskip("torch")
+    w = _pw()
+    with pytest.raises(ValueError, match="CUDA"):
+        qmm.qmm_gemv(w, torch.zeros(2, 256, dtype=torch.int16), torch.zeros(2, 64, dtype=torch.int16))
+    with pytest.raises(ValueError, match="CUDA"):
+        qmm.qmm_gemv(w, torch.zeros(0, 256, dtype=torch.int16), torch.zeros(0, 64, dtype=torch.int16))

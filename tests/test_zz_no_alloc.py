@@ -65,7 +65,7 @@ def test_noalloc_refuses_more_pairs_than_its_array_holds():
     t, topk = 16385, 4                         # 65540 pairs > 65536
     ids = torch.zeros((t, topk), dtype=torch.int32, device="cuda")
     x = torch.zeros((t, 64), dtype=torch.int16, device="cuda")
-    y = torch.zeros((1, 16), dtype=torch.int16, device="cuda")
+    y = torch.zeros((t, topk, 16), dtype=torch.int16, device="cuda")
     with pytest.raises(qmm.QmmError) as e:
         qmm.qmm_grouped_gemv_noalloc(w, x, ids, y)
     assert e.value.status == 2                 # QMM_ERR_UNSUPPORTED_SHAPE, nothing launched
