@@ -13,6 +13,9 @@ Timing: W untimed warm-up steps, then K steps replayed from a CUDA graph of
 back-to-back launches, bracketed by a barrier and synchronisation, timed with
 CUDA events on the launching stream, max over ranks.  The weights rotate over
 enough device copies to exceed 4x the L2 size, so every step streams from HBM.
+``per_launch`` gives the spread: an event after every graph replay yields
+each replay's per-launch time, reported as median, standard deviation,
+minimum and maximum over the replays.
 
 ``e2e``: the same GEMV through ``qmm_gemv_host`` (the call a serving loop
 makes with host buffers): every step brings the token's activations in from
@@ -191,8 +194,10 @@ def graph_of(launch, count: int):
     return g
 
 
-def time_graph(g, reps: int, world: int, sampler=None):
-    """Replay `g` reps times; returns (seconds, clocks dict or None)."""
+def time_graph(g, reps: int, world: int, sampler=None, rep_ms=None):
+    """Replay `g` reps times; returns (seconds, clocks dict or None).  With a
+    list `rep_ms`, an event after every replay also records each replay's
+    milliseconds into it (for the spread of the per-launch time)."""
     import torch
     barrier(world)
     torch.cuda.synchronize()
@@ -200,14 +205,19 @@ def time_graph(g, reps: int, world: int, sampler=None):
         sampler.start()
     st = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    marks = [torch.cuda.Event(enable_timing=True) for _ in range(reps)] if rep_ms is not None else None
     e0.record(st)
-    for _ in range(reps):
+    for i in range(reps):
         g.replay()
+        if marks is not None:
+            marks[i].record(st)
     e1.record(st)
     e1.synchronize()
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
     barrier(world)
+    if marks is not None:
+        rep_ms.extend((e0 if i == 0 else marks[i - 1]).elapsed_time(marks[i]) for i in range(reps))
     return e0.elapsed_time(e1) / 1e3, clocks
 
 
@@ -236,12 +246,17 @@ def gemv_workload(p, x_bits, steps, warmup, world, l2, sampler=None, graph_len=1
     wreps = max(1, math.ceil(warmup / glen))
     time_graph(g, wreps, world)
     reps = max(1, steps // glen)
-    secs, clocks = time_graph(g, reps, world, sampler)
+    rep_ms = []
+    secs, clocks = time_graph(g, reps, world, sampler, rep_ms)
     launches = reps * glen
     assert qmm.qmm_sync_check() == 0
     per = secs / launches
     del g
-    return {"variant": variant, "launches": launches, "seconds": secs, "s_per_launch": per,
+    us = np.asarray(rep_ms, dtype=np.float64) * 1e3 / glen  # per-launch microseconds of each replay
+    stats = {"median_us": round(float(np.median(us)), 4), "sd_us": round(float(np.std(us)), 4),
+             "min_us": round(float(us.min()), 4), "max_us": round(float(us.max()), 4), "replays": reps,
+             "launches_per_replay": glen}
+    return {"variant": variant, "launches": launches, "seconds": secs, "s_per_launch": per, "per_launch": stats,
             "bytes_per_launch": base.nbytes, "gbs": base.nbytes / per / 1e9, "copies": R,
             "rotating_bytes": R * base.nbytes, "clocks": clocks, "m": m, "n": p.n, "k": p.k}
 
@@ -627,6 +642,7 @@ def main():
                          else "fallback 6650 GB/s", "kernel": r["variant"],
                          "algorithmic_bytes_per_launch": r["bytes_per_launch"]},
             "clocks": r["clocks"],
+            "per_launch": r["per_launch"],
             "e2e": {"value": round(e2e["gbs"], 2), "unit": "GB/s", "h2d_bytes_per_step": e2e["h2d"],
                     "d2h_bytes_per_step": e2e["d2h"]},
             "gpu_launches": launches}
