@@ -1,0 +1,66 @@
+"""Host logic of bench.py that needs no GPU: the clock/throttle record taken
+during the timed region, and the number of rotating weight copies."""
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+class _Done:
+    """Stands in for the finished nvidia-smi sampler process."""
+    def terminate(self):
+        pass
+
+    def wait(self, timeout=None):
+        return 0
+
+
+def _stop(tmp_path, monkeypatch, lines):
+    path = tmp_path / "clk.csv"
+    path.write_text("".join(ln + "\n" for ln in lines))
+    s = bench.ClockSampler(0)
+    s.proc, s.path = _Done(), str(path)
+    monkeypatch.setattr(bench.time, "sleep", lambda _s: None)
+    return s.stop()
+
+
+NA, ACT = "Not Active", "Active"
+
+
+def _row(mhz, reasons=(NA, NA, NA, NA), mx=1965):
+    return ", ".join(["0", str(mhz), str(mx), "650.1", "0x0"] + list(reasons))
+
+
+def test_clock_record_takes_the_median_of_the_loaded_samples(tmp_path, monkeypatch):
+    r = _stop(tmp_path, monkeypatch, [_row(345), _row(1965), _row(1950), _row(1965), _row(1900), _row(1965)])
+    assert r["sm_max_mhz"] == 1965 and r["reasons"] == [] and r["samples"] == 6
+    assert r["sm_mhz"] == 1965                     # top half: 1965, 1965, 1965
+
+
+def test_clock_record_names_every_reason_seen(tmp_path, monkeypatch):
+    r = _stop(tmp_path, monkeypatch, [_row(1900, (NA, NA, NA, ACT)), _row(1300, (ACT, NA, NA, ACT)),
+                         _row(1800, (NA, NA, ACT, NA))])
+    assert r["reasons"] == ["hw_slowdown", "sw_power_cap", "sw_thermal_slowdown"]
+
+
+def test_clock_record_skips_unreadable_fields_and_short_lines(tmp_path, monkeypatch):
+    r = _stop(tmp_path, monkeypatch, ["garbage", _row("[N/A]"), _row(1965), "0, 1, 2"])
+    assert r["samples"] == 2 and r["sm_mhz"] == 1965
+    assert _stop(tmp_path, monkeypatch, [])["reasons"] == ["no samples"]
+
+
+def test_rotating_copies_exceed_four_l2_and_respect_the_cap():
+    l2 = 126 << 20
+    for nbytes in (73728, 20971520, 47513600, 655360000):
+        r = bench.rotating_copies(nbytes, l2)
+        assert r * nbytes >= min(4 * l2, (6 << 30) // nbytes * nbytes) and r >= 1
+        assert r * nbytes <= max(6 << 30, nbytes)
+    assert bench.rotating_copies(47513600, l2) == 12     # 570 MB for the in_proj headline
+
+
+def test_replica_throughput_counts_every_rank():
+    assert bench.replica_throughput(1000, 10, 1e-6, 1) == 10.0
+    assert bench.replica_throughput(1000, 10, 1e-6, 4) == 40.0
