@@ -22,8 +22,11 @@ makes with host buffers): every step brings the token's activations in from
 pinned host memory and writes y back to pinned host memory, timed the same
 way.
 
-``--impl reference`` times the CPU oracle (plain C, one host thread) on a
-bounded sample of the same workload instead.
+``cpu_baseline`` is the CPU oracle (plain C, fp64) on one host thread over a
+quarter of the rows; ``cpu_baseline_all_cores`` runs the same oracle on every
+usable host core at once over disjoint row ranges; both name the host CPU.
+``--impl reference`` times the CPU oracle (one host thread) on a bounded
+sample of the same workload instead.
 """
 from __future__ import annotations
 
@@ -310,7 +313,54 @@ def cpu_oracle_gemv(p, x_bits, budget_s=10.0, rows=None):
             break
     dt = time.perf_counter() - t0
     return {"value": sub.nbytes * reps / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": "%d of %d rows x %d reps (%.1f s, one thread)" % (rows, p.n, reps, dt)}
+            "sample": "%d of %d rows x %d reps (%.1f s, one thread)" % (rows, p.n, reps, dt),
+            "cpu": host_cpu()}
+
+
+def host_cpu():
+    """Model name and usable core count of the host the oracle ran on."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"model": model, "nproc": len(os.sched_getaffinity(0))}
+
+
+def cpu_oracle_gemv_all_cores(p, x_bits, budget_s=10.0, threads=None):
+    """The oracle as it stands on every usable host core at once: a row
+    sample cut into one disjoint row range per thread, each thread calling
+    the oracle on its range (the C call releases the interpreter lock), as a
+    parallel loop over output rows would."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    threads = threads or len(os.sched_getaffinity(0))
+    rows = min(p.n, max(16 * threads, p.n // 4))
+    db, sb = oracle.data_bytes(p.fmt, 1, p.k), oracle.scale_bytes(p.fmt, 1, p.k)
+    cuts = [rows * i // threads for i in range(threads + 1)]
+    parts = [type(p)(p.fmt, r1 - r0, p.k, p.data[r0 * db: r1 * db],
+                     None if p.scales is None else p.scales[r0 * sb: r1 * sb], p.global_scale)
+             for r0, r1 in zip(cuts[:-1], cuts[1:]) if r1 > r0]
+
+    def run(q):
+        t0, reps = time.perf_counter(), 0
+        while True:
+            oracle.matmul(q.fmt, q.n, q.k, q.data, q.scales, q.global_scale, x_bits)
+            reps += 1
+            if time.perf_counter() - t0 >= budget_s:
+                return q.nbytes * reps, time.perf_counter() - t0
+
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(max_workers=len(parts)) as ex:
+        done = list(ex.map(run, parts))
+    wall = time.perf_counter() - t0
+    return {"value": sum(b for b, _ in done) / wall / 1e9, "unit": "GB/s", "cores": len(parts), "kind": "oracle",
+            "sample": "%d of %d rows in %d disjoint ranges, one thread each (%.1f s)" % (rows, p.n, len(parts), wall),
+            "cpu": host_cpu()}
 
 
 def timed_launches(launch, count, reps, warm_reps, world):
@@ -650,6 +700,8 @@ def main():
         line["workloads"] = extra_workloads(args, world, l2, peaks)
     if rank == 0:
         line["cpu_baseline"] = cpu_oracle_gemv(p, x, budget_s=args.cpu_budget) if world == 1 else None
+        if world == 1:
+            line["cpu_baseline_all_cores"] = cpu_oracle_gemv_all_cores(p, x, budget_s=args.cpu_budget)
         print(json.dumps(line))
     if world > 1:
         import torch.distributed as dist

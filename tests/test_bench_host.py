@@ -64,3 +64,15 @@ def test_rotating_copies_exceed_four_l2_and_respect_the_cap():
 def test_replica_throughput_counts_every_rank():
     assert bench.replica_throughput(1000, 10, 1e-6, 1) == 10.0
     assert bench.replica_throughput(1000, 10, 1e-6, 4) == 40.0
+
+
+def test_all_core_oracle_baseline_covers_disjoint_row_ranges():
+    import numpy as np
+    from packed_bit_weight_b200 import synth
+    rng = np.random.default_rng(0)
+    p = synth.gen_fp4(rng, 64, 256)
+    x = synth.gen_x(rng, 1, 256)
+    r = bench.cpu_oracle_gemv_all_cores(p, x, budget_s=0.05, threads=3)
+    assert r["cores"] == 3 and r["value"] > 0 and r["kind"] == "oracle" and r["unit"] == "GB/s"
+    assert "48 of 64 rows in 3 disjoint ranges" in r["sample"]
+    assert r["cpu"]["nproc"] >= 1 and r["cpu"]["model"]
