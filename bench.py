@@ -24,7 +24,9 @@ way.
 
 ``cpu_baseline`` is the CPU oracle (plain C, fp64) on one host thread over a
 quarter of the rows; ``cpu_baseline_all_cores`` runs the same oracle on every
-usable host core at once over disjoint row ranges; both name the host CPU.
+usable host core at once over disjoint row ranges; ``cpu_baseline_gemm`` is
+the oracle on a 256-row x 64-token sample of the prefill GEMM, in TFLOP/s;
+all name the host CPU.
 ``--impl reference`` times the CPU oracle (one host thread) on a bounded
 sample of the same workload instead.
 """
@@ -315,6 +317,30 @@ def cpu_oracle_gemv(p, x_bits, budget_s=10.0, rows=None):
     return {"value": sub.nbytes * reps / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
             "sample": "%d of %d rows x %d reps (%.1f s, one thread)" % (rows, p.n, reps, dt),
             "cpu": host_cpu()}
+
+
+def cpu_oracle_gemm(budget_s=10.0, rows=256, tokens=64):
+    """The oracle on a bounded sample of the prefill GEMM (2048 x 18560 x
+    4096, FP4-G16): the first `rows` weight rows against the first `tokens`
+    activation rows, one host thread, repeated for about budget_s."""
+    import oracle
+    from packed_bit_weight_b200 import synth
+    p, x = synth.make_prefill()
+    rows, tokens = min(rows, p.n), min(tokens, x.shape[0])
+    sub = type(p)(p.fmt, rows, p.k, p.data[: oracle.data_bytes(p.fmt, rows, p.k)],
+                  None if p.scales is None else p.scales[: oracle.scale_bytes(p.fmt, rows, p.k)], p.global_scale)
+    xs = np.ascontiguousarray(x[:tokens])
+    t0, reps = time.perf_counter(), 0
+    while True:
+        oracle.matmul(sub.fmt, sub.n, sub.k, sub.data, sub.scales, sub.global_scale, xs)
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    flops = 2.0 * tokens * rows * p.k * reps
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+            "sample": "%d of %d rows x %d of %d tokens, k = %d, x %d reps (%.1f s, one thread)"
+                      % (rows, p.n, tokens, x.shape[0], p.k, reps, dt), "cpu": host_cpu()}
 
 
 def host_cpu():
@@ -702,6 +728,7 @@ def main():
         line["cpu_baseline"] = cpu_oracle_gemv(p, x, budget_s=args.cpu_budget) if world == 1 else None
         if world == 1:
             line["cpu_baseline_all_cores"] = cpu_oracle_gemv_all_cores(p, x, budget_s=args.cpu_budget)
+            line["cpu_baseline_gemm"] = cpu_oracle_gemm(budget_s=args.cpu_budget)
         print(json.dumps(line))
     if world > 1:
         import torch.distributed as dist

@@ -76,3 +76,9 @@ def test_all_core_oracle_baseline_covers_disjoint_row_ranges():
     assert r["cores"] == 3 and r["value"] > 0 and r["kind"] == "oracle" and r["unit"] == "GB/s"
     assert "48 of 64 rows in 3 disjoint ranges" in r["sample"]
     assert r["cpu"]["nproc"] >= 1 and r["cpu"]["model"]
+
+
+def test_gemm_oracle_baseline_reports_tflops_of_its_sample():
+    r = bench.cpu_oracle_gemm(budget_s=0.01, rows=32, tokens=4)
+    assert r["unit"] == "TFLOP/s" and r["value"] > 0 and r["cores"] == 1 and r["kind"] == "oracle"
+    assert r["sample"].startswith("32 of 18560 rows x 4 of 2048 tokens, k = 4096")
