@@ -517,14 +517,18 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
   if constexpr (PF && FMT != 1) {
     // Both ranges start 16 rows past a 16-byte-aligned base (16-byte
     // aligned); their lengths are rounded down to whole 16-byte units, as the
-    // bulk prefetch needs, and stay inside row n-1.
+    // bulk prefetch needs, stay inside row n-1, and go out in pieces of at
+    // most 32 KB.
     const int64_t t2 = (int64_t)blockIdx.x + pf_ahead;
     if (pf_ahead > 0 && threadIdx.x == 0 && t2 * 16 < n) {
       const int64_t rows = min((int64_t)16, (int64_t)n - t2 * 16);
       const int64_t sbr = (FMT == 2) ? 2 * srow : (FMT == 4) ? (srow >> 1) : srow;  // scale bytes per row
-      const uint32_t cbytes = (uint32_t)(rows * crow) & ~15u, sbytes = (uint32_t)(rows * sbr) & ~15u;
-      if (cbytes) prefetch_l2_bulk(codes + t2 * 16 * crow, cbytes);
-      if (sbytes) prefetch_l2_bulk(scales + t2 * 16 * sbr, sbytes);
+      auto prefetch = [](const uint8_t* p, int64_t bytes) {
+        bytes &= ~(int64_t)15;
+        for (int64_t o = 0; o < bytes; o += 32768) prefetch_l2_bulk(p + o, (uint32_t)min((int64_t)32768, bytes - o));
+      };
+      prefetch(codes + t2 * 16 * crow, rows * crow);
+      prefetch(scales + t2 * 16 * sbr, rows * sbr);
     }
   }
   uint4 qa[SPW], qb[SPW];
