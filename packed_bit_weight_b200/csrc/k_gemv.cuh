@@ -490,19 +490,10 @@ __device__ __forceinline__ void ldg_tile_store(float (&red)[WPC][16][16], const 
 // bytes of two segments with one 256-bit load per row, and their scales with
 // one load (8 B fp16, 4 B E4M3, 2 B E8M0), the segment pairing of
 // ldg_tile_mma's WIDE layout.
-//
-// PF (opt-in): the CTAs of the first resident wave also bulk-prefetch into L2
-// the tile of the CTA pf_ahead blocks later (its 16 code rows and 16 scale
-// rows are two contiguous byte ranges), so HBM keeps streaming the later
-// tiles while the first wave multiplies after the dependency wait, and those
-// tiles' register loads then hit L2.  pf_ahead is the number of CTAs resident
-// at once; 0 turns the prefetch off.
-template <int FMT, int NT, int SPW, int WPC = kLdgWarps, int MINB = 2, bool WIDE = false, bool XW = false,
-          bool PF = false>
+template <int FMT, int NT, int SPW, int WPC = kLdgWarps, int MINB = 2, bool WIDE = false, bool XW = false>
 __global__ void __launch_bounds__(WPC * 32, MINB)
     gemv_fp4_ldg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
-                        const uint16_t* __restrict__ x, uint16_t* __restrict__ y, int n, int k, int m, float g,
-                        int pf_ahead) {
+                        const uint16_t* __restrict__ x, uint16_t* __restrict__ y, int n, int k, int m, float g) {
   static_assert(!WIDE || SPW % 2 == 0, "WIDE pairs segments");
   __shared__ float red[WPC][16][16];  // [warp][token][row]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -514,23 +505,6 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
   const int64_t crow = k >> 1, srow = k >> 4;
 
   pdl_launch_dependents();
-  if constexpr (PF && FMT != 1) {
-    // Both ranges start 16 rows past a 16-byte-aligned base (16-byte
-    // aligned); their lengths are rounded down to whole 16-byte units, as the
-    // bulk prefetch needs, stay inside row n-1, and go out in pieces of at
-    // most 32 KB.
-    const int64_t t2 = (int64_t)blockIdx.x + pf_ahead;
-    if (pf_ahead > 0 && threadIdx.x == 0 && t2 * 16 < n) {
-      const int64_t rows = min((int64_t)16, (int64_t)n - t2 * 16);
-      const int64_t sbr = (FMT == 2) ? 2 * srow : (FMT == 4) ? (srow >> 1) : srow;  // scale bytes per row
-      auto prefetch = [](const uint8_t* p, int64_t bytes) {
-        bytes &= ~(int64_t)15;
-        for (int64_t o = 0; o < bytes; o += 32768) prefetch_l2_bulk(p + o, (uint32_t)min((int64_t)32768, bytes - o));
-      };
-      prefetch(codes + t2 * 16 * crow, rows * crow);
-      prefetch(scales + t2 * 16 * sbr, rows * sbr);
-    }
-  }
   uint4 qa[SPW], qb[SPW];
   uint32_t sa[SPW], sb[SPW];
   if (WIDE) {

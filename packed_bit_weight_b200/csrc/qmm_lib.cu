@@ -168,8 +168,7 @@ static qmm_status launch_gemv_tma(const qmm_weights* w, const uint16_t* x, int m
   return launch_status();
 }
 
-template <int FMT, int NT, int SPW, int WPC = kLdgWarps, int MINB = 2, bool WIDE = false, bool XW = false,
-          bool PF = false>
+template <int FMT, int NT, int SPW, int WPC = kLdgWarps, int MINB = 2, bool WIDE = false, bool XW = false>
 static qmm_status launch_gemv_ldg(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st) {
   const int n = (int)w->n, k = (int)w->k;
   const int tiles = (n + 15) / 16;
@@ -179,26 +178,10 @@ static qmm_status launch_gemv_ldg(const qmm_weights* w, const uint16_t* x, int m
   const char* nopdl = getenv("QMM_GEMV_NOPDL");
   const char* pad = getenv("QMM_GEMV_SMEM_PAD");
   const int pad_bytes = pad ? atoi(pad) : 0;
-  auto kern = gemv_fp4_ldg_kernel<FMT, NT, SPW, WPC, MINB, WIDE, XW, PF>;
+  auto kern = gemv_fp4_ldg_kernel<FMT, NT, SPW, WPC, MINB, WIDE, XW>;
   if (pad_bytes > 0 &&
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pad_bytes) != cudaSuccess)
     return QMM_ERR_CUDA;
-  // PF: prefetch distance = CTAs resident at once (QMM_GEMV_L2PF=<n> > 1
-  // sets it directly, for sweeps)
-  int pf_ahead = 0;
-  if constexpr (PF) {
-    const char* e = getenv("QMM_GEMV_L2PF");
-    pf_ahead = e ? atoi(e) : 0;
-    if (pf_ahead <= 1) {
-      int dev = 0, sms = 0, per_sm = 0;
-      if (cudaGetDevice(&dev) != cudaSuccess ||
-          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-          cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, WPC * 32, pad_bytes > 0 ? pad_bytes : 0) !=
-              cudaSuccess)
-        return QMM_ERR_CUDA;
-      pf_ahead = sms * per_sm;
-    }
-  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(tiles);
   cfg.blockDim = dim3(WPC * 32);
@@ -212,14 +195,9 @@ static qmm_status launch_gemv_ldg(const qmm_weights* w, const uint16_t* x, int m
   const uint8_t* codes = static_cast<const uint8_t*>(w->data);
   const uint8_t* scales = static_cast<const uint8_t*>(w->scales);
   const float g = w->global_scale;
-  if (cudaLaunchKernelEx(&cfg, kern, codes, scales, x, y, n, k, m, g, pf_ahead) != cudaSuccess)
-    return QMM_ERR_CUDA;
-  if (PF)
-    set_variant("gemv_fp4_ldg<fmt=%d,nt=%d,spw=%d,wpc=%d,minb=%d,wide=%d,xw=%d,tiles=%d,l2pf=%d>", FMT, NT, SPW, WPC,
-                MINB, WIDE ? 1 : 0, XW ? 1 : 0, tiles, pf_ahead);
-  else
-    set_variant("gemv_fp4_ldg<fmt=%d,nt=%d,spw=%d,wpc=%d,minb=%d,wide=%d,xw=%d,tiles=%d>", FMT, NT, SPW, WPC, MINB,
-                WIDE ? 1 : 0, XW ? 1 : 0, tiles);
+  if (cudaLaunchKernelEx(&cfg, kern, codes, scales, x, y, n, k, m, g) != cudaSuccess) return QMM_ERR_CUDA;
+  set_variant("gemv_fp4_ldg<fmt=%d,nt=%d,spw=%d,wpc=%d,minb=%d,wide=%d,xw=%d,tiles=%d>", FMT, NT, SPW, WPC, MINB,
+              WIDE ? 1 : 0, XW ? 1 : 0, tiles);
   return launch_status();
 }
 
@@ -243,14 +221,6 @@ static qmm_status launch_gemv_ldg_pick(bool wide, const qmm_weights* w, const ui
   // them off: measurement knob)
   const char* xe = getenv("QMM_GEMV_XW");
   const bool xw = (reinterpret_cast<uintptr_t>(x) & 31u) == 0 && !(xe && xe[0] == '0');
-  // QMM_GEMV_L2PF=1 (or a prefetch distance in CTAs): the first wave's L2
-  // prefetch of the later tiles (opt-in; 128-byte-row layout, 256-bit x).
-  // At 4 warps per tile it asks for 5 CTAs per SM, which keeps FP4-G16 at
-  // the default's 96 registers (106 otherwise, and 4 CTAs per SM; MXFP4
-  // would spill at 96 and keeps its own bound).
-  const char* pf = getenv("QMM_GEMV_L2PF");
-  if (pf && pf[0] && pf[0] != '0' && xw && !wide)
-    return launch_gemv_ldg<FMT, NT, SPW, WPC, (WPC == 4 && FMT != 4 ? 5 : MINB), false, true, true>(w, x, m, y, st);
   if constexpr (SPW % 2 == 0) {
     if (wide && xw) return launch_gemv_ldg<FMT, NT, SPW, WPC, MINB, true, true>(w, x, m, y, st);
     if (wide) return launch_gemv_ldg<FMT, NT, SPW, WPC, MINB, true>(w, x, m, y, st);
