@@ -69,3 +69,5 @@ def test_reference_arm_rank0_prints_one_line():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+    assert d["steps"] == 5 and d["warmup"] == 3 and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["sample"].startswith("5 timed + 3 untimed steps")
