@@ -1,7 +1,12 @@
-"""Host-side argument checks of qmm_gemv_host, run without a GPU: every case
-here returns before the library touches CUDA (descriptor, batch size, null
-and alignment checks come first), with fake device addresses that are never
-dereferenced."""
+"""Host-side argument checks, run without a GPU.
+
+The C entry points (qmm_gemv_host, qmm_gemm, qmm_grouped_gemv, qmm_route,
+qmm_moe_routed, qmm_router_topk, qmm_quantize, qmm_workspace_bytes) check
+descriptors, sizes, null pointers and alignment before they touch CUDA; the
+cases here all return there, with fake device addresses that are never
+dereferenced.  The Python binding's own checks (host vs device tensors,
+contiguity, and that every tensor holds the bytes its call touches) run on
+CPU tensors, which reach them before the device check."""
 import ctypes
 
 import numpy as np
