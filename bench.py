@@ -747,7 +747,7 @@ def main():
     e2e = gemv_e2e(p, x, max(200, min(5000, args.steps // 4)), world)
     line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": launches,
             "warmup": args.warmup, "ms_per_step": per_launch * 1e3, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "fp16-in/fp32-acc (4-bit packed weights)", "data": "synthetic",
+            "vs_baseline": None, "dtype": "f16", "acc_dtype": "f32", "data": "synthetic",
             "config": dict(config, l2="rotating %d weight copies = %.0f MB > 4x L2 (%d MB)" %
                            (r["copies"], r["rotating_bytes"] / 1e6, l2 >> 20),
                            timing="CUDA graph of 100 back-to-back launches, replayed"),
