@@ -2,31 +2,32 @@
 """Throughput of the packed 4-bit weight path on B200.
 
 Headline workload: the FP4-G16 (fp16 group scale) GEMV at the Mamba-2 8B
-in_proj shape, n = 18560, k = 4096, one decode token (m = 1).  A step is one
-call of the fused dequantise-and-multiply (stream packed blocks, decode,
-multiply-accumulate, reduce, store y) for one token.  ``value`` is packed
-weight bytes per second over all ranks.  The other workloads of the path
-(m = 4/16 sweeps, IQ4_NL, dequantisation, prefill GEMM, routed experts) are
-measured the same way and reported under ``workloads``.
+in_proj shape, n = 18560, k = 4096, one decode token (m = 1).  A step is
+what one decode token costs in this projection: the fused
+dequantise-and-multiply (stream packed blocks, decode, multiply-accumulate,
+reduce, store y) of each of the model's 56 layers, every layer on its own
+copy of the weights (2.66 GB resident, so every launch streams from HBM).
+``value`` is packed weight bytes per second over all ranks.  The other
+workloads of the path (m = 4/16 sweeps, IQ4_NL, dequantisation, prefill
+GEMM, routed experts) are measured per launch and reported under
+``workloads``.
 
-Timing: W untimed warm-up steps, then K steps replayed from a CUDA graph of
-back-to-back launches, bracketed by a barrier and synchronisation, timed with
-CUDA events on the launching stream, max over ranks.  The weights rotate over
-enough device copies to exceed 4x the L2 size, so every step streams from HBM.
-``per_launch`` gives the spread: an event after every graph replay yields
-each replay's per-launch time, reported as median, standard deviation,
-minimum and maximum over the replays.
+Timing: the 56 launches of a step are captured back to back in one CUDA
+graph (programmatic dependent launch between them); W untimed replays, then
+K timed replays bracketed by a barrier and synchronisation, timed with CUDA
+events on the launching stream, max over ranks.  ``per_launch`` gives the
+spread: an event after every replay yields each step's per-launch time,
+reported as median, standard deviation, minimum and maximum over the steps.
 
-``e2e``: the same GEMV through ``qmm_gemv_host`` (the call a serving loop
-makes with host buffers): every step brings the token's activations in from
-pinned host memory and writes y back to pinned host memory, timed the same
-way.
+``e2e``: the same step through ``qmm_gemv_host`` (the call a serving loop
+makes with host buffers): each of the 56 calls brings its activations in
+from pinned host memory and writes y back to pinned host memory.
 
 ``cpu_baseline`` is the CPU oracle (plain C, fp64) on one host thread over a
-quarter of the rows; ``cpu_baseline_all_cores`` runs the same oracle on every
-usable host core at once over disjoint row ranges; ``cpu_baseline_gemm`` is
-the oracle on a 256-row x 64-token sample of the prefill GEMM, in TFLOP/s;
-all name the host CPU.
+quarter of the in_proj rows; ``cpu_baseline_all_cores`` runs the same oracle
+on every usable host core at once over disjoint row ranges;
+``cpu_baselines`` times the oracle on every other workload (a bounded
+sample of each, stated); all name the host CPU.
 ``--impl reference`` times the CPU oracle instead (one host thread): W
 untimed and K timed steps, each step a block of consecutive weight rows of
 the same matrix, the block sized so the whole run takes about six times
@@ -51,6 +52,7 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 
 METRIC = "packed 4-bit GEMV weight GB/s vs HBM peak (M=1); prefill GEMM TFLOP/s (M=2048)"
+LAYERS = 56  # Mamba-2 8B layers: one in_proj GEMV each per decode token
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # ncu DRAM traffic per launch (read + write bytes) of the dominant kernel, by
@@ -231,15 +233,59 @@ def time_graph(g, reps: int, world: int, sampler=None, rep_ms=None):
 # ---------------------------------------------------------------------------
 # workloads
 # ---------------------------------------------------------------------------
-def gemv_workload(p, x_bits, steps, warmup, world, l2, sampler=None, graph_len=100):
-    """Device-resident GEMV throughput; returns dict."""
-    import torch
+def weight_copies(p, count):
+    """`count` distinct device copies of one packed matrix (the seeded host
+    matrix uploaded once, the rest device-side clones: the bytes every launch
+    streams are the same, at different addresses)."""
     from packed_bit_weight_b200 import qmm
     base = qmm.PackedWeights.from_host(p)
-    R = rotating_copies(base.nbytes, l2)
-    ws = [base] + [qmm.PackedWeights(base.fmt, base.n, base.k, base.data.clone(),
-                                     None if base.scales is None else base.scales.clone(), base.global_scale)
-                   for _ in range(R - 1)]
+    return [base] + [qmm.PackedWeights(base.fmt, base.n, base.k, base.data.clone(),
+                                       None if base.scales is None else base.scales.clone(), base.global_scale)
+                     for _ in range(count - 1)]
+
+
+def gemv_step_workload(p, x_bits, steps, warmup, world, layers, sampler=None):
+    """Device-resident decode step: one launch per layer, each on its own
+    weight copy, back to back in one CUDA graph (programmatic dependent
+    launch between them); the graph is replayed once per step.  Returns
+    dict with per-step and per-launch times."""
+    import torch
+    from packed_bit_weight_b200 import qmm
+    ws = weight_copies(p, layers)
+    m = x_bits.shape[0]
+    x = torch.from_numpy(x_bits.view(np.int16)).cuda()
+    y = torch.empty((m, p.n), dtype=torch.int16, device="cuda")
+
+    def launch(i):
+        qmm.qmm_gemv(ws[i], x, y)
+
+    g = graph_of(launch, layers)
+    variant = qmm.qmm_last_variant()
+    time_graph(g, warmup, world)
+    rep_ms = []
+    secs, clocks = time_graph(g, steps, world, sampler, rep_ms)
+    assert qmm.qmm_sync_check() == 0
+    del g
+    us = np.asarray(rep_ms, dtype=np.float64) * 1e3 / layers  # per-launch microseconds of each step
+    stats = {"median_us": round(float(np.median(us)), 4), "sd_us": round(float(np.std(us)), 4),
+             "min_us": round(float(us.min()), 4), "max_us": round(float(us.max()), 4), "steps": steps,
+             "launches_per_step": layers}
+    nbytes = ws[0].nbytes
+    return {"variant": variant, "launches": steps * layers, "seconds": secs, "s_per_launch": secs / (steps * layers),
+            "per_launch": stats, "bytes_per_launch": nbytes, "bytes_per_step": nbytes * layers,
+            "gbs": nbytes * layers * steps / secs / 1e9, "copies": layers, "resident_bytes": layers * nbytes,
+            "clocks": clocks, "m": m, "n": p.n, "k": p.k}
+
+
+def gemv_workload(p, x_bits, steps, warmup, world, l2, sampler=None, graph_len=100):
+    """Device-resident GEMV throughput of one matrix shape: rotating weight
+    copies (> 4x L2), a graph of up to graph_len back-to-back launches,
+    replayed; returns dict."""
+    import torch
+    from packed_bit_weight_b200 import qmm
+    R = rotating_copies(qmm.qmm_packed_bytes(p.fmt, p.n, p.k), l2)
+    ws = weight_copies(p, R)
+    base = ws[0]
     m = x_bits.shape[0]
     x = torch.from_numpy(x_bits.view(np.int16)).cuda()
     y = torch.empty((m, p.n), dtype=torch.int16, device="cuda")
@@ -268,13 +314,14 @@ def gemv_workload(p, x_bits, steps, warmup, world, l2, sampler=None, graph_len=1
             "rotating_bytes": R * base.nbytes, "clocks": clocks, "m": m, "n": p.n, "k": p.k}
 
 
-def gemv_e2e(p, x_bits, steps, world):
-    """Same GEMV through the public API with host buffers (qmm_gemv_host):
-    pinned x host->device, the product, y device->host, every step, in one
-    library call per step."""
+def gemv_e2e(p, x_bits, steps, world, layers):
+    """The decode step through the public API with host buffers
+    (qmm_gemv_host), one call per layer on its own weight copy: every call
+    brings that layer's activations in from pinned host memory and writes
+    its y back to pinned host memory."""
     import torch
     from packed_bit_weight_b200 import qmm
-    w = qmm.PackedWeights.from_host(p)
+    ws = weight_copies(p, layers)
     m = x_bits.shape[0]
     xh = torch.from_numpy(x_bits.view(np.int16).copy()).pin_memory()
     yh = torch.empty((m, p.n), dtype=torch.int16).pin_memory()
@@ -284,9 +331,10 @@ def gemv_e2e(p, x_bits, steps, world):
     st = torch.cuda.current_stream()
 
     def step():
-        qmm.qmm_gemv_host(w, xh, yh, xd, yd, stream=st)
+        for w in ws:
+            qmm.qmm_gemv_host(w, xh, yh, xd, yd, stream=st)
 
-    for _ in range(20):
+    for _ in range(3):
         step()
     torch.cuda.synchronize()
     barrier(world)
@@ -296,9 +344,10 @@ def gemv_e2e(p, x_bits, steps, world):
         step()
     e1.record(st)
     e1.synchronize()
+    assert qmm.qmm_sync_check() == 0
     secs = max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
-    return {"seconds": secs, "steps": steps, "h2d": xh.numel() * 2, "d2h": yh.numel() * 2,
-            "gbs": world * w.nbytes * steps / secs / 1e9}
+    return {"seconds": secs, "steps": steps, "h2d": layers * xh.numel() * 2, "d2h": layers * yh.numel() * 2,
+            "gbs": world * ws[0].nbytes * layers * steps / secs / 1e9}
 
 
 def cpu_oracle_gemv(p, x_bits, budget_s=10.0, rows=None):
@@ -694,8 +743,8 @@ def profile_case(name: str) -> int:
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
-    ap.add_argument("--warmup", type=int, default=500)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extra", action="store_true", help="headline workload only")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
@@ -710,7 +759,7 @@ def main():
     from packed_bit_weight_b200 import synth
     wl = synth.FP4_IN_PROJ
     config = {"workload": wl.name, "format": "FP4-G16 (E2M1 codes, fp16 scale per 16 k)", "n": 18560, "k": 4096,
-              "m": 1, "seed": wl.seed, "parallelism": "replicas"}
+              "m": 1, "seed": wl.seed, "layers_per_step": LAYERS, "parallelism": "replicas"}
 
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -738,28 +787,32 @@ def main():
     p, x = synth.make_gemv(wl)
     sampler = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[0])
                            if "CUDA_VISIBLE_DEVICES" in os.environ else local)
-    r = gemv_workload(p, x, args.steps, args.warmup, world, l2, sampler)
+    r = gemv_step_workload(p, x, args.steps, args.warmup, world, LAYERS, sampler)
     secs = max_over_ranks(r["seconds"], world)
     launches = r["launches"]
-    value = replica_throughput(r["bytes_per_launch"], launches, secs, world)
+    value = replica_throughput(r["bytes_per_step"], args.steps, secs, world)
     per_launch = secs / launches
     achieved = r["bytes_per_launch"] / per_launch / 1e9
-    e2e = gemv_e2e(p, x, max(200, min(5000, args.steps // 4)), world)
-    line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": launches,
-            "warmup": args.warmup, "ms_per_step": per_launch * 1e3, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f16", "acc_dtype": "f32", "data": "synthetic",
-            "config": dict(config, l2="rotating %d weight copies = %.0f MB > 4x L2 (%d MB)" %
-                           (r["copies"], r["rotating_bytes"] / 1e6, l2 >> 20),
-                           timing="CUDA graph of 100 back-to-back launches, replayed"),
+    e2e = gemv_e2e(p, x, max(20, min(500, args.steps)), world, LAYERS)
+    line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16", "acc_dtype": "f32", "data": "synthetic",
+            "config": config,
+            "step": "one decode token through the in_proj GEMV of all %d layers: %d launches back to back in one "
+                    "CUDA graph, each on its own copy of the weights (%.2f GB resident, > 4x L2 of %d MB, so every "
+                    "launch streams from HBM); the graph is replayed once per step" %
+                    (LAYERS, LAYERS, r["resident_bytes"] / 1e9, l2 >> 20),
+            "bytes_per_step": r["bytes_per_step"],
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": TRAFFIC.get(r["variant"]),
                          "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_src if peak_src == "measured"
                          else "fallback 6650 GB/s", "kernel": r["variant"],
-                         "algorithmic_bytes_per_launch": r["bytes_per_launch"]},
+                         "algorithmic_bytes_per_launch": r["bytes_per_launch"],
+                         "launch_us": round(per_launch * 1e6, 4)},
             "clocks": r["clocks"],
             "per_launch": r["per_launch"],
             "e2e": {"value": round(e2e["gbs"], 2), "unit": "GB/s", "h2d_bytes_per_step": e2e["h2d"],
-                    "d2h_bytes_per_step": e2e["d2h"]},
+                    "d2h_bytes_per_step": e2e["d2h"], "steps": e2e["steps"]},
             "gpu_launches": launches}
     if not args.no_extra:
         line["workloads"] = extra_workloads(args, world, l2, peaks)

@@ -286,7 +286,7 @@ __global__ void __launch_bounds__(kIqWarps * 32, 4)
     grouped_iq4_kernel(const uint8_t* __restrict__ data, int64_t dstride, const uint8_t* __restrict__ data2,
                        int64_t dstride2, const uint16_t* __restrict__ x, int x_per_pair, int topk,
                        const int32_t* __restrict__ offsets, const int32_t* __restrict__ perm, int m_plain,
-                       void* __restrict__ yout, const float* __restrict__ gw, int n, int k, int E, int pf_items) {
+                       void* __restrict__ yout, const float* __restrict__ gw, int n, int k, int E) {
   extern __shared__ __align__(16) uint8_t smem_iq[];
   const uint32_t lut = smem_addr(smem_iq);
   float* red = reinterpret_cast<float*>(smem_iq + kIqLutBytes);  // [warp][32 token slots][16 rows]
@@ -306,23 +306,7 @@ __global__ void __launch_bounds__(kIqWarps * 32, 4)
   const int64_t rowb = (int64_t)(k >> 5) * 18;  // bytes per row
   const int items = tiles * E;
   constexpr int kHalves = (MODE == IQ_SWIGLU) ? 2 : 1;
-  // L2 prefetch of the weight tile(s) of the item this CTA takes pf_items
-  // items later: the warps hold only one pass of loads in registers, so the
-  // bulk prefetch keeps HBM busy while they decode.  16 rows of one expert are
-  // one contiguous byte range.
-  auto prefetch_item = [&](int it) {
-    if (it >= items) return;
-    const int e2 = it / tiles, t2 = it % tiles;
-    if (offsets && offsets[e2 + 1] <= offsets[e2]) return;  // expert without tokens
-    const uint32_t bytes = (uint32_t)((int64_t)min(16, n - t2 * 16) * rowb) & ~15u;
-    if (!bytes) return;
-    prefetch_l2_bulk(data + (int64_t)e2 * dstride + (int64_t)t2 * 16 * rowb, bytes);
-    if (kHalves == 2) prefetch_l2_bulk(data2 + (int64_t)e2 * dstride2 + (int64_t)t2 * 16 * rowb, bytes);
-  };
-  if (pf_items > 0 && threadIdx.x == 0)
-    for (int a = 0; a < pf_items; a++) prefetch_item(blockIdx.x + a * gridDim.x);
   for (int item = blockIdx.x; item < items; item += gridDim.x) {
-    if (pf_items > 0 && threadIdx.x == 0) prefetch_item(item + pf_items * gridDim.x);
     const int e = item / tiles, tile = item % tiles;
     int start = 0, cnt = m_plain;
     if (offsets) {

@@ -264,8 +264,16 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
 // Bulk prefetch of a global byte range into L2 (no shared memory, no
 // completion; a hint): address 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
-               : "memory");
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes));
+}
+
+// The same prefetch, issued only when `on` is nonzero (a predicated
+// instruction, no branch).
+__device__ __forceinline__ void prefetch_l2_bulk_if(const void* p, uint32_t bytes, uint32_t on) {
+  asm volatile(
+      "{\n .reg .pred q;\n setp.ne.u32 q, %2, 0;\n @q cp.async.bulk.prefetch.L2.global [%0], %1;\n}" ::"l"(
+          reinterpret_cast<uint64_t>(p)),
+      "r"(bytes), "r"(on));
 }
 
 // bar.sync on a named barrier that also returns the OR of every thread's flag.

@@ -19,9 +19,6 @@
 #include "k_gemv.cuh"
 #include "k_gemm.cuh"
 #include "k_grouped.cuh"
-#include "k_gemv_ring.cuh"
-#include "k_iq4p.cuh"
-#include "k_iq4w.cuh"
 #include "k_iq4t.cuh"
 #include "k_quant.cuh"
 #include "k_moe.cuh"
@@ -136,68 +133,40 @@ static int grid_for(int64_t items, int per_block, int sms, int waves = 8) {
 // ---------------------------------------------------------------------------
 // GEMV dispatch
 // ---------------------------------------------------------------------------
-template <int FMT, int MT, int NT>
-static qmm_status launch_gemv_tma(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st,
-                                  const DevInfo* di) {
-  using C = GemvTmaCfg<FMT, MT>;
-  const int n = (int)w->n, k = (int)w->k;
-  CUtensorMap tc, ts;
-  if (!make_map_2d(&tc, w->data, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)k / 2, (uint64_t)n, 128, C::RT,
-                   CU_TENSOR_MAP_SWIZZLE_128B))
-    return QMM_ERR_CUDA;
-  if (FMT == 2) {
-    if (!make_map_2d(&ts, w->scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)k / 16, (uint64_t)n, 16, C::RT,
-                     CU_TENSOR_MAP_SWIZZLE_NONE))
-      return QMM_ERR_CUDA;
-  } else {
-    if (!make_map_2d(&ts, w->scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)k / 16, (uint64_t)n, 16, C::RT,
-                     CU_TENSOR_MAP_SWIZZLE_NONE))
-      return QMM_ERR_CUDA;
-  }
-  const size_t budget = di->smem_optin - 1024;  // room for the static shared words
-  int depth = 16;
-  while (depth > 2 && C::smem_bytes(depth) > budget) depth--;
-  const size_t smem = C::smem_bytes(depth);
-  auto kern = gemv_fp4_tma_kernel<FMT, MT, NT>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return QMM_ERR_CUDA;
-  const int tiles = (n + C::RT - 1) / C::RT;
-  const int grid = tiles < di->sms ? tiles : di->sms;
-  kern<<<grid, kGemvThreads, smem, st>>>(tc, ts, x, y, n, k, m, w->global_scale, tiles, depth);
-  set_variant("gemv_fp4_tma<fmt=%d,rt=%d,nt=%d,depth=%d,grid=%d>", FMT, C::RT, NT, depth, grid);
-  return launch_status();
-}
-
 template <int FMT, int NT, int SPW, int WPC = kLdgWarps, int MINB = 2, bool WIDE = false, bool XW = false>
-static qmm_status launch_gemv_ldg(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st) {
+static qmm_status launch_gemv_ldg(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st,
+                                  const DevInfo* di) {
   const int n = (int)w->n, k = (int)w->k;
   const int tiles = (n + 15) / 16;
-  // Measurement knobs: QMM_GEMV_NOPDL=1 drops programmatic dependent launch,
-  // QMM_GEMV_SMEM_PAD=<bytes> reserves unused shared memory per CTA (caps
-  // the CTAs per SM).
-  const char* nopdl = getenv("QMM_GEMV_NOPDL");
-  const char* pad = getenv("QMM_GEMV_SMEM_PAD");
-  const int pad_bytes = pad ? atoi(pad) : 0;
   auto kern = gemv_fp4_ldg_kernel<FMT, NT, SPW, WPC, MINB, WIDE, XW>;
-  if (pad_bytes > 0 &&
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pad_bytes) != cudaSuccess)
+  // CTAs resident at once (one wave): the first wave prefetches the second
+  // into L2 after its dependency wait.  QMM_GEMV_L2PF=0 turns it off (A/B).
+  static int per_sm = -1;
+  if (per_sm < 0 && cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, WPC * 32, 0) != cudaSuccess)
     return QMM_ERR_CUDA;
+  const char* pfe = getenv("QMM_GEMV_L2PF");
+  const int wave = per_sm * di->sms;
+  // first-wave CTAs whose tile one wave later is whole (16 rows); codes of a
+  // tile in at most two 32 KB pieces (k <= 8192), offsets within 32 bits
+  int pf_ctas = std::max(0, std::min(wave, n / 16 - wave));
+  if ((pfe && pfe[0] == '0') || k > 8192 || (int64_t)2 * wave * 8 * k >= ((int64_t)1 << 32)) pf_ctas = 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(tiles);
   cfg.blockDim = dim3(WPC * 32);
-  cfg.dynamicSmemBytes = pad_bytes > 0 ? pad_bytes : 0;
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = (nopdl && nopdl[0] == '1') ? 0 : 1;
+  cfg.numAttrs = 1;
   const uint8_t* codes = static_cast<const uint8_t*>(w->data);
   const uint8_t* scales = static_cast<const uint8_t*>(w->scales);
   const float g = w->global_scale;
-  if (cudaLaunchKernelEx(&cfg, kern, codes, scales, x, y, n, k, m, g) != cudaSuccess) return QMM_ERR_CUDA;
-  set_variant("gemv_fp4_ldg<fmt=%d,nt=%d,spw=%d,wpc=%d,minb=%d,wide=%d,xw=%d,tiles=%d>", FMT, NT, SPW, WPC, MINB,
-              WIDE ? 1 : 0, XW ? 1 : 0, tiles);
+  if (cudaLaunchKernelEx(&cfg, kern, codes, scales, x, y, n, k, m, g, wave, pf_ctas) != cudaSuccess)
+    return QMM_ERR_CUDA;
+  set_variant("gemv_fp4_ldg<fmt=%d,nt=%d,spw=%d,wpc=%d,minb=%d,wide=%d,xw=%d,tiles=%d,l2pf=%d>", FMT, NT, SPW, WPC,
+              MINB, WIDE ? 1 : 0, XW ? 1 : 0, tiles, pf_ctas > 0 ? 1 : 0);
   return launch_status();
 }
 
@@ -216,157 +185,72 @@ static bool ldg_wide_ok(const qmm_weights* w) {
 
 template <int FMT, int NT, int SPW, int WPC, int MINB>
 static qmm_status launch_gemv_ldg_pick(bool wide, const qmm_weights* w, const uint16_t* x, int m, uint16_t* y,
-                                       cudaStream_t st) {
+                                       cudaStream_t st, const DevInfo* di) {
   // 256-bit activation loads when x is 32-byte aligned (QMM_GEMV_XW=0 turns
   // them off: measurement knob)
   const char* xe = getenv("QMM_GEMV_XW");
   const bool xw = (reinterpret_cast<uintptr_t>(x) & 31u) == 0 && !(xe && xe[0] == '0');
   if constexpr (SPW % 2 == 0) {
-    if (wide && xw) return launch_gemv_ldg<FMT, NT, SPW, WPC, MINB, true, true>(w, x, m, y, st);
-    if (wide) return launch_gemv_ldg<FMT, NT, SPW, WPC, MINB, true>(w, x, m, y, st);
+    if (wide && xw) return launch_gemv_ldg<FMT, NT, SPW, WPC, MINB, true, true>(w, x, m, y, st, di);
+    if (wide) return launch_gemv_ldg<FMT, NT, SPW, WPC, MINB, true>(w, x, m, y, st, di);
   }
-  if (xw) return launch_gemv_ldg<FMT, NT, SPW, WPC, MINB, false, true>(w, x, m, y, st);
-  return launch_gemv_ldg<FMT, NT, SPW, WPC, MINB, false>(w, x, m, y, st);
-}
-
-// Persistent ring GEMV (k_gemv_ring.cuh): one CTA per SM, whole 16-row tiles
-// in a ring of 2..4 stages (at most 96 KB, so the next launch's CTA fits
-// beside it), programmatic dependent launch.  Needs k % 256 == 0 and a tile of
-// at most 48 KB (k <= 4096 with fp16 scales).  Measurement knobs:
-// QMM_RING_STAGES=<2..4>, QMM_GEMV_NOPDL=1.
-template <int FMT, int NT, int CW, int SPW, bool XSM>
-static qmm_status launch_gemv_ring(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st,
-                                   const DevInfo* di) {
-  const int64_t n = w->n, k = w->k;
-  if (k % 256 || k < 256 || k > 128 * CW * SPW || n < 1 || n > INT32_MAX - 16) return QMM_ERR_UNSUPPORTED_SHAPE;
-  const uint32_t stage = ring_stage_bytes(FMT, (int)k);
-  int stages = (int)std::min<uint32_t>(kRingMaxStages, kRingStageBudget / stage);
-  if (const char* e = getenv("QMM_RING_STAGES")) stages = atoi(e);
-  if (stages < 2 || stages > kRingMaxStages) return QMM_ERR_UNSUPPORTED_SHAPE;
-  const uint32_t xs_bytes = XSM ? 2u * (uint32_t)m * (uint32_t)k : 0u;
-  if (xs_bytes > kRingXsMax) return QMM_ERR_UNSUPPORTED_SHAPE;
-  const uint32_t smem = ring_smem_bytes<CW, NT>(FMT, (int)k, stages, xs_bytes);
-  if (smem > di->smem_optin) return QMM_ERR_UNSUPPORTED_SHAPE;
-  auto kern = gemv_fp4_ring_kernel<FMT, NT, CW, SPW, XSM>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return QMM_ERR_CUDA;
-  const int64_t tiles = (n + 15) / 16;
-  const int64_t grid = std::min<int64_t>(tiles, (int64_t)di->sms);
-  const char* nopdl = getenv("QMM_GEMV_NOPDL");
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(32 * (CW + 1));
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = (nopdl && nopdl[0] == '1') ? 0 : 1;
-  if (cudaLaunchKernelEx(&cfg, kern, static_cast<const uint8_t*>(w->data), static_cast<const uint8_t*>(w->scales), x,
-                         y, (int)n, (int)k, m, w->global_scale, stages) != cudaSuccess)
-    return QMM_ERR_CUDA;
-  set_variant("gemv_fp4_ring<fmt=%d,nt=%d,cw=%d,xsm=%d,stages=%d,grid=%d,smem=%u>", FMT, NT, CW, (int)XSM, stages,
-              (int)grid, smem);
-  return launch_status();
-}
-
-// Two tiles per CTA (k_gemv.cuh, gemv_fp4_dual_kernel): one in registers, one
-// bulk-copied into shared memory, so the whole matrix is in flight in one wave.
-template <int FMT, int NT, int SPW, int WPC, int MINB>
-static qmm_status launch_gemv_dual(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st,
-                                   const DevInfo* di) {
-  const int64_t n = w->n, k = w->k;
-  if (k != 128 * WPC * SPW || n < 1 || n > INT32_MAX - 32) return QMM_ERR_UNSUPPORTED_SHAPE;
-  const uint32_t smem = dual_smem_bytes<FMT>((int)k);
-  if (smem > di->smem_optin) return QMM_ERR_UNSUPPORTED_SHAPE;
-  auto kern = gemv_fp4_dual_kernel<FMT, NT, SPW, WPC, MINB>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return QMM_ERR_CUDA;
-  const int64_t blocks = (n + 31) / 32;
-  const char* nopdl = getenv("QMM_GEMV_NOPDL");
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)blocks);
-  cfg.blockDim = dim3(WPC * 32);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = (nopdl && nopdl[0] == '1') ? 0 : 1;
-  if (cudaLaunchKernelEx(&cfg, kern, static_cast<const uint8_t*>(w->data), static_cast<const uint8_t*>(w->scales), x,
-                         y, (int)n, (int)k, m, w->global_scale) != cudaSuccess)
-    return QMM_ERR_CUDA;
-  set_variant("gemv_fp4_dual<fmt=%d,nt=%d,spw=%d,wpc=%d,minb=%d,blocks=%d,smem=%u>", FMT, NT, SPW, WPC, MINB,
-              (int)blocks, smem);
-  return launch_status();
-}
-
-template <int FMT>
-static qmm_status gemv_dual_auto(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st,
-                                 const DevInfo* di) {
-  if (m > 8 || w->k % 512) return QMM_ERR_UNSUPPORTED_SHAPE;
-  switch (w->k / 512) {
-    case 4: return launch_gemv_dual<FMT, 1, 4, 4, 4>(w, x, m, y, st, di);
-    case 6: return launch_gemv_dual<FMT, 1, 6, 4, 4>(w, x, m, y, st, di);
-    case 8: return launch_gemv_dual<FMT, 1, 8, 4, 4>(w, x, m, y, st, di);
-    default: return QMM_ERR_UNSUPPORTED_SHAPE;
-  }
+  if (xw) return launch_gemv_ldg<FMT, NT, SPW, WPC, MINB, false, true>(w, x, m, y, st, di);
+  return launch_gemv_ldg<FMT, NT, SPW, WPC, MINB, false>(w, x, m, y, st, di);
 }
 
 // Pick the warps per tile (WPC) and segments per warp (SPW, <= 8 at m <= 8,
 // <= 4 at m <= 16) for k = 128 * WPC * SPW; fewer, fuller warps keep more
 // bytes in flight per register.  Returns UNSUPPORTED_SHAPE for other k.
 template <int FMT, int NT>
-static qmm_status gemv_ldg_auto(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st) {
+static qmm_status gemv_ldg_auto(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st,
+                                const DevInfo* di) {
   const int segs = (int)(w->k / 128);
   if (w->k % 128) return QMM_ERR_UNSUPPORTED_SHAPE;
   const bool wide = ldg_wide_ok(w);
   if (NT == 1) {
     if (segs % 4 == 0 && segs / 4 <= 8) {
       switch (segs / 4) {
-        case 1: return launch_gemv_ldg_pick<FMT, 1, 1, 4, 4>(wide, w, x, m, y, st);
-        case 2: return launch_gemv_ldg_pick<FMT, 1, 2, 4, 4>(wide, w, x, m, y, st);
-        case 3: return launch_gemv_ldg_pick<FMT, 1, 3, 4, 4>(wide, w, x, m, y, st);
-        case 4: return launch_gemv_ldg_pick<FMT, 1, 4, 4, 4>(wide, w, x, m, y, st);
-        case 5: return launch_gemv_ldg_pick<FMT, 1, 5, 4, 4>(wide, w, x, m, y, st);
-        case 6: return launch_gemv_ldg_pick<FMT, 1, 6, 4, 4>(wide, w, x, m, y, st);
-        case 7: return launch_gemv_ldg_pick<FMT, 1, 7, 4, 4>(wide, w, x, m, y, st);
-        default: return launch_gemv_ldg_pick<FMT, 1, 8, 4, 4>(wide, w, x, m, y, st);
+        case 1: return launch_gemv_ldg_pick<FMT, 1, 1, 4, 4>(wide, w, x, m, y, st, di);
+        case 2: return launch_gemv_ldg_pick<FMT, 1, 2, 4, 4>(wide, w, x, m, y, st, di);
+        case 3: return launch_gemv_ldg_pick<FMT, 1, 3, 4, 4>(wide, w, x, m, y, st, di);
+        case 4: return launch_gemv_ldg_pick<FMT, 1, 4, 4, 4>(wide, w, x, m, y, st, di);
+        case 5: return launch_gemv_ldg_pick<FMT, 1, 5, 4, 4>(wide, w, x, m, y, st, di);
+        case 6: return launch_gemv_ldg_pick<FMT, 1, 6, 4, 4>(wide, w, x, m, y, st, di);
+        case 7: return launch_gemv_ldg_pick<FMT, 1, 7, 4, 4>(wide, w, x, m, y, st, di);
+        default: return launch_gemv_ldg_pick<FMT, 1, 8, 4, 4>(wide, w, x, m, y, st, di);
       }
     }
     if (segs % 8 == 0 && segs / 8 <= 8) {
       switch (segs / 8) {
-        case 5: return launch_gemv_ldg_pick<FMT, 1, 5, 8, 2>(wide, w, x, m, y, st);
-        case 6: return launch_gemv_ldg_pick<FMT, 1, 6, 8, 2>(wide, w, x, m, y, st);
-        case 7: return launch_gemv_ldg_pick<FMT, 1, 7, 8, 2>(wide, w, x, m, y, st);
-        case 8: return launch_gemv_ldg_pick<FMT, 1, 8, 8, 2>(wide, w, x, m, y, st);
+        case 5: return launch_gemv_ldg_pick<FMT, 1, 5, 8, 2>(wide, w, x, m, y, st, di);
+        case 6: return launch_gemv_ldg_pick<FMT, 1, 6, 8, 2>(wide, w, x, m, y, st, di);
+        case 7: return launch_gemv_ldg_pick<FMT, 1, 7, 8, 2>(wide, w, x, m, y, st, di);
+        case 8: return launch_gemv_ldg_pick<FMT, 1, 8, 8, 2>(wide, w, x, m, y, st, di);
         default: break;  // smaller counts took the 4-warp path
       }
     }
     if (segs % 16 == 0 && segs / 16 <= 8) {
       switch (segs / 16) {
-        case 5: return launch_gemv_ldg_pick<FMT, 1, 5, 16, 1>(wide, w, x, m, y, st);
-        case 6: return launch_gemv_ldg_pick<FMT, 1, 6, 16, 1>(wide, w, x, m, y, st);
-        case 7: return launch_gemv_ldg_pick<FMT, 1, 7, 16, 1>(wide, w, x, m, y, st);
-        case 8: return launch_gemv_ldg_pick<FMT, 1, 8, 16, 1>(wide, w, x, m, y, st);
+        case 5: return launch_gemv_ldg_pick<FMT, 1, 5, 16, 1>(wide, w, x, m, y, st, di);
+        case 6: return launch_gemv_ldg_pick<FMT, 1, 6, 16, 1>(wide, w, x, m, y, st, di);
+        case 7: return launch_gemv_ldg_pick<FMT, 1, 7, 16, 1>(wide, w, x, m, y, st, di);
+        case 8: return launch_gemv_ldg_pick<FMT, 1, 8, 16, 1>(wide, w, x, m, y, st, di);
         default: break;
       }
     }
   } else {
     if (segs % 8 == 0 && segs / 8 <= 4) {
       switch (segs / 8) {
-        case 1: return launch_gemv_ldg_pick<FMT, 2, 1, 8, 2>(wide, w, x, m, y, st);
-        case 2: return launch_gemv_ldg_pick<FMT, 2, 2, 8, 2>(wide, w, x, m, y, st);
-        case 3: return launch_gemv_ldg_pick<FMT, 2, 3, 8, 2>(wide, w, x, m, y, st);
-        default: return launch_gemv_ldg_pick<FMT, 2, 4, 8, 2>(wide, w, x, m, y, st);
+        case 1: return launch_gemv_ldg_pick<FMT, 2, 1, 8, 2>(wide, w, x, m, y, st, di);
+        case 2: return launch_gemv_ldg_pick<FMT, 2, 2, 8, 2>(wide, w, x, m, y, st, di);
+        case 3: return launch_gemv_ldg_pick<FMT, 2, 3, 8, 2>(wide, w, x, m, y, st, di);
+        default: return launch_gemv_ldg_pick<FMT, 2, 4, 8, 2>(wide, w, x, m, y, st, di);
       }
     }
     if (segs % 16 == 0 && segs / 16 <= 4) {
       switch (segs / 16) {
-        case 3: return launch_gemv_ldg_pick<FMT, 2, 3, 16, 1>(wide, w, x, m, y, st);
-        case 4: return launch_gemv_ldg_pick<FMT, 2, 4, 16, 1>(wide, w, x, m, y, st);
+        case 3: return launch_gemv_ldg_pick<FMT, 2, 3, 16, 1>(wide, w, x, m, y, st, di);
+        case 4: return launch_gemv_ldg_pick<FMT, 2, 4, 16, 1>(wide, w, x, m, y, st, di);
         default: break;
       }
     }
@@ -374,40 +258,18 @@ static qmm_status gemv_ldg_auto(const qmm_weights* w, const uint16_t* x, int m, 
   return QMM_ERR_UNSUPPORTED_SHAPE;
 }
 
-template <int FMT, int NT, int WPC, int DEPTH, int MINB = 2>
-static qmm_status launch_gemv_cpa(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st,
-                                  const DevInfo* di) {
-  const int n = (int)w->n, k = (int)w->k;
-  const int tiles = (n + 15) / 16;
-  const size_t smem = (size_t)WPC * 16 * 16 * 4 + (size_t)WPC * DEPTH * kCpaSlotBytes;
-  auto kern = gemv_fp4_cpa_kernel<FMT, NT, WPC, DEPTH, MINB>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return QMM_ERR_CUDA;
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, WPC * 32, smem) != cudaSuccess || per_sm < 1)
-    return QMM_ERR_CUDA;
-  const int grid = tiles < per_sm * di->sms ? tiles : per_sm * di->sms;
-  kern<<<grid, WPC * 32, smem, st>>>(static_cast<const uint8_t*>(w->data), static_cast<const uint8_t*>(w->scales), x, y,
-                                      n, k, m, w->global_scale, tiles);
-  set_variant("gemv_fp4_cpa<fmt=%d,nt=%d,wpc=%d,depth=%d,minb=%d,grid=%d>", FMT, NT, WPC, DEPTH, MINB, grid);
-  return launch_status();
-}
-
-// Variant override for measurements: QMM_GEMV_VARIANT=cpa|tma|ldg|generic.
+// Kernel override, for tests that cover the kernels a shape does not reach by
+// default: QMM_GEMV_VARIANT=ldg|generic (FP4 formats), iq4|iq4t (IQ4_NL:
+// streaming or tile-resident kernel).  Unset: the default dispatch.
+enum { PICK_DEFAULT = 0, PICK_LDG = 2, PICK_GENERIC = 3, PICK_IQ4_STREAM = 5, PICK_IQ4_TILE = 10 };
 static int gemv_variant_env() {
   const char* v = getenv("QMM_GEMV_VARIANT");
-  if (!v) return 0;
-  if (!strcmp(v, "tma")) return 1;
-  if (!strcmp(v, "ldg")) return 2;
-  if (!strcmp(v, "generic")) return 3;
-  if (!strcmp(v, "cpa")) return 4;
-  if (!strcmp(v, "iq4")) return 5;
-  if (!strcmp(v, "iq4p")) return 6;
-  if (!strcmp(v, "ring")) return 7;
-  if (!strcmp(v, "dual")) return 8;
-  if (!strcmp(v, "iq4w")) return 9;
-  if (!strcmp(v, "iq4t")) return 10;
-  return 0;
+  if (!v) return PICK_DEFAULT;
+  if (!strcmp(v, "ldg")) return PICK_LDG;
+  if (!strcmp(v, "generic")) return PICK_GENERIC;
+  if (!strcmp(v, "iq4")) return PICK_IQ4_STREAM;
+  if (!strcmp(v, "iq4t")) return PICK_IQ4_TILE;
+  return PICK_DEFAULT;
 }
 
 // Tile-resident IQ4_NL kernel (k_iq4t.cuh); UNSUPPORTED_SHAPE launches nothing.
@@ -416,136 +278,26 @@ static qmm_status launch_iq4_tile(const qmm_weights* w0, const qmm_weights* w1, 
                                   int64_t topk, const int32_t* offsets, const int32_t* perm, int64_t P, int m_plain,
                                   void* y, const float* gw, cudaStream_t st, const int32_t* ids = nullptr);
 
-// Warp-per-tile IQ4_NL kernel (k_iq4w.cuh); UNSUPPORTED_SHAPE launches nothing.
-template <int MODE>
-static qmm_status launch_iq4_warp(const qmm_weights* w0, const qmm_weights* w1, const uint16_t* x, int x_per_pair,
-                                  int64_t topk, const int32_t* offsets, const int32_t* perm, int m_plain, void* y,
-                                  const float* gw, cudaStream_t st, const DevInfo* di);
-
-// Persistent IQ4_NL kernel (k_iq4p.cuh).  Returns QMM_ERR_UNSUPPORTED_SHAPE,
-// having launched nothing, when the shape is outside what it takes.
-template <int MODE>
-static qmm_status launch_iq4_persist(const qmm_weights* w0, const qmm_weights* w1, const uint16_t* x, int x_per_pair,
-                                     int64_t topk, const int32_t* ids, int64_t P, int m_plain, void* y,
-                                     const float* gw, cudaStream_t st, const DevInfo* di);
-
 static qmm_status launch_iq4_stream(const qmm_weights* w, const uint16_t* x, int x_per_pair, int64_t topk,
                                    const int32_t* offsets, const int32_t* perm, int m_plain, uint16_t* y,
                                    cudaStream_t st, const DevInfo* di);
-
-// Persistent streaming GEMV, launched with programmatic stream serialization
-// (PDL) so its weight prefetch overlaps the previous kernel's tail.
-template <int FMT, int NT, int WPC, int P, int MINB>
-static qmm_status launch_gemv_stream(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st,
-                                     const DevInfo* di) {
-  const int n = (int)w->n, k = (int)w->k;
-  const int tiles = (n + 15) / 16;
-  auto kern = gemv_fp4_stream_kernel<FMT, NT, WPC, P, MINB>;
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, WPC * 32, 0) != cudaSuccess || per_sm < 1)
-    return QMM_ERR_CUDA;
-  const int grid = tiles < per_sm * di->sms ? tiles : per_sm * di->sms;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(WPC * 32);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const uint8_t* codes = static_cast<const uint8_t*>(w->data);
-  const uint8_t* scales = static_cast<const uint8_t*>(w->scales);
-  const float g = w->global_scale;
-  if (cudaLaunchKernelEx(&cfg, kern, codes, scales, x, y, n, k, m, g, tiles) != cudaSuccess) return QMM_ERR_CUDA;
-  set_variant("gemv_fp4_stream<fmt=%d,nt=%d,wpc=%d,p=%d,minb=%d,grid=%d>", FMT, NT, WPC, P, MINB, grid);
-  return launch_status();
-}
-
-// Measurement hook: QMM_GEMV_CFG picks one compiled configuration of the
-// streaming kernels for k = 4096, m <= 8 (used by the tuning sweep only).
-template <int FMT>
-static bool gemv_cfg_env(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st,
-                         const DevInfo* di, qmm_status* out) {
-  const char* c = getenv("QMM_GEMV_CFG");
-  if (!c || w->k != 4096 || m > 8) return false;
-  if (!strcmp(c, "ldg_w8_s4_b2")) *out = launch_gemv_ldg<FMT, 1, 4, 8, 2>(w, x, m, y, st);
-  else if (!strcmp(c, "ldg_w16_s2_b2")) *out = launch_gemv_ldg<FMT, 1, 2, 16, 2>(w, x, m, y, st);
-  else if (!strcmp(c, "ldg_w8_s4_b3")) *out = launch_gemv_ldg<FMT, 1, 4, 8, 3>(w, x, m, y, st);
-  else if (!strcmp(c, "ldg_w4_s8_b4")) *out = launch_gemv_ldg<FMT, 1, 8, 4, 4>(w, x, m, y, st);
-  else if (!strcmp(c, "cpa_w8_d8_b2")) *out = launch_gemv_cpa<FMT, 1, 8, 8, 2>(w, x, m, y, st, di);
-  else if (!strcmp(c, "cpa_w8_d4_b3")) *out = launch_gemv_cpa<FMT, 1, 8, 4, 3>(w, x, m, y, st, di);
-  else if (!strcmp(c, "cpa_w16_d4_b2")) *out = launch_gemv_cpa<FMT, 1, 16, 4, 2>(w, x, m, y, st, di);
-  else if (!strcmp(c, "cpa_w4_d8_b4")) *out = launch_gemv_cpa<FMT, 1, 4, 8, 4>(w, x, m, y, st, di);
-  else if (!strcmp(c, "str_w4_p4_b4")) *out = launch_gemv_stream<FMT, 1, 4, 4, 4>(w, x, m, y, st, di);
-  else if (!strcmp(c, "str_w4_p8_b3")) *out = launch_gemv_stream<FMT, 1, 4, 8, 3>(w, x, m, y, st, di);
-  else if (!strcmp(c, "str_w8_p4_b2")) *out = launch_gemv_stream<FMT, 1, 8, 4, 2>(w, x, m, y, st, di);
-  else if (!strcmp(c, "str_w8_p2_b3")) *out = launch_gemv_stream<FMT, 1, 8, 2, 3>(w, x, m, y, st, di);
-  else if (!strcmp(c, "str_w2_p8_b6")) *out = launch_gemv_stream<FMT, 1, 2, 8, 6>(w, x, m, y, st, di);
-  else return false;
-  return true;
-}
 
 template <int FMT>
 static qmm_status gemv_fmt(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st,
                            const DevInfo* di) {
   const int64_t n = w->n, k = w->k;
-  // FP4-G16 (fp16 or E4M3 scale per 16) has every streaming variant; MXFP4
-  // the register kernel and the generic one
-  constexpr bool kG16 = FMT == 2 || FMT == 3;
-  if constexpr (kG16) {
-    qmm_status cs;
-    if (gemv_cfg_env<FMT>(w, x, m, y, st, di, &cs)) return cs;
-  }
   const int pick = gemv_variant_env();
-  if constexpr (kG16) {
-    if (pick == 8) {
-      const qmm_status s = gemv_dual_auto<FMT>(w, x, m, y, st, di);
-      if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
-    }
-    if (pick == 7) {
-      const bool xsm = 2 * m * k <= (int64_t)kRingXsMax;
-      const char* cwe = getenv("QMM_RING_CW");  // measurement knob: 16 consumer warps at m <= 8
-      const qmm_status s = (m > 8) ? launch_gemv_ring<FMT, 2, 8, 4, false>(w, x, m, y, st, di)
-                           : (cwe && atoi(cwe) == 16) ? launch_gemv_ring<FMT, 1, 16, 2, false>(w, x, m, y, st, di)
-                           : xsm ? launch_gemv_ring<FMT, 1, 8, 4, true>(w, x, m, y, st, di)
-                                 : launch_gemv_ring<FMT, 1, 8, 4, false>(w, x, m, y, st, di);
-      if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
-    }
-  }
   if constexpr (FMT != 1) {  // the register kernel decodes E2M1 codes only
-    if (pick == 0 || pick == 2) {
-      const qmm_status s = (m <= 8) ? gemv_ldg_auto<FMT, 1>(w, x, m, y, st) : gemv_ldg_auto<FMT, 2>(w, x, m, y, st);
+    if (pick == PICK_DEFAULT || pick == PICK_LDG) {
+      const qmm_status s = (m <= 8) ? gemv_ldg_auto<FMT, 1>(w, x, m, y, st, di) : gemv_ldg_auto<FMT, 2>(w, x, m, y, st, di);
       if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
     }
   }
-  if constexpr (kG16) {
-    const int segs = (int)(k / 128);
-    const bool cpa_ok = k % 1024 == 0 && k >= 1024;
-    if (cpa_ok && pick == 4 && segs % 8 == 0) {
-      if (m <= 8) return launch_gemv_cpa<FMT, 1, 8, 8>(w, x, m, y, st, di);
-      return launch_gemv_cpa<FMT, 2, 8, 8>(w, x, m, y, st, di);
-    }
-    const bool tma_ok = k % kChunkK == 0 && k >= 8 * kChunkK && n >= 16;
-    if (tma_ok && (pick == 0 || pick == 1)) {
-      if (m <= 8) return launch_gemv_tma<FMT, 1, 1>(w, x, m, y, st, di);
-      return launch_gemv_tma<FMT, 1, 2>(w, x, m, y, st, di);
-    }
-  }
-  if (FMT == 1 && pick == 10) {
+  if (FMT == 1 && pick == PICK_IQ4_TILE) {
     const qmm_status s = launch_iq4_tile<IQ_OUT_F16>(w, nullptr, x, 0, 1, nullptr, nullptr, 0, m, y, nullptr, st);
     if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
   }
-  if (FMT == 1 && pick == 9) {
-    const qmm_status s = launch_iq4_warp<IQ_OUT_F16>(w, nullptr, x, 0, 1, nullptr, nullptr, m, y, nullptr, st, di);
-    if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
-  }
-  if (FMT == 1 && pick == 6) {  // persistent kernel: measured slower than the streaming one, kept selectable
-    const qmm_status s = launch_iq4_persist<IQ_OUT_F16>(w, nullptr, x, 0, 1, nullptr, 0, m, y, nullptr, st, di);
-    if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
-  }
-  if (FMT == 1 && k % 128 == 0 && (pick == 0 || pick == 5)) {
+  if (FMT == 1 && k % 128 == 0 && (pick == PICK_DEFAULT || pick == PICK_IQ4_STREAM)) {
     const qmm_status s = launch_iq4_stream(w, x, 0, 1, nullptr, nullptr, m, y, st, di);
     set_variant("gemv_iq4_stream");
     return s;
@@ -662,53 +414,10 @@ static qmm_status launch_iq4_mode(const qmm_weights* w, const qmm_weights* w2, c
     return QMM_ERR_CUDA;
   const int64_t items = ((w->n + 15) / 16) * w->num_experts;
   const int64_t grid = items < (int64_t)per_sm * di->sms ? items : (int64_t)per_sm * di->sms;
-  int pf = 0;  // items of L2 prefetch ahead per CTA (measurement knob QMM_IQ4_PF)
-  if (const char* e = getenv("QMM_IQ4_PF")) pf = atoi(e);
-  if (pf < 0 || pf > 8) return QMM_ERR_INVALID_ARG;
   grouped_iq4_kernel<MODE><<<(unsigned)grid, kIqWarps * 32, smem, st>>>(
       static_cast<const uint8_t*>(w->data), w->expert_data_stride,
       w2 ? static_cast<const uint8_t*>(w2->data) : nullptr, w2 ? w2->expert_data_stride : 0, x, x_per_pair,
-      (int)topk, offsets, perm, m_plain, y, gw, (int)w->n, (int)w->k, (int)w->num_experts, pf);
-  return launch_status();
-}
-
-// Warp-per-tile IQ4_NL kernel (k_iq4w.cuh): persistent, two CTAs of 8 warps
-// per SM, items from the routing sort (offsets/perm) or the plain product.
-template <int MODE>
-static qmm_status launch_iq4_warp(const qmm_weights* w0, const qmm_weights* w1, const uint16_t* x, int x_per_pair,
-                                  int64_t topk, const int32_t* offsets, const int32_t* perm, int m_plain, void* y,
-                                  const float* gw, cudaStream_t st, const DevInfo* di) {
-  const int64_t n = w0->n, k = w0->k;
-  if (w0->fmt != QMM_FMT_IQ4_NL || (w1 && w1->fmt != QMM_FMT_IQ4_NL)) return QMM_ERR_UNSUPPORTED_SHAPE;
-  if (k % 128 || k < 128 || n < 1 || n > INT32_MAX / 2 || k > INT32_MAX / 2) return QMM_ERR_UNSUPPORTED_SHAPE;
-  if (offsets && w0->num_experts > kIqwMaxExperts) return QMM_ERR_UNSUPPORTED_SHAPE;
-  const size_t smem = kIqLutBytes;
-  if (cudaFuncSetAttribute(iq4_warp_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-      cudaSuccess)
-    return QMM_ERR_CUDA;
-  int64_t grid = 2 * (int64_t)di->sms;
-  if (!offsets) {
-    const int64_t items = ((n + 31) / 32) * ((m_plain + 15) / 16);  // tile pairs x token groups
-    grid = std::min<int64_t>(grid, (items + kIqwWarps - 1) / kIqwWarps);
-  }
-  IqwArgs a;
-  a.data0 = static_cast<const uint8_t*>(w0->data);
-  a.data1 = w1 ? static_cast<const uint8_t*>(w1->data) : nullptr;
-  a.dstride0 = w0->expert_data_stride;
-  a.dstride1 = w1 ? w1->expert_data_stride : 0;
-  a.x = x;
-  a.x_per_pair = x_per_pair;
-  a.topk = (int)topk;
-  a.offsets = offsets;
-  a.perm = perm;
-  a.m_plain = m_plain;
-  a.y = y;
-  a.gw = gw;
-  a.n = (int)n;
-  a.k = (int)k;
-  a.E = offsets ? (int)w0->num_experts : 1;
-  iq4_warp_kernel<MODE><<<(unsigned)std::max<int64_t>(grid, 1), kIqwWarps * 32, smem, st>>>(a);
-  set_variant("iq4_warp<mode=%d,grid=%d>", MODE, (int)grid);
+      (int)topk, offsets, perm, m_plain, y, gw, (int)w->n, (int)w->k, (int)w->num_experts);
   return launch_status();
 }
 
@@ -795,67 +504,6 @@ static qmm_status launch_iq4_tile(const qmm_weights* w0, const qmm_weights* w1, 
     return launch_iq4_tile_cfg<MODE, 4, 1, 128, false>(w0, w1, x, x_per_pair, topk, offsets, perm, P, m_plain, y, gw,
                                                        st, ids);
   return QMM_ERR_UNSUPPORTED_SHAPE;
-}
-
-template <int MODE>
-static qmm_status launch_iq4_persist(const qmm_weights* w0, const qmm_weights* w1, const uint16_t* x, int x_per_pair,
-                                     int64_t topk, const int32_t* ids, int64_t P, int m_plain, void* y,
-                                     const float* gw, cudaStream_t st, const DevInfo* di) {
-  const int64_t n = w0->n, k = w0->k;
-  const int E = ids ? (int)w0->num_experts : 1;
-  const int H = (MODE == IQ_SWIGLU) ? 2 : 1;
-  if (w0->fmt != QMM_FMT_IQ4_NL || (w1 && w1->fmt != QMM_FMT_IQ4_NL)) return QMM_ERR_UNSUPPORTED_SHAPE;
-  if (k % 128 || n % 16 || k > (1 << 20) || n > INT32_MAX / 2) return QMM_ERR_UNSUPPORTED_SHAPE;
-  if (ids && (P > kPxMaxPairs || E > kRouteMaxExperts)) return QMM_ERR_UNSUPPORTED_SHAPE;
-  if (!ids && m_plain > 16) return QMM_ERR_UNSUPPORTED_SHAPE;
-  const int steps = (int)(k / 128);
-  int W = (steps + 1) / 2;  // about two 128-wide super-steps per consumer warp per tile
-  if (W > kPxMaxWarps) W = kPxMaxWarps;
-  if (W < 1) W = 1;
-  const uint32_t limit = 232448u - 256u;  // opt-in shared memory per block, less the static part
-  int S = 0, XB = 0;
-  for (int xb = kPxMaxXBuf; xb >= 1 && !S; xb--)
-    for (int s = kPxMaxStages; s >= 2; s--)
-      if (px_layout((int)k, E, (int)P, W, s, xb, H).total <= limit) {
-        S = s;
-        XB = xb;
-        break;
-      }
-  if (!S) return QMM_ERR_UNSUPPORTED_SHAPE;
-  const PxLayout L = px_layout((int)k, E, (int)P, W, S, XB, H);
-  if (cudaFuncSetAttribute(iq4_persist_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total) !=
-      cudaSuccess)
-    return QMM_ERR_CUDA;
-  PxArgs a;
-  a.data0 = static_cast<const uint8_t*>(w0->data);
-  a.data1 = w1 ? static_cast<const uint8_t*>(w1->data) : nullptr;
-  a.dstride0 = w0->expert_data_stride;
-  a.dstride1 = w1 ? w1->expert_data_stride : 0;
-  a.x = x;
-  a.x_per_pair = x_per_pair;
-  a.topk = (int)topk;
-  a.ids = ids;
-  a.P = (int)P;
-  a.m_plain = m_plain;
-  a.y = y;
-  a.gw = gw;
-  a.n = (int)n;
-  a.k = (int)k;
-  a.E = E;
-  a.W = W;
-  a.S = S;
-  a.XB = XB;
-  // items exist only for routed experts, known on the device: one CTA per SM
-  // (plain product: no more CTAs than items)
-  int64_t grid = di->sms;
-  if (!ids) {
-    const int64_t items = (n / 16) * ((m_plain + 15) / 16);
-    if (items < grid) grid = items;
-  }
-  if (grid < 1) grid = 1;
-  iq4_persist_kernel<MODE><<<(unsigned)grid, 32 * (W + 1), L.total, st>>>(a);
-  set_variant("iq4_persist<mode=%d,W=%d,S=%d,XB=%d,grid=%d>", MODE, W, S, XB, (int)grid);
-  return launch_status();
 }
 
 static qmm_status launch_iq4_stream(const qmm_weights* w, const uint16_t* x, int x_per_pair, int64_t topk,
@@ -1188,17 +836,11 @@ qmm_status qmm_grouped_gemv(const qmm_weights* experts, const uint16_t* x, int32
   if (!aligned16(ws)) return QMM_ERR_MISALIGNED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int pick = gemv_variant_env();
-  if (experts->fmt == QMM_FMT_IQ4_NL && experts->k > 0 && pick == 6) {
-    // persistent kernel (buckets the ids itself, no routing pass); measured
-    // slower than route + streaming kernel on the routed-expert shapes
-    s = launch_iq4_persist<IQ_OUT_F16>(experts, nullptr, x, x_per_pair, topk, topk_ids, P, 0, y, nullptr, st, di);
-    if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
-  }
   // IQ4_NL: the tile-resident kernel (its weight loads overlap the previous
   // kernel when most experts have pairs); up to kIqtInKernelRoutePairs pairs
   // each CTA finds its expert's pairs itself, so no routing pass runs.
   // QMM_GEMV_VARIANT=iq4 keeps the streaming kernel.
-  const bool iq4_tile = pick == 10 || pick == 0;
+  const bool iq4_tile = pick == PICK_IQ4_TILE || pick == PICK_DEFAULT;
   if (experts->fmt == QMM_FMT_IQ4_NL && experts->k > 0 && iq4_tile && P <= kIqtInKernelRoutePairs) {
     s = launch_iq4_tile<IQ_OUT_F16>(experts, nullptr, x, x_per_pair, topk, nullptr, nullptr, P, 0, y, nullptr, st,
                                     topk_ids);
@@ -1224,14 +866,7 @@ qmm_status qmm_grouped_gemv(const qmm_weights* experts, const uint16_t* x, int32
       return s;
     }
   }
-  if (experts->fmt == QMM_FMT_IQ4_NL && pick == 9) {
-    s = launch_iq4_warp<IQ_OUT_F16>(experts, nullptr, x, x_per_pair, topk, offsets, perm, 0, y, nullptr, st, di);
-    if (s != QMM_ERR_UNSUPPORTED_SHAPE) {
-      set_variant("route+grouped_iq4_warp");
-      return s;
-    }
-  }
-  if (experts->fmt == QMM_FMT_IQ4_NL && experts->k % 128 == 0 && (pick == 0 || pick == 5)) {
+  if (experts->fmt == QMM_FMT_IQ4_NL && experts->k % 128 == 0 && (pick == PICK_DEFAULT || pick == PICK_IQ4_STREAM)) {
     s = launch_iq4_stream(experts, x, x_per_pair, topk, offsets, perm, 0, y, st, di);
     set_variant("route+grouped_iq4_stream");
     return s;
@@ -1347,26 +982,12 @@ qmm_status qmm_moe_routed(const qmm_weights* gate, const qmm_weights* up, const 
   uint16_t* h = reinterpret_cast<uint16_t*>(p);
   p += align256(2 * (size_t)P * (size_t)f);
   float* yg = reinterpret_cast<float*>(p);
-  if (f > 0 && gemv_variant_env() == 6) {
-    // persistent kernels (each buckets the ids itself): gate/up + SiLU, then
-    // the g-scaled down product, then the slot sum
-    s = launch_iq4_persist<IQ_SWIGLU>(gate, up, x, 0, topk, topk_ids, P, 0, h, nullptr, st, di);
-    if (s == QMM_OK)
-      s = launch_iq4_persist<IQ_SCALED_F32>(down, nullptr, h, 1, topk, topk_ids, P, 0, yg, topk_weights, st, di);
-    if (s == QMM_OK) {
-      combine_kernel<<<grid_for(t * (d / 8), 256, di->sms), 256, 0, st>>>(yg, topk_ids, (int)E, (int)t, (int)topk,
-                                                                           (int)d, out);
-      set_variant("moe:gate_up_swiglu_iq4_persist+down_scaled_iq4_persist+combine");
-      return launch_status();
-    }
-    if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
-  }
   // tile-resident kernels (measured faster than the streaming ones at 1, 4,
   // 16 and 64 tokens); up to kIqtInKernelRoutePairs pairs each CTA finds its
   // expert's pairs itself, so no routing pass runs.  QMM_GEMV_VARIANT=iq4
   // keeps the streaming kernels.
   const int pick = gemv_variant_env();
-  const bool tile = pick == 10 || pick == 0;
+  const bool tile = pick == PICK_IQ4_TILE || pick == PICK_DEFAULT;
   if (f > 0 && tile && P <= kIqtInKernelRoutePairs) {
     s = launch_iq4_tile<IQ_SWIGLU>(gate, up, x, 0, topk, nullptr, nullptr, P, 0, h, nullptr, st, topk_ids);
     if (s == QMM_OK)
@@ -1396,18 +1017,6 @@ qmm_status qmm_moe_routed(const qmm_weights* gate, const qmm_weights* up, const 
       combine_kernel<<<grid_for(t * (d / 8), 256, di->sms), 256, 0, st>>>(yg, topk_ids, (int)E, (int)t, (int)topk,
                                                                            (int)d, out);
       set_variant("moe:route+gate_up_swiglu_iq4_tile+down_scaled_iq4_tile+combine");
-      return launch_status();
-    }
-    if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
-  }
-  if (pick == 9) {  // warp-per-tile kernels
-    s = launch_iq4_warp<IQ_SWIGLU>(gate, up, x, 0, topk, offsets, perm, 0, h, nullptr, st, di);
-    if (s == QMM_OK)
-      s = launch_iq4_warp<IQ_SCALED_F32>(down, nullptr, h, 1, topk, offsets, perm, 0, yg, topk_weights, st, di);
-    if (s == QMM_OK) {
-      combine_kernel<<<grid_for(t * (d / 8), 256, di->sms), 256, 0, st>>>(yg, topk_ids, (int)E, (int)t, (int)topk,
-                                                                           (int)d, out);
-      set_variant("moe:route+gate_up_swiglu_iq4_warp+down_scaled_iq4_warp+combine");
       return launch_status();
     }
     if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;

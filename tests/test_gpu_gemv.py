@@ -35,10 +35,10 @@ def test_gemv_vs_oracle(fmt, n, k, m):
 def test_fast_path_is_used_for_streaming_shapes():
     p, x = _case(synth.FMT_FP4G16_F16, 1000, 4096, 1, 5)
     run_gemv(dev(p), x)
-    assert qmm.qmm_last_variant().startswith(("gemv_fp4_cpa", "gemv_fp4_ldg", "gemv_fp4_tma"))
+    assert qmm.qmm_last_variant().startswith("gemv_fp4_ldg")
 
 
-@pytest.mark.parametrize("variant", ["cpa", "tma", "ldg", "generic", "ring", "dual"])
+@pytest.mark.parametrize("variant", ["ldg", "generic"])
 @pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3])
 @pytest.mark.parametrize("n,k,m", [(1000, 4096, 1), (333, 8192, 3), (64, 2048, 16), (517, 3072, 9)])
 def test_every_streaming_variant_vs_oracle(variant, fmt, n, k, m, monkeypatch):
@@ -46,9 +46,7 @@ def test_every_streaming_variant_vs_oracle(variant, fmt, n, k, m, monkeypatch):
     p, x = _case(fmt, n, k, m, 2000 + n + k + m + fmt)
     y = run_gemv(dev(p), x)
     v = qmm.qmm_last_variant()
-    want = {"cpa": "gemv_fp4_cpa", "tma": "gemv_fp4_tma", "ldg": "gemv_fp4_ldg", "generic": "gemv_generic",
-            "ring": "gemv_fp4_ring" if k <= 4096 else "gemv_generic",  # ring: tiles of <= 48 KB
-            "dual": "gemv_fp4_dual" if m <= 8 and k in (2048, 3072, 4096) else "gemv_generic"}[variant]
+    want = {"ldg": "gemv_fp4_ldg", "generic": "gemv_generic"}[variant]
     assert v.startswith(want), v
     yref, absy = oracle.matmul(fmt, n, k, p.data, p.scales, p.global_scale, x)
     check_tol(y, yref, absy, v)
@@ -113,7 +111,7 @@ def test_config2_in_proj_full(fmt):
     p, x = synth.make_gemv(synth.FP4_IN_PROJ, fmt)
     w = dev(p)
     y = run_gemv(w, x)
-    assert qmm.qmm_last_variant().startswith(("gemv_fp4_cpa", "gemv_fp4_ldg", "gemv_fp4_tma"))
+    assert qmm.qmm_last_variant().startswith("gemv_fp4_ldg")
     yref, absy = oracle.matmul(fmt, p.n, p.k, p.data, p.scales, p.global_scale, x)
     check_tol(y, yref, absy, "in_proj")
     y2 = run_gemv(w, x)
@@ -166,38 +164,21 @@ def test_gemv_edge_cases():
     assert e.value.status == 3
 
 
-@pytest.mark.parametrize("variant", [None, "iq4p", "iq4w", "iq4t", "generic"])
+@pytest.mark.parametrize("variant", [None, "iq4t", "generic"])
 @pytest.mark.parametrize("n,k,m", [(256, 512, 1), (2000, 4096, 5), (48, 2560, 16), (4096, 8192, 2)])
 def test_iq4nl_kernels_vs_oracle(variant, n, k, m, monkeypatch):
     """Each IQ4_NL GEMV kernel: the streaming kernel (default for k % 128 ==
-    0), the persistent kernel (k % 128 == 0 and n % 16 == 0 while 16
-    activation rows and two weight tiles fit in shared memory, k <= 2560 or
-    so; a shape it does not take goes to the generic kernel) and the generic
-    one."""
+    0), the tile-resident one (k <= 4096; a shape it does not take goes to
+    the generic kernel) and the generic one."""
     if variant:
         monkeypatch.setenv("QMM_GEMV_VARIANT", variant)
     p, x = _case(synth.FMT_IQ4_NL, n, k, m, 3000 + n + k + m)
     y = run_gemv(dev(p), x)
     v = qmm.qmm_last_variant()
-    want = {None: ("gemv_iq4_stream",), "iq4p": ("iq4_persist",) if k <= 2560 else ("gemv_generic",),
-            "iq4w": ("iq4_warp",), "iq4t": ("iq4_tile",) if k <= 4096 else ("gemv_generic",),
+    want = {None: ("gemv_iq4_stream",), "iq4t": ("iq4_tile",) if k <= 4096 else ("gemv_generic",),
             "generic": ("gemv_generic",)}[variant]
     assert v.startswith(want), v
     yref, absy = oracle.matmul(synth.FMT_IQ4_NL, n, k, p.data, None, 1.0, x)
-    check_tol(y, yref, absy, v)
-
-
-@pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3])
-@pytest.mark.parametrize("n,k,m", [(1010, 4096, 1), (1010, 3072, 5), (31, 2048, 8), (17, 4096, 2), (16, 4096, 1)])
-def test_dual_tile_kernel_ragged(fmt, n, k, m, monkeypatch):
-    """Two tiles per CTA (registers + a bulk copy into shared memory): a last
-    CTA whose second tile is partial, absent, or the only partial one."""
-    monkeypatch.setenv("QMM_GEMV_VARIANT", "dual")
-    p, x = _case(fmt, n, k, m, 4000 + n + k + m + fmt)
-    y = run_gemv(dev(p), x)
-    v = qmm.qmm_last_variant()
-    assert v.startswith("gemv_fp4_dual"), v
-    yref, absy = oracle.matmul(fmt, n, k, p.data, p.scales, p.global_scale, x)
     check_tol(y, yref, absy, v)
 
 

@@ -108,15 +108,13 @@ def test_grouped_rejects_small_workspace():
     assert e.value.status == 8
 
 
-@pytest.mark.parametrize("variant", [None, "iq4", "iq4p", "iq4w", "iq4t"])
+@pytest.mark.parametrize("variant", [None, "iq4", "iq4t"])
 @pytest.mark.parametrize("E,n,k,t,topk,per_pair", [(3, 64, 256, 50, 2, False), (5, 48, 384, 200, 3, True),
                                                     (2, 16, 128, 2100, 2, False), (32, 32, 128, 1, 4, True)])
 def test_grouped_iq4_many_pairs_per_expert(variant, E, n, k, t, topk, per_pair, monkeypatch):
     """IQ4_NL experts with more than 16 pairs each (several token groups per
     expert, whose row tiles land on different CTAs), with the default
-    (tile-resident) kernel and the opt-in ones;
-    t * topk = 4200 is past the persistent kernel's pair limit (a forced
-    variant that does not take a shape leaves it to the generic kernel)."""
+    (tile-resident) kernel and the streaming one."""
     if variant:
         monkeypatch.setenv("QMM_GEMV_VARIANT", variant)
     rng = np.random.default_rng(E * 1000 + n + k + t)
@@ -126,11 +124,7 @@ def test_grouped_iq4_many_pairs_per_expert(variant, E, n, k, t, topk, per_pair, 
     y, st = _grouped(dev(p), x, ids, per_pair)
     v = qmm.qmm_last_variant()
     assert st == 0, v
-    if variant == "iq4p":
-        assert v.startswith("iq4_persist" if t * topk <= 4096 else "route+grouped_gemv_generic"), v
-    elif variant == "iq4w":
-        assert v.startswith("route+grouped_iq4_warp"), v
-    elif variant == "iq4t":
+    if variant == "iq4t":
         assert "grouped_iq4_tile" in v, v
     elif variant == "iq4":
         assert v.startswith("route+grouped_iq4_stream"), v
