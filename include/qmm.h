@@ -44,8 +44,11 @@
  *     qmm_sync_check() reports and clears it.
  *   - Device base pointers must be 16-byte aligned (QMM_ERR_MISALIGNED
  *     otherwise).
- *   - Calls on different streams may run concurrently; they share no state
- *     besides the error word.
+ *   - Calls on different streams may run concurrently.  What they share:
+ *     the per-device error word; the fixed scratch array of
+ *     qmm_grouped_gemv_noalloc (two calls of that entry point whose kernels
+ *     overlap race on it); and nothing else on the device.  The record read
+ *     by qmm_last_variant() is kept per host thread.
  */
 #ifndef QMM_H_
 #define QMM_H_
@@ -139,15 +142,24 @@ qmm_status qmm_dequant(const qmm_weights* w, uint16_t* out, void* stream);
  *   w       device, [n][k] fp16 (k a multiple of the format's group)
  *   data    device, qmm_data_bytes(fmt, n, k) bytes, written completely
  *   scales  device, qmm_scale_bytes(fmt, n, k) bytes (NULL for IQ4_NL)
+ * The call ends with an empty kernel launched without programmatic
+ * dependent launch, so a qmm_gemv or expert call that follows on the same
+ * stream (those read W before their dependency wait) starts only after the
+ * encoded bytes are complete and visible.
  * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, NOT_SM100, CUDA. */
 qmm_status qmm_quantize(int32_t fmt, const uint16_t* w, int64_t n, int64_t k, void* data, void* scales,
                         void* stream);
 
 /* Fused dequantise-and-multiply for decode batches: y[m][n] = sum_k
  * x[m][k] * W[n][k] with the decoded fp16 weights, fp32 accumulation, one
- * rounding of the sum to fp16.  For FP4G16_E4M3 the global scale g is applied
- * to the fp32 sum instead of to each weight (the difference from the
- * per-weight definition is one fp16 rounding of each weight).
+ * rounding of the sum to fp16.  The weights are the FP16-decoded ones the
+ * FP4-G16 model card's runtime holds resident ("Mamb2_8B_FP4_Recall_SQ3.25",
+ * section "Storage and runtime memory": the decoded FP16 weights stay
+ * resident and no packed-resident FP4 matmul kernel is provided); this call
+ * is that product with W left packed in GPU memory and decoded inside the
+ * kernel.  For FP4G16_E4M3 the global scale g is applied to the fp32 sum
+ * instead of to each weight (the difference from the per-weight definition
+ * is one fp16 rounding of each weight).
  * The FP4 kernels are launched with programmatic dependent launch: they start
  * reading W while the kernel before them on the stream is still running (x
  * and y wait for it).  So W must not be written by the kernel that
@@ -182,8 +194,13 @@ qmm_status qmm_gemv(const qmm_weights* w, const uint16_t* x, int64_t m, uint16_t
 qmm_status qmm_gemv_host(const qmm_weights* w, const uint16_t* x_host, int64_t m, uint16_t* y_host,
                          uint16_t* x_dev, uint16_t* y_dev, void* stream);
 
-/* The same product for a prefill window (m up to any size; the kernel is a
- * tensor-core GEMM that decodes weight tiles into shared memory).
+/* The same product for a prefill window: every token of a window of m
+ * tokens at once (the FP4-G16 model card scores 2,048-token windows,
+ * "Mamb2_8B_FP4_Recall_SQ3.25", section "Measured quality"; the weights are
+ * the decoded ones of section "Storage and runtime memory", as for
+ * qmm_gemv).  m may be any size; from m = 64 (k % 64 == 0) the kernel is a
+ * tensor-core GEMM that decodes weight tiles into shared memory, below that
+ * the decode-batch kernel over 16-token slices.
  *   x       device, [m][k] fp16;  y device, [m][n] fp16
  * Errors: as qmm_gemv. */
 qmm_status qmm_gemm(const qmm_weights* w, const uint16_t* x, int64_t m, uint16_t* y, void* ws,
@@ -242,7 +259,14 @@ qmm_status qmm_grouped_gemv(const qmm_weights* experts, const uint16_t* x, int32
  *
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress, with that device current) and caches it; make that
- * first call before any stream capture.  Every call on a device uses the
+ * first call before any stream capture.  The cache holds one address per
+ * device for the life of the process: after cudaDeviceReset (or anything
+ * else that destroys and recreates the device's primary context) the
+ * address is stale, so do not call this entry point again in that process.
+ * The expert products run on the library's generic grouped kernel (one warp
+ * per 16-row tile, any format), not on the IQ4_NL kernels qmm_grouped_gemv
+ * uses by default: the results agree within the same tolerance, the speed
+ * does not.  Every call on a device uses the
  * same array and it keeps the last call's contents (each call rewrites every
  * entry it reads, so nothing needs clearing): two calls whose kernels
  * overlap on the GPU -- on different streams, or from different host

@@ -273,6 +273,34 @@ __device__ __forceinline__ void ldg_tile_store(float (&red)[WPC][16][16], const 
   }
 }
 
+// Loads of one lane's SPW segments (128-bit layout: 16 code bytes of rows ra
+// and rb at 16*tig of each 64-byte segment, and the two group scales they
+// use; rows past n read as zero codes, scale 1 for MXFP4).
+template <int FMT, int SPW>
+__device__ __forceinline__ void ldg_tile_load(uint4 (&qa)[SPW], uint4 (&qb)[SPW], uint32_t (&sa)[SPW],
+                                              uint32_t (&sb)[SPW], const uint8_t* __restrict__ codes,
+                                              const uint8_t* __restrict__ scales, int64_t ra, int64_t rb, bool va,
+                                              bool vb, int seg0, int tig, int64_t crow, int64_t srow) {
+#pragma unroll
+  for (int i = 0; i < SPW; i++) {
+    const int seg = seg0 + i;
+    const int64_t cb = (int64_t)seg * 64 + tig * 16;
+    const int64_t gi = (int64_t)seg * 8 + tig * 2;  // first of the two group scales
+    qa[i] = va ? ldg_stream128(codes + ra * crow + cb) : make_uint4(0, 0, 0, 0);
+    qb[i] = vb ? ldg_stream128(codes + rb * crow + cb) : make_uint4(0, 0, 0, 0);
+    if (FMT == 2) {
+      sa[i] = va ? ldg_stream32(scales + (ra * srow + gi) * 2) : 0u;
+      sb[i] = vb ? ldg_stream32(scales + (rb * srow + gi) * 2) : 0u;
+    } else if (FMT == 4) {  // the lane's 32 k are one MXFP4 group: one E8M0 byte (127 = 1 for rows past n)
+      sa[i] = e8m0_f16_factor_pair(va ? ldg_stream8(scales + ra * (srow >> 1) + seg * 4 + tig) : 127u);
+      sb[i] = e8m0_f16_factor_pair(vb ? ldg_stream8(scales + rb * (srow >> 1) + seg * 4 + tig) : 127u);
+    } else {
+      sa[i] = va ? e4m3x2_to_f16x2(ldg_stream16(scales + ra * srow + gi)) : 0u;
+      sb[i] = vb ? e4m3x2_to_f16x2(ldg_stream16(scales + rb * srow + gi)) : 0u;
+    }
+  }
+}
+
 // WIDE (k % 256 == 0, SPW even, codes 32-byte aligned): each lane loads its
 // bytes of two segments with one 256-bit load per row, and their scales with
 // one load (8 B fp16, 4 B E4M3, 2 B E8M0), the segment pairing of
@@ -280,8 +308,7 @@ __device__ __forceinline__ void ldg_tile_store(float (&red)[WPC][16][16], const 
 template <int FMT, int NT, int SPW, int WPC = kLdgWarps, int MINB = 2, bool WIDE = false, bool XW = false>
 __global__ void __launch_bounds__(WPC * 32, MINB)
     gemv_fp4_ldg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
-                        const uint16_t* __restrict__ x, uint16_t* __restrict__ y, int n, int k, int m, float g,
-                        int wave, int pf_ctas) {
+                        const uint16_t* __restrict__ x, uint16_t* __restrict__ y, int n, int k, int m, float g) {
   static_assert(!WIDE || SPW % 2 == 0, "WIDE pairs segments");
   __shared__ float red[WPC][16][16];  // [warp][token][row]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -321,48 +348,9 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
       }
     }
   } else {
-#pragma unroll
-  for (int i = 0; i < SPW; i++) {
-    const int seg = seg0 + i;
-    const int64_t cb = (int64_t)seg * 64 + tig * 16;
-    const int64_t gi = (int64_t)seg * 8 + tig * 2;  // first of the two group scales
-    qa[i] = va ? ldg_stream128(codes + ra * crow + cb) : make_uint4(0, 0, 0, 0);
-    qb[i] = vb ? ldg_stream128(codes + rb * crow + cb) : make_uint4(0, 0, 0, 0);
-    if (FMT == 2) {
-      sa[i] = va ? ldg_stream32(scales + (ra * srow + gi) * 2) : 0u;
-      sb[i] = vb ? ldg_stream32(scales + (rb * srow + gi) * 2) : 0u;
-    } else if (FMT == 4) {  // the lane's 32 k are one MXFP4 group: one E8M0 byte (127 = 1 for rows past n)
-      sa[i] = e8m0_f16_factor_pair(va ? ldg_stream8(scales + ra * (srow >> 1) + seg * 4 + tig) : 127u);
-      sb[i] = e8m0_f16_factor_pair(vb ? ldg_stream8(scales + rb * (srow >> 1) + seg * 4 + tig) : 127u);
-    } else {
-      sa[i] = va ? e4m3x2_to_f16x2(ldg_stream16(scales + ra * srow + gi)) : 0u;
-      sb[i] = vb ? e4m3x2_to_f16x2(ldg_stream16(scales + rb * srow + gi)) : 0u;
-    }
-  }
+    ldg_tile_load<FMT, SPW>(qa, qb, sa, sb, codes, scales, ra, rb, va, vb, seg0, tig, crow, srow);
   }
   pdl_wait();  // x may be the previous kernel's output; y may still be read by it
-  // The CTAs of the first resident wave (the `wave` lowest block indices)
-  // hold all their weights in registers when the dependency wait releases
-  // and then decode and multiply at once, with no further loads in flight:
-  // HBM would idle until the second wave's CTAs start.  So thread 0 of each
-  // asks the copy engine to bring the tile of the CTA one wave later into L2
-  // (its 16 code rows, one contiguous range, in at most two pieces of
-  // 32 KB, and its 16 scale rows; 16-byte-aligned starts and lengths), so
-  // those CTAs' loads hit L2.  Only whole tiles are prefetched: the host
-  // passes pf_ctas, the number of first-wave CTAs whose next-wave tile has
-  // all 16 rows (0 where k > 8192 or the 32-bit offsets could overflow).
-  // Branch-free (predicated prefetches), which keeps the kernel at its
-  // register count.
-  {
-    const uint32_t on = threadIdx.x == 0 && (int)blockIdx.x < pf_ctas;
-    const uint32_t t2 = blockIdx.x + (uint32_t)wave;
-    const uint32_t ctb = 8u * (uint32_t)k;                                          // code bytes of a tile
-    const uint32_t stb = (FMT == 2) ? 2u * k : (FMT == 4) ? (uint32_t)k >> 1 : (uint32_t)k;  // scale bytes
-    const uint8_t* pc = codes + t2 * ctb;
-    prefetch_l2_bulk_if(pc, min(32768u, ctb), on);
-    prefetch_l2_bulk_if(pc + 32768, ctb - 32768u, on & (ctb > 32768u));
-    prefetch_l2_bulk_if(scales + t2 * stb, stb, on);
-  }
   float acc[NT][4];
 #pragma unroll
   for (int j = 0; j < NT; j++)
@@ -370,6 +358,73 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
     for (int c = 0; c < 4; c++) acc[j][c] = 0.f;
   ldg_tile_mma<FMT, NT, SPW, WIDE, XW>(acc, qa, qb, sa, sb, seg0, grp, tig, x, k, m);
   ldg_tile_store<FMT, NT, WPC>(red, acc, warp, grp, tig, n0, n, m, g, y);
+}
+
+// ---------------------------------------------------------------------------
+// Split-K for narrow matrices.  When n has too few 16-row tiles to fill the
+// GPU (out_proj: 256 tiles of k = 8192 on 148 SMs), the CS CTAs of a
+// thread-block cluster (launch attribute, CS = 2..8) share one tile: CTA c
+// of the cluster multiplies k range c of CS equal ranges (its WPC warps
+// split it as in gemv_fp4_ldg, the same loads and MMAs), the CTA's warps are
+// summed in warp order into `part`, and after a cluster barrier the CTAs
+// read each other's `part` through distributed shared memory: CTA c adds, in
+// rank order 0..CS-1, the outputs whose index is c mod CS and stores them.
+// A second cluster barrier keeps every CTA's `part` alive until all reads
+// are done.  The order of every sum is fixed, so results are deterministic.
+// Programmatic dependent launch as in gemv_fp4_ldg (weights before the wait).
+// ---------------------------------------------------------------------------
+template <int FMT, int NT, int SPW, int WPC, int MINB, bool XW>
+__global__ void __launch_bounds__(WPC * 32, MINB)
+    gemv_fp4_splitk_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                           const uint16_t* __restrict__ x, uint16_t* __restrict__ y, int n, int k, int m, float g) {
+  __shared__ float red[WPC][16][16];  // [warp][token][row]
+  __shared__ float part[16][16];      // [token][row]: this CTA's k range, warps summed
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int grp = lane >> 2, tig = lane & 3;
+  const int cs = (int)cluster_nctarank(), c = (int)cluster_ctarank();
+  const int n0 = (blockIdx.x / cs) * 16;
+  const int ra = n0 + grp, rb = ra + 8;
+  const bool va = ra < n, vb = rb < n;
+  const int seg0 = (c * WPC + warp) * SPW;
+  const int64_t crow = k >> 1, srow = k >> 4;
+
+  pdl_launch_dependents();
+  uint4 qa[SPW], qb[SPW];
+  uint32_t sa[SPW], sb[SPW];
+  ldg_tile_load<FMT, SPW>(qa, qb, sa, sb, codes, scales, ra, rb, va, vb, seg0, tig, crow, srow);
+  pdl_wait();  // x may be the previous kernel's output; y may still be read by it
+
+  float acc[NT][4];
+#pragma unroll
+  for (int j = 0; j < NT; j++)
+#pragma unroll
+    for (int q = 0; q < 4; q++) acc[j][q] = 0.f;
+  ldg_tile_mma<FMT, NT, SPW, false, XW>(acc, qa, qb, sa, sb, seg0, grp, tig, x, k, m);
+#pragma unroll
+  for (int j = 0; j < NT; j++) {
+    const int t0 = 8 * j + 2 * tig;
+    red[warp][t0][grp] = acc[j][0];
+    red[warp][t0 + 1][grp] = acc[j][1];
+    red[warp][t0][grp + 8] = acc[j][2];
+    red[warp][t0 + 1][grp + 8] = acc[j][3];
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < 16 * m; idx += WPC * 32) {
+    const int row = idx & 15, tok = idx >> 4;
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < WPC; w++) v += red[w][tok][row];
+    part[tok][row] = v;
+  }
+  cluster_sync();
+  const float gs = (FMT == 3) ? g : 1.0f;
+  for (int idx = c + cs * (int)threadIdx.x; idx < 16 * m; idx += cs * WPC * 32) {
+    const int row = idx & 15, tok = idx >> 4;
+    float v = 0.f;
+    for (int r = 0; r < cs; r++) v += ld_dsmem_f32(&part[tok][row], (uint32_t)r);
+    if (n0 + row < n) y[(int64_t)tok * n + n0 + row] = f32_to_f16_bits(v * gs);
+  }
+  cluster_sync();
 }
 
 }  // namespace qmm

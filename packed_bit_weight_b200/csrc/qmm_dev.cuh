@@ -252,28 +252,32 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* m, 
       : "memory");
 }
 
-// Contiguous bulk copy global -> this CTA's shared memory through the TMA
-// engine, completing `bytes` of transaction on `bar`.  Both addresses 16-byte
-// aligned, bytes a multiple of 16 (callers check).  No multicast.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
-               : "memory");
+// ---------------------------------------------------------------------------
+// Thread-block clusters: rank, barrier, distributed shared memory reads
+// (plain loads from a peer CTA's shared memory on this GPU; no multicast).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
 }
-
-// Bulk prefetch of a global byte range into L2 (no shared memory, no
-// completion; a hint): address 16-byte aligned, bytes a multiple of 16.
-__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes));
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
 }
-
-// The same prefetch, issued only when `on` is nonzero (a predicated
-// instruction, no branch).
-__device__ __forceinline__ void prefetch_l2_bulk_if(const void* p, uint32_t bytes, uint32_t on) {
-  asm volatile(
-      "{\n .reg .pred q;\n setp.ne.u32 q, %2, 0;\n @q cp.async.bulk.prefetch.L2.global [%0], %1;\n}" ::"l"(
-          reinterpret_cast<uint64_t>(p)),
-      "r"(bytes), "r"(on));
+// Every thread of every CTA of the cluster arrives, then waits for all: the
+// shared-memory writes before it are visible cluster-wide after it.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// fp32 at the same shared-memory offset as `local` in the CTA of rank r.
+__device__ __forceinline__ float ld_dsmem_f32(const float* local, uint32_t r) {
+  uint32_t remote;
+  float v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(local)), "r"(r));
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
 }
 
 // bar.sync on a named barrier that also returns the OR of every thread's flag.

@@ -130,6 +130,11 @@ static int grid_for(int64_t items, int per_block, int sms, int waves = 8) {
   return (int)b;
 }
 
+// An empty kernel: launched without programmatic dependent launch after a
+// kernel that writes packed weights, so that a following kernel which reads
+// weights before its dependency wait overlaps nothing that writes them.
+__global__ void ordering_kernel() {}
+
 // ---------------------------------------------------------------------------
 // GEMV dispatch
 // ---------------------------------------------------------------------------
@@ -139,17 +144,6 @@ static qmm_status launch_gemv_ldg(const qmm_weights* w, const uint16_t* x, int m
   const int n = (int)w->n, k = (int)w->k;
   const int tiles = (n + 15) / 16;
   auto kern = gemv_fp4_ldg_kernel<FMT, NT, SPW, WPC, MINB, WIDE, XW>;
-  // CTAs resident at once (one wave): the first wave prefetches the second
-  // into L2 after its dependency wait.  QMM_GEMV_L2PF=0 turns it off (A/B).
-  static int per_sm = -1;
-  if (per_sm < 0 && cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, WPC * 32, 0) != cudaSuccess)
-    return QMM_ERR_CUDA;
-  const char* pfe = getenv("QMM_GEMV_L2PF");
-  const int wave = per_sm * di->sms;
-  // first-wave CTAs whose tile one wave later is whole (16 rows); codes of a
-  // tile in at most two 32 KB pieces (k <= 8192), offsets within 32 bits
-  int pf_ctas = std::max(0, std::min(wave, n / 16 - wave));
-  if ((pfe && pfe[0] == '0') || k > 8192 || (int64_t)2 * wave * 8 * k >= ((int64_t)1 << 32)) pf_ctas = 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(tiles);
   cfg.blockDim = dim3(WPC * 32);
@@ -163,10 +157,9 @@ static qmm_status launch_gemv_ldg(const qmm_weights* w, const uint16_t* x, int m
   const uint8_t* codes = static_cast<const uint8_t*>(w->data);
   const uint8_t* scales = static_cast<const uint8_t*>(w->scales);
   const float g = w->global_scale;
-  if (cudaLaunchKernelEx(&cfg, kern, codes, scales, x, y, n, k, m, g, wave, pf_ctas) != cudaSuccess)
-    return QMM_ERR_CUDA;
-  set_variant("gemv_fp4_ldg<fmt=%d,nt=%d,spw=%d,wpc=%d,minb=%d,wide=%d,xw=%d,tiles=%d,l2pf=%d>", FMT, NT, SPW, WPC,
-              MINB, WIDE ? 1 : 0, XW ? 1 : 0, tiles, pf_ctas > 0 ? 1 : 0);
+  if (cudaLaunchKernelEx(&cfg, kern, codes, scales, x, y, n, k, m, g) != cudaSuccess) return QMM_ERR_CUDA;
+  set_variant("gemv_fp4_ldg<fmt=%d,nt=%d,spw=%d,wpc=%d,minb=%d,wide=%d,xw=%d,tiles=%d>", FMT, NT, SPW, WPC, MINB,
+              WIDE ? 1 : 0, XW ? 1 : 0, tiles);
   return launch_status();
 }
 
@@ -258,6 +251,77 @@ static qmm_status gemv_ldg_auto(const qmm_weights* w, const uint16_t* x, int m, 
   return QMM_ERR_UNSUPPORTED_SHAPE;
 }
 
+// Split-K GEMV (k_gemv.cuh, gemv_fp4_splitk_kernel): clusters of cs CTAs
+// share a 16-row tile, 4 warps per CTA, spw segments per warp.
+template <int FMT, int NT, int SPW, bool XW>
+static qmm_status launch_gemv_splitk(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st,
+                                     int cs) {
+  const int n = (int)w->n, k = (int)w->k;
+  const int64_t tiles = (n + 15) / 16;
+  if (tiles * cs > INT32_MAX) return QMM_ERR_UNSUPPORTED_SHAPE;
+  constexpr int kMinb = NT == 1 ? 4 : 2;
+  auto kern = gemv_fp4_splitk_kernel<FMT, NT, SPW, 4, kMinb, XW>;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(tiles * cs));
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = (unsigned)cs;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  if (cudaLaunchKernelEx(&cfg, kern, static_cast<const uint8_t*>(w->data), static_cast<const uint8_t*>(w->scales), x,
+                         y, n, k, m, w->global_scale) != cudaSuccess)
+    return QMM_ERR_CUDA;
+  set_variant("gemv_fp4_splitk<fmt=%d,nt=%d,spw=%d,wpc=4,cs=%d,xw=%d,tiles=%lld>", FMT, NT, SPW, cs, XW ? 1 : 0,
+              (long long)tiles);
+  return launch_status();
+}
+
+// Clusters per tile for a narrow matrix: the smallest power of two (2..8)
+// that gives at least four CTAs per SM, with whole 4-warp CTAs of 1..8
+// segments per warp (1..4 at m > 8); 0 = no split (wide enough, or k does
+// not divide).  QMM_GEMV_SPLITK=<cs> forces cs (0 turns split-K off).
+static int splitk_clusters(int64_t n, int64_t k, int m, int sms) {
+  const int64_t tiles = (n + 15) / 16, segs = k / 128;
+  const int max_spw = m > 8 ? 4 : 8;
+  auto ok = [&](int cs) {
+    return k % 128 == 0 && segs % (4 * cs) == 0 && segs / (4 * cs) >= 1 && segs / (4 * cs) <= max_spw;
+  };
+  if (const char* e = getenv("QMM_GEMV_SPLITK")) {
+    const int cs = atoi(e);
+    return (cs == 2 || cs == 4 || cs == 8) && ok(cs) ? cs : 0;
+  }
+  if (tiles >= 2 * (int64_t)sms) return 0;
+  for (int cs = 2; cs <= 8; cs *= 2)
+    if (ok(cs) && tiles * cs >= 4 * (int64_t)sms) return cs;
+  for (int cs = 8; cs >= 2; cs /= 2)
+    if (ok(cs)) return cs;
+  return 0;
+}
+
+template <int FMT, int NT>
+static qmm_status gemv_splitk_auto(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st,
+                                   int cs) {
+  const int spw = (int)(w->k / 128) / (4 * cs);
+  const bool xw = (reinterpret_cast<uintptr_t>(x) & 31u) == 0;
+  switch (spw) {
+    case 1: return xw ? launch_gemv_splitk<FMT, NT, 1, true>(w, x, m, y, st, cs) : launch_gemv_splitk<FMT, NT, 1, false>(w, x, m, y, st, cs);
+    case 2: return xw ? launch_gemv_splitk<FMT, NT, 2, true>(w, x, m, y, st, cs) : launch_gemv_splitk<FMT, NT, 2, false>(w, x, m, y, st, cs);
+    case 4: return xw ? launch_gemv_splitk<FMT, NT, 4, true>(w, x, m, y, st, cs) : launch_gemv_splitk<FMT, NT, 4, false>(w, x, m, y, st, cs);
+    case 8:
+      if constexpr (NT == 1)
+        return xw ? launch_gemv_splitk<FMT, NT, 8, true>(w, x, m, y, st, cs) : launch_gemv_splitk<FMT, NT, 8, false>(w, x, m, y, st, cs);
+      return QMM_ERR_UNSUPPORTED_SHAPE;
+    default: return QMM_ERR_UNSUPPORTED_SHAPE;
+  }
+}
+
 // Kernel override, for tests that cover the kernels a shape does not reach by
 // default: QMM_GEMV_VARIANT=ldg|generic (FP4 formats), iq4|iq4t (IQ4_NL:
 // streaming or tile-resident kernel).  Unset: the default dispatch.
@@ -287,7 +351,15 @@ static qmm_status gemv_fmt(const qmm_weights* w, const uint16_t* x, int m, uint1
                            const DevInfo* di) {
   const int64_t n = w->n, k = w->k;
   const int pick = gemv_variant_env();
-  if constexpr (FMT != 1) {  // the register kernel decodes E2M1 codes only
+  if constexpr (FMT != 1) {  // the register kernels decode E2M1 codes only
+    if (pick == PICK_DEFAULT) {
+      const int cs = splitk_clusters(n, k, m, di->sms);
+      if (cs) {
+        const qmm_status s = (m <= 8) ? gemv_splitk_auto<FMT, 1>(w, x, m, y, st, cs)
+                                      : gemv_splitk_auto<FMT, 2>(w, x, m, y, st, cs);
+        if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
+      }
+    }
     if (pick == PICK_DEFAULT || pick == PICK_LDG) {
       const qmm_status s = (m <= 8) ? gemv_ldg_auto<FMT, 1>(w, x, m, y, st, di) : gemv_ldg_auto<FMT, 2>(w, x, m, y, st, di);
       if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
@@ -657,6 +729,12 @@ qmm_status qmm_quantize(int32_t fmt, const uint16_t* w, int64_t n, int64_t k, vo
     quantize_fp4_kernel<2><<<grid_for(ng, 128, di->sms), 128, 0, st>>>(w, d, sc, ng);
     set_variant("quantize_fp4<fmt=2>");
   }
+  if (cudaGetLastError() != cudaSuccess) return QMM_ERR_CUDA;
+  // The GEMV and expert kernels read W before their dependency wait, so the
+  // kernel right before them must not be the one that wrote W: this empty
+  // kernel (plain launch, it starts after the encoder has finished) takes
+  // that place.
+  ordering_kernel<<<1, 32, 0, st>>>();
   return launch_status();
 }
 
@@ -787,7 +865,8 @@ static size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
 
 static qmm_status check_routing(const int32_t* ids, int64_t t, int64_t topk, int64_t num_experts) {
   if (t < 0 || topk < 0 || num_experts < 1) return QMM_ERR_INVALID_ARG;
-  if (num_experts > kRouteMaxExperts || t * topk > INT32_MAX / 2) return QMM_ERR_UNSUPPORTED_SHAPE;
+  // bound the factors before multiplying them (no int64 overflow)
+  if (num_experts > kRouteMaxExperts || (topk > 0 && t > (INT32_MAX / 2) / topk)) return QMM_ERR_UNSUPPORTED_SHAPE;
   if (t * topk > 0 && !ids) return QMM_ERR_INVALID_ARG;
   if (ids && !aligned16(ids)) return QMM_ERR_MISALIGNED;
   return QMM_OK;
@@ -884,6 +963,7 @@ qmm_status qmm_grouped_gemv(const qmm_weights* experts, const uint16_t* x, int32
 size_t qmm_workspace_bytes(int32_t op, const qmm_weights* w, int64_t m, int64_t t, int64_t topk) {
   if (op == QMM_OP_GROUPED || op == QMM_OP_MOE) {
     if (!w || w->num_experts < 1 || t < 0 || topk < 0 || w->n < 0 || w->k < 0) return 0;
+    if (topk > 0 && t > (INT32_MAX / 2) / topk) return 0;  // the call itself refuses these sizes
     size_t b = align256(4 * (size_t)(w->num_experts + 1)) + align256(4 * (size_t)(t * topk));
     if (op == QMM_OP_MOE)  // h [t*topk][f] fp16, g-scaled slot outputs [t*topk][d] fp32
       b += align256(2 * (size_t)(t * topk) * (size_t)w->n) + align256(4 * (size_t)(t * topk) * (size_t)w->k);

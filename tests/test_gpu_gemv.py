@@ -35,7 +35,10 @@ def test_gemv_vs_oracle(fmt, n, k, m):
 def test_fast_path_is_used_for_streaming_shapes():
     p, x = _case(synth.FMT_FP4G16_F16, 1000, 4096, 1, 5)
     run_gemv(dev(p), x)
-    assert qmm.qmm_last_variant().startswith("gemv_fp4_ldg")
+    assert qmm.qmm_last_variant().startswith("gemv_fp4_splitk")   # 63 tiles: split across clusters
+    p, x = _case(synth.FMT_FP4G16_F16, 18560, 4096, 1, 5)
+    run_gemv(dev(p), x)
+    assert qmm.qmm_last_variant().startswith("gemv_fp4_ldg")      # 1160 tiles: one CTA per tile
 
 
 @pytest.mark.parametrize("variant", ["ldg", "generic"])
@@ -74,9 +77,10 @@ def test_register_kernel_both_load_layouts(wide, fmt, n, k, m, monkeypatch):
 
 
 @pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_MXFP4])
-def test_codes_16_byte_aligned_take_the_128_bit_layout(fmt):
+def test_codes_16_byte_aligned_take_the_128_bit_layout(fmt, monkeypatch):
     """Codes that are 16- but not 32-byte aligned (legal in the ABI) must not
     reach the 256-bit loads."""
+    monkeypatch.setenv("QMM_GEMV_VARIANT", "ldg")
     n, k, m = 300, 4096, 2
     p, x = _case(fmt, n, k, m, 91 + fmt)
     w = dev(p)
@@ -200,7 +204,7 @@ def test_mxfp4_small_and_normal_scales(variant, m, monkeypatch):
     x = synth.gen_x(rng, m, k)
     y = run_gemv(dev(p), x)
     v = qmm.qmm_last_variant()
-    assert v.startswith("gemv_generic" if variant else "gemv_fp4_ldg"), v
+    assert v.startswith(("gemv_generic",) if variant else ("gemv_fp4_ldg", "gemv_fp4_splitk")), v
     yref, absy = oracle.matmul(p.fmt, n, k, p.data, p.scales, 1.0, x)
     check_tol(y, yref, absy, v)
 
@@ -283,6 +287,7 @@ def test_gemv_host_argument_errors():
 def test_register_kernel_128_bit_activation_loads(fmt, n, k, m, how, monkeypatch):
     """The 16-byte activation loads: forced by QMM_GEMV_XW=0, or taken
     because x is 16- but not 32-byte aligned (legal in the ABI)."""
+    monkeypatch.setenv("QMM_GEMV_VARIANT", "ldg")
     p, xb = _case(fmt, n, k, m, 7000 + n + k + m + fmt)
     w = dev(p)
     if how == "knob":
@@ -302,3 +307,64 @@ def test_register_kernel_128_bit_activation_loads(fmt, n, k, m, how, monkeypatch
     assert v.startswith("gemv_fp4_ldg") and "xw=0" in v, v
     yref, absy = oracle.matmul(fmt, n, k, p.data, p.scales, p.global_scale, xb)
     check_tol(y, yref, absy, v)
+
+
+@pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3, synth.FMT_MXFP4])
+@pytest.mark.parametrize("n,k,m,cs", [(100, 4096, 1, 2), (100, 4096, 1, 4), (100, 4096, 1, 8), (333, 8192, 3, 2),
+                                      (333, 8192, 3, 8), (77, 2048, 16, 2), (77, 2048, 16, 4), (30, 1024, 9, 2),
+                                      (77, 2048, 16, 8), (50, 1536, 5, 4), (40, 3072, 2, 2), (17, 512, 1, 2)])
+def test_split_k_clusters_vs_oracle(fmt, n, k, m, cs, monkeypatch):
+    """Split-K over a cluster of cs CTAs per 16-row tile (ragged n, m = 1..16),
+    reduced through distributed shared memory; split counts that do not
+    divide the shape into whole 4-warp CTAs (k = 2048 at cs = 8, k = 1536,
+    3072, 512) fall back to the unsplit kernel.  Deterministic: two calls
+    give the same bits."""
+    monkeypatch.setenv("QMM_GEMV_SPLITK", str(cs))
+    p, x = _case(fmt, n, k, m, 8000 + n + k + m + cs + fmt)
+    w = dev(p)
+    y = run_gemv(w, x)
+    v = qmm.qmm_last_variant()
+    segs = k // 128
+    spw = segs // (4 * cs)
+    split = segs % (4 * cs) == 0 and spw in ((1, 2, 4, 8) if m <= 8 else (1, 2, 4))
+    assert v.startswith("gemv_fp4_splitk" if split else "gemv_fp4_ldg"), v
+    if split:
+        assert "cs=%d" % cs in v, v
+    yref, absy = oracle.matmul(fmt, n, k, p.data, p.scales, p.global_scale, x)
+    check_tol(y, yref, absy, v)
+    assert np.array_equal(run_gemv(w, x), y)
+
+
+@pytest.mark.parametrize("m", [1, 4, 16])
+def test_out_proj_takes_split_k_by_default(m):
+    """The 4096 x 8192 out_proj (256 tiles) is split across clusters; the full
+    output matches the oracle."""
+    mats = synth.make_sweep(mats=[("out_proj", 4096, 8192)])
+    p, xall = mats["out_proj"]
+    y = run_gemv(dev(p), xall[:m])
+    v = qmm.qmm_last_variant()
+    assert v.startswith("gemv_fp4_splitk"), v
+    yref, absy = oracle.matmul(p.fmt, p.n, p.k, p.data, p.scales, p.global_scale, xall[:m])
+    check_tol(y, yref, absy, v)
+
+
+@pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_MXFP4])
+@pytest.mark.parametrize("m", [1, 12])
+def test_split_k_with_16_byte_aligned_activations(fmt, m):
+    """x 16- but not 32-byte aligned: the split-K kernel takes the 128-bit
+    activation loads (xw=0)."""
+    n, k = 200, 4096
+    p, xb = _case(fmt, n, k, m, 9100 + m + fmt)
+    w = dev(p)
+    buf = torch.zeros(m * k + 32, dtype=torch.int16, device="cuda")
+    off = 8 if buf.data_ptr() % 32 == 0 else 0
+    xs = buf[off:off + m * k].view(m, k)
+    assert xs.data_ptr() % 32 == 16
+    xs.copy_(to_dev_u16(xb))
+    yd = torch.empty((m, n), dtype=torch.int16, device="cuda")
+    qmm.qmm_gemv(w, xs, yd)
+    assert qmm.qmm_sync_check() == 0
+    v = qmm.qmm_last_variant()
+    assert v.startswith("gemv_fp4_splitk") and "xw=0" in v, v
+    yref, absy = oracle.matmul(fmt, n, k, p.data, p.scales, p.global_scale, xb)
+    check_tol(from_dev_u16(yd), yref, absy, v)

@@ -94,3 +94,32 @@ def test_quantize_rejects_e4m3_and_ragged_k():
     w2 = torch.zeros((2, 48), dtype=torch.int16, device="cuda")
     with pytest.raises(qmm.QmmError):
         qmm.qmm_quantize(synth.FMT_MXFP4, w2, data, sc)
+
+
+@pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_MXFP4])
+def test_quantize_then_gemv_back_to_back_on_one_stream(fmt):
+    """qmm_quantize writes packed W and qmm_gemv, next on the same stream
+    with nothing in between, reads W before its dependency wait: the GEMV
+    must see the encoded bytes (the oracle's product of the oracle's
+    encoding), also when the same buffers held other weights just before."""
+    from gpu_util import check_tol
+    rng = np.random.default_rng(77 + fmt)
+    n, k, m = 4096, 4096, 2
+    w_old, w_new = _weights(rng, n, k), _weights(rng, n, k)
+    x_bits = synth.gen_x(rng, m, k)
+    data = torch.empty((qmm.qmm_data_bytes(fmt, n, k),), dtype=torch.uint8, device="cuda")
+    scales = torch.empty((qmm.qmm_scale_bytes(fmt, n, k),), dtype=torch.uint8, device="cuda")
+    x = to_dev_u16(x_bits)
+    y = torch.empty((m, n), dtype=torch.int16, device="cuda")
+    pw = qmm.PackedWeights(fmt, n, k, data, scales)
+    st = torch.cuda.current_stream()
+    qmm.qmm_quantize(fmt, to_dev_u16(w_old).view(n, k), data, scales, stream=st)
+    wd = to_dev_u16(w_new).view(n, k)
+    torch.cuda.synchronize()
+    for _ in range(3):
+        qmm.qmm_quantize(fmt, wd, data, scales, stream=st)
+        qmm.qmm_gemv(pw, x, y, stream=st)
+    assert qmm.qmm_sync_check() == 0
+    od, os_ = oracle.quantize(fmt, n, k, w_new)
+    yref, absy = oracle.matmul(fmt, n, k, od, os_, 1.0, x_bits)
+    check_tol(from_dev_u16(y), yref, absy, "quantize->gemv " + qmm.qmm_last_variant())

@@ -107,6 +107,11 @@ def test_grouped_argument_errors():
     assert call(_stack(), ids=_vp(FAKE + 4)) == MISALIGNED
     assert call(_stack(), per_pair=2) == INVALID
     assert call(_stack(fmt=2, scale_stride=4)) == INVALID                  # FP4 scale stride below one matrix
+    # t * topk would overflow int64: refused on the bounds, before any product
+    assert call(_stack(), t=1 << 62, topk=1 << 40) == UNSUPPORTED
+    assert call(_stack(), t=(1 << 30), topk=2) == UNSUPPORTED               # more pairs than INT32_MAX / 2
+    assert L.qmm_grouped_gemv_noalloc(ctypes.byref(_stack()), _vp(FAKE), 0, ids, 1 << 62, 1 << 40, _vp(FAKE),
+                                      None) == UNSUPPORTED
 
 
 def test_route_argument_errors():
@@ -155,6 +160,7 @@ def test_workspace_size_rejects_bad_descriptors():
     assert L.qmm_workspace_bytes(qmm.OP_GROUPED, None, 0, 8, 2) == 0
     assert L.qmm_workspace_bytes(qmm.OP_GROUPED, ctypes.byref(_stack()), 0, -1, 2) == 0
     assert L.qmm_workspace_bytes(qmm.OP_GROUPED, ctypes.byref(_stack()), 0, 8, 2) > 0
+    assert L.qmm_workspace_bytes(qmm.OP_GROUPED, ctypes.byref(_stack()), 0, 1 << 62, 1 << 40) == 0  # no overflow
 
 
 def _pw(fmt=2, n=64, k=256, experts=1, short=0, scales_short=0):

@@ -5,9 +5,10 @@ qmm_grouped_gemv_noalloc serves callers that cannot allocate device memory
 serving loop that must not block in the allocator) and therefore cannot pass
 the routing workspace that qmm_grouped_gemv takes.  Its routing scratch is a
 fixed array inside the library.  This file checks, through the C ABI, that
-two calls in a row give the same results as the workspace entry point, within
-the tolerance the other parity tests use, and that calls beyond the array's
-limit are refused.  It is collected last on purpose.
+two calls in a row give the oracle's results and the workspace entry point's,
+within the tolerance the other parity tests use, that further calls take no
+device memory, and that calls beyond the array's limit are refused.  It is
+collected last on purpose.
 """
 import numpy as np
 import pytest
@@ -28,7 +29,23 @@ def _case(seed, fmt, E, n, k, t, topk, per_pair):
     return p, x, ids
 
 
-def test_noalloc_matches_workspace_entry_point_on_two_calls():
+def _oracle_y(p, fmt, n, k, x_bits, ids_np, per_pair):
+    """The oracle's product for every (token, slot) and its tolerance scale
+    sum_k |w_k x_k|."""
+    t, topk = ids_np.shape
+    yref, absy = np.empty((t, topk, n)), np.empty((t, topk, n))
+    for tok in range(t):
+        for s in range(topk):
+            e = ids_np[tok, s]
+            de = p.data[e * p.data_stride:(e + 1) * p.data_stride]
+            se = None if p.scales is None else p.scales[e * p.scale_stride:(e + 1) * p.scale_stride]
+            xr = x_bits[tok, s][None] if per_pair else x_bits[tok][None]
+            yr, ar = oracle.matmul(fmt, n, k, de, se, p.global_scale, xr)
+            yref[tok, s], absy[tok, s] = yr[0], ar[0]
+    return yref, absy
+
+
+def test_noalloc_matches_oracle_and_workspace_entry_point_on_two_calls():
     # two different calls in a row: the second reuses the library's scratch
     # array after the first and must not see anything left over from it
     cases = [(71, synth.FMT_IQ4_NL, 8, 96, 256, 40, 4, False),
@@ -45,17 +62,29 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
         qmm.qmm_grouped_gemv_noalloc(w, x, ids, y_na, x_per_pair=per_pair)
         assert qmm.qmm_sync_check() == 0
         assert qmm.qmm_last_variant().startswith("noalloc:")
-        # tolerance scale sum_k |w_k x_k| of every output, from the oracle
-        absy = np.empty((t, topk, n))
-        for tok in range(t):
-            for s in range(topk):
-                e = ids_np[tok, s]
-                de = p.data[e * p.data_stride:(e + 1) * p.data_stride]
-                se = None if p.scales is None else p.scales[e * p.scale_stride:(e + 1) * p.scale_stride]
-                xr = x_bits[tok, s][None] if per_pair else x_bits[tok][None]
-                absy[tok, s] = oracle.matmul(fmt, n, k, de, se, p.global_scale, xr)[1][0]
-        a, b = f16(from_dev_u16(y_na)), f16(from_dev_u16(y_ws))
-        assert (np.abs(a - b) <= REL * absy + ABS).all()
+        yref, absy = _oracle_y(p, fmt, n, k, x_bits, ids_np, per_pair)
+        got = f16(from_dev_u16(y_na))
+        assert (np.abs(got - yref) <= REL * absy + ABS).all()            # against the oracle
+        assert (np.abs(got - f16(from_dev_u16(y_ws))) <= REL * absy + ABS).all()  # and the workspace call
+
+
+def test_noalloc_call_takes_no_device_memory():
+    """After a first call (which may load the kernels' code), further calls
+    leave the device's free memory unchanged."""
+    p, x_bits, ids_np = _case(73, synth.FMT_IQ4_NL, 8, 96, 256, 40, 4, False)
+    w = dev(p)
+    x = to_dev_u16(x_bits)
+    ids = torch.from_numpy(ids_np).cuda()
+    y = torch.zeros((40, 4, 96), dtype=torch.int16, device="cuda")
+    qmm.qmm_grouped_gemv_noalloc(w, x, ids, y)
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        qmm.qmm_grouped_gemv_noalloc(w, x, ids, y)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert qmm.qmm_sync_check() == 0
+    assert free1 == free0
 
 
 def test_noalloc_refuses_more_pairs_than_its_array_holds():
