@@ -347,6 +347,24 @@ size_t qmm_workspace_bytes(int32_t op, const qmm_weights* w, int64_t m, int64_t 
  * Returns QMM_OK, QMM_ERR_TIMEOUT, QMM_ERR_DEVICE_FAULT or QMM_ERR_CUDA. */
 qmm_status qmm_sync_check(void* stream);
 
+/* Test hooks for the failure path of the pipelined kernels (not needed in
+ * normal use; the pages have no counterpart).  Every mbarrier wait of the
+ * tensor-core GEMMs is bounded by a device-wide limit on %globaltimer; when
+ * a wait runs out, the kernel sets QMM_ERR_TIMEOUT in the error word, lets
+ * its own copies and MMAs finish, frees its tensor memory and returns, so
+ * the context stays usable.  These hooks let a test exercise that path
+ * without faulting anything:
+ *   QMM_DEBUG_WAIT_LIMIT_NS     value = the limit in ns (1e3 .. 1e10;
+ *                               2e9 by default)
+ *   QMM_DEBUG_WITHHOLD_X_TILES  value = 1: the GEMMs' activation loader
+ *                               issues no tile load, so their waits run out
+ *                               (nothing is written to y); 0: normal
+ * Both are device-wide (current device), copied synchronously, and stay set
+ * until changed.  Errors: INVALID_ARG (unknown hook or value), NOT_SM100,
+ * CUDA. */
+enum { QMM_DEBUG_WAIT_LIMIT_NS = 1, QMM_DEBUG_WITHHOLD_X_TILES = 2 };
+qmm_status qmm_debug_set(int32_t what, int64_t value);
+
 /* Static text for a status code. */
 const char* qmm_status_string(int32_t status);
 

@@ -213,7 +213,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       prefetch_tmap(&tm_x);
       int issued = 0;
-      for (int ks = 0; ks < ksteps; ks++) {
+      const int kissue = (g_test_flags & kTestWithholdXTiles) ? 0 : ksteps;  // test switch: issue nothing
+      for (int ks = 0; ks < kissue; ks++) {
         const int s = ks % STAGES;
         const uint32_t ph = (uint32_t)(ks / STAGES) & 1u;
         if (s_abort || !mbar_wait(bars + 8 * (STAGES + s), ph ^ 1u)) { s_abort = 1; break; }
@@ -449,7 +450,8 @@ __global__ void __launch_bounds__(kGemmPThreads, 1)
     if (lane == 0) {
       prefetch_tmap(&tm_x);
       int gs = 0, issued = 0;
-      for (int li = 0; li < my_tiles && !s_abort; li++) {
+      const int tissue = (g_test_flags & kTestWithholdXTiles) ? 0 : my_tiles;  // test switch: issue nothing
+      for (int li = 0; li < tissue && !s_abort; li++) {
         const int tile = (int)blockIdx.x + li * G;
         const int m0 = (tile / n_tiles) * kBM;
         for (int ks = 0; ks < ksteps; ks++, gs++) {

@@ -15,8 +15,17 @@ enum : unsigned { ERR_TIMEOUT = 1u, ERR_BAD_EXPERT = 2u };
 // One word per device that loads the library.
 __device__ unsigned int g_err_word;
 
-// A pipeline wait gives up after this many nanoseconds of %globaltimer.
+// A pipeline wait gives up after this many nanoseconds of %globaltimer
+// (2 s; a test may lower it through qmm_debug_set).
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+__device__ unsigned long long g_wait_limit_ns = kWaitLimitNs;
+
+// Test switches (qmm_debug_set), 0 in normal use.  kTestWithholdXTiles: the
+// tensor-core GEMMs' activation loader issues no tile load, so the MMA
+// issuer's wait for the first stage runs out and the kernel takes its
+// timeout path (raise the error word, drain, free tensor memory, return).
+enum : unsigned { kTestWithholdXTiles = 1u };
+__device__ unsigned int g_test_flags;
 
 __device__ __forceinline__ void raise_error(unsigned bits) { atomicOr(&g_err_word, bits); }
 
@@ -221,13 +230,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity has completed.  Gives up after
-// kWaitLimitNs, raises ERR_TIMEOUT and returns false.
+// g_wait_limit_ns, raises ERR_TIMEOUT and returns false.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
+  const unsigned long long limit = *(volatile unsigned long long*)&g_wait_limit_ns;
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit) {
       raise_error(ERR_TIMEOUT);
       return false;
     }

@@ -1111,6 +1111,23 @@ qmm_status qmm_moe_routed(const qmm_weights* gate, const qmm_weights* up, const 
   return launch_status();
 }
 
+qmm_status qmm_debug_set(int32_t what, int64_t value) {
+  DevInfo* di = nullptr;
+  qmm_status s = device_info(&di);
+  if (s != QMM_OK) return s;
+  if (what == QMM_DEBUG_WAIT_LIMIT_NS) {
+    if (value < 1000 || value > 10000000000ll) return QMM_ERR_INVALID_ARG;
+    const unsigned long long v = (unsigned long long)value;
+    return cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v)) == cudaSuccess ? QMM_OK : QMM_ERR_CUDA;
+  }
+  if (what == QMM_DEBUG_WITHHOLD_X_TILES) {
+    if (value != 0 && value != 1) return QMM_ERR_INVALID_ARG;
+    const unsigned int v = value ? kTestWithholdXTiles : 0u;
+    return cudaMemcpyToSymbol(g_test_flags, &v, sizeof(v)) == cudaSuccess ? QMM_OK : QMM_ERR_CUDA;
+  }
+  return QMM_ERR_INVALID_ARG;
+}
+
 qmm_status qmm_sync_check(void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return QMM_ERR_CUDA;

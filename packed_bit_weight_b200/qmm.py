@@ -71,6 +71,7 @@ def _lib():
             "qmm_moe_routed": (i32, [W, W, W, vp, vp, vp, i64, i64, vp, vp, sz, vp]),
             "qmm_workspace_bytes": (sz, [i32, W, i64, i64, i64]),
             "qmm_sync_check": (i32, [vp]),
+            "qmm_debug_set": (i32, [i32, i64]),
             "qmm_status_string": (ctypes.c_char_p, [i32]),
             "qmm_last_variant": (ctypes.c_char_p, []),
             "qmm_version": (ctypes.c_char_p, []),
@@ -365,6 +366,15 @@ def qmm_moe_routed(gate: PackedWeights, up: PackedWeights, down: PackedWeights, 
                                  _ptr(topk_ids, 4, "topk_ids"), _ptr(topk_weights, 4, "topk_weights"), t, topk,
                                  _ptr(out, 2, "out"), wp, wb, _stream(stream)), "qmm_moe_routed")
     return out
+
+
+DEBUG_WAIT_LIMIT_NS = 1
+DEBUG_WITHHOLD_X_TILES = 2
+
+
+def qmm_debug_set(what: int, value: int) -> None:
+    """Test hooks of the bounded pipeline waits (include/qmm.h)."""
+    _check(_lib().qmm_debug_set(int(what), int(value)), "qmm_debug_set")
 
 
 def qmm_sync_check(stream=None) -> int:
