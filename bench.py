@@ -394,6 +394,68 @@ def cpu_oracle_gemm(budget_s=10.0, rows=256, tokens=64):
                       % (rows, p.n, tokens, x.shape[0], p.k, reps, dt), "cpu": host_cpu()}
 
 
+def cpu_oracle_configs(budget_s=2.5):
+    """The oracle as it stands, one host thread, on every other workload of
+    the path: each timed by repeating one bounded call until about budget_s
+    has passed (at least once).  GEMV rows count packed weight bytes per
+    second; the routed experts count the bytes of the experts their sample
+    hits (the GPU metric's definition; the oracle itself multiplies pair by
+    pair)."""
+    import oracle
+    from packed_bit_weight_b200 import synth
+    cpu = host_cpu()
+
+    def timed(fn):
+        t0, reps = time.perf_counter(), 0
+        while True:
+            fn()
+            reps += 1
+            if time.perf_counter() - t0 >= budget_s:
+                return reps, time.perf_counter() - t0
+
+    def rows_of(p, rows):
+        return type(p)(p.fmt, rows, p.k, p.data[: oracle.data_bytes(p.fmt, rows, p.k)],
+                       None if p.scales is None else p.scales[: oracle.scale_bytes(p.fmt, rows, p.k)],
+                       p.global_scale)
+
+    out = {}
+    p, x = synth.make_gemv(synth.IQ4_TINY)
+    reps, dt = timed(lambda: oracle.matmul(p.fmt, p.n, p.k, p.data, None, 1.0, x))
+    out["iq4nl_gemv_tiny_256x512_m1"] = {
+        "value": p.nbytes * reps / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+        "sample": "the whole 256 x 512 matrix, m = 1, x %d reps (%.1f s, one thread)" % (reps, dt), "cpu": cpu}
+    for name, (p, xall) in synth.make_sweep().items():
+        sub = p if name == "out_proj" else rows_of(p, 1024)
+        for m in (1, 4, 16):
+            xs = np.ascontiguousarray(xall[:m])
+            reps, dt = timed(lambda: oracle.matmul(sub.fmt, sub.n, sub.k, sub.data, sub.scales, sub.global_scale, xs))
+            out["fp4g16_gemv_%s_m%d" % (name, m)] = {
+                "value": sub.nbytes * reps / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                "sample": "%s, m = %d, x %d reps (%.1f s, one thread)" % (
+                    "the whole %d x %d matrix" % (p.n, p.k) if sub is p else "rows 0..%d of %d" % (sub.n - 1, p.n),
+                    m, reps, dt), "cpu": cpu}
+    wgu, wdn, x_gu, x_dn, ids = synth.make_experts()
+    tt = 4  # tokens of the sample
+    ids_s = np.ascontiguousarray(ids[:tt])
+    xg = np.ascontiguousarray(x_gu[:tt])
+    xd = np.ascontiguousarray(x_dn[:tt].reshape(tt * ids.shape[1], -1))
+    ids_d = np.ascontiguousarray(ids_s.reshape(-1, 1))
+
+    def experts():
+        oracle.grouped_gemv(wgu.fmt, wgu.n, wgu.k, wgu.data, wgu.data_stride, None, 0, 1.0, wgu.experts, xg, ids_s)
+        oracle.grouped_gemv(wdn.fmt, wdn.n, wdn.k, wdn.data, wdn.data_stride, None, 0, 1.0, wdn.experts, xd, ids_d)
+
+    reps, dt = timed(experts)
+    hit = len(set(ids_s.reshape(-1).tolist()))
+    hit_bytes = hit * (wgu.data_stride + wdn.data_stride)
+    out["iq4nl_grouped_experts_t64_top4"] = {
+        "value": hit_bytes * reps / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+        "pairs_per_s": tt * ids.shape[1] * reps / dt,
+        "sample": "tokens 0..%d of 64 (%d pairs, %d experts hit), gate+up then down, x %d reps (%.1f s, one thread)"
+                  % (tt - 1, tt * ids.shape[1], hit, reps, dt), "cpu": cpu}
+    return out
+
+
 def oracle_steps(p, x_bits, steps, warmup, total_s):
     """The reference arm: `warmup` untimed and `steps` timed steps of the
     oracle on one host thread, each step one block of consecutive weight rows
@@ -821,6 +883,7 @@ def main():
         if world == 1:
             line["cpu_baseline_all_cores"] = cpu_oracle_gemv_all_cores(p, x, budget_s=args.cpu_budget)
             line["cpu_baseline_gemm"] = cpu_oracle_gemm(budget_s=args.cpu_budget)
+            line["cpu_baselines"] = cpu_oracle_configs(budget_s=args.cpu_budget / 4)
         print(json.dumps(line))
     if world > 1:
         import torch.distributed as dist
