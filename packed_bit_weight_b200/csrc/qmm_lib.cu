@@ -283,26 +283,54 @@ static qmm_status launch_gemv_splitk(const qmm_weights* w, const uint16_t* x, in
   return launch_status();
 }
 
-// Clusters per tile for a narrow matrix: the smallest power of two (2..8)
-// that gives at least four CTAs per SM, with whole 4-warp CTAs of 1..8
-// segments per warp (1..4 at m > 8); 0 = no split (wide enough, or k does
-// not divide).  QMM_GEMV_SPLITK=<cs> forces cs (0 turns split-K off).
-static int splitk_clusters(int64_t n, int64_t k, int m, int sms) {
-  const int64_t tiles = (n + 15) / 16, segs = k / 128;
+// Clusters per tile (0 = no split), from a sweep on B200 (per-launch time,
+// n x k at m = 1: 256 x 4096 3.35 -> 2.47 us at cs = 4, 256 x 8192 3.86 ->
+// 2.74 at cs = 8, 1024 x 4096 3.62 -> 3.12 at cs = 4, 2048 x 4096 4.36 ->
+// 3.33 at cs = 2; 4096 x 8192 (out_proj) 5.25 unsplit, 6.4-11.8 split).  At
+// m <= 8 a matrix of at most 64 tiles takes cs = 256 / tiles rounded down to
+// a power of two, at most 8 and at most k / 1024 (two or more segments per
+// warp); 65..128 tiles with k <= 4096 take cs = 2.  At m > 8 the split lost
+// everywhere the unsplit kernel has a configuration, so it serves only the
+// shapes that kernel does not take (k = 16384 at m = 16: 646 -> 3.9 us,
+// instead of the generic kernel).  Each choice needs whole 4-warp CTAs of
+// 1..8 segments per warp (1..4 at m > 8).  QMM_GEMV_SPLITK=<cs> forces a
+// count (0 turns split-K off); a count the shape does not divide is ignored.
+static bool splitk_fits(int64_t k, int m, int cs) {
+  const int64_t segs = k / 128;
   const int max_spw = m > 8 ? 4 : 8;
-  auto ok = [&](int cs) {
-    return k % 128 == 0 && segs % (4 * cs) == 0 && segs / (4 * cs) >= 1 && segs / (4 * cs) <= max_spw;
-  };
+  return k % 128 == 0 && segs % (4 * cs) == 0 && segs / (4 * cs) >= 1 && segs / (4 * cs) <= max_spw &&
+         (segs / (4 * cs)) != 3 && (segs / (4 * cs)) != 5 && (segs / (4 * cs)) != 6 && (segs / (4 * cs)) != 7;
+}
+static int splitk_clusters(int64_t n, int64_t k, int m, bool unsplit_ok) {
+  const int64_t tiles = (n + 15) / 16;
   if (const char* e = getenv("QMM_GEMV_SPLITK")) {
     const int cs = atoi(e);
-    return (cs == 2 || cs == 4 || cs == 8) && ok(cs) ? cs : 0;
+    return (cs == 2 || cs == 4 || cs == 8) && splitk_fits(k, m, cs) ? cs : 0;
   }
-  if (tiles >= 2 * (int64_t)sms) return 0;
-  for (int cs = 2; cs <= 8; cs *= 2)
-    if (ok(cs) && tiles * cs >= 4 * (int64_t)sms) return cs;
-  for (int cs = 8; cs >= 2; cs /= 2)
-    if (ok(cs)) return cs;
-  return 0;
+  if (!unsplit_ok) {  // the shape has no unsplit configuration: any count that fits
+    for (int cs = 2; cs <= 8; cs *= 2)
+      if (splitk_fits(k, m, cs)) return cs;
+    return 0;
+  }
+  if (m > 8) return 0;
+  int cs = 0;
+  if (tiles <= 64) {
+    for (int c = 8; c >= 2 && !cs; c /= 2)
+      if (tiles * c <= 256 && k / 1024 >= c && splitk_fits(k, m, c)) cs = c;
+  } else if (tiles <= 128 && k <= 4096 && splitk_fits(k, m, 2)) {
+    cs = 2;
+  }
+  return cs;
+}
+
+// Whether gemv_ldg_auto has a configuration for this k and batch (its cases).
+static bool ldg_config_exists(int64_t k, int m) {
+  if (k % 128) return false;
+  const int64_t segs = k / 128;
+  if (m <= 8)
+    return (segs % 4 == 0 && segs / 4 >= 1 && segs / 4 <= 8) || (segs % 8 == 0 && segs / 8 >= 5 && segs / 8 <= 8) ||
+           (segs % 16 == 0 && segs / 16 >= 5 && segs / 16 <= 8);
+  return (segs % 8 == 0 && segs / 8 >= 1 && segs / 8 <= 4) || (segs % 16 == 0 && segs / 16 >= 3 && segs / 16 <= 4);
 }
 
 template <int FMT, int NT>
@@ -353,7 +381,7 @@ static qmm_status gemv_fmt(const qmm_weights* w, const uint16_t* x, int m, uint1
   const int pick = gemv_variant_env();
   if constexpr (FMT != 1) {  // the register kernels decode E2M1 codes only
     if (pick == PICK_DEFAULT) {
-      const int cs = splitk_clusters(n, k, m, di->sms);
+      const int cs = splitk_clusters(n, k, m, ldg_config_exists(k, m));
       if (cs) {
         const qmm_status s = (m <= 8) ? gemv_splitk_auto<FMT, 1>(w, x, m, y, st, cs)
                                       : gemv_splitk_auto<FMT, 2>(w, x, m, y, st, cs);

@@ -65,3 +65,56 @@ def run_gemv(w: qmm.PackedWeights, x_bits: np.ndarray, canary: int = 64) -> np.n
     tail = yb[m * w.n:].cpu()
     assert bool((tail == 0x5A5A).all()), "write past the end of y"
     return from_dev_u16(y)
+
+
+def oracle_matmul_rows(fmt, n, k, data, scales, global_scale, x_bits, threads=None):
+    """oracle.matmul over row blocks on several host threads (each ctypes call
+    releases the interpreter lock): the same per-row definition, for full
+    outputs of the large matrices.  Returns (y, absy), [m][n]."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+    threads = threads or max(1, len(os.sched_getaffinity(0)))
+    db, sb = oracle.data_bytes(fmt, 1, k), oracle.scale_bytes(fmt, 1, k)
+    cuts = np.linspace(0, n, threads + 1).astype(np.int64)
+
+    def part(i):
+        r0, r1 = int(cuts[i]), int(cuts[i + 1])
+        if r1 <= r0:
+            return r0, None, None
+        sc = None if scales is None else scales[r0 * sb:r1 * sb]
+        y, a = oracle.matmul(fmt, r1 - r0, k, data[r0 * db:r1 * db], sc, global_scale, x_bits)
+        return r0, y, a
+
+    m = x_bits.shape[0]
+    y, a = np.empty((m, n)), np.empty((m, n))
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        for r0, yy, aa in ex.map(part, range(threads)):
+            if yy is not None:
+                y[:, r0:r0 + yy.shape[1]], a[:, r0:r0 + aa.shape[1]] = yy, aa
+    return y, a
+
+
+def oracle_grouped_full(w, x_bits, ids, per_pair, threads=None):
+    """The oracle's grouped product for every (token, slot, row), over
+    tokens on several host threads.  Returns (y, absy), [t][topk][n]."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+    threads = threads or max(1, len(os.sched_getaffinity(0)))
+    t, topk = ids.shape
+
+    def one(tok):
+        if per_pair:   # one activation row per pair: pairs as tokens of one slot
+            xs = np.ascontiguousarray(x_bits[tok])
+            ii = np.ascontiguousarray(ids[tok].reshape(topk, 1))
+        else:
+            xs = np.ascontiguousarray(x_bits[tok][None])
+            ii = np.ascontiguousarray(ids[tok][None])
+        yy, aa = oracle.grouped_gemv(w.fmt, w.n, w.k, w.data, w.data_stride, w.scales,
+                                     0 if w.scales is None else w.scale_stride, w.global_scale, w.experts, xs, ii)
+        return tok, yy.reshape(topk, w.n), aa.reshape(topk, w.n)
+
+    y, a = np.empty((t, topk, w.n)), np.empty((t, topk, w.n))
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        for tok, yy, aa in ex.map(one, range(t)):
+            y[tok], a[tok] = yy, aa
+    return y, a

@@ -148,6 +148,20 @@ def test_config3_sweep(m):
         del w
 
 
+@pytest.mark.parametrize("m", [1, 16])
+def test_lm_head_full_output(m):
+    """The whole 256000 x 4096 LM head output at m = 1 and 16 against the
+    oracle, element by element (the oracle over row blocks on the host's
+    cores)."""
+    from gpu_util import oracle_matmul_rows
+    mats = synth.make_sweep(mats=[("lm_head", 256000, 4096)])
+    p, xall = mats["lm_head"]
+    x = np.ascontiguousarray(xall[:m])
+    y = run_gemv(dev(p), x)
+    yref, absy = oracle_matmul_rows(p.fmt, p.n, p.k, p.data, p.scales, p.global_scale, x)
+    check_tol(y, yref, absy, "lm_head m=%d %s" % (m, qmm.qmm_last_variant()))
+
+
 def test_gemv_edge_cases():
     p, x = _case(synth.FMT_FP4G16_F16, 64, 256, 2, 3)
     w = dev(p)
@@ -335,24 +349,27 @@ def test_split_k_clusters_vs_oracle(fmt, n, k, m, cs, monkeypatch):
     assert np.array_equal(run_gemv(w, x), y)
 
 
-@pytest.mark.parametrize("m", [1, 4, 16])
-def test_out_proj_takes_split_k_by_default(m):
-    """The 4096 x 8192 out_proj (256 tiles) is split across clusters; the full
-    output matches the oracle."""
-    mats = synth.make_sweep(mats=[("out_proj", 4096, 8192)])
-    p, xall = mats["out_proj"]
-    y = run_gemv(dev(p), xall[:m])
+@pytest.mark.parametrize("n,k,m,split", [(256, 8192, 1, True), (1000, 4096, 3, True), (2000, 4096, 1, True),
+                                         (4096, 8192, 1, False), (4096, 8192, 16, False), (256, 4096, 16, False),
+                                         (128, 16384, 16, True), (64, 32768, 2, True)])
+def test_split_k_default_dispatch(n, k, m, split):
+    """Narrow matrices at m <= 8 take split-K by default, out_proj (256
+    tiles) and m > 8 do not, except where the unsplit kernel has no
+    configuration for k (k = 16384 at m = 16, k = 32768)."""
+    p, x = _case(synth.FMT_FP4G16_F16, n, k, m, 8500 + n + k + m)
+    y = run_gemv(dev(p), x)
     v = qmm.qmm_last_variant()
-    assert v.startswith("gemv_fp4_splitk"), v
-    yref, absy = oracle.matmul(p.fmt, p.n, p.k, p.data, p.scales, p.global_scale, xall[:m])
+    assert v.startswith("gemv_fp4_splitk" if split else "gemv_fp4_ldg"), v
+    yref, absy = oracle.matmul(p.fmt, n, k, p.data, p.scales, p.global_scale, x)
     check_tol(y, yref, absy, v)
 
 
 @pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_MXFP4])
 @pytest.mark.parametrize("m", [1, 12])
-def test_split_k_with_16_byte_aligned_activations(fmt, m):
+def test_split_k_with_16_byte_aligned_activations(fmt, m, monkeypatch):
     """x 16- but not 32-byte aligned: the split-K kernel takes the 128-bit
     activation loads (xw=0)."""
+    monkeypatch.setenv("QMM_GEMV_SPLITK", "4")
     n, k = 200, 4096
     p, xb = _case(fmt, n, k, m, 9100 + m + fmt)
     w = dev(p)

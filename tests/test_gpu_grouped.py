@@ -96,6 +96,19 @@ def test_config4_experts_sampled():
                 check_tol(y[tok, s, rows], ys, as_, "config4")
 
 
+def test_config4_experts_full_output():
+    """Every (token, slot, row) of the routed-expert workload (32 experts,
+    gate+up 1792 x 2560 and down 2560 x 896, 64 tokens top-4) against the
+    oracle element by element."""
+    from gpu_util import oracle_grouped_full
+    wgu, wdn, x_gu, x_dn, ids = synth.make_experts()
+    for w, x, per_pair in ((wgu, x_gu, False), (wdn, x_dn, True)):
+        y, st = _grouped(dev(w), x, ids, per_pair)
+        assert st == 0
+        yref, absy = oracle_grouped_full(w, x, ids, per_pair)
+        check_tol(y, yref, absy, "config4 full %s" % qmm.qmm_last_variant())
+
+
 def test_grouped_rejects_small_workspace():
     rng = np.random.default_rng(2)
     p = synth.gen_iq4nl(rng, 32, 64, experts=4)
