@@ -119,11 +119,6 @@ __device__ __forceinline__ void cp_commit_g() { asm volatile("cp.async.commit_gr
 __device__ __forceinline__ void cp_wait_g(int) {
   asm volatile("cp.async.wait_group %0;" ::"n"(kGemmPSlots - 1) : "memory");
 }
-__device__ __forceinline__ uint2 lds64(uint32_t addr) {
-  uint2 v;
-  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
-  return v;
-}
 
 // Copy the packed codes (32 bytes) and scales (8 or 4 bytes) of weight row
 // `row` for the k step starting at k0 into this thread's ring slot.  Rows

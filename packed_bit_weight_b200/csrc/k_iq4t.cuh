@@ -159,6 +159,39 @@ __device__ __forceinline__ void iqt_window(uint32_t (&win)[6], const uint8_t* ro
   }
 }
 
+// The same 24-byte window read from the CTA's shared-memory copy of the tile
+// (row = shared address of the row; rows 16-byte aligned when W16, so the
+// window's alignment is the global one).
+template <bool W16>
+__device__ __forceinline__ void iqt_window_smem(uint32_t (&win)[6], uint32_t row, int blk, int s) {
+  const uint32_t p = row + ((uint32_t)(blk * 18) & ~7u);
+  if (W16 && !(s & 1)) {
+    const uint4 a = lds128(p);
+    const uint2 b = lds64(p + 16);
+    win[0] = a.x; win[1] = a.y; win[2] = a.z; win[3] = a.w; win[4] = b.x; win[5] = b.y;
+  } else if (W16) {
+    const uint2 a = lds64(p);
+    const uint4 b = lds128(p + 8);
+    win[0] = a.x; win[1] = a.y; win[2] = b.x; win[3] = b.y; win[4] = b.z; win[5] = b.w;
+  } else {
+    const uint2 a = lds64(p), b = lds64(p + 8), c = lds64(p + 16);
+    win[0] = a.x; win[1] = a.y; win[2] = b.x; win[3] = b.y; win[4] = c.x; win[5] = c.y;
+  }
+}
+
+template <int S, int SPW, bool W16>
+__device__ __forceinline__ void iqt_load_smem(uint32_t (&w)[SPW][S][2][6], const uint32_t (&rs)[S][2], int s0,
+                                              int tig) {
+#pragma unroll
+  for (int u = 0; u < SPW; u++) {
+    const int blk = 4 * (s0 + u) + tig;
+#pragma unroll
+    for (int s = 0; s < S; s++)
+#pragma unroll
+      for (int r = 0; r < 2; r++) iqt_window_smem<W16>(w[u][s][r], rs[s][r], blk, s0 + u);
+  }
+}
+
 template <int S, int SPW, bool W16>
 __device__ __forceinline__ void iqt_load(uint32_t (&w)[SPW][S][2][6], const uint8_t* const (&rp)[S][2], int s0,
                                          int tig) {
@@ -200,10 +233,20 @@ __device__ __forceinline__ int iqt_collect_pairs(const IqtArgs& a, int e, int* s
   return *s_cnt;
 }
 
-template <int MODE, int S, int SPW, int MAXREG, bool W16>
+// STG: the item's tiles (16 rows of each source, one contiguous byte range
+// each) are brought into shared memory by the copy engine (one bulk copy per
+// source, completing on an mbarrier) instead of each lane loading its
+// windows from global memory: a warp's window loads from global memory touch
+// eight rows' lines each and were the largest share of the L1 data-pipe
+// wavefronts; from shared memory a 16-byte window load of eight rows costs
+// the minimum four.  The copies are issued when the global loads would have
+// been (before the dependency wait when speculative), and every exit waits
+// for them, so no copy is in flight when the CTA leaves.
+template <int MODE, int S, int SPW, int MAXREG, bool W16, bool STG = false>
 __global__ void __launch_bounds__(iqt_max_threads(MAXREG)) __maxnreg__(MAXREG) iq4_tile_kernel(const IqtArgs a) {
   __shared__ int s_pairs[kIqtMaxPairs];
   __shared__ int s_cnt;
+  __shared__ __align__(8) unsigned long long s_wbar;
   static_assert(MODE != IQ_SWIGLU || S % 2 == 0, "SwiGLU items are gate and up tiles of the same rows");
   constexpr int kOut = (MODE == IQ_SWIGLU) ? S / 2 : S;  // output tiles per item
   extern __shared__ __align__(16) uint8_t smem_iqt[];
@@ -212,6 +255,37 @@ __global__ void __launch_bounds__(iqt_max_threads(MAXREG)) __maxnreg__(MAXREG) i
   const int wpc = blockDim.x >> 5;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, grp = lane >> 2, tig = lane & 3;
   const int e = blockIdx.x / a.items_per_expert, item = blockIdx.x - e * a.items_per_expert;
+  const int64_t rowb = (int64_t)(a.k >> 5) * 18;
+  // STG: shared-memory copy of the sources after the table and the partial
+  // sums; source s holds its 16 rows contiguously (rows past n hold stale
+  // bytes: their outputs are never stored)
+  const uint32_t stage = lut + (uint32_t)kIqLutBytes + (uint32_t)wpc * S * kIqtGroup * 16u * 4u;
+  const uint32_t wbar = smem_addr(&s_wbar);
+  auto issue_copies = [&]() {  // thread 0
+    uint32_t bytes[S];
+    uint32_t total = 0;
+#pragma unroll
+    for (int s = 0; s < S; s++) {
+      const int r0 = (MODE == IQ_SWIGLU) ? (item * kOut + (s >> 1)) * 16 : (item * S + s) * 16;
+      const int rows = max(0, min(16, a.n - r0));
+      bytes[s] = (uint32_t)(rows * rowb);
+      total += bytes[s];
+    }
+    mbar_arrive_expect_tx(wbar, total);
+#pragma unroll
+    for (int s = 0; s < S; s++) {
+      if (!bytes[s]) continue;
+      const int r0 = (MODE == IQ_SWIGLU) ? (item * kOut + (s >> 1)) * 16 : (item * S + s) * 16;
+      const uint8_t* base = (MODE == IQ_SWIGLU && (s & 1)) ? a.data1 + (int64_t)e * a.dstride1
+                                                            : a.data0 + (int64_t)e * a.dstride0;
+      bulk_load(stage + (uint32_t)s * 16u * (uint32_t)rowb, base + (int64_t)r0 * rowb, bytes[s], wbar);
+    }
+  };
+  if (STG && threadIdx.x == 0) {
+    mbar_init(wbar, 1);
+    fence_mbar_init();
+    if (a.spec) issue_copies();
+  }
   pdl_launch_dependents();
   int start = 0, cnt = a.m_plain;
   if (!a.spec) {  // most experts may be empty: find out before any other work
@@ -223,6 +297,7 @@ __global__ void __launch_bounds__(iqt_max_threads(MAXREG)) __maxnreg__(MAXREG) i
       cnt = a.offsets[e + 1] - start;
     }
     if (cnt <= 0) return;
+    if (STG && threadIdx.x == 0) issue_copies();
   }
   // pair table: entry v (an index byte) = (kv[v & 15], kv[v >> 4]) as f16x2,
   // one copy per bank; each store covers four banks
@@ -237,7 +312,6 @@ __global__ void __launch_bounds__(iqt_max_threads(MAXREG)) __maxnreg__(MAXREG) i
   // re-reads the last row and stores nothing)
   int row0[S];
   const uint8_t* rp[S][2];
-  const int64_t rowb = (int64_t)(a.k >> 5) * 18;
 #pragma unroll
   for (int s = 0; s < S; s++) {
     const uint8_t* base;
@@ -254,7 +328,7 @@ __global__ void __launch_bounds__(iqt_max_threads(MAXREG)) __maxnreg__(MAXREG) i
   const int s0 = warp * SPW;
   uint32_t w[SPW][S][2][6];
   if (a.spec) {
-    iqt_load<S, SPW, W16>(w, rp, s0, tig);
+    if (!STG) iqt_load<S, SPW, W16>(w, rp, s0, tig);
     pdl_wait();  // routing, activations and the output buffer follow the previous kernel
     if (a.ids) {
       cnt = iqt_collect_pairs(a, e, s_pairs, &s_cnt);
@@ -262,11 +336,29 @@ __global__ void __launch_bounds__(iqt_max_threads(MAXREG)) __maxnreg__(MAXREG) i
       start = a.offsets[e];
       cnt = a.offsets[e + 1] - start;
     }
-    if (cnt <= 0) return;  // the whole CTA: an expert without pairs
-  } else {
+    if (cnt <= 0) {  // the whole CTA (cnt is the same in every thread): an expert without pairs
+      if (STG) {       // let our copies land before leaving
+        __syncthreads();  // (the barrier's initialisation is visible to every thread)
+        mbar_wait(wbar, 0);
+      }
+      return;
+    }
+  } else if (!STG) {
     iqt_load<S, SPW, W16>(w, rp, s0, tig);
   }
   __syncthreads();  // the pair table is complete
+  if (STG) {
+    // the copies have landed (a wait that runs out raises the error word; the
+    // CTA still waits, bounded again, before it reads or leaves)
+    if (!mbar_wait(wbar, 0)) mbar_wait(wbar, 0);
+    uint32_t rs[S][2];
+#pragma unroll
+    for (int s = 0; s < S; s++) {
+      rs[s][0] = stage + (uint32_t)(s * 16 + grp) * (uint32_t)rowb;
+      rs[s][1] = rs[s][0] + 8u * (uint32_t)rowb;
+    }
+    iqt_load_smem<S, SPW, W16>(w, rs, s0, tig);
+  }
   const uint32_t lut_lane = lut + 4u * lane;
 
   for (int g0 = 0; g0 < cnt; g0 += kIqtGroup) {

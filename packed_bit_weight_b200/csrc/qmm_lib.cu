@@ -28,11 +28,19 @@ namespace qmm {
 static thread_local char t_variant[160] = "";
 
 static void set_variant(const char* fmt, ...) __attribute__((format(printf, 1, 2)));
+static void prefix_variant(const char* prefix);
 static void set_variant(const char* fmt, ...) {
   va_list ap;
   va_start(ap, fmt);
   vsnprintf(t_variant, sizeof(t_variant), fmt, ap);
   va_end(ap);
+}
+
+// Record the dispatch path in front of the kernel variant just recorded.
+static void prefix_variant(const char* prefix) {
+  char kern[sizeof(t_variant)];
+  snprintf(kern, sizeof(kern), "%s", t_variant);
+  snprintf(t_variant, sizeof(t_variant), "%s%s", prefix, kern);
 }
 
 struct DevInfo {
@@ -526,7 +534,7 @@ static qmm_status launch_iq4_mode(const qmm_weights* w, const qmm_weights* w2, c
 // dependency wait when most experts are expected to have pairs (P >= 4E:
 // fewer than 2 % of the experts empty for uniform routing) or for the plain
 // product; QMM_IQ4T_SPEC=0/1 forces either (measurement knob).
-template <int MODE, int S, int SPW, int kMaxReg, bool W16>
+template <int MODE, int S, int SPW, int kMaxReg, bool W16, bool STG = false>
 static qmm_status launch_iq4_tile_cfg(const qmm_weights* w0, const qmm_weights* w1, const uint16_t* x, int x_per_pair,
                                       int64_t topk, const int32_t* offsets, const int32_t* perm, int64_t P,
                                       int m_plain, void* y, const float* gw, cudaStream_t st, const int32_t* ids) {
@@ -539,8 +547,8 @@ static qmm_status launch_iq4_tile_cfg(const qmm_weights* w0, const qmm_weights* 
   const int64_t grid = E * ipe;
   if (ids && P > kIqtMaxPairs) return QMM_ERR_UNSUPPORTED_SHAPE;
   if (grid < 1 || grid > INT32_MAX) return QMM_ERR_UNSUPPORTED_SHAPE;
-  auto kern = iq4_tile_kernel<MODE, S, SPW, kMaxReg, W16>;
-  const uint32_t smem = iqt_smem_bytes(S, wpc);
+  auto kern = iq4_tile_kernel<MODE, S, SPW, kMaxReg, W16, STG>;
+  const uint32_t smem = iqt_smem_bytes(S, wpc) + (STG ? (uint32_t)S * 16u * (uint32_t)(w0->k / 32 * 18) : 0u);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return QMM_ERR_CUDA;
   IqtArgs a;
@@ -575,8 +583,8 @@ static qmm_status launch_iq4_tile_cfg(const qmm_weights* w0, const qmm_weights* 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return QMM_ERR_CUDA;
-  set_variant("iq4_tile<mode=%d,s=%d,spw=%d,wpc=%d,w16=%d,spec=%d,route=%s,grid=%d>", MODE, S, SPW, wpc, W16 ? 1 : 0,
-              a.spec, ids ? "in_kernel" : "sorted", (int)grid);
+  set_variant("iq4_tile<mode=%d,s=%d,spw=%d,wpc=%d,w16=%d,stg=%d,spec=%d,route=%s,grid=%d>", MODE, S, SPW, wpc,
+              W16 ? 1 : 0, STG ? 1 : 0, a.spec, ids ? "in_kernel" : "sorted", (int)grid);
   return launch_status();
 }
 
@@ -597,12 +605,27 @@ static qmm_status launch_iq4_tile(const qmm_weights* w0, const qmm_weights* w1, 
   // CTAs of up to 10 warps per SM).  Otherwise four tiles, one super-step per
   // warp, 128 registers.  Four tiles at one super-step per warp for k = 2560
   // would need 20 warps of ~128 registers (more than an SM holds).
-  if (steps % 2 == 0 && steps / 2 <= iqt_max_threads(96) / 32)
+  // Shared-memory staging of the tiles (k_iq4t.cuh, STG) wherever every
+  // source tile is a whole number of 16-byte units (rows * 9k/16 bytes:
+  // whole tiles, an even k / 128, or an even number of rows in the last
+  // tile).  QMM_IQ4T_STAGE=0/1 forces it off / on where it fits.
+  const int64_t rem = n % 16;
+  bool stg = rem == 0 || (steps % 2 == 0) || (rem % 2 == 0);
+  if (const char* e = getenv("QMM_IQ4T_STAGE")) stg = stg && e[0] == '1';
+  if (steps % 2 == 0 && steps / 2 <= iqt_max_threads(96) / 32) {
+    if (stg)
+      return launch_iq4_tile_cfg<MODE, 2, 2, 96, true, true>(w0, w1, x, x_per_pair, topk, offsets, perm, P, m_plain, y,
+                                                             gw, st, ids);
     return launch_iq4_tile_cfg<MODE, 2, 2, 96, true>(w0, w1, x, x_per_pair, topk, offsets, perm, P, m_plain, y, gw,
                                                      st, ids);
-  if (steps <= iqt_max_threads(128) / 32)
+  }
+  if (steps <= iqt_max_threads(128) / 32) {
+    if (stg)
+      return launch_iq4_tile_cfg<MODE, 4, 1, 128, false, true>(w0, w1, x, x_per_pair, topk, offsets, perm, P, m_plain,
+                                                               y, gw, st, ids);
     return launch_iq4_tile_cfg<MODE, 4, 1, 128, false>(w0, w1, x, x_per_pair, topk, offsets, perm, P, m_plain, y, gw,
                                                        st, ids);
+  }
   return QMM_ERR_UNSUPPORTED_SHAPE;
 }
 
@@ -952,7 +975,7 @@ qmm_status qmm_grouped_gemv(const qmm_weights* experts, const uint16_t* x, int32
     s = launch_iq4_tile<IQ_OUT_F16>(experts, nullptr, x, x_per_pair, topk, nullptr, nullptr, P, 0, y, nullptr, st,
                                     topk_ids);
     if (s != QMM_ERR_UNSUPPORTED_SHAPE) {
-      set_variant("grouped_iq4_tile+in_kernel_route");
+      prefix_variant("grouped_iq4_tile+in_kernel_route:");
       return s;
     }
   }
@@ -969,7 +992,7 @@ qmm_status qmm_grouped_gemv(const qmm_weights* experts, const uint16_t* x, int32
   if (experts->fmt == QMM_FMT_IQ4_NL && iq4_tile) {  // more pairs: after the routing sort
     s = launch_iq4_tile<IQ_OUT_F16>(experts, nullptr, x, x_per_pair, topk, offsets, perm, P, 0, y, nullptr, st);
     if (s != QMM_ERR_UNSUPPORTED_SHAPE) {
-      set_variant("route+grouped_iq4_tile");
+      prefix_variant("route+grouped_iq4_tile:");
       return s;
     }
   }

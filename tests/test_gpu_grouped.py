@@ -157,21 +157,26 @@ def test_grouped_iq4_many_pairs_per_expert(variant, E, n, k, t, topk, per_pair, 
     check_tol(y, yref, absy, "grouped iq4 %s" % v)
 
 
+@pytest.mark.parametrize("stage", ["0", "1"])
 @pytest.mark.parametrize("spec", ["0", "1"])
 @pytest.mark.parametrize("E,n,k,t,topk,per_pair", [(32, 1792, 2560, 64, 4, False), (32, 2560, 896, 64, 4, True),
                                                     (32, 2560, 896, 1, 4, True), (7, 1000, 1152, 37, 3, False),
                                                     (4, 72, 4096, 20, 2, False), (2, 72, 4096, 16, 2, False),
-                                                    (3, 100, 896, 10, 3, True)])
-def test_grouped_iq4_tile_kernel(spec, E, n, k, t, topk, per_pair, monkeypatch):
+                                                    (3, 100, 896, 10, 3, True), (3, 99, 896, 10, 3, False),
+                                                    (5, 83, 2560, 12, 2, False)])
+def test_grouped_iq4_tile_kernel(stage, spec, E, n, k, t, topk, per_pair, monkeypatch):
     """The tile-resident IQ4_NL kernel with its weight loads before and after
-    the dependency wait, items of two tiles (two super-steps per warp, k %
-    256 == 0) or four (one super-step per warp: k = 896, 1152), ragged last
-    items (n = 1000, 72), the routed-expert shapes (gate+up 1792 x 2560, down
-    2560 x 896 at 64 and 1 tokens), and routing inside the kernel (at most 32
-    pairs; 16 tokens x 2 over 2 experts puts more than one token group on an
-    expert)."""
+    the dependency wait, its windows read from global memory or from the
+    tiles' shared-memory copy (stage; a last tile whose bytes are not whole
+    16-byte units, 99 rows at k = 896, stays on global loads), items of two
+    tiles (two super-steps per warp, k % 256 == 0) or four (one super-step
+    per warp: k = 896, 1152), ragged last items (n = 1000, 72, 99, 83), the
+    routed-expert shapes (gate+up 1792 x 2560, down 2560 x 896 at 64 and 1
+    tokens), and routing inside the kernel (at most 32 pairs; 16 tokens x 2
+    over 2 experts puts more than one token group on an expert)."""
     monkeypatch.setenv("QMM_GEMV_VARIANT", "iq4t")
     monkeypatch.setenv("QMM_IQ4T_SPEC", spec)
+    monkeypatch.setenv("QMM_IQ4T_STAGE", stage)
     rng = np.random.default_rng(E * 7 + n + k + t)
     p = synth.gen_weights(rng, synth.FMT_IQ4_NL, n, k, experts=E)
     x = synth.gen_x(rng, t, topk, k) if per_pair else synth.gen_x(rng, t, k)
@@ -179,6 +184,8 @@ def test_grouped_iq4_tile_kernel(spec, E, n, k, t, topk, per_pair, monkeypatch):
     y, st = _grouped(dev(p), x, ids, per_pair)
     v = qmm.qmm_last_variant()
     assert st == 0 and "grouped_iq4_tile" in v, v
+    fits = n % 16 == 0 or (k // 128) % 2 == 0 or (n % 16) % 2 == 0
+    assert ("stg=1" in v) == (stage == "1" and fits), v
     if per_pair:
         xs = x.reshape(t * topk, k)
         yref = np.empty((t * topk, n)); absy = np.empty((t * topk, n))
