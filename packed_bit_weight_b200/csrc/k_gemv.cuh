@@ -114,6 +114,25 @@ __global__ void __launch_bounds__(128) gemv_generic_kernel(const uint8_t* __rest
 // a CTA that starts while the previous kernel drains already streams its
 // weights; activations are read and y written only after the wait.
 // ---------------------------------------------------------------------------
+// The same streaming loads as volatile asm: kept after griddepcontrol.wait
+// when they are written after it (a plain asm load may be hoisted above).
+__device__ __forceinline__ uint4 ldg_stream128_after(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint32_t ldg_stream32_after(const void* p) {
+  uint32_t v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint32_t ldg_stream16_after(const void* p) {
+  unsigned short v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.u16 %0, [%1];" : "=h"(v) : "l"(p));
+  return v;
+}
 __device__ __forceinline__ uint4 ldg_stream128(const void* p) {
   uint4 v;
   asm("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -273,6 +292,43 @@ __device__ __forceinline__ void ldg_tile_store(float (&red)[WPC][16][16], const 
   }
 }
 
+// Segments [I0, I1) of ldg_tile_load, FP4-G16 scales (fp16 or E4M3), with
+// volatile loads (AFTER: issued after the dependency wait and kept there).
+template <int FMT, int SPW, int I0, int I1, bool AFTER>
+__device__ __forceinline__ void ldg_tile_load_part(uint4 (&qa)[SPW], uint4 (&qb)[SPW], uint32_t (&sa)[SPW],
+                                                   uint32_t (&sb)[SPW], const uint8_t* __restrict__ codes,
+                                                   const uint8_t* __restrict__ scales, int64_t ra, int64_t rb,
+                                                   bool va, bool vb, int seg0, int tig, int64_t crow, int64_t srow) {
+  static_assert(FMT == 2 || FMT == 3, "FP4-G16 scales");
+#pragma unroll
+  for (int i = I0; i < I1; i++) {
+    const int seg = seg0 + i;
+    const int64_t cb = (int64_t)seg * 64 + tig * 16;
+    const int64_t gi = (int64_t)seg * 8 + tig * 2;
+    if (AFTER) {
+      qa[i] = va ? ldg_stream128_after(codes + ra * crow + cb) : make_uint4(0, 0, 0, 0);
+      qb[i] = vb ? ldg_stream128_after(codes + rb * crow + cb) : make_uint4(0, 0, 0, 0);
+      if (FMT == 2) {
+        sa[i] = va ? ldg_stream32_after(scales + (ra * srow + gi) * 2) : 0u;
+        sb[i] = vb ? ldg_stream32_after(scales + (rb * srow + gi) * 2) : 0u;
+      } else {
+        sa[i] = va ? e4m3x2_to_f16x2(ldg_stream16_after(scales + ra * srow + gi)) : 0u;
+        sb[i] = vb ? e4m3x2_to_f16x2(ldg_stream16_after(scales + rb * srow + gi)) : 0u;
+      }
+    } else {
+      qa[i] = va ? ldg_stream128(codes + ra * crow + cb) : make_uint4(0, 0, 0, 0);
+      qb[i] = vb ? ldg_stream128(codes + rb * crow + cb) : make_uint4(0, 0, 0, 0);
+      if (FMT == 2) {
+        sa[i] = va ? ldg_stream32(scales + (ra * srow + gi) * 2) : 0u;
+        sb[i] = vb ? ldg_stream32(scales + (rb * srow + gi) * 2) : 0u;
+      } else {
+        sa[i] = va ? e4m3x2_to_f16x2(ldg_stream16(scales + ra * srow + gi)) : 0u;
+        sb[i] = vb ? e4m3x2_to_f16x2(ldg_stream16(scales + rb * srow + gi)) : 0u;
+      }
+    }
+  }
+}
+
 // Loads of one lane's SPW segments (128-bit layout: 16 code bytes of rows ra
 // and rb at 16*tig of each 64-byte segment, and the two group scales they
 // use; rows past n read as zero codes, scale 1 for MXFP4).
@@ -305,7 +361,14 @@ __device__ __forceinline__ void ldg_tile_load(uint4 (&qa)[SPW], uint4 (&qb)[SPW]
 // bytes of two segments with one 256-bit load per row, and their scales with
 // one load (8 B fp16, 4 B E4M3, 2 B E8M0), the segment pairing of
 // ldg_tile_mma's WIDE layout.
-template <int FMT, int NT, int SPW, int WPC = kLdgWarps, int MINB = 2, bool WIDE = false, bool XW = false>
+// PRE < SPW (FP4-G16, 128-bit layout): only the first PRE segments of each
+// warp are loaded before the dependency wait, the rest right after it, so
+// that when the resident wave's CTAs are released together their remaining
+// loads keep HBM busy while they decode what arrived (in_proj on B200:
+// 9.83 vs 10.01 us per launch at PRE = 4 of 8; the 103 registers this takes
+// leave 4 CTAs per SM instead of 5, part of the effect).
+template <int FMT, int NT, int SPW, int WPC = kLdgWarps, int MINB = 2, bool WIDE = false, bool XW = false,
+          int PRE = SPW>
 __global__ void __launch_bounds__(WPC * 32, MINB)
     gemv_fp4_ldg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
                         const uint16_t* __restrict__ x, uint16_t* __restrict__ y, int n, int k, int m, float g) {
@@ -347,10 +410,14 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
         sb[2 * p] = e4m3x2_to_f16x2(s1 & 0xFFFFu); sb[2 * p + 1] = e4m3x2_to_f16x2(s1 >> 16);
       }
     }
+  } else if constexpr (PRE < SPW && !WIDE && (FMT == 2 || FMT == 3)) {
+    ldg_tile_load_part<FMT, SPW, 0, PRE, false>(qa, qb, sa, sb, codes, scales, ra, rb, va, vb, seg0, tig, crow, srow);
+    pdl_wait();  // x may be the previous kernel's output; y may still be read by it
+    ldg_tile_load_part<FMT, SPW, PRE, SPW, true>(qa, qb, sa, sb, codes, scales, ra, rb, va, vb, seg0, tig, crow, srow);
   } else {
     ldg_tile_load<FMT, SPW>(qa, qb, sa, sb, codes, scales, ra, rb, va, vb, seg0, tig, crow, srow);
   }
-  pdl_wait();  // x may be the previous kernel's output; y may still be read by it
+  if (PRE >= SPW || WIDE || !(FMT == 2 || FMT == 3)) pdl_wait();  // x may be the previous kernel's output
   float acc[NT][4];
 #pragma unroll
   for (int j = 0; j < NT; j++)

@@ -42,6 +42,32 @@
 
 namespace qmm {
 
+// The bank-replicated pair table in device memory, generated at compile
+// time: entry (v, lane) at word 32 v + lane is the f16x2 pair (kv[v & 15],
+// kv[v >> 4]) of the printed IQ4_NL table (every value an integer, so its
+// fp16 is exact).  A CTA brings it into shared memory with one bulk copy
+// instead of 2048 stores and conversions.
+constexpr int8_t kIqKv[16] = {-127, -104, -83, -65, -49, -35, -22, -10, 1, 13, 25, 38, 53, 69, 89, 113};
+constexpr uint32_t iq_f16_of_int(int v) {  // fp16 bits of a small integer (|v| < 2048), exact
+  if (v == 0) return 0u;
+  const uint32_t sgn = v < 0 ? 0x8000u : 0u;
+  uint32_t a = (uint32_t)(v < 0 ? -v : v);
+  int e = 0;
+  while ((a >> (e + 1)) != 0u) e++;                       // a in [2^e, 2^(e+1))
+  const uint32_t mant = ((a << 10) >> e) & 0x3FFu;        // the 10 fraction bits (exact: e <= 10)
+  return sgn | ((uint32_t)(e + 15) << 10) | mant;
+}
+struct IqPairTable {
+  uint32_t w[256 * 32];
+  constexpr IqPairTable() : w() {
+    for (int i = 0; i < 256 * 32; i++) {
+      const int v = i >> 5;
+      w[i] = iq_f16_of_int(kIqKv[v & 15]) | (iq_f16_of_int(kIqKv[v >> 4]) << 16);
+    }
+  }
+};
+__device__ __align__(128) const IqPairTable g_iq_pair_table = IqPairTable();
+
 constexpr int kIqtGroup = 16;      // token slots per pass (two MMA n-tiles)
 constexpr int kIqtMaxPairs = 1024;  // in-kernel routing: at most this many (token, slot) pairs
 // ... and the dispatch uses it up to one warp's worth: warp 0 reads the ids
@@ -271,7 +297,8 @@ __global__ void __launch_bounds__(iqt_max_threads(MAXREG)) __maxnreg__(MAXREG) i
       bytes[s] = (uint32_t)(rows * rowb);
       total += bytes[s];
     }
-    mbar_arrive_expect_tx(wbar, total);
+    mbar_arrive_expect_tx(wbar, total + (uint32_t)kIqLutBytes);
+    bulk_load(lut, &g_iq_pair_table, (uint32_t)kIqLutBytes, wbar);
 #pragma unroll
     for (int s = 0; s < S; s++) {
       if (!bytes[s]) continue;
@@ -300,8 +327,9 @@ __global__ void __launch_bounds__(iqt_max_threads(MAXREG)) __maxnreg__(MAXREG) i
     if (STG && threadIdx.x == 0) issue_copies();
   }
   // pair table: entry v (an index byte) = (kv[v & 15], kv[v >> 4]) as f16x2,
-  // one copy per bank; each store covers four banks
-  for (int i = threadIdx.x; i < 256 * 8; i += blockDim.x) {
+  // one copy per bank; each store covers four banks (STG: copied in with the
+  // tiles instead)
+  for (int i = threadIdx.x; !STG && i < 256 * 8; i += blockDim.x) {
     const int v = i >> 3;
     const uint32_t lo = __half_as_ushort(__int2half_rn(c_iq4nl_kv[v & 15]));
     const uint32_t hi = __half_as_ushort(__int2half_rn(c_iq4nl_kv[v >> 4]));

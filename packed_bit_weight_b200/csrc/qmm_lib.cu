@@ -151,7 +151,10 @@ static qmm_status launch_gemv_ldg(const qmm_weights* w, const uint16_t* x, int m
                                   const DevInfo* di) {
   const int n = (int)w->n, k = (int)w->k;
   const int tiles = (n + 15) / 16;
-  auto kern = gemv_fp4_ldg_kernel<FMT, NT, SPW, WPC, MINB, WIDE, XW>;
+  // half of each warp's 8 segments after the dependency wait (FP4-G16, the
+  // 4-warp configuration of k = 4096)
+  constexpr int kPre = (NT == 1 && SPW == 8 && WPC == 4 && !WIDE && (FMT == 2 || FMT == 3)) ? 4 : SPW;
+  auto kern = gemv_fp4_ldg_kernel<FMT, NT, SPW, WPC, MINB, WIDE, XW, kPre>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(tiles);
   cfg.blockDim = dim3(WPC * 32);
@@ -166,8 +169,8 @@ static qmm_status launch_gemv_ldg(const qmm_weights* w, const uint16_t* x, int m
   const uint8_t* scales = static_cast<const uint8_t*>(w->scales);
   const float g = w->global_scale;
   if (cudaLaunchKernelEx(&cfg, kern, codes, scales, x, y, n, k, m, g) != cudaSuccess) return QMM_ERR_CUDA;
-  set_variant("gemv_fp4_ldg<fmt=%d,nt=%d,spw=%d,wpc=%d,minb=%d,wide=%d,xw=%d,tiles=%d>", FMT, NT, SPW, WPC, MINB,
-              WIDE ? 1 : 0, XW ? 1 : 0, tiles);
+  set_variant("gemv_fp4_ldg<fmt=%d,nt=%d,spw=%d,wpc=%d,minb=%d,wide=%d,xw=%d,pre=%d,tiles=%d>", FMT, NT, SPW, WPC,
+              MINB, WIDE ? 1 : 0, XW ? 1 : 0, kPre, tiles);
   return launch_status();
 }
 
