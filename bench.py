@@ -21,7 +21,9 @@ reported as median, standard deviation, minimum and maximum over the steps.
 
 ``e2e``: the same step through ``qmm_gemv_host`` (the call a serving loop
 makes with host buffers): each of the 56 calls brings its activations in
-from pinned host memory and writes y back to pinned host memory.
+from pinned host memory and writes y back to pinned host memory; the step's
+56 calls are captured in one CUDA graph and replayed, and the transfers
+across the bus happen in every replay.
 
 ``cpu_baseline`` is the CPU oracle (plain C, fp64) on one host thread over a
 quarter of the in_proj rows; ``cpu_baseline_all_cores`` runs the same oracle
@@ -318,7 +320,10 @@ def gemv_e2e(p, x_bits, steps, world, layers):
     """The decode step through the public API with host buffers
     (qmm_gemv_host), one call per layer on its own weight copy: every call
     brings that layer's activations in from pinned host memory and writes
-    its y back to pinned host memory."""
+    its y back to pinned host memory.  The 56 calls of a step are captured in
+    one CUDA graph, as a serving loop would replay them; the transfers across
+    the bus happen in every replay (the kernels read and write the pinned
+    buffers through their device mapping)."""
     import torch
     from packed_bit_weight_b200 import qmm
     ws = weight_copies(p, layers)
@@ -328,24 +333,15 @@ def gemv_e2e(p, x_bits, steps, world, layers):
     xd = torch.empty_like(xh, device="cuda")
     yd = torch.empty((m, p.n), dtype=torch.int16, device="cuda")
 
-    st = torch.cuda.current_stream()
+    def launch(i):
+        qmm.qmm_gemv_host(ws[i], xh, yh, xd, yd, stream=torch.cuda.current_stream())
 
-    def step():
-        for w in ws:
-            qmm.qmm_gemv_host(w, xh, yh, xd, yd, stream=st)
-
-    for _ in range(3):
-        step()
-    torch.cuda.synchronize()
-    barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(st)
-    for _ in range(steps):
-        step()
-    e1.record(st)
-    e1.synchronize()
+    g = graph_of(launch, layers)
+    time_graph(g, 3, world)
+    secs, _ = time_graph(g, steps, world)
     assert qmm.qmm_sync_check() == 0
-    secs = max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
+    del g
+    secs = max_over_ranks(secs, world)
     return {"seconds": secs, "steps": steps, "h2d": layers * xh.numel() * 2, "d2h": layers * yh.numel() * 2,
             "gbs": world * ws[0].nbytes * layers * steps / secs / 1e9}
 

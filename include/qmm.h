@@ -180,7 +180,12 @@ qmm_status qmm_gemv(const qmm_weights* w, const uint16_t* x, int64_t m, uint16_t
  * (cudaHostAlloc, torch pin_memory) are used in place through their device
  * mapping: a copy kernel reads x_host into x_dev while the GEMV, launched
  * with programmatic dependent launch, already streams W, and the GEMV stores
- * y straight into y_host (y_dev is then unused).  Pageable buffers go through
+ * y straight into y_host (y_dev is then unused).  The copy kernel is itself
+ * launched with programmatic dependent launch: it reads x_host while the
+ * kernel before it on the stream still runs and writes x_dev only after that
+ * kernel has finished, so x_host must not be written by the kernel
+ * immediately preceding this call on the stream (any other operation in
+ * between restores full ordering).  Pageable buffers go through
  * cudaMemcpyAsync (synchronous to the host) and y_dev.  y_host holds the
  * result once the stream reaches the end of this call's work.
  *   x_host  host, [m][k] fp16 (16-byte aligned for the in-place path)

@@ -103,17 +103,24 @@ __global__ void __launch_bounds__(256) dequant_iq4nl_kernel(const uint8_t* __res
   }
 }
 
-// y[i] = 0 for i < count (a product over an empty k axis).
-// Copy of n16 16-byte words (the activations of a host round trip, read
-// from page-locked host memory through its device mapping).  Lets a kernel
-// launched after it with programmatic dependent launch start at once: the
-// GEMV then streams its weights while this copy crosses the bus.
+// Copy n16 16-byte units from src (page-locked host memory through its device
+// mapping) to dst, one unit per thread (the grid covers n16).  Launched with
+// programmatic dependent launch: the read across the bus starts while the
+// kernel before it on the stream (the previous call's GEMV, which may still
+// read dst) runs; dst is written only after griddepcontrol.wait.  It lets the
+// GEMV launched after it start at once (launch_dependents first): the GEMV
+// streams its weights while this copy crosses the bus, and waits for it
+// before it reads x.
 __global__ void fetch16_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, int64_t n16) {
   asm volatile("griddepcontrol.launch_dependents;" :::);
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += (int64_t)gridDim.x * blockDim.x)
-    dst[i] = src[i];
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  uint4 v = make_uint4(0, 0, 0, 0);
+  if (i < n16) v = src[i];
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (i < n16) dst[i] = v;
 }
 
+// y[i] = 0 for i < count (a product over an empty k axis).
 __global__ void zero_fill_kernel(uint16_t* __restrict__ y, int64_t count) {
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < count; i += (int64_t)gridDim.x * blockDim.x)
     y[i] = 0;

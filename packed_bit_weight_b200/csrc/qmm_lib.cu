@@ -865,10 +865,19 @@ qmm_status qmm_gemv_host(const qmm_weights* w, const uint16_t* x_host, int64_t m
   void* ya = mapped_host_alias(y_host, yb);
   if (xb) {
     if (xa && xb % 16 == 0) {
-      const int64_t n16 = (int64_t)(xb / 16);
-      fetch16_kernel<<<(unsigned)std::min<int64_t>((n16 + 255) / 256, di->sms), 256, 0, st>>>(
-          static_cast<const uint4*>(xa), reinterpret_cast<uint4*>(x_dev), n16);
-      if (cudaGetLastError() != cudaSuccess) return QMM_ERR_CUDA;
+      const int64_t n16 = (int64_t)(xb / 16);  // at most 16 x 2^30 / 16: the grid covers it
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)((n16 + 255) / 256));
+      cfg.blockDim = dim3(256);
+      cfg.stream = st;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      if (cudaLaunchKernelEx(&cfg, fetch16_kernel, static_cast<const uint4*>(xa), reinterpret_cast<uint4*>(x_dev),
+                             n16) != cudaSuccess)
+        return QMM_ERR_CUDA;
     } else if (cudaMemcpyAsync(x_dev, x_host, xb, cudaMemcpyHostToDevice, st) != cudaSuccess) {
       return QMM_ERR_CUDA;
     }
