@@ -60,8 +60,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # ncu DRAM traffic per launch (read + write bytes) of the dominant kernel, by
 # variant string; a variant not listed here reports traffic null.
 TRAFFIC = {
-    # profiles/gemv_fp4_ldg_in_proj_18560x4096_m1.md: 47,552,512 B read + 1,792 B written
-    "gemv_fp4_ldg<fmt=2,nt=1,spw=8,wpc=4,minb=4,wide=0,xw=1,tiles=1160>": 47554304,
+    # profiles/gemv_fp4_ldg_in_proj_18560x4096_m1.md: 47,552,256 B read + 7,936 B written
+    "gemv_fp4_ldg<fmt=2,nt=1,spw=8,wpc=4,minb=4,wide=0,xw=1,pre=4,tiles=1160>": 47560192,
 }
 
 

@@ -364,9 +364,10 @@ __device__ __forceinline__ void ldg_tile_load(uint4 (&qa)[SPW], uint4 (&qb)[SPW]
 // PRE < SPW (FP4-G16, 128-bit layout): only the first PRE segments of each
 // warp are loaded before the dependency wait, the rest right after it, so
 // that when the resident wave's CTAs are released together their remaining
-// loads keep HBM busy while they decode what arrived (in_proj on B200:
-// 9.83 vs 10.01 us per launch at PRE = 4 of 8; the 103 registers this takes
-// leave 4 CTAs per SM instead of 5, part of the effect).
+// loads keep HBM busy while they decode what arrived (on B200 at PRE = 4 of
+// 8: in_proj 9.83 vs 10.01 us per launch, out_proj 4.97 vs 5.26; at in_proj's
+// configuration the 103 registers this takes leave 4 CTAs per SM instead of
+// 5, part of the effect).
 template <int FMT, int NT, int SPW, int WPC = kLdgWarps, int MINB = 2, bool WIDE = false, bool XW = false,
           int PRE = SPW>
 __global__ void __launch_bounds__(WPC * 32, MINB)
