@@ -235,6 +235,20 @@ def time_graph(g, reps: int, world: int, sampler=None, rep_ms=None):
 # ---------------------------------------------------------------------------
 # workloads
 # ---------------------------------------------------------------------------
+def input_manifest(p, x_bits, seed):
+    """SHA-256 of each generated input buffer of the timed workload (packed
+    codes, scales, activations) with the seed that drew them, so that two
+    results can be checked to have run on the same bytes."""
+    import hashlib
+
+    def sha(a):
+        return None if a is None else hashlib.sha256(np.ascontiguousarray(a).tobytes()).hexdigest()
+
+    return {"seed": seed, "w_data_sha256": sha(p.data), "w_scales_sha256": sha(p.scales),
+            "x_sha256": sha(x_bits), "w_data_bytes": int(p.data.nbytes),
+            "w_scales_bytes": 0 if p.scales is None else int(p.scales.nbytes), "x_bytes": int(x_bits.nbytes)}
+
+
 def weight_copies(p, count):
     """`count` distinct device copies of one packed matrix (the seeded host
     matrix uploaded once, the rest device-side clones: the bytes every launch
@@ -270,6 +284,7 @@ def gemv_step_workload(p, x_bits, steps, warmup, world, layers, sampler=None):
     del g
     us = np.asarray(rep_ms, dtype=np.float64) * 1e3 / layers  # per-launch microseconds of each step
     stats = {"median_us": round(float(np.median(us)), 4), "sd_us": round(float(np.std(us)), 4),
+             "p10_us": round(float(np.percentile(us, 10)), 4), "p90_us": round(float(np.percentile(us, 90)), 4),
              "min_us": round(float(us.min()), 4), "max_us": round(float(us.max()), 4), "steps": steps,
              "launches_per_step": layers}
     nbytes = ws[0].nbytes
@@ -279,10 +294,11 @@ def gemv_step_workload(p, x_bits, steps, warmup, world, layers, sampler=None):
             "clocks": clocks, "m": m, "n": p.n, "k": p.k}
 
 
-def gemv_workload(p, x_bits, steps, warmup, world, l2, sampler=None, graph_len=100):
+def gemv_workload(p, x_bits, steps, warmup, world, l2, sampler=None, graph_len=100, op="gemv"):
     """Device-resident GEMV throughput of one matrix shape: rotating weight
     copies (> 4x L2), a graph of up to graph_len back-to-back launches,
-    replayed; returns dict."""
+    replayed; returns dict.  op="gemm" makes each launch a qmm_gemm call
+    (batches beyond the decode GEMV's 16 tokens)."""
     import torch
     from packed_bit_weight_b200 import qmm
     R = rotating_copies(qmm.qmm_packed_bytes(p.fmt, p.n, p.k), l2)
@@ -292,8 +308,10 @@ def gemv_workload(p, x_bits, steps, warmup, world, l2, sampler=None, graph_len=1
     x = torch.from_numpy(x_bits.view(np.int16)).cuda()
     y = torch.empty((m, p.n), dtype=torch.int16, device="cuda")
 
+    call = qmm.qmm_gemm if op == "gemm" else qmm.qmm_gemv
+
     def launch(i):
-        qmm.qmm_gemv(ws[i % R], x, y)
+        call(ws[i % R], x, y)
 
     glen = max(1, min(graph_len, steps))
     g = graph_of(launch, glen)
@@ -699,6 +717,13 @@ def extra_workloads(args, world, l2, peaks):
             out["fp4g16_gemv_%s_m%d" % (name, m)] = {
                 "variant": r["variant"], "gbs": r["gbs"], "frac_hbm": r["gbs"] / peaks["hbm_gbs"],
                 "us_per_launch": r["s_per_launch"] * 1e6, "tflops": 2 * m * p.n * p.k / r["s_per_launch"] / 1e12}
+        # larger decode batches through qmm_gemm (x rows drawn like the sweep's)
+        for m in (32, 64):
+            xm = synth.gen_x(np.random.default_rng(60 + m), m, p.k)
+            r = gemv_workload(p, xm, steps, warm, world, l2, op="gemm")
+            out["fp4g16_gemm_%s_m%d" % (name, m)] = {
+                "variant": r["variant"], "gbs": r["gbs"], "frac_hbm": r["gbs"] / peaks["hbm_gbs"],
+                "us_per_launch": r["s_per_launch"] * 1e6, "tflops": 2 * m * p.n * p.k / r["s_per_launch"] / 1e12}
     del mats
     p, x = synth.make_gemv(synth.FP4_IN_PROJ, synth.FMT_FP4G16_E4M3)
     r = gemv_workload(p, x, steps, warm, world, l2)
@@ -871,7 +896,8 @@ def main():
             "per_launch": r["per_launch"],
             "e2e": {"value": round(e2e["gbs"], 2), "unit": "GB/s", "h2d_bytes_per_step": e2e["h2d"],
                     "d2h_bytes_per_step": e2e["d2h"], "steps": e2e["steps"]},
-            "gpu_launches": launches}
+            "gpu_launches": launches,
+            "inputs": input_manifest(p, x, wl.seed)}
     if not args.no_extra:
         line["workloads"] = extra_workloads(args, world, l2, peaks)
     if rank == 0:

@@ -203,9 +203,11 @@ qmm_status qmm_gemv_host(const qmm_weights* w, const uint16_t* x_host, int64_t m
  * tokens at once (the FP4-G16 model card scores 2,048-token windows,
  * "Mamb2_8B_FP4_Recall_SQ3.25", section "Measured quality"; the weights are
  * the decoded ones of section "Storage and runtime memory", as for
- * qmm_gemv).  m may be any size; from m = 64 (k % 64 == 0) the kernel is a
- * tensor-core GEMM that decodes weight tiles into shared memory, below that
- * the decode-batch kernel over 16-token slices.
+ * qmm_gemv).  m may be any size.  From 256 tokens (k % 64 == 0) the kernel
+ * is a tensor-core GEMM that decodes weight tiles into shared memory; below
+ * that either that GEMM or the qmm_gemv kernels over 16-token slices of x,
+ * whichever a cost model of the two puts first for the shape (few rows or
+ * few tokens favour the slices); qmm_last_variant names the path taken.
  *   x       device, [m][k] fp16;  y device, [m][n] fp16
  * Errors: as qmm_gemv. */
 qmm_status qmm_gemm(const qmm_weights* w, const uint16_t* x, int64_t m, uint16_t* y, void* ws,

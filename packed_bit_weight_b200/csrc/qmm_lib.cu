@@ -8,6 +8,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -490,21 +491,26 @@ static qmm_status launch_gemm_tc_persistent(const qmm_weights* w, const uint16_t
   return launch_gemm_tc_persistent_mh<FMT, 1>(w, x, m, y, st, di);
 }
 
-// Any shape the tensor-core kernel does not take: the decode-batch kernel
-// over 16-token slices of x (a GPU path, recorded as such).
+// Any shape the tensor-core kernel does not take, and small batches: the
+// decode GEMV dispatch (register kernels, split-K, IQ4_NL kernels) over
+// 16-token slices of x, one launch per slice.  Slice j reads x rows
+// [16j, 16j + 16) and writes the same rows of y; both stay 32-byte aligned
+// (16 rows of k or n fp16 values are 32 k or 32 n bytes).
+// (A four-n-tile register kernel over 32-token slices measured no better:
+// in_proj m = 32 39.0 vs 37.6 us, LM head 519 vs 508 us, out_proj 18.7 vs
+// 19.8 us on B200.)
 template <int FMT>
 static qmm_status gemm_by_gemv(const qmm_weights* w, const uint16_t* x, int64_t m, uint16_t* y, cudaStream_t st,
                                const DevInfo* di) {
+  const int64_t slices = (m + 15) / 16;
   for (int64_t m0 = 0; m0 < m; m0 += 16) {
     const int mm = (int)((m - m0) < 16 ? (m - m0) : 16);
-    qmm_weights w1 = *w;
-    const int64_t tiles = (w->n + 15) / 16;
-    gemv_generic_kernel<FMT><<<(unsigned)((tiles + 3) / 4), 128, 0, st>>>(
-        static_cast<const uint8_t*>(w1.data), static_cast<const uint8_t*>(w1.scales), w1.global_scale,
-        x + m0 * w->k, y + m0 * w->n, w->n, w->k, mm);
-    if (cudaGetLastError() != cudaSuccess) return QMM_ERR_CUDA;
+    const qmm_status s = gemv_fmt<FMT>(w, x + m0 * w->k, mm, y + m0 * w->n, st, di);
+    if (s != QMM_OK) return s;
   }
-  set_variant("gemm_by_gemv_generic<fmt=%d>", FMT);
+  char pre[64];
+  snprintf(pre, sizeof(pre), "gemm_by_gemv[slices=%lld]:", (long long)slices);
+  prefix_variant(pre);
   return QMM_OK;
 }
 
@@ -889,6 +895,24 @@ qmm_status qmm_gemv_host(const qmm_weights* w, const uint16_t* x_host, int64_t m
   return QMM_OK;
 }
 
+// Batches under 256 tokens: tensor-core GEMM or the decode GEMV over 16-token
+// slices, whichever a cost model calibrated on B200 puts first.  The GEMM
+// (128 x 256 tiles, one per SM at a time) is decode-bound at about 22,800
+// weights per us per SM, so it costs its waves of tiles whatever m is; the
+// GEMV streams the packed bytes once per slice at about 2.5 TB/s (the 16-token
+// rate) plus ~3 us of launch and tail.  qmm_gemm per launch, us, tc / slices:
+// in_proj 18560x4096 m = 32: 46.0 / 37.7, m = 48: 46.7 / 55.7; out_proj
+// 4096x8192 (16 tiles) m = 128: 87.7 / 75.7; LM head 256000x4096 m = 17:
+// 292 / 365.  From 256 tokens the GEMM's 256-token tiles always lead.
+static bool gemm_prefers_tc(int64_t m, int64_t n, int64_t k, size_t packed_bytes, int sms) {
+  if (m >= 256) return true;
+  const double tiles = (double)((m + 127) / 128) * (double)((n + 255) / 256);
+  const double waves = ceil(tiles / (double)sms);
+  const double tc_us = 5.0 + waves * 256.0 * (double)k / 22800.0;
+  const double gemv_us = (double)((m + 15) / 16) * (3.0 + (double)packed_bytes / 2.5e6);
+  return tc_us < gemv_us;
+}
+
 qmm_status qmm_gemm(const qmm_weights* w, const uint16_t* x, int64_t m, uint16_t* y, void* ws, size_t ws_bytes,
                     void* stream) {
   (void)ws;
@@ -904,10 +928,15 @@ qmm_status qmm_gemm(const qmm_weights* w, const uint16_t* x, int64_t m, uint16_t
   if (!aligned16(y) || (x && !aligned16(x))) return QMM_ERR_MISALIGNED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (w->k == 0) return zero_output(y, m * w->n, st, di);
-  const bool tc = w->k % kGemmBK == 0 && m >= 64;
-  // persistent kernel when k is a multiple of its 256-wide staging chunk;
-  // QMM_GEMM_VARIANT=tile selects the one-tile-per-CTA kernel (measurements)
+  // QMM_GEMM_VARIANT=tc / gemv forces either path at any m (measurements),
+  // =tile the one-tile-per-CTA tensor-core kernel.
   const char* gv = getenv("QMM_GEMM_VARIANT");
+  const bool force_tc = gv && (!strcmp(gv, "tc") || !strcmp(gv, "tile"));
+  const bool force_gemv = gv && !strcmp(gv, "gemv");
+  const size_t packed = qmm_packed_bytes(w->fmt, w->n, w->k);
+  const bool tc = w->k % kGemmBK == 0 && !force_gemv &&
+                  (force_tc || gemm_prefers_tc(m, w->n, w->k, packed, di->sms));
+  // persistent kernel when k is a multiple of its 256-wide staging chunk
   const bool persist = !(gv && !strcmp(gv, "tile")) && w->k % (kGemmChunkSteps * kGemmBK) == 0;
   switch (w->fmt) {
     case QMM_FMT_IQ4_NL:  // the persistent kernel only (256-wide staging chunk = 8 blocks = 144 bytes a row)

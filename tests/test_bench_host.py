@@ -82,3 +82,19 @@ def test_gemm_oracle_baseline_reports_tflops_of_its_sample():
     r = bench.cpu_oracle_gemm(budget_s=0.01, rows=32, tokens=4)
     assert r["unit"] == "TFLOP/s" and r["value"] > 0 and r["cores"] == 1 and r["kind"] == "oracle"
     assert r["sample"].startswith("32 of 18560 rows x 4 of 2048 tokens, k = 4096")
+
+
+def test_input_manifest_pins_the_seeded_generators():
+    """The bench records the SHA-256 of every generated input buffer; the
+    seeded generators must keep drawing the same bytes (an input that changes
+    shows up here before it shows up as a different timing)."""
+    from packed_bit_weight_b200 import synth
+    p, x = synth.make_gemv(synth.IQ4_TINY)
+    m = bench.input_manifest(p, x, synth.IQ4_TINY.seed)
+    assert m["w_data_sha256"] == "813fb1eda2d42bdad81bb5712c038bfe886fb361cf73a380175e96423c2fd45e"
+    assert m["x_sha256"] == "a7fee885ac3cea9ead24bc682ae86dc698fae11aba47f6cafd6f0eb423e63a51"
+    assert m["w_scales_sha256"] is None and m["w_data_bytes"] == 256 * 16 * 18 and m["x_bytes"] == 1024
+    p, x = synth.make_gemv(synth.FP4_IN_PROJ)
+    m = bench.input_manifest(p, x, synth.FP4_IN_PROJ.seed)
+    assert m["w_data_bytes"] == 18560 * 4096 // 2 and m["w_scales_bytes"] == 18560 * 4096 // 16 * 2
+    assert m["x_bytes"] == 2 * 4096 and len(m["w_scales_sha256"]) == 64

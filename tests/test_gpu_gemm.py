@@ -70,6 +70,28 @@ def test_gemm_small_m_uses_decode_kernel_and_agrees():
     check_tol(y, yref, absy, "small m")
 
 
+@pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3, synth.FMT_MXFP4, synth.FMT_IQ4_NL])
+@pytest.mark.parametrize("m", [17, 32, 33, 48, 63])
+@pytest.mark.parametrize("variant", [None, "tc", "gemv"])
+def test_gemm_decode_batches_17_to_63(fmt, m, variant, monkeypatch):
+    """Batches between the decode GEMV's 16 tokens and the tensor-core
+    tiles: the default (16-token GEMV slices), the tensor-core kernel forced
+    at small m (rows past m masked), and the slices forced; 16-row tiles with
+    a ragged tail of rows (n = 1000), k spanning several 128-wide segments."""
+    if variant:
+        monkeypatch.setenv("QMM_GEMM_VARIANT", variant)
+    rng = np.random.default_rng(700 + m + 10 * fmt)
+    n, k = 1000, 1024
+    p = synth.gen_weights(rng, fmt, n, k)
+    x = synth.gen_x(rng, m, k)
+    y = run_gemm(dev(p), x)
+    v = qmm.qmm_last_variant()
+    assert v.startswith("gemm_fp4_tc_persistent" if variant == "tc" else
+                        "gemm_by_gemv[slices=%d]:" % ((m + 15) // 16)), v
+    yref, absy = oracle.matmul(p.fmt, p.n, p.k, p.data, p.scales, p.global_scale, x)
+    check_tol(y, yref, absy, "gemm m=%d fmt=%d %s" % (m, fmt, variant))
+
+
 def test_gemm_iq4nl():
     rng = np.random.default_rng(6)
     p = synth.gen_iq4nl(rng, 100, 256)
@@ -96,6 +118,23 @@ def test_config5_prefill_full_size_sampled(fmt):
     check_tol(y[np.arange(2048), col], ys, as_, "prefill last column")
     y2 = run_gemm(w, x)
     assert np.array_equal(y, y2)  # deterministic
+
+
+@pytest.mark.parametrize("m,path", [(32, "gemm_by_gemv[slices=2]:"), (48, "gemm_fp4_tc_persistent")])
+def test_in_proj_decode_batches_sampled(m, path):
+    """The in_proj matrix (18560 x 4096) at decode batches of 32 and 48: the
+    dispatch takes the GEMV slices at 32 tokens and the tensor-core GEMM at
+    48 (the measured crossover); sampled outputs against the oracle, every
+    token of the first and last rows."""
+    p, _ = synth.make_gemv(synth.FP4_IN_PROJ)
+    x = synth.gen_x(np.random.default_rng(90 + m), m, p.k)
+    y = run_gemm(dev(p), x)
+    assert qmm.qmm_last_variant().startswith(path), qmm.qmm_last_variant()
+    rng = np.random.default_rng(91)
+    mi = np.concatenate([np.arange(m), np.arange(m), rng.integers(0, m, 1000)])
+    ri = np.concatenate([np.zeros(m, np.int64), np.full(m, p.n - 1), rng.integers(0, p.n, 1000)])
+    ys, as_ = oracle.matmul_sampled(p.fmt, p.n, p.k, p.data, p.scales, p.global_scale, x, mi, ri)
+    check_tol(y[mi, ri], ys, as_, "in_proj m=%d sampled" % m)
 
 
 def test_gemm_mxfp4_small_and_normal_scales():
