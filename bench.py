@@ -754,19 +754,20 @@ def extra_workloads(args, world, l2, peaks):
 
 def profile_case(name: str) -> int:
     """Small cases for ncu captures (a few hundred MB on the device, a handful
-    of launches): gemv (in_proj, m=1, 4 rotating copies > L2), gemm (the
+    of launches): gemv / gemv16 (in_proj, m = 1 / 16, 4 rotating copies >
+    L2), gemm (the
     2048-token prefill, two launches), grouped (routed experts, 2 rotating
     sets), moe (router + routed-expert block, 2 rotating sets), dequant
     (in_proj)."""
     import torch
     from packed_bit_weight_b200 import qmm, synth
-    if name == "gemv":
-        p, x = synth.make_gemv(synth.FP4_IN_PROJ)
+    if name in ("gemv", "gemv16"):
+        p, x = synth.make_gemv(synth.FP4_IN_PROJ, m=16 if name == "gemv16" else 1)
         base = qmm.PackedWeights.from_host(p)
         ws = [base] + [qmm.PackedWeights(base.fmt, base.n, base.k, base.data.clone(), base.scales.clone())
                        for _ in range(3)]
         xd = torch.from_numpy(x.view(np.int16)).cuda()
-        y = torch.empty((1, p.n), dtype=torch.int16, device="cuda")
+        y = torch.empty((x.shape[0], p.n), dtype=torch.int16, device="cuda")
         for i in range(8):
             qmm.qmm_gemv(ws[i % 4], xd, y)
     elif name in ("gemm", "gemm_tile"):

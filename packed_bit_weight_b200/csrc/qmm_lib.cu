@@ -154,8 +154,8 @@ static qmm_status launch_gemv_ldg(const qmm_weights* w, const uint16_t* x, int m
   const int tiles = (n + 15) / 16;
   // half of each warp's 8 segments after the dependency wait (FP4-G16, the
   // 4- and 8-warp configurations of k = 4096 and 8192: in_proj 9.83 vs 10.01
-  // us, out_proj 4.97 vs 5.26 us per launch on B200)
-  constexpr int kPre = (NT == 1 && SPW == 8 && (WPC == 4 || WPC == 8) && !WIDE && (FMT == 2 || FMT == 3)) ? 4 : SPW;
+  // us, out_proj 4.97 vs 5.26 us per launch on B200; also at two n-tiles)
+  constexpr int kPre = (SPW == 8 && (WPC == 4 || WPC == 8) && !WIDE && (FMT == 2 || FMT == 3)) ? 4 : SPW;
   auto kern = gemv_fp4_ldg_kernel<FMT, NT, SPW, WPC, MINB, WIDE, XW, kPre>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(tiles);
@@ -204,9 +204,10 @@ static qmm_status launch_gemv_ldg_pick(bool wide, const qmm_weights* w, const ui
   return launch_gemv_ldg<FMT, NT, SPW, WPC, MINB, false>(w, x, m, y, st, di);
 }
 
-// Pick the warps per tile (WPC) and segments per warp (SPW, <= 8 at m <= 8,
-// <= 4 at m <= 16) for k = 128 * WPC * SPW; fewer, fuller warps keep more
-// bytes in flight per register.  Returns UNSUPPORTED_SHAPE for other k.
+// Pick the warps per tile (WPC) and segments per warp (SPW <= 8) for k =
+// 128 * WPC * SPW (k <= 16384 at m <= 8, k <= 8192 at m <= 16); fewer,
+// fuller warps keep more bytes in flight per register.  Returns
+// UNSUPPORTED_SHAPE for other k.
 template <int FMT, int NT>
 static qmm_status gemv_ldg_auto(const qmm_weights* w, const uint16_t* x, int m, uint16_t* y, cudaStream_t st,
                                 const DevInfo* di) {
@@ -245,19 +246,30 @@ static qmm_status gemv_ldg_auto(const qmm_weights* w, const uint16_t* x, int m, 
       }
     }
   } else {
-    if (segs % 8 == 0 && segs / 8 <= 4) {
-      switch (segs / 8) {
-        case 1: return launch_gemv_ldg_pick<FMT, 2, 1, 8, 2>(wide, w, x, m, y, st, di);
-        case 2: return launch_gemv_ldg_pick<FMT, 2, 2, 8, 2>(wide, w, x, m, y, st, di);
-        case 3: return launch_gemv_ldg_pick<FMT, 2, 3, 8, 2>(wide, w, x, m, y, st, di);
-        default: return launch_gemv_ldg_pick<FMT, 2, 4, 8, 2>(wide, w, x, m, y, st, di);
+    // 9..16 tokens: the same shapes as one n-tile (4 warps of up to 8
+    // segments, then 8 warps), which keep twice the segments in flight per
+    // warp of the earlier 8-warp / 16-warp choice at 4 segments (on B200:
+    // LM head m = 16 224 vs 254 us, out_proj 8.5 vs 9.9 us, in_proj 17.0 vs
+    // 19.1 us, 8192 x 2048 4.7 vs 6.3 us).  k > 8192 is left to split-K.
+    if (segs % 4 == 0 && segs / 4 <= 8) {
+      switch (segs / 4) {
+        case 1: return launch_gemv_ldg_pick<FMT, 2, 1, 4, 4>(wide, w, x, m, y, st, di);
+        case 2: return launch_gemv_ldg_pick<FMT, 2, 2, 4, 4>(wide, w, x, m, y, st, di);
+        case 3: return launch_gemv_ldg_pick<FMT, 2, 3, 4, 4>(wide, w, x, m, y, st, di);
+        case 4: return launch_gemv_ldg_pick<FMT, 2, 4, 4, 4>(wide, w, x, m, y, st, di);
+        case 5: return launch_gemv_ldg_pick<FMT, 2, 5, 4, 4>(wide, w, x, m, y, st, di);
+        case 6: return launch_gemv_ldg_pick<FMT, 2, 6, 4, 4>(wide, w, x, m, y, st, di);
+        case 7: return launch_gemv_ldg_pick<FMT, 2, 7, 4, 4>(wide, w, x, m, y, st, di);
+        default: return launch_gemv_ldg_pick<FMT, 2, 8, 4, 4>(wide, w, x, m, y, st, di);
       }
     }
-    if (segs % 16 == 0 && segs / 16 <= 4) {
-      switch (segs / 16) {
-        case 3: return launch_gemv_ldg_pick<FMT, 2, 3, 16, 1>(wide, w, x, m, y, st, di);
-        case 4: return launch_gemv_ldg_pick<FMT, 2, 4, 16, 1>(wide, w, x, m, y, st, di);
-        default: break;
+    if (segs % 8 == 0 && segs / 8 <= 8) {
+      switch (segs / 8) {
+        case 5: return launch_gemv_ldg_pick<FMT, 2, 5, 8, 2>(wide, w, x, m, y, st, di);
+        case 6: return launch_gemv_ldg_pick<FMT, 2, 6, 8, 2>(wide, w, x, m, y, st, di);
+        case 7: return launch_gemv_ldg_pick<FMT, 2, 7, 8, 2>(wide, w, x, m, y, st, di);
+        case 8: return launch_gemv_ldg_pick<FMT, 2, 8, 8, 2>(wide, w, x, m, y, st, di);
+        default: break;  // smaller counts took the 4-warp path
       }
     }
   }
@@ -343,7 +355,7 @@ static bool ldg_config_exists(int64_t k, int m) {
   if (m <= 8)
     return (segs % 4 == 0 && segs / 4 >= 1 && segs / 4 <= 8) || (segs % 8 == 0 && segs / 8 >= 5 && segs / 8 <= 8) ||
            (segs % 16 == 0 && segs / 16 >= 5 && segs / 16 <= 8);
-  return (segs % 8 == 0 && segs / 8 >= 1 && segs / 8 <= 4) || (segs % 16 == 0 && segs / 16 >= 3 && segs / 16 <= 4);
+  return (segs % 4 == 0 && segs / 4 >= 1 && segs / 4 <= 8) || (segs % 8 == 0 && segs / 8 >= 5 && segs / 8 <= 8);
 }
 
 template <int FMT, int NT>
@@ -899,7 +911,7 @@ qmm_status qmm_gemv_host(const qmm_weights* w, const uint16_t* x_host, int64_t m
 // slices, whichever a cost model calibrated on B200 puts first.  The GEMM
 // (128 x 256 tiles, one per SM at a time) is decode-bound at about 22,800
 // weights per us per SM, so it costs its waves of tiles whatever m is; the
-// GEMV streams the packed bytes once per slice at about 2.5 TB/s (the 16-token
+// GEMV streams the packed bytes once per slice at about 2.9 TB/s (the 16-token
 // rate) plus ~3 us of launch and tail.  qmm_gemm per launch, us, tc / slices:
 // in_proj 18560x4096 m = 32: 46.0 / 37.7, m = 48: 46.7 / 55.7; out_proj
 // 4096x8192 (16 tiles) m = 128: 87.7 / 75.7; LM head 256000x4096 m = 17:
@@ -909,7 +921,7 @@ static bool gemm_prefers_tc(int64_t m, int64_t n, int64_t k, size_t packed_bytes
   const double tiles = (double)((m + 127) / 128) * (double)((n + 255) / 256);
   const double waves = ceil(tiles / (double)sms);
   const double tc_us = 5.0 + waves * 256.0 * (double)k / 22800.0;
-  const double gemv_us = (double)((m + 15) / 16) * (3.0 + (double)packed_bytes / 2.5e6);
+  const double gemv_us = (double)((m + 15) / 16) * (3.0 + (double)packed_bytes / 2.9e6);
   return tc_us < gemv_us;
 }
 
