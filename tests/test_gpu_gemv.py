@@ -41,6 +41,25 @@ def test_fast_path_is_used_for_streaming_shapes():
     assert qmm.qmm_last_variant().startswith("gemv_fp4_ldg")      # 1160 tiles: one CTA per tile
 
 
+@pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3, synth.FMT_MXFP4])
+@pytest.mark.parametrize("k,spw,wpc", [(512, 1, 4), (1024, 2, 4), (1536, 3, 4), (2048, 4, 4), (2560, 5, 4),
+                                       (3072, 6, 4), (3584, 7, 4), (4096, 8, 4), (5120, 5, 8), (6144, 6, 8),
+                                       (7168, 7, 8), (8192, 8, 8)])
+@pytest.mark.parametrize("m", [9, 16])
+def test_every_two_n_tile_configuration(fmt, k, spw, wpc, m, monkeypatch):
+    """Every configuration of the register kernel at 9..16 tokens (two
+    n-tiles): 4 warps of 1..8 segments for k <= 4096, 8 warps of 5..8 for
+    k = 5120..8192; 40 rows (a ragged tile), m = 9 (a half-empty second
+    n-tile) and 16."""
+    monkeypatch.setenv("QMM_GEMV_VARIANT", "ldg")
+    p, x = _case(fmt, 40, k, m, 2600 + k + m + fmt)
+    y = run_gemv(dev(p), x)
+    v = qmm.qmm_last_variant()
+    assert v.startswith("gemv_fp4_ldg<fmt=%d,nt=2,spw=%d,wpc=%d," % (fmt, spw, wpc)), v
+    yref, absy = oracle.matmul(fmt, p.n, k, p.data, p.scales, p.global_scale, x)
+    check_tol(y, yref, absy, v)
+
+
 @pytest.mark.parametrize("variant", ["ldg", "generic"])
 @pytest.mark.parametrize("fmt", [synth.FMT_FP4G16_F16, synth.FMT_FP4G16_E4M3])
 @pytest.mark.parametrize("n,k,m", [(1000, 4096, 1), (333, 8192, 3), (64, 2048, 16), (517, 3072, 9)])
