@@ -418,9 +418,20 @@ static qmm_status gemv_fmt(const qmm_weights* w, const uint16_t* x, int m, uint1
       if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
     }
   }
-  if (FMT == 1 && pick == PICK_IQ4_TILE) {
-    const qmm_status s = launch_iq4_tile<IQ_OUT_F16>(w, nullptr, x, 0, 1, nullptr, nullptr, 0, m, y, nullptr, st);
-    if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
+  // Plain IQ4_NL GEMV: the tile-resident kernel, except where the streaming
+  // one measured faster on B200 (us per launch, streaming / tile): very tall
+  // matrices at small m (LM head 256000 x 4096 m = 1 / 4: 269 / 325, 312 /
+  // 340; in_proj 18560 x 4096 m = 1: 24.0 / 24.8) and short rows at m > 8
+  // (256 x 512 m = 16: 3.6 / 5.0; 2560 x 896: 5.9 / 6.6).  Elsewhere the
+  // tile kernel leads: 256 x 512 m = 1 2.5 vs 3.1, 4096 x 4096 m = 1 6.2 vs
+  // 10.6, in_proj m = 16 32.6 vs 41.0, LM head m = 16 430 vs 513.
+  if constexpr (FMT == 1) {
+    const int64_t tiles = (n + 15) / 16;
+    const bool stream_first = (m > 8 && k < 2048) || (tiles >= 4096 && m <= 8) || (tiles >= 1024 && m == 1);
+    if (pick == PICK_IQ4_TILE || (pick == PICK_DEFAULT && !stream_first)) {
+      const qmm_status s = launch_iq4_tile<IQ_OUT_F16>(w, nullptr, x, 0, 1, nullptr, nullptr, 0, m, y, nullptr, st);
+      if (s != QMM_ERR_UNSUPPORTED_SHAPE) return s;
+    }
   }
   if (FMT == 1 && k % 128 == 0 && (pick == PICK_DEFAULT || pick == PICK_IQ4_STREAM)) {
     const qmm_status s = launch_iq4_stream(w, x, 0, 1, nullptr, nullptr, m, y, st, di);
@@ -606,13 +617,13 @@ static qmm_status launch_iq4_tile_cfg(const qmm_weights* w0, const qmm_weights* 
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return QMM_ERR_CUDA;
   set_variant("iq4_tile<mode=%d,s=%d,spw=%d,wpc=%d,w16=%d,stg=%d,spec=%d,route=%s,grid=%d>", MODE, S, SPW, wpc,
-              W16 ? 1 : 0, STG ? 1 : 0, a.spec, ids ? "in_kernel" : "sorted", (int)grid);
+              W16 ? 1 : 0, STG ? 1 : 0, a.spec, ids ? "in_kernel" : offsets ? "sorted" : "none", (int)grid);
   return launch_status();
 }
 
-// Needs k % 128 == 0 and k <= 4096 (at most 16 warps of at most two
-// super-steps); returns QMM_ERR_UNSUPPORTED_SHAPE, having launched nothing,
-// otherwise.
+// Needs k % 256 == 0 and k <= 5376 (at most 21 warps of two super-steps)
+// or k % 128 == 0 and k <= 2048 (at most 16 warps of one); returns
+// QMM_ERR_UNSUPPORTED_SHAPE, having launched nothing, otherwise.
 template <int MODE>
 static qmm_status launch_iq4_tile(const qmm_weights* w0, const qmm_weights* w1, const uint16_t* x, int x_per_pair,
                                   int64_t topk, const int32_t* offsets, const int32_t* perm, int64_t P, int m_plain,

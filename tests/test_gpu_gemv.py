@@ -202,17 +202,25 @@ def test_gemv_edge_cases():
 
 
 @pytest.mark.parametrize("variant", [None, "iq4t", "generic"])
-@pytest.mark.parametrize("n,k,m", [(256, 512, 1), (2000, 4096, 5), (48, 2560, 16), (4096, 8192, 2)])
+@pytest.mark.parametrize("n,k,m", [(256, 512, 1), (2000, 4096, 5), (48, 2560, 16), (4096, 8192, 2),
+                                   (17600, 1024, 1), (300, 896, 12), (256, 512, 16)])
 def test_iq4nl_kernels_vs_oracle(variant, n, k, m, monkeypatch):
-    """Each IQ4_NL GEMV kernel: the streaming kernel (default for k % 128 ==
-    0), the tile-resident one (k <= 4096; a shape it does not take goes to
-    the generic kernel) and the generic one."""
+    """Each IQ4_NL GEMV kernel: the default choice between the tile-resident
+    and the streaming kernel, the tile-resident one forced (k <= 5376 in
+    steps of 256, or k <= 2048; a shape it does not take goes to the generic
+    kernel) and the generic one."""
     if variant:
         monkeypatch.setenv("QMM_GEMV_VARIANT", variant)
     p, x = _case(synth.FMT_IQ4_NL, n, k, m, 3000 + n + k + m)
     y = run_gemv(dev(p), x)
     v = qmm.qmm_last_variant()
-    want = {None: ("gemv_iq4_stream",), "iq4t": ("iq4_tile",) if k <= 4096 else ("gemv_generic",),
+    # default: the tile kernel where it takes the shape (k <= 4096), except
+    # very tall matrices at small m and short rows at m > 8
+    tiles = (n + 15) // 16
+    stream_first = (m > 8 and k < 2048) or (tiles >= 4096 and m <= 8) or (tiles >= 1024 and m == 1)
+    tile_ok = (k % 256 == 0 and k <= 5376) or (k % 128 == 0 and k <= 2048)
+    default = ("iq4_tile",) if tile_ok and not stream_first else ("gemv_iq4_stream",)
+    want = {None: default, "iq4t": ("iq4_tile",) if tile_ok else ("gemv_generic",),
             "generic": ("gemv_generic",)}[variant]
     assert v.startswith(want), v
     yref, absy = oracle.matmul(synth.FMT_IQ4_NL, n, k, p.data, None, 1.0, x)
