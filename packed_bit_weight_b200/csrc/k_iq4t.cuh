@@ -93,6 +93,7 @@ struct IqtArgs {
   int n, k, E;
   int items_per_expert;  // CTAs per expert
   int spec;              // 1: weight loads before the dependency wait
+  int compact;           // ids with P <= 32 and P < E: CTA slot j takes the j-th distinct expert in the ids
 };
 
 // Shared memory: the pair table, then the partial sums [warp][source][slot][row].
@@ -237,11 +238,31 @@ __host__ __device__ constexpr int iqt_max_threads(int maxreg) { return (65536 / 
 // In-kernel routing (a.ids): warp 0 collects the pairs p whose id is this
 // CTA's expert, in increasing p (the order of the stable routing sort), into
 // shared memory; any id outside [0, E) raises ERR_BAD_EXPERT and is left out.
-// Returns the count to every thread (ends with a barrier).
-__device__ __forceinline__ int iqt_collect_pairs(const IqtArgs& a, int e, int* s_pairs, int* s_cnt) {
+// Compact grids (a.compact, P <= 32): the CTA's expert slot e is replaced by
+// the e-th distinct valid id in order of first occurrence (none: -1, no
+// pairs), so only as many experts' CTAs are launched as there are pairs.
+// Returns the count to every thread and e through *s_e (ends with a barrier).
+__device__ __forceinline__ int iqt_collect_pairs(const IqtArgs& a, int& e, int* s_pairs, int* s_cnt, int* s_e) {
   if ((threadIdx.x >> 5) == 0) {
     const int lane = threadIdx.x & 31;
     const unsigned lt = (1u << lane) - 1u;
+    if (a.compact) {
+      const int id = lane < a.P ? a.ids[lane] : -1;
+      const bool valid = lane < a.P && id >= 0 && id < a.E;
+      const unsigned same = __match_any_sync(0xFFFFFFFFu, valid ? id : -1 - lane);  // invalid lanes: own keys
+      const bool first = valid && (__ffs(same) - 1) == lane;
+      const unsigned firsts = __ballot_sync(0xFFFFFFFFu, first);
+      const unsigned mine = __ballot_sync(0xFFFFFFFFu, first && __popc(firsts & lt) == e);
+      const int ej = mine ? __shfl_sync(0xFFFFFFFFu, id, __ffs(mine) - 1) : -1;
+      const unsigned mask = __ballot_sync(0xFFFFFFFFu, valid && id == ej && ej >= 0);
+      if (valid && id == ej && ej >= 0) s_pairs[__popc(mask & lt)] = lane;
+      const bool bad = lane < a.P && !valid;
+      if (__any_sync(0xFFFFFFFFu, bad) && lane == 0 && e == 0 && blockIdx.x == 0) raise_error(ERR_BAD_EXPERT);
+      if (lane == 0) {
+        *s_cnt = __popc(mask);
+        *s_e = ej;
+      }
+    } else {
     int n = 0;
     bool bad = false;
     for (int p0 = 0; p0 < a.P; p0 += 32) {
@@ -253,9 +274,14 @@ __device__ __forceinline__ int iqt_collect_pairs(const IqtArgs& a, int e, int* s
       n += __popc(mask);
     }
     if (__any_sync(0xFFFFFFFFu, bad) && lane == 0 && e == 0 && blockIdx.x == 0) raise_error(ERR_BAD_EXPERT);
-    if (lane == 0) *s_cnt = n;
+    if (lane == 0) {
+      *s_cnt = n;
+      *s_e = e;
+    }
+    }
   }
   __syncthreads();
+  e = *s_e;
   return *s_cnt;
 }
 
@@ -271,7 +297,7 @@ __device__ __forceinline__ int iqt_collect_pairs(const IqtArgs& a, int e, int* s
 template <int MODE, int S, int SPW, int MAXREG, bool W16, bool STG = false>
 __global__ void __launch_bounds__(iqt_max_threads(MAXREG)) __maxnreg__(MAXREG) iq4_tile_kernel(const IqtArgs a) {
   __shared__ int s_pairs[kIqtMaxPairs];
-  __shared__ int s_cnt;
+  __shared__ int s_cnt, s_e;
   __shared__ __align__(8) unsigned long long s_wbar;
   static_assert(MODE != IQ_SWIGLU || S % 2 == 0, "SwiGLU items are gate and up tiles of the same rows");
   constexpr int kOut = (MODE == IQ_SWIGLU) ? S / 2 : S;  // output tiles per item
@@ -280,7 +306,8 @@ __global__ void __launch_bounds__(iqt_max_threads(MAXREG)) __maxnreg__(MAXREG) i
   float* red = reinterpret_cast<float*>(smem_iqt + kIqLutBytes);  // [warp][source][slot][row]
   const int wpc = blockDim.x >> 5;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, grp = lane >> 2, tig = lane & 3;
-  const int e = blockIdx.x / a.items_per_expert, item = blockIdx.x - e * a.items_per_expert;
+  int e = blockIdx.x / a.items_per_expert;  // compact grids: a slot, made an expert by iqt_collect_pairs
+  const int item = blockIdx.x - e * a.items_per_expert;
   const int64_t rowb = (int64_t)(a.k >> 5) * 18;
   // STG: shared-memory copy of the sources after the table and the partial
   // sums; source s holds its 16 rows contiguously (rows past n hold stale
@@ -318,7 +345,7 @@ __global__ void __launch_bounds__(iqt_max_threads(MAXREG)) __maxnreg__(MAXREG) i
   if (!a.spec) {  // most experts may be empty: find out before any other work
     pdl_wait();
     if (a.ids) {
-      cnt = iqt_collect_pairs(a, e, s_pairs, &s_cnt);
+      cnt = iqt_collect_pairs(a, e, s_pairs, &s_cnt, &s_e);
     } else if (a.offsets) {
       start = a.offsets[e];
       cnt = a.offsets[e + 1] - start;
@@ -359,7 +386,7 @@ __global__ void __launch_bounds__(iqt_max_threads(MAXREG)) __maxnreg__(MAXREG) i
     if (!STG) iqt_load<S, SPW, W16>(w, rp, s0, tig);
     pdl_wait();  // routing, activations and the output buffer follow the previous kernel
     if (a.ids) {
-      cnt = iqt_collect_pairs(a, e, s_pairs, &s_cnt);
+      cnt = iqt_collect_pairs(a, e, s_pairs, &s_cnt, &s_e);
     } else if (a.offsets) {
       start = a.offsets[e];
       cnt = a.offsets[e + 1] - start;

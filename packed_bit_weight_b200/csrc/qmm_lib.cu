@@ -577,7 +577,12 @@ static qmm_status launch_iq4_tile_cfg(const qmm_weights* w0, const qmm_weights* 
   const int64_t ipe = (tiles + kOut - 1) / kOut;
   if (wpc * 32 > iqt_max_threads(kMaxReg)) return QMM_ERR_UNSUPPORTED_SHAPE;
   const int64_t E = (offsets || ids) ? w0->num_experts : 1;
-  const int64_t grid = E * ipe;
+  // in-kernel routing with fewer pairs than experts (decode: one token's
+  // top-k): CTAs only for as many experts as there are pairs, each slot
+  // taking the next distinct expert of the ids (MoE block t = 1: 224 instead
+  // of 1,792 gate/up CTAs)
+  const bool compact = ids && P <= 32 && P < E;
+  const int64_t grid = (compact ? P : E) * ipe;
   if (ids && P > kIqtMaxPairs) return QMM_ERR_UNSUPPORTED_SHAPE;
   if (grid < 1 || grid > INT32_MAX) return QMM_ERR_UNSUPPORTED_SHAPE;
   auto kern = iq4_tile_kernel<MODE, S, SPW, kMaxReg, W16, STG>;
@@ -605,6 +610,8 @@ static qmm_status launch_iq4_tile_cfg(const qmm_weights* w0, const qmm_weights* 
   a.items_per_expert = (int)ipe;
   a.spec = ((!offsets && !ids) || P >= 4 * E) ? 1 : 0;
   if (const char* e = getenv("QMM_IQ4T_SPEC")) a.spec = (e[0] == '1') ? 1 : 0;
+  a.compact = compact ? 1 : 0;
+  if (compact) a.spec = 0;  // a slot's expert is known only after the ids are read
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
   cfg.blockDim = dim3(wpc * 32);
@@ -617,7 +624,8 @@ static qmm_status launch_iq4_tile_cfg(const qmm_weights* w0, const qmm_weights* 
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return QMM_ERR_CUDA;
   set_variant("iq4_tile<mode=%d,s=%d,spw=%d,wpc=%d,w16=%d,stg=%d,spec=%d,route=%s,grid=%d>", MODE, S, SPW, wpc,
-              W16 ? 1 : 0, STG ? 1 : 0, a.spec, ids ? "in_kernel" : offsets ? "sorted" : "none", (int)grid);
+              W16 ? 1 : 0, STG ? 1 : 0, a.spec, compact ? "in_kernel_compact" : ids ? "in_kernel" : offsets ? "sorted" : "none",
+              (int)grid);
   return launch_status();
 }
 

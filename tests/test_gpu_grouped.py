@@ -201,6 +201,46 @@ def test_grouped_iq4_tile_kernel(stage, spec, E, n, k, t, topk, per_pair, monkey
 
 
 
+@pytest.mark.parametrize("E,n,k,t,topk,per_pair,bad", [(32, 100, 512, 3, 4, False, False),
+                                                        (64, 48, 256, 5, 6, True, False),
+                                                        (32, 1792, 2560, 1, 4, False, False),
+                                                        (40, 64, 896, 3, 4, False, True),
+                                                        (33, 16, 256, 8, 4, False, False)])
+def test_grouped_iq4_compact_in_kernel_routing(E, n, k, t, topk, per_pair, bad):
+    """Fewer pairs than experts (decode): the tile kernel launches CTAs for
+    as many experts as there are pairs, slot j taking the j-th distinct id in
+    order of first occurrence; tokens that share experts (3 tokens x 4 of 32)
+    leave slots empty; an id outside [0, E) is flagged and its row left
+    unwritten while every other pair is computed."""
+    rng = np.random.default_rng(E * 11 + n + k + t)
+    p = synth.gen_weights(rng, synth.FMT_IQ4_NL, n, k, experts=E)
+    x = synth.gen_x(rng, t, topk, k) if per_pair else synth.gen_x(rng, t, k)
+    ids = synth.gen_topk(rng, t, topk, E)
+    if t >= 3:
+        ids[2] = ids[0]  # a token with the same experts as another
+    if bad:
+        ids[1, 2] = E + 3
+    y, st = _grouped(dev(p), x, ids, per_pair)
+    v = qmm.qmm_last_variant()
+    assert "in_kernel_compact" in v, v
+    assert st == (7 if bad else 0), v
+    valid = (ids >= 0) & (ids < E)
+    assert np.all(y[~valid] == 0x5A5A), v
+    safe = np.where(valid, ids, 0)
+    if per_pair:
+        xs = x.reshape(t * topk, k)
+        yref = np.empty((t * topk, n)); absy = np.empty((t * topk, n))
+        for e in range(E):
+            sel = np.flatnonzero(safe.reshape(-1) == e)
+            if len(sel):
+                de = p.data[e * p.data_stride:(e + 1) * p.data_stride]
+                yref[sel], absy[sel] = oracle.matmul(synth.FMT_IQ4_NL, n, k, de, None, 1.0, xs[sel])
+        yref, absy = yref.reshape(t, topk, n), absy.reshape(t, topk, n)
+    else:
+        yref, absy = oracle.grouped_gemv(synth.FMT_IQ4_NL, n, k, p.data, p.data_stride, None, 0, 1.0, E, x, safe)
+    check_tol(y[valid], yref[valid], absy[valid], "compact %s" % v)
+
+
 @pytest.mark.parametrize("variant", [None, "iq4"])
 def test_grouped_iq4_out_of_range_ids_are_left_out_and_flagged(variant, monkeypatch):
     """IQ4_NL experts with ids outside [0, E): the default kernel routes in
