@@ -120,6 +120,12 @@ __global__ void __launch_bounds__(kRouterThreads) router_topk_kernel(const uint1
 // expert id is out of range were never computed and are left out.
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ yg, const int32_t* __restrict__ ids,
                                                       int E, int t, int topk, int n, uint16_t* __restrict__ out) {
+  // launched with programmatic dependent launch: resident while the down
+  // pass finishes, reads its output only after it (MoE block t = 4 44.4 vs
+  // 45.2 us on B200; the router launched the same way measured 0.6 us slower
+  // at t = 1 and stays a plain launch)
+  asm volatile("griddepcontrol.launch_dependents;" :::);
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int64_t per_tok = n / 8;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < (int64_t)t * per_tok;
        i += (int64_t)gridDim.x * blockDim.x) {

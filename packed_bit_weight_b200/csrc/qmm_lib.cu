@@ -14,6 +14,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "../../include/qmm.h"
 #include "k_dequant.cuh"
@@ -129,6 +130,24 @@ static bool make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt
   CUresult r = g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// Launch with programmatic dependent launch (the kernel waits on the previous
+// one with griddepcontrol.wait before touching its outputs).
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 static int grid_for(int64_t items, int per_block, int sms, int waves = 8) {
@@ -1198,8 +1217,9 @@ qmm_status qmm_moe_routed(const qmm_weights* gate, const qmm_weights* up, const 
       s = launch_iq4_tile<IQ_SCALED_F32>(down, nullptr, h, 1, topk, nullptr, nullptr, P, 0, yg, topk_weights, st,
                                          topk_ids);
     if (s == QMM_OK) {
-      combine_kernel<<<grid_for(t * (d / 8), 256, di->sms), 256, 0, st>>>(yg, topk_ids, (int)E, (int)t, (int)topk,
-                                                                           (int)d, out);
+      if (launch_pdl(combine_kernel, dim3((unsigned)grid_for(t * (d / 8), 256, di->sms)), dim3(256), 0, st,
+                     (const float*)yg, topk_ids, (int)E, (int)t, (int)topk, (int)d, out) != cudaSuccess)
+        return QMM_ERR_CUDA;
       set_variant("moe:gate_up_swiglu_iq4_tile+down_scaled_iq4_tile+combine(in-kernel routing)");
       return launch_status();
     }
@@ -1218,8 +1238,9 @@ qmm_status qmm_moe_routed(const qmm_weights* gate, const qmm_weights* up, const 
     if (s == QMM_OK)
       s = launch_iq4_tile<IQ_SCALED_F32>(down, nullptr, h, 1, topk, offsets, perm, P, 0, yg, topk_weights, st);
     if (s == QMM_OK) {
-      combine_kernel<<<grid_for(t * (d / 8), 256, di->sms), 256, 0, st>>>(yg, topk_ids, (int)E, (int)t, (int)topk,
-                                                                           (int)d, out);
+      if (launch_pdl(combine_kernel, dim3((unsigned)grid_for(t * (d / 8), 256, di->sms)), dim3(256), 0, st,
+                     (const float*)yg, topk_ids, (int)E, (int)t, (int)topk, (int)d, out) != cudaSuccess)
+        return QMM_ERR_CUDA;
       set_variant("moe:route+gate_up_swiglu_iq4_tile+down_scaled_iq4_tile+combine");
       return launch_status();
     }
@@ -1230,7 +1251,9 @@ qmm_status qmm_moe_routed(const qmm_weights* gate, const qmm_weights* up, const 
   if ((s = launch_iq4_mode<IQ_SCALED_F32>(down, nullptr, h, 1, topk, offsets, perm, 0, yg, topk_weights, st, di)) !=
       QMM_OK)
     return s;
-  combine_kernel<<<grid_for(t * (d / 8), 256, di->sms), 256, 0, st>>>(yg, topk_ids, (int)E, (int)t, (int)topk, (int)d, out);
+  if (launch_pdl(combine_kernel, dim3((unsigned)grid_for(t * (d / 8), 256, di->sms)), dim3(256), 0, st,
+                 (const float*)yg, topk_ids, (int)E, (int)t, (int)topk, (int)d, out) != cudaSuccess)
+    return QMM_ERR_CUDA;
   set_variant("moe:route+gate_up_swiglu_iq4+down_scaled_iq4+combine");
   return launch_status();
 }
