@@ -98,7 +98,7 @@ def test_input_manifest_pins_the_seeded_generators():
     m = bench.input_manifest(p, x, synth.FP4_IN_PROJ.seed)
     assert m["w_data_bytes"] == 18560 * 4096 // 2 and m["w_scales_bytes"] == 18560 * 4096 // 16 * 2
     assert m["x_bytes"] == 2 * 4096
-    # the headline workload's bytes, as recorded by bench runs on the GPU machine
+    # the headline workload's bytes: the hashes its bench lines record
     assert m["w_data_sha256"] == "07e75c9359e62a11bd8c8294416246a722595e0f36c5feec2d61081bf6f967fe"
     assert m["w_scales_sha256"] == "4d534c0f7b8502b73dc8aab103f5c188980a7fed4b67bda941892f97ab8c03d5"
     assert m["x_sha256"] == "12904c048eb2e764a96b57dc6966c304b4da34aeafe420f5e20e7bf9433e9d7a"
