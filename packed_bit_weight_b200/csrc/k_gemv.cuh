@@ -199,7 +199,9 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 // 2w+h holds k = 256w + 64*tig + 32h + [0, 32) instead of 128s + 32*tig.
 // XW: the token row's 64 bytes per segment as two 256-bit loads (x rows
 // 32-byte aligned).
-template <int FMT, int NT, int SPW, bool WIDE = false, bool XW = false>
+// MX1 (MXFP4): every group of the warp's segments has f1 = 1 (its scale is
+// an fp16 value), so one multiply by f2 gives the same bits as two.
+template <int FMT, int NT, int SPW, bool WIDE = false, bool XW = false, bool MX1 = false>
 __device__ __forceinline__ void ldg_tile_mma(float (&acc)[NT][4], const uint4 (&qa)[SPW], const uint4 (&qb)[SPW],
                                              const uint32_t (&sa)[SPW], const uint32_t (&sb)[SPW], int seg0, int grp,
                                              int tig, const uint16_t* __restrict__ x, int k, int m) {
@@ -252,7 +254,10 @@ __device__ __forceinline__ void ldg_tile_mma(float (&acc)[NT][4], const uint4 (&
 #pragma unroll
     for (int st = 0; st < 8; st++) {
       uint32_t a0, a1, a2, a3;
-      if (FMT == 4) {  // the lane's one group: code * f1 exact, * f2 rounds once
+      if (FMT == 4 && MX1) {  // f1 = 1: code * f2 rounds once
+        a0 = hmul2(wa[2 * st], sa1); a2 = hmul2(wa[2 * st + 1], sa1);
+        a1 = hmul2(wb[2 * st], sb1); a3 = hmul2(wb[2 * st + 1], sb1);
+      } else if (FMT == 4) {  // the lane's one group: code * f1 exact, * f2 rounds once
         a0 = hmul2(hmul2(wa[2 * st], sa0), sa1); a2 = hmul2(hmul2(wa[2 * st + 1], sa0), sa1);
         a1 = hmul2(hmul2(wb[2 * st], sb0), sb1); a3 = hmul2(hmul2(wb[2 * st + 1], sb0), sb1);
       } else {  // group st/4 of the lane's two
@@ -424,7 +429,20 @@ __global__ void __launch_bounds__(WPC * 32, MINB)
   for (int j = 0; j < NT; j++)
 #pragma unroll
     for (int c = 0; c < 4; c++) acc[j][c] = 0.f;
-  ldg_tile_mma<FMT, NT, SPW, WIDE, XW>(acc, qa, qb, sa, sb, seg0, grp, tig, x, k, m);
+  if constexpr (FMT == 4) {
+    // the common case, every scale of the warp's segments an fp16 value
+    // (factor f1 = 1, low half 0x3C00), takes one multiply per pair; one
+    // vote per warp and tile, so the branch never diverges
+    bool one = true;
+#pragma unroll
+    for (int i = 0; i < SPW; i++) one = one && (sa[i] & 0xFFFFu) == 0x3C00u && (sb[i] & 0xFFFFu) == 0x3C00u;
+    if (__all_sync(0xFFFFFFFFu, one))
+      ldg_tile_mma<FMT, NT, SPW, WIDE, XW, true>(acc, qa, qb, sa, sb, seg0, grp, tig, x, k, m);
+    else
+      ldg_tile_mma<FMT, NT, SPW, WIDE, XW, false>(acc, qa, qb, sa, sb, seg0, grp, tig, x, k, m);
+  } else {
+    ldg_tile_mma<FMT, NT, SPW, WIDE, XW>(acc, qa, qb, sa, sb, seg0, grp, tig, x, k, m);
+  }
   ldg_tile_store<FMT, NT, WPC>(red, acc, warp, grp, tig, n0, n, m, g, y);
 }
 
