@@ -250,6 +250,33 @@ def test_mxfp4_small_and_normal_scales(variant, m, monkeypatch):
     check_tol(y, yref, absy, v)
 
 
+@pytest.mark.parametrize("m", [1, 4, 16])
+def test_mxfp4_one_multiply_path_gives_the_two_factor_bits(m, monkeypatch):
+    """A warp whose scales are all fp16 values multiplies once, a warp with
+    any other scale multiplies by both factors; the two give the same bits.
+    One tile, two versions of the scales that differ in one group of row 0
+    (in range / out of range): rows 1..15 come out bit-identical, although
+    the warp holding that group switches paths, and both versions agree
+    with the oracle."""
+    monkeypatch.setenv("QMM_GEMV_VARIANT", "ldg")
+    rng = np.random.default_rng(4321 + m)
+    n, k = 16, 4096
+    p = synth.gen_fp4(rng, n, k, synth.FMT_MXFP4)
+    sc = rng.integers(118, 136, size=p.scales.size).astype(np.uint8)  # every group an fp16 value
+    sc_b = sc.copy()
+    sc_b[5] = 60                                                        # row 0, group 5: 2^-67
+    x = synth.gen_x(rng, m, k)
+    ys = []
+    for scales in (sc, sc_b):
+        q = synth.Packed(p.fmt, n, k, p.data, scales)
+        y = run_gemv(dev(q), x)
+        assert qmm.qmm_last_variant().startswith("gemv_fp4_ldg<fmt=4"), qmm.qmm_last_variant()
+        yref, absy = oracle.matmul(q.fmt, n, k, q.data, q.scales, 1.0, x)
+        check_tol(y, yref, absy, "mxfp4 one-multiply m=%d" % m)
+        ys.append(y)
+    assert np.array_equal(ys[0][:, 1:], ys[1][:, 1:])
+
+
 @pytest.mark.parametrize("variant", [None, "generic"])
 def test_mxfp4_huge_scales_overflow_like_the_oracle(variant, monkeypatch):
     """E8M0 bytes 143..254 turn codes >= 1 into fp16 infinities; 0xFF is NaN.
