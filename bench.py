@@ -755,10 +755,9 @@ def extra_workloads(args, world, l2, peaks):
 def profile_case(name: str) -> int:
     """Small cases for ncu captures (a few hundred MB on the device, a handful
     of launches): gemv / gemv16 (in_proj, m = 1 / 16, 4 rotating copies >
-    L2), gemm (the
-    2048-token prefill, two launches), grouped (routed experts, 2 rotating
-    sets), moe (router + routed-expert block, 2 rotating sets), dequant
-    (in_proj)."""
+    L2), gemm (the 2048-token prefill, two launches), grouped (routed
+    experts, 2 rotating sets), moe / moe1 (router + routed-expert block at
+    64 / 1 tokens, 2 rotating sets), dequant (in_proj)."""
     import torch
     from packed_bit_weight_b200 import qmm, synth
     if name in ("gemv", "gemv16"):
@@ -793,8 +792,8 @@ def profile_case(name: str) -> int:
             gu, dn = sets[i % 2]
             qmm.qmm_grouped_gemv(gu, xg, d_ids, ygu, x_per_pair=False, ws=ws)
             qmm.qmm_grouped_gemv(dn, xdn, d_ids, ydn, x_per_pair=True, ws=ws)
-    elif name == "moe":
-        wgu, wdn, x, wr, br = synth.make_moe()
+    elif name in ("moe", "moe1"):
+        wgu, wdn, x, wr, br = synth.make_moe(t=1 if name == "moe1" else 64)
         f = wgu.n // 2
         sets = [(qmm.PackedWeights.from_host(wgu), qmm.PackedWeights.from_host(wdn)) for _ in range(2)]
         xd = torch.from_numpy(x.view(np.int16)).cuda()

@@ -3,8 +3,8 @@
 // (MoE)": s = Softmax(x W_router + b), top-4 experts with weights g_i,
 // F(x) = (SiLU(x W_gate) * (x W_up)) W_down, routed output sum_i g_i F_i(x)).
 //
-// router_topk_kernel: one CTA of 32 warps per token; warps take experts,
-//   lanes split k;
+// router_topk_kernel: one thread-block cluster of CS CTAs of 32 warps per
+//   token; the CTAs split k, warps take experts, lanes split each CTA's k;
 //   every fp16 x fp16 product is exact in fp32 and the dot product is
 //   accumulated in fp64, then rounded once, with the bias, to an fp32 logit;
 //   softmax in fp32;
@@ -22,13 +22,18 @@ namespace qmm {
 constexpr int kRouterMaxExperts = 256;
 constexpr int kRouterMaxTopk = 16;
 
-// Router logits: 32 warps per token; warp w takes experts w, w+32, ...; lanes
-// take 8 consecutive k of every 256.  Each fp16 x fp16 product is exact in
-// fp32 and is added in fp64, into two partial sums (alternate chunks: two
+// Router logits: a cluster of CS CTAs per token (launch attribute; CS = 1
+// without one); CTA c of the cluster takes the 256-wide k chunks c, c + CS,
+// ...; in each CTA warp w takes experts w, w+32, ..., and lanes take 8
+// consecutive k of every chunk.  Each fp16 x fp16 product is exact in fp32
+// and is added in fp64, into two partial sums (alternate chunks: two
 // independent add chains); four chunks' loads are issued before their
-// products.  (Eight warps with four experts each measured 11 us per token:
-// the fp64 adds and conversions are long-latency and two warps per scheduler
-// did not hide them.)
+// products.  The CTAs' fp64 partial sums meet in CTA 0 through distributed
+// shared memory and are added in rank order (deterministic), then rounded
+// once with the bias.  (Eight warps with four experts each measured 11 us
+// per token: the fp64 adds and conversions are long-latency and two warps
+// per scheduler did not hide them.  One CTA per token: 7.0 us per launch at
+// one token, the cluster spreads that over CS SMs.)
 constexpr int kRouterThreads = 1024;
 
 __device__ __forceinline__ void router_acc8(double& s, const uint4& xv, const uint4& wv) {
@@ -48,42 +53,51 @@ __global__ void __launch_bounds__(kRouterThreads) router_topk_kernel(const uint1
                                                                      float* __restrict__ g,
                                                                      float* __restrict__ logits_out) {
   __shared__ float z[kRouterMaxExperts];
+  __shared__ double zp[kRouterMaxExperts];  // this CTA's partial sums
   // a kernel launched after this one with programmatic dependent launch (the
   // routed-expert kernels) may start now; it waits for these results
   asm volatile("griddepcontrol.launch_dependents;" :::);
-  const int tok = blockIdx.x;
+  const int cs = (int)cluster_nctarank(), c = (int)cluster_ctarank();
+  const int tok = (int)blockIdx.x / cs;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int kWarps = kRouterThreads / 32;
   const uint16_t* xr = x + (int64_t)tok * k;
+  const int step = 256 * cs;
   for (int e = warp; e < E; e += kWarps) {
     const uint16_t* wr = w + (int64_t)e * k;
     double s0 = 0.0, s1 = 0.0;
-    int kk = lane * 8;
-    for (; kk + 3 * 256 < k; kk += 4 * 256) {
+    int kk = 256 * c + lane * 8;
+    for (; kk + 3 * step < k; kk += 4 * step) {
       uint4 xv[4], wv[4];
 #pragma unroll
       for (int u = 0; u < 4; u++) {
-        xv[u] = *reinterpret_cast<const uint4*>(xr + kk + u * 256);
-        wv[u] = *reinterpret_cast<const uint4*>(wr + kk + u * 256);
+        xv[u] = *reinterpret_cast<const uint4*>(xr + kk + u * step);
+        wv[u] = *reinterpret_cast<const uint4*>(wr + kk + u * step);
       }
       router_acc8(s0, xv[0], wv[0]);
       router_acc8(s1, xv[1], wv[1]);
       router_acc8(s0, xv[2], wv[2]);
       router_acc8(s1, xv[3], wv[3]);
     }
-    for (; kk < k; kk += 256)
+    for (; kk < k; kk += step)
       router_acc8(s0, *reinterpret_cast<const uint4*>(xr + kk), *reinterpret_cast<const uint4*>(wr + kk));
     double v = s0 + s1;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
-    if (lane == 0) {
+    if (lane == 0) zp[e] = v;
+  }
+  cluster_sync();  // every CTA's partials are written (also a CTA barrier)
+  if (c == 0) {
+    for (int e = threadIdx.x; e < E; e += kRouterThreads) {
+      double v = 0.0;
+      for (int r = 0; r < cs; r++) v += ld_dsmem_f64(&zp[e], (uint32_t)r);
       const float zz = __double2float_rn(v + (double)b[e]);
       z[e] = zz;
       if (logits_out) logits_out[(int64_t)tok * E + e] = zz;
     }
   }
-  __syncthreads();
-  if (warp != 0) return;
+  cluster_sync();  // the partials stay until CTA 0 has read them; z is complete
+  if (c != 0 || warp != 0) return;
   float mx = -INFINITY;
   for (int e = lane; e < E; e += 32) mx = fmaxf(mx, z[e]);
 #pragma unroll

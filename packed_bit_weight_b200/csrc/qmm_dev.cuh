@@ -296,6 +296,14 @@ __device__ __forceinline__ uint32_t cluster_nctarank() {
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+// fp64 at the same shared-memory offset as `local` in the CTA of rank r.
+__device__ __forceinline__ double ld_dsmem_f64(const double* local, uint32_t r) {
+  uint32_t remote;
+  double v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(local)), "r"(r));
+  asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v) : "r"(remote) : "memory");
+  return v;
+}
 // fp32 at the same shared-memory offset as `local` in the CTA of rank r.
 __device__ __forceinline__ float ld_dsmem_f32(const float* local, uint32_t r) {
   uint32_t remote;

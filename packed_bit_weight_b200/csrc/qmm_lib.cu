@@ -1167,9 +1167,32 @@ qmm_status qmm_router_topk(const uint16_t* x, const uint16_t* w_router, const fl
   if ((x && !aligned16(x)) || (w_router && !aligned16(w_router)) || !aligned16(bias) || !aligned16(topk_ids) ||
       !aligned16(topk_weights) || (logits && !aligned16(logits)))
     return QMM_ERR_MISALIGNED;
-  router_topk_kernel<<<(unsigned)t, kRouterThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      x, w_router, bias, (int)k, (int)num_experts, (int)topk, topk_ids, topk_weights, logits);
-  set_variant("router_topk");
+  // a cluster of cs CTAs per token splits k: 8 for a few tokens, 2 for more
+  // (router alone on B200, us per launch at cs = 1 / 2 / 4 / 8: one token
+  // 7.8 / 6.4 / 6.2 / 5.8; 64 tokens 8.4 / 7.0 / 10.2 / 17.0).
+  // QMM_ROUTER_CS=1/2/4/8 forces a size (measurement knob).
+  int cs = t <= 4 ? 8 : 2;
+  if (const char* e = getenv("QMM_ROUTER_CS")) {
+    const int v = atoi(e);
+    if (v == 1 || v == 2 || v == 4 || v == 8) cs = v;
+  }
+  if ((int64_t)t * cs > INT32_MAX) cs = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(t * cs));
+  cfg.blockDim = dim3(kRouterThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, router_topk_kernel, x, w_router, bias, (int)k, (int)num_experts, (int)topk, topk_ids,
+                         topk_weights, logits) != cudaSuccess)
+    return QMM_ERR_CUDA;
+  set_variant("router_topk<cs=%d>", cs);
   return launch_status();
 }
 
