@@ -54,6 +54,19 @@ def test_router_vs_oracle(t, k, E, topk):
     _check_router(x, w, b, topk)
 
 
+@pytest.mark.parametrize("cs", ["1", "2", "4", "8"])
+@pytest.mark.parametrize("t,k,E,topk", [(1, 2560, 32, 4), (6, 520, 7, 3), (3, 24, 40, 40)])
+def test_router_every_cluster_size(cs, t, k, E, topk, monkeypatch):
+    """The router's k split over 1, 2, 4 or 8 CTAs per token (k = 24 leaves
+    most CTAs of a cluster without a chunk; k = 520 a ragged last chunk)."""
+    monkeypatch.setenv("QMM_ROUTER_CS", cs)
+    rng = np.random.default_rng(t * 1000 + k + E + int(cs))
+    x = synth.gen_x(rng, t, k)
+    w, b = synth.gen_router(rng, E, k)
+    _check_router(x, w, b, topk)
+    assert qmm.qmm_last_variant() == "router_topk<cs=%s>" % cs
+
+
 def test_router_ties_go_to_the_lower_index():
     rng = np.random.default_rng(5)
     x = synth.gen_x(rng, 4, 256)
