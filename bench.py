@@ -755,9 +755,10 @@ def extra_workloads(args, world, l2, peaks):
 def profile_case(name: str) -> int:
     """Small cases for ncu captures (a few hundred MB on the device, a handful
     of launches): gemv / gemv16 (in_proj, m = 1 / 16, 4 rotating copies >
-    L2), gemm (the 2048-token prefill, two launches), grouped (routed
-    experts, 2 rotating sets), moe / moe1 (router + routed-expert block at
-    64 / 1 tokens, 2 rotating sets), dequant (in_proj)."""
+    L2), gemm / gemm_iq4 (the 2048-token prefill, FP4-G16 / IQ4_NL, two
+    launches), grouped (routed experts, 2 rotating sets), moe / moe1 (router
+    + routed-expert block at 64 / 1 tokens, 2 rotating sets), dequant
+    (in_proj)."""
     import torch
     from packed_bit_weight_b200 import qmm, synth
     if name in ("gemv", "gemv16"):
@@ -769,10 +770,10 @@ def profile_case(name: str) -> int:
         y = torch.empty((x.shape[0], p.n), dtype=torch.int16, device="cuda")
         for i in range(8):
             qmm.qmm_gemv(ws[i % 4], xd, y)
-    elif name in ("gemm", "gemm_tile"):
+    elif name in ("gemm", "gemm_tile", "gemm_iq4"):
         if name == "gemm_tile":
             os.environ["QMM_GEMM_VARIANT"] = "tile"
-        p, x = synth.make_prefill()
+        p, x = synth.make_prefill(synth.FMT_IQ4_NL if name == "gemm_iq4" else synth.FMT_FP4G16_F16)
         w = qmm.PackedWeights.from_host(p)
         xd = torch.from_numpy(x.view(np.int16)).cuda()
         y = torch.empty((x.shape[0], p.n), dtype=torch.int16, device="cuda")
