@@ -263,21 +263,21 @@ __device__ __forceinline__ int iqt_collect_pairs(const IqtArgs& a, int& e, int* 
         *s_e = ej;
       }
     } else {
-    int n = 0;
-    bool bad = false;
-    for (int p0 = 0; p0 < a.P; p0 += 32) {
-      const int p = p0 + lane;
-      const int id = p < a.P ? a.ids[p] : -1;
-      bad |= p < a.P && (id < 0 || id >= a.E);
-      const unsigned mask = __ballot_sync(0xFFFFFFFFu, id == e);
-      if (id == e) s_pairs[n + __popc(mask & lt)] = p;
-      n += __popc(mask);
-    }
-    if (__any_sync(0xFFFFFFFFu, bad) && lane == 0 && e == 0 && blockIdx.x == 0) raise_error(ERR_BAD_EXPERT);
-    if (lane == 0) {
-      *s_cnt = n;
-      *s_e = e;
-    }
+      int n = 0;
+      bool bad = false;
+      for (int p0 = 0; p0 < a.P; p0 += 32) {
+        const int p = p0 + lane;
+        const int id = p < a.P ? a.ids[p] : -1;
+        bad |= p < a.P && (id < 0 || id >= a.E);
+        const unsigned mask = __ballot_sync(0xFFFFFFFFu, id == e);
+        if (id == e) s_pairs[n + __popc(mask & lt)] = p;
+        n += __popc(mask);
+      }
+      if (__any_sync(0xFFFFFFFFu, bad) && lane == 0 && e == 0 && blockIdx.x == 0) raise_error(ERR_BAD_EXPERT);
+      if (lane == 0) {
+        *s_cnt = n;
+        *s_e = e;
+      }
     }
   }
   __syncthreads();
