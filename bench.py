@@ -704,13 +704,16 @@ def dequant_workload(world, l2, peaks):
             "us_per_launch": per * 1e6}
 
 
-def extra_workloads(args, world, l2, peaks):
-    """Every other workload of the path, device-resident, kernel throughput."""
+def extra_workloads(args, world, l2, peaks, only=None):
+    """Every other workload of the path, device-resident, kernel throughput.
+    only = 1, 3, 4 or 5: just that configuration's workloads (the IQ4_NL
+    tiny GEMV; the out_proj / LM head batch sweep; the routed experts and
+    MoE blocks; the prefill GEMMs)."""
     from packed_bit_weight_b200 import synth
     out = {}
     steps = max(200, args.steps // 10)
     warm = max(3, args.warmup // 10)
-    mats = synth.make_sweep()
+    mats = synth.make_sweep() if only in (None, 3) else {}
     for name, (p, xall) in mats.items():
         for m in (1, 4, 16):
             r = gemv_workload(p, xall[:m], steps, warm, world, l2)
@@ -725,30 +728,36 @@ def extra_workloads(args, world, l2, peaks):
                 "variant": r["variant"], "gbs": r["gbs"], "frac_hbm": r["gbs"] / peaks["hbm_gbs"],
                 "us_per_launch": r["s_per_launch"] * 1e6, "tflops": 2 * m * p.n * p.k / r["s_per_launch"] / 1e12}
     del mats
-    p, x = synth.make_gemv(synth.FP4_IN_PROJ, synth.FMT_FP4G16_E4M3)
-    r = gemv_workload(p, x, steps, warm, world, l2)
-    out["fp4g16_e4m3_gemv_in_proj_m1"] = {"variant": r["variant"], "gbs": r["gbs"],
-                                          "frac_hbm": r["gbs"] / peaks["hbm_gbs"],
-                                          "us_per_launch": r["s_per_launch"] * 1e6}
-    p, x = synth.make_gemv(synth.FP4_IN_PROJ, synth.FMT_MXFP4)
-    r = gemv_workload(p, x, steps, warm, world, l2)
-    out["mxfp4_gemv_in_proj_m1"] = {"variant": r["variant"], "gbs": r["gbs"], "frac_hbm": r["gbs"] / peaks["hbm_gbs"],
-                                    "us_per_launch": r["s_per_launch"] * 1e6,
-                                    "note": "E2M1 codes + one E8M0 byte per 32 (4.25 bits per weight)"}
-    p, x = synth.make_gemv(synth.IQ4_TINY)
-    r = gemv_workload(p, x, steps, warm, world, l2)
-    out["iq4nl_gemv_tiny_256x512_m1"] = {"variant": r["variant"], "gbs": r["gbs"],
-                                         "us_per_launch": r["s_per_launch"] * 1e6, "note": "fits in L2"}
-    out["fp4g16_prefill_gemm_2048x18560x4096"] = gemm_workload(synth.FMT_FP4G16_F16, world, l2, peaks)
-    out["fp4g16_e4m3_prefill_gemm_2048x18560x4096"] = gemm_workload(synth.FMT_FP4G16_E4M3, world, l2, peaks)
-    out["mxfp4_prefill_gemm_2048x18560x4096"] = gemm_workload(synth.FMT_MXFP4, world, l2, peaks)
-    out["iq4nl_prefill_gemm_2048x18560x4096"] = gemm_workload(synth.FMT_IQ4_NL, world, l2, peaks)
-    out["iq4nl_grouped_experts_t64_top4"] = grouped_workload(world, l2, peaks)
-    out["iq4nl_moe_block_t64_top4"] = moe_workload(world, l2, peaks, t=64)
-    out["iq4nl_moe_block_t1_top4"] = moe_workload(world, l2, peaks, t=1)
-    out["fp4g16_dequant_in_proj"] = dequant_workload(world, l2, peaks)
-    out["fp4g16_quantize_in_proj"] = quantize_workload(synth.FMT_FP4G16_F16, world, l2, peaks)
-    out["iq4nl_quantize_in_proj"] = quantize_workload(synth.FMT_IQ4_NL, world, l2, peaks)
+    if only is None:
+        p, x = synth.make_gemv(synth.FP4_IN_PROJ, synth.FMT_FP4G16_E4M3)
+        r = gemv_workload(p, x, steps, warm, world, l2)
+        out["fp4g16_e4m3_gemv_in_proj_m1"] = {"variant": r["variant"], "gbs": r["gbs"],
+                                              "frac_hbm": r["gbs"] / peaks["hbm_gbs"],
+                                              "us_per_launch": r["s_per_launch"] * 1e6}
+        p, x = synth.make_gemv(synth.FP4_IN_PROJ, synth.FMT_MXFP4)
+        r = gemv_workload(p, x, steps, warm, world, l2)
+        out["mxfp4_gemv_in_proj_m1"] = {"variant": r["variant"], "gbs": r["gbs"],
+                                        "frac_hbm": r["gbs"] / peaks["hbm_gbs"],
+                                        "us_per_launch": r["s_per_launch"] * 1e6,
+                                        "note": "E2M1 codes + one E8M0 byte per 32 (4.25 bits per weight)"}
+    if only in (None, 1):
+        p, x = synth.make_gemv(synth.IQ4_TINY)
+        r = gemv_workload(p, x, steps, warm, world, l2)
+        out["iq4nl_gemv_tiny_256x512_m1"] = {"variant": r["variant"], "gbs": r["gbs"],
+                                             "us_per_launch": r["s_per_launch"] * 1e6, "note": "fits in L2"}
+    if only in (None, 5):
+        out["fp4g16_prefill_gemm_2048x18560x4096"] = gemm_workload(synth.FMT_FP4G16_F16, world, l2, peaks)
+        out["fp4g16_e4m3_prefill_gemm_2048x18560x4096"] = gemm_workload(synth.FMT_FP4G16_E4M3, world, l2, peaks)
+        out["mxfp4_prefill_gemm_2048x18560x4096"] = gemm_workload(synth.FMT_MXFP4, world, l2, peaks)
+        out["iq4nl_prefill_gemm_2048x18560x4096"] = gemm_workload(synth.FMT_IQ4_NL, world, l2, peaks)
+    if only in (None, 4):
+        out["iq4nl_grouped_experts_t64_top4"] = grouped_workload(world, l2, peaks)
+        out["iq4nl_moe_block_t64_top4"] = moe_workload(world, l2, peaks, t=64)
+        out["iq4nl_moe_block_t1_top4"] = moe_workload(world, l2, peaks, t=1)
+    if only is None:
+        out["fp4g16_dequant_in_proj"] = dequant_workload(world, l2, peaks)
+        out["fp4g16_quantize_in_proj"] = quantize_workload(synth.FMT_FP4G16_F16, world, l2, peaks)
+        out["iq4nl_quantize_in_proj"] = quantize_workload(synth.FMT_IQ4_NL, world, l2, peaks)
     return out
 
 
@@ -833,10 +842,22 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="headline workload only")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--profile-case", default=None,
-                    help="run one small case for an ncu capture and exit (gemv, gemm, gemm_tile, grouped, dequant)")
+                    help="run one small case for an ncu capture and exit (gemv, gemv16, gemm, gemm_tile, gemm_iq4, "
+                         "grouped, moe, moe1, dequant)")
+    ap.add_argument("--config", type=int, default=None, choices=[1, 3, 4, 5],
+                    help="print only that configuration's workloads (1: IQ4_NL tiny GEMV, 3: out_proj / LM head "
+                         "batches, 4: routed experts and MoE blocks, 5: prefill GEMMs); the headline (2) is the "
+                         "default line")
     args = ap.parse_args()
     if args.profile_case:
         return profile_case(args.profile_case)
+    if args.config is not None:
+        world, rank, local = dist_init()
+        peaks, _ = load_peaks()
+        w = extra_workloads(args, world, l2_bytes(), peaks, only=args.config)
+        if rank == 0:
+            print(json.dumps({"config_id": args.config, "n_gpus": world, "workloads": w}))
+        return 0
     if args.warmup < 3:
         args.warmup = 3
 
