@@ -102,3 +102,34 @@ def test_input_manifest_pins_the_seeded_generators():
     assert m["w_data_sha256"] == "07e75c9359e62a11bd8c8294416246a722595e0f36c5feec2d61081bf6f967fe"
     assert m["w_scales_sha256"] == "4d534c0f7b8502b73dc8aab103f5c188980a7fed4b67bda941892f97ab8c03d5"
     assert m["x_sha256"] == "12904c048eb2e764a96b57dc6966c304b4da34aeafe420f5e20e7bf9433e9d7a"
+
+
+def test_config_selection_runs_only_that_configurations_workloads(monkeypatch):
+    """`--config N` (extra_workloads(only=N)) measures exactly configuration
+    N's workloads; no selection measures every workload."""
+    import types
+
+    import numpy as np
+    from packed_bit_weight_b200 import synth
+
+    class P:
+        n, k = 16, 32
+
+    monkeypatch.setattr(synth, "make_sweep", lambda *a, **k: {"out_proj": (P(), np.zeros((16, 32), np.uint16)),
+                                                               "lm_head": (P(), np.zeros((16, 32), np.uint16))})
+    monkeypatch.setattr(synth, "make_gemv", lambda *a, **k: (P(), np.zeros((1, 32), np.uint16)))
+    fake = {"variant": "v", "gbs": 1.0, "s_per_launch": 1e-6}
+    monkeypatch.setattr(bench, "gemv_workload", lambda *a, **k: fake)
+    for name in ("gemm_workload", "grouped_workload", "moe_workload", "dequant_workload", "quantize_workload"):
+        monkeypatch.setattr(bench, name, lambda *a, **k: {"x": 1})
+    args = types.SimpleNamespace(steps=20, warmup=5)
+    peaks = {"hbm_gbs": 1.0}
+    keys = {n: set(bench.extra_workloads(args, 1, 1 << 27, peaks, only=n)) for n in (1, 3, 4, 5)}
+    assert keys[1] == {"iq4nl_gemv_tiny_256x512_m1"}
+    assert keys[3] == {"fp4g16_%s_%s_m%d" % (op, mat, m) for mat in ("out_proj", "lm_head")
+                       for op, ms in (("gemv", (1, 4, 16)), ("gemm", (32, 64))) for m in ms}
+    assert keys[4] == {"iq4nl_grouped_experts_t64_top4", "iq4nl_moe_block_t64_top4", "iq4nl_moe_block_t1_top4"}
+    assert keys[5] == {"%s_prefill_gemm_2048x18560x4096" % f for f in ("fp4g16", "fp4g16_e4m3", "mxfp4", "iq4nl")}
+    full = set(bench.extra_workloads(args, 1, 1 << 27, peaks))
+    assert full >= keys[1] | keys[3] | keys[4] | keys[5]
+    assert {"fp4g16_e4m3_gemv_in_proj_m1", "mxfp4_gemv_in_proj_m1", "fp4g16_dequant_in_proj"} <= full
