@@ -366,10 +366,14 @@ qmm_status qmm_sync_check(void* stream);
  *   QMM_DEBUG_WITHHOLD_X_TILES  value = 1: the GEMMs' activation loader
  *                               issues no tile load, so their waits run out
  *                               (nothing is written to y); 0: normal
- * Both are device-wide (current device), copied synchronously, and stay set
+ *   QMM_DEBUG_WITHHOLD_TILE_COPIES  value = 1: the routed-expert tile kernel
+ *                               issues none of its bulk copies, so its wait
+ *                               for them runs out (y is left meaningless);
+ *                               0: normal
+ * All are device-wide (current device), copied synchronously, and stay set
  * until changed.  Errors: INVALID_ARG (unknown hook or value), NOT_SM100,
  * CUDA. */
-enum { QMM_DEBUG_WAIT_LIMIT_NS = 1, QMM_DEBUG_WITHHOLD_X_TILES = 2 };
+enum { QMM_DEBUG_WAIT_LIMIT_NS = 1, QMM_DEBUG_WITHHOLD_X_TILES = 2, QMM_DEBUG_WITHHOLD_TILE_COPIES = 3 };
 qmm_status qmm_debug_set(int32_t what, int64_t value);
 
 /* Static text for a status code. */

@@ -325,6 +325,7 @@ __global__ void __launch_bounds__(iqt_max_threads(MAXREG)) __maxnreg__(MAXREG) i
       total += bytes[s];
     }
     mbar_arrive_expect_tx(wbar, total + (uint32_t)kIqLutBytes);
+    if (g_test_flags & kTestWithholdTileCopies) return;  // test switch: the copies never come
     bulk_load(lut, &g_iq_pair_table, (uint32_t)kIqLutBytes, wbar);
 #pragma unroll
     for (int s = 0; s < S; s++) {

@@ -1290,9 +1290,12 @@ qmm_status qmm_debug_set(int32_t what, int64_t value) {
     const unsigned long long v = (unsigned long long)value;
     return cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v)) == cudaSuccess ? QMM_OK : QMM_ERR_CUDA;
   }
-  if (what == QMM_DEBUG_WITHHOLD_X_TILES) {
+  if (what == QMM_DEBUG_WITHHOLD_X_TILES || what == QMM_DEBUG_WITHHOLD_TILE_COPIES) {
     if (value != 0 && value != 1) return QMM_ERR_INVALID_ARG;
-    const unsigned int v = value ? kTestWithholdXTiles : 0u;
+    const unsigned int bit = (what == QMM_DEBUG_WITHHOLD_X_TILES) ? kTestWithholdXTiles : kTestWithholdTileCopies;
+    unsigned int v = 0u;
+    if (cudaMemcpyFromSymbol(&v, g_test_flags, sizeof(v)) != cudaSuccess) return QMM_ERR_CUDA;
+    v = value ? (v | bit) : (v & ~bit);
     return cudaMemcpyToSymbol(g_test_flags, &v, sizeof(v)) == cudaSuccess ? QMM_OK : QMM_ERR_CUDA;
   }
   return QMM_ERR_INVALID_ARG;

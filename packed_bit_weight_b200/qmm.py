@@ -370,6 +370,7 @@ def qmm_moe_routed(gate: PackedWeights, up: PackedWeights, down: PackedWeights, 
 
 DEBUG_WAIT_LIMIT_NS = 1
 DEBUG_WITHHOLD_X_TILES = 2
+DEBUG_WITHHOLD_TILE_COPIES = 3
 
 
 def qmm_debug_set(what: int, value: int) -> None:
