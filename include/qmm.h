@@ -370,7 +370,8 @@ qmm_status qmm_sync_check(void* stream);
  *                               issues none of its bulk copies, so its wait
  *                               for them runs out (y is left meaningless);
  *                               0: normal
- * All are device-wide (current device), copied synchronously, and stay set
+ * The first two are device-wide (current device) and copied synchronously,
+ * the third applies to every later launch of this process; all stay set
  * until changed.  Errors: INVALID_ARG (unknown hook or value), NOT_SM100,
  * CUDA. */
 enum { QMM_DEBUG_WAIT_LIMIT_NS = 1, QMM_DEBUG_WITHHOLD_X_TILES = 2, QMM_DEBUG_WITHHOLD_TILE_COPIES = 3 };

@@ -94,6 +94,7 @@ struct IqtArgs {
   int items_per_expert;  // CTAs per expert
   int spec;              // 1: weight loads before the dependency wait
   int compact;           // ids with P <= 32 and P < E: CTA slot j takes the j-th distinct expert in the ids
+  int withhold;          // test switch (qmm_debug_set, from the host): the bulk copies are not issued
 };
 
 // Shared memory: the pair table, then the partial sums [warp][source][slot][row].
@@ -325,7 +326,7 @@ __global__ void __launch_bounds__(iqt_max_threads(MAXREG)) __maxnreg__(MAXREG) i
       total += bytes[s];
     }
     mbar_arrive_expect_tx(wbar, total + (uint32_t)kIqLutBytes);
-    if (g_test_flags & kTestWithholdTileCopies) return;  // test switch: the copies never come
+    if (a.withhold) return;  // test switch: the copies never come
     bulk_load(lut, &g_iq_pair_table, (uint32_t)kIqLutBytes, wbar);
 #pragma unroll
     for (int s = 0; s < S; s++) {

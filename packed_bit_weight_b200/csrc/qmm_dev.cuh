@@ -24,9 +24,9 @@ __device__ unsigned long long g_wait_limit_ns = kWaitLimitNs;
 // tensor-core GEMMs' activation loader issues no tile load, so the MMA
 // issuer's wait for the first stage runs out and the kernel takes its
 // timeout path (raise the error word, drain, free tensor memory, return).
-// kTestWithholdTileCopies: the routed-expert tile kernel announces its bulk
-// copies on its mbarrier but issues none, so its wait for them runs out.
-enum : unsigned { kTestWithholdXTiles = 1u, kTestWithholdTileCopies = 2u };
+// (The routed-expert tile kernel's switch, which withholds its bulk copies,
+// is a launch argument instead: IqtArgs::withhold.)
+enum : unsigned { kTestWithholdXTiles = 1u };
 __device__ unsigned int g_test_flags;
 
 __device__ __forceinline__ void raise_error(unsigned bits) { atomicOr(&g_err_word, bits); }

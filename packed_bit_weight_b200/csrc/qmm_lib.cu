@@ -52,6 +52,9 @@ struct DevInfo {
   size_t smem_optin = 0;
 };
 static DevInfo g_dev[64];
+// qmm_debug_set(QMM_DEBUG_WITHHOLD_TILE_COPIES): passed to the tile kernel as
+// a launch argument (process-wide; tests only)
+static bool g_withhold_tile_copies = false;
 static std::mutex g_mu;
 
 static qmm_status device_info(DevInfo** out) {
@@ -630,6 +633,7 @@ static qmm_status launch_iq4_tile_cfg(const qmm_weights* w0, const qmm_weights* 
   a.spec = ((!offsets && !ids) || P >= 4 * E) ? 1 : 0;
   if (const char* e = getenv("QMM_IQ4T_SPEC")) a.spec = (e[0] == '1') ? 1 : 0;
   a.compact = compact ? 1 : 0;
+  a.withhold = g_withhold_tile_copies ? 1 : 0;
   if (compact) a.spec = 0;  // a slot's expert is known only after the ids are read
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
@@ -1290,13 +1294,15 @@ qmm_status qmm_debug_set(int32_t what, int64_t value) {
     const unsigned long long v = (unsigned long long)value;
     return cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v)) == cudaSuccess ? QMM_OK : QMM_ERR_CUDA;
   }
-  if (what == QMM_DEBUG_WITHHOLD_X_TILES || what == QMM_DEBUG_WITHHOLD_TILE_COPIES) {
+  if (what == QMM_DEBUG_WITHHOLD_X_TILES) {
     if (value != 0 && value != 1) return QMM_ERR_INVALID_ARG;
-    const unsigned int bit = (what == QMM_DEBUG_WITHHOLD_X_TILES) ? kTestWithholdXTiles : kTestWithholdTileCopies;
-    unsigned int v = 0u;
-    if (cudaMemcpyFromSymbol(&v, g_test_flags, sizeof(v)) != cudaSuccess) return QMM_ERR_CUDA;
-    v = value ? (v | bit) : (v & ~bit);
+    const unsigned int v = value ? kTestWithholdXTiles : 0u;
     return cudaMemcpyToSymbol(g_test_flags, &v, sizeof(v)) == cudaSuccess ? QMM_OK : QMM_ERR_CUDA;
+  }
+  if (what == QMM_DEBUG_WITHHOLD_TILE_COPIES) {  // a launch argument of the tile kernel (no device read)
+    if (value != 0 && value != 1) return QMM_ERR_INVALID_ARG;
+    g_withhold_tile_copies = value != 0;
+    return QMM_OK;
   }
   return QMM_ERR_INVALID_ARG;
 }
