@@ -133,3 +133,25 @@ def test_config_selection_runs_only_that_configurations_workloads(monkeypatch):
     full = set(bench.extra_workloads(args, 1, 1 << 27, peaks))
     assert full >= keys[1] | keys[3] | keys[4] | keys[5]
     assert {"fp4g16_e4m3_gemv_in_proj_m1", "mxfp4_gemv_in_proj_m1", "fp4g16_dequant_in_proj"} <= full
+
+
+def test_reference_arm_prints_the_contract_line():
+    """`bench.py --impl reference` (the oracle on the host cores) prints one
+    JSON line with the contract's keys, the headline's config and input
+    manifest, and e2e equal to its own value."""
+    import json
+    import subprocess
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--steps", "3",
+                        "--warmup", "3", "--cpu-budget", "0.05"], capture_output=True, text=True, timeout=600,
+                       cwd=root, env={k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE")})
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+                "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e", "gpu_launches", "inputs"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["steps"] == 3 and line["warmup"] == 3 and line["value"] > 0
+    assert line["config"]["workload"] == "fp4g16_gemv_mamba2_8b_in_proj_18560x4096_m1"
+    assert line["e2e"]["value"] == line["value"] and line["e2e"]["h2d_bytes_per_step"] == 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
+    assert line["inputs"]["w_data_sha256"].startswith("07e75c9359e62a11")
